@@ -1,0 +1,194 @@
+/*
+ * attn.h - C ABI of the B200 (sm_100a) masked attention forward.
+ *
+ * Computes, for every sequence b of a ragged batch, every query head h and every
+ * query row i,
+ *
+ *     out[i, h, :] = softmax_j( scale * q[i, h, :] . k[j, h / g, :]  +  mask[i, j] ) . v[j, h / g, :]
+ *     lse[i, h]    = ln sum_{j visible} exp( scale * q[i, h, :] . k[j, h / g, :] )
+ *
+ * with g = hq / hkv (grouped-query attention) and mask[i, j] in {0, -inf}. A row
+ * that sees no key gets out = 0 and lse = -inf. The masks are the kinds defined on:
+ *   - "feat: support custom mask for flash attention" (sglang-jax PR #20), Highlights:
+ *     ragged, paged attention with an optional custom mask or a causal flag;
+ *   - "[Attention] feat: support PrefixLM" (aphrodite-engine #1526), Highlights:
+ *     PrefixLM mask (bidirectional prefix, causal suffix) and prefix_len;
+ *   - "Custom mask slows down attention." (flashinfer #724): bit-packed custom masks;
+ *   - "Feature request: chunk-causal mask type for Flex Flash Attention" (MagiAttention
+ *     #316), Current pattern / Desired representation / Proposed API: q/k range lists,
+ *     attn_type_map, chunk-causal ranges with a chunk size;
+ *   - "feat: add Gemma2 sliding-window (local/global) attention" (mlxcel PR #555),
+ *     Summary: local mask = causal AND within the window.
+ *
+ * Coordinates. L_q and L_k are the query and key lengths of one sequence. Query row i
+ * (0-based inside its sequence) sits at key position pos(i) = i + L_k - L_q, i.e. the
+ * queries are the last L_q tokens of the sequence. All ranges are half-open.
+ *
+ * Usage. attn_plan() validates the problem and the mask descriptor, classifies every
+ * 128 x 128 (query, key) tile as empty, full or partial, writes the tile-transposed
+ * masks of the partial tiles and a balanced work list into a device workspace that the
+ * plan owns. attn_masked_fwd() then runs the forward on a stream; it allocates nothing
+ * and may be called any number of times with the same plan (e.g. the same lengths and
+ * mask for every layer). attn_plan_destroy() frees the plan.
+ *
+ * Errors. Every call returns an attn_status_t; nothing is thrown across the ABI and
+ * nothing exits the process. attn_status_string() names a status.
+ */
+#ifndef MASKED_ATTN_B200_ATTN_H
+#define MASKED_ATTN_B200_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A cudaStream_t. NULL is the legacy default stream. */
+typedef struct CUstream_st* attn_stream_t;
+
+typedef enum {
+  ATTN_OK = 0,
+  ATTN_ERR_INVALID_ARG = 1,    /* a null pointer, a negative or inconsistent size, a bad range */
+  ATTN_ERR_UNSUPPORTED = 2,    /* head_dim not in {64, 128, 256}, page_size not in {16, 32, 64, 128} */
+  ATTN_ERR_MASK_TOO_SMALL = 3, /* CUSTOM: the packed mask holds fewer words than the lengths need */
+  ATTN_ERR_OOM = 4,            /* cudaMalloc of the plan workspace failed */
+  ATTN_ERR_CUDA = 5,           /* any other CUDA runtime error (launch, copy, no device) */
+  ATTN_ERR_TIMEOUT = 6         /* a bounded wait inside the kernel expired (see attn_plan_check_status) */
+} attn_status_t;
+
+typedef enum {
+  ATTN_MASK_FULL = 0,           /* every key */
+  ATTN_MASK_CAUSAL = 1,         /* j <= pos(i) */
+  ATTN_MASK_SLIDING_WINDOW = 2, /* j <= pos(i) and pos(i) - j < window */
+  ATTN_MASK_PREFIX_LM = 3,      /* j < prefix_len  or  j <= pos(i) */
+  ATTN_MASK_CHUNK_CAUSAL = 4,   /* CAUSAL range over [0, chunk.q_start) plus the chunk-causal range `chunk` */
+  ATTN_MASK_RANGES = 5,         /* union of typed (q_range, k_range) pairs, per sequence */
+  ATTN_MASK_CUSTOM = 6          /* bit-packed boolean mask, per sequence, shared by all heads */
+} attn_mask_kind_t;
+
+/* Range types. 0 and 1 are the attn_type_map values FULL and CAUSAL printed on the
+ * chunk-causal feature request; 4 is this library's code for CHUNK_CAUSAL. */
+typedef enum {
+  ATTN_RANGE_FULL = 0,          /* every (i, j) in q_range x k_range */
+  ATTN_RANGE_CAUSAL = 1,        /* and j <= i, both in sequence-local coordinates */
+  ATTN_RANGE_CHUNK_CAUSAL = 4   /* query chunk c = (i - q_start) / chunk_size sees keys
+                                   [k_start, min(q_start + (c+1)*chunk_size, q_end)) within k_range */
+} attn_range_type_t;
+
+/* One (q_range, k_range) pair in sequence-local coordinates, half-open.
+ * 0 <= q_start <= q_end <= L_q, 0 <= k_start <= k_end <= L_k; chunk_size >= 1 for
+ * CHUNK_CAUSAL (ignored otherwise). Overlapping pairs are OR-ed. */
+typedef struct {
+  int32_t q_start, q_end, k_start, k_end, type, chunk_size;
+} attn_range_t;
+
+/* Mask descriptor. Only the fields of `kind` are read. */
+typedef struct {
+  int32_t kind;                     /* attn_mask_kind_t */
+  int32_t window;                   /* SLIDING_WINDOW: >= 1 (keys including the query's own position) */
+  int32_t prefix_len;               /* PREFIX_LM when prefix_lens is NULL: >= 0 */
+  const int32_t* prefix_lens;       /* PREFIX_LM: host [batch] per-sequence prefix lengths, or NULL */
+  attn_range_t chunk;               /* CHUNK_CAUSAL: the chunk-causal range, the same for every
+                                       sequence; rows and keys past a sequence's end are dropped,
+                                       the chunk arithmetic uses the values as given */
+  const attn_range_t* ranges;       /* RANGES: host, all sequences' ranges concatenated */
+  const int32_t* cu_ranges;         /* RANGES: host [batch+1]; sequence b owns ranges[cu_ranges[b] .. cu_ranges[b+1]) */
+  const uint32_t* mask_bits;        /* CUSTOM: DEVICE pointer. Sequence b's mask starts at word
+                                       mask_word_offsets[b] and is row-major [L_q][W], W = ceil(L_k/32);
+                                       key j of row i is bit (j % 32) of word i*W + j/32, least
+                                       significant bit first. Bits past L_k are ignored. */
+  const int64_t* mask_word_offsets; /* CUSTOM: host [batch+1] word offsets (non-decreasing) */
+  int64_t mask_words_total;         /* CUSTOM: number of readable words at mask_bits */
+} attn_mask_desc_t;
+
+/* Problem shape. Host arrays are read during attn_plan() only. */
+typedef struct {
+  int32_t batch;                    /* number of sequences, >= 0 */
+  int32_t hq, hkv;                  /* query / key-value heads, hq % hkv == 0 */
+  int32_t head_dim;                 /* 64, 128 or 256 (the value head dim is the same) */
+  float scale;                      /* softmax scale; <= 0 selects 1/sqrt(head_dim) */
+  const int32_t* cu_seqlens_q;      /* host [batch+1] query token offsets (non-decreasing, from 0) */
+  const int32_t* cu_seqlens_k;      /* host [batch+1] key token offsets; contiguous K/V only, else NULL */
+  const int32_t* kv_lens;           /* host [batch] key lengths; paged K/V only, else NULL */
+  const int32_t* page_table;        /* DEVICE int32 [batch][max_pages_per_seq]; paged only. Entry p of
+                                       row b holds the cache page of keys [p*page_size, (p+1)*page_size).
+                                       Entries outside [0, num_pages) read as zeros. Must stay valid
+                                       while forwards that use the plan run. */
+  int32_t page_size;                /* paged: 16, 32, 64 or 128 */
+  int32_t max_pages_per_seq;        /* paged: row length of page_table */
+  int32_t num_pages;                /* paged: pages in the K and V caches */
+} attn_problem_t;
+
+typedef struct attn_plan attn_plan_t; /* opaque */
+
+typedef struct {
+  int64_t unmasked_pairs;           /* visible (i, j) pairs summed over sequences, for ONE head */
+  int64_t tiles_empty, tiles_full, tiles_partial; /* 128 x 128 tile classes over valid rectangles */
+  int64_t mask_tiles;               /* 2 KiB tile-transposed mask tiles the forward reads */
+  int64_t work_items, jobs;         /* forward work list: items and (item, key tile) jobs */
+  int32_t ctas;                     /* persistent CTAs the forward launches */
+  int32_t heads_per_tile;           /* query heads packed into one 128-row tile (short queries) */
+  int32_t tiles_per_cta;            /* 128-row query tiles one CTA works on at once (1 or 2) */
+  int32_t reserved;
+} attn_plan_stats_t;
+
+/* Validate and plan. `stream` orders the plan's device work (the CUSTOM mask scan and
+ * the uploads); attn_plan returns after that work has finished. On success *out_plan
+ * owns a device workspace. Errors: INVALID_ARG, UNSUPPORTED, MASK_TOO_SMALL, OOM, CUDA.
+ * Defined by the pages listed at the top of this file; the validation rules follow the
+ * custom_mask review comments of "feat: support custom mask for flash attention"
+ * (conflicting options rejected; a custom mask shorter than the lengths need rejected). */
+attn_status_t attn_plan(const attn_problem_t* problem, const attn_mask_desc_t* mask,
+                        attn_stream_t stream, attn_plan_t** out_plan);
+
+/* Run the forward asynchronously on `stream`. All pointers are DEVICE pointers,
+ * 16-byte aligned, and must stay valid until the stream work completes:
+ *   q   bf16 [total_q][hq][head_dim]             (total_q = cu_seqlens_q[batch])
+ *   k,v bf16 [total_k][hkv][head_dim]            contiguous (total_k = cu_seqlens_k[batch]), or
+ *       bf16 [num_pages][page_size][hkv][head_dim] paged caches
+ *   out bf16 [total_q][hq][head_dim]             written for every valid row
+ *   lse fp32 [total_q][hq]                       natural log, scale included; may be NULL
+ * Allocates nothing. Errors: INVALID_ARG (null/misaligned pointer), CUDA (launch). */
+attn_status_t attn_masked_fwd(const attn_plan_t* plan, const void* q, const void* k, const void* v,
+                              void* out, float* lse, attn_stream_t stream);
+
+/* Copy the 128 x 128 tile classes (0 empty, 1 full, 2 partial) in the order sequence,
+ * query tile, key tile (row-major) into host_dst[0 .. n). *n_needed (may be NULL)
+ * receives the total count; a short buffer gets a prefix. */
+attn_status_t attn_plan_get_tile_classes(const attn_plan_t* plan, uint8_t* host_dst, size_t n,
+                                         size_t* n_needed);
+
+/* Plan statistics (host memory). */
+attn_status_t attn_plan_get_stats(const attn_plan_t* plan, attn_plan_stats_t* stats);
+
+/* Synchronise `stream`, then read and clear the plan's device status word. Returns
+ * ATTN_ERR_TIMEOUT if a bounded wait of an earlier forward expired (its output is then
+ * undefined), ATTN_ERR_CUDA on a CUDA error, else ATTN_OK. */
+attn_status_t attn_plan_check_status(const attn_plan_t* plan, attn_stream_t stream);
+
+/* Testing hook for the failure path: flags bit 0 makes the next forwards skip the
+ * arrival that publishes the first query tile, so that a bounded wait expires and the
+ * kernel returns through its abort path; timeout_ns (> 0) sets the per-wait limit
+ * (default 2 s). 0 / 0 restores the defaults. */
+attn_status_t attn_plan_set_debug(attn_plan_t* plan, int32_t flags, int64_t timeout_ns);
+
+/* Free the plan and its device workspace (after the forwards that use it finished). */
+attn_status_t attn_plan_destroy(attn_plan_t* plan);
+
+/* Host-only classification for the analytic kinds (everything but CUSTOM): the same
+ * validation and 128 x 128 tile classes as attn_plan, without any CUDA call (the device
+ * page_table pointer may be NULL here). classes
+ * may be NULL to query *n_needed; *unmasked_pairs (may be NULL) receives the per-head
+ * visible pair count. CUSTOM returns UNSUPPORTED (its bits live on the device). */
+attn_status_t attn_classify_host(const attn_problem_t* problem, const attn_mask_desc_t* mask,
+                                 uint8_t* classes, size_t n, size_t* n_needed,
+                                 int64_t* unmasked_pairs);
+
+const char* attn_status_string(attn_status_t status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MASKED_ATTN_B200_ATTN_H */

@@ -1,0 +1,276 @@
+"""B200 (sm_100a) masked attention forward.
+
+Thin Python binding over the C ABI declared in ``include/attn.h``: every function
+here only marshals arguments (torch tensors supply device memory and streams);
+all of the computation happens in ``libattn_b200.so``. Importing succeeds without a
+GPU; calls that need one fail with a RuntimeError. If the library has not been
+built, every call raises instead of falling back to anything else.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import numpy as np
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libattn_b200.so")
+
+ATTN_OK = 0
+STATUS = {0: "ATTN_OK", 1: "ATTN_ERR_INVALID_ARG", 2: "ATTN_ERR_UNSUPPORTED", 3: "ATTN_ERR_MASK_TOO_SMALL",
+          4: "ATTN_ERR_OOM", 5: "ATTN_ERR_CUDA", 6: "ATTN_ERR_TIMEOUT"}
+MASK_KIND = {"FULL": 0, "CAUSAL": 1, "SLIDING_WINDOW": 2, "PREFIX_LM": 3, "CHUNK_CAUSAL": 4, "RANGES": 5,
+             "CUSTOM": 6}
+RANGE_FULL, RANGE_CAUSAL, RANGE_CHUNK_CAUSAL = 0, 1, 4
+
+# every symbol include/attn.h declares
+EXPORTS = ("attn_plan", "attn_masked_fwd", "attn_plan_get_tile_classes", "attn_plan_get_stats",
+           "attn_plan_check_status", "attn_plan_set_debug", "attn_plan_destroy", "attn_classify_host",
+           "attn_status_string")
+
+
+class AttnError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS.get(status, status)}")
+
+
+class attn_range_t(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in ("q_start", "q_end", "k_start", "k_end", "type", "chunk_size")]
+
+
+class attn_mask_desc_t(ctypes.Structure):
+    _fields_ = [("kind", ctypes.c_int32), ("window", ctypes.c_int32), ("prefix_len", ctypes.c_int32),
+                ("prefix_lens", ctypes.c_void_p), ("chunk", attn_range_t), ("ranges", ctypes.c_void_p),
+                ("cu_ranges", ctypes.c_void_p), ("mask_bits", ctypes.c_void_p),
+                ("mask_word_offsets", ctypes.c_void_p), ("mask_words_total", ctypes.c_int64)]
+
+
+class attn_problem_t(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int32), ("hq", ctypes.c_int32), ("hkv", ctypes.c_int32),
+                ("head_dim", ctypes.c_int32), ("scale", ctypes.c_float), ("cu_seqlens_q", ctypes.c_void_p),
+                ("cu_seqlens_k", ctypes.c_void_p), ("kv_lens", ctypes.c_void_p), ("page_table", ctypes.c_void_p),
+                ("page_size", ctypes.c_int32), ("max_pages_per_seq", ctypes.c_int32), ("num_pages", ctypes.c_int32)]
+
+
+class attn_plan_stats_t(ctypes.Structure):
+    _fields_ = [("unmasked_pairs", ctypes.c_int64), ("tiles_empty", ctypes.c_int64), ("tiles_full", ctypes.c_int64),
+                ("tiles_partial", ctypes.c_int64), ("mask_tiles", ctypes.c_int64), ("work_items", ctypes.c_int64),
+                ("jobs", ctypes.c_int64), ("ctas", ctypes.c_int32), ("heads_per_tile", ctypes.c_int32),
+                ("tiles_per_cta", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded library; raises if it was not built (no fallback exists)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(_LIB_PATH):
+            raise RuntimeError(f"{_LIB_PATH} is missing: build it with "
+                               "`python -m masked_flash_attention_attn_b200.build`")
+        L = ctypes.CDLL(_LIB_PATH)
+        vp, i32, i64, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+        L.attn_plan.argtypes = [ctypes.POINTER(attn_problem_t), ctypes.POINTER(attn_mask_desc_t), vp,
+                                ctypes.POINTER(vp)]
+        L.attn_masked_fwd.argtypes = [vp, vp, vp, vp, vp, vp, vp]
+        L.attn_plan_get_tile_classes.argtypes = [vp, vp, sz, ctypes.POINTER(sz)]
+        L.attn_plan_get_stats.argtypes = [vp, ctypes.POINTER(attn_plan_stats_t)]
+        L.attn_plan_check_status.argtypes = [vp, vp]
+        L.attn_plan_set_debug.argtypes = [vp, i32, i64]
+        L.attn_plan_destroy.argtypes = [vp]
+        L.attn_classify_host.argtypes = [ctypes.POINTER(attn_problem_t), ctypes.POINTER(attn_mask_desc_t), vp, sz,
+                                         ctypes.POINTER(sz), ctypes.POINTER(i64)]
+        L.attn_status_string.argtypes = [i32]
+        L.attn_status_string.restype = ctypes.c_char_p
+        for n in EXPORTS[:-1]:
+            getattr(L, n).restype = i32
+        _lib = L
+    return _lib
+
+
+def _check(st: int, where: str):
+    if st != ATTN_OK:
+        raise AttnError(st, where)
+
+
+def _ptr(a) -> Optional[int]:
+    if a is None:
+        return None
+    if isinstance(a, np.ndarray):
+        return a.ctypes.data
+    return a.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream if torch.cuda.is_available() else None
+    return getattr(stream, "cuda_stream", stream)
+
+
+class _Marshal:
+    """Host arrays of one call, kept alive while the C side reads them."""
+
+    def __init__(self):
+        self.keep = []
+
+    def arr(self, x, dtype):
+        if x is None:
+            return None
+        a = np.ascontiguousarray(np.asarray(x, dtype=dtype))
+        self.keep.append(a)
+        return a.ctypes.data
+
+
+def _problem(m: _Marshal, *, hq, hkv, head_dim, cu_seqlens_q, cu_seqlens_k=None, kv_lens=None, page_table=None,
+             page_size=0, num_pages=0, scale=0.0):
+    cq = np.asarray(cu_seqlens_q, dtype=np.int32)
+    pr = attn_problem_t()
+    pr.batch = len(cq) - 1
+    pr.hq, pr.hkv, pr.head_dim, pr.scale = hq, hkv, head_dim, float(scale)
+    pr.cu_seqlens_q = m.arr(cq, np.int32)
+    pr.cu_seqlens_k = m.arr(cu_seqlens_k, np.int32)
+    pr.kv_lens = m.arr(kv_lens, np.int32)
+    if page_table is not None:
+        pr.page_table = _ptr(page_table)
+        pr.max_pages_per_seq = int(page_table.shape[1])
+        pr.page_size, pr.num_pages = int(page_size), int(num_pages)
+    return pr
+
+
+def _mask_desc(m: _Marshal, mask, device_bits=None):
+    """``mask``: an object with the attributes kind, window, prefix_len, prefix_lens, chunk,
+    ranges (per-sequence lists of 6-tuples), bits, word_offsets (see include/attn.h)."""
+    d = attn_mask_desc_t()
+    d.kind = MASK_KIND[mask.kind]
+    d.window = int(getattr(mask, "window", 0) or 0)
+    d.prefix_len = int(getattr(mask, "prefix_len", 0) or 0)
+    d.prefix_lens = m.arr(getattr(mask, "prefix_lens", None), np.int32)
+    ch = getattr(mask, "chunk", None)
+    if ch is not None:
+        d.chunk = attn_range_t(*[int(x) for x in ch])
+    rs = getattr(mask, "ranges", None)
+    if rs is not None:
+        flat = [tuple(int(x) for x in r) for per in rs for r in per]
+        cu = np.zeros(len(rs) + 1, np.int32)
+        cu[1:] = np.cumsum([len(per) for per in rs])
+        arr = (attn_range_t * max(1, len(flat)))(*[attn_range_t(*r) for r in flat])
+        m.keep.append(arr)
+        d.ranges = ctypes.addressof(arr)
+        d.cu_ranges = m.arr(cu, np.int32)
+    if mask.kind == "CUSTOM":
+        d.mask_word_offsets = m.arr(mask.word_offsets, np.int64)
+        d.mask_bits = _ptr(device_bits)
+        d.mask_words_total = int(device_bits.numel()) if device_bits is not None else 0
+    return d
+
+
+class Plan:
+    """Owns an attn_plan_t. Keeps the device page table (read by every forward) alive."""
+
+    def __init__(self, handle, page_table, hq, head_dim, total_q):
+        self.handle = handle
+        self._page_table = page_table
+        self.hq, self.head_dim, self.total_q = hq, head_dim, total_q
+
+    def __del__(self):
+        if getattr(self, "handle", None):
+            try:
+                attn_plan_destroy(self)
+            except Exception:
+                pass
+
+    @property
+    def stats(self) -> dict:
+        return attn_plan_get_stats(self)
+
+
+def attn_plan(*, hq: int, hkv: int, head_dim: int, cu_seqlens_q, mask, cu_seqlens_k=None, kv_lens=None,
+              page_table=None, page_size: int = 0, num_pages: int = 0, scale: float = 0.0, stream=None) -> Plan:
+    """attn_plan(): validate, classify tiles, build the work list. ``page_table`` is a device
+    int32 tensor [batch, max_pages]; CUSTOM ``mask.bits`` may be host (numpy) or device words."""
+    import torch
+    m = _Marshal()
+    pr = _problem(m, hq=hq, hkv=hkv, head_dim=head_dim, cu_seqlens_q=cu_seqlens_q, cu_seqlens_k=cu_seqlens_k,
+                  kv_lens=kv_lens, page_table=page_table, page_size=page_size, num_pages=num_pages, scale=scale)
+    dev_bits = None
+    if mask.kind == "CUSTOM":
+        b = mask.bits
+        if isinstance(b, np.ndarray):
+            dev_bits = torch.from_numpy(np.ascontiguousarray(b.astype(np.uint32).view(np.int32))).cuda()
+        else:
+            dev_bits = b
+    d = _mask_desc(m, mask, dev_bits)
+    h = ctypes.c_void_p()
+    _check(lib().attn_plan(ctypes.byref(pr), ctypes.byref(d), _stream(stream), ctypes.byref(h)), "attn_plan")
+    total_q = int(np.asarray(cu_seqlens_q)[-1])
+    return Plan(h.value, page_table, hq, head_dim, total_q)
+
+
+def attn_masked_fwd(plan: Plan, q, k, v, out, lse=None, stream=None) -> None:
+    """attn_masked_fwd(): enqueue the forward on ``stream`` (default: torch's current stream)."""
+    _check(lib().attn_masked_fwd(plan.handle, _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _stream(stream)),
+           "attn_masked_fwd")
+
+
+def attn_plan_get_tile_classes(plan: Plan) -> np.ndarray:
+    n = ctypes.c_size_t()
+    _check(lib().attn_plan_get_tile_classes(plan.handle, None, 0, ctypes.byref(n)), "attn_plan_get_tile_classes")
+    out = np.zeros(n.value, dtype=np.uint8)
+    _check(lib().attn_plan_get_tile_classes(plan.handle, out.ctypes.data, n.value, None),
+           "attn_plan_get_tile_classes")
+    return out
+
+
+def attn_plan_get_stats(plan: Plan) -> dict:
+    s = attn_plan_stats_t()
+    _check(lib().attn_plan_get_stats(plan.handle, ctypes.byref(s)), "attn_plan_get_stats")
+    return {n: getattr(s, n) for n, _ in attn_plan_stats_t._fields_ if n != "reserved"}
+
+
+def attn_plan_check_status(plan: Plan, stream=None) -> int:
+    """Synchronises the stream; returns the status code (0 ok, 6 a bounded wait expired)."""
+    return int(lib().attn_plan_check_status(plan.handle, _stream(stream)))
+
+
+def attn_plan_set_debug(plan: Plan, flags: int, timeout_ns: int = 0) -> None:
+    _check(lib().attn_plan_set_debug(plan.handle, int(flags), int(timeout_ns)), "attn_plan_set_debug")
+
+
+def attn_plan_destroy(plan: Plan) -> None:
+    if plan.handle:
+        h, plan.handle = plan.handle, None
+        _check(lib().attn_plan_destroy(h), "attn_plan_destroy")
+
+
+def attn_classify_host(*, hq: int, hkv: int, head_dim: int, cu_seqlens_q, mask, cu_seqlens_k=None, kv_lens=None,
+                       page_size: int = 0, max_pages_per_seq: int = 0, num_pages: int = 0):
+    """Host-only tile classes (analytic kinds). Returns (classes uint8, unmasked pairs per head)."""
+    m = _Marshal()
+    pr = _problem(m, hq=hq, hkv=hkv, head_dim=head_dim, cu_seqlens_q=cu_seqlens_q, cu_seqlens_k=cu_seqlens_k,
+                  kv_lens=kv_lens)
+    if kv_lens is not None:
+        pr.page_size, pr.max_pages_per_seq, pr.num_pages = page_size, max_pages_per_seq, num_pages
+    d = _mask_desc(m, mask)
+    n, pairs = ctypes.c_size_t(), ctypes.c_int64()
+    _check(lib().attn_classify_host(ctypes.byref(pr), ctypes.byref(d), None, 0, ctypes.byref(n), ctypes.byref(pairs)),
+           "attn_classify_host")
+    out = np.zeros(n.value, dtype=np.uint8)
+    _check(lib().attn_classify_host(ctypes.byref(pr), ctypes.byref(d), out.ctypes.data, n.value, None, None),
+           "attn_classify_host")
+    return out, int(pairs.value)
+
+
+def attn_status_string(status: int) -> str:
+    return lib().attn_status_string(int(status)).decode()
+
+
+def forward(plan: Plan, q, k, v, stream=None):
+    """Allocate out / lse with torch and run attn_masked_fwd (convenience)."""
+    import torch
+    out = torch.empty(q.shape[0], plan.hq, plan.head_dim, dtype=torch.bfloat16, device=q.device)
+    lse = torch.empty(q.shape[0], plan.hq, dtype=torch.float32, device=q.device)
+    attn_masked_fwd(plan, q, k, v, out, lse, stream)
+    return out, lse

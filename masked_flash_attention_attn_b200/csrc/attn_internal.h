@@ -1,0 +1,98 @@
+// Internal types shared by the host planner (attn_plan.cpp), the forward kernel
+// (attn_fwd.cu) and the CUSTOM-mask scan (attn_custom.cu). Not part of the ABI.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <vector>
+
+#include "attn.h"
+
+namespace mfa {
+
+constexpr int kTile = 128;          // query rows and keys per tile, and per classification tile
+constexpr int kMaskTileBytes = 2048;  // 128 rows x 128 bits
+
+// mask field of a Job
+constexpr int32_t kMaskFull = -1;   // tile fully visible: no mask arithmetic
+constexpr int32_t kMaskNone = -2;   // tile fully hidden for this query tile (pairing filler)
+
+// One unit of forward work: up to two 128-row query tiles that share one key/value
+// head and iterate over the same key tiles. Row r of tile t is query head
+// head[t] + r / R at token tok[t] + r % R, valid when r % R < rows[t]
+// (R = 128 / heads_per_tile).
+struct alignas(16) WorkItem {
+  int32_t seq;
+  int32_t kv_head;
+  int32_t k_base;      // contiguous: first key row of the sequence; paged: seq * max_pages_per_seq
+  int32_t kv_len;      // valid keys of the sequence
+  int32_t tok[2];
+  int32_t rows[2];
+  int32_t head[2];
+  int32_t job_start;
+  int32_t job_count;
+  int32_t npages;      // paged: pages that hold the sequence's keys
+  int32_t pad;
+};
+static_assert(sizeof(WorkItem) == 64, "WorkItem layout");
+
+// One key tile of a work item and, per query tile, how to mask it.
+struct alignas(16) Job {
+  int32_t k_tile;
+  int32_t mask[2];     // kMaskFull, kMaskNone or the index of a 2 KiB mask tile
+  int32_t pad;
+};
+static_assert(sizeof(Job) == 16, "Job layout");
+
+// ---- CUSTOM mask scan on the device ----------------------------------------------------
+struct CustomSeq {
+  int64_t word_off;    // first word of the sequence's packed mask
+  int64_t cnt_off;     // first count of the sequence in the count array
+  int32_t lq, lk;
+  int32_t n_rb, n_kt;  // row blocks of R rows, key tiles of 128
+};
+struct CountTask { int32_t seq, rb, kt0, pad; };   // one row block x up to 32 key tiles
+struct RepackTask { int32_t seq, rb, kt, idx; };    // one mask tile to write
+
+cudaError_t launch_custom_count(const uint32_t* bits, const CustomSeq* seqs, const CountTask* tasks,
+                                int ntasks, int R, int32_t* counts, cudaStream_t stream);
+cudaError_t launch_custom_repack(const uint32_t* bits, const CustomSeq* seqs, const RepackTask* tasks,
+                                 int ntasks, int R, uint4* tiles, cudaStream_t stream);
+
+}  // namespace mfa
+
+struct attn_plan {
+  // problem
+  int32_t batch = 0, hq = 0, hkv = 0, d = 0;
+  float scale = 0.f;
+  bool paged = false;
+  int32_t page_size = 0, max_pages = 0, num_pages = 0;
+  const int32_t* page_table = nullptr;   // device
+  int64_t total_q = 0, total_kv_rows = 0;
+  // kernel shape
+  int32_t nq = 1;        // query tiles per CTA
+  int32_t hp = 1;        // heads packed per query tile
+  int32_t R = 128;       // rows per head in a query tile
+  int32_t ctas = 0;
+  // host results
+  std::vector<uint8_t> classes;
+  attn_plan_stats_t stats{};
+  // device workspace (one allocation)
+  void* ws = nullptr;
+  size_t ws_bytes = 0;
+  int32_t* d_status = nullptr;
+  const mfa::WorkItem* d_items = nullptr;
+  const mfa::Job* d_jobs = nullptr;
+  const int32_t* d_cta_off = nullptr;
+  const int32_t* d_cta_items = nullptr;
+  const uint4* d_mask_tiles = nullptr;
+  // debug hooks
+  int32_t debug_flags = 0;
+  int64_t timeout_ns = 2000000000LL;
+  int device = 0;
+};
+
+// forward launcher (attn_fwd.cu)
+attn_status_t mfa_launch_forward(const attn_plan_t* plan, const void* q, const void* k, const void* v,
+                                 void* out, float* lse, cudaStream_t stream);

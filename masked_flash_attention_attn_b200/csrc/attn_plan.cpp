@@ -1,0 +1,780 @@
+// Host planner and C ABI of the masked attention forward.
+//
+// attn_plan() turns a problem + mask descriptor into:
+//   * the class of every 128 x 128 (query, key) tile over its valid sub-rectangle
+//     (empty / full / partial): empty tiles are never loaded, full tiles skip all mask
+//     arithmetic, partial tiles get a 2 KiB tile-transposed bit mask (row r's 128 bits
+//     at byte 16 r, bit c of the row = key c of the tile) that one thread per row reads
+//     with a single 16-byte load. This replaces the per-element, uncoalesced custom-mask
+//     reads that "Custom mask slows down attention." (flashinfer #724) blames for a 2x
+//     slowdown, and generalises the block mask of "[Attention] feat: support PrefixLM"
+//     (build_block_mask) to every kind;
+//   * a work list of (query tiles, key-tile run) items, balanced over the persistent CTAs
+//     of the forward by longest-processing-time-first assignment, so that ragged lengths
+//     ("feat: support custom mask for flash attention": ragged paged attention) do not
+//     leave SMs idle.
+//
+// Analytic kinds are reduced to per-row half-open key intervals on the host; range lists
+// ("Feature request: chunk-causal mask type for Flex Flash Attention") are merged per row,
+// so the union of many ranges classifies exactly even when no single range covers a tile.
+// CUSTOM masks are scanned on the device (attn_custom.cu).
+#include <algorithm>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <new>
+#include <numeric>
+#include <queue>
+#include <stdexcept>
+#include <utility>
+#include <vector>
+
+#include "attn_internal.h"
+
+namespace {
+
+using namespace mfa;
+
+struct Iv {
+  int32_t a, b;
+};
+
+constexpr int32_t kClassEmpty = 0, kClassFull = 1, kClassPartial = 2;
+
+// Validated view of the problem.
+struct Shape {
+  int B = 0, hq = 0, hkv = 0, d = 0;
+  float scale = 0.f;
+  bool paged = false;
+  int ps = 0, maxp = 0, npages = 0;
+  std::vector<int32_t> lq, lk, qoff, koff;
+  int64_t total_q = 0, total_kv_rows = 0;
+};
+
+attn_status_t validate_problem(const attn_problem_t* p, Shape& s, bool need_device_ptrs = true) {
+  if (!p) return ATTN_ERR_INVALID_ARG;
+  if (p->batch < 0 || p->hq <= 0 || p->hkv <= 0) return ATTN_ERR_INVALID_ARG;
+  if (p->hq % p->hkv != 0) return ATTN_ERR_INVALID_ARG;
+  if (p->head_dim != 64 && p->head_dim != 128 && p->head_dim != 256) return ATTN_ERR_UNSUPPORTED;
+  if (std::isnan(p->scale) || std::isinf(p->scale)) return ATTN_ERR_INVALID_ARG;
+  s.B = p->batch;
+  s.hq = p->hq;
+  s.hkv = p->hkv;
+  s.d = p->head_dim;
+  s.scale = p->scale > 0.f ? p->scale : 1.0f / std::sqrt(float(p->head_dim));
+  if (s.B > 0 && !p->cu_seqlens_q) return ATTN_ERR_INVALID_ARG;
+  s.paged = p->cu_seqlens_k == nullptr;
+  if (s.paged) {
+    if (s.B > 0 && (!p->kv_lens || (need_device_ptrs && !p->page_table))) return ATTN_ERR_INVALID_ARG;
+    if (p->page_size != 16 && p->page_size != 32 && p->page_size != 64 && p->page_size != 128)
+      return ATTN_ERR_UNSUPPORTED;
+    if (p->max_pages_per_seq < 0 || p->num_pages < 0) return ATTN_ERR_INVALID_ARG;
+    if (int64_t(p->num_pages) * p->page_size > INT32_MAX) return ATTN_ERR_UNSUPPORTED;
+    s.ps = p->page_size;
+    s.maxp = p->max_pages_per_seq;
+    s.npages = p->num_pages;
+  } else if (p->kv_lens) {
+    return ATTN_ERR_INVALID_ARG;  // both layouts given
+  }
+  if (s.B > 0 && p->cu_seqlens_q[0] != 0) return ATTN_ERR_INVALID_ARG;
+  s.lq.resize(s.B);
+  s.lk.resize(s.B);
+  s.qoff.resize(s.B);
+  s.koff.resize(s.B);
+  for (int b = 0; b < s.B; ++b) {
+    int64_t q0 = p->cu_seqlens_q[b], q1 = p->cu_seqlens_q[b + 1];
+    if (q1 < q0) return ATTN_ERR_INVALID_ARG;
+    s.lq[b] = int32_t(q1 - q0);
+    s.qoff[b] = int32_t(q0);
+    if (s.paged) {
+      int64_t n = p->kv_lens[b];
+      if (n < 0) return ATTN_ERR_INVALID_ARG;
+      if (n > int64_t(s.maxp) * s.ps) return ATTN_ERR_INVALID_ARG;  // more keys than the page row holds
+      s.lk[b] = int32_t(n);
+      if (int64_t(b) * s.maxp > INT32_MAX) return ATTN_ERR_UNSUPPORTED;
+      s.koff[b] = b * s.maxp;
+    } else {
+      if (b == 0 && p->cu_seqlens_k[0] != 0) return ATTN_ERR_INVALID_ARG;
+      int64_t k0 = p->cu_seqlens_k[b], k1 = p->cu_seqlens_k[b + 1];
+      if (k1 < k0) return ATTN_ERR_INVALID_ARG;
+      s.lk[b] = int32_t(k1 - k0);
+      s.koff[b] = int32_t(k0);
+    }
+  }
+  s.total_q = s.B ? p->cu_seqlens_q[s.B] : 0;
+  s.total_kv_rows = s.paged ? int64_t(s.npages) * s.ps : (s.B ? p->cu_seqlens_k[s.B] : 0);
+  return ATTN_OK;
+}
+
+bool range_ok(const attn_range_t& r) {
+  if (r.q_start < 0 || r.q_end < r.q_start || r.k_start < 0 || r.k_end < r.k_start) return false;
+  if (r.type != ATTN_RANGE_FULL && r.type != ATTN_RANGE_CAUSAL && r.type != ATTN_RANGE_CHUNK_CAUSAL)
+    return false;
+  if (r.type == ATTN_RANGE_CHUNK_CAUSAL && r.chunk_size < 1) return false;
+  return true;
+}
+
+attn_status_t validate_mask(const attn_mask_desc_t* m, const Shape& s) {
+  if (!m) return ATTN_ERR_INVALID_ARG;
+  switch (m->kind) {
+    case ATTN_MASK_FULL:
+    case ATTN_MASK_CAUSAL:
+      return ATTN_OK;
+    case ATTN_MASK_SLIDING_WINDOW:
+      return m->window >= 1 ? ATTN_OK : ATTN_ERR_INVALID_ARG;
+    case ATTN_MASK_PREFIX_LM:
+      if (m->prefix_lens) {
+        for (int b = 0; b < s.B; ++b)
+          if (m->prefix_lens[b] < 0) return ATTN_ERR_INVALID_ARG;
+        return ATTN_OK;
+      }
+      return m->prefix_len >= 0 ? ATTN_OK : ATTN_ERR_INVALID_ARG;
+    case ATTN_MASK_CHUNK_CAUSAL:
+      if (m->chunk.type != ATTN_RANGE_CHUNK_CAUSAL || !range_ok(m->chunk)) return ATTN_ERR_INVALID_ARG;
+      return ATTN_OK;
+    case ATTN_MASK_RANGES: {
+      if (s.B > 0 && (!m->cu_ranges || m->cu_ranges[0] != 0)) return ATTN_ERR_INVALID_ARG;
+      for (int b = 0; b < s.B; ++b) {
+        if (m->cu_ranges[b + 1] < m->cu_ranges[b]) return ATTN_ERR_INVALID_ARG;
+        if (m->cu_ranges[b + 1] > m->cu_ranges[b] && !m->ranges) return ATTN_ERR_INVALID_ARG;
+        for (int32_t r = m->cu_ranges[b]; r < m->cu_ranges[b + 1]; ++r) {
+          const attn_range_t& g = m->ranges[r];
+          if (!range_ok(g) || g.q_end > s.lq[b] || g.k_end > s.lk[b]) return ATTN_ERR_INVALID_ARG;
+        }
+      }
+      return ATTN_OK;
+    }
+    case ATTN_MASK_CUSTOM: {
+      if (s.B == 0) return ATTN_OK;
+      if (!m->mask_word_offsets) return ATTN_ERR_INVALID_ARG;
+      if (m->mask_words_total < 0) return ATTN_ERR_INVALID_ARG;
+      int64_t need_end = 0;
+      for (int b = 0; b < s.B; ++b) {
+        int64_t o0 = m->mask_word_offsets[b], o1 = m->mask_word_offsets[b + 1];
+        if (o0 < 0 || o1 < o0) return ATTN_ERR_INVALID_ARG;
+        int64_t need = int64_t(s.lq[b]) * ((int64_t(s.lk[b]) + 31) / 32);
+        // "custom_mask length must be larger than total kv length" (sglang-jax PR #20 review)
+        if (o1 - o0 < need) return ATTN_ERR_MASK_TOO_SMALL;
+        need_end = std::max(need_end, o0 + need);
+      }
+      if (need_end > m->mask_words_total) return ATTN_ERR_MASK_TOO_SMALL;
+      if (need_end > 0 && !m->mask_bits) return ATTN_ERR_INVALID_ARG;
+      return ATTN_OK;
+    }
+    default:
+      return ATTN_ERR_INVALID_ARG;
+  }
+}
+
+// Per-row key intervals of the analytic kinds (everything but CUSTOM).
+class RowSource {
+ public:
+  RowSource(const attn_mask_desc_t* m, const Shape& s) : m_(m), s_(s) {}
+
+  // Build the merged per-row intervals of sequence b for the range kinds.
+  void prepare(int b) {
+    if (m_->kind != ATTN_MASK_RANGES && m_->kind != ATTN_MASK_CHUNK_CAUSAL) return;
+    const int lq = s_.lq[b], lk = s_.lk[b];
+    std::vector<attn_range_t> rs;
+    if (m_->kind == ATTN_MASK_RANGES) {
+      for (int32_t r = m_->cu_ranges[b]; r < m_->cu_ranges[b + 1]; ++r) rs.push_back(m_->ranges[r]);
+    } else {
+      const attn_range_t& c = m_->chunk;
+      rs.push_back(attn_range_t{0, c.q_start, 0, c.q_start, ATTN_RANGE_CAUSAL, 0});
+      rs.push_back(c);
+    }
+    off_.assign(size_t(lq) + 1, 0);
+    for (const auto& r : rs) {
+      int32_t a = std::min(r.q_start, lq), e = std::min(r.q_end, lq);
+      for (int32_t i = a; i < e; ++i) off_[i + 1]++;
+    }
+    for (int i = 0; i < lq; ++i) off_[i + 1] += off_[i];
+    iv_.assign(off_[lq], Iv{0, 0});
+    std::vector<int64_t> fill(off_.begin(), off_.end() - 1);
+    for (const auto& r : rs) {
+      int32_t a = std::min(r.q_start, lq), e = std::min(r.q_end, lq);
+      for (int32_t i = a; i < e; ++i) {
+        int64_t lo = std::max<int64_t>(r.k_start, 0), hi = std::min<int64_t>(r.k_end, lk);
+        if (r.type == ATTN_RANGE_CAUSAL) {
+          hi = std::min<int64_t>(hi, int64_t(i) + 1);
+        } else if (r.type == ATTN_RANGE_CHUNK_CAUSAL) {
+          int64_t c = (int64_t(i) - r.q_start) / r.chunk_size;
+          int64_t end = std::min<int64_t>(int64_t(r.q_start) + (c + 1) * int64_t(r.chunk_size), r.q_end);
+          hi = std::min(hi, end);
+        }
+        iv_[fill[i]++] = lo < hi ? Iv{int32_t(lo), int32_t(hi)} : Iv{0, 0};
+      }
+    }
+    // merge each row in place (sort by start; drop empties; coalesce overlaps/adjacency)
+    std::vector<int64_t> noff(size_t(lq) + 1, 0);
+    int64_t w = 0;
+    for (int i = 0; i < lq; ++i) {
+      auto first = iv_.begin() + off_[i], last = iv_.begin() + off_[i + 1];
+      std::sort(first, last, [](const Iv& x, const Iv& y) { return x.a < y.a; });
+      int64_t row_start = w;
+      for (auto it = first; it != last; ++it) {
+        if (it->a >= it->b) continue;
+        if (w > row_start && it->a <= iv_[w - 1].b) {
+          iv_[w - 1].b = std::max(iv_[w - 1].b, it->b);
+        } else {
+          iv_[w++] = *it;
+        }
+      }
+      noff[i + 1] = w;
+    }
+    iv_.resize(w);
+    off_.swap(noff);
+  }
+
+  // Intervals of row i of sequence b (sorted, disjoint, non-empty, inside [0, L_k)).
+  int row(int b, int i, const Iv** out) {
+    const int64_t lq = s_.lq[b], lk = s_.lk[b];
+    const int64_t pos = int64_t(i) + lk - lq;
+    int n = 0;
+    auto emit = [&](int64_t a, int64_t e) {
+      a = std::max<int64_t>(a, 0);
+      e = std::min<int64_t>(e, lk);
+      if (a < e) buf_[n++] = Iv{int32_t(a), int32_t(e)};
+    };
+    switch (m_->kind) {
+      case ATTN_MASK_FULL:
+        emit(0, lk);
+        break;
+      case ATTN_MASK_CAUSAL:
+        emit(0, pos + 1);
+        break;
+      case ATTN_MASK_SLIDING_WINDOW:
+        emit(pos - int64_t(m_->window) + 1, pos + 1);
+        break;
+      case ATTN_MASK_PREFIX_LM: {
+        int64_t p = m_->prefix_lens ? m_->prefix_lens[b] : m_->prefix_len;
+        emit(0, std::max(p, pos + 1));
+        break;
+      }
+      default:
+        *out = iv_.data() + off_[i];
+        return int(off_[i + 1] - off_[i]);
+    }
+    *out = buf_;
+    return n;
+  }
+
+ private:
+  const attn_mask_desc_t* m_;
+  const Shape& s_;
+  std::vector<int64_t> off_;
+  std::vector<Iv> iv_;
+  Iv buf_[2];
+};
+
+// Visible-pair counts of every (row block of R rows, key tile) of one sequence.
+void count_sequence(RowSource& src, int b, const Shape& s, int R, std::vector<int32_t>& cnt) {
+  const int lq = s.lq[b], lk = s.lk[b];
+  const int n_rb = (lq + R - 1) / R, n_kt = (lk + kTile - 1) / kTile;
+  cnt.assign(size_t(n_rb) * n_kt, 0);
+  std::vector<int32_t> diff(size_t(n_kt) + 1);
+  for (int rb = 0; rb < n_rb; ++rb) {
+    int32_t* c = cnt.data() + size_t(rb) * n_kt;
+    std::fill(diff.begin(), diff.end(), 0);
+    const int r_end = std::min(lq, (rb + 1) * R);
+    for (int i = rb * R; i < r_end; ++i) {
+      const Iv* iv;
+      int n = src.row(b, i, &iv);
+      for (int t = 0; t < n; ++t) {
+        const int a = iv[t].a, e = iv[t].b;
+        const int ka = a / kTile, kb = (e - 1) / kTile;
+        if (ka == kb) {
+          c[ka] += e - a;
+        } else {
+          c[ka] += (ka + 1) * kTile - a;
+          c[kb] += e - kb * kTile;
+          diff[ka + 1] += 1;
+          diff[kb] -= 1;
+        }
+      }
+    }
+    int32_t run = 0;
+    for (int kt = 0; kt < n_kt; ++kt) {
+      run += diff[kt];
+      c[kt] += run * kTile;
+    }
+  }
+}
+
+inline int32_t classify(int64_t cnt, int64_t total) {
+  return cnt == 0 ? kClassEmpty : (cnt == total ? kClassFull : kClassPartial);
+}
+
+// 128 x 128 classes of one sequence from its R-row block counts.
+void report_classes(const std::vector<int32_t>& cnt, int lq, int lk, int R, std::vector<uint8_t>& out,
+                    attn_plan_stats_t& st) {
+  const int n_rb = (lq + R - 1) / R, n_kt = (lk + kTile - 1) / kTile;
+  const int n_qt = (lq + kTile - 1) / kTile, per = kTile / R;
+  for (int qt = 0; qt < n_qt; ++qt) {
+    const int64_t rows = std::min(kTile, lq - qt * kTile);
+    for (int kt = 0; kt < n_kt; ++kt) {
+      int64_t c = 0;
+      for (int rb = qt * per; rb < std::min(n_rb, (qt + 1) * per); ++rb) c += cnt[size_t(rb) * n_kt + kt];
+      const int64_t cols = std::min(kTile, lk - kt * kTile);
+      const int32_t k = classify(c, rows * cols);
+      out.push_back(uint8_t(k));
+      st.unmasked_pairs += c;
+      if (k == kClassEmpty) st.tiles_empty++;
+      else if (k == kClassFull) st.tiles_full++;
+      else st.tiles_partial++;
+    }
+  }
+}
+
+struct TileRef {
+  int32_t seq, rb, kt, idx;
+};
+
+// Work list for all sequences given their R-row block counts.
+struct WorkList {
+  std::vector<WorkItem> items;
+  std::vector<Job> jobs;
+  std::vector<TileRef> mask_tiles;   // in index order
+  std::vector<int32_t> cta_off, cta_items;
+};
+
+void build_work(const Shape& s, int R, int hp, int nq, const std::vector<std::vector<int32_t>>& cnts,
+                int num_sms, WorkList& wl) {
+  const int g = s.hq / s.hkv;
+  const int G = g / hp;  // head groups per kv head
+  for (int b = 0; b < s.B; ++b) {
+    const int lq = s.lq[b], lk = s.lk[b];
+    if (lq == 0) continue;
+    const int n_rb = (lq + R - 1) / R, n_kt = (lk + kTile - 1) / kTile;
+    const std::vector<int32_t>& cnt = cnts[b];
+    std::vector<int32_t> tidx(size_t(n_rb) * n_kt, -1);
+    auto kclass = [&](int rb, int kt) -> int32_t {
+      const int64_t rows = std::min(R, lq - rb * R), cols = std::min(kTile, lk - kt * kTile);
+      return classify(cnt[size_t(rb) * n_kt + kt], rows * cols);
+    };
+    auto mask_of = [&](int rb, int kt) -> int32_t {
+      if (rb < 0) return kMaskNone;
+      const int32_t k = kclass(rb, kt);
+      if (k == kClassEmpty) return kMaskNone;
+      // a full tile that extends past L_k still needs its key columns cut
+      if (k == kClassFull && (kt + 1) * kTile <= lk) return kMaskFull;
+      int32_t& t = tidx[size_t(rb) * n_kt + kt];
+      if (t < 0) {
+        t = int32_t(wl.mask_tiles.size());
+        wl.mask_tiles.push_back(TileRef{b, rb, kt, t});
+      }
+      return t;
+    };
+    auto add_item = [&](int kh, int rb0, int hg0, int rb1, int hg1) {
+      WorkItem it{};
+      it.seq = b;
+      it.kv_head = kh;
+      it.k_base = s.koff[b];
+      it.kv_len = lk;
+      it.npages = s.paged ? (lk + s.ps - 1) / s.ps : 0;
+      const int rbs[2] = {rb0, rb1}, hgs[2] = {hg0, hg1};
+      for (int t = 0; t < 2; ++t) {
+        const int rb = rbs[t] >= 0 ? rbs[t] : rb0, hg = rbs[t] >= 0 ? hgs[t] : hg0;
+        it.tok[t] = s.qoff[b] + rb * R;
+        it.rows[t] = rbs[t] >= 0 ? std::min(R, lq - rb * R) : 0;
+        it.head[t] = kh * g + hg * hp;
+      }
+      it.job_start = int32_t(wl.jobs.size());
+      for (int kt = 0; kt < n_kt; ++kt) {
+        Job j{};
+        j.k_tile = kt;
+        j.mask[0] = mask_of(rb0, kt);
+        j.mask[1] = nq == 2 ? mask_of(rb1, kt) : kMaskNone;
+        if (j.mask[0] == kMaskNone && j.mask[1] == kMaskNone) continue;
+        wl.jobs.push_back(j);
+      }
+      if (wl.jobs.size() == size_t(it.job_start)) {
+        // every row of the item is fully masked: one hidden job writes out = 0, lse = -inf
+        wl.jobs.push_back(Job{0, {kMaskNone, kMaskNone}, 0});
+      }
+      it.job_count = int32_t(wl.jobs.size()) - it.job_start;
+      wl.items.push_back(it);
+    };
+    for (int kh = 0; kh < s.hkv; ++kh) {
+      if (nq == 2 && G >= 2) {
+        for (int rb = 0; rb < n_rb; ++rb)
+          for (int hg = 0; hg < G; hg += 2) add_item(kh, rb, hg, hg + 1 < G ? rb : -1, hg + 1);
+      } else if (nq == 2) {
+        for (int rb = 0; rb < n_rb; rb += 2) add_item(kh, rb, 0, rb + 1 < n_rb ? rb + 1 : -1, 0);
+      } else {
+        for (int rb = 0; rb < n_rb; ++rb)
+          for (int hg = 0; hg < G; ++hg) add_item(kh, rb, hg, -1, 0);
+      }
+    }
+  }
+  // longest-processing-time-first onto persistent CTAs
+  const int n_items = int(wl.items.size());
+  const int C = std::max(1, std::min(num_sms, n_items));
+  std::vector<int32_t> order(n_items);
+  std::iota(order.begin(), order.end(), 0);
+  std::stable_sort(order.begin(), order.end(), [&](int32_t x, int32_t y) {
+    return wl.items[x].job_count > wl.items[y].job_count;
+  });
+  using Load = std::pair<int64_t, int32_t>;
+  std::priority_queue<Load, std::vector<Load>, std::greater<Load>> heap;
+  for (int c = 0; c < C; ++c) heap.push(Load{0, c});
+  std::vector<std::vector<int32_t>> per(C);
+  for (int32_t it : order) {
+    Load l = heap.top();
+    heap.pop();
+    per[l.second].push_back(it);
+    l.first += int64_t(wl.items[it].job_count) + 1;
+    heap.push(l);
+  }
+  wl.cta_off.assign(size_t(C) + 1, 0);
+  wl.cta_items.clear();
+  for (int c = 0; c < C; ++c) {
+    wl.cta_items.insert(wl.cta_items.end(), per[c].begin(), per[c].end());
+    wl.cta_off[c + 1] = int32_t(wl.cta_items.size());
+  }
+}
+
+// Tile-transposed bits of one mask tile from the row intervals.
+void write_mask_tile(RowSource& src, const Shape& s, int R, const TileRef& t, uint32_t* dst) {
+  std::memset(dst, 0, kMaskTileBytes);
+  const int lq = s.lq[t.seq], lk = s.lk[t.seq];
+  const int c0 = t.kt * kTile, c1 = std::min(lk, c0 + kTile);
+  for (int lr = 0; lr < R; ++lr) {
+    const int i = t.rb * R + lr;
+    if (i >= lq) break;
+    uint32_t w[4] = {0, 0, 0, 0};
+    const Iv* iv;
+    const int n = src.row(t.seq, i, &iv);
+    for (int k = 0; k < n; ++k) {
+      const int a = std::max(iv[k].a, c0), e = std::min(iv[k].b, c1);
+      for (int j = a; j < e; ++j) w[(j - c0) >> 5] |= 1u << ((j - c0) & 31);
+    }
+    for (int r = lr; r < kTile; r += R) std::memcpy(dst + 4 * r, w, 16);
+  }
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct Staging {
+  size_t off_items, off_jobs, off_cta_off, off_cta_items, off_tiles, total;
+};
+
+Staging layout(const WorkList& wl) {
+  Staging st{};
+  st.off_items = 256;
+  st.off_jobs = align256(st.off_items + wl.items.size() * sizeof(WorkItem));
+  st.off_cta_off = align256(st.off_jobs + wl.jobs.size() * sizeof(Job));
+  st.off_cta_items = align256(st.off_cta_off + wl.cta_off.size() * sizeof(int32_t));
+  st.off_tiles = align256(st.off_cta_items + wl.cta_items.size() * sizeof(int32_t));
+  st.total = st.off_tiles + wl.mask_tiles.size() * size_t(kMaskTileBytes);
+  return st;
+}
+
+int choose_hp(const Shape& s) {
+  const int g = s.hq / s.hkv;
+  int lmax = 0;
+  for (int b = 0; b < s.B; ++b) lmax = std::max(lmax, s.lq[b]);
+  int hp = 1;
+  while (hp * 2 <= g && g % (hp * 2) == 0 && kTile / (hp * 2) >= std::max(lmax, 8)) hp *= 2;
+  return hp;
+}
+
+attn_status_t cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return ATTN_OK;
+  if (e == cudaErrorMemoryAllocation) return ATTN_ERR_OOM;
+  return ATTN_ERR_CUDA;
+}
+
+// CUSTOM: counts of every (row block, key tile) from the packed bits on the device.
+attn_status_t custom_counts(const attn_mask_desc_t* m, const Shape& s, int R, cudaStream_t stream,
+                            std::vector<std::vector<int32_t>>& cnts) {
+  std::vector<CustomSeq> seqs(s.B);
+  std::vector<CountTask> tasks;
+  int64_t total = 0;
+  for (int b = 0; b < s.B; ++b) {
+    CustomSeq& c = seqs[b];
+    c.word_off = m->mask_word_offsets[b];
+    c.lq = s.lq[b];
+    c.lk = s.lk[b];
+    c.n_rb = (c.lq + R - 1) / R;
+    c.n_kt = (c.lk + kTile - 1) / kTile;
+    c.cnt_off = total;
+    total += int64_t(c.n_rb) * c.n_kt;
+    for (int rb = 0; rb < c.n_rb; ++rb)
+      for (int kt = 0; kt < c.n_kt; kt += 32) tasks.push_back(CountTask{b, rb, kt, 0});
+  }
+  for (int b = 0; b < s.B; ++b) cnts[b].assign(size_t(seqs[b].n_rb) * seqs[b].n_kt, 0);
+  if (tasks.empty()) return ATTN_OK;
+  void* tmp = nullptr;
+  const size_t bytes_seqs = align256(seqs.size() * sizeof(CustomSeq));
+  const size_t bytes_tasks = align256(tasks.size() * sizeof(CountTask));
+  const size_t bytes = bytes_seqs + bytes_tasks + size_t(total) * sizeof(int32_t);
+  cudaError_t e = cudaMalloc(&tmp, bytes);
+  if (e != cudaSuccess) return cuda_status(e);
+  auto* d_seqs = reinterpret_cast<CustomSeq*>(tmp);
+  auto* d_tasks = reinterpret_cast<CountTask*>(static_cast<char*>(tmp) + bytes_seqs);
+  auto* d_cnt = reinterpret_cast<int32_t*>(static_cast<char*>(tmp) + bytes_seqs + bytes_tasks);
+  std::vector<int32_t> host(total);
+  e = cudaMemcpyAsync(d_seqs, seqs.data(), seqs.size() * sizeof(CustomSeq), cudaMemcpyHostToDevice, stream);
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(d_tasks, tasks.data(), tasks.size() * sizeof(CountTask), cudaMemcpyHostToDevice, stream);
+  if (e == cudaSuccess) e = cudaMemsetAsync(d_cnt, 0, size_t(total) * sizeof(int32_t), stream);
+  if (e == cudaSuccess) e = launch_custom_count(m->mask_bits, d_seqs, d_tasks, int(tasks.size()), R, d_cnt, stream);
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(host.data(), d_cnt, size_t(total) * sizeof(int32_t), cudaMemcpyDeviceToHost, stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+  cudaFree(tmp);
+  if (e != cudaSuccess) return cuda_status(e);
+  for (int b = 0; b < s.B; ++b)
+    std::copy(host.begin() + seqs[b].cnt_off, host.begin() + seqs[b].cnt_off + cnts[b].size(), cnts[b].begin());
+  return ATTN_OK;
+}
+
+attn_status_t custom_repack(const attn_mask_desc_t* m, const Shape& s, int R, const WorkList& wl,
+                            uint4* d_tiles, cudaStream_t stream) {
+  if (wl.mask_tiles.empty()) return ATTN_OK;
+  std::vector<CustomSeq> seqs(s.B);
+  for (int b = 0; b < s.B; ++b) {
+    seqs[b].word_off = m->mask_word_offsets[b];
+    seqs[b].lq = s.lq[b];
+    seqs[b].lk = s.lk[b];
+    seqs[b].n_rb = (s.lq[b] + R - 1) / R;
+    seqs[b].n_kt = (s.lk[b] + kTile - 1) / kTile;
+  }
+  std::vector<RepackTask> tasks(wl.mask_tiles.size());
+  for (size_t i = 0; i < tasks.size(); ++i) {
+    const TileRef& t = wl.mask_tiles[i];
+    tasks[i] = RepackTask{t.seq, t.rb, t.kt, t.idx};
+  }
+  void* tmp = nullptr;
+  const size_t bytes_seqs = align256(seqs.size() * sizeof(CustomSeq));
+  cudaError_t e = cudaMalloc(&tmp, bytes_seqs + tasks.size() * sizeof(RepackTask));
+  if (e != cudaSuccess) return cuda_status(e);
+  auto* d_seqs = reinterpret_cast<CustomSeq*>(tmp);
+  auto* d_tasks = reinterpret_cast<RepackTask*>(static_cast<char*>(tmp) + bytes_seqs);
+  e = cudaMemcpyAsync(d_seqs, seqs.data(), seqs.size() * sizeof(CustomSeq), cudaMemcpyHostToDevice, stream);
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(d_tasks, tasks.data(), tasks.size() * sizeof(RepackTask), cudaMemcpyHostToDevice, stream);
+  if (e == cudaSuccess)
+    e = launch_custom_repack(m->mask_bits, d_seqs, d_tasks, int(tasks.size()), R, d_tiles, stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+  cudaFree(tmp);
+  return cuda_status(e);
+}
+
+attn_status_t plan_impl(const attn_problem_t* problem, const attn_mask_desc_t* mask, cudaStream_t stream,
+                        attn_plan_t** out_plan) {
+  if (!out_plan) return ATTN_ERR_INVALID_ARG;
+  *out_plan = nullptr;
+  Shape s;
+  attn_status_t st = validate_problem(problem, s);
+  if (st != ATTN_OK) return st;
+  st = validate_mask(mask, s);
+  if (st != ATTN_OK) return st;
+
+  int dev = 0, num_sms = 148;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return ATTN_ERR_CUDA;
+
+  auto plan = new attn_plan_t();
+  plan->device = dev;
+  plan->batch = s.B;
+  plan->hq = s.hq;
+  plan->hkv = s.hkv;
+  plan->d = s.d;
+  plan->scale = s.scale;
+  plan->paged = s.paged;
+  plan->page_size = s.ps;
+  plan->max_pages = s.maxp;
+  plan->num_pages = s.npages;
+  plan->page_table = s.paged ? problem->page_table : nullptr;
+  plan->total_q = s.total_q;
+  plan->total_kv_rows = s.total_kv_rows;
+  plan->nq = s.d <= 128 ? 2 : 1;
+  plan->hp = choose_hp(s);
+  plan->R = kTile / plan->hp;
+  const int R = plan->R;
+
+  std::vector<std::vector<int32_t>> cnts(s.B);
+  RowSource src(mask, s);
+  if (mask->kind == ATTN_MASK_CUSTOM) {
+    st = custom_counts(mask, s, R, stream, cnts);
+    if (st != ATTN_OK) {
+      delete plan;
+      return st;
+    }
+  } else {
+    for (int b = 0; b < s.B; ++b) {
+      src.prepare(b);
+      count_sequence(src, b, s, R, cnts[b]);
+    }
+  }
+  for (int b = 0; b < s.B; ++b) report_classes(cnts[b], s.lq[b], s.lk[b], R, plan->classes, plan->stats);
+
+  WorkList wl;
+  build_work(s, R, plan->hp, plan->nq, cnts, num_sms, wl);
+  plan->ctas = int32_t(wl.cta_off.size()) - 1;
+  plan->stats.mask_tiles = int64_t(wl.mask_tiles.size());
+  plan->stats.work_items = int64_t(wl.items.size());
+  plan->stats.jobs = int64_t(wl.jobs.size());
+  plan->stats.ctas = plan->ctas;
+  plan->stats.heads_per_tile = plan->hp;
+  plan->stats.tiles_per_cta = plan->nq;
+
+  const Staging lay = layout(wl);
+  std::vector<char> host(lay.off_tiles, 0);
+  std::memcpy(host.data() + lay.off_items, wl.items.data(), wl.items.size() * sizeof(WorkItem));
+  std::memcpy(host.data() + lay.off_jobs, wl.jobs.data(), wl.jobs.size() * sizeof(Job));
+  std::memcpy(host.data() + lay.off_cta_off, wl.cta_off.data(), wl.cta_off.size() * sizeof(int32_t));
+  std::memcpy(host.data() + lay.off_cta_items, wl.cta_items.data(), wl.cta_items.size() * sizeof(int32_t));
+  std::vector<uint32_t> tiles;
+  if (mask->kind != ATTN_MASK_CUSTOM && !wl.mask_tiles.empty()) {
+    tiles.resize(wl.mask_tiles.size() * (kMaskTileBytes / 4));
+    int cur = -1;
+    for (const TileRef& t : wl.mask_tiles) {
+      if (t.seq != cur) {
+        src.prepare(t.seq);
+        cur = t.seq;
+      }
+      write_mask_tile(src, s, R, t, tiles.data() + size_t(t.idx) * (kMaskTileBytes / 4));
+    }
+  }
+
+  e = cudaMalloc(&plan->ws, lay.total);
+  if (e != cudaSuccess) {
+    delete plan;
+    return cuda_status(e);
+  }
+  plan->ws_bytes = lay.total;
+  char* base = static_cast<char*>(plan->ws);
+  plan->d_status = reinterpret_cast<int32_t*>(base);
+  plan->d_items = reinterpret_cast<const WorkItem*>(base + lay.off_items);
+  plan->d_jobs = reinterpret_cast<const Job*>(base + lay.off_jobs);
+  plan->d_cta_off = reinterpret_cast<const int32_t*>(base + lay.off_cta_off);
+  plan->d_cta_items = reinterpret_cast<const int32_t*>(base + lay.off_cta_items);
+  plan->d_mask_tiles = reinterpret_cast<const uint4*>(base + lay.off_tiles);
+  e = cudaMemcpyAsync(base, host.data(), host.size(), cudaMemcpyHostToDevice, stream);
+  if (e == cudaSuccess && !tiles.empty())
+    e = cudaMemcpyAsync(base + lay.off_tiles, tiles.data(), tiles.size() * 4, cudaMemcpyHostToDevice, stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+  st = cuda_status(e);
+  if (st == ATTN_OK && mask->kind == ATTN_MASK_CUSTOM)
+    st = custom_repack(mask, s, R, wl, reinterpret_cast<uint4*>(base + lay.off_tiles), stream);
+  if (st != ATTN_OK) {
+    cudaFree(plan->ws);
+    delete plan;
+    return st;
+  }
+  *out_plan = plan;
+  return ATTN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+attn_status_t attn_plan(const attn_problem_t* problem, const attn_mask_desc_t* mask, attn_stream_t stream,
+                        attn_plan_t** out_plan) {
+  try {
+    return plan_impl(problem, mask, reinterpret_cast<cudaStream_t>(stream), out_plan);
+  } catch (const std::bad_alloc&) {
+    return ATTN_ERR_OOM;
+  } catch (...) {
+    return ATTN_ERR_INVALID_ARG;
+  }
+}
+
+attn_status_t attn_masked_fwd(const attn_plan_t* plan, const void* q, const void* k, const void* v, void* out,
+                              float* lse, attn_stream_t stream) {
+  if (!plan) return ATTN_ERR_INVALID_ARG;
+  if (plan->total_q == 0) return ATTN_OK;
+  if (!q || !k || !v || !out) return ATTN_ERR_INVALID_ARG;
+  auto mis = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) != 0; };
+  if (mis(q) || mis(k) || mis(v) || mis(out) || (lse && (reinterpret_cast<uintptr_t>(lse) & 3)))
+    return ATTN_ERR_INVALID_ARG;
+  return mfa_launch_forward(plan, q, k, v, out, lse, reinterpret_cast<cudaStream_t>(stream));
+}
+
+attn_status_t attn_plan_get_tile_classes(const attn_plan_t* plan, uint8_t* host_dst, size_t n, size_t* n_needed) {
+  if (!plan) return ATTN_ERR_INVALID_ARG;
+  if (n_needed) *n_needed = plan->classes.size();
+  if (n && !host_dst) return ATTN_ERR_INVALID_ARG;
+  std::memcpy(host_dst, plan->classes.data(), std::min(n, plan->classes.size()));
+  return ATTN_OK;
+}
+
+attn_status_t attn_plan_get_stats(const attn_plan_t* plan, attn_plan_stats_t* stats) {
+  if (!plan || !stats) return ATTN_ERR_INVALID_ARG;
+  *stats = plan->stats;
+  return ATTN_OK;
+}
+
+attn_status_t attn_plan_check_status(const attn_plan_t* plan, attn_stream_t stream) {
+  if (!plan) return ATTN_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  int32_t host[4] = {0, 0, 0, 0};
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e == cudaSuccess) e = cudaMemcpy(host, plan->d_status, sizeof(host), cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess) e = cudaMemset(plan->d_status, 0, sizeof(host));
+  if (e != cudaSuccess) return ATTN_ERR_CUDA;
+  if (host[0] != 0) return ATTN_ERR_TIMEOUT;
+  return ATTN_OK;
+}
+
+attn_status_t attn_plan_set_debug(attn_plan_t* plan, int32_t flags, int64_t timeout_ns) {
+  if (!plan || flags < 0 || timeout_ns < 0) return ATTN_ERR_INVALID_ARG;
+  plan->debug_flags = flags;
+  plan->timeout_ns = timeout_ns > 0 ? timeout_ns : 2000000000LL;
+  return ATTN_OK;
+}
+
+attn_status_t attn_plan_destroy(attn_plan_t* plan) {
+  if (!plan) return ATTN_OK;
+  cudaError_t e = cudaSuccess;
+  if (plan->ws) e = cudaFree(plan->ws);
+  delete plan;
+  return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+attn_status_t attn_classify_host(const attn_problem_t* problem, const attn_mask_desc_t* mask, uint8_t* classes,
+                                 size_t n, size_t* n_needed, int64_t* unmasked_pairs) {
+  try {
+    Shape s;
+    attn_status_t st = validate_problem(problem, s, /*need_device_ptrs=*/false);
+    if (st != ATTN_OK) return st;
+    st = validate_mask(mask, s);
+    if (st != ATTN_OK) return st;
+    if (mask->kind == ATTN_MASK_CUSTOM) return ATTN_ERR_UNSUPPORTED;
+    RowSource src(mask, s);
+    std::vector<uint8_t> out;
+    attn_plan_stats_t stats{};
+    std::vector<int32_t> cnt;
+    for (int b = 0; b < s.B; ++b) {
+      src.prepare(b);
+      count_sequence(src, b, s, kTile, cnt);
+      report_classes(cnt, s.lq[b], s.lk[b], kTile, out, stats);
+    }
+    if (n_needed) *n_needed = out.size();
+    if (unmasked_pairs) *unmasked_pairs = stats.unmasked_pairs;
+    if (classes) std::memcpy(classes, out.data(), std::min(n, out.size()));
+    return ATTN_OK;
+  } catch (const std::bad_alloc&) {
+    return ATTN_ERR_OOM;
+  }
+}
+
+const char* attn_status_string(attn_status_t status) {
+  switch (status) {
+    case ATTN_OK: return "ok";
+    case ATTN_ERR_INVALID_ARG: return "invalid argument";
+    case ATTN_ERR_UNSUPPORTED: return "unsupported configuration";
+    case ATTN_ERR_MASK_TOO_SMALL: return "custom mask buffer too small for the lengths";
+    case ATTN_ERR_OOM: return "out of device memory";
+    case ATTN_ERR_CUDA: return "CUDA runtime error";
+    case ATTN_ERR_TIMEOUT: return "a bounded wait in the kernel expired";
+    default: return "unknown status";
+  }
+}
+
+}  // extern "C"
