@@ -1,0 +1,401 @@
+"""Benchmark of the masked attention forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config 1..5]
+
+Default workload: the Gemma2-style local/global pair -- 4 ragged sequences with lengths
+uniform in [1024, 8192] (seed 2), Hq=16, Hkv=8, d=256, bf16 N(0,1) inputs -- run with
+SLIDING_WINDOW(4096) and with CAUSAL on the same tensors. One step = both forwards.
+
+Metric: effective TFLOP/s = 4 * d * (unmasked pairs) * Hq / time, summed over the masks of
+the step (masked pairs are not counted). Prints ONE JSON line on rank 0.
+
+Multi-GPU (torchrun, one rank per GPU): every rank runs its own independent batch of the
+same workload (seed offset by rank); there is no collective on the data path. Timing is
+the max over ranks of CUDA-event time; the value is the work of all ranks / that time.
+
+--impl reference times the fp64 CPU oracle on a bounded row sample of the same workload
+(rank 0 only), the baseline arm of this build.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "effective masked-attn TFLOP/s (unmasked pairs) and % of B200 bf16 tensor peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_BYTES = 126 * 1024 * 1024
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured (MEASURED_PEAKS.json)"
+    return dict(FALLBACK_PEAKS), "fallback (no MEASURED_PEAKS.json)"
+
+
+def workload(cfg: int, rank: int):
+    import workloads as W
+    seed = cfg + 7919 * rank
+    return W.config(cfg, seed=seed)
+
+
+def flops_of(stats, wl):
+    return 4.0 * wl.d * stats["unmasked_pairs"] * wl.hq
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for f in ("attn_fwd.cu", "tmem_ldst.inc", "attn_internal.h"):
+        with open(os.path.join(ROOT, "masked_flash_attention_attn_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_for(workload_name):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on this kernel source."""
+    path = os.path.join(ROOT, "profiles", "fwd_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    e = d.get(workload_name)
+    if not e or e.get("kernel_source_hash") != kernel_source_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{device_index}.csv")
+        try:
+            import torch
+            uuid = "GPU-" + str(torch.cuda.get_device_properties(device_index).uuid)
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", uuid, f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.fh, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.fh.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                p = [x.strip() for x in line.split(",")]
+                if len(p) < 9:
+                    continue
+                try:
+                    rows.append((float(p[1]), float(p[2]), p[5:9]))
+                except ValueError:
+                    continue
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, r in rows for i in range(4) if r[i].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows)}
+
+
+def oracle_sample(wl, specs, budget_s, rows_per_block=128):
+    """Time the fp64 oracle on row blocks (one query head each, cycling through sequences,
+    heads and the masks of the step) until budget_s has passed. Returns (pairs*heads, seconds, desc)."""
+    import oracle
+    from oracle import masks as OM
+    from oracle import attention as OA
+    import torch
+    g = wl.hq // wl.hkv
+    pairs, t_used, blocks = 0, 0.0, 0
+    b_order = sorted(range(wl.batch), key=lambda b: -wl.lq(b))
+    kv = {}
+    while t_used < budget_s:
+        b = b_order[blocks % len(b_order)]
+        spec = specs[blocks % len(specs)]
+        h = (blocks // len(b_order)) % wl.hq
+        lq, lk = wl.lq(b), wl.lk(b)
+        r1 = lq - (blocks * 977) % max(1, lq - rows_per_block)
+        r0 = max(0, r1 - rows_per_block)
+        if b not in kv:
+            kk, vv = wl.kv_of_seq(b)
+            kv[b] = (kk.to(torch.float64).numpy(), vv.to(torch.float64).numpy())
+        kk, vv = kv[b]
+        q0 = int(wl.cu_seqlens_q[b])
+        t0 = time.perf_counter()
+        m = OM.dense_mask_rows(spec, b, lq, lk, r0, r1)
+        qq = wl.q[q0 + r0:q0 + r1, h].to(torch.float64).numpy()
+        OA.attention_one_head(qq, kk[:, h // g], vv[:, h // g], m, wl.scale)
+        t_used += time.perf_counter() - t0
+        pairs += int(m.sum())
+        blocks += 1
+    desc = (f"{blocks} blocks of <= {rows_per_block} query rows x 1 head over all keys, cycling the "
+            f"{len(specs)} masks of the step; fp64 NumPy")
+    return pairs, t_used, desc
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    wl = workload(args.config, 0)
+    specs = wl.masks
+    per_step = max(0.25, min(4.0, 150.0 / max(1, args.steps)))  # whole run within a few minutes
+    for _ in range(args.warmup):
+        oracle_sample(wl, specs, 0.2)
+    pairs, secs = 0, 0.0
+    desc = None
+    for _ in range(args.steps):
+        p, s, desc = oracle_sample(wl, specs, per_step)
+        pairs, secs = pairs + p, secs + s
+    flops = 4.0 * wl.d * pairs
+    val = flops / secs / 1e12
+    cores = blas_threads()
+    line = {"metric": METRIC, "value": val, "unit": "TFLOP/s", "impl": "reference", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / max(1, args.steps),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": config_of(wl, args, world),
+            "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                             "sample": f"{args.steps} steps x ~{per_step:.0f} s: {desc}"},
+            "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def config_of(wl, args, world):
+    tq = int(wl.cu_seqlens_q[-1])
+    tk = int(wl.cu_seqlens_k[-1]) if not wl.paged else int(wl.k_cache.shape[0] * wl.page_size)
+    in_bytes = 2 * (tq * wl.hq * wl.d + 2 * tk * wl.hkv * wl.d)
+    return {"workload": wl.name, "batch": wl.batch,
+            "lengths_q": [wl.lq(b) for b in range(wl.batch)][:64],
+            "hq": wl.hq, "hkv": wl.hkv, "head_dim": wl.d,
+            "masks": [m.kind + (f"({m.window})" if m.kind == "SLIDING_WINDOW" else "") for m in wl.masks],
+            "seed": wl.seed, "parallelism": f"dp{world} (independent batches, no collective)",
+            "l2": f"inputs {in_bytes / 2**20:.0f} MiB vs 126 MiB L2; no flush" if in_bytes > L2_BYTES
+            else "inputs fit L2; L2 flushed between steps"}
+
+
+def device_inputs(wl, dev):
+    q = wl.q.to(dev)
+    if wl.paged:
+        return q, wl.k_cache.to(dev), wl.v_cache.to(dev)
+    return q, wl.k.to(dev), wl.v.to(dev)
+
+
+def make_plan(M, wl, spec, dev):
+    import torch
+    kw = dict(hq=wl.hq, hkv=wl.hkv, head_dim=wl.d, cu_seqlens_q=wl.cu_seqlens_q, mask=spec, scale=wl.scale)
+    if wl.paged:
+        kw.update(kv_lens=wl.kv_lens, page_table=torch.from_numpy(wl.page_table).to(dev),
+                  page_size=wl.page_size, num_pages=wl.k_cache.shape[0])
+    else:
+        kw.update(cu_seqlens_k=wl.cu_seqlens_k)
+    return M.attn_plan(**kw)
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    import masked_flash_attention_attn_b200 as M
+
+    if not os.path.exists(M._LIB_PATH):
+        raise RuntimeError("libattn_b200.so is not built: run `python -m masked_flash_attention_attn_b200.build`")
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    wl = workload(args.config, rank)
+    stream = torch.cuda.current_stream()
+    q, k, v = device_inputs(wl, dev)
+    plans = [make_plan(M, wl, spec, dev) for spec in wl.masks]
+    stats = [M.attn_plan_get_stats(p) for p in plans]
+    flops = [flops_of(s, wl) for s in stats]
+    tq = q.shape[0]
+    outs = [torch.empty(tq, wl.hq, wl.d, dtype=torch.bfloat16, device=dev) for _ in plans]
+    lses = [torch.empty(tq, wl.hq, dtype=torch.float32, device=dev) for _ in plans]
+    in_bytes = q.numel() * 2 + k.numel() * 2 + v.numel() * 2
+    flush = torch.empty(256 * 2**20, dtype=torch.uint8, device=dev) if in_bytes <= L2_BYTES else None
+
+    def step(events=None):
+        for i, p in enumerate(plans):
+            if flush is not None:
+                flush.fill_(i)
+            if events is not None:
+                events[i][0].record(stream)
+            M.attn_masked_fwd(p, q, k, v, outs[i], lses[i], stream)
+            if events is not None:
+                events[i][1].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    for p in plans:
+        st = M.attn_plan_check_status(p)
+        if st != 0:
+            raise RuntimeError(f"forward reported {M.STATUS.get(st, st)}")
+    ev = [[[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in plans] for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local_rank)
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for s in range(args.steps):
+        step(ev[s])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    if world > 1:
+        dist.barrier()
+    ms = t_start.elapsed_time(t_end)
+    launch_ms = [[ev[s][i][0].elapsed_time(ev[s][i][1]) for s in range(args.steps)] for i in range(len(plans))]
+    for p in plans:
+        st = M.attn_plan_check_status(p)
+        if st != 0:
+            raise RuntimeError(f"forward reported {M.STATUS.get(st, st)}")
+
+    # ---- end to end through the public API: pinned host inputs in, results out, every step ----
+    hq_, hk_, hv_ = (t.cpu().pin_memory() for t in (q, k, v))
+    ho = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs]
+    hl = [torch.empty(l.shape, dtype=l.dtype).pin_memory() for l in lses]
+    e2e_steps = max(3, min(args.steps, 20))
+
+    def e2e_step():
+        q.copy_(hq_, non_blocking=True)
+        k.copy_(hk_, non_blocking=True)
+        v.copy_(hv_, non_blocking=True)
+        for i, p in enumerate(plans):
+            M.attn_masked_fwd(p, q, k, v, outs[i], lses[i], stream)
+            ho[i].copy_(outs[i], non_blocking=True)
+            hl[i].copy_(lses[i], non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    h2d = in_bytes
+    d2h = sum(o.numel() * 2 + l.numel() * 4 for o, l in zip(outs, lses))
+
+    # ---- reduce over ranks (reporting only) ----
+    step_flops = sum(flops)
+    tot = torch.tensor([ms, e2e_ms], dtype=torch.float64, device=dev)
+    work = torch.tensor([step_flops], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(tot, op=dist.ReduceOp.MAX)
+        dist.all_reduce(work, op=dist.ReduceOp.SUM)
+    ms, e2e_ms = float(tot[0]), float(tot[1])
+    total_flops = float(work[0])
+    if rank != 0:
+        return
+    value = total_flops * args.steps / (ms * 1e-3) / 1e12
+    e2e_val = total_flops * e2e_steps / (e2e_ms * 1e-3) / 1e12
+    pk, pk_src = peaks()
+    # the kernel runs back to back for the whole timed region: the sustained GEMM peak applies
+    peak = float(pk.get("bf16_tflops_sustained", pk.get("bf16_tflops")))
+    avg_launch_ms = sum(sum(x) for x in launch_ms) / sum(len(x) for x in launch_ms)
+    achieved = (sum(flops) / len(flops)) / (avg_launch_ms * 1e-3) / 1e12
+    tr = traffic_for(wl.name)
+    mask_bytes = sum(s["mask_tile_reads"] for s in stats) * 2048.0
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) bf16, lengths from seed)",
+        "config": config_of(wl, args, world),
+        "pct_of_peak": 100.0 * value / world / peak,
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": tr,
+                     "peak_source": pk_src + " bf16_tflops_sustained",
+                     "kernel": f"masked_attn_fwd_kernel d={wl.d}",
+                     "algorithmic_flops_per_launch": sum(flops) / len(flops),
+                     "avg_launch_ms": avg_launch_ms},
+        "per_mask": [{"mask": m.kind, "unmasked_pairs_per_head": s["unmasked_pairs"], "tflops_per_s":
+                      f / (statistics.mean(x) * 1e-3) / 1e12, "ms": statistics.mean(x),
+                      "tiles_e_f_p": [s["tiles_empty"], s["tiles_full"], s["tiles_partial"]]}
+                     for m, s, f, x in zip(wl.masks, stats, flops, launch_ms)],
+        "mask_gbs": mask_bytes / (sum(statistics.mean(x) for x in launch_ms) * 1e-3) / 1e9,
+        "e2e": {"value": e2e_val, "unit": "TFLOP/s", "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+                "steps": e2e_steps},
+        "gpu_launches": len(plans) * args.steps,
+        "clocks": clocks,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        pairs, secs, desc = oracle_sample(wl, wl.masks, args.cpu_seconds)
+        line["cpu_baseline"] = {"value": 4.0 * wl.d * pairs / secs / 1e12, "unit": "TFLOP/s",
+                                "cores": blas_threads(), "kind": "oracle", "sample": desc,
+                                "seconds": secs}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", type=int, default=2, choices=[1, 2, 3, 4, 5])
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

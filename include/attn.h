@@ -127,6 +127,7 @@ typedef struct {
   int64_t tiles_empty, tiles_full, tiles_partial; /* 128 x 128 tile classes over valid rectangles */
   int64_t mask_tiles;               /* 2 KiB tile-transposed mask tiles the forward reads */
   int64_t work_items, jobs;         /* forward work list: items and (item, key tile) jobs */
+  int64_t mask_tile_reads;          /* 2 KiB mask tiles one forward reads (per query tile and job) */
   int32_t ctas;                     /* persistent CTAs the forward launches */
   int32_t heads_per_tile;           /* query heads packed into one 128-row tile (short queries) */
   int32_t tiles_per_cta;            /* 128-row query tiles one CTA works on at once (1 or 2) */

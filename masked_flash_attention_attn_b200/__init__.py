@@ -56,7 +56,7 @@ class attn_problem_t(ctypes.Structure):
 class attn_plan_stats_t(ctypes.Structure):
     _fields_ = [("unmasked_pairs", ctypes.c_int64), ("tiles_empty", ctypes.c_int64), ("tiles_full", ctypes.c_int64),
                 ("tiles_partial", ctypes.c_int64), ("mask_tiles", ctypes.c_int64), ("work_items", ctypes.c_int64),
-                ("jobs", ctypes.c_int64), ("ctas", ctypes.c_int32), ("heads_per_tile", ctypes.c_int32),
+                ("jobs", ctypes.c_int64), ("mask_tile_reads", ctypes.c_int64), ("ctas", ctypes.c_int32), ("heads_per_tile", ctypes.c_int32),
                 ("tiles_per_cta", ctypes.c_int32), ("reserved", ctypes.c_int32)]
 
 

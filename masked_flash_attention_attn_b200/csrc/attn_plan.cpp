@@ -618,6 +618,8 @@ attn_status_t plan_impl(const attn_problem_t* problem, const attn_mask_desc_t* m
   plan->stats.mask_tiles = int64_t(wl.mask_tiles.size());
   plan->stats.work_items = int64_t(wl.items.size());
   plan->stats.jobs = int64_t(wl.jobs.size());
+  for (const Job& j : wl.jobs)
+    for (int t = 0; t < 2; ++t) plan->stats.mask_tile_reads += j.mask[t] >= 0 ? 1 : 0;
   plan->stats.ctas = plan->ctas;
   plan->stats.heads_per_tile = plan->hp;
   plan->stats.tiles_per_cta = plan->nq;
