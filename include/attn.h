@@ -54,7 +54,8 @@ typedef enum {
   ATTN_ERR_MASK_TOO_SMALL = 3, /* CUSTOM: the packed mask holds fewer words than the lengths need */
   ATTN_ERR_OOM = 4,            /* cudaMalloc of the plan workspace failed */
   ATTN_ERR_CUDA = 5,           /* any other CUDA runtime error (launch, copy, no device) */
-  ATTN_ERR_TIMEOUT = 6         /* a bounded wait inside the kernel expired (see attn_plan_check_status) */
+  ATTN_ERR_TIMEOUT = 6,        /* a bounded wait inside the kernel expired (see attn_plan_check_status) */
+  ATTN_ERR_TOO_LARGE = 7       /* attn_masked_fwd_noalloc: the work list and masks exceed its fixed scratch */
 } attn_status_t;
 
 typedef enum {
@@ -187,6 +188,33 @@ attn_status_t attn_classify_host(const attn_problem_t* problem, const attn_mask_
                                  int64_t* unmasked_pairs);
 
 const char* attn_status_string(attn_status_t status);
+
+/* Forward for callers that cannot allocate device memory. No page of the masked-attention
+ * pages has a counterpart of this call; it exists for embedders such as serving runtimes
+ * that own every device allocation through their own pool or are not allowed to call
+ * cudaMalloc / cudaFree at run time. It plans and runs in one call, like attn_plan()
+ * followed by attn_masked_fwd() and attn_plan_destroy(), but the work list, the partial-
+ * tile masks and the status word live in one fixed device array of
+ * ATTN_NOALLOC_SCRATCH_BYTES (32 MiB) inside the library, which every GPU that loads the
+ * library keeps until the process exits. It calls no cudaMalloc / cudaFree and no other
+ * device allocator; the host-side planning uses ordinary host memory.
+ *   - Arguments as in attn_plan() and attn_masked_fwd(); mask kinds FULL, CAUSAL,
+ *     SLIDING_WINDOW, PREFIX_LM, CHUNK_CAUSAL and RANGES (CUSTOM returns
+ *     ATTN_ERR_UNSUPPORTED: its device scan needs a workspace of its own).
+ *   - A problem whose plan needs more than the fixed array returns ATTN_ERR_TOO_LARGE
+ *     before any device work is enqueued.
+ *   - The plan is copied into the array on `stream` and the forward is enqueued behind it;
+ *     the call returns once the host copy source has been consumed.
+ *   - The first call on a device looks up the array's device address (once per device,
+ *     with that device current); make that first call before any stream capture.
+ *   - Every call reuses the same array and overwrites what the previous call left there
+ *     (the status word is cleared each time), so calls whose work overlaps on the GPU --
+ *     different streams, or another host thread -- race; serialise them on one stream.
+ * Errors: INVALID_ARG, UNSUPPORTED, TOO_LARGE, CUDA. */
+#define ATTN_NOALLOC_SCRATCH_BYTES (32u << 20)
+attn_status_t attn_masked_fwd_noalloc(const attn_problem_t* problem, const attn_mask_desc_t* mask,
+                                      const void* q, const void* k, const void* v, void* out, float* lse,
+                                      attn_stream_t stream);
 
 #ifdef __cplusplus
 }

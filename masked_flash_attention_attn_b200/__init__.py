@@ -18,7 +18,8 @@ _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libattn_b2
 
 ATTN_OK = 0
 STATUS = {0: "ATTN_OK", 1: "ATTN_ERR_INVALID_ARG", 2: "ATTN_ERR_UNSUPPORTED", 3: "ATTN_ERR_MASK_TOO_SMALL",
-          4: "ATTN_ERR_OOM", 5: "ATTN_ERR_CUDA", 6: "ATTN_ERR_TIMEOUT"}
+          4: "ATTN_ERR_OOM", 5: "ATTN_ERR_CUDA", 6: "ATTN_ERR_TIMEOUT", 7: "ATTN_ERR_TOO_LARGE"}
+NOALLOC_SCRATCH_BYTES = 32 << 20
 MASK_KIND = {"FULL": 0, "CAUSAL": 1, "SLIDING_WINDOW": 2, "PREFIX_LM": 3, "CHUNK_CAUSAL": 4, "RANGES": 5,
              "CUSTOM": 6}
 RANGE_FULL, RANGE_CAUSAL, RANGE_CHUNK_CAUSAL = 0, 1, 4
@@ -26,7 +27,7 @@ RANGE_FULL, RANGE_CAUSAL, RANGE_CHUNK_CAUSAL = 0, 1, 4
 # every symbol include/attn.h declares
 EXPORTS = ("attn_plan", "attn_masked_fwd", "attn_plan_get_tile_classes", "attn_plan_get_stats",
            "attn_plan_check_status", "attn_plan_set_debug", "attn_plan_destroy", "attn_classify_host",
-           "attn_status_string")
+           "attn_status_string", "attn_masked_fwd_noalloc")
 
 
 class AttnError(RuntimeError):
@@ -84,8 +85,11 @@ def lib() -> ctypes.CDLL:
                                          ctypes.POINTER(sz), ctypes.POINTER(i64)]
         L.attn_status_string.argtypes = [i32]
         L.attn_status_string.restype = ctypes.c_char_p
-        for n in EXPORTS[:-1]:
-            getattr(L, n).restype = i32
+        L.attn_masked_fwd_noalloc.argtypes = [ctypes.POINTER(attn_problem_t), ctypes.POINTER(attn_mask_desc_t),
+                                              vp, vp, vp, vp, vp, vp]
+        for n in EXPORTS:
+            if n != "attn_status_string":
+                getattr(L, n).restype = i32
         _lib = L
     return _lib
 
@@ -261,6 +265,23 @@ def attn_classify_host(*, hq: int, hkv: int, head_dim: int, cu_seqlens_q, mask, 
     _check(lib().attn_classify_host(ctypes.byref(pr), ctypes.byref(d), out.ctypes.data, n.value, None, None),
            "attn_classify_host")
     return out, int(pairs.value)
+
+
+def attn_masked_fwd_noalloc(*, hq: int, hkv: int, head_dim: int, cu_seqlens_q, mask, q, k, v, out, lse=None,
+                            cu_seqlens_k=None, kv_lens=None, page_table=None, page_size: int = 0,
+                            num_pages: int = 0, scale: float = 0.0, stream=None) -> None:
+    """attn_masked_fwd_noalloc(): plan + forward in one call without any device allocation.
+
+    For callers that may not allocate device memory (e.g. a runtime that owns every device
+    allocation through its own pool): the plan goes into a fixed 32 MiB array inside the
+    library instead of a cudaMalloc'd workspace. Calls that overlap on the GPU race on that
+    array; keep them on one stream. CUSTOM masks are not accepted here."""
+    m = _Marshal()
+    pr = _problem(m, hq=hq, hkv=hkv, head_dim=head_dim, cu_seqlens_q=cu_seqlens_q, cu_seqlens_k=cu_seqlens_k,
+                  kv_lens=kv_lens, page_table=page_table, page_size=page_size, num_pages=num_pages, scale=scale)
+    d = _mask_desc(m, mask)
+    _check(lib().attn_masked_fwd_noalloc(ctypes.byref(pr), ctypes.byref(d), _ptr(q), _ptr(k), _ptr(v), _ptr(out),
+                                         _ptr(lse), _stream(stream)), "attn_masked_fwd_noalloc")
 
 
 def attn_status_string(status: int) -> str:

@@ -655,3 +655,64 @@ attn_status_t mfa_launch_forward(const attn_plan_t* plan, const void* q, const v
     return plan->paged ? launch<Cfg<256, 1, 5, true>>(plan, p, stream) : launch<Cfg<256, 1, 5, false>>(plan, p, stream);
   }
 }
+
+// ---- allocation-free forward ------------------------------------------------------------
+// For embedders that may not allocate device memory: the plan of each call is copied into
+// this fixed array instead of a cudaMalloc'd workspace. Host code never dereferences the
+// symbol: it passes the address that cudaGetSymbolAddress returns for the current device.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[ATTN_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[kMaxDevices] = {};
+
+// Device address of g_noalloc_scratch on the current device, looked up once per device.
+attn_status_t noalloc_scratch(int dev, void** out) {
+  if (dev < 0 || dev >= kMaxDevices) return ATTN_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_addr[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) return ATTN_ERR_CUDA;
+    g_noalloc_addr[dev] = ptr;
+  }
+  *out = g_noalloc_addr[dev];
+  return ATTN_OK;
+}
+}  // namespace
+
+extern "C" attn_status_t attn_masked_fwd_noalloc(const attn_problem_t* problem, const attn_mask_desc_t* mask,
+                                                 const void* q, const void* k, const void* v, void* out,
+                                                 float* lse, attn_stream_t stream_handle) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_handle);
+  int dev = 0, num_sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  void* scratch = nullptr;
+  attn_status_t st = noalloc_scratch(dev, &scratch);
+  if (st != ATTN_OK) return st;
+  mfa_host_plan hp;
+  st = mfa_plan_host(problem, mask, num_sms, &hp);
+  if (st != ATTN_OK) return st;
+  if (hp.bytes.size() > size_t(ATTN_NOALLOC_SCRATCH_BYTES)) return ATTN_ERR_TOO_LARGE;
+  if (hp.meta.total_q == 0) return ATTN_OK;
+  if (!q || !k || !v || !out) return ATTN_ERR_INVALID_ARG;
+  auto mis = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) != 0; };
+  if (mis(q) || mis(k) || mis(v) || mis(out) || (lse && (reinterpret_cast<uintptr_t>(lse) & 3)))
+    return ATTN_ERR_INVALID_ARG;
+  // the bytes start with a zeroed status word: each call clears what the previous one left
+  if (cudaMemcpyAsync(scratch, hp.bytes.data(), hp.bytes.size(), cudaMemcpyHostToDevice, stream) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  char* base = static_cast<char*>(scratch);
+  attn_plan_t& plan = hp.meta;
+  plan.d_status = reinterpret_cast<int32_t*>(base);
+  plan.d_items = reinterpret_cast<const mfa::WorkItem*>(base + hp.off_items);
+  plan.d_jobs = reinterpret_cast<const mfa::Job*>(base + hp.off_jobs);
+  plan.d_cta_off = reinterpret_cast<const int32_t*>(base + hp.off_cta_off);
+  plan.d_cta_items = reinterpret_cast<const int32_t*>(base + hp.off_cta_items);
+  plan.d_mask_tiles = reinterpret_cast<const uint4*>(base + hp.off_tiles);
+  // (a copy from pageable host memory returns once the source has been staged, so the host
+  // bytes may go away when this function returns)
+  return mfa_launch_forward(&plan, q, k, v, out, lse, stream);
+}

@@ -93,6 +93,16 @@ struct attn_plan {
   int device = 0;
 };
 
+// Host-only plan used by attn_masked_fwd_noalloc: the bytes attn_plan would upload, laid
+// out as [status | items | jobs | cta_off | cta_items | mask tiles] from offset 0 (attn_plan.cpp).
+struct mfa_host_plan {
+  attn_plan_t meta;            // problem and kernel shape; device pointers left unset
+  std::vector<char> bytes;
+  size_t off_items = 0, off_jobs = 0, off_cta_off = 0, off_cta_items = 0, off_tiles = 0;
+};
+attn_status_t mfa_plan_host(const attn_problem_t* problem, const attn_mask_desc_t* mask, int num_sms,
+                            mfa_host_plan* out);
+
 // forward launcher (attn_fwd.cu)
 attn_status_t mfa_launch_forward(const attn_plan_t* plan, const void* q, const void* k, const void* v,
                                  void* out, float* lse, cudaStream_t stream);

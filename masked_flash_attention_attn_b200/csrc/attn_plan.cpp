@@ -674,6 +674,71 @@ attn_status_t plan_impl(const attn_problem_t* problem, const attn_mask_desc_t* m
 
 }  // namespace
 
+// Host-only planning for attn_masked_fwd_noalloc (analytic kinds): the same validation,
+// classification, work list and mask tiles as attn_plan, written into host bytes in the
+// workspace layout instead of a device allocation.
+attn_status_t mfa_plan_host(const attn_problem_t* problem, const attn_mask_desc_t* mask, int num_sms,
+                            mfa_host_plan* out) {
+  try {
+    if (mask && mask->kind == ATTN_MASK_CUSTOM) return ATTN_ERR_UNSUPPORTED;
+    Shape s;
+    attn_status_t st = validate_problem(problem, s);
+    if (st != ATTN_OK) return st;
+    st = validate_mask(mask, s);
+    if (st != ATTN_OK) return st;
+    attn_plan_t& m = out->meta;
+    m.batch = s.B;
+    m.hq = s.hq;
+    m.hkv = s.hkv;
+    m.d = s.d;
+    m.scale = s.scale;
+    m.paged = s.paged;
+    m.page_size = s.ps;
+    m.max_pages = s.maxp;
+    m.num_pages = s.npages;
+    m.page_table = s.paged ? problem->page_table : nullptr;
+    m.total_q = s.total_q;
+    m.total_kv_rows = s.total_kv_rows;
+    m.nq = s.d <= 128 ? 2 : 1;
+    m.hp = choose_hp(s);
+    m.R = kTile / m.hp;
+    const int R = m.R;
+    std::vector<std::vector<int32_t>> cnts(s.B);
+    RowSource src(mask, s);
+    for (int b = 0; b < s.B; ++b) {
+      src.prepare(b);
+      count_sequence(src, b, s, R, cnts[b]);
+    }
+    WorkList wl;
+    build_work(s, R, m.hp, m.nq, cnts, num_sms, wl);
+    m.ctas = int32_t(wl.cta_off.size()) - 1;
+    const Staging lay = layout(wl);
+    out->off_items = lay.off_items;
+    out->off_jobs = lay.off_jobs;
+    out->off_cta_off = lay.off_cta_off;
+    out->off_cta_items = lay.off_cta_items;
+    out->off_tiles = lay.off_tiles;
+    out->bytes.assign(lay.total, 0);
+    char* h = out->bytes.data();
+    std::memcpy(h + lay.off_items, wl.items.data(), wl.items.size() * sizeof(WorkItem));
+    std::memcpy(h + lay.off_jobs, wl.jobs.data(), wl.jobs.size() * sizeof(Job));
+    std::memcpy(h + lay.off_cta_off, wl.cta_off.data(), wl.cta_off.size() * sizeof(int32_t));
+    std::memcpy(h + lay.off_cta_items, wl.cta_items.data(), wl.cta_items.size() * sizeof(int32_t));
+    int cur = -1;
+    for (const TileRef& t : wl.mask_tiles) {
+      if (t.seq != cur) {
+        src.prepare(t.seq);
+        cur = t.seq;
+      }
+      write_mask_tile(src, s, R, t,
+                      reinterpret_cast<uint32_t*>(h + lay.off_tiles + size_t(t.idx) * kMaskTileBytes));
+    }
+    return ATTN_OK;
+  } catch (const std::bad_alloc&) {
+    return ATTN_ERR_OOM;
+  }
+}
+
 extern "C" {
 
 attn_status_t attn_plan(const attn_problem_t* problem, const attn_mask_desc_t* mask, attn_stream_t stream,
@@ -775,6 +840,7 @@ const char* attn_status_string(attn_status_t status) {
     case ATTN_ERR_OOM: return "out of device memory";
     case ATTN_ERR_CUDA: return "CUDA runtime error";
     case ATTN_ERR_TIMEOUT: return "a bounded wait in the kernel expired";
+    case ATTN_ERR_TOO_LARGE: return "the plan exceeds the fixed scratch of attn_masked_fwd_noalloc";
     default: return "unknown status";
   }
 }
