@@ -328,8 +328,15 @@ def run_ours(args, rank, world, local_rank):
     value = total_flops * args.steps / (ms * 1e-3) / 1e12
     e2e_val = total_flops * e2e_steps / (e2e_ms * 1e-3) / 1e12
     pk, pk_src = peaks()
-    # the kernel runs back to back for the whole timed region: the sustained GEMM peak applies
-    peak = float(pk.get("bf16_tflops_sustained", pk.get("bf16_tflops")))
+    # The timed regions here are short (well under the seconds a GEMM needs to settle at the
+    # power cap) and the SM clock stays near its maximum (see "clocks"), so the burst cuBLAS
+    # figure is the denominator; the sustained one is used only when the sampled clock fell
+    # below 90 % of the maximum.
+    burst = float(pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    sustained = float(pk.get("bf16_tflops_sustained", burst))
+    use_sustained = clocks is not None and clocks["sm_mhz"] < 0.9 * clocks["sm_max_mhz"]
+    peak = sustained if use_sustained else burst
+    pk_src += " bf16_tflops_sustained" if use_sustained else " bf16_tflops (burst)"
     avg_launch_ms = sum(sum(x) for x in launch_ms) / sum(len(x) for x in launch_ms)
     achieved = (sum(flops) / len(flops)) / (avg_launch_ms * 1e-3) / 1e12
     tr = traffic_for(wl.name)
@@ -342,7 +349,7 @@ def run_ours(args, rank, world, local_rank):
         "pct_of_peak": 100.0 * value / world / peak,
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": tr,
-                     "peak_source": pk_src + " bf16_tflops_sustained",
+                     "peak_source": pk_src,
                      "kernel": f"masked_attn_fwd_kernel d={wl.d}",
                      "algorithmic_flops_per_launch": sum(flops) / len(flops),
                      "avg_launch_ms": avg_launch_ms},

@@ -132,7 +132,7 @@ typedef struct {
   int32_t ctas;                     /* persistent CTAs the forward launches */
   int32_t heads_per_tile;           /* query heads packed into one 128-row tile (short queries) */
   int32_t tiles_per_cta;            /* 128-row query tiles one CTA works on at once (1 or 2) */
-  int32_t reserved;
+  int32_t cluster_size;             /* CTAs that cooperate on one work item (2: a pair of SMs) */
 } attn_plan_stats_t;
 
 /* Validate and plan. `stream` orders the plan's device work (the CUSTOM mask scan and

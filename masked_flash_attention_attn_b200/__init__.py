@@ -27,7 +27,7 @@ RANGE_FULL, RANGE_CAUSAL, RANGE_CHUNK_CAUSAL = 0, 1, 4
 # every symbol include/attn.h declares
 EXPORTS = ("attn_plan", "attn_masked_fwd", "attn_plan_get_tile_classes", "attn_plan_get_stats",
            "attn_plan_check_status", "attn_plan_set_debug", "attn_plan_destroy", "attn_classify_host",
-           "attn_status_string", "attn_masked_fwd_noalloc")
+           "attn_status_string", "attn_masked_fwd_noalloc", "attn_test_exp2_poly")
 
 
 class AttnError(RuntimeError):
@@ -58,7 +58,7 @@ class attn_plan_stats_t(ctypes.Structure):
     _fields_ = [("unmasked_pairs", ctypes.c_int64), ("tiles_empty", ctypes.c_int64), ("tiles_full", ctypes.c_int64),
                 ("tiles_partial", ctypes.c_int64), ("mask_tiles", ctypes.c_int64), ("work_items", ctypes.c_int64),
                 ("jobs", ctypes.c_int64), ("mask_tile_reads", ctypes.c_int64), ("ctas", ctypes.c_int32), ("heads_per_tile", ctypes.c_int32),
-                ("tiles_per_cta", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+                ("tiles_per_cta", ctypes.c_int32), ("cluster_size", ctypes.c_int32)]
 
 
 _lib = None
@@ -85,6 +85,7 @@ def lib() -> ctypes.CDLL:
                                          ctypes.POINTER(sz), ctypes.POINTER(i64)]
         L.attn_status_string.argtypes = [i32]
         L.attn_status_string.restype = ctypes.c_char_p
+        L.attn_test_exp2_poly.argtypes = [vp, vp, i64, vp]
         L.attn_masked_fwd_noalloc.argtypes = [ctypes.POINTER(attn_problem_t), ctypes.POINTER(attn_mask_desc_t),
                                               vp, vp, vp, vp, vp, vp]
         for n in EXPORTS:
@@ -231,7 +232,7 @@ def attn_plan_get_tile_classes(plan: Plan) -> np.ndarray:
 def attn_plan_get_stats(plan: Plan) -> dict:
     s = attn_plan_stats_t()
     _check(lib().attn_plan_get_stats(plan.handle, ctypes.byref(s)), "attn_plan_get_stats")
-    return {n: getattr(s, n) for n, _ in attn_plan_stats_t._fields_ if n != "reserved"}
+    return {n: getattr(s, n) for n, _ in attn_plan_stats_t._fields_}
 
 
 def attn_plan_check_status(plan: Plan, stream=None) -> int:
@@ -282,6 +283,11 @@ def attn_masked_fwd_noalloc(*, hq: int, hkv: int, head_dim: int, cu_seqlens_q, m
     d = _mask_desc(m, mask)
     _check(lib().attn_masked_fwd_noalloc(ctypes.byref(pr), ctypes.byref(d), _ptr(q), _ptr(k), _ptr(v), _ptr(out),
                                          _ptr(lse), _stream(stream)), "attn_masked_fwd_noalloc")
+
+
+def attn_test_exp2_poly(x, y, stream=None) -> None:
+    """Test hook: y = 2^x by the forward kernel's polynomial exp2 (device fp32 tensors)."""
+    _check(lib().attn_test_exp2_poly(_ptr(x), _ptr(y), int(x.numel()), _stream(stream)), "attn_test_exp2_poly")
 
 
 def attn_status_string(status: int) -> str:

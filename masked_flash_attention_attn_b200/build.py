@@ -30,10 +30,11 @@ def nvcc() -> str:
     return cand
 
 
-def _compile(src: str, verbose: bool) -> str:
-    obj = os.path.join(BUILD, src + ".o")
+def _compile(src: str, verbose: bool, defines=()) -> str:
+    obj = os.path.join(BUILD, src + "".join("." + d for d in defines) + ".o")
     cmd = [nvcc(), "-c", os.path.join(CSRC, src), "-o", obj, "-O3", "-std=c++17", "-lineinfo",
-           "-Xcompiler", "-fPIC", "-I", os.path.join(ROOT, "include"), "-I", CSRC, *ARCH]
+           "-Xcompiler", "-fPIC", "-I", os.path.join(ROOT, "include"), "-I", CSRC, *ARCH,
+           *[f"-D{d}" for d in defines]]
     if src.endswith(".cu"):
         cmd += ["-Xptxas", "-v"] if verbose else []
     else:
@@ -46,20 +47,24 @@ def _compile(src: str, verbose: bool) -> str:
     return obj
 
 
-def build(verbose: bool = False) -> str:
+def build(verbose: bool = False, defines=(), out: str = LIB) -> str:
+    """Compile and link; ``defines`` are extra NAME=VALUE macros, ``out`` the library path."""
     os.makedirs(BUILD, exist_ok=True)
     with cf.ThreadPoolExecutor(len(SOURCES)) as ex:
-        objs = list(ex.map(lambda s: _compile(s, verbose), SOURCES))
-    tmp = LIB + ".tmp"
+        objs = list(ex.map(lambda s: _compile(s, verbose, tuple(defines)), SOURCES))
+    tmp = out + ".tmp"
     cmd = [nvcc(), "-shared", "-o", tmp, *objs, *ARCH, "-lcudart_static", "-ldl", "-lpthread", "-lrt"]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, out)
+    return out
 
 
 if __name__ == "__main__":
     ap = argparse.ArgumentParser()
     ap.add_argument("--verbose", action="store_true")
-    print(build(ap.parse_args().verbose))
+    ap.add_argument("-D", dest="defines", action="append", default=[], help="extra macro NAME=VALUE")
+    ap.add_argument("--out", default=LIB)
+    a = ap.parse_args()
+    print(build(a.verbose, a.defines, a.out))

@@ -37,6 +37,7 @@
 #include <mutex>
 
 #include "attn_internal.h"
+#include "attn_testing.h"
 
 namespace mfa {
 namespace {
@@ -59,9 +60,10 @@ struct Params {
   int64_t timeout_ns;
 };
 
-template <int D_, int NQ_, int STAGES_, bool PAGED_>
+template <int D_, int NQ_, int STAGES_, bool PAGED_, int EMU_ = 0>
 struct Cfg {
   static constexpr int D = D_, NQ = NQ_, STAGES = STAGES_;
+  static constexpr int EMU = EMU_;               // of every 8 column pairs, EMU use exp2_poly
   static constexpr bool PAGED = PAGED_;
   static constexpr int CH = D < 128 ? D : 128;   // columns of one ring chunk
   static constexpr int NCH = D / CH;             // ring chunks per K or V tile
@@ -80,6 +82,10 @@ struct Cfg {
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;  // [0] TMEM base, [1] abort flag
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + slack to align the base to 1 KiB
   static constexpr int THREADS = 128 * (1 + NQ);
+  // register split for NQ = 2: 128 threads at REG_LOW, 256 at REG_HIGH
+  static constexpr bool REG_SPLIT = NQ == 2;
+  static constexpr int REG_LOW = 64, REG_HIGH = 208;
+  static constexpr int REG_SPLIT_TOTAL = 128 * REG_LOW + 128 * NQ * REG_HIGH;
   static constexpr int TM_O = 256;
   static constexpr uint32_t IDESC_QK =  // M=128, N=128, bf16 x bf16 -> fp32, both K-major
       (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(128 >> 3) << 17) | (uint32_t(128 >> 4) << 24);
@@ -136,24 +142,25 @@ __device__ __forceinline__ void st_volatile_shared(uint32_t addr, uint32_t v) {
 }
 
 struct Guard {
-  uint32_t abort_addr;
+  uint32_t abort_addr;       // this CTA's abort flag (shared::cta)
+  uint32_t abort_peer;       // the cluster peer's abort flag (shared::cluster), 0 when alone
   int32_t* status;
   int64_t timeout_ns;
 };
 
-// Slow path of wait_bounded: spin on try_wait until the phase completes, the shared abort
-// flag is raised (returns false) or timeout_ns passes (raises the flag, records `code`).
-__device__ __noinline__ bool wait_slow(uint32_t bar, uint32_t parity, uint32_t abort_addr, int32_t* status,
-                                       int64_t timeout_ns, int32_t code) {
+// Slow path of the bounded waits: spin until the phase completes, the abort flag is raised
+// (returns false) or timeout_ns passes (raises this CTA's and the peer's flags, records `code`).
+__device__ __forceinline__ bool wait_slow(uint32_t bar, uint32_t parity, const Guard& g, int32_t code) {
   const uint64_t t0 = gtime();
   while (true) {
 #pragma unroll 1
     for (int i = 0; i < 16; ++i)
       if (mbar_try_wait(bar, parity)) return true;
-    if (ld_volatile_shared(abort_addr) != 0u) return false;
-    if (gtime() - t0 > uint64_t(timeout_ns)) {
-      st_volatile_shared(abort_addr, 1u);
-      atomicCAS(status, 0, code);
+    if (ld_volatile_shared(g.abort_addr) != 0u) return false;
+    if (gtime() - t0 > uint64_t(g.timeout_ns)) {
+      st_volatile_shared(g.abort_addr, 1u);
+      if (g.abort_peer) asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(g.abort_peer), "r"(1u) : "memory");
+      atomicCAS(g.status, 0, code);
       return false;
     }
   }
@@ -162,12 +169,12 @@ __device__ __noinline__ bool wait_slow(uint32_t bar, uint32_t parity, uint32_t a
 // Wait for the phase of `parity` to complete; false when the CTA is aborting.
 __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, const Guard& g, int32_t code) {
   if (mbar_try_wait(bar, parity)) return true;
-  return wait_slow(bar, parity, g.abort_addr, g.status, g.timeout_ns, code);
+  return wait_slow(bar, parity, g, code);
 }
 
 // Wait without looking at the abort flag (used to let in-flight async work land before
 // the CTA exits); still bounded.
-__device__ __noinline__ void wait_drain(uint32_t bar, uint32_t parity, int64_t timeout_ns) {
+__device__ __forceinline__ void wait_drain(uint32_t bar, uint32_t parity, int64_t timeout_ns) {
   const uint64_t t0 = gtime();
   while (!mbar_try_wait(bar, parity)) {
     if (gtime() - t0 > uint64_t(timeout_ns)) return;
@@ -215,6 +222,79 @@ __device__ __forceinline__ void mma_commit(uint32_t bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
 }
 
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+// shared::cluster address of the same variable in cluster CTA `rank`
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Arrive on a barrier given by its shared::cluster address (this CTA's or the peer's).
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+// Warp-level publication of TMEM writes to the pair leader: every lane has waited for its
+// tcgen05.st and fenced them; after the warp converges one lane arrives (barrier count is
+// one per warp of both CTAs).
+__device__ __forceinline__ void warp_arrive_leader(uint32_t cluster_addr) {
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive_remote(cluster_addr);
+}
+
+// 2-SM MMA of a CTA pair (issued by the pair's leader): A rows split over the two CTAs,
+// B rows (N) split over the two CTAs, D rows split, all at the same offsets in both CTAs.
+__device__ __forceinline__ void mma2_ss(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(acc)
+      : "memory");
+}
+
+__device__ __forceinline__ void mma2_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc)
+      : "memory");
+}
+
+// arrive on the barrier at this offset in both CTAs of the pair when the MMAs complete
+__device__ __forceinline__ void mma2_commit_both(uint32_t bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(bar),
+      "h"(uint16_t(3))
+      : "memory");
+}
+
+__device__ __forceinline__ void mma2_commit_self(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+
+// TMA load into this CTA's shared memory whose completion is counted on the pair leader's
+// barrier (`bar` is a shared::cluster address); no multicast.
+__device__ __forceinline__ void tma2_load_3d(uint32_t dst, const CUtensorMap* tm, int32_t c0, int32_t c1, int32_t c2,
+                                             uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(
+          dst),
+      "l"(reinterpret_cast<uint64_t>(tm)), "r"(c0), "r"(c1), "r"(c2), "r"(bar)
+      : "memory");
+}
+
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
@@ -228,12 +308,195 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// 2^x on the FMA/ALU pipes, for the share of the softmax exponentials that the kernel takes
+// off the MUFU unit. Cody-Waite style reduction x = n + f, n = round(x) (the 1.5 * 2^23
+// addition leaves n in the low mantissa bits), f in [-1/2, 1/2]; 2^f by the degree-3
+// polynomial of least maximum relative error (Remez exchange; coefficients and the fit
+// are produced by gen_exp2_poly.py next to this file, max relative error 7.5e-5); 2^n is
+// applied by adding n to the exponent field. x is clamped at -125 so the result stays a
+// normal float (>= ~2e-38, i.e. zero for every use here).
+#define EXP2_POLY_C0 0x1.fff692p-1f  // 0.999928057
+#define EXP2_POLY_C1 0x1.62f31ap-1f  // 0.693260968
+#define EXP2_POLY_C2 0x1.f0de1ap-3f  // 0.242611125
+#define EXP2_POLY_C3 0x1.c3f76p-5f   // 0.0551716685
+__device__ __forceinline__ float exp2_poly(float x) {
+  x = fmaxf(x, -125.0f);
+  const float y = x + 12582912.0f;      // 1.5 * 2^23: y = 1.5 * 2^23 + round(x)
+  const float f = x - (y - 12582912.0f);
+  float p = fmaf(EXP2_POLY_C3, f, EXP2_POLY_C2);
+  p = fmaf(p, f, EXP2_POLY_C1);
+  p = fmaf(p, f, EXP2_POLY_C0);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(y) << 23));
+}
+
+// Packed fp32x2 arithmetic (sm_100): one instruction for two lanes of a float2.
+__device__ __forceinline__ uint64_t pk2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void unpk2(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
+// exp2_poly on a packed pair (same arithmetic as exp2_poly, two lanes per instruction).
+__device__ __forceinline__ uint64_t exp2_poly2(float x0, float x1) {
+  x0 = fmaxf(x0, -125.0f);
+  x1 = fmaxf(x1, -125.0f);
+  const uint64_t magic = pk2(12582912.0f, 12582912.0f);
+  const uint64_t x = pk2(x0, x1);
+  const uint64_t y = fadd2(x, magic);
+  const uint64_t nmagic = pk2(-12582912.0f, -12582912.0f);
+  const uint64_t r = fadd2(y, nmagic);             // round(x)
+  float r0, r1;
+  unpk2(r, r0, r1);
+  const uint64_t f = fadd2(x, pk2(-r0, -r1));      // x - round(x)
+  uint64_t p = ffma2(pk2(EXP2_POLY_C3, EXP2_POLY_C3), f, pk2(EXP2_POLY_C2, EXP2_POLY_C2));
+  p = ffma2(p, f, pk2(EXP2_POLY_C1, EXP2_POLY_C1));
+  p = ffma2(p, f, pk2(EXP2_POLY_C0, EXP2_POLY_C0));
+  float p0, p1, y0, y1;
+  unpk2(p, p0, p1);
+  unpk2(y, y0, y1);
+  return pk2(__int_as_float(__float_as_int(p0) + (__float_as_int(y0) << 23)),
+             __int_as_float(__float_as_int(p1) + (__float_as_int(y1) << 23)));
+}
+
 // Two fp32 -> one bf16x2 word (round to nearest even); `lo` lands in the low half, which
 // is the lower column / key index in every layout used here.
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
+}
+
+
+// ---- per-row softmax steps shared by both kernels ---------------------------------------
+// One thread owns one row (= one TMEM lane). m_run is the reference maximum in the
+// scaled log2 domain (scores * scale * log2 e); it is raised only when a tile's maximum
+// exceeds it by more than 8, so P <= 2^8 and O / l are rescaled rarely (exact either way:
+// O and l always share the same reference).
+struct RowState {
+  float m_run, l_run;
+};
+
+// S row (128 fp32 columns at t_s) -> masked online-softmax step -> P (bf16, written over
+// the first 64 columns of t_s). Returns the factor alpha by which O and l must be
+// multiplied (1 when the reference did not move); `need` tells whether it moved.
+template <int EMU>
+__device__ __forceinline__ float softmax_tile(uint32_t t_s, int mi, const uint4& bits, float sl2, RowState& st,
+                                              bool& need) {
+  float s[128];
+  {
+    uint32_t su[128];
+    tmem_ld32x32(t_s + 0, su + 0);
+    tmem_ld32x32(t_s + 32, su + 32);
+    tmem_ld32x32(t_s + 64, su + 64);
+    tmem_ld32x32(t_s + 96, su + 96);
+    tmem_wait_ld();
+#pragma unroll
+    for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(su[c]);
+  }
+  if (mi != kMaskFull) {
+    const uint32_t wv[4] = {bits.x, bits.y, bits.z, bits.w};
+#pragma unroll
+    for (int c = 0; c < 128; ++c)
+      if (!((wv[c >> 5] >> (c & 31)) & 1u)) s[c] = -INFINITY;
+  }
+  float mx = s[0];
+#pragma unroll
+  for (int c = 1; c < 128; ++c) mx = fmaxf(mx, s[c]);
+  const float m_new = mx * sl2;
+  need = m_new > st.m_run + 8.0f;
+  float alpha = 1.f;
+  if (need) {
+    alpha = ex2(st.m_run - m_new);
+    st.m_run = m_new;
+    st.l_run *= alpha;
+  }
+  const float mref = st.m_run == -INFINITY ? 0.f : st.m_run;
+  const uint64_t sl2x2 = pk2(sl2, sl2), nm2 = pk2(-mref, -mref);
+  uint64_t lsum2 = pk2(0.f, 0.f);
+#pragma unroll
+  for (int cc = 0; cc < 4; ++cc) {
+    uint32_t pk[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      float x0, x1;
+      unpk2(ffma2(pk2(s[cc * 32 + 2 * e], s[cc * 32 + 2 * e + 1]), sl2x2, nm2), x0, x1);
+      uint64_t p01;
+      if ((e & 7) < EMU) {
+        p01 = exp2_poly2(x0, x1);
+      } else {
+        p01 = pk2(ex2(x0), ex2(x1));
+      }
+      lsum2 = fadd2(lsum2, p01);
+      float p0, p1;
+      unpk2(p01, p0, p1);
+      pk[e] = pack_bf16(p0, p1);
+    }
+    tmem_st32x16(t_s + cc * 16, pk);
+  }
+  {
+    float a, b;
+    unpk2(lsum2, a, b);
+    st.l_run += a + b;
+  }
+  tmem_wait_st();
+  return alpha;
+}
+
+// O row (D fp32 columns at t_o) *= alpha; warp-collective.
+template <int D>
+__device__ __forceinline__ void rescale_o(uint32_t t_o, float alpha) {
+#pragma unroll 1
+  for (int cc = 0; cc < D / 32; ++cc) {
+    uint32_t o[32];
+    tmem_ld32x32(t_o + cc * 32, o);
+    tmem_wait_ld();
+#pragma unroll
+    for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+    tmem_st32x32(t_o + cc * 32, o);
+  }
+  tmem_wait_st();
+}
+
+// out = O / l (bf16), lse = ln 2 * (m + log2 l); rows that saw no key get 0 and -inf.
+// A row saw a key iff its reference maximum is finite (the polynomial exp2 leaves ~2^-125,
+// not 0, for masked entries, so l > 0 alone does not tell). Warp-collective TMEM reads;
+// the global stores are guarded by `valid`.
+template <int D>
+__device__ __forceinline__ void store_row(uint32_t t_o, const RowState& st, bool valid, int64_t row,
+                                          __nv_bfloat16* out, float* lse) {
+  const bool seen = st.m_run != -INFINITY;
+  const float inv = seen ? 1.f / st.l_run : 0.f;
+#pragma unroll 1
+  for (int cc = 0; cc < D / 32; ++cc) {
+    uint32_t o[32];
+    tmem_ld32x32(t_o + cc * 32, o);
+    tmem_wait_ld();
+    uint32_t pk[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e)
+      pk[e] = pack_bf16(__uint_as_float(o[2 * e]) * inv, __uint_as_float(o[2 * e + 1]) * inv);
+    if (valid) {
+      uint4* dst = reinterpret_cast<uint4*>(out + row * D + cc * 32);
+      dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+      dst[2] = make_uint4(pk[8], pk[9], pk[10], pk[11]);
+      dst[3] = make_uint4(pk[12], pk[13], pk[14], pk[15]);
+    }
+  }
+  if (valid && lse) lse[row] = seen ? (st.m_run + log2f(st.l_run)) * 0.69314718055994531f : -INFINITY;
 }
 
 // ---- the kernel ----------------------------------------------------------------------------
@@ -250,7 +513,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_fwd_kernel(const __
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem_raw + (sbase - raw) + C::OFF_MISC);
   const uint32_t bar0 = sbase + C::OFF_BAR;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const Guard guard{smem_u32(misc + 1), p.status, p.timeout_ns};
+  const Guard guard{smem_u32(misc + 1), 0u, p.status, p.timeout_ns};
 #define BAR(i) (bar0 + 8u * uint32_t(i))
 
   if (tid == 0) {
@@ -286,6 +549,10 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_fwd_kernel(const __
   const uint32_t tmem = misc[0];
   const int i_begin = p.cta_off[blockIdx.x], i_end = p.cta_off[blockIdx.x + 1];
 
+  // Registers move from the producer / MMA warpgroup to the softmax warpgroups (NQ = 2);
+  // the host launches only when the block's launch registers cover the split.
+  if (warp < 4) {
+  if constexpr (C::REG_SPLIT) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::REG_LOW));
   if (warp == 0) {
     // ================================ TMA producer ================================
     if (lane == 0) {
@@ -320,13 +587,18 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_fwd_kernel(const __
                             BAR(C::B_KVFULL + slot));
             } else {
               const int ps = p.page_size, ppt = 128 / ps;
-              for (int pg = 0; pg < ppt; ++pg) {
+              // all page ids of the tile are requested before the first is used
+              int32_t page[8];
+#pragma unroll
+              for (int pg = 0; pg < 8; ++pg) {
                 const int idx = kt * ppt + pg;
+                page[pg] = (pg < ppt && idx < it.npages) ? __ldg(p.page_table + it.k_base + idx) : -1;
+              }
+#pragma unroll
+              for (int pg = 0; pg < 8; ++pg) {
+                if (pg >= ppt) break;
                 int32_t row = p.num_pages * ps;  // fully out of bounds: the box reads zeros
-                if (idx < it.npages) {
-                  const int32_t page = __ldg(p.page_table + it.k_base + idx);
-                  if (page >= 0 && page < p.num_pages) row = page * ps;
-                }
+                if (page[pg] >= 0 && page[pg] < p.num_pages) row = page[pg] * ps;
                 for (int c = 0; c < C::NBOX; ++c)
                   tma_load_3d(dst + c * C::BOX_BYTES + pg * ps * 128, tm, h * C::CH + c * 64, it.kv_head, row,
                               BAR(C::B_KVFULL + slot));
@@ -374,18 +646,21 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_fwd_kernel(const __
           const uint32_t slot = (sj + t) & 1;
           const uint32_t qbase = sbase + C::OFF_Q + q * C::Q_BYTES;
 #pragma unroll
-          for (int kk = 0; kk < C::D / 16; ++kk) {
-            const int col = kk * 16;
-            const int h = col / C::CH, c = (col % C::CH) / 64, w = col % 64;
-            const uint64_t a = sdesc(qbase + (col / 64) * C::BOX_BYTES + w * 2, 16, 1024);
-            const uint64_t b = sdesc(sbase + C::OFF_RING + ((rk + h) % C::STAGES) * C::CHUNK_BYTES +
-                                         c * C::BOX_BYTES + w * 2,
-                                     16, 1024);
-            mma_ss(tmem + 128 * slot, a, b, C::IDESC_QK, kk > 0 ? 1u : 0u);
+          for (int h = 0; h < C::NCH; ++h) {
+#pragma unroll
+            for (int kq = 0; kq < C::CH / 16; ++kq) {
+              const int col = h * C::CH + kq * 16;
+              const int c = (col % C::CH) / 64, w = col % 64;
+              const uint64_t a = sdesc(qbase + (col / 64) * C::BOX_BYTES + w * 2, 16, 1024);
+              const uint64_t b = sdesc(sbase + C::OFF_RING + ((rk + h) % C::STAGES) * C::CHUNK_BYTES +
+                                           c * C::BOX_BYTES + w * 2,
+                                       16, 1024);
+              mma_ss(tmem + 128 * slot, a, b, C::IDESC_QK, col > 0 ? 1u : 0u);
+            }
+            // the chunk is free once these MMAs complete (commit tracks all earlier MMAs)
+            if (q == C::NQ - 1) mma_commit(BAR(C::B_KVEMPTY + (rk + h) % C::STAGES));
           }
           mma_commit(BAR(C::B_SFULL + slot));
-          if (q == C::NQ - 1)
-            for (int h = 0; h < C::NCH; ++h) mma_commit(BAR(C::B_KVEMPTY + (rk + h) % C::STAGES));
           if (t == T - 1) mma_commit(BAR(C::B_QEMPTY));
           return true;
         };
@@ -410,10 +685,9 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_fwd_kernel(const __
               mma_ts(tmem + C::TM_O + q * C::D + h * 128, tmem + 128 * slot + kk * 8, b, C::IDESC_PV,
                      (u < C::NQ && kk == 0) ? 0u : 1u);
             }
+            if (q == C::NQ - 1) mma_commit(BAR(C::B_KVEMPTY + (rv + h) % C::STAGES));
           }
           mma_commit(BAR(C::B_PVDONE + q));
-          if (q == C::NQ - 1)
-            for (int h = 0; h < C::NCH; ++h) mma_commit(BAR(C::B_KVEMPTY + (rv + h) % C::STAGES));
           return true;
         };
         bool ok = qk(0);
@@ -430,7 +704,9 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_fwd_kernel(const __
       wait_drain(BAR(C::B_DRAIN), 0, p.timeout_ns);
     }
     __syncwarp();
-  } else if (warp >= 4) {
+  }
+  } else {
+    if constexpr (C::REG_SPLIT) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(C::REG_HIGH));
     // ================================ softmax warpgroup ================================
     const int q = warp / 4 - 1;                       // query tile of this warpgroup
     const int r = tid - 128 * (1 + q);                // row of the tile = TMEM lane
@@ -442,7 +718,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_fwd_kernel(const __
     for (int ii = i_begin; ok && ii < i_end; ++ii) {
       const WorkItem it = p.items[p.cta_items[ii]];
       const int T = C::NQ * it.job_count;
-      float m_run = -INFINITY, l_run = 0.f;
+      RowState st{-INFINITY, 0.f};
       for (int t = q; t < T; t += C::NQ) {
         const uint32_t g = sj + t, slot = g & 1;
         const int mi = p.jobs[it.job_start + t / C::NQ].mask[q];
@@ -454,51 +730,8 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_fwd_kernel(const __
           break;
         }
         tc_fence_after();
-        const uint32_t t_s = tmem + lane_base + 128 * slot;
-        float s[128];
-        {
-          uint32_t su[128];
-          tmem_ld32x32(t_s + 0, su + 0);
-          tmem_ld32x32(t_s + 32, su + 32);
-          tmem_ld32x32(t_s + 64, su + 64);
-          tmem_ld32x32(t_s + 96, su + 96);
-          tmem_wait_ld();
-#pragma unroll
-          for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(su[c]);
-        }
-        if (mi != kMaskFull) {
-          const uint32_t wv[4] = {bits.x, bits.y, bits.z, bits.w};
-#pragma unroll
-          for (int c = 0; c < 128; ++c)
-            if (!((wv[c >> 5] >> (c & 31)) & 1u)) s[c] = -INFINITY;
-        }
-        float mx = s[0];
-#pragma unroll
-        for (int c = 1; c < 128; ++c) mx = fmaxf(mx, s[c]);
-        const float m_new = mx * sl2;
-        const bool need = m_new > m_run + 8.0f;
-        float alpha = 1.f;
-        if (need) {
-          alpha = ex2(m_run - m_new);
-          m_run = m_new;
-          l_run *= alpha;
-        }
-        const float mref = m_run == -INFINITY ? 0.f : m_run;
-        float lsum = 0.f;
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-          uint32_t pk[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const float p0 = ex2(fmaf(s[cc * 32 + 2 * e], sl2, -mref));
-            const float p1 = ex2(fmaf(s[cc * 32 + 2 * e + 1], sl2, -mref));
-            lsum += p0 + p1;
-            pk[e] = pack_bf16(p0, p1);
-          }
-          tmem_st32x16(t_s + cc * 16, pk);
-        }
-        l_run += lsum;
-        tmem_wait_st();
+        bool need;
+        const float alpha = softmax_tile<C::EMU>(tmem + lane_base + 128 * slot, mi, bits, sl2, st, need);
         if (t >= C::NQ) {
           // the previous P V of this tile must be done before O is touched or P is published
           if (!__all_sync(0xffffffffu, wait_bounded(BAR(C::B_PVDONE + q), pvc & 1, guard, kWaitPvDone))) {
@@ -507,49 +740,18 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_fwd_kernel(const __
           }
           ++pvc;
           tc_fence_after();
-          if (__any_sync(0xffffffffu, need)) {
-#pragma unroll 1
-            for (int cc = 0; cc < C::D / 32; ++cc) {
-              uint32_t o[32];
-              tmem_ld32x32(t_o + cc * 32, o);
-              tmem_wait_ld();
-#pragma unroll
-              for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-              tmem_st32x32(t_o + cc * 32, o);
-            }
-            tmem_wait_st();
-          }
+          if (__any_sync(0xffffffffu, need)) rescale_o<C::D>(t_o, alpha);
         }
         tc_fence_before();
         mbar_arrive(BAR(C::B_PFULL + slot));
       }
       if (!ok) break;
-      // ---- epilogue: out = O / l, lse = ln(2) (m + log2 l) ----
+      // ---- epilogue ----
       if (!__all_sync(0xffffffffu, wait_bounded(BAR(C::B_PVDONE + q), pvc & 1, guard, kWaitPvDone))) break;
       ++pvc;
       tc_fence_after();
       const int lr = r % p.R, hh = r / p.R;
-      const bool valid = lr < it.rows[q];
-      const int64_t row = int64_t(it.tok[q] + lr) * p.hq + it.head[q] + hh;
-      const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-#pragma unroll 1
-      for (int cc = 0; cc < C::D / 32; ++cc) {
-        uint32_t o[32];
-        tmem_ld32x32(t_o + cc * 32, o);
-        tmem_wait_ld();
-        uint32_t pk[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e)
-          pk[e] = pack_bf16(__uint_as_float(o[2 * e]) * inv, __uint_as_float(o[2 * e + 1]) * inv);
-        if (valid) {
-          uint4* dst = reinterpret_cast<uint4*>(p.out + row * C::D + cc * 32);
-          dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-          dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-          dst[2] = make_uint4(pk[8], pk[9], pk[10], pk[11]);
-          dst[3] = make_uint4(pk[12], pk[13], pk[14], pk[15]);
-        }
-      }
-      if (valid && p.lse) p.lse[row] = l_run > 0.f ? (m_run + log2f(l_run)) * 0.69314718055994531f : -INFINITY;
+      store_row<C::D>(t_o, st, lr < it.rows[q], int64_t(it.tok[q] + lr) * p.hq + it.head[q] + hh, p.out, p.lse);
       tc_fence_before();
       mbar_arrive(BAR(C::B_OEMPTY + q));
       sj += T;
@@ -562,6 +764,288 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_fwd_kernel(const __
   if (warp == 1) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem) : "memory");
 }
 
+// ================================ cluster-pair kernel (head_dim 256) ================================
+// Two CTAs on the two SMs of a pair cooperate on one work item: CTA r owns query tile r
+// (128 rows) and its TMEM rows; the pair's leader (r = 0) issues 2-SM MMAs of M = 256:
+//   S  = Q K^T : A = each CTA's Q tile, B = each CTA's HALF of the key tile (keys 64r..64r+63)
+//   O += P V   : A = each CTA's P (TMEM), B = each CTA's HALF of the value columns
+// so every CTA streams half of K and half of V per key tile, and one query tile per CTA
+// keeps two S buffers (the next S = Q K^T runs while the softmax works on the current one).
+// Both CTAs' TMA loads count on the leader's "full" barriers; the leader's commits arrive
+// on both CTAs' barriers; the softmax warpgroups of both CTAs arrive on the leader's "P
+// ready" and "O free" barriers. No TMA load multicasts.
+template <int D_, int STAGES_, bool PAGED_, int EMU_ = 0>
+struct PairCfg {
+  static constexpr int D = D_, STAGES = STAGES_, EMU = EMU_;
+  static constexpr bool PAGED = PAGED_;
+  static constexpr int QBOX = D / 64;              // 64-column boxes of a Q tile and of a K half
+  static constexpr int VBOX = D / 128;             // 64-column boxes of a V half (D / 2 columns)
+  static constexpr int Q_BYTES = QBOX * 128 * 128;
+  static constexpr int KH_BOX = 64 * 128;          // 64 keys x 128 bytes
+  static constexpr int VH_BOX = 128 * 128;         // 128 keys x 128 bytes
+  static constexpr int SLOT_BYTES = QBOX * KH_BOX; // == VBOX * VH_BOX
+  static_assert(QBOX * KH_BOX == VBOX * VH_BOX, "K and V halves fill one ring slot");
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_RING = Q_BYTES;
+  static constexpr int OFF_BAR = OFF_RING + STAGES * SLOT_BYTES;
+  static constexpr int B_QFULL = 0, B_QEMPTY = 1, B_KVFULL = 2, B_KVEMPTY = B_KVFULL + STAGES,
+                       B_SFULL = B_KVEMPTY + STAGES, B_PFULL = B_SFULL + 2, B_PVDONE = B_PFULL + 2,
+                       B_OEMPTY = B_PVDONE + 1, B_DRAIN = B_OEMPTY + 1, NBAR = B_DRAIN + 1;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
+  static constexpr int THREADS = 256;
+  static constexpr int TM_O = 256;
+  static constexpr uint32_t IDESC_QK =  // M=256 (pair), N=128, bf16 -> fp32, both K-major
+      (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(128 >> 3) << 17) | (uint32_t(256 >> 4) << 24);
+  static constexpr uint32_t IDESC_PV =  // M=256, N=D, A (P) from TMEM, B (V) MN-major
+      (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) | (uint32_t(D >> 3) << 17) | (uint32_t(256 >> 4) << 24);
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+  static_assert(256 + D <= 512, "TMEM budget");
+};
+
+template <class C>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::THREADS, 1)
+    masked_attn_fwd_pair_kernel(const __grid_constant__ Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t sbase = (raw + 1023u) & ~1023u;
+  uint32_t* misc = reinterpret_cast<uint32_t*>(smem_raw + (sbase - raw) + C::OFF_MISC);
+  const uint32_t bar0 = sbase + C::OFF_BAR;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+#define BAR(i) (bar0 + 8u * uint32_t(i))
+  const uint32_t lbar0 = mapa_shared(bar0, 0);   // the leader's barriers, cluster addresses
+#define LBAR(i) (lbar0 + 8u * uint32_t(i))
+  const Guard guard{smem_u32(misc + 1), mapa_shared(smem_u32(misc + 1), rank ^ 1u), p.status, p.timeout_ns};
+
+  if (tid == 0) {
+    mbar_init(BAR(C::B_QFULL), 1);
+    mbar_init(BAR(C::B_QEMPTY), 1);
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(BAR(C::B_KVFULL + s), 1);
+      mbar_init(BAR(C::B_KVEMPTY + s), 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(BAR(C::B_SFULL + s), 1);
+      mbar_init(BAR(C::B_PFULL + s), 8);   // one arrival per softmax warp of both CTAs
+    }
+    mbar_init(BAR(C::B_PVDONE), 1);
+    mbar_init(BAR(C::B_OEMPTY), 8);
+    mbar_init(BAR(C::B_DRAIN), 1);
+    misc[1] = 0u;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    prefetch_tmap(&p.tm_q);
+    prefetch_tmap(&p.tm_k);
+    prefetch_tmap(&p.tm_v);
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(smem_u32(misc))
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  cluster_sync();
+  tc_fence_after();
+  const uint32_t tmem = misc[0];
+  const int cl = blockIdx.x / 2;
+  const int i_begin = p.cta_off[cl], i_end = p.cta_off[cl + 1];
+
+  if (warp == 0) {
+    // ================================ TMA producer (both CTAs) ================================
+    if (lane == 0) {
+      uint32_t rc = 0;
+      int n = 0, q_last = -1;
+      for (int ii = i_begin; ii < i_end; ++ii, ++n) {
+        const WorkItem it = p.items[p.cta_items[ii]];
+        if (!wait_bounded(BAR(C::B_QEMPTY), (n & 1) ^ 1, guard, kWaitQEmpty)) break;
+        if (!((p.debug_flags & 1) && n == 0)) {
+          if (leader) mbar_expect_tx(BAR(C::B_QFULL), 2 * C::Q_BYTES);
+          q_last = n;
+          for (int hh = 0; hh < p.hp; ++hh)
+            for (int c = 0; c < C::QBOX; ++c)
+              tma2_load_3d(sbase + C::OFF_Q + c * 16384 + hh * p.R * 128, &p.tm_q, c * 64, it.head[rank] + hh,
+                           it.tok[rank], LBAR(C::B_QFULL));
+        }
+        const int T = it.job_count;
+        auto load_half = [&](bool is_v, int j) -> bool {
+          const int kt = p.jobs[it.job_start + j].k_tile;
+          const uint32_t slot = rc % C::STAGES;
+          if (!wait_bounded(BAR(C::B_KVEMPTY + slot), ((rc / C::STAGES) & 1) ^ 1, guard, kWaitKvEmpty)) return false;
+          if (leader) mbar_expect_tx(BAR(C::B_KVFULL + slot), 2 * C::SLOT_BYTES);
+          const uint32_t dst = sbase + C::OFF_RING + slot * C::SLOT_BYTES;
+          const uint32_t fb = LBAR(C::B_KVFULL + slot);
+          // K half: keys kt*128 + 64 rank .. +63, all D columns; V half: all 128 keys,
+          // columns rank*D/2 .. +D/2
+          const int key0 = kt * 128 + (is_v ? 0 : 64 * int(rank));
+          const int nkeys = is_v ? 128 : 64;
+          const int nbox = is_v ? C::VBOX : C::QBOX;
+          const int box_bytes = is_v ? C::VH_BOX : C::KH_BOX;
+          const int col0 = is_v ? int(rank) * (C::D / 2) : 0;
+          const CUtensorMap* tm = is_v ? &p.tm_v : &p.tm_k;
+          if constexpr (!C::PAGED) {
+            for (int c = 0; c < nbox; ++c)
+              tma2_load_3d(dst + c * box_bytes, tm, col0 + c * 64, it.kv_head, it.k_base + key0, fb);
+          } else {
+            const int ps = p.page_size;
+            const int rows = ps < nkeys ? ps : nkeys;  // rows per box
+            const int nb = nkeys / rows;               // boxes per 64-column block
+            int32_t page[8];
+#pragma unroll
+            for (int pg = 0; pg < 8; ++pg) {
+              const int idx = (key0 + pg * rows) / ps;
+              page[pg] = (pg < nb && idx < it.npages) ? __ldg(p.page_table + it.k_base + idx) : -1;
+            }
+#pragma unroll
+            for (int pg = 0; pg < 8; ++pg) {
+              if (pg >= nb) break;
+              int32_t row = p.num_pages * ps;  // fully out of bounds: the box reads zeros
+              if (page[pg] >= 0 && page[pg] < p.num_pages) row = page[pg] * ps + (key0 + pg * rows) % ps;
+              for (int c = 0; c < nbox; ++c)
+                tma2_load_3d(dst + c * box_bytes + pg * rows * 128, tm, col0 + c * 64, it.kv_head, row, fb);
+            }
+          }
+          ++rc;
+          return true;
+        };
+        bool ok = load_half(false, 0);
+        if (ok && T > 1) ok = load_half(false, 1);
+        for (int u = 0; ok && u < T; ++u) {
+          ok = load_half(true, u);
+          if (ok && u + 2 < T) ok = load_half(false, u + 2);
+        }
+        if (!ok) break;
+      }
+      // let the copies land before the CTA may exit: the leader's barriers count both CTAs' bytes
+      if (leader) {
+        for (uint32_t r = rc > uint32_t(C::STAGES) ? rc - C::STAGES : 0u; r < rc; ++r)
+          wait_drain(BAR(C::B_KVFULL + r % C::STAGES), (r / C::STAGES) & 1, p.timeout_ns);
+        if (q_last >= 0) wait_drain(BAR(C::B_QFULL), q_last & 1, p.timeout_ns);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ================================ MMA issuer (leader only) ================================
+    if (lane == 0 && leader) {
+      uint32_t rc = 0, sj = 0;
+      int n = 0;
+      for (int ii = i_begin; ii < i_end; ++ii, ++n) {
+        const WorkItem it = p.items[p.cta_items[ii]];
+        if (!wait_bounded(BAR(C::B_QFULL), n & 1, guard, kWaitQFull)) break;
+        tc_fence_after();
+        const int T = it.job_count;
+        auto qk = [&](int t) -> bool {
+          const uint32_t slot = (sj + t) & 1, rk = rc;
+          if (!wait_bounded(BAR(C::B_KVFULL + rc % C::STAGES), (rc / C::STAGES) & 1, guard, kWaitKvFull))
+            return false;
+          ++rc;
+          tc_fence_after();
+          const uint32_t kb = sbase + C::OFF_RING + (rk % C::STAGES) * C::SLOT_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < C::D / 16; ++kk) {
+            const int col = kk * 16;
+            const uint64_t a = sdesc(sbase + C::OFF_Q + (col / 64) * 16384 + (col % 64) * 2, 16, 1024);
+            const uint64_t b = sdesc(kb + (col / 64) * C::KH_BOX + (col % 64) * 2, 16, 1024);
+            mma2_ss(tmem + 128 * slot, a, b, C::IDESC_QK, kk > 0 ? 1u : 0u);
+          }
+          mma2_commit_both(BAR(C::B_KVEMPTY + rk % C::STAGES));
+          mma2_commit_both(BAR(C::B_SFULL + slot));
+          if (t == T - 1) mma2_commit_both(BAR(C::B_QEMPTY));
+          return true;
+        };
+        auto pv = [&](int u) -> bool {
+          const uint32_t g = sj + u, slot = g & 1, rv = rc;
+          if (!wait_bounded(BAR(C::B_PFULL + slot), (g >> 1) & 1, guard, kWaitPFull)) return false;
+          if (u == 0 && !wait_bounded(BAR(C::B_OEMPTY), (n & 1) ^ 1, guard, kWaitOEmpty)) return false;
+          if (!wait_bounded(BAR(C::B_KVFULL + rc % C::STAGES), (rc / C::STAGES) & 1, guard, kWaitKvFull))
+            return false;
+          ++rc;
+          tc_fence_after();
+          const uint32_t vb = sbase + C::OFF_RING + (rv % C::STAGES) * C::SLOT_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint64_t b = sdesc(vb + kk * 2048, C::VH_BOX, 1024);
+            mma2_ts(tmem + C::TM_O, tmem + 128 * slot + kk * 8, b, C::IDESC_PV, (u == 0 && kk == 0) ? 0u : 1u);
+          }
+          mma2_commit_both(BAR(C::B_KVEMPTY + rv % C::STAGES));
+          mma2_commit_both(BAR(C::B_PVDONE));
+          return true;
+        };
+        bool ok = qk(0);
+        if (ok && T > 1) ok = qk(1);
+        for (int u = 0; ok && u < T; ++u) {
+          ok = pv(u);
+          if (ok && u + 2 < T) ok = qk(u + 2);
+        }
+        if (!ok) break;
+        sj += T;
+      }
+      mma2_commit_self(BAR(C::B_DRAIN));
+      wait_drain(BAR(C::B_DRAIN), 0, p.timeout_ns);
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ================================ softmax warpgroup (both CTAs) ================================
+    const int r = tid - 128;
+    const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
+    const uint32_t t_o = tmem + lane_base + C::TM_O;
+    const float sl2 = p.scale_log2;
+    uint32_t sj = 0, pvc = 0;
+    bool ok = true;
+    for (int ii = i_begin; ok && ii < i_end; ++ii) {
+      const WorkItem it = p.items[p.cta_items[ii]];
+      const int T = it.job_count;
+      RowState st{-INFINITY, 0.f};
+      for (int t = 0; t < T; ++t) {
+        const uint32_t g = sj + t, slot = g & 1;
+        const int mi = p.jobs[it.job_start + t].mask[rank];
+        uint4 bits = make_uint4(0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu);
+        if (mi >= 0) bits = __ldg(p.mask_tiles + int64_t(mi) * 128 + r);
+        else if (mi == kMaskNone) bits = make_uint4(0u, 0u, 0u, 0u);
+        if (!__all_sync(0xffffffffu, wait_bounded(BAR(C::B_SFULL + slot), (g >> 1) & 1, guard, kWaitSFull))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        bool need;
+        const float alpha = softmax_tile<C::EMU>(tmem + lane_base + 128 * slot, mi, bits, sl2, st, need);
+        if (t >= 1) {
+          if (!__all_sync(0xffffffffu, wait_bounded(BAR(C::B_PVDONE), pvc & 1, guard, kWaitPvDone))) {
+            ok = false;
+            break;
+          }
+          ++pvc;
+          tc_fence_after();
+          if (__any_sync(0xffffffffu, need)) rescale_o<C::D>(t_o, alpha);
+        }
+        tc_fence_before();
+        warp_arrive_leader(LBAR(C::B_PFULL + slot));
+      }
+      if (!ok) break;
+      if (!__all_sync(0xffffffffu, wait_bounded(BAR(C::B_PVDONE), pvc & 1, guard, kWaitPvDone))) break;
+      ++pvc;
+      tc_fence_after();
+      const int lr = r % p.R, hh = r / p.R;
+      store_row<C::D>(t_o, st, lr < it.rows[rank], int64_t(it.tok[rank] + lr) * p.hq + it.head[rank] + hh, p.out,
+                      p.lse);
+      tc_fence_before();
+      warp_arrive_leader(LBAR(C::B_OEMPTY));
+      sj += T;
+    }
+  }
+#undef LBAR
+#undef BAR
+  tc_fence_before();
+  cluster_sync();
+  tc_fence_after();
+  if (warp == 1) asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, 512;" ::"r"(tmem) : "memory");
+}
+
+__global__ void exp2_poly_kernel(const float* __restrict__ x, float* __restrict__ y, int64_t n) {
+  for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < n; i += int64_t(gridDim.x) * blockDim.x)
+    y[i] = exp2_poly(x[i]);
+}
+
 // Rows of a problem without any key at all: out = 0, lse = -inf.
 __global__ void fill_empty_kernel(float* lse, int64_t n) {
   for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < n; i += int64_t(gridDim.x) * blockDim.x)
@@ -569,6 +1053,11 @@ __global__ void fill_empty_kernel(float* lse, int64_t n) {
 }
 
 // ---- host side ---------------------------------------------------------------------------
+
+// Column pairs (of every 8) whose exponentials the d <= 128 kernels take off the MUFU unit.
+#ifndef MFA_EMU_D128
+#define MFA_EMU_D128 0
+#endif
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -599,12 +1088,33 @@ template <class C>
 attn_status_t launch(const attn_plan_t* plan, Params& p, cudaStream_t stream) {
   static std::once_flag once;
   static cudaError_t attr = cudaSuccess;
+  static bool regs_ok = true;
   std::call_once(once, [] {
     attr = cudaFuncSetAttribute(masked_attn_fwd_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 C::SMEM_BYTES);
+    if (attr == cudaSuccess && C::REG_SPLIT) {
+      // setmaxnreg.inc draws on the registers the block was launched with: the split must fit
+      cudaFuncAttributes fa{};
+      attr = cudaFuncGetAttributes(&fa, masked_attn_fwd_kernel<C>);
+      regs_ok = attr == cudaSuccess && fa.numRegs * C::THREADS >= C::REG_SPLIT_TOTAL;
+    }
+  });
+  if (attr != cudaSuccess || !regs_ok) return ATTN_ERR_CUDA;
+  masked_attn_fwd_kernel<C><<<plan->ctas, C::THREADS, C::SMEM_BYTES, stream>>>(p);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+template <class C>
+attn_status_t launch_pair(const attn_plan_t* plan, Params& p, cudaStream_t stream) {
+  static std::once_flag once;
+  static cudaError_t attr = cudaSuccess;
+  std::call_once(once, [] {
+    attr = cudaFuncSetAttribute(masked_attn_fwd_pair_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                C::SMEM_BYTES);
   });
   if (attr != cudaSuccess) return ATTN_ERR_CUDA;
-  masked_attn_fwd_kernel<C><<<plan->ctas, C::THREADS, C::SMEM_BYTES, stream>>>(p);
+  // grid = 2 CTAs per work unit; the kernel's cluster shape (2, 1, 1) is compiled in
+  masked_attn_fwd_pair_kernel<C><<<2 * plan->ctas, C::THREADS, C::SMEM_BYTES, stream>>>(p);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
@@ -625,10 +1135,13 @@ attn_status_t mfa_launch_forward(const attn_plan_t* plan, const void* q, const v
     return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
   }
   Params p{};
-  const uint32_t kv_box = plan->paged ? uint32_t(plan->page_size) : 128u;
+  // rows per K / V box: a page, a whole 128-key tile, or (pair kernel) a 64-key half tile
+  const uint32_t ps = uint32_t(plan->page_size);
+  uint32_t k_box = plan->paged ? ps : 128u, v_box = k_box;
+  if (plan->cluster == 2) k_box = k_box < 64u ? k_box : 64u;
   if (!encode3d(&p.tm_q, q, D, plan->hq, plan->total_q, uint32_t(plan->R)) ||
-      !encode3d(&p.tm_k, k, D, plan->hkv, plan->total_kv_rows, kv_box) ||
-      !encode3d(&p.tm_v, v, D, plan->hkv, plan->total_kv_rows, kv_box))
+      !encode3d(&p.tm_k, k, D, plan->hkv, plan->total_kv_rows, k_box) ||
+      !encode3d(&p.tm_v, v, D, plan->hkv, plan->total_kv_rows, v_box))
     return ATTN_ERR_CUDA;
   p.items = plan->d_items;
   p.jobs = plan->d_jobs;
@@ -648,12 +1161,22 @@ attn_status_t mfa_launch_forward(const attn_plan_t* plan, const void* q, const v
   p.scale_log2 = plan->scale * 1.4426950408889634f;
   p.timeout_ns = plan->timeout_ns;
   if (D == 64) {
-    return plan->paged ? launch<Cfg<64, 2, 10, true>>(plan, p, stream) : launch<Cfg<64, 2, 10, false>>(plan, p, stream);
+    return plan->paged ? launch<Cfg<64, 2, 10, true, MFA_EMU_D128>>(plan, p, stream)
+                       : launch<Cfg<64, 2, 10, false, MFA_EMU_D128>>(plan, p, stream);
   } else if (D == 128) {
-    return plan->paged ? launch<Cfg<128, 2, 5, true>>(plan, p, stream) : launch<Cfg<128, 2, 5, false>>(plan, p, stream);
+    return plan->paged ? launch<Cfg<128, 2, 5, true, MFA_EMU_D128>>(plan, p, stream)
+                       : launch<Cfg<128, 2, 5, false, MFA_EMU_D128>>(plan, p, stream);
   } else {
-    return plan->paged ? launch<Cfg<256, 1, 5, true>>(plan, p, stream) : launch<Cfg<256, 1, 5, false>>(plan, p, stream);
+    return plan->paged ? launch_pair<PairCfg<256, 5, true>>(plan, p, stream)
+                       : launch_pair<PairCfg<256, 5, false>>(plan, p, stream);
   }
+}
+
+extern "C" attn_status_t attn_test_exp2_poly(const float* x, float* y, int64_t n, attn_stream_t stream) {
+  if (n < 0 || (n > 0 && (!x || !y))) return ATTN_ERR_INVALID_ARG;
+  if (n == 0) return ATTN_OK;
+  mfa::exp2_poly_kernel<<<296, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(x, y, n);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
 // ---- allocation-free forward ------------------------------------------------------------

@@ -71,7 +71,8 @@ struct attn_plan {
   const int32_t* page_table = nullptr;   // device
   int64_t total_q = 0, total_kv_rows = 0;
   // kernel shape
-  int32_t nq = 1;        // query tiles per CTA
+  int32_t nq = 1;        // query tiles per work item
+  int32_t cluster = 1;   // CTAs per work item (2: the cluster-pair kernel, one tile per CTA)
   int32_t hp = 1;        // heads packed per query tile
   int32_t R = 128;       // rows per head in a query tile
   int32_t ctas = 0;

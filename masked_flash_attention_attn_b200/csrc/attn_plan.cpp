@@ -470,6 +470,11 @@ Staging layout(const WorkList& wl) {
   return st;
 }
 
+// Kernel shape: every work item holds two 128-row query tiles; head_dim 256 runs them on a
+// pair of SMs (one tile per CTA, 2-SM MMAs: each SM streams half of K and V), head_dim 64
+// and 128 on one SM (two softmax warpgroups share its exponential unit better; measured).
+void choose_shape(const Shape& s, attn_plan_t& m);
+
 int choose_hp(const Shape& s) {
   const int g = s.hq / s.hkv;
   int lmax = 0;
@@ -477,6 +482,13 @@ int choose_hp(const Shape& s) {
   int hp = 1;
   while (hp * 2 <= g && g % (hp * 2) == 0 && kTile / (hp * 2) >= std::max(lmax, 8)) hp *= 2;
   return hp;
+}
+
+void choose_shape(const Shape& s, attn_plan_t& m) {
+  m.nq = 2;
+  m.cluster = s.d == 256 ? 2 : 1;
+  m.hp = choose_hp(s);
+  m.R = kTile / m.hp;
 }
 
 attn_status_t cuda_status(cudaError_t e) {
@@ -591,9 +603,7 @@ attn_status_t plan_impl(const attn_problem_t* problem, const attn_mask_desc_t* m
   plan->page_table = s.paged ? problem->page_table : nullptr;
   plan->total_q = s.total_q;
   plan->total_kv_rows = s.total_kv_rows;
-  plan->nq = s.d <= 128 ? 2 : 1;
-  plan->hp = choose_hp(s);
-  plan->R = kTile / plan->hp;
+  choose_shape(s, *plan);
   const int R = plan->R;
 
   std::vector<std::vector<int32_t>> cnts(s.B);
@@ -613,16 +623,17 @@ attn_status_t plan_impl(const attn_problem_t* problem, const attn_mask_desc_t* m
   for (int b = 0; b < s.B; ++b) report_classes(cnts[b], s.lq[b], s.lk[b], R, plan->classes, plan->stats);
 
   WorkList wl;
-  build_work(s, R, plan->hp, plan->nq, cnts, num_sms, wl);
-  plan->ctas = int32_t(wl.cta_off.size()) - 1;
+  build_work(s, R, plan->hp, plan->nq, cnts, num_sms / plan->cluster, wl);
+  plan->ctas = int32_t(wl.cta_off.size()) - 1;   // work units: CTAs, or CTA pairs
   plan->stats.mask_tiles = int64_t(wl.mask_tiles.size());
   plan->stats.work_items = int64_t(wl.items.size());
   plan->stats.jobs = int64_t(wl.jobs.size());
   for (const Job& j : wl.jobs)
     for (int t = 0; t < 2; ++t) plan->stats.mask_tile_reads += j.mask[t] >= 0 ? 1 : 0;
-  plan->stats.ctas = plan->ctas;
+  plan->stats.ctas = plan->ctas * plan->cluster;
   plan->stats.heads_per_tile = plan->hp;
-  plan->stats.tiles_per_cta = plan->nq;
+  plan->stats.tiles_per_cta = plan->nq / plan->cluster;
+  plan->stats.cluster_size = plan->cluster;
 
   const Staging lay = layout(wl);
   std::vector<char> host(lay.off_tiles, 0);
@@ -699,9 +710,7 @@ attn_status_t mfa_plan_host(const attn_problem_t* problem, const attn_mask_desc_
     m.page_table = s.paged ? problem->page_table : nullptr;
     m.total_q = s.total_q;
     m.total_kv_rows = s.total_kv_rows;
-    m.nq = s.d <= 128 ? 2 : 1;
-    m.hp = choose_hp(s);
-    m.R = kTile / m.hp;
+    choose_shape(s, m);
     const int R = m.R;
     std::vector<std::vector<int32_t>> cnts(s.B);
     RowSource src(mask, s);
@@ -710,7 +719,7 @@ attn_status_t mfa_plan_host(const attn_problem_t* problem, const attn_mask_desc_
       count_sequence(src, b, s, R, cnts[b]);
     }
     WorkList wl;
-    build_work(s, R, m.hp, m.nq, cnts, num_sms, wl);
+    build_work(s, R, m.hp, m.nq, cnts, num_sms / m.cluster, wl);
     m.ctas = int32_t(wl.cta_off.size()) - 1;
     const Staging lay = layout(wl);
     out->off_items = lay.off_items;

@@ -157,3 +157,21 @@ def test_bounded_wait_timeout_reports_and_context_survives():
     assert M.attn_plan_check_status(plan) == 0
     ref_o, ref_l = oracle.masked_attention(wl, wl.masks[0])
     G.compare(out.float().cpu(), lse.cpu(), ref_o, ref_l, "after timeout")
+
+
+def test_exp2_polynomial_error_bound():
+    """The FMA-pipe exp2 used for part of the softmax: relative error <= 7.5e-5 (the Remez fit's
+    bound, plus fp32 evaluation rounding) against fp64 2^x on the range the softmax feeds it,
+    tiny and exact-zero behaviour below it."""
+    import masked_flash_attention_attn_b200 as M
+    x = torch.cat([torch.linspace(-120.0, 8.0, 2_000_001), torch.tensor([-125.0, -1e4, -float("inf"), 0.0, 1.0])])
+    xd = x.cuda()
+    y = torch.empty_like(xd)
+    M.attn_test_exp2_poly(xd, y)
+    y = y.cpu().double()
+    ref = torch.exp2(x.double())
+    body = x >= -120
+    rel = ((y[body] - ref[body]).abs() / ref[body]).max().item()
+    assert rel <= 8e-5, rel
+    assert torch.all(y[~body] <= 2.0 ** -120) and torch.all(y[~body] >= 0)
+    assert y[-2].item() == pytest.approx(1.0, rel=8e-5) and y[-1].item() == pytest.approx(2.0, rel=8e-5)
