@@ -209,6 +209,19 @@ def config_of(wl, args, world):
             else "inputs fit L2; L2 flushed between steps"}
 
 
+def reduce_over_ranks(times_ms, work, device):
+    """Max over ranks of each timing and sum over ranks of the work (for the JSON line only;
+    nothing on the data path is exchanged)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(list(times_ms), dtype=torch.float64, device=device)
+    w = torch.tensor([float(work)], dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        dist.all_reduce(w, op=dist.ReduceOp.SUM)
+    return [float(x) for x in t], float(w[0])
+
+
 def device_inputs(wl, dev):
     q = wl.q.to(dev)
     if wl.paged:
@@ -315,14 +328,7 @@ def run_ours(args, rank, world, local_rank):
     d2h = sum(o.numel() * 2 + l.numel() * 4 for o, l in zip(outs, lses))
 
     # ---- reduce over ranks (reporting only) ----
-    step_flops = sum(flops)
-    tot = torch.tensor([ms, e2e_ms], dtype=torch.float64, device=dev)
-    work = torch.tensor([step_flops], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(tot, op=dist.ReduceOp.MAX)
-        dist.all_reduce(work, op=dist.ReduceOp.SUM)
-    ms, e2e_ms = float(tot[0]), float(tot[1])
-    total_flops = float(work[0])
+    (ms, e2e_ms), total_flops = reduce_over_ranks([ms, e2e_ms], sum(flops), dev)
     if rank != 0:
         return
     value = total_flops * args.steps / (ms * 1e-3) / 1e12
@@ -374,7 +380,7 @@ def run_ours(args, rank, world, local_rank):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", type=int, default=2, choices=[1, 2, 3, 4, 5])

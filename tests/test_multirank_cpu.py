@@ -1,0 +1,58 @@
+"""Multi-rank host logic of bench.py on CPU: two gloo ranks (world size 2).
+
+Each rank runs an independent batch (no data-path collective); only the report is reduced:
+the max over ranks of the timings and the sum of the work. The reference arm runs on rank 0
+only; other ranks return without work."""
+import multiprocessing as mp
+import os
+import socket
+
+import pytest
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import torch.distributed as dist
+    import bench
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        times, work = bench.reduce_over_ranks([1.0 + rank, 10.0 * (rank + 1)], 100.0 * (rank + 1), "cpu")
+        seed_notes = bench.workload(2, rank).notes
+        q.put((rank, times, work, seed_notes))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_rank_reduction_and_independent_batches():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=240) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, times, work, _ in res:
+        assert times == [2.0, 20.0]          # max over ranks
+        assert work == 300.0                 # sum over ranks
+    assert res[0][3] != res[1][3]            # every rank draws its own batch
+
+
+def test_reference_arm_runs_on_rank0_only(capsys):
+    import argparse
+    import bench
+    bench.run_reference(argparse.Namespace(config=2, steps=1, warmup=0), rank=1, world=2)
+    assert capsys.readouterr().out == ""
+
+
+def test_single_process_reduction_is_identity():
+    import bench
+    assert bench.reduce_over_ranks([3.0, 4.0], 7.0, "cpu") == ([3.0, 4.0], 7.0)
