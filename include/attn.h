@@ -68,11 +68,15 @@ typedef enum {
   ATTN_MASK_CUSTOM = 6          /* bit-packed boolean mask, per sequence, shared by all heads */
 } attn_mask_kind_t;
 
-/* Range types. 0 and 1 are the attn_type_map values FULL and CAUSAL printed on the
- * chunk-causal feature request; 4 is this library's code for CHUNK_CAUSAL. */
+/* Range types. 0-3 are the attn_type_map values FULL, CAUSAL, INV_CAUSAL and BI_CAUSAL
+ * printed on the chunk-causal feature request (Why existing mask types are not enough:
+ * BI_CAUSAL is an "aligned band/intersection"); 4 is this library's code for CHUNK_CAUSAL. */
 typedef enum {
   ATTN_RANGE_FULL = 0,          /* every (i, j) in q_range x k_range */
   ATTN_RANGE_CAUSAL = 1,        /* and j <= i, both in sequence-local coordinates */
+  ATTN_RANGE_INV_CAUSAL = 2,    /* and j - k_start >= i - q_start (triangle aligned to the top-left corner) */
+  ATTN_RANGE_BI_CAUSAL = 3,     /* INV_CAUSAL and j - k_end <= i - q_end (the band between the
+                                   top-left and bottom-right aligned diagonals) */
   ATTN_RANGE_CHUNK_CAUSAL = 4   /* query chunk c = (i - q_start) / chunk_size sees keys
                                    [k_start, min(q_start + (c+1)*chunk_size, q_end)) within k_range */
 } attn_range_type_t;

@@ -22,7 +22,7 @@ STATUS = {0: "ATTN_OK", 1: "ATTN_ERR_INVALID_ARG", 2: "ATTN_ERR_UNSUPPORTED", 3:
 NOALLOC_SCRATCH_BYTES = 32 << 20
 MASK_KIND = {"FULL": 0, "CAUSAL": 1, "SLIDING_WINDOW": 2, "PREFIX_LM": 3, "CHUNK_CAUSAL": 4, "RANGES": 5,
              "CUSTOM": 6}
-RANGE_FULL, RANGE_CAUSAL, RANGE_CHUNK_CAUSAL = 0, 1, 4
+RANGE_FULL, RANGE_CAUSAL, RANGE_INV_CAUSAL, RANGE_BI_CAUSAL, RANGE_CHUNK_CAUSAL = 0, 1, 2, 3, 4
 
 # every symbol include/attn.h declares
 EXPORTS = ("attn_plan", "attn_masked_fwd", "attn_plan_get_tile_classes", "attn_plan_get_stats",

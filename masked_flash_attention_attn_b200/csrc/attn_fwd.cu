@@ -190,6 +190,23 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* tm,
       : "memory");
 }
 
+// L2 eviction priority for the pair kernel's TMA loads: K/V tiles are re-read by every
+// query tile of their (sequence, head), Q tiles once per item (measured: +0.7 % at d=256;
+// the single-CTA kernel loads without hints, where they measured neutral to -3.5 %).
+#ifndef MFA_L2_HINTS
+#define MFA_L2_HINTS 1
+#endif
+__device__ __forceinline__ uint64_t l2_policy_evict_last() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* tm) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tm)) : "memory");
 }
@@ -292,6 +309,16 @@ __device__ __forceinline__ void tma2_load_3d(uint32_t dst, const CUtensorMap* tm
       "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(
           dst),
       "l"(reinterpret_cast<uint64_t>(tm)), "r"(c0), "r"(c1), "r"(c2), "r"(bar)
+      : "memory");
+}
+
+__device__ __forceinline__ void tma2_load_3d_hint(uint32_t dst, const CUtensorMap* tm, int32_t c0, int32_t c1,
+                                                  int32_t c2, uint32_t bar, uint64_t pol) {
+  if (!MFA_L2_HINTS) return tma2_load_3d(dst, tm, c0, c1, c2, bar);
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(
+          dst),
+      "l"(reinterpret_cast<uint64_t>(tm)), "r"(c0), "r"(c1), "r"(c2), "r"(bar), "l"(pol)
       : "memory");
 }
 
@@ -854,6 +881,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::THREADS, 1)
   if (warp == 0) {
     // ================================ TMA producer (both CTAs) ================================
     if (lane == 0) {
+      const uint64_t pol_kv = l2_policy_evict_last(), pol_q = l2_policy_evict_first();
       uint32_t rc = 0;
       int n = 0, q_last = -1;
       for (int ii = i_begin; ii < i_end; ++ii, ++n) {
@@ -864,8 +892,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::THREADS, 1)
           q_last = n;
           for (int hh = 0; hh < p.hp; ++hh)
             for (int c = 0; c < C::QBOX; ++c)
-              tma2_load_3d(sbase + C::OFF_Q + c * 16384 + hh * p.R * 128, &p.tm_q, c * 64, it.head[rank] + hh,
-                           it.tok[rank], LBAR(C::B_QFULL));
+              tma2_load_3d_hint(sbase + C::OFF_Q + c * 16384 + hh * p.R * 128, &p.tm_q, c * 64, it.head[rank] + hh,
+                                it.tok[rank], LBAR(C::B_QFULL), pol_q);
         }
         const int T = it.job_count;
         auto load_half = [&](bool is_v, int j) -> bool {
@@ -885,7 +913,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::THREADS, 1)
           const CUtensorMap* tm = is_v ? &p.tm_v : &p.tm_k;
           if constexpr (!C::PAGED) {
             for (int c = 0; c < nbox; ++c)
-              tma2_load_3d(dst + c * box_bytes, tm, col0 + c * 64, it.kv_head, it.k_base + key0, fb);
+              tma2_load_3d_hint(dst + c * box_bytes, tm, col0 + c * 64, it.kv_head, it.k_base + key0, fb, pol_kv);
           } else {
             const int ps = p.page_size;
             const int rows = ps < nkeys ? ps : nkeys;  // rows per box
@@ -902,7 +930,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::THREADS, 1)
               int32_t row = p.num_pages * ps;  // fully out of bounds: the box reads zeros
               if (page[pg] >= 0 && page[pg] < p.num_pages) row = page[pg] * ps + (key0 + pg * rows) % ps;
               for (int c = 0; c < nbox; ++c)
-                tma2_load_3d(dst + c * box_bytes + pg * rows * 128, tm, col0 + c * 64, it.kv_head, row, fb);
+                tma2_load_3d_hint(dst + c * box_bytes + pg * rows * 128, tm, col0 + c * 64, it.kv_head, row, fb,
+                                  pol_kv);
             }
           }
           ++rc;

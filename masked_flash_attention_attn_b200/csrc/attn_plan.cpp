@@ -108,7 +108,8 @@ attn_status_t validate_problem(const attn_problem_t* p, Shape& s, bool need_devi
 
 bool range_ok(const attn_range_t& r) {
   if (r.q_start < 0 || r.q_end < r.q_start || r.k_start < 0 || r.k_end < r.k_start) return false;
-  if (r.type != ATTN_RANGE_FULL && r.type != ATTN_RANGE_CAUSAL && r.type != ATTN_RANGE_CHUNK_CAUSAL)
+  if (r.type != ATTN_RANGE_FULL && r.type != ATTN_RANGE_CAUSAL && r.type != ATTN_RANGE_INV_CAUSAL &&
+      r.type != ATTN_RANGE_BI_CAUSAL && r.type != ATTN_RANGE_CHUNK_CAUSAL)
     return false;
   if (r.type == ATTN_RANGE_CHUNK_CAUSAL && r.chunk_size < 1) return false;
   return true;
@@ -197,6 +198,10 @@ class RowSource {
         int64_t lo = std::max<int64_t>(r.k_start, 0), hi = std::min<int64_t>(r.k_end, lk);
         if (r.type == ATTN_RANGE_CAUSAL) {
           hi = std::min<int64_t>(hi, int64_t(i) + 1);
+        } else if (r.type == ATTN_RANGE_INV_CAUSAL || r.type == ATTN_RANGE_BI_CAUSAL) {
+          lo = std::max<int64_t>(lo, int64_t(r.k_start) + (int64_t(i) - r.q_start));
+          if (r.type == ATTN_RANGE_BI_CAUSAL)
+            hi = std::min<int64_t>(hi, int64_t(r.k_end) - (int64_t(r.q_end) - i) + 1);
         } else if (r.type == ATTN_RANGE_CHUNK_CAUSAL) {
           int64_t c = (int64_t(i) - r.q_start) / r.chunk_size;
           int64_t end = std::min<int64_t>(int64_t(r.q_start) + (c + 1) * int64_t(r.chunk_size), r.q_end);

@@ -18,7 +18,13 @@ Sources for each kind
                   Attention", Current pattern / Proposed API: a list of
                   (q_range, k_range, type) whose union is the mask.
                   FULL: every (i, j) in q_range x k_range; CAUSAL: additionally
-                  j <= i in sequence-local coordinates.
+                  j <= i in sequence-local coordinates. The same page names
+                  INV_CAUSAL and BI_CAUSAL (attn_type_map 2, 3; "Why existing mask
+                  types are not enough": BI_CAUSAL is an aligned band/intersection):
+                  INV_CAUSAL keeps j - k_start >= i - q_start (the causal triangle
+                  aligned to the top-left corner of the range rectangle); BI_CAUSAL
+                  additionally keeps j - k_end <= i - q_end (bottom-right aligned
+                  causal), i.e. the band between the two aligned diagonals.
   CHUNK_CAUSAL    same page, Desired representation: query chunk c of
                   [q_start + c*cs, q_start + (c+1)*cs) attends keys
                   [k_start, q_start + (c+1)*cs), the chunk end clipped to q_end
@@ -34,7 +40,7 @@ from __future__ import annotations
 import numpy as np
 
 CLASS_EMPTY, CLASS_FULL, CLASS_PARTIAL = 0, 1, 2
-R_FULL, R_CAUSAL, R_CHUNK = 0, 1, 4
+R_FULL, R_CAUSAL, R_INV_CAUSAL, R_BI_CAUSAL, R_CHUNK = 0, 1, 2, 3, 4
 TILE = 128
 
 
@@ -64,6 +70,10 @@ def _range_or_into(m: np.ndarray, rng, r0: int, r1: int) -> None:
         sub = np.ones((b - a, d - c), dtype=bool)
     elif typ == R_CAUSAL:
         sub = j <= i
+    elif typ == R_INV_CAUSAL:
+        sub = (j - ks) >= (i - qs)
+    elif typ == R_BI_CAUSAL:
+        sub = ((j - ks) >= (i - qs)) & ((j - ke) <= (i - qe))
     elif typ == R_CHUNK:
         ch = (i - qs) // cs
         end = np.minimum(qs + (ch + 1) * cs, qe)

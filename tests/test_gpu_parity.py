@@ -175,3 +175,25 @@ def test_exp2_polynomial_error_bound():
     assert rel <= 8e-5, rel
     assert torch.all(y[~body] <= 2.0 ** -120) and torch.all(y[~body] >= 0)
     assert y[-2].item() == pytest.approx(1.0, rel=8e-5) and y[-1].item() == pytest.approx(2.0, rel=8e-5)
+
+
+@pytest.mark.parametrize("d", [128, 256])
+def test_inv_and_bi_causal_ranges(d):
+    """The INV_CAUSAL / BI_CAUSAL range types on non-square, overlapping ranges."""
+    rng = np.random.default_rng(d)
+    lq = np.array([300, 517, 129])
+    lk = np.array([420, 517, 700])
+    ranges = []
+    for b in range(3):
+        rs = []
+        for t in (W.RANGE_INV_CAUSAL, W.RANGE_BI_CAUSAL, W.RANGE_BI_CAUSAL, W.RANGE_FULL):
+            a, c = sorted(rng.integers(0, lq[b] + 1, size=2).tolist())
+            e, f = sorted(rng.integers(0, lk[b] + 1, size=2).tolist())
+            rs.append((a, c, e, f, t, 0))
+        ranges.append(rs)
+    gen = torch.Generator().manual_seed(d)
+    cq, ck = W.cu_from_lengths(lq), W.cu_from_lengths(lk)
+    wl = W.Workload(name="invbi", hq=4, hkv=2, d=d, scale=1.0 / np.sqrt(d), cu_seqlens_q=cq,
+                    q=W.randn_bf16(gen, int(cq[-1]), 4, d), masks=[W.MaskSpec("RANGES", ranges=ranges)],
+                    cu_seqlens_k=ck, k=W.randn_bf16(gen, int(ck[-1]), 2, d), v=W.randn_bf16(gen, int(ck[-1]), 2, d))
+    G.check_full(wl, wl.masks[0], f"inv/bi d={d}")

@@ -258,3 +258,38 @@ def test_tile_classes_ragged_valid_rectangle():
     # pos(i) = i - 1: rows 128, 129 of tile (1,1) see key 128 only for i = 129
     assert list(OM.tile_classes(spec, [(130, 129)])) == [2, 0, 1, 2]
     assert list(OM.tile_classes(spec, [(0, 5)])) == []
+
+
+# ---- INV_CAUSAL and BI_CAUSAL range types (the page names them; readings in the header) ----
+
+def _one_range(typ, qs, qe, ks, ke, L=None):
+    L = L or max(qe, ke)
+    return OM.dense_mask(_ranges_spec([[(qs, qe, ks, ke, typ, 0)]]), 0, L, L)
+
+
+def test_inv_causal_square_is_transposed_causal():
+    L = 37
+    inv = _one_range(W.RANGE_INV_CAUSAL, 0, L, 0, L)
+    ca = _one_range(W.RANGE_CAUSAL, 0, L, 0, L)
+    assert np.array_equal(inv, ca.T)
+    assert np.array_equal(inv | ca, np.ones((L, L), bool))     # together they cover the square
+    assert np.array_equal(inv & ca, np.eye(L, dtype=bool))     # and meet on the diagonal
+
+
+def test_bi_causal_is_an_aligned_band():
+    # square: the band of width 1 is the diagonal; with L_k - L_q = 5 every row keeps 6 keys
+    assert np.array_equal(_one_range(W.RANGE_BI_CAUSAL, 0, 20, 0, 20), np.eye(20, dtype=bool))
+    m = _one_range(W.RANGE_BI_CAUSAL, 3, 13, 2, 17, L=20)
+    rows = m.sum(1)
+    assert list(rows[3:13]) == [6] * 10 and rows[:3].sum() == 0 and rows[13:].sum() == 0
+    for i in range(3, 13):
+        keys = np.nonzero(m[i])[0]
+        # top-left aligned lower edge, bottom-right aligned upper edge
+        assert keys[0] == 2 + (i - 3) and keys[-1] == 16 - (12 - i)
+    # BI = INV_CAUSAL and the bottom-right aligned causal triangle (equal to CAUSAL here: k_end = q_end)
+    inv = _one_range(W.RANGE_INV_CAUSAL, 4, 15, 1, 15, L=15)
+    ca = _one_range(W.RANGE_CAUSAL, 4, 15, 1, 15, L=15)
+    assert np.array_equal(_one_range(W.RANGE_BI_CAUSAL, 4, 15, 1, 15, L=15), inv & ca)
+    # a band is not prefix + chunk-local attention (the page's point)
+    cc = OM.dense_mask(_ranges_spec([[(0, 20, 0, 20, W.RANGE_CHUNK_CAUSAL, 2)]]), 0, 20, 20)
+    assert not np.array_equal(_one_range(W.RANGE_BI_CAUSAL, 0, 20, 0, 20), cc)

@@ -40,10 +40,12 @@ from typing import List, Optional, Sequence, Tuple
 import numpy as np
 import torch
 
-# range types of the range-list descriptor (0/1 follow the attn_type_map values
-# printed on the chunk-causal page; 4 is this library's code for CHUNK_CAUSAL)
+# range types of the range-list descriptor (0-3 follow the attn_type_map values printed
+# on the chunk-causal page; 4 is this library's code for CHUNK_CAUSAL)
 RANGE_FULL = 0
 RANGE_CAUSAL = 1
+RANGE_INV_CAUSAL = 2
+RANGE_BI_CAUSAL = 3
 RANGE_CHUNK_CAUSAL = 4
 
 KINDS = ("FULL", "CAUSAL", "SLIDING_WINDOW", "PREFIX_LM", "CHUNK_CAUSAL", "RANGES", "CUSTOM")
@@ -348,7 +350,8 @@ def random_mask_spec(rng: np.random.Generator, kind: str, lq, lk) -> MaskSpec:
             for _ in range(int(rng.integers(0, 6))):
                 a, c = sorted(rng.integers(0, int(lq[b]) + 1, size=2).tolist())
                 e, f = sorted(rng.integers(0, int(lk[b]) + 1, size=2).tolist())
-                t = int(rng.choice([RANGE_FULL, RANGE_CAUSAL, RANGE_CHUNK_CAUSAL]))
+                t = int(rng.choice([RANGE_FULL, RANGE_CAUSAL, RANGE_INV_CAUSAL, RANGE_BI_CAUSAL,
+                                    RANGE_CHUNK_CAUSAL]))
                 rs.append((a, c, e, f, t, int(rng.integers(1, 6)) if t == RANGE_CHUNK_CAUSAL else 0))
             per.append(rs)
         return MaskSpec(kind, ranges=per)
