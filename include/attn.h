@@ -65,7 +65,8 @@ typedef enum {
   ATTN_MASK_PREFIX_LM = 3,      /* j < prefix_len  or  j <= pos(i) */
   ATTN_MASK_CHUNK_CAUSAL = 4,   /* CAUSAL range over [0, chunk.q_start) plus the chunk-causal range `chunk` */
   ATTN_MASK_RANGES = 5,         /* union of typed (q_range, k_range) pairs, per sequence */
-  ATTN_MASK_CUSTOM = 6          /* bit-packed boolean mask, per sequence, shared by all heads */
+  ATTN_MASK_CUSTOM = 6,         /* bit-packed boolean mask, per sequence, shared by all heads */
+  ATTN_MASK_BLOCK_SPARSE = 7    /* block-sparse (BSR) mask: listed (block_q x block_k) blocks are visible */
 } attn_mask_kind_t;
 
 /* Range types. 0-3 are the attn_type_map values FULL, CAUSAL, INV_CAUSAL and BI_CAUSAL
@@ -105,6 +106,14 @@ typedef struct {
                                        significant bit first. Bits past L_k are ignored. */
   const int64_t* mask_word_offsets; /* CUSTOM: host [batch+1] word offsets (non-decreasing) */
   int64_t mask_words_total;         /* CUSTOM: number of readable words at mask_bits */
+  int32_t block_q, block_k;         /* BLOCK_SPARSE: block height (query rows) and width (keys), >= 1 */
+  const int32_t* bsr_row_ptr;       /* BLOCK_SPARSE: host CSR row pointer over the block rows of all
+                                       sequences in order (sequence b has ceil(L_q / block_q) block
+                                       rows); length = total block rows + 1, starting at 0 */
+  const int32_t* bsr_col_idx;       /* BLOCK_SPARSE: host block-column indices (sequence-local, in
+                                       [0, ceil(L_k / block_k))); query i, key j is visible iff
+                                       block (i / block_q, j / block_k) is listed ("Custom mask slows
+                                       down attention.": the sparse API, equivalent to a custom mask) */
 } attn_mask_desc_t;
 
 /* Problem shape. Host arrays are read during attn_plan() only. */

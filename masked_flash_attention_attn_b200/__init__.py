@@ -21,7 +21,7 @@ STATUS = {0: "ATTN_OK", 1: "ATTN_ERR_INVALID_ARG", 2: "ATTN_ERR_UNSUPPORTED", 3:
           4: "ATTN_ERR_OOM", 5: "ATTN_ERR_CUDA", 6: "ATTN_ERR_TIMEOUT", 7: "ATTN_ERR_TOO_LARGE"}
 NOALLOC_SCRATCH_BYTES = 32 << 20
 MASK_KIND = {"FULL": 0, "CAUSAL": 1, "SLIDING_WINDOW": 2, "PREFIX_LM": 3, "CHUNK_CAUSAL": 4, "RANGES": 5,
-             "CUSTOM": 6}
+             "CUSTOM": 6, "BLOCK_SPARSE": 7}
 RANGE_FULL, RANGE_CAUSAL, RANGE_INV_CAUSAL, RANGE_BI_CAUSAL, RANGE_CHUNK_CAUSAL = 0, 1, 2, 3, 4
 
 # every symbol include/attn.h declares
@@ -44,7 +44,9 @@ class attn_mask_desc_t(ctypes.Structure):
     _fields_ = [("kind", ctypes.c_int32), ("window", ctypes.c_int32), ("prefix_len", ctypes.c_int32),
                 ("prefix_lens", ctypes.c_void_p), ("chunk", attn_range_t), ("ranges", ctypes.c_void_p),
                 ("cu_ranges", ctypes.c_void_p), ("mask_bits", ctypes.c_void_p),
-                ("mask_word_offsets", ctypes.c_void_p), ("mask_words_total", ctypes.c_int64)]
+                ("mask_word_offsets", ctypes.c_void_p), ("mask_words_total", ctypes.c_int64),
+                ("block_q", ctypes.c_int32), ("block_k", ctypes.c_int32), ("bsr_row_ptr", ctypes.c_void_p),
+                ("bsr_col_idx", ctypes.c_void_p)]
 
 
 class attn_problem_t(ctypes.Structure):
@@ -147,7 +149,8 @@ def _problem(m: _Marshal, *, hq, hkv, head_dim, cu_seqlens_q, cu_seqlens_k=None,
 
 def _mask_desc(m: _Marshal, mask, device_bits=None):
     """``mask``: an object with the attributes kind, window, prefix_len, prefix_lens, chunk,
-    ranges (per-sequence lists of 6-tuples), bits, word_offsets (see include/attn.h)."""
+    ranges (per-sequence lists of 6-tuples), bits, word_offsets, block_q, block_k,
+    bsr_row_ptr, bsr_col_idx (see include/attn.h)."""
     d = attn_mask_desc_t()
     d.kind = MASK_KIND[mask.kind]
     d.window = int(getattr(mask, "window", 0) or 0)
@@ -165,6 +168,10 @@ def _mask_desc(m: _Marshal, mask, device_bits=None):
         m.keep.append(arr)
         d.ranges = ctypes.addressof(arr)
         d.cu_ranges = m.arr(cu, np.int32)
+    if mask.kind == "BLOCK_SPARSE":
+        d.block_q, d.block_k = int(mask.block_q), int(mask.block_k)
+        d.bsr_row_ptr = m.arr(mask.bsr_row_ptr, np.int32)
+        d.bsr_col_idx = m.arr(mask.bsr_col_idx if len(mask.bsr_col_idx) else np.zeros(1), np.int32)
     if mask.kind == "CUSTOM":
         d.mask_word_offsets = m.arr(mask.word_offsets, np.int64)
         d.mask_bits = _ptr(device_bits)

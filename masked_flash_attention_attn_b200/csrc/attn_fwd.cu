@@ -207,6 +207,10 @@ __device__ __forceinline__ uint64_t l2_policy_evict_first() {
   return pol;
 }
 
+__device__ __forceinline__ void prefetch_l1(const void* ptr) {
+  asm volatile("prefetch.global.L1 [%0];" ::"l"(ptr));
+}
+
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* tm) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tm)) : "memory");
 }
@@ -588,6 +592,11 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_fwd_kernel(const __
       int q_last = -1;            // last item whose Q load was armed
       for (int ii = i_begin; ii < i_end; ++ii, ++n) {
         const WorkItem it = p.items[p.cta_items[ii]];
+        if constexpr (C::PAGED) {
+          // first page-table lines of this item and of the next one
+          prefetch_l1(p.page_table + it.k_base);
+          if (ii + 1 < i_end) prefetch_l1(p.page_table + p.items[p.cta_items[ii + 1]].k_base);
+        }
         if (!wait_bounded(BAR(C::B_QEMPTY), (n & 1) ^ 1, guard, kWaitQEmpty)) break;
         if (!((p.debug_flags & 1) && n == 0)) {
           mbar_expect_tx(BAR(C::B_QFULL), C::NQ * C::Q_BYTES);
@@ -614,6 +623,12 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_fwd_kernel(const __
                             BAR(C::B_KVFULL + slot));
             } else {
               const int ps = p.page_size, ppt = 128 / ps;
+              // the page ids of the key tile two ahead go to L1 now; this tile's ids were
+              // prefetched the same way, so the loads below hit L1
+              if (!is_v && h == 0) {
+                const int ahead = (kt + 2) * ppt;
+                if (ahead < it.npages) prefetch_l1(p.page_table + it.k_base + ahead);
+              }
               // all page ids of the tile are requested before the first is used
               int32_t page[8];
 #pragma unroll
@@ -918,6 +933,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::THREADS, 1)
             const int ps = p.page_size;
             const int rows = ps < nkeys ? ps : nkeys;  // rows per box
             const int nb = nkeys / rows;               // boxes per 64-column block
+            if (!is_v) {
+              const int ahead = ((kt + 2) * 128) / ps;   // page-table line of the key tile two ahead
+              if (ahead < it.npages) prefetch_l1(p.page_table + it.k_base + ahead);
+            }
             int32_t page[8];
 #pragma unroll
             for (int pg = 0; pg < 8; ++pg) {

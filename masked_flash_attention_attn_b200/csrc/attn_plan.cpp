@@ -145,6 +145,24 @@ attn_status_t validate_mask(const attn_mask_desc_t* m, const Shape& s) {
       }
       return ATTN_OK;
     }
+    case ATTN_MASK_BLOCK_SPARSE: {
+      if (m->block_q < 1 || m->block_k < 1) return ATTN_ERR_INVALID_ARG;
+      if (s.B == 0) return ATTN_OK;
+      if (!m->bsr_row_ptr || m->bsr_row_ptr[0] != 0) return ATTN_ERR_INVALID_ARG;
+      int64_t row = 0;
+      for (int b = 0; b < s.B; ++b) {
+        const int64_t nbr = (int64_t(s.lq[b]) + m->block_q - 1) / m->block_q;
+        const int64_t nbc = (int64_t(s.lk[b]) + m->block_k - 1) / m->block_k;
+        for (int64_t r = row; r < row + nbr; ++r) {
+          if (m->bsr_row_ptr[r + 1] < m->bsr_row_ptr[r]) return ATTN_ERR_INVALID_ARG;
+          if (m->bsr_row_ptr[r + 1] > m->bsr_row_ptr[r] && !m->bsr_col_idx) return ATTN_ERR_INVALID_ARG;
+          for (int32_t e = m->bsr_row_ptr[r]; e < m->bsr_row_ptr[r + 1]; ++e)
+            if (m->bsr_col_idx[e] < 0 || m->bsr_col_idx[e] >= nbc) return ATTN_ERR_INVALID_ARG;
+        }
+        row += nbr;
+      }
+      return ATTN_OK;
+    }
     case ATTN_MASK_CUSTOM: {
       if (s.B == 0) return ATTN_OK;
       if (!m->mask_word_offsets) return ATTN_ERR_INVALID_ARG;
@@ -172,8 +190,9 @@ class RowSource {
  public:
   RowSource(const attn_mask_desc_t* m, const Shape& s) : m_(m), s_(s) {}
 
-  // Build the merged per-row intervals of sequence b for the range kinds.
+  // Build the merged per-row intervals of sequence b for the range and block-sparse kinds.
   void prepare(int b) {
+    if (m_->kind == ATTN_MASK_BLOCK_SPARSE) return prepare_bsr(b);
     if (m_->kind != ATTN_MASK_RANGES && m_->kind != ATTN_MASK_CHUNK_CAUSAL) return;
     const int lq = s_.lq[b], lk = s_.lk[b];
     std::vector<attn_range_t> rs;
@@ -229,6 +248,36 @@ class RowSource {
     }
     iv_.resize(w);
     off_.swap(noff);
+  }
+
+  // Block-sparse: every row of block row R shares the intervals of R's listed block columns.
+  void prepare_bsr(int b) {
+    const int lq = s_.lq[b], lk = s_.lk[b], bq = m_->block_q, bk = m_->block_k;
+    int64_t row0 = 0;
+    for (int x = 0; x < b; ++x) row0 += (int64_t(s_.lq[x]) + bq - 1) / bq;
+    const int nbr = (lq + bq - 1) / bq;
+    std::vector<Iv> brow;
+    off_.assign(size_t(lq) + 1, 0);
+    iv_.clear();
+    for (int R = 0; R < nbr; ++R) {
+      brow.clear();
+      for (int32_t e = m_->bsr_row_ptr[row0 + R]; e < m_->bsr_row_ptr[row0 + R + 1]; ++e) {
+        const int64_t a = int64_t(m_->bsr_col_idx[e]) * bk;
+        brow.push_back(Iv{int32_t(a), int32_t(std::min<int64_t>(a + bk, lk))});
+      }
+      std::sort(brow.begin(), brow.end(), [](const Iv& x, const Iv& y) { return x.a < y.a; });
+      std::vector<Iv> merged;
+      for (const Iv& v : brow) {
+        if (v.a >= v.b) continue;
+        if (!merged.empty() && v.a <= merged.back().b) merged.back().b = std::max(merged.back().b, v.b);
+        else merged.push_back(v);
+      }
+      const int r_end = std::min(lq, (R + 1) * bq);
+      for (int i = R * bq; i < r_end; ++i) {
+        iv_.insert(iv_.end(), merged.begin(), merged.end());
+        off_[i + 1] = int64_t(iv_.size());
+      }
+    }
   }
 
   // Intervals of row i of sequence b (sorted, disjoint, non-empty, inside [0, L_k)).

@@ -30,6 +30,11 @@ Sources for each kind
                   [k_start, q_start + (c+1)*cs), the chunk end clipped to q_end
                   and the keys to k_range. The convenience kind adds a CAUSAL
                   range over [0, q_start) before the chunked part.
+  BLOCK_SPARSE    "Custom mask slows down attention." (the sparse API the thread
+                  recommends for long sequences, equivalent to a custom mask): query i
+                  sees key j iff block (i // block_q, j // block_k) is listed in the
+                  sequence's block rows (CSR over all sequences' block rows in order;
+                  bsr_seq_row0[b] is sequence b's first block row).
   CUSTOM          "Custom mask slows down attention." (bit-packed mask) and
                   "feat: support custom mask for flash attention" (custom_mask):
                   row-major [L_q][ceil(L_k/32)] uint32 words, key j is bit j%32
@@ -107,6 +112,15 @@ def dense_mask_rows(spec, b: int, lq: int, lk: int, r0: int, r1: int) -> np.ndar
         m = np.zeros((r1 - r0, lk), dtype=bool)
         for rg in ranges:
             _range_or_into(m, rg, r0, r1)
+        return m
+    if kind == "BLOCK_SPARSE":
+        bq, bk = int(spec.block_q), int(spec.block_k)
+        row0 = int(spec.bsr_seq_row0[b])      # first block row of sequence b in the CSR
+        m = np.zeros((r1 - r0, lk), dtype=bool)
+        for R in range(r0 // bq, -(-r1 // bq)):
+            a, e = max(r0, R * bq), min(r1, (R + 1) * bq)
+            for c in spec.bsr_col_idx[spec.bsr_row_ptr[row0 + R]:spec.bsr_row_ptr[row0 + R + 1]]:
+                m[a - r0:e - r0, int(c) * bk:min(lk, (int(c) + 1) * bk)] = True
         return m
     if kind == "CUSTOM":
         w = (lk + 31) // 32

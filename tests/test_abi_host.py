@@ -54,7 +54,7 @@ def _lengths(wl):
     return [(wl.lq(b), wl.lk(b)) for b in range(wl.batch)]
 
 
-@pytest.mark.parametrize("kind", ["FULL", "CAUSAL", "SLIDING_WINDOW", "PREFIX_LM", "CHUNK_CAUSAL", "RANGES"])
+@pytest.mark.parametrize("kind", ["FULL", "CAUSAL", "SLIDING_WINDOW", "PREFIX_LM", "CHUNK_CAUSAL", "RANGES", "BLOCK_SPARSE"])
 @pytest.mark.parametrize("seed", range(6))
 def test_host_classes_match_oracle_random(attn_lib, kind, seed):
     wl = W.random_small(seed=100 * seed + 7, kind=kind, batch=4, lmin=1, lmax=700, equal_qk=(seed % 2 == 0))

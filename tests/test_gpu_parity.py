@@ -15,7 +15,7 @@ from tests import gpu_helpers as G
 
 pytestmark = pytest.mark.gpu
 
-KINDS = ["FULL", "CAUSAL", "SLIDING_WINDOW", "PREFIX_LM", "CHUNK_CAUSAL", "RANGES", "CUSTOM"]
+KINDS = ["FULL", "CAUSAL", "SLIDING_WINDOW", "PREFIX_LM", "CHUNK_CAUSAL", "RANGES", "CUSTOM", "BLOCK_SPARSE"]
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -197,3 +197,22 @@ def test_inv_and_bi_causal_ranges(d):
                     q=W.randn_bf16(gen, int(cq[-1]), 4, d), masks=[W.MaskSpec("RANGES", ranges=ranges)],
                     cu_seqlens_k=ck, k=W.randn_bf16(gen, int(ck[-1]), 2, d), v=W.randn_bf16(gen, int(ck[-1]), 2, d))
     G.check_full(wl, wl.masks[0], f"inv/bi d={d}")
+
+
+def test_block_sparse_equals_custom_of_its_blocks():
+    """The sparse (BSR) descriptor and the packed custom mask of the same blocks plan the same
+    tiles and give bit-identical outputs ("Custom mask slows down attention.": equivalence)."""
+    wl = W.random_small(seed=77, kind="BLOCK_SPARSE", batch=3, hq=4, hkv=2, d=128, lmin=50, lmax=500)
+    spec = wl.masks[0]
+    out_b, lse_b, plan_b = G.run(wl, spec)
+    words, offs = [], [0]
+    for b in range(wl.batch):
+        m = oracle.dense_mask(spec, b, wl.lq(b), wl.lk(b))
+        w = W.pack_rows(m).reshape(-1)
+        words.append(w)
+        offs.append(offs[-1] + w.size)
+    cu = W.MaskSpec("CUSTOM", bits=np.concatenate(words).astype(np.uint32), word_offsets=np.asarray(offs, np.int64))
+    out_c, lse_c, plan_c = G.run(wl, cu)
+    import masked_flash_attention_attn_b200 as M
+    assert np.array_equal(M.attn_plan_get_tile_classes(plan_b), M.attn_plan_get_tile_classes(plan_c))
+    assert torch.equal(out_b, out_c) and torch.equal(lse_b, lse_c)

@@ -38,7 +38,7 @@ def _brute(q, k, v, mask, scale):
 
 
 @pytest.mark.parametrize("kind", ["FULL", "CAUSAL", "SLIDING_WINDOW", "PREFIX_LM", "CHUNK_CAUSAL",
-                                  "RANGES", "CUSTOM"])
+                                  "RANGES", "CUSTOM", "BLOCK_SPARSE"])
 def test_brute_force_tiny(kind):
     wl = W.random_small(seed=11 + len(kind), kind=kind, batch=3, hq=4, hkv=2, d=8, lmin=1, lmax=13)
     spec = wl.masks[0]

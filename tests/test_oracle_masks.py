@@ -293,3 +293,37 @@ def test_bi_causal_is_an_aligned_band():
     # a band is not prefix + chunk-local attention (the page's point)
     cc = OM.dense_mask(_ranges_spec([[(0, 20, 0, 20, W.RANGE_CHUNK_CAUSAL, 2)]]), 0, 20, 20)
     assert not np.array_equal(_one_range(W.RANGE_BI_CAUSAL, 0, 20, 0, 20), cc)
+
+
+# ---- BLOCK_SPARSE ("Custom mask slows down attention.": the sparse API ≡ a custom mask) ----
+
+def test_block_sparse_equals_custom_mask_of_its_blocks():
+    rng = np.random.default_rng(12)
+    lq, lk = np.array([200, 77, 300]), np.array([260, 77, 129])
+    spec = W.random_mask_spec(rng, "BLOCK_SPARSE", lq, lk)
+    bq, bk = spec.block_q, spec.block_k
+    for b in range(3):
+        m = OM.dense_mask(spec, b, int(lq[b]), int(lk[b]))
+        # expand the listed blocks by hand (a separate statement of the same definition)
+        exp = np.zeros_like(m)
+        nbr = -(-int(lq[b]) // bq)
+        for R in range(nbr):
+            r = int(spec.bsr_seq_row0[b]) + R
+            for c in spec.bsr_col_idx[spec.bsr_row_ptr[r]:spec.bsr_row_ptr[r + 1]]:
+                exp[R * bq:(R + 1) * bq, c * bk:(c + 1) * bk] = True
+        assert np.array_equal(m, exp)
+        bits = W.pack_rows(m).reshape(-1)
+        cu = W.MaskSpec("CUSTOM", bits=bits, word_offsets=np.array([0, bits.size], np.int64))
+        assert np.array_equal(OM.dense_mask(cu, 0, int(lq[b]), int(lk[b])), m)
+
+
+def test_block_sparse_all_blocks_is_full_and_none_is_empty():
+    lq, lk, bq, bk = 130, 300, 64, 128
+    nbr, nbc = 3, 3
+    full = W.MaskSpec("BLOCK_SPARSE", block_q=bq, block_k=bk,
+                      bsr_row_ptr=np.arange(0, nbc * nbr + 1, nbc, dtype=np.int32),
+                      bsr_col_idx=np.tile(np.arange(nbc, dtype=np.int32), nbr), bsr_seq_row0=np.array([0]))
+    assert OM.dense_mask(full, 0, lq, lk).all()
+    none = W.MaskSpec("BLOCK_SPARSE", block_q=bq, block_k=bk, bsr_row_ptr=np.zeros(nbr + 1, np.int32),
+                      bsr_col_idx=np.zeros(0, np.int32), bsr_seq_row0=np.array([0]))
+    assert not OM.dense_mask(none, 0, lq, lk).any()

@@ -26,6 +26,8 @@ pages they come from:
   CUSTOM(bits, word_offsets)            "Custom mask slows down attention." (bit-packed
                                         custom mask); "feat: support custom mask for
                                         flash attention" (custom_mask input)
+  BLOCK_SPARSE(block_q, block_k, BSR)   "Custom mask slows down attention." (the sparse API
+                                        recommended for long sequences): listed blocks visible
 
 Packed CUSTOM layout: for each sequence, row-major ``[L_q][ceil(L_k/32)]``
 uint32 words; key ``j`` of row ``i`` is bit ``j % 32`` (least significant bit
@@ -48,7 +50,7 @@ RANGE_INV_CAUSAL = 2
 RANGE_BI_CAUSAL = 3
 RANGE_CHUNK_CAUSAL = 4
 
-KINDS = ("FULL", "CAUSAL", "SLIDING_WINDOW", "PREFIX_LM", "CHUNK_CAUSAL", "RANGES", "CUSTOM")
+KINDS = ("FULL", "CAUSAL", "SLIDING_WINDOW", "PREFIX_LM", "CHUNK_CAUSAL", "RANGES", "CUSTOM", "BLOCK_SPARSE")
 
 Range = Tuple[int, int, int, int, int, int]  # q_start, q_end, k_start, k_end, type, chunk_size
 
@@ -63,6 +65,11 @@ class MaskSpec:
     ranges: Optional[List[List[Range]]] = None         # RANGES: per-sequence lists
     bits: Optional[np.ndarray] = None                  # CUSTOM: uint32 words
     word_offsets: Optional[np.ndarray] = None          # CUSTOM: int64 [B+1]
+    block_q: int = 0                                   # BLOCK_SPARSE block height
+    block_k: int = 0                                   # BLOCK_SPARSE block width
+    bsr_row_ptr: Optional[np.ndarray] = None           # BLOCK_SPARSE: int32 [total block rows + 1]
+    bsr_col_idx: Optional[np.ndarray] = None           # BLOCK_SPARSE: int32 block columns
+    bsr_seq_row0: Optional[np.ndarray] = None          # BLOCK_SPARSE: first block row of each sequence
 
     def __post_init__(self):
         if self.kind not in KINDS:
@@ -355,6 +362,18 @@ def random_mask_spec(rng: np.random.Generator, kind: str, lq, lk) -> MaskSpec:
                 rs.append((a, c, e, f, t, int(rng.integers(1, 6)) if t == RANGE_CHUNK_CAUSAL else 0))
             per.append(rs)
         return MaskSpec(kind, ranges=per)
+    if kind == "BLOCK_SPARSE":
+        bq, bk = int(rng.choice([16, 64, 128, 100])), int(rng.choice([32, 128, 77]))
+        ptr, cols, row0 = [0], [], []
+        for b in range(B):
+            nbr, nbc = -(-int(lq[b]) // bq), -(-int(lk[b]) // bk)
+            row0.append(len(ptr) - 1)
+            for _ in range(nbr):
+                sel = np.nonzero(rng.random(nbc) < rng.choice([0.1, 0.5, 0.9]))[0]
+                cols.extend(rng.permutation(sel).tolist())   # unsorted on purpose
+                ptr.append(len(cols))
+        return MaskSpec(kind, block_q=bq, block_k=bk, bsr_row_ptr=np.asarray(ptr, np.int32),
+                        bsr_col_idx=np.asarray(cols, np.int32), bsr_seq_row0=np.asarray(row0, np.int64))
     if kind == "CUSTOM":
         words, offs = [], [0]
         for b in range(B):
