@@ -215,29 +215,16 @@ __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* tm) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tm)) : "memory");
 }
 
-// Shared-memory matrix descriptor, 128-byte swizzle, sm_100 version field = 1.
-__device__ __forceinline__ uint64_t sdesc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
-  return uint64_t((addr & 0x3FFFFu) >> 4) | (uint64_t(lbo >> 4) << 16) | (uint64_t(sbo >> 4) << 32) |
-         (1ull << 46) | (2ull << 61);
+// Descriptors split into words: the high word (stride byte offset 1024, version 1, 128-byte
+// swizzle) is the same for every operand here; the low word holds the start address and
+// the leading byte offset, so stepping through a tile is one 32-bit add per operand.
+constexpr uint32_t kDescHi = (1024u >> 4) | (1u << 14) | (2u << 29);
+__device__ __forceinline__ uint32_t desc_lo(uint32_t addr, uint32_t lbo) {
+  return ((addr & 0x3FFFFu) >> 4) | ((lbo >> 4) << 16);
 }
+__device__ __forceinline__ uint64_t desc_of(uint32_t lo) { return (uint64_t(kDescHi) << 32) | lo; }
 
-__device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a), "l"(b), "r"(idesc), "r"(acc)
-      : "memory");
-}
 
-__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t idesc, uint32_t acc) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc)
-      : "memory");
-}
 
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
@@ -273,25 +260,10 @@ __device__ __forceinline__ void warp_arrive_leader(uint32_t cluster_addr) {
   if ((threadIdx.x & 31) == 0) mbar_arrive_remote(cluster_addr);
 }
 
-// 2-SM MMA of a CTA pair (issued by the pair's leader): A rows split over the two CTAs,
-// B rows (N) split over the two CTAs, D rows split, all at the same offsets in both CTAs.
-__device__ __forceinline__ void mma2_ss(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a), "l"(b), "r"(idesc), "r"(acc)
-      : "memory");
-}
+// 2-SM MMAs of a CTA pair (mma2_*_x* in mma_groups.inc, issued by the pair's leader): A rows
+// split over the two CTAs, B rows (N) split over the two CTAs, D rows split, all at the same
+// offsets in both CTAs.
 
-__device__ __forceinline__ void mma2_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t idesc, uint32_t acc) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc)
-      : "memory");
-}
 
 // arrive on the barrier at this offset in both CTAs of the pair when the MMAs complete
 __device__ __forceinline__ void mma2_commit_both(uint32_t bar) {
@@ -332,6 +304,7 @@ __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 #include "tmem_ldst.inc"
+#include "mma_groups.inc"
 
 __device__ __forceinline__ float ex2(float x) {
   float y;
@@ -686,19 +659,14 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_fwd_kernel(const __
             tc_fence_after();
           }
           const uint32_t slot = (sj + t) & 1;
-          const uint32_t qbase = sbase + C::OFF_Q + q * C::Q_BYTES;
+          const uint32_t d_s = tmem + 128 * slot;
+          const uint32_t qlo = desc_lo(sbase + C::OFF_Q + q * C::Q_BYTES, 16);
+          static_assert(C::NCH == 1, "single-CTA kernel: one ring chunk per K or V tile");
 #pragma unroll
           for (int h = 0; h < C::NCH; ++h) {
-#pragma unroll
-            for (int kq = 0; kq < C::CH / 16; ++kq) {
-              const int col = h * C::CH + kq * 16;
-              const int c = (col % C::CH) / 64, w = col % 64;
-              const uint64_t a = sdesc(qbase + (col / 64) * C::BOX_BYTES + w * 2, 16, 1024);
-              const uint64_t b = sdesc(sbase + C::OFF_RING + ((rk + h) % C::STAGES) * C::CHUNK_BYTES +
-                                           c * C::BOX_BYTES + w * 2,
-                                       16, 1024);
-              mma_ss(tmem + 128 * slot, a, b, C::IDESC_QK, col > 0 ? 1u : 0u);
-            }
+            const uint32_t klo = desc_lo(sbase + C::OFF_RING + ((rk + h) % C::STAGES) * C::CHUNK_BYTES, 16);
+            if constexpr (C::D == 128) mma_ss_x8_k128(d_s, desc_of(qlo), desc_of(klo), C::IDESC_QK, 0u);
+            else mma_ss_x4_k64(d_s, desc_of(qlo), desc_of(klo), C::IDESC_QK, 0u);
             // the chunk is free once these MMAs complete (commit tracks all earlier MMAs)
             if (q == C::NQ - 1) mma_commit(BAR(C::B_KVEMPTY + (rk + h) % C::STAGES));
           }
@@ -718,15 +686,12 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_fwd_kernel(const __
                 return false;
           }
           tc_fence_after();
+          const uint32_t first = u < C::NQ ? 1u : 0u;
 #pragma unroll
           for (int h = 0; h < C::NCH; ++h) {
-            const uint32_t vbase = sbase + C::OFF_RING + ((rv + h) % C::STAGES) * C::CHUNK_BYTES;
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-              const uint64_t b = sdesc(vbase + kk * 2048, C::BOX_BYTES, 1024);
-              mma_ts(tmem + C::TM_O + q * C::D + h * 128, tmem + 128 * slot + kk * 8, b, C::IDESC_PV,
-                     (u < C::NQ && kk == 0) ? 0u : 1u);
-            }
+            const uint32_t vlo = desc_lo(sbase + C::OFF_RING + ((rv + h) % C::STAGES) * C::CHUNK_BYTES, C::BOX_BYTES);
+            const uint32_t d_o = tmem + C::TM_O + q * C::D + h * 128, a_p = tmem + 128 * slot;
+            mma_ts_x8(d_o, a_p, desc_of(vlo), C::IDESC_PV, first ^ 1u);
             if (q == C::NQ - 1) mma_commit(BAR(C::B_KVEMPTY + (rv + h) % C::STAGES));
           }
           mma_commit(BAR(C::B_PVDONE + q));
@@ -988,14 +953,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::THREADS, 1)
             return false;
           ++rc;
           tc_fence_after();
-          const uint32_t kb = sbase + C::OFF_RING + (rk % C::STAGES) * C::SLOT_BYTES;
-#pragma unroll
-          for (int kk = 0; kk < C::D / 16; ++kk) {
-            const int col = kk * 16;
-            const uint64_t a = sdesc(sbase + C::OFF_Q + (col / 64) * 16384 + (col % 64) * 2, 16, 1024);
-            const uint64_t b = sdesc(kb + (col / 64) * C::KH_BOX + (col % 64) * 2, 16, 1024);
-            mma2_ss(tmem + 128 * slot, a, b, C::IDESC_QK, kk > 0 ? 1u : 0u);
-          }
+          const uint32_t qlo = desc_lo(sbase + C::OFF_Q, 16);
+          const uint32_t klo = desc_lo(sbase + C::OFF_RING + (rk % C::STAGES) * C::SLOT_BYTES, 16);
+          const uint32_t d_s = tmem + 128 * slot;
+          static_assert(C::D == 256, "pair kernel issue groups are laid out for head_dim 256");
+          mma2_ss_x16_k256(d_s, desc_of(qlo), desc_of(klo), C::IDESC_QK, 0u);
           mma2_commit_both(BAR(C::B_KVEMPTY + rk % C::STAGES));
           mma2_commit_both(BAR(C::B_SFULL + slot));
           if (t == T - 1) mma2_commit_both(BAR(C::B_QEMPTY));
@@ -1009,12 +971,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::THREADS, 1)
             return false;
           ++rc;
           tc_fence_after();
-          const uint32_t vb = sbase + C::OFF_RING + (rv % C::STAGES) * C::SLOT_BYTES;
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint64_t b = sdesc(vb + kk * 2048, C::VH_BOX, 1024);
-            mma2_ts(tmem + C::TM_O, tmem + 128 * slot + kk * 8, b, C::IDESC_PV, (u == 0 && kk == 0) ? 0u : 1u);
-          }
+          const uint32_t vlo = desc_lo(sbase + C::OFF_RING + (rv % C::STAGES) * C::SLOT_BYTES, C::VH_BOX);
+          const uint32_t a_p = tmem + 128 * slot, acc0 = u == 0 ? 0u : 1u;
+          mma2_ts_x8(tmem + C::TM_O, a_p, desc_of(vlo), C::IDESC_PV, acc0);
           mma2_commit_both(BAR(C::B_KVEMPTY + rv % C::STAGES));
           mma2_commit_both(BAR(C::B_PVDONE));
           return true;
