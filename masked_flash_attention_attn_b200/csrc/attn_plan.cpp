@@ -31,6 +31,11 @@
 
 #include "attn_internal.h"
 
+// 1: balance items group by group (see build_work); 0: plain longest-processing-time-first
+#ifndef MFA_SCHED_GROUPED
+#define MFA_SCHED_GROUPED 1
+#endif
+
 namespace {
 
 using namespace mfa;
@@ -461,12 +466,24 @@ void build_work(const Shape& s, int R, int hp, int nq, const std::vector<std::ve
       }
     }
   }
-  // longest-processing-time-first onto persistent CTAs
+  // Greedy balancing onto persistent CTAs: each item goes to the least-loaded CTA. Items are
+  // taken group by group -- a group being one (sequence, key/value head), the largest
+  // groups first -- and, inside a group, longest first. Items of one group then run at
+  // about the same time on different CTAs and share their K/V tiles in L2 (pure
+  // longest-first interleaves every group and re-reads K/V from DRAM once it exceeds L2);
+  // with one item per group this is plain longest-processing-time-first.
   const int n_items = int(wl.items.size());
   const int C = std::max(1, std::min(num_sms, n_items));
   std::vector<int32_t> order(n_items);
   std::iota(order.begin(), order.end(), 0);
+  auto group = [&](int32_t i) { return int64_t(wl.items[i].seq) * s.hkv + wl.items[i].kv_head; };
+  std::vector<int64_t> gcost(size_t(s.B) * s.hkv, 0);
+  for (const WorkItem& it : wl.items) gcost[size_t(it.seq) * s.hkv + it.kv_head] += it.job_count;
   std::stable_sort(order.begin(), order.end(), [&](int32_t x, int32_t y) {
+    if (MFA_SCHED_GROUPED && group(x) != group(y)) {
+      const int64_t cx = gcost[group(x)], cy = gcost[group(y)];
+      return cx != cy ? cx > cy : group(x) < group(y);
+    }
     return wl.items[x].job_count > wl.items[y].job_count;
   });
   using Load = std::pair<int64_t, int32_t>;
