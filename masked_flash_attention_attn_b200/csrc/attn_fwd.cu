@@ -375,6 +375,13 @@ __device__ __forceinline__ uint64_t exp2_poly2(float x0, float x1) {
              __int_as_float(__float_as_int(p1) + (__float_as_int(y1) << 23)));
 }
 
+// Three-operand maximum (sm_100 adds the 3-input form of max.f32).
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 // Two fp32 -> one bf16x2 word (round to nearest even); `lo` lands in the low half, which
 // is the lower column / key index in every layout used here.
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
@@ -416,9 +423,16 @@ __device__ __forceinline__ float softmax_tile(uint32_t t_s, int mi, const uint4&
     for (int c = 0; c < 128; ++c)
       if (!((wv[c >> 5] >> (c & 31)) & 1u)) s[c] = -INFINITY;
   }
-  float mx = s[0];
+  // row maximum: eight independent chains of 3-input max, then a small tree (one thread
+  // owns the row, so a single 127-long dependent chain would cost its full latency)
+  float m8[8];
 #pragma unroll
-  for (int c = 1; c < 128; ++c) mx = fmaxf(mx, s[c]);
+  for (int k = 0; k < 8; ++k) m8[k] = fmaxf(s[k], s[k + 8]);
+#pragma unroll
+  for (int j = 1; j < 8; ++j)
+#pragma unroll
+    for (int k = 0; k < 8; ++k) m8[k] = max3f(m8[k], s[16 * j + k], s[16 * j + 8 + k]);
+  const float mx = max3f(max3f(m8[0], m8[1], m8[2]), max3f(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
   const float m_new = mx * sl2;
   need = m_new > st.m_run + 8.0f;
   float alpha = 1.f;
@@ -429,7 +443,7 @@ __device__ __forceinline__ float softmax_tile(uint32_t t_s, int mi, const uint4&
   }
   const float mref = st.m_run == -INFINITY ? 0.f : st.m_run;
   const uint64_t sl2x2 = pk2(sl2, sl2), nm2 = pk2(-mref, -mref);
-  uint64_t lsum2 = pk2(0.f, 0.f);
+  uint64_t lsum2[4] = {pk2(0.f, 0.f), pk2(0.f, 0.f), pk2(0.f, 0.f), pk2(0.f, 0.f)};  // 4 independent sums
 #pragma unroll
   for (int cc = 0; cc < 4; ++cc) {
     uint32_t pk[16];
@@ -443,7 +457,7 @@ __device__ __forceinline__ float softmax_tile(uint32_t t_s, int mi, const uint4&
       } else {
         p01 = pk2(ex2(x0), ex2(x1));
       }
-      lsum2 = fadd2(lsum2, p01);
+      lsum2[e & 3] = fadd2(lsum2[e & 3], p01);
       float p0, p1;
       unpk2(p01, p0, p1);
       pk[e] = pack_bf16(p0, p1);
@@ -452,7 +466,7 @@ __device__ __forceinline__ float softmax_tile(uint32_t t_s, int mi, const uint4&
   }
   {
     float a, b;
-    unpk2(lsum2, a, b);
+    unpk2(fadd2(fadd2(lsum2[0], lsum2[1]), fadd2(lsum2[2], lsum2[3])), a, b);
     st.l_run += a + b;
   }
   tmem_wait_st();
