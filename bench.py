@@ -204,7 +204,8 @@ def config_of(wl, args, world):
             "lengths_q": [wl.lq(b) for b in range(wl.batch)][:64],
             "hq": wl.hq, "hkv": wl.hkv, "head_dim": wl.d,
             "masks": [m.kind + (f"({m.window})" if m.kind == "SLIDING_WINDOW" else "") for m in wl.masks],
-            "seed": wl.seed, "parallelism": f"dp{world} (independent batches, no collective)",
+            "seed": wl.seed, "kv_splits": getattr(args, "kv_splits", 0),
+            "parallelism": f"dp{world} (independent batches, no collective)",
             "l2": f"inputs {in_bytes / 2**20:.0f} MiB vs 126 MiB L2; no flush" if in_bytes > L2_BYTES
             else "inputs fit L2; L2 flushed between steps"}
 
@@ -229,9 +230,10 @@ def device_inputs(wl, dev):
     return q, wl.k.to(dev), wl.v.to(dev)
 
 
-def make_plan(M, wl, spec, dev):
+def make_plan(M, wl, spec, dev, kv_splits=0):
     import torch
-    kw = dict(hq=wl.hq, hkv=wl.hkv, head_dim=wl.d, cu_seqlens_q=wl.cu_seqlens_q, mask=spec, scale=wl.scale)
+    kw = dict(hq=wl.hq, hkv=wl.hkv, head_dim=wl.d, cu_seqlens_q=wl.cu_seqlens_q, mask=spec, scale=wl.scale,
+              kv_splits=kv_splits)
     if wl.paged:
         kw.update(kv_lens=wl.kv_lens, page_table=torch.from_numpy(wl.page_table).to(dev),
                   page_size=wl.page_size, num_pages=wl.k_cache.shape[0])
@@ -252,7 +254,7 @@ def run_ours(args, rank, world, local_rank):
     wl = workload(args.config, rank)
     stream = torch.cuda.current_stream()
     q, k, v = device_inputs(wl, dev)
-    plans = [make_plan(M, wl, spec, dev) for spec in wl.masks]
+    plans = [make_plan(M, wl, spec, dev, args.kv_splits) for spec in wl.masks]
     stats = [M.attn_plan_get_stats(p) for p in plans]
     flops = [flops_of(s, wl) for s in stats]
     tq = q.shape[0]
@@ -361,12 +363,14 @@ def run_ours(args, rank, world, local_rank):
                      "avg_launch_ms": avg_launch_ms},
         "per_mask": [{"mask": m.kind, "unmasked_pairs_per_head": s["unmasked_pairs"], "tflops_per_s":
                       f / (statistics.mean(x) * 1e-3) / 1e12, "ms": statistics.mean(x),
-                      "tiles_e_f_p": [s["tiles_empty"], s["tiles_full"], s["tiles_partial"]]}
+                      "tiles_e_f_p": [s["tiles_empty"], s["tiles_full"], s["tiles_partial"]],
+                      "kv_splits_max": s["kv_splits_max"], "merge_tiles": s["merge_tiles"]}
                      for m, s, f, x in zip(wl.masks, stats, flops, launch_ms)],
         "mask_gbs": mask_bytes / (sum(statistics.mean(x) for x in launch_ms) * 1e-3) / 1e9,
         "e2e": {"value": e2e_val, "unit": "TFLOP/s", "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                 "steps": e2e_steps},
-        "gpu_launches": len(plans) * args.steps,
+        # the forward kernel per plan and step, plus the split-KV merge kernel where a plan split
+        "gpu_launches": sum(1 + (s["merge_tiles"] > 0) for s in stats) * args.steps,
         "clocks": clocks,
     }
     if world == 1 and not args.no_cpu_baseline:
@@ -383,7 +387,10 @@ def main():
     ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--config", type=int, default=2, choices=[1, 2, 3, 4, 5])
+    ap.add_argument("--config", type=int, default=2, choices=[1, 2, 3, 4, 5, 6],
+                    help="1-5: the benchmark workloads; 6: long-context tree verify (split-KV case)")
+    ap.add_argument("--kv-splits", type=int, default=0,
+                    help="split-KV: 0 automatic, 1 never, N >= 2 at most N key ranges per query tile")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()

@@ -132,6 +132,15 @@ typedef struct {
   int32_t page_size;                /* paged: 16, 32, 64 or 128 */
   int32_t max_pages_per_seq;        /* paged: row length of page_table */
   int32_t num_pages;                /* paged: pages in the K and V caches */
+  int32_t kv_splits;                /* split-KV: 0 = automatic, 1 = never split, N >= 2 = split a work
+                                       item's key tiles into at most N ranges. A split item writes
+                                       fp32 partial results (out / l and lse per range) into the plan
+                                       workspace and a second kernel merges them by their lse:
+                                       lse = ln sum_r exp(lse_r), out = sum_r exp(lse_r - lse) out_r.
+                                       Automatic splits only when the longest item exceeds 1.5x the
+                                       per-CTA share of the work (few long items: short queries over
+                                       long keys, the tree-verify case of "Custom mask slows down
+                                       attention."). Must be >= 0. */
 } attn_problem_t;
 
 typedef struct attn_plan attn_plan_t; /* opaque */
@@ -146,6 +155,8 @@ typedef struct {
   int32_t heads_per_tile;           /* query heads packed into one 128-row tile (short queries) */
   int32_t tiles_per_cta;            /* 128-row query tiles one CTA works on at once (1 or 2) */
   int32_t cluster_size;             /* CTAs that cooperate on one work item (2: a pair of SMs) */
+  int32_t kv_splits_max;            /* largest number of key ranges any query tile was split into (1: none) */
+  int32_t merge_tiles;              /* 128-row query tiles whose partial results the merge kernel combines */
 } attn_plan_stats_t;
 
 /* Validate and plan. `stream` orders the plan's device work (the CUSTOM mask scan and
@@ -199,6 +210,14 @@ attn_status_t attn_plan_destroy(attn_plan_t* plan);
 attn_status_t attn_classify_host(const attn_problem_t* problem, const attn_mask_desc_t* mask,
                                  uint8_t* classes, size_t n, size_t* n_needed,
                                  int64_t* unmasked_pairs);
+
+/* Host-only dry run of attn_plan() for the analytic kinds (everything but CUSTOM): the
+ * same validation, tile classes, work list and split-KV choice for a GPU of `num_sms`
+ * SMs, reported as the statistics attn_plan_get_stats() would give; no CUDA call, no
+ * device memory (the device page_table pointer may be NULL). Errors: INVALID_ARG
+ * (num_sms <= 0 or as attn_plan), UNSUPPORTED (CUSTOM, or as attn_plan), OOM. */
+attn_status_t attn_plan_dry_run(const attn_problem_t* problem, const attn_mask_desc_t* mask, int32_t num_sms,
+                                attn_plan_stats_t* stats);
 
 const char* attn_status_string(attn_status_t status);
 

@@ -27,7 +27,7 @@ RANGE_FULL, RANGE_CAUSAL, RANGE_INV_CAUSAL, RANGE_BI_CAUSAL, RANGE_CHUNK_CAUSAL 
 # every symbol include/attn.h declares
 EXPORTS = ("attn_plan", "attn_masked_fwd", "attn_plan_get_tile_classes", "attn_plan_get_stats",
            "attn_plan_check_status", "attn_plan_set_debug", "attn_plan_destroy", "attn_classify_host",
-           "attn_status_string", "attn_masked_fwd_noalloc", "attn_test_exp2_poly")
+           "attn_status_string", "attn_masked_fwd_noalloc", "attn_test_exp2_poly", "attn_plan_dry_run")
 
 
 class AttnError(RuntimeError):
@@ -53,14 +53,16 @@ class attn_problem_t(ctypes.Structure):
     _fields_ = [("batch", ctypes.c_int32), ("hq", ctypes.c_int32), ("hkv", ctypes.c_int32),
                 ("head_dim", ctypes.c_int32), ("scale", ctypes.c_float), ("cu_seqlens_q", ctypes.c_void_p),
                 ("cu_seqlens_k", ctypes.c_void_p), ("kv_lens", ctypes.c_void_p), ("page_table", ctypes.c_void_p),
-                ("page_size", ctypes.c_int32), ("max_pages_per_seq", ctypes.c_int32), ("num_pages", ctypes.c_int32)]
+                ("page_size", ctypes.c_int32), ("max_pages_per_seq", ctypes.c_int32), ("num_pages", ctypes.c_int32),
+                ("kv_splits", ctypes.c_int32)]
 
 
 class attn_plan_stats_t(ctypes.Structure):
     _fields_ = [("unmasked_pairs", ctypes.c_int64), ("tiles_empty", ctypes.c_int64), ("tiles_full", ctypes.c_int64),
                 ("tiles_partial", ctypes.c_int64), ("mask_tiles", ctypes.c_int64), ("work_items", ctypes.c_int64),
                 ("jobs", ctypes.c_int64), ("mask_tile_reads", ctypes.c_int64), ("ctas", ctypes.c_int32), ("heads_per_tile", ctypes.c_int32),
-                ("tiles_per_cta", ctypes.c_int32), ("cluster_size", ctypes.c_int32)]
+                ("tiles_per_cta", ctypes.c_int32), ("cluster_size", ctypes.c_int32),
+                ("kv_splits_max", ctypes.c_int32), ("merge_tiles", ctypes.c_int32)]
 
 
 _lib = None
@@ -88,6 +90,8 @@ def lib() -> ctypes.CDLL:
         L.attn_status_string.argtypes = [i32]
         L.attn_status_string.restype = ctypes.c_char_p
         L.attn_test_exp2_poly.argtypes = [vp, vp, i64, vp]
+        L.attn_plan_dry_run.argtypes = [ctypes.POINTER(attn_problem_t), ctypes.POINTER(attn_mask_desc_t), i32,
+                                        ctypes.POINTER(attn_plan_stats_t)]
         L.attn_masked_fwd_noalloc.argtypes = [ctypes.POINTER(attn_problem_t), ctypes.POINTER(attn_mask_desc_t),
                                               vp, vp, vp, vp, vp, vp]
         for n in EXPORTS:
@@ -132,11 +136,12 @@ class _Marshal:
 
 
 def _problem(m: _Marshal, *, hq, hkv, head_dim, cu_seqlens_q, cu_seqlens_k=None, kv_lens=None, page_table=None,
-             page_size=0, num_pages=0, scale=0.0):
+             page_size=0, num_pages=0, scale=0.0, kv_splits=0):
     cq = np.asarray(cu_seqlens_q, dtype=np.int32)
     pr = attn_problem_t()
     pr.batch = len(cq) - 1
     pr.hq, pr.hkv, pr.head_dim, pr.scale = hq, hkv, head_dim, float(scale)
+    pr.kv_splits = int(kv_splits)
     pr.cu_seqlens_q = m.arr(cq, np.int32)
     pr.cu_seqlens_k = m.arr(cu_seqlens_k, np.int32)
     pr.kv_lens = m.arr(kv_lens, np.int32)
@@ -200,13 +205,16 @@ class Plan:
 
 
 def attn_plan(*, hq: int, hkv: int, head_dim: int, cu_seqlens_q, mask, cu_seqlens_k=None, kv_lens=None,
-              page_table=None, page_size: int = 0, num_pages: int = 0, scale: float = 0.0, stream=None) -> Plan:
+              page_table=None, page_size: int = 0, num_pages: int = 0, scale: float = 0.0, kv_splits: int = 0,
+              stream=None) -> Plan:
     """attn_plan(): validate, classify tiles, build the work list. ``page_table`` is a device
-    int32 tensor [batch, max_pages]; CUSTOM ``mask.bits`` may be host (numpy) or device words."""
+    int32 tensor [batch, max_pages]; CUSTOM ``mask.bits`` may be host (numpy) or device words;
+    ``kv_splits``: 0 automatic, 1 never, N >= 2 at most N key ranges per query tile."""
     import torch
     m = _Marshal()
     pr = _problem(m, hq=hq, hkv=hkv, head_dim=head_dim, cu_seqlens_q=cu_seqlens_q, cu_seqlens_k=cu_seqlens_k,
-                  kv_lens=kv_lens, page_table=page_table, page_size=page_size, num_pages=num_pages, scale=scale)
+                  kv_lens=kv_lens, page_table=page_table, page_size=page_size, num_pages=num_pages, scale=scale,
+                  kv_splits=kv_splits)
     dev_bits = None
     if mask.kind == "CUSTOM":
         b = mask.bits
@@ -257,12 +265,28 @@ def attn_plan_destroy(plan: Plan) -> None:
         _check(lib().attn_plan_destroy(h), "attn_plan_destroy")
 
 
+def attn_plan_dry_run(*, hq: int, hkv: int, head_dim: int, cu_seqlens_q, mask, num_sms: int = 148,
+                      cu_seqlens_k=None, kv_lens=None, page_size: int = 0, max_pages_per_seq: int = 0,
+                      num_pages: int = 0, kv_splits: int = 0) -> dict:
+    """Host-only attn_plan() (analytic kinds) for a GPU of ``num_sms`` SMs: the plan statistics."""
+    m = _Marshal()
+    pr = _problem(m, hq=hq, hkv=hkv, head_dim=head_dim, cu_seqlens_q=cu_seqlens_q, cu_seqlens_k=cu_seqlens_k,
+                  kv_lens=kv_lens, kv_splits=kv_splits)
+    if kv_lens is not None:
+        pr.page_size, pr.max_pages_per_seq, pr.num_pages = page_size, max_pages_per_seq, num_pages
+    d = _mask_desc(m, mask)
+    st = attn_plan_stats_t()
+    _check(lib().attn_plan_dry_run(ctypes.byref(pr), ctypes.byref(d), int(num_sms), ctypes.byref(st)),
+           "attn_plan_dry_run")
+    return {n: getattr(st, n) for n, _ in attn_plan_stats_t._fields_}
+
+
 def attn_classify_host(*, hq: int, hkv: int, head_dim: int, cu_seqlens_q, mask, cu_seqlens_k=None, kv_lens=None,
-                       page_size: int = 0, max_pages_per_seq: int = 0, num_pages: int = 0):
+                       page_size: int = 0, max_pages_per_seq: int = 0, num_pages: int = 0, kv_splits: int = 0):
     """Host-only tile classes (analytic kinds). Returns (classes uint8, unmasked pairs per head)."""
     m = _Marshal()
     pr = _problem(m, hq=hq, hkv=hkv, head_dim=head_dim, cu_seqlens_q=cu_seqlens_q, cu_seqlens_k=cu_seqlens_k,
-                  kv_lens=kv_lens)
+                  kv_lens=kv_lens, kv_splits=kv_splits)
     if kv_lens is not None:
         pr.page_size, pr.max_pages_per_seq, pr.num_pages = page_size, max_pages_per_seq, num_pages
     d = _mask_desc(m, mask)

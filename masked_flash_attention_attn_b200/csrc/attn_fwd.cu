@@ -54,6 +54,8 @@ struct Params {
   const int32_t* page_table;
   __nv_bfloat16* out;
   float* lse;
+  float* part_o;       // split-KV partial slots (kSlotRows x D fp32 each), or null
+  float* part_lse;     // split-KV partial lse (kSlotRows fp32 per slot), or null
   int32_t* status;
   int32_t hq, R, hp, page_size, num_pages, debug_flags;
   float scale_log2;
@@ -517,6 +519,29 @@ __device__ __forceinline__ void store_row(uint32_t t_o, const RowState& st, bool
   if (valid && lse) lse[row] = seen ? (st.m_run + log2f(st.l_run)) * 0.69314718055994531f : -INFINITY;
 }
 
+// Split-KV: the row's result over this item's key range, out / l in fp32 and its lse
+// (natural log), into partial slot row `srow`; merged later by merge_partials_kernel.
+template <int D>
+__device__ __forceinline__ void store_partial(uint32_t t_o, const RowState& st, bool valid, int64_t srow, float* po,
+                                              float* plse) {
+  const bool seen = st.m_run != -INFINITY;
+  const float inv = seen ? 1.f / st.l_run : 0.f;
+#pragma unroll 1
+  for (int cc = 0; cc < D / 32; ++cc) {
+    uint32_t o[32];
+    tmem_ld32x32(t_o + cc * 32, o);
+    tmem_wait_ld();
+    if (valid) {
+      float4* dst = reinterpret_cast<float4*>(po + srow * D + cc * 32);
+#pragma unroll
+      for (int e = 0; e < 8; ++e)
+        dst[e] = make_float4(__uint_as_float(o[4 * e]) * inv, __uint_as_float(o[4 * e + 1]) * inv,
+                             __uint_as_float(o[4 * e + 2]) * inv, __uint_as_float(o[4 * e + 3]) * inv);
+    }
+  }
+  if (valid) plse[srow] = seen ? (st.m_run + log2f(st.l_run)) * 0.69314718055994531f : -INFINITY;
+}
+
 // ---- the kernel ----------------------------------------------------------------------------
 
 enum : int32_t {
@@ -772,7 +797,10 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_fwd_kernel(const __
       ++pvc;
       tc_fence_after();
       const int lr = r % p.R, hh = r / p.R;
-      store_row<C::D>(t_o, st, lr < it.rows[q], int64_t(it.tok[q] + lr) * p.hq + it.head[q] + hh, p.out, p.lse);
+      if (it.part < 0)
+        store_row<C::D>(t_o, st, lr < it.rows[q], int64_t(it.tok[q] + lr) * p.hq + it.head[q] + hh, p.out, p.lse);
+      else
+        store_partial<C::D>(t_o, st, lr < it.rows[q], int64_t(it.part + q) * kSlotRows + r, p.part_o, p.part_lse);
       tc_fence_before();
       mbar_arrive(BAR(C::B_OEMPTY + q));
       sj += T;
@@ -1047,8 +1075,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::THREADS, 1)
       ++pvc;
       tc_fence_after();
       const int lr = r % p.R, hh = r / p.R;
-      store_row<C::D>(t_o, st, lr < it.rows[rank], int64_t(it.tok[rank] + lr) * p.hq + it.head[rank] + hh, p.out,
-                      p.lse);
+      if (it.part < 0)
+        store_row<C::D>(t_o, st, lr < it.rows[rank], int64_t(it.tok[rank] + lr) * p.hq + it.head[rank] + hh, p.out,
+                        p.lse);
+      else
+        store_partial<C::D>(t_o, st, lr < it.rows[rank], int64_t(it.part + int(rank)) * kSlotRows + r, p.part_o,
+                            p.part_lse);
       tc_fence_before();
       warp_arrive_leader(LBAR(C::B_OEMPTY));
       sj += T;
@@ -1065,6 +1097,58 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::THREADS, 1)
 __global__ void exp2_poly_kernel(const float* __restrict__ x, float* __restrict__ y, int64_t n) {
   for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < n; i += int64_t(gridDim.x) * blockDim.x)
     y[i] = exp2_poly(x[i]);
+}
+
+// Split-KV merge. With lse_r the partial lse of key range r and o_r its out / l:
+// lse = m + ln sum_r exp(lse_r - m) (m = max_r lse_r), out = sum_r exp(lse_r - lse) o_r;
+// a row that saw no key in any range gets out = 0, lse = -inf. Grid (merge tiles,
+// kSlotRows / 8): one warp per row; the lanes first share out the range weights (kept in
+// shared memory), then each lane sums the ranges for its 4-column groups.
+constexpr int kMergeRowsPerBlock = 8;
+__global__ void __launch_bounds__(32 * kMergeRowsPerBlock) merge_partials_kernel(
+    const MergeTile* __restrict__ tiles, const float* __restrict__ part_o, const float* __restrict__ part_lse, int D,
+    int R, int hq, __nv_bfloat16* __restrict__ out, float* __restrict__ lse) {
+  __shared__ float wsh[kMergeRowsPerBlock][kMaxSplits];
+  const MergeTile t = tiles[blockIdx.x];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int r = blockIdx.y * kMergeRowsPerBlock + warp;
+  const int lr = r % R, hh = r / R;
+  if (lr >= t.rows) return;
+  const int64_t orow = int64_t(t.tok + lr) * hq + t.head + hh;
+  float m = -INFINITY;
+  for (int k = lane; k < t.nsplit; k += 32) m = fmaxf(m, part_lse[int64_t(t.slot0 + k * t.stride) * kSlotRows + r]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if (m == -INFINITY) {
+    for (int c = 4 * lane; c < D; c += 128) *reinterpret_cast<uint2*>(out + orow * D + c) = make_uint2(0u, 0u);
+    if (lse && lane == 0) lse[orow] = -INFINITY;
+    return;
+  }
+  float wsum = 0.f;
+  for (int k = lane; k < t.nsplit; k += 32) {
+    const float w = expf(part_lse[int64_t(t.slot0 + k * t.stride) * kSlotRows + r] - m);
+    wsh[warp][k] = w;
+    wsum += w;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, o);
+  __syncwarp();
+  const float inv = 1.f / wsum;
+  for (int c = 4 * lane; c < D; c += 128) {
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+    for (int k = 0; k < t.nsplit; ++k) {
+      const float w = wsh[warp][k];
+      const float4 o = *reinterpret_cast<const float4*>(part_o + (int64_t(t.slot0 + k * t.stride) * kSlotRows + r) * D + c);
+      acc.x = fmaf(w, o.x, acc.x);
+      acc.y = fmaf(w, o.y, acc.y);
+      acc.z = fmaf(w, o.z, acc.z);
+      acc.w = fmaf(w, o.w, acc.w);
+    }
+    *reinterpret_cast<uint2*>(out + orow * D + c) =
+        make_uint2(pack_bf16(acc.x * inv, acc.y * inv), pack_bf16(acc.z * inv, acc.w * inv));
+  }
+  if (lse && lane == 0) lse[orow] = m + logf(wsum);
 }
 
 // Rows of a problem without any key at all: out = 0, lse = -inf.
@@ -1172,6 +1256,8 @@ attn_status_t mfa_launch_forward(const attn_plan_t* plan, const void* q, const v
   p.page_table = plan->page_table;
   p.out = static_cast<__nv_bfloat16*>(out);
   p.lse = lse;
+  p.part_o = plan->d_part_o;
+  p.part_lse = plan->d_part_lse;
   p.status = plan->d_status;
   p.hq = plan->hq;
   p.R = plan->R;
@@ -1181,16 +1267,22 @@ attn_status_t mfa_launch_forward(const attn_plan_t* plan, const void* q, const v
   p.debug_flags = plan->debug_flags;
   p.scale_log2 = plan->scale * 1.4426950408889634f;
   p.timeout_ns = plan->timeout_ns;
+  attn_status_t st;
   if (D == 64) {
-    return plan->paged ? launch<Cfg<64, 2, 10, true, MFA_EMU_D128>>(plan, p, stream)
-                       : launch<Cfg<64, 2, 10, false, MFA_EMU_D128>>(plan, p, stream);
+    st = plan->paged ? launch<Cfg<64, 2, 10, true, MFA_EMU_D128>>(plan, p, stream)
+                     : launch<Cfg<64, 2, 10, false, MFA_EMU_D128>>(plan, p, stream);
   } else if (D == 128) {
-    return plan->paged ? launch<Cfg<128, 2, 5, true, MFA_EMU_D128>>(plan, p, stream)
-                       : launch<Cfg<128, 2, 5, false, MFA_EMU_D128>>(plan, p, stream);
+    st = plan->paged ? launch<Cfg<128, 2, 5, true, MFA_EMU_D128>>(plan, p, stream)
+                     : launch<Cfg<128, 2, 5, false, MFA_EMU_D128>>(plan, p, stream);
   } else {
-    return plan->paged ? launch_pair<PairCfg<256, 5, true>>(plan, p, stream)
-                       : launch_pair<PairCfg<256, 5, false>>(plan, p, stream);
+    st = plan->paged ? launch_pair<PairCfg<256, 5, true>>(plan, p, stream)
+                     : launch_pair<PairCfg<256, 5, false>>(plan, p, stream);
   }
+  if (st != ATTN_OK || plan->n_merge == 0) return st;
+  const dim3 grid(plan->n_merge, kSlotRows / kMergeRowsPerBlock);
+  merge_partials_kernel<<<grid, 32 * kMergeRowsPerBlock, 0, stream>>>(plan->d_merge, plan->d_part_o, plan->d_part_lse,
+                                                                     D, plan->R, plan->hq, p.out, lse);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
 extern "C" attn_status_t attn_test_exp2_poly(const float* x, float* y, int64_t n, attn_stream_t stream) {

@@ -33,9 +33,25 @@ struct alignas(16) WorkItem {
   int32_t job_start;
   int32_t job_count;
   int32_t npages;      // paged: pages that hold the sequence's keys
-  int32_t pad;
+  int32_t part;        // -1: write out / lse; else query tile t writes partial slot part + t
 };
 static_assert(sizeof(WorkItem) == 64, "WorkItem layout");
+
+// A query tile whose key tiles were split over several work items (split-KV): its rows'
+// partial results sit in slots slot0, slot0 + stride, ... (nsplit of them) and are merged
+// into out / lse by the merge kernel. Rows as in WorkItem (tile row r: token tok + r % R,
+// head head + r / R, valid when r % R < rows).
+struct alignas(16) MergeTile {
+  int32_t tok, head, rows;
+  int32_t slot0, nsplit, stride;
+  int32_t pad[2];
+};
+static_assert(sizeof(MergeTile) == 32, "MergeTile layout");
+
+// Partial-result slots: 128 rows x head_dim fp32 (out / l) and 128 fp32 lse values each.
+constexpr int kSlotRows = 128;
+// Most key ranges one query tile is split into (the merge kernel keeps that many weights per row).
+constexpr int kMaxSplits = 256;
 
 // One key tile of a work item and, per query tile, how to mask it.
 struct alignas(16) Job {
@@ -88,6 +104,11 @@ struct attn_plan {
   const int32_t* d_cta_off = nullptr;
   const int32_t* d_cta_items = nullptr;
   const uint4* d_mask_tiles = nullptr;
+  // split-KV: partial slots and the tiles to merge (none when nothing was split)
+  float* d_part_o = nullptr;
+  float* d_part_lse = nullptr;
+  const mfa::MergeTile* d_merge = nullptr;
+  int32_t n_merge = 0;
   // debug hooks
   int32_t debug_flags = 0;
   int64_t timeout_ns = 2000000000LL;

@@ -54,6 +54,7 @@ struct Shape {
   int ps = 0, maxp = 0, npages = 0;
   std::vector<int32_t> lq, lk, qoff, koff;
   int64_t total_q = 0, total_kv_rows = 0;
+  int kv_splits = 0;   // 0 automatic, 1 never, N >= 2 at most N key ranges per query tile
 };
 
 attn_status_t validate_problem(const attn_problem_t* p, Shape& s, bool need_device_ptrs = true) {
@@ -62,6 +63,8 @@ attn_status_t validate_problem(const attn_problem_t* p, Shape& s, bool need_devi
   if (p->hq % p->hkv != 0) return ATTN_ERR_INVALID_ARG;
   if (p->head_dim != 64 && p->head_dim != 128 && p->head_dim != 256) return ATTN_ERR_UNSUPPORTED;
   if (std::isnan(p->scale) || std::isinf(p->scale)) return ATTN_ERR_INVALID_ARG;
+  if (p->kv_splits < 0) return ATTN_ERR_INVALID_ARG;
+  s.kv_splits = p->kv_splits;
   s.B = p->batch;
   s.hq = p->hq;
   s.hkv = p->hkv;
@@ -395,10 +398,103 @@ struct WorkList {
   std::vector<Job> jobs;
   std::vector<TileRef> mask_tiles;   // in index order
   std::vector<int32_t> cta_off, cta_items;
+  std::vector<MergeTile> merge;      // split-KV: query tiles to merge
+  int32_t slots = 0;                 // split-KV: partial-result slots
+  int32_t splits_max = 1;
 };
 
+// Greedy least-loaded assignment of costs (taken in the given order) onto `units`: the
+// largest load, i.e. the modelled makespan.
+int64_t greedy_makespan(const std::vector<int64_t>& costs, int units) {
+  using Load = std::pair<int64_t, int32_t>;
+  std::priority_queue<Load, std::vector<Load>, std::greater<Load>> heap;
+  for (int c = 0; c < units; ++c) heap.push(Load{0, c});
+  int64_t worst = 0;
+  for (int64_t x : costs) {
+    Load l = heap.top();
+    heap.pop();
+    l.first += x;
+    worst = std::max(worst, l.first);
+    heap.push(l);
+  }
+  return worst;
+}
+
+// Split-KV. A work item's key tiles may be cut into n consecutive ranges, each a work item
+// of its own that writes partial results (out / l and lse per row) to its own slots; the
+// merge kernel combines them by lse. Forced (kv_splits = N >= 2): every item with >= 2 key
+// tiles into min(N, tiles) ranges. Automatic (kv_splits = 0): a cost model in key-tile
+// units -- an item (or range) costs its tiles + 2 (Q load, pipeline start, epilogue), the
+// merge costs one tile per partial slot spread over all units -- picks the range length
+// P = ceil(longest / n), n = 1 .. 64, whose longest-first greedy schedule plus merge is
+// shortest; the split is kept only when that beats the unsplit makespan by more than 15 %.
+void split_items(const Shape& s, int units, int nq, WorkList& wl) {
+  if (s.kv_splits == 1 || wl.items.empty()) return;
+  auto pieces_of = [&](const WorkItem& it, int64_t P) -> int {
+    int n = 1;
+    if (s.kv_splits >= 2) n = it.job_count >= 2 ? std::min(s.kv_splits, it.job_count) : 1;
+    else if (P > 0) n = int((it.job_count + P - 1) / P);
+    return std::max(1, std::min(n, kMaxSplits));
+  };
+  int64_t best_P = 0;   // 0: no split
+  if (s.kv_splits == 0) {
+    int64_t longest = 0;
+    for (const WorkItem& it : wl.items) longest = std::max<int64_t>(longest, it.job_count);
+    auto cost = [&](int64_t P) {
+      std::vector<int64_t> costs;
+      int64_t slots = 0;
+      for (const WorkItem& it : wl.items) {
+        const int n = P > 0 ? pieces_of(it, P) : 1;
+        for (int c = 0; c < n; ++c)
+          costs.push_back(int64_t(it.job_count) * (c + 1) / n - int64_t(it.job_count) * c / n + 2);
+        if (n > 1) slots += int64_t(n) * nq;
+      }
+      std::sort(costs.begin(), costs.end(), std::greater<int64_t>());
+      return greedy_makespan(costs, units) + (slots + units - 1) / units;
+    };
+    const int64_t base = cost(0);
+    int64_t total = 0;
+    for (const WorkItem& it : wl.items) total += it.job_count + 2;
+    if (100 * base <= 115 * ((total + units - 1) / units)) return;   // already balanced
+    int64_t best = base;
+    for (int n = 2; n <= 64; ++n) {
+      const int64_t P = std::max<int64_t>(4, (longest + n - 1) / n);
+      const int64_t c = cost(P);
+      if (c < best) {
+        best = c;
+        best_P = P;
+      }
+      if (P == 4) break;
+    }
+    if (best_P == 0 || 100 * best >= 85 * base) return;
+  }
+  std::vector<WorkItem> out;
+  out.reserve(wl.items.size());
+  for (const WorkItem& it : wl.items) {
+    const int n = pieces_of(it, best_P);
+    if (n <= 1) {
+      out.push_back(it);
+      continue;
+    }
+    const int32_t slot0 = wl.slots;
+    for (int c = 0; c < n; ++c) {
+      WorkItem p = it;
+      const int32_t j0 = int32_t(int64_t(it.job_count) * c / n), j1 = int32_t(int64_t(it.job_count) * (c + 1) / n);
+      p.job_start = it.job_start + j0;
+      p.job_count = j1 - j0;
+      p.part = slot0 + c * nq;
+      out.push_back(p);
+    }
+    wl.slots += n * nq;
+    for (int t = 0; t < nq; ++t)
+      if (it.rows[t] > 0) wl.merge.push_back(MergeTile{it.tok[t], it.head[t], it.rows[t], slot0 + t, n, nq, {0, 0}});
+    wl.splits_max = std::max(wl.splits_max, n);
+  }
+  wl.items.swap(out);
+}
+
 void build_work(const Shape& s, int R, int hp, int nq, const std::vector<std::vector<int32_t>>& cnts,
-                int num_sms, WorkList& wl) {
+                int num_sms, WorkList& wl, bool allow_split = true) {
   const int g = s.hq / s.hkv;
   const int G = g / hp;  // head groups per kv head
   for (int b = 0; b < s.B; ++b) {
@@ -426,6 +522,7 @@ void build_work(const Shape& s, int R, int hp, int nq, const std::vector<std::ve
     };
     auto add_item = [&](int kh, int rb0, int hg0, int rb1, int hg1) {
       WorkItem it{};
+      it.part = -1;
       it.seq = b;
       it.kv_head = kh;
       it.k_base = s.koff[b];
@@ -466,6 +563,7 @@ void build_work(const Shape& s, int R, int hp, int nq, const std::vector<std::ve
       }
     }
   }
+  if (allow_split) split_items(s, num_sms, nq, wl);
   // Greedy balancing onto persistent CTAs: each item goes to the least-loaded CTA. Items are
   // taken group by group -- a group being one (sequence, key/value head), the largest
   // groups first -- and, inside a group, longest first. Items of one group then run at
@@ -527,17 +625,21 @@ void write_mask_tile(RowSource& src, const Shape& s, int R, const TileRef& t, ui
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 struct Staging {
-  size_t off_items, off_jobs, off_cta_off, off_cta_items, off_tiles, total;
+  size_t off_items, off_jobs, off_cta_off, off_cta_items, off_tiles, off_merge, off_part_lse, off_part_o, total;
 };
 
-Staging layout(const WorkList& wl) {
+// [status | items | jobs | cta_off | cta_items | mask tiles | merge tiles | partial lse | partial out]
+Staging layout(const WorkList& wl, int d) {
   Staging st{};
   st.off_items = 256;
   st.off_jobs = align256(st.off_items + wl.items.size() * sizeof(WorkItem));
   st.off_cta_off = align256(st.off_jobs + wl.jobs.size() * sizeof(Job));
   st.off_cta_items = align256(st.off_cta_off + wl.cta_off.size() * sizeof(int32_t));
   st.off_tiles = align256(st.off_cta_items + wl.cta_items.size() * sizeof(int32_t));
-  st.total = st.off_tiles + wl.mask_tiles.size() * size_t(kMaskTileBytes);
+  st.off_merge = align256(st.off_tiles + wl.mask_tiles.size() * size_t(kMaskTileBytes));
+  st.off_part_lse = align256(st.off_merge + wl.merge.size() * sizeof(MergeTile));
+  st.off_part_o = align256(st.off_part_lse + size_t(wl.slots) * kSlotRows * sizeof(float));
+  st.total = st.off_part_o + size_t(wl.slots) * kSlotRows * size_t(d) * sizeof(float);
   return st;
 }
 
@@ -645,6 +747,25 @@ attn_status_t custom_repack(const attn_mask_desc_t* m, const Shape& s, int R, co
   return cuda_status(e);
 }
 
+// Work-list part of the plan statistics.
+void work_stats(const attn_plan_t& m, const WorkList& wl, attn_plan_stats_t& st) {
+  st.mask_tiles = int64_t(wl.mask_tiles.size());
+  st.work_items = int64_t(wl.items.size());
+  int64_t jobs = 0;
+  for (const WorkItem& it : wl.items) jobs += it.job_count;   // a split item's ranges share its jobs
+  st.jobs = jobs;
+  st.mask_tile_reads = 0;
+  for (const WorkItem& it : wl.items)
+    for (int j = it.job_start; j < it.job_start + it.job_count; ++j)
+      for (int t = 0; t < 2; ++t) st.mask_tile_reads += wl.jobs[j].mask[t] >= 0 ? 1 : 0;
+  st.ctas = m.ctas * m.cluster;
+  st.heads_per_tile = m.hp;
+  st.tiles_per_cta = m.nq / m.cluster;
+  st.cluster_size = m.cluster;
+  st.kv_splits_max = wl.splits_max;
+  st.merge_tiles = int32_t(wl.merge.size());
+}
+
 attn_status_t plan_impl(const attn_problem_t* problem, const attn_mask_desc_t* mask, cudaStream_t stream,
                         attn_plan_t** out_plan) {
   if (!out_plan) return ATTN_ERR_INVALID_ARG;
@@ -696,17 +817,9 @@ attn_status_t plan_impl(const attn_problem_t* problem, const attn_mask_desc_t* m
   WorkList wl;
   build_work(s, R, plan->hp, plan->nq, cnts, num_sms / plan->cluster, wl);
   plan->ctas = int32_t(wl.cta_off.size()) - 1;   // work units: CTAs, or CTA pairs
-  plan->stats.mask_tiles = int64_t(wl.mask_tiles.size());
-  plan->stats.work_items = int64_t(wl.items.size());
-  plan->stats.jobs = int64_t(wl.jobs.size());
-  for (const Job& j : wl.jobs)
-    for (int t = 0; t < 2; ++t) plan->stats.mask_tile_reads += j.mask[t] >= 0 ? 1 : 0;
-  plan->stats.ctas = plan->ctas * plan->cluster;
-  plan->stats.heads_per_tile = plan->hp;
-  plan->stats.tiles_per_cta = plan->nq / plan->cluster;
-  plan->stats.cluster_size = plan->cluster;
+  work_stats(*plan, wl, plan->stats);
 
-  const Staging lay = layout(wl);
+  const Staging lay = layout(wl, s.d);
   std::vector<char> host(lay.off_tiles, 0);
   std::memcpy(host.data() + lay.off_items, wl.items.data(), wl.items.size() * sizeof(WorkItem));
   std::memcpy(host.data() + lay.off_jobs, wl.jobs.data(), wl.jobs.size() * sizeof(Job));
@@ -738,9 +851,18 @@ attn_status_t plan_impl(const attn_problem_t* problem, const attn_mask_desc_t* m
   plan->d_cta_off = reinterpret_cast<const int32_t*>(base + lay.off_cta_off);
   plan->d_cta_items = reinterpret_cast<const int32_t*>(base + lay.off_cta_items);
   plan->d_mask_tiles = reinterpret_cast<const uint4*>(base + lay.off_tiles);
+  if (!wl.merge.empty()) {
+    plan->d_merge = reinterpret_cast<const MergeTile*>(base + lay.off_merge);
+    plan->n_merge = int32_t(wl.merge.size());
+    plan->d_part_lse = reinterpret_cast<float*>(base + lay.off_part_lse);
+    plan->d_part_o = reinterpret_cast<float*>(base + lay.off_part_o);
+  }
   e = cudaMemcpyAsync(base, host.data(), host.size(), cudaMemcpyHostToDevice, stream);
   if (e == cudaSuccess && !tiles.empty())
     e = cudaMemcpyAsync(base + lay.off_tiles, tiles.data(), tiles.size() * 4, cudaMemcpyHostToDevice, stream);
+  if (e == cudaSuccess && !wl.merge.empty())
+    e = cudaMemcpyAsync(base + lay.off_merge, wl.merge.data(), wl.merge.size() * sizeof(MergeTile),
+                        cudaMemcpyHostToDevice, stream);
   if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
   st = cuda_status(e);
   if (st == ATTN_OK && mask->kind == ATTN_MASK_CUSTOM)
@@ -790,9 +912,9 @@ attn_status_t mfa_plan_host(const attn_problem_t* problem, const attn_mask_desc_
       count_sequence(src, b, s, R, cnts[b]);
     }
     WorkList wl;
-    build_work(s, R, m.hp, m.nq, cnts, num_sms / m.cluster, wl);
+    build_work(s, R, m.hp, m.nq, cnts, num_sms / m.cluster, wl, /*allow_split=*/false);
     m.ctas = int32_t(wl.cta_off.size()) - 1;
-    const Staging lay = layout(wl);
+    const Staging lay = layout(wl, s.d);
     out->off_items = lay.off_items;
     out->off_jobs = lay.off_jobs;
     out->off_cta_off = lay.off_cta_off;
@@ -820,6 +942,41 @@ attn_status_t mfa_plan_host(const attn_problem_t* problem, const attn_mask_desc_
 }
 
 extern "C" {
+
+attn_status_t attn_plan_dry_run(const attn_problem_t* problem, const attn_mask_desc_t* mask, int32_t num_sms,
+                                attn_plan_stats_t* stats) {
+  try {
+    if (!stats || num_sms <= 0) return ATTN_ERR_INVALID_ARG;
+    if (mask && mask->kind == ATTN_MASK_CUSTOM) return ATTN_ERR_UNSUPPORTED;
+    Shape s;
+    attn_status_t st = validate_problem(problem, s, /*need_device_ptrs=*/false);
+    if (st != ATTN_OK) return st;
+    st = validate_mask(mask, s);
+    if (st != ATTN_OK) return st;
+    attn_plan_t m;
+    m.batch = s.B;
+    m.hq = s.hq;
+    m.hkv = s.hkv;
+    m.d = s.d;
+    choose_shape(s, m);
+    attn_plan_stats_t out{};
+    std::vector<std::vector<int32_t>> cnts(s.B);
+    RowSource src(mask, s);
+    for (int b = 0; b < s.B; ++b) {
+      src.prepare(b);
+      count_sequence(src, b, s, m.R, cnts[b]);
+      report_classes(cnts[b], s.lq[b], s.lk[b], m.R, m.classes, out);
+    }
+    WorkList wl;
+    build_work(s, m.R, m.hp, m.nq, cnts, num_sms / m.cluster, wl);
+    m.ctas = int32_t(wl.cta_off.size()) - 1;
+    work_stats(m, wl, out);
+    *stats = out;
+    return ATTN_OK;
+  } catch (const std::bad_alloc&) {
+    return ATTN_ERR_OOM;
+  }
+}
 
 attn_status_t attn_plan(const attn_problem_t* problem, const attn_mask_desc_t* mask, attn_stream_t stream,
                         attn_plan_t** out_plan) {

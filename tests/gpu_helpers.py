@@ -20,9 +20,9 @@ def device_inputs(wl, dev="cuda"):
     return q, wl.k.to(dev), wl.v.to(dev)
 
 
-def make_plan(wl, spec, dev="cuda", stream=None):
+def make_plan(wl, spec, dev="cuda", stream=None, kv_splits=0):
     kw = dict(hq=wl.hq, hkv=wl.hkv, head_dim=wl.d, cu_seqlens_q=wl.cu_seqlens_q, mask=spec, scale=wl.scale,
-              stream=stream)
+              stream=stream, kv_splits=kv_splits)
     if wl.paged:
         kw.update(kv_lens=wl.kv_lens, page_table=torch.from_numpy(wl.page_table).to(dev),
                   page_size=wl.page_size, num_pages=wl.k_cache.shape[0])
@@ -31,11 +31,11 @@ def make_plan(wl, spec, dev="cuda", stream=None):
     return M.attn_plan(**kw)
 
 
-def run(wl, spec, inputs=None, extra_rows=0, canary=None):
+def run(wl, spec, inputs=None, extra_rows=0, canary=None, kv_splits=0):
     """Plan + forward; returns (out fp32 [total_q, hq, d], lse [total_q, hq], plan).
     ``extra_rows`` canary-filled rows follow the real ones in the output buffers."""
     q, k, v = inputs if inputs is not None else device_inputs(wl)
-    plan = make_plan(wl, spec)
+    plan = make_plan(wl, spec, kv_splits=kv_splits)
     tq = int(wl.cu_seqlens_q[-1])
     out = torch.empty(tq + extra_rows, wl.hq, wl.d, dtype=torch.bfloat16, device="cuda")
     lse = torch.empty(tq + extra_rows, wl.hq, dtype=torch.float32, device="cuda")
@@ -68,9 +68,9 @@ def lengths(wl):
     return [(wl.lq(b), wl.lk(b)) for b in range(wl.batch)]
 
 
-def check_full(wl, spec, what=""):
+def check_full(wl, spec, what="", kv_splits=0):
     """Whole-output comparison against the full oracle (small problems)."""
-    out, lse, plan = run(wl, spec)
+    out, lse, plan = run(wl, spec, kv_splits=kv_splits)
     ref_out, ref_lse = oracle.masked_attention(wl, spec)
     cls = M.attn_plan_get_tile_classes(plan)
     assert np.array_equal(cls, oracle.tile_classes(spec, lengths(wl))), f"{what}: tile classes"

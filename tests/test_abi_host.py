@@ -160,3 +160,43 @@ def test_empty_and_degenerate_lengths(attn_lib):
     cls, pairs = M.attn_classify_host(hq=2, hkv=1, head_dim=64, cu_seqlens_q=np.array([0], np.int32),
                                       cu_seqlens_k=np.array([0], np.int32), mask=W.MaskSpec("FULL"))
     assert len(cls) == 0
+
+
+def test_dry_run_split_kv_decisions(attn_lib):
+    """Split-KV planning on the host (attn_plan_dry_run): few long work items are cut into
+    key ranges, the ranges cover each item's key tiles exactly once, and balanced
+    workloads are left alone."""
+    M = attn_lib
+    lq, lk = [64] * 4, [23740, 25265, 24931, 22072]          # 4 requests x 8 KV heads = 32 items
+    base = dict(hq=32, hkv=8, head_dim=128, cu_seqlens_q=W.cu_from_lengths(lq),
+                cu_seqlens_k=W.cu_from_lengths(lk), mask=W.MaskSpec("CAUSAL"))
+    never = M.attn_plan_dry_run(kv_splits=1, **base)
+    assert never["work_items"] == 32 and never["kv_splits_max"] == 1 and never["merge_tiles"] == 0
+    auto = M.attn_plan_dry_run(kv_splits=0, **base)
+    assert auto["kv_splits_max"] >= 3 and auto["work_items"] >= 128
+    assert auto["merge_tiles"] == 64                          # 32 items x 2 query tiles
+    assert auto["jobs"] == never["jobs"] and auto["mask_tile_reads"] == never["mask_tile_reads"]
+    assert auto["unmasked_pairs"] == never["unmasked_pairs"]
+    for n in (2, 7):
+        forced = M.attn_plan_dry_run(kv_splits=n, **base)
+        assert forced["work_items"] == 32 * n and forced["kv_splits_max"] == n
+        assert forced["jobs"] == never["jobs"]
+    # fewer SMs than items: no split is worth it
+    assert M.attn_plan_dry_run(kv_splits=0, num_sms=32, **base)["kv_splits_max"] == 1
+    # the balanced benchmark workloads (analytic masks) are not split
+    for c in (1, 2, 4, 5):
+        wl = W.config(c)
+        for spec in wl.masks:
+            if spec.kind == "CUSTOM":
+                continue
+            st = M.attn_plan_dry_run(hq=wl.hq, hkv=wl.hkv, head_dim=wl.d, cu_seqlens_q=wl.cu_seqlens_q,
+                                     cu_seqlens_k=wl.cu_seqlens_k, mask=spec)
+            assert st["kv_splits_max"] == 1 and st["merge_tiles"] == 0, (c, spec.kind)
+    assert _err_dry(M, kv_splits=-1, **base) == 1
+    assert _err_dry(M, num_sms=0, **base) == 1
+
+
+def _err_dry(M, **kw):
+    with pytest.raises(M.AttnError) as e:
+        M.attn_plan_dry_run(**kw)
+    return e.value.status

@@ -291,12 +291,22 @@ def block_dense_custom(seed: int = 5, L: int = 29576, dense_rows: int = 24576, b
                        1.0 / np.sqrt(d), masks)
 
 
+def tree_verify_long_paged(seed: int = 6, requests: int = 4) -> Workload:
+    """Long-context tree verify (split-KV case): the tree-verify recipe with 4 requests and
+    prefixes P ~ U[16384, 32768]; 32 (request, KV head) work items alone would fill 32 of
+    148 SMs, so the key range of every item is split."""
+    wl = tree_verify_paged(seed=seed, requests=requests, plo=16384, phi=32768)
+    wl.name = "tree_verify_long_paged_d128"
+    return wl
+
+
 CONFIGS = {
     1: prefix_lm_small,
     2: gemma2_local_global,
     3: tree_verify_paged,
     4: chunk_causal_interleaved,
     5: block_dense_custom,
+    6: tree_verify_long_paged,
 }
 
 
