@@ -9,6 +9,8 @@ Contents
   masks.py      dense boolean mask per descriptor kind, bit unpacking,
                 128x128 tile classes and unmasked-pair counts from the dense mask
   attention.py  O = softmax(scale * Q K^T + mask) V and the row log-sum-exp, fp64
+  backward.py   dQ, dK, dV of that forward for a given dO (chain rule through the row
+                softmax), fp64
 
 Every function is pinned by the CPU tests (tests/test_oracle_*.py) to facts
 the pages or the mathematics fix: the pages' worked chunk-causal example,
@@ -18,7 +20,9 @@ tiny inputs and the library softmax on unmasked rows.
 from .masks import (dense_mask_rows, dense_mask, unpack_rows, tile_classes, unmasked_pairs,
                     CLASS_EMPTY, CLASS_FULL, CLASS_PARTIAL)
 from .attention import attention_one_head, masked_attention, sampled_attention
+from .backward import attention_backward_one_head, masked_attention_backward
 
 __all__ = ["dense_mask_rows", "dense_mask", "unpack_rows", "tile_classes", "unmasked_pairs",
            "CLASS_EMPTY", "CLASS_FULL", "CLASS_PARTIAL",
-           "attention_one_head", "masked_attention", "sampled_attention"]
+           "attention_one_head", "masked_attention", "sampled_attention",
+           "attention_backward_one_head", "masked_attention_backward"]

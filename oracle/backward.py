@@ -1,0 +1,73 @@
+"""fp64 gradients of the masked attention forward (oracle; test infrastructure only).
+
+The forward (oracle.attention) is, per sequence and query head h with key/value head
+kh = floor(h / g), g = Hq / Hkv:
+
+    s_ij = scale * q_i . k_j,  p_ij = exp(s_ij - lse_i) on visible (i, j), 0 elsewhere,
+    out_i = sum_j p_ij v_j.
+
+For a loss whose gradient with respect to out is dout (lse treated as an output without
+a gradient of its own), the chain rule through the row softmax gives
+
+    dv_j  = sum_i p_ij dout_i
+    dp_ij = dout_i . v_j
+    D_i   = sum_j p_ij dp_ij  ( = dout_i . out_i )
+    ds_ij = p_ij (dp_ij - D_i)
+    dq_i  = scale * sum_j ds_ij k_j
+    dk_j  = scale * sum_i ds_ij q_i
+
+and dk, dv of a key/value head are the sums over the g query heads that read it. A row
+that sees no key has p = 0 and contributes nothing. These are the textbook derivatives of
+softmax(scale Q K^T + mask) V; nothing here is taken from the CUDA path.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+from .attention import attention_one_head, _f64
+from .masks import dense_mask
+
+
+def attention_backward_one_head(q, k, v, mask, scale, dout):
+    """q [n, d], k, v [L_k, d], mask bool [n, L_k], dout [n, d]; fp64.
+    Returns (dq [n, d], dk [L_k, d], dv [L_k, d])."""
+    out, lse = attention_one_head(q, k, v, mask, scale)
+    has = np.isfinite(lse)
+    s = scale * (q @ k.T)
+    p = np.where(mask & has[:, None], np.exp(np.where(mask, s, 0.0) - np.where(has, lse, 0.0)[:, None]), 0.0)
+    dv = p.T @ dout
+    dp = dout @ v.T
+    big_d = np.sum(p * dp, axis=1)
+    ds = p * (dp - big_d[:, None])
+    dq = scale * (ds @ k)
+    dk = scale * (ds.T @ q)
+    return dq, dk, dv
+
+
+def masked_attention_backward(wl, spec, dout):
+    """Gradients over a contiguous workload: dout [total_q, Hq, d] (torch or numpy).
+    Returns (dq fp64 [total_q, Hq, d], dk, dv fp64 [total_k, Hkv, d])."""
+    if wl.paged:
+        raise ValueError("backward oracle: contiguous K/V only")
+    dout = dout.to(__import__("torch").float64).numpy() if hasattr(dout, "numpy") else np.asarray(dout, np.float64)
+    g = wl.hq // wl.hkv
+    total_q, total_k = int(wl.cu_seqlens_q[-1]), int(wl.cu_seqlens_k[-1])
+    dq = np.zeros((total_q, wl.hq, wl.d))
+    dk = np.zeros((total_k, wl.hkv, wl.d))
+    dv = np.zeros((total_k, wl.hkv, wl.d))
+    for b in range(wl.batch):
+        lq, lk = wl.lq(b), wl.lk(b)
+        q0, k0 = int(wl.cu_seqlens_q[b]), int(wl.cu_seqlens_k[b])
+        if lq == 0 or lk == 0:
+            continue
+        m = dense_mask(spec, b, lq, lk)
+        kk, vv = wl.kv_of_seq(b)
+        kk, vv = _f64(kk), _f64(vv)
+        for h in range(wl.hq):
+            kh = h // g
+            a, bk, bv = attention_backward_one_head(_f64(wl.q[q0:q0 + lq, h]), kk[:, kh], vv[:, kh], m, wl.scale,
+                                                    dout[q0:q0 + lq, h])
+            dq[q0:q0 + lq, h] = a
+            dk[k0:k0 + lk, kh] += bk
+            dv[k0:k0 + lk, kh] += bv
+    return dq, dk, dv

@@ -1,0 +1,121 @@
+"""Pins of the fp64 backward oracle (oracle/backward.py) to facts outside itself:
+central finite differences of the pinned forward oracle, the autograd of the library
+softmax / matmul on unmasked and causal rows, the softmax-gradient invariant
+(sum_j ds_ij = 0, hence sum_j dk_j = 0), zero gradients for rows that see no key, and
+the grouped-query sum. Planted mistakes (a dropped D term, a missing scale, a transposed
+ds) must each fail one of them."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import oracle.backward as OB
+import workloads as W
+
+
+def _case(seed, n=5, lk=7, d=4, density=0.6, empty_row=True):
+    rng = np.random.default_rng(seed)
+    q, k, v, do = (rng.standard_normal(s) for s in ((n, d), (lk, d), (lk, d), (n, d)))
+    mask = rng.random((n, lk)) < density
+    mask[0, :] = True
+    if empty_row:
+        mask[1, :] = False
+    return q, k, v, do, mask
+
+
+def _loss(q, k, v, mask, scale, do):
+    out, _ = oracle.attention_one_head(q, k, v, mask, scale)
+    return float(np.sum(out * do))
+
+
+def _fd(f, x, h=1e-6):
+    g = np.zeros_like(x)
+    for idx in np.ndindex(*x.shape):
+        xp, xm = x.copy(), x.copy()
+        xp[idx] += h
+        xm[idx] -= h
+        g[idx] = (f(xp) - f(xm)) / (2 * h)
+    return g
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_finite_differences(seed):
+    q, k, v, do, mask = _case(seed)
+    scale = 0.7
+    dq, dk, dv = OB.attention_backward_one_head(q, k, v, mask, scale, do)
+    assert np.allclose(dq, _fd(lambda x: _loss(x, k, v, mask, scale, do), q), rtol=1e-6, atol=1e-8)
+    assert np.allclose(dk, _fd(lambda x: _loss(q, x, v, mask, scale, do), k), rtol=1e-6, atol=1e-8)
+    assert np.allclose(dv, _fd(lambda x: _loss(q, k, x, mask, scale, do), v), rtol=1e-6, atol=1e-8)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_library_autograd(causal):
+    rng = np.random.default_rng(7)
+    n, d = 9, 6
+    q, k, v, do = (rng.standard_normal((n, d)) for _ in range(4))
+    scale = 0.4
+    mask = np.tril(np.ones((n, n), bool)) if causal else np.ones((n, n), bool)
+    tq, tk, tv = (torch.tensor(x, dtype=torch.float64, requires_grad=True) for x in (q, k, v))
+    add = torch.zeros(n, n, dtype=torch.float64).masked_fill(torch.from_numpy(~mask), float("-inf"))
+    out = torch.softmax(scale * tq @ tk.T + add, dim=-1) @ tv
+    out.backward(torch.from_numpy(do))
+    dq, dk, dv = OB.attention_backward_one_head(q, k, v, mask, scale, do)
+    for a, b in ((dq, tq.grad), (dk, tk.grad), (dv, tv.grad)):
+        assert np.allclose(a, b.numpy(), rtol=1e-12, atol=1e-12)
+
+
+def test_invariants():
+    q, k, v, do, mask = _case(3, n=12, lk=20, d=8)
+    dq, dk, dv = OB.attention_backward_one_head(q, k, v, mask, 0.5, do)
+    assert np.allclose(dk.sum(axis=0), 0.0, atol=1e-12)      # sum_j ds_ij = 0 for every row
+    assert np.all(dq[1] == 0.0)                               # row 1 sees no key
+    # dv_j = sum_i p_ij dout_i: the column sums of p are the weights of dout
+    out, lse = oracle.attention_one_head(q, k, v, mask, 0.5)
+    assert np.allclose(dv.sum(axis=0), (do * np.isfinite(lse)[:, None]).sum(axis=0), atol=1e-12)
+
+
+def test_gqa_sum_over_query_heads():
+    wl = W.random_small(seed=4, kind="CAUSAL", batch=2, hq=4, hkv=2, d=16, lmin=3, lmax=20)
+    rng = np.random.default_rng(4)
+    do = rng.standard_normal((int(wl.cu_seqlens_q[-1]), wl.hq, wl.d))
+    dq, dk, dv = oracle.masked_attention_backward(wl, wl.masks[0], do)
+    b, g = 1, 2
+    lq, lk = wl.lq(b), wl.lk(b)
+    q0, k0 = int(wl.cu_seqlens_q[b]), int(wl.cu_seqlens_k[b])
+    m = oracle.dense_mask(wl.masks[0], b, lq, lk)
+    kk, vv = (t.to(torch.float64).numpy() for t in wl.kv_of_seq(b))
+    acc_k = np.zeros((lk, wl.d))
+    for h in (2, 3):   # the query heads of key/value head 1
+        _, a, _ = OB.attention_backward_one_head(wl.q[q0:q0 + lq, h].double().numpy(), kk[:, 1], vv[:, 1], m,
+                                                 wl.scale, do[q0:q0 + lq, h])
+        acc_k += a
+    assert np.allclose(dk[k0:k0 + lk, 1], acc_k, atol=1e-12)
+
+
+def test_planted_mistakes_are_caught(monkeypatch):
+    good = OB.attention_backward_one_head
+
+    def no_d_term(q, k, v, mask, scale, dout):
+        out, lse = oracle.attention_one_head(q, k, v, mask, scale)
+        has = np.isfinite(lse)
+        p = np.where(mask & has[:, None], np.exp(np.where(mask, scale * q @ k.T, 0) - np.where(has, lse, 0)[:, None]), 0)
+        ds = p * (dout @ v.T)
+        return scale * ds @ k, scale * ds.T @ q, p.T @ dout
+
+    def no_scale(q, k, v, mask, scale, dout):
+        a, b, c = good(q, k, v, mask, scale, dout)
+        return a / scale, b / scale, c
+
+    def transposed(q, k, v, mask, scale, dout):
+        a, b, c = good(q, k, v, mask, scale, dout)
+        return a, b[::-1].copy(), c
+
+    caught = 0
+    for bad in (no_d_term, no_scale, transposed):
+        monkeypatch.setattr(OB, "attention_backward_one_head", bad)
+        try:
+            test_finite_differences(0)
+        except AssertionError:
+            caught += 1
+        monkeypatch.setattr(OB, "attention_backward_one_head", good)
+    assert caught == 3
