@@ -58,7 +58,7 @@ def flops_of(stats, wl):
 
 def kernel_source_hash():
     h = hashlib.sha256()
-    for f in ("attn_fwd.cu", "tmem_ldst.inc", "attn_internal.h"):
+    for f in ("attn_fwd.cu", "device_common.cuh", "mma_groups.inc", "tmem_ldst.inc", "attn_internal.h"):
         with open(os.path.join(ROOT, "masked_flash_attention_attn_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]

@@ -179,6 +179,31 @@ attn_status_t attn_plan(const attn_problem_t* problem, const attn_mask_desc_t* m
 attn_status_t attn_masked_fwd(const attn_plan_t* plan, const void* q, const void* k, const void* v,
                               void* out, float* lse, attn_stream_t stream);
 
+/* Plan the forward AND the backward pass (gradients of out with respect to q, k, v).
+ * Same arguments and errors as attn_plan(); the plan serves attn_masked_fwd() and
+ * attn_masked_bwd(). Backward support: contiguous K/V and head_dim 64 or 128, otherwise
+ * UNSUPPORTED. It adds a second device workspace: the dQ and dK/dV work lists over
+ * 128 x 128 tiles of one head, the partial-tile masks in query-major and key-major form,
+ * and an fp32 [total_q][hq] buffer for the row terms dout . out. */
+attn_status_t attn_plan_bwd(const attn_problem_t* problem, const attn_mask_desc_t* mask,
+                            attn_stream_t stream, attn_plan_t** out_plan);
+
+/* Backward of attn_masked_fwd for a loss with gradient dout on out (lse has no gradient
+ * of its own):
+ *     dv_j = sum_i p_ij dout_i,  ds_ij = p_ij (dout_i . v_j - dout_i . out_i),
+ *     dq_i = scale sum_j ds_ij k_j,  dk_j = scale sum_i ds_ij q_i,
+ * p_ij = exp(scale q_i . k_j - lse_i) on visible pairs; dk, dv of a key/value head sum over
+ * its query heads. Asynchronous on `stream`; all DEVICE pointers, 16-byte aligned:
+ *   q, out, dout  bf16 [total_q][hq][head_dim]; lse fp32 [total_q][hq] as attn_masked_fwd wrote it
+ *   k, v          bf16 [total_k][hkv][head_dim]
+ *   dq            bf16 [total_q][hq][head_dim]  (0 on rows that see no key)
+ *   dk, dv        bf16 [total_k][hkv][head_dim] (0 on keys that no query sees)
+ * The plan must come from attn_plan_bwd(). Allocates nothing. Errors: INVALID_ARG (plan
+ * without backward lists, null or misaligned pointer), CUDA. */
+attn_status_t attn_masked_bwd(const attn_plan_t* plan, const void* q, const void* k, const void* v,
+                              const void* out, const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                              attn_stream_t stream);
+
 /* Copy the 128 x 128 tile classes (0 empty, 1 full, 2 partial) in the order sequence,
  * query tile, key tile (row-major) into host_dst[0 .. n). *n_needed (may be NULL)
  * receives the total count; a short buffer gets a prefix. */

@@ -27,7 +27,8 @@ RANGE_FULL, RANGE_CAUSAL, RANGE_INV_CAUSAL, RANGE_BI_CAUSAL, RANGE_CHUNK_CAUSAL 
 # every symbol include/attn.h declares
 EXPORTS = ("attn_plan", "attn_masked_fwd", "attn_plan_get_tile_classes", "attn_plan_get_stats",
            "attn_plan_check_status", "attn_plan_set_debug", "attn_plan_destroy", "attn_classify_host",
-           "attn_status_string", "attn_masked_fwd_noalloc", "attn_test_exp2_poly", "attn_plan_dry_run")
+           "attn_status_string", "attn_masked_fwd_noalloc", "attn_test_exp2_poly", "attn_plan_dry_run",
+           "attn_plan_bwd", "attn_masked_bwd")
 
 
 class AttnError(RuntimeError):
@@ -90,6 +91,9 @@ def lib() -> ctypes.CDLL:
         L.attn_status_string.argtypes = [i32]
         L.attn_status_string.restype = ctypes.c_char_p
         L.attn_test_exp2_poly.argtypes = [vp, vp, i64, vp]
+        L.attn_plan_bwd.argtypes = [ctypes.POINTER(attn_problem_t), ctypes.POINTER(attn_mask_desc_t), vp,
+                                    ctypes.POINTER(vp)]
+        L.attn_masked_bwd.argtypes = [vp] * 11
         L.attn_plan_dry_run.argtypes = [ctypes.POINTER(attn_problem_t), ctypes.POINTER(attn_mask_desc_t), i32,
                                         ctypes.POINTER(attn_plan_stats_t)]
         L.attn_masked_fwd_noalloc.argtypes = [ctypes.POINTER(attn_problem_t), ctypes.POINTER(attn_mask_desc_t),
@@ -206,7 +210,7 @@ class Plan:
 
 def attn_plan(*, hq: int, hkv: int, head_dim: int, cu_seqlens_q, mask, cu_seqlens_k=None, kv_lens=None,
               page_table=None, page_size: int = 0, num_pages: int = 0, scale: float = 0.0, kv_splits: int = 0,
-              stream=None) -> Plan:
+              stream=None, backward: bool = False) -> Plan:
     """attn_plan(): validate, classify tiles, build the work list. ``page_table`` is a device
     int32 tensor [batch, max_pages]; CUSTOM ``mask.bits`` may be host (numpy) or device words;
     ``kv_splits``: 0 automatic, 1 never, N >= 2 at most N key ranges per query tile."""
@@ -224,7 +228,11 @@ def attn_plan(*, hq: int, hkv: int, head_dim: int, cu_seqlens_q, mask, cu_seqlen
             dev_bits = b
     d = _mask_desc(m, mask, dev_bits)
     h = ctypes.c_void_p()
-    _check(lib().attn_plan(ctypes.byref(pr), ctypes.byref(d), _stream(stream), ctypes.byref(h)), "attn_plan")
+    if backward:   # attn_plan_bwd(): forward and backward work lists
+        _check(lib().attn_plan_bwd(ctypes.byref(pr), ctypes.byref(d), _stream(stream), ctypes.byref(h)),
+               "attn_plan_bwd")
+    else:
+        _check(lib().attn_plan(ctypes.byref(pr), ctypes.byref(d), _stream(stream), ctypes.byref(h)), "attn_plan")
     total_q = int(np.asarray(cu_seqlens_q)[-1])
     return Plan(h.value, page_table, hq, head_dim, total_q)
 
@@ -233,6 +241,13 @@ def attn_masked_fwd(plan: Plan, q, k, v, out, lse=None, stream=None) -> None:
     """attn_masked_fwd(): enqueue the forward on ``stream`` (default: torch's current stream)."""
     _check(lib().attn_masked_fwd(plan.handle, _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _stream(stream)),
            "attn_masked_fwd")
+
+
+def attn_masked_bwd(plan: Plan, q, k, v, out, lse, dout, dq, dk, dv, stream=None) -> None:
+    """attn_masked_bwd(): enqueue dq, dk, dv for the gradient dout of out (plan from
+    attn_plan(..., backward=True))."""
+    _check(lib().attn_masked_bwd(plan.handle, _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dout), _ptr(dq),
+                                 _ptr(dk), _ptr(dv), _stream(stream)), "attn_masked_bwd")
 
 
 def attn_plan_get_tile_classes(plan: Plan) -> np.ndarray:
@@ -332,3 +347,13 @@ def forward(plan: Plan, q, k, v, stream=None):
     lse = torch.empty(q.shape[0], plan.hq, dtype=torch.float32, device=q.device)
     attn_masked_fwd(plan, q, k, v, out, lse, stream)
     return out, lse
+
+
+def backward(plan: Plan, q, k, v, out, lse, dout, stream=None):
+    """Allocate dq / dk / dv with torch and run attn_masked_bwd (convenience)."""
+    import torch
+    dq = torch.empty_like(q)
+    dk = torch.empty_like(k)
+    dv = torch.empty_like(v)
+    attn_masked_bwd(plan, q, k, v, out, lse, dout, dq, dk, dv, stream)
+    return dq, dk, dv

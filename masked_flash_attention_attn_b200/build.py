@@ -19,7 +19,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libattn_b200.so")
-SOURCES = ["attn_plan.cpp", "attn_custom.cu", "attn_fwd.cu"]
+SOURCES = ["attn_plan.cpp", "attn_custom.cu", "attn_fwd.cu", "attn_bwd.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

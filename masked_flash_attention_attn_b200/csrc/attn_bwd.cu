@@ -1,0 +1,624 @@
+// Masked attention backward for sm_100a (B200): dQ, dK and dV of the forward in attn_fwd.cu.
+//
+// With p_ij = exp(scale q_i . k_j - lse_i) on visible pairs (0 elsewhere), dp_ij = dout_i . v_j,
+// delta_i = dout_i . out_i and ds_ij = p_ij (dp_ij - delta_i):
+//     dq_i = scale sum_j ds_ij k_j,   dk_j = scale sum_i ds_ij q_i,   dv_j = sum_i p_ij dout_i,
+// dk and dv of a key/value head summed over the query heads that read it. Three kernels:
+//   bwd_delta_kernel    delta_i for every (row, query head): one warp per row.
+//   dQ kernel           one persistent CTA per SM over dQ items (a 128-row query tile of one
+//                       query head and its non-empty key tiles): S = Q K^T and dP = dO V^T
+//                       into TMEM, the elementwise warpgroup turns them into dS (bf16, written
+//                       over S), then dQ += dS K accumulates in TMEM.
+//   dK/dV kernel        one persistent CTA per SM over dK/dV items (a 128-key tile of one
+//                       key/value head and every (query head, query tile) that sees it):
+//                       S^T = K Q^T and dP^T = V dO^T into TMEM, the warpgroup writes P^T and
+//                       dS^T (bf16) over them, then dV += P^T dO and dK += dS^T Q accumulate in
+//                       TMEM.
+// Both recompute P from the forward's lse instead of storing it. Warp roles as in the
+// forward: warp 0 TMA producer, warp 1 MMA issuer (one thread), warps 4-7 the elementwise
+// warpgroup, one TMEM lane (= one tile row) per thread. Tiles are 128 rows of one head,
+// 64-column boxes with the 128-byte swizzle; a ring of STAGES tile slots streams the
+// per-job operands (dQ: K and V tiles; dK/dV: Q and dO tiles). TMEM: S at column 0, dP at
+// 128, the accumulators from 256 (dQ: D columns; dK/dV: dV then dK). Every mbarrier wait is
+// bounded as in the forward.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_bf16.h>
+
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "attn_internal.h"
+
+namespace mfa {
+namespace {
+
+#include "device_common.cuh"
+
+struct BwdParams {
+  CUtensorMap tm_a;   // per item:  dQ: Q    dK/dV: K
+  CUtensorMap tm_b;   // per item:  dQ: dO   dK/dV: V
+  CUtensorMap tm_c;   // per job:   dQ: K    dK/dV: Q
+  CUtensorMap tm_d;   // per job:   dQ: V    dK/dV: dO
+  const BwdItem* items;
+  const BwdJob* jobs;
+  const int32_t* cta_off;
+  const int32_t* cta_items;
+  const uint4* mask_tiles;
+  const float* lse;     // [total_q][hq], natural log
+  const float* delta;   // [total_q][hq]
+  __nv_bfloat16* g0;    // dQ: dq;  dK/dV: dk
+  __nv_bfloat16* g1;    // dK/dV: dv
+  int32_t* status;
+  int32_t hq, hkv;
+  float scale, scale_log2;
+  int64_t timeout_ns;
+};
+
+template <int D_>
+struct BwdCfg {
+  static constexpr int D = D_;
+  static constexpr int NBOX = D / 64;                  // 64-column boxes per tile
+  static constexpr int BOX_BYTES = 128 * 128;          // 128 rows x 128 bytes
+  static constexpr int TILE_BYTES = NBOX * BOX_BYTES;  // one 128-row tile of one head
+  static constexpr int STAGES = D == 128 ? 4 : 8;      // ring tile slots (two per job)
+  static constexpr int OFF_A = 0, OFF_B = TILE_BYTES, OFF_RING = 2 * TILE_BYTES;
+  static constexpr int OFF_ROWV = OFF_RING + STAGES * TILE_BYTES;  // dK/dV: per warp 128 lse2 + 128 delta
+  static constexpr int OFF_BAR = OFF_ROWV + 4 * 2 * 128 * 4;
+  static constexpr int B_AFULL = 0, B_AEMPTY = 1, B_RFULL = 2, B_REMPTY = B_RFULL + STAGES,
+                       B_SFULL = B_REMPTY + STAGES, B_PFULL = B_SFULL + 1, B_ACCFULL = B_PFULL + 1,
+                       B_ACCEMPTY = B_ACCFULL + 1, B_DRAIN = B_ACCEMPTY + 1, NBAR = B_DRAIN + 1;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;       // [0] TMEM base, [1] abort flag
+  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;   // + slack to align the base to 1 KiB
+  static constexpr int THREADS = 256;
+  static constexpr int TM_S = 0, TM_P = 128, TM_ACC = 256;
+  static constexpr uint32_t IDESC_SS =  // M=128, N=128, bf16 x bf16 -> fp32, both K-major
+      (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(128 >> 3) << 17) | (uint32_t(128 >> 4) << 24);
+  static constexpr uint32_t IDESC_TS =  // M=128, N=D, A from TMEM, B MN-major
+      (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) | (uint32_t(D >> 3) << 17) | (uint32_t(128 >> 4) << 24);
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+  static_assert(TM_ACC + 2 * D <= 512, "TMEM budget");
+};
+
+enum : int32_t {
+  kBwdWaitAEmpty = 0x200, kBwdWaitREmpty, kBwdWaitAFull, kBwdWaitRFull, kBwdWaitPFull, kBwdWaitAccEmpty,
+  kBwdWaitSFull, kBwdWaitAccFull
+};
+
+// C[128 x 128] (TMEM, fp32) = A[128 x D] . B[128 x D]^T, both tiles K-major in shared memory.
+template <int D>
+__device__ __forceinline__ void mma_tile_ss(uint32_t d, uint32_t a_smem, uint32_t b_smem, uint32_t idesc) {
+  if constexpr (D == 128) mma_ss_x8_k128(d, desc_of(desc_lo(a_smem, 16)), desc_of(desc_lo(b_smem, 16)), idesc, 0u);
+  else mma_ss_x4_k64(d, desc_of(desc_lo(a_smem, 16)), desc_of(desc_lo(b_smem, 16)), idesc, 0u);
+}
+
+// C[128 x D] (+)= A[128 x 128] (bf16 in TMEM) . B[128 x D] (tile in shared memory, MN-major).
+template <int D>
+__device__ __forceinline__ void mma_tile_ts(uint32_t d, uint32_t a_tmem, uint32_t b_smem, uint32_t idesc,
+                                            uint32_t acc) {
+  mma_ts_x8(d, a_tmem, desc_of(desc_lo(b_smem, 128 * 128)), idesc, acc);
+}
+
+__device__ __forceinline__ bool mask_bit(const uint4& bits, int c) {
+  const uint32_t w = c < 64 ? (c < 32 ? bits.x : bits.y) : (c < 96 ? bits.z : bits.w);
+  return (w >> (c & 31)) & 1u;
+}
+
+// One 128-row x D tile of bf16 gradients from TMEM (fp32, times `mul`) to global memory.
+template <int D>
+__device__ __forceinline__ void store_grad_row(uint32_t t_acc, float mul, bool valid, __nv_bfloat16* dst) {
+#pragma unroll 1
+  for (int cc = 0; cc < D / 32; ++cc) {
+    uint32_t o[32];
+    tmem_ld32x32(t_acc + cc * 32, o);
+    tmem_wait_ld();
+    uint32_t pk[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e)
+      pk[e] = pack_bf16(__uint_as_float(o[2 * e]) * mul, __uint_as_float(o[2 * e + 1]) * mul);
+    if (valid) {
+      uint4* q = reinterpret_cast<uint4*>(dst + cc * 32);
+      q[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      q[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+      q[2] = make_uint4(pk[8], pk[9], pk[10], pk[11]);
+      q[3] = make_uint4(pk[12], pk[13], pk[14], pk[15]);
+    }
+  }
+}
+
+// delta[r][h] = dout[r][h] . out[r][h] (fp32), one warp per (row, head).
+__global__ void bwd_delta_kernel(const __nv_bfloat16* __restrict__ out, const __nv_bfloat16* __restrict__ dout,
+                                 float* __restrict__ delta, int64_t rows, int D) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = int64_t(gridDim.x) * (blockDim.x >> 5);
+  for (int64_t r = int64_t(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); r < rows; r += warps) {
+    float acc = 0.f;
+    for (int c = 2 * lane; c < D; c += 64) {
+      const __nv_bfloat162 o = *reinterpret_cast<const __nv_bfloat162*>(out + r * D + c);
+      const __nv_bfloat162 g = *reinterpret_cast<const __nv_bfloat162*>(dout + r * D + c);
+      acc = fmaf(__low2float(o), __low2float(g), acc);
+      acc = fmaf(__high2float(o), __high2float(g), acc);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) delta[r] = acc;
+  }
+}
+
+// ================================ dQ ================================
+template <class C>
+__global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd_dq_kernel(const __grid_constant__ BwdParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t sbase = (raw + 1023u) & ~1023u;
+  uint32_t* misc = reinterpret_cast<uint32_t*>(smem_raw + (sbase - raw) + C::OFF_MISC);
+  const uint32_t bar0 = sbase + C::OFF_BAR;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const Guard guard{smem_u32(misc + 1), 0u, p.status, p.timeout_ns};
+#define BAR(i) (bar0 + 8u * uint32_t(i))
+  if (tid == 0) {
+    mbar_init(BAR(C::B_AFULL), 1);
+    mbar_init(BAR(C::B_AEMPTY), 1);
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(BAR(C::B_RFULL + s), 1);
+      mbar_init(BAR(C::B_REMPTY + s), 1);
+    }
+    mbar_init(BAR(C::B_SFULL), 1);
+    mbar_init(BAR(C::B_PFULL), 128);
+    mbar_init(BAR(C::B_ACCFULL), 1);
+    mbar_init(BAR(C::B_ACCEMPTY), 128);
+    mbar_init(BAR(C::B_DRAIN), 1);
+    misc[1] = 0u;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    prefetch_tmap(&p.tm_a);
+    prefetch_tmap(&p.tm_b);
+    prefetch_tmap(&p.tm_c);
+    prefetch_tmap(&p.tm_d);
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(smem_u32(misc))
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = misc[0];
+  const int i_begin = p.cta_off[blockIdx.x], i_end = p.cta_off[blockIdx.x + 1];
+
+  if (warp == 0) {
+    // ---- TMA producer: Q and dO once per item, then K and V tiles of every job ----
+    if (lane == 0) {
+      uint32_t rc = 0;
+      int n = 0, a_last = -1;
+      bool ok = true;
+      for (int ii = i_begin; ok && ii < i_end; ++ii, ++n) {
+        const BwdItem it = p.items[p.cta_items[ii]];
+        if (!wait_bounded(BAR(C::B_AEMPTY), (n & 1) ^ 1, guard, kBwdWaitAEmpty)) break;
+        mbar_expect_tx(BAR(C::B_AFULL), 2 * C::TILE_BYTES);
+        a_last = n;
+        for (int c = 0; c < C::NBOX; ++c) {
+          tma_load_3d(sbase + C::OFF_A + c * C::BOX_BYTES, &p.tm_a, c * 64, it.head, it.tok, BAR(C::B_AFULL));
+          tma_load_3d(sbase + C::OFF_B + c * C::BOX_BYTES, &p.tm_b, c * 64, it.head, it.tok, BAR(C::B_AFULL));
+        }
+        for (int j = 0; ok && j < it.job_count; ++j) {
+          const BwdJob jb = p.jobs[it.job_start + j];
+          for (int op = 0; op < 2; ++op, ++rc) {
+            const uint32_t slot = rc % C::STAGES;
+            if (!wait_bounded(BAR(C::B_REMPTY + slot), ((rc / C::STAGES) & 1) ^ 1, guard, kBwdWaitREmpty)) {
+              ok = false;
+              break;
+            }
+            mbar_expect_tx(BAR(C::B_RFULL + slot), C::TILE_BYTES);
+            const CUtensorMap* tm = op == 0 ? &p.tm_c : &p.tm_d;
+            for (int c = 0; c < C::NBOX; ++c)
+              tma_load_3d(sbase + C::OFF_RING + slot * C::TILE_BYTES + c * C::BOX_BYTES, tm, c * 64, it.kv_head,
+                          jb.tok, BAR(C::B_RFULL + slot));
+          }
+        }
+      }
+      for (uint32_t r = rc > uint32_t(C::STAGES) ? rc - C::STAGES : 0u; r < rc; ++r)
+        wait_drain(BAR(C::B_RFULL + r % C::STAGES), (r / C::STAGES) & 1, p.timeout_ns);
+      if (a_last >= 0) wait_drain(BAR(C::B_AFULL), a_last & 1, p.timeout_ns);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ---- MMA issuer ----
+    if (lane == 0) {
+      uint32_t rc = 0, gj = 0;
+      int n = 0;
+      bool ok = true;
+      for (int ii = i_begin; ok && ii < i_end; ++ii, ++n) {
+        const BwdItem it = p.items[p.cta_items[ii]];
+        if (!wait_bounded(BAR(C::B_AFULL), n & 1, guard, kBwdWaitAFull)) break;
+        tc_fence_after();
+        for (int j = 0; j < it.job_count; ++j, ++gj) {
+          const uint32_t rk = rc, rv = rc + 1;
+          rc += 2;
+          if (!wait_bounded(BAR(C::B_RFULL + rk % C::STAGES), (rk / C::STAGES) & 1, guard, kBwdWaitRFull) ||
+              !wait_bounded(BAR(C::B_RFULL + rv % C::STAGES), (rv / C::STAGES) & 1, guard, kBwdWaitRFull)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t k_tile = sbase + C::OFF_RING + (rk % C::STAGES) * C::TILE_BYTES;
+          const uint32_t v_tile = sbase + C::OFF_RING + (rv % C::STAGES) * C::TILE_BYTES;
+          mma_tile_ss<C::D>(tmem + C::TM_S, sbase + C::OFF_A, k_tile, C::IDESC_SS);   // S = Q K^T
+          mma_tile_ss<C::D>(tmem + C::TM_P, sbase + C::OFF_B, v_tile, C::IDESC_SS);   // dP = dO V^T
+          mma_commit(BAR(C::B_REMPTY + rv % C::STAGES));
+          mma_commit(BAR(C::B_SFULL));
+          if (!wait_bounded(BAR(C::B_PFULL), gj & 1, guard, kBwdWaitPFull)) {
+            ok = false;
+            break;
+          }
+          if (j == 0 && !wait_bounded(BAR(C::B_ACCEMPTY), (n & 1) ^ 1, guard, kBwdWaitAccEmpty)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          mma_tile_ts<C::D>(tmem + C::TM_ACC, tmem + C::TM_S, k_tile, C::IDESC_TS, j > 0 ? 1u : 0u);  // dQ += dS K
+          mma_commit(BAR(C::B_REMPTY + rk % C::STAGES));
+        }
+        if (!ok) break;
+        mma_commit(BAR(C::B_ACCFULL));
+        mma_commit(BAR(C::B_AEMPTY));
+      }
+      mma_commit(BAR(C::B_DRAIN));
+      wait_drain(BAR(C::B_DRAIN), 0, p.timeout_ns);
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ---- elementwise warpgroup: thread r owns row r of the query tile ----
+    const int r = tid - 128;
+    const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
+    const float sl2 = p.scale_log2;
+    uint32_t gj = 0;
+    int n = 0;
+    bool ok = true;
+    for (int ii = i_begin; ok && ii < i_end; ++ii, ++n) {
+      const BwdItem it = p.items[p.cta_items[ii]];
+      const bool valid = r < it.rows;
+      const int64_t grow = int64_t(it.tok + r) * p.hq + it.head;
+      float lse2 = INFINITY, dlt = 0.f;   // lse2 = +inf: the row contributes nothing
+      if (valid) {
+        const float l = p.lse[grow];
+        lse2 = l == -INFINITY ? INFINITY : l * 1.4426950408889634f;
+        dlt = p.delta[grow];
+      }
+      for (int j = 0; j < it.job_count; ++j, ++gj) {
+        const int mi = p.jobs[it.job_start + j].mask;
+        uint4 bits = make_uint4(0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu);
+        if (mi >= 0) bits = __ldg(p.mask_tiles + int64_t(mi) * 128 + r);
+        else if (mi == kMaskNone) bits = make_uint4(0u, 0u, 0u, 0u);
+        if (!__all_sync(0xffffffffu, wait_bounded(BAR(C::B_SFULL), gj & 1, guard, kBwdWaitSFull))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t sv[32], dv[32];
+          tmem_ld32x32(tmem + lane_base + C::TM_S + 32 * c, sv);
+          tmem_ld32x32(tmem + lane_base + C::TM_P + 32 * c, dv);
+          tmem_wait_ld();
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            float ds[2];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const int col = 32 * c + 2 * e + h;
+              const float pr = mask_bit(bits, col) ? ex2(fmaf(__uint_as_float(sv[2 * e + h]), sl2, -lse2)) : 0.f;
+              ds[h] = pr * (__uint_as_float(dv[2 * e + h]) - dlt);
+            }
+            pk[e] = pack_bf16(ds[0], ds[1]);
+          }
+          // dS of columns 32c .. 32c+31 over S columns 16c .. 16c+15 (already read)
+          tmem_st32x16(tmem + lane_base + C::TM_S + 16 * c, pk);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(BAR(C::B_PFULL));
+      }
+      if (!ok) break;
+      if (!__all_sync(0xffffffffu, wait_bounded(BAR(C::B_ACCFULL), n & 1, guard, kBwdWaitAccFull))) break;
+      tc_fence_after();
+      store_grad_row<C::D>(tmem + lane_base + C::TM_ACC, p.scale, valid, p.g0 + grow * C::D);
+      tc_fence_before();
+      mbar_arrive(BAR(C::B_ACCEMPTY));
+    }
+  }
+#undef BAR
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem) : "memory");
+}
+
+// ================================ dK / dV ================================
+template <class C>
+__global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd_dkv_kernel(const __grid_constant__ BwdParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t sbase = (raw + 1023u) & ~1023u;
+  uint8_t* sgen = smem_raw + (sbase - raw);
+  uint32_t* misc = reinterpret_cast<uint32_t*>(sgen + C::OFF_MISC);
+  const uint32_t bar0 = sbase + C::OFF_BAR;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const Guard guard{smem_u32(misc + 1), 0u, p.status, p.timeout_ns};
+#define BAR(i) (bar0 + 8u * uint32_t(i))
+  if (tid == 0) {
+    mbar_init(BAR(C::B_AFULL), 1);
+    mbar_init(BAR(C::B_AEMPTY), 1);
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(BAR(C::B_RFULL + s), 1);
+      mbar_init(BAR(C::B_REMPTY + s), 1);
+    }
+    mbar_init(BAR(C::B_SFULL), 1);
+    mbar_init(BAR(C::B_PFULL), 128);
+    mbar_init(BAR(C::B_ACCFULL), 1);
+    mbar_init(BAR(C::B_ACCEMPTY), 128);
+    mbar_init(BAR(C::B_DRAIN), 1);
+    misc[1] = 0u;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    prefetch_tmap(&p.tm_a);
+    prefetch_tmap(&p.tm_b);
+    prefetch_tmap(&p.tm_c);
+    prefetch_tmap(&p.tm_d);
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(smem_u32(misc))
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = misc[0];
+  const int i_begin = p.cta_off[blockIdx.x], i_end = p.cta_off[blockIdx.x + 1];
+
+  if (warp == 0) {
+    // ---- TMA producer: K and V once per item, then Q and dO tiles of every job ----
+    if (lane == 0) {
+      uint32_t rc = 0;
+      int n = 0, a_last = -1;
+      bool ok = true;
+      for (int ii = i_begin; ok && ii < i_end; ++ii, ++n) {
+        const BwdItem it = p.items[p.cta_items[ii]];
+        if (!wait_bounded(BAR(C::B_AEMPTY), (n & 1) ^ 1, guard, kBwdWaitAEmpty)) break;
+        mbar_expect_tx(BAR(C::B_AFULL), 2 * C::TILE_BYTES);
+        a_last = n;
+        for (int c = 0; c < C::NBOX; ++c) {
+          tma_load_3d(sbase + C::OFF_A + c * C::BOX_BYTES, &p.tm_a, c * 64, it.kv_head, it.tok, BAR(C::B_AFULL));
+          tma_load_3d(sbase + C::OFF_B + c * C::BOX_BYTES, &p.tm_b, c * 64, it.kv_head, it.tok, BAR(C::B_AFULL));
+        }
+        for (int j = 0; ok && j < it.job_count; ++j) {
+          const BwdJob jb = p.jobs[it.job_start + j];
+          for (int op = 0; op < 2; ++op, ++rc) {
+            const uint32_t slot = rc % C::STAGES;
+            if (!wait_bounded(BAR(C::B_REMPTY + slot), ((rc / C::STAGES) & 1) ^ 1, guard, kBwdWaitREmpty)) {
+              ok = false;
+              break;
+            }
+            mbar_expect_tx(BAR(C::B_RFULL + slot), C::TILE_BYTES);
+            const CUtensorMap* tm = op == 0 ? &p.tm_c : &p.tm_d;
+            for (int c = 0; c < C::NBOX; ++c)
+              tma_load_3d(sbase + C::OFF_RING + slot * C::TILE_BYTES + c * C::BOX_BYTES, tm, c * 64, jb.head, jb.tok,
+                          BAR(C::B_RFULL + slot));
+          }
+        }
+      }
+      for (uint32_t r = rc > uint32_t(C::STAGES) ? rc - C::STAGES : 0u; r < rc; ++r)
+        wait_drain(BAR(C::B_RFULL + r % C::STAGES), (r / C::STAGES) & 1, p.timeout_ns);
+      if (a_last >= 0) wait_drain(BAR(C::B_AFULL), a_last & 1, p.timeout_ns);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ---- MMA issuer ----
+    if (lane == 0) {
+      uint32_t rc = 0, gj = 0;
+      int n = 0;
+      bool ok = true;
+      for (int ii = i_begin; ok && ii < i_end; ++ii, ++n) {
+        const BwdItem it = p.items[p.cta_items[ii]];
+        if (!wait_bounded(BAR(C::B_AFULL), n & 1, guard, kBwdWaitAFull)) break;
+        tc_fence_after();
+        for (int j = 0; j < it.job_count; ++j, ++gj) {
+          const uint32_t rq = rc, rd = rc + 1;
+          rc += 2;
+          if (!wait_bounded(BAR(C::B_RFULL + rq % C::STAGES), (rq / C::STAGES) & 1, guard, kBwdWaitRFull) ||
+              !wait_bounded(BAR(C::B_RFULL + rd % C::STAGES), (rd / C::STAGES) & 1, guard, kBwdWaitRFull)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t q_tile = sbase + C::OFF_RING + (rq % C::STAGES) * C::TILE_BYTES;
+          const uint32_t do_tile = sbase + C::OFF_RING + (rd % C::STAGES) * C::TILE_BYTES;
+          mma_tile_ss<C::D>(tmem + C::TM_S, sbase + C::OFF_A, q_tile, C::IDESC_SS);    // S^T = K Q^T
+          mma_tile_ss<C::D>(tmem + C::TM_P, sbase + C::OFF_B, do_tile, C::IDESC_SS);   // dP^T = V dO^T
+          mma_commit(BAR(C::B_SFULL));
+          if (!wait_bounded(BAR(C::B_PFULL), gj & 1, guard, kBwdWaitPFull)) {
+            ok = false;
+            break;
+          }
+          if (j == 0 && !wait_bounded(BAR(C::B_ACCEMPTY), (n & 1) ^ 1, guard, kBwdWaitAccEmpty)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t acc = j > 0 ? 1u : 0u;
+          mma_tile_ts<C::D>(tmem + C::TM_ACC, tmem + C::TM_S, do_tile, C::IDESC_TS, acc);         // dV += P^T dO
+          mma_tile_ts<C::D>(tmem + C::TM_ACC + C::D, tmem + C::TM_P, q_tile, C::IDESC_TS, acc);   // dK += dS^T Q
+          mma_commit(BAR(C::B_REMPTY + rq % C::STAGES));
+          mma_commit(BAR(C::B_REMPTY + rd % C::STAGES));
+        }
+        if (!ok) break;
+        mma_commit(BAR(C::B_ACCFULL));
+        mma_commit(BAR(C::B_AEMPTY));
+      }
+      mma_commit(BAR(C::B_DRAIN));
+      wait_drain(BAR(C::B_DRAIN), 0, p.timeout_ns);
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ---- elementwise warpgroup: thread r owns key row r of the key tile ----
+    const int r = tid - 128;
+    const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
+    const float sl2 = p.scale_log2;
+    // this warp's copy of the job's per-query-row terms (no barrier across warps)
+    float* rl2 = reinterpret_cast<float*>(sgen + C::OFF_ROWV) + (warp - 4) * 256;
+    float* rdl = rl2 + 128;
+    uint32_t gj = 0;
+    int n = 0;
+    bool ok = true;
+    for (int ii = i_begin; ok && ii < i_end; ++ii, ++n) {
+      const BwdItem it = p.items[p.cta_items[ii]];
+      for (int j = 0; j < it.job_count; ++j, ++gj) {
+        const BwdJob jb = p.jobs[it.job_start + j];
+        __syncwarp();   // the previous job's reads of rl2 / rdl are done
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int qr = 4 * lane + k;
+          float l2 = INFINITY, dl = 0.f;
+          if (qr < jb.rows) {
+            const int64_t g = int64_t(jb.tok + qr) * p.hq + jb.head;
+            const float l = p.lse[g];
+            l2 = l == -INFINITY ? INFINITY : l * 1.4426950408889634f;
+            dl = p.delta[g];
+          }
+          rl2[qr] = l2;
+          rdl[qr] = dl;
+        }
+        __syncwarp();
+        uint4 bits = make_uint4(0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu);
+        if (jb.mask >= 0) bits = __ldg(p.mask_tiles + int64_t(jb.mask) * 128 + r);
+        else if (jb.mask == kMaskNone) bits = make_uint4(0u, 0u, 0u, 0u);
+        if (!__all_sync(0xffffffffu, wait_bounded(BAR(C::B_SFULL), gj & 1, guard, kBwdWaitSFull))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t sv[32], dv[32];
+          tmem_ld32x32(tmem + lane_base + C::TM_S + 32 * c, sv);
+          tmem_ld32x32(tmem + lane_base + C::TM_P + 32 * c, dv);
+          tmem_wait_ld();
+          uint32_t pp[16], pd[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            float pr[2], ds[2];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const int col = 32 * c + 2 * e + h;   // query row of the tile
+              pr[h] = mask_bit(bits, col) ? ex2(fmaf(__uint_as_float(sv[2 * e + h]), sl2, -rl2[col])) : 0.f;
+              ds[h] = pr[h] * (__uint_as_float(dv[2 * e + h]) - rdl[col]);
+            }
+            pp[e] = pack_bf16(pr[0], pr[1]);
+            pd[e] = pack_bf16(ds[0], ds[1]);
+          }
+          // P^T over S^T columns 16c.., dS^T over dP^T columns 16c.. (both already read)
+          tmem_st32x16(tmem + lane_base + C::TM_S + 16 * c, pp);
+          tmem_st32x16(tmem + lane_base + C::TM_P + 16 * c, pd);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(BAR(C::B_PFULL));
+      }
+      if (!ok) break;
+      if (!__all_sync(0xffffffffu, wait_bounded(BAR(C::B_ACCFULL), n & 1, guard, kBwdWaitAccFull))) break;
+      tc_fence_after();
+      const bool valid = r < it.rows;
+      const int64_t grow = int64_t(it.tok + r) * p.hkv + it.kv_head;
+      store_grad_row<C::D>(tmem + lane_base + C::TM_ACC, 1.f, valid, p.g1 + grow * C::D);           // dv
+      store_grad_row<C::D>(tmem + lane_base + C::TM_ACC + C::D, p.scale, valid, p.g0 + grow * C::D);  // dk
+      tc_fence_before();
+      mbar_arrive(BAR(C::B_ACCEMPTY));
+    }
+  }
+#undef BAR
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem) : "memory");
+}
+
+template <class C, bool DKV>
+attn_status_t launch_bwd(int ctas, const BwdParams& p, cudaStream_t stream) {
+  static std::once_flag once;
+  static cudaError_t attr = cudaSuccess;
+  std::call_once(once, [] {
+    attr = DKV ? cudaFuncSetAttribute(masked_attn_bwd_dkv_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      C::SMEM_BYTES)
+               : cudaFuncSetAttribute(masked_attn_bwd_dq_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      C::SMEM_BYTES);
+  });
+  if (attr != cudaSuccess) return ATTN_ERR_CUDA;
+  if (DKV) masked_attn_bwd_dkv_kernel<C><<<ctas, C::THREADS, C::SMEM_BYTES, stream>>>(p);
+  else masked_attn_bwd_dq_kernel<C><<<ctas, C::THREADS, C::SMEM_BYTES, stream>>>(p);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+}  // namespace
+}  // namespace mfa
+
+attn_status_t mfa_launch_backward(const attn_plan_t* plan, const void* q, const void* k, const void* v,
+                                  const void* out, const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                                  cudaStream_t stream) {
+  using namespace mfa;
+  const int D = plan->d;
+  const int64_t qrows = plan->total_q * plan->hq, krows = plan->total_kv_rows * plan->hkv;
+  if (plan->total_q == 0 || plan->total_kv_rows == 0) {
+    // nothing to attend: every gradient is zero
+    cudaError_t e = cudaMemsetAsync(dq, 0, size_t(qrows) * D * 2, stream);
+    if (e == cudaSuccess) e = cudaMemsetAsync(dk, 0, size_t(krows) * D * 2, stream);
+    if (e == cudaSuccess) e = cudaMemsetAsync(dv, 0, size_t(krows) * D * 2, stream);
+    return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+  }
+  bwd_delta_kernel<<<4 * 148, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(out),
+                                                static_cast<const __nv_bfloat16*>(dout), plan->d_bdelta, qrows, D);
+  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  BwdParams pq{}, pk{};
+  if (!encode3d(&pq.tm_a, q, D, plan->hq, plan->total_q, 128) ||
+      !encode3d(&pq.tm_b, dout, D, plan->hq, plan->total_q, 128) ||
+      !encode3d(&pq.tm_c, k, D, plan->hkv, plan->total_kv_rows, 128) ||
+      !encode3d(&pq.tm_d, v, D, plan->hkv, plan->total_kv_rows, 128))
+    return ATTN_ERR_CUDA;
+  pk.tm_a = pq.tm_c;   // K
+  pk.tm_b = pq.tm_d;   // V
+  pk.tm_c = pq.tm_a;   // Q
+  pk.tm_d = pq.tm_b;   // dO
+  for (BwdParams* p : {&pq, &pk}) {
+    p->lse = lse;
+    p->delta = plan->d_bdelta;
+    p->status = plan->d_status;
+    p->hq = plan->hq;
+    p->hkv = plan->hkv;
+    p->scale = plan->scale;
+    p->scale_log2 = plan->scale * 1.4426950408889634f;
+    p->timeout_ns = plan->timeout_ns;
+  }
+  pq.items = plan->d_bq_items;
+  pq.jobs = plan->d_bq_jobs;
+  pq.cta_off = plan->d_bq_cta_off;
+  pq.cta_items = plan->d_bq_cta_items;
+  pq.mask_tiles = plan->d_bmask_q;
+  pq.g0 = static_cast<__nv_bfloat16*>(dq);
+  pk.items = plan->d_bkv_items;
+  pk.jobs = plan->d_bkv_jobs;
+  pk.cta_off = plan->d_bkv_cta_off;
+  pk.cta_items = plan->d_bkv_cta_items;
+  pk.mask_tiles = plan->d_bmask_k;
+  pk.g0 = static_cast<__nv_bfloat16*>(dk);
+  pk.g1 = static_cast<__nv_bfloat16*>(dv);
+  attn_status_t st;
+  if (D == 64) {
+    st = launch_bwd<BwdCfg<64>, false>(plan->bq_ctas, pq, stream);
+    if (st == ATTN_OK) st = launch_bwd<BwdCfg<64>, true>(plan->bkv_ctas, pk, stream);
+  } else {
+    st = launch_bwd<BwdCfg<128>, false>(plan->bq_ctas, pq, stream);
+    if (st == ATTN_OK) st = launch_bwd<BwdCfg<128>, true>(plan->bkv_ctas, pk, stream);
+  }
+  return st;
+}

@@ -61,6 +61,28 @@ struct alignas(16) Job {
 };
 static_assert(sizeof(Job) == 16, "Job layout");
 
+// ---- backward work lists (attn_plan_bwd) -------------------------------------------------
+// dQ items: one 128-row query tile of one query head against its non-empty key tiles.
+// dK/dV items: one 128-key tile of one key/value head against every (query head of its
+// group, query tile) that sees it. Tiles here are always 128 rows of one head.
+struct alignas(16) BwdItem {
+  int32_t seq, kv_head;
+  int32_t head;        // dQ: the query head
+  int32_t tok;         // dQ: first query token of the tile; dK/dV: first key row of the tile
+  int32_t rows;        // valid rows of the tile (queries, or keys)
+  int32_t job_start, job_count;
+  int32_t pad;
+};
+static_assert(sizeof(BwdItem) == 32, "BwdItem layout");
+
+struct alignas(16) BwdJob {
+  int32_t tok;         // dQ: first key row of the key tile; dK/dV: first query token of the query tile
+  int32_t mask;        // kMaskFull, kMaskNone, or a mask tile (dQ: query-major; dK/dV: key-major)
+  int32_t head;        // dK/dV: the query head
+  int32_t rows;        // dK/dV: valid query rows of the query tile
+};
+static_assert(sizeof(BwdJob) == 16, "BwdJob layout");
+
 // ---- CUSTOM mask scan on the device ----------------------------------------------------
 struct CustomSeq {
   int64_t word_off;    // first word of the sequence's packed mask
@@ -109,6 +131,21 @@ struct attn_plan {
   float* d_part_lse = nullptr;
   const mfa::MergeTile* d_merge = nullptr;
   int32_t n_merge = 0;
+  // backward (attn_plan_bwd; one more workspace allocation)
+  bool has_bwd = false;
+  void* bws = nullptr;
+  int32_t bq_ctas = 0, bkv_ctas = 0;
+  const mfa::BwdItem* d_bq_items = nullptr;
+  const mfa::BwdJob* d_bq_jobs = nullptr;
+  const int32_t* d_bq_cta_off = nullptr;
+  const int32_t* d_bq_cta_items = nullptr;
+  const mfa::BwdItem* d_bkv_items = nullptr;
+  const mfa::BwdJob* d_bkv_jobs = nullptr;
+  const int32_t* d_bkv_cta_off = nullptr;
+  const int32_t* d_bkv_cta_items = nullptr;
+  const uint4* d_bmask_q = nullptr;   // query-major 2 KiB tiles (row = query, bits = keys)
+  const uint4* d_bmask_k = nullptr;   // the same tiles transposed (row = key, bits = queries)
+  float* d_bdelta = nullptr;          // [total_q][hq]: dout . out per row
   // debug hooks
   int32_t debug_flags = 0;
   int64_t timeout_ns = 2000000000LL;
@@ -128,3 +165,8 @@ attn_status_t mfa_plan_host(const attn_problem_t* problem, const attn_mask_desc_
 // forward launcher (attn_fwd.cu)
 attn_status_t mfa_launch_forward(const attn_plan_t* plan, const void* q, const void* k, const void* v,
                                  void* out, float* lse, cudaStream_t stream);
+
+// backward launcher (attn_bwd.cu)
+attn_status_t mfa_launch_backward(const attn_plan_t* plan, const void* q, const void* k, const void* v,
+                                  const void* out, const float* lse, const void* dout, void* dq, void* dk,
+                                  void* dv, cudaStream_t stream);

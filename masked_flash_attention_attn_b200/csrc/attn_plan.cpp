@@ -715,9 +715,9 @@ attn_status_t custom_counts(const attn_mask_desc_t* m, const Shape& s, int R, cu
   return ATTN_OK;
 }
 
-attn_status_t custom_repack(const attn_mask_desc_t* m, const Shape& s, int R, const WorkList& wl,
+attn_status_t custom_repack(const attn_mask_desc_t* m, const Shape& s, int R, const std::vector<TileRef>& mask_tiles,
                             uint4* d_tiles, cudaStream_t stream) {
-  if (wl.mask_tiles.empty()) return ATTN_OK;
+  if (mask_tiles.empty()) return ATTN_OK;
   std::vector<CustomSeq> seqs(s.B);
   for (int b = 0; b < s.B; ++b) {
     seqs[b].word_off = m->mask_word_offsets[b];
@@ -726,9 +726,9 @@ attn_status_t custom_repack(const attn_mask_desc_t* m, const Shape& s, int R, co
     seqs[b].n_rb = (s.lq[b] + R - 1) / R;
     seqs[b].n_kt = (s.lk[b] + kTile - 1) / kTile;
   }
-  std::vector<RepackTask> tasks(wl.mask_tiles.size());
+  std::vector<RepackTask> tasks(mask_tiles.size());
   for (size_t i = 0; i < tasks.size(); ++i) {
-    const TileRef& t = wl.mask_tiles[i];
+    const TileRef& t = mask_tiles[i];
     tasks[i] = RepackTask{t.seq, t.rb, t.kt, t.idx};
   }
   void* tmp = nullptr;
@@ -766,8 +766,200 @@ void work_stats(const attn_plan_t& m, const WorkList& wl, attn_plan_stats_t& st)
   st.merge_tiles = int32_t(wl.merge.size());
 }
 
+// ---- backward planning ----------------------------------------------------------------
+
+// Longest-first greedy assignment of items (costs) onto units: per-unit offsets and lists.
+void assign_lpt(const std::vector<int64_t>& cost, int units, std::vector<int32_t>& off, std::vector<int32_t>& list) {
+  const int n = int(cost.size());
+  const int C = std::max(1, std::min(units, n));
+  std::vector<int32_t> order(n);
+  std::iota(order.begin(), order.end(), 0);
+  std::stable_sort(order.begin(), order.end(), [&](int32_t x, int32_t y) { return cost[x] > cost[y]; });
+  using Load = std::pair<int64_t, int32_t>;
+  std::priority_queue<Load, std::vector<Load>, std::greater<Load>> heap;
+  for (int c = 0; c < C; ++c) heap.push(Load{0, c});
+  std::vector<std::vector<int32_t>> per(C);
+  for (int32_t it : order) {
+    Load l = heap.top();
+    heap.pop();
+    per[l.second].push_back(it);
+    l.first += cost[it];
+    heap.push(l);
+  }
+  off.assign(size_t(C) + 1, 0);
+  list.clear();
+  for (int c = 0; c < C; ++c) {
+    list.insert(list.end(), per[c].begin(), per[c].end());
+    off[c + 1] = int32_t(list.size());
+  }
+}
+
+// Backward lists over 128-row tiles of one head (cnts: per sequence, (query tile, key tile)
+// visible-pair counts with R = 128). A tile gets a mask tile when it is partial, or full but
+// cut by the end of the keys or of the queries (the dK/dV kernel must not let the rows past
+// L_q, which belong to the next sequence, into its sums).
+struct BwdLists {
+  std::vector<BwdItem> q_items, kv_items;
+  std::vector<BwdJob> q_jobs, kv_jobs;
+  std::vector<int32_t> q_off, q_list, kv_off, kv_list;
+  std::vector<TileRef> tiles;
+};
+
+void build_bwd(const Shape& s, const std::vector<std::vector<int32_t>>& cnts, int num_sms, BwdLists& bl) {
+  const int g = s.hq / s.hkv;
+  std::vector<int64_t> q_cost, kv_cost;
+  for (int b = 0; b < s.B; ++b) {
+    const int lq = s.lq[b], lk = s.lk[b];
+    const int n_qt = (lq + kTile - 1) / kTile, n_kt = (lk + kTile - 1) / kTile;
+    const std::vector<int32_t>& cnt = cnts[b];
+    std::vector<int32_t> tidx(size_t(n_qt) * n_kt, -1);
+    auto mask_of = [&](int qt, int kt) -> int32_t {
+      const int64_t rows = std::min(kTile, lq - qt * kTile), cols = std::min(kTile, lk - kt * kTile);
+      const int32_t k = classify(cnt[size_t(qt) * n_kt + kt], rows * cols);
+      if (k == kClassEmpty) return kMaskNone;
+      if (k == kClassFull && (kt + 1) * kTile <= lk && (qt + 1) * kTile <= lq) return kMaskFull;
+      int32_t& t = tidx[size_t(qt) * n_kt + kt];
+      if (t < 0) {
+        t = int32_t(bl.tiles.size());
+        bl.tiles.push_back(TileRef{b, qt, kt, t});
+      }
+      return t;
+    };
+    for (int kh = 0; kh < s.hkv; ++kh) {
+      // dQ items
+      for (int h = kh * g; h < (kh + 1) * g; ++h)
+        for (int qt = 0; qt < n_qt; ++qt) {
+          BwdItem it{b, kh, h, s.qoff[b] + qt * kTile, std::min(kTile, lq - qt * kTile), int32_t(bl.q_jobs.size()), 0, 0};
+          for (int kt = 0; kt < n_kt; ++kt) {
+            const int32_t m = mask_of(qt, kt);
+            if (m != kMaskNone) bl.q_jobs.push_back(BwdJob{s.koff[b] + kt * kTile, m, h, 0});
+          }
+          if (bl.q_jobs.size() == size_t(it.job_start))   // no key anywhere: one hidden job writes dq = 0
+            bl.q_jobs.push_back(BwdJob{s.koff[b], kMaskNone, h, 0});
+          it.job_count = int32_t(bl.q_jobs.size()) - it.job_start;
+          q_cost.push_back(it.job_count + 2);
+          bl.q_items.push_back(it);
+        }
+      // dK/dV items
+      for (int kt = 0; kt < n_kt; ++kt) {
+        BwdItem it{b, kh, kh * g, s.koff[b] + kt * kTile, std::min(kTile, lk - kt * kTile),
+                   int32_t(bl.kv_jobs.size()), 0, 0};
+        for (int h = kh * g; h < (kh + 1) * g; ++h)
+          for (int qt = 0; qt < n_qt; ++qt) {
+            const int32_t m = mask_of(qt, kt);
+            if (m != kMaskNone)
+              bl.kv_jobs.push_back(BwdJob{s.qoff[b] + qt * kTile, m, h, std::min(kTile, lq - qt * kTile)});
+          }
+        if (bl.kv_jobs.size() == size_t(it.job_start))   // no query sees the tile: dk = dv = 0
+          bl.kv_jobs.push_back(BwdJob{s.qoff[b], kMaskNone, kh * g, 0});
+        it.job_count = int32_t(bl.kv_jobs.size()) - it.job_start;
+        kv_cost.push_back(it.job_count + 2);
+        bl.kv_items.push_back(it);
+      }
+    }
+  }
+  assign_lpt(q_cost, num_sms, bl.q_off, bl.q_list);
+  assign_lpt(kv_cost, num_sms, bl.kv_off, bl.kv_list);
+}
+
+// Row-major 2 KiB tile (row r: 4 words, bit c = key c) -> the transposed tile (row c, bit r).
+void transpose_tile(const uint32_t* src, uint32_t* dst) {
+  std::memset(dst, 0, kMaskTileBytes);
+  for (int r = 0; r < kTile; ++r)
+    for (int c = 0; c < kTile; ++c)
+      if ((src[4 * r + (c >> 5)] >> (c & 31)) & 1u) dst[4 * c + (r >> 5)] |= 1u << (r & 31);
+}
+
+attn_status_t plan_backward(const attn_mask_desc_t* mask, const Shape& s, RowSource& src, int num_sms,
+                            cudaStream_t stream, attn_plan_t* plan) {
+  if (s.paged || (s.d != 64 && s.d != 128)) return ATTN_ERR_UNSUPPORTED;
+  std::vector<std::vector<int32_t>> cnts(s.B);
+  if (mask->kind == ATTN_MASK_CUSTOM) {
+    attn_status_t st = custom_counts(mask, s, kTile, stream, cnts);
+    if (st != ATTN_OK) return st;
+  } else {
+    for (int b = 0; b < s.B; ++b) {
+      src.prepare(b);
+      count_sequence(src, b, s, kTile, cnts[b]);
+    }
+  }
+  BwdLists bl;
+  build_bwd(s, cnts, num_sms, bl);
+  const size_t nt = bl.tiles.size();
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align256(off + bytes);
+    return o;
+  };
+  const size_t o_qi = take(bl.q_items.size() * sizeof(BwdItem)), o_qj = take(bl.q_jobs.size() * sizeof(BwdJob)),
+               o_qo = take(bl.q_off.size() * 4), o_ql = take(bl.q_list.size() * 4),
+               o_ki = take(bl.kv_items.size() * sizeof(BwdItem)), o_kj = take(bl.kv_jobs.size() * sizeof(BwdJob)),
+               o_ko = take(bl.kv_off.size() * 4), o_kl = take(bl.kv_list.size() * 4),
+               o_mq = take(nt * kMaskTileBytes), o_mk = take(nt * kMaskTileBytes),
+               o_dl = take(size_t(std::max<int64_t>(1, s.total_q)) * s.hq * sizeof(float));
+  std::vector<char> host(o_mq, 0);
+  std::memcpy(host.data() + o_qi, bl.q_items.data(), bl.q_items.size() * sizeof(BwdItem));
+  std::memcpy(host.data() + o_qj, bl.q_jobs.data(), bl.q_jobs.size() * sizeof(BwdJob));
+  std::memcpy(host.data() + o_qo, bl.q_off.data(), bl.q_off.size() * 4);
+  std::memcpy(host.data() + o_ql, bl.q_list.data(), bl.q_list.size() * 4);
+  std::memcpy(host.data() + o_ki, bl.kv_items.data(), bl.kv_items.size() * sizeof(BwdItem));
+  std::memcpy(host.data() + o_kj, bl.kv_jobs.data(), bl.kv_jobs.size() * sizeof(BwdJob));
+  std::memcpy(host.data() + o_ko, bl.kv_off.data(), bl.kv_off.size() * 4);
+  std::memcpy(host.data() + o_kl, bl.kv_list.data(), bl.kv_list.size() * 4);
+  void* ws = nullptr;
+  cudaError_t e = cudaMalloc(&ws, off);
+  if (e != cudaSuccess) return cuda_status(e);
+  char* base = static_cast<char*>(ws);
+  std::vector<uint32_t> qmaj(nt * (kMaskTileBytes / 4)), kmaj(nt * (kMaskTileBytes / 4));
+  e = cudaMemcpyAsync(base, host.data(), host.size(), cudaMemcpyHostToDevice, stream);
+  attn_status_t st = cuda_status(e);
+  if (st == ATTN_OK && nt) {
+    if (mask->kind == ATTN_MASK_CUSTOM) {
+      st = custom_repack(mask, s, kTile, bl.tiles, reinterpret_cast<uint4*>(base + o_mq), stream);
+      if (st == ATTN_OK)
+        st = cuda_status(cudaMemcpy(qmaj.data(), base + o_mq, nt * kMaskTileBytes, cudaMemcpyDeviceToHost));
+    } else {
+      int cur = -1;
+      for (const TileRef& t : bl.tiles) {
+        if (t.seq != cur) {
+          src.prepare(t.seq);
+          cur = t.seq;
+        }
+        write_mask_tile(src, s, kTile, t, qmaj.data() + size_t(t.idx) * (kMaskTileBytes / 4));
+      }
+      st = cuda_status(cudaMemcpyAsync(base + o_mq, qmaj.data(), nt * kMaskTileBytes, cudaMemcpyHostToDevice, stream));
+    }
+    for (size_t i = 0; st == ATTN_OK && i < nt; ++i)
+      transpose_tile(qmaj.data() + i * (kMaskTileBytes / 4), kmaj.data() + i * (kMaskTileBytes / 4));
+    if (st == ATTN_OK)
+      st = cuda_status(cudaMemcpyAsync(base + o_mk, kmaj.data(), nt * kMaskTileBytes, cudaMemcpyHostToDevice, stream));
+  }
+  if (st == ATTN_OK) st = cuda_status(cudaStreamSynchronize(stream));
+  if (st != ATTN_OK) {
+    cudaFree(ws);
+    return st;
+  }
+  plan->has_bwd = true;
+  plan->bws = ws;
+  plan->bq_ctas = int32_t(bl.q_off.size()) - 1;
+  plan->bkv_ctas = int32_t(bl.kv_off.size()) - 1;
+  plan->d_bq_items = reinterpret_cast<const BwdItem*>(base + o_qi);
+  plan->d_bq_jobs = reinterpret_cast<const BwdJob*>(base + o_qj);
+  plan->d_bq_cta_off = reinterpret_cast<const int32_t*>(base + o_qo);
+  plan->d_bq_cta_items = reinterpret_cast<const int32_t*>(base + o_ql);
+  plan->d_bkv_items = reinterpret_cast<const BwdItem*>(base + o_ki);
+  plan->d_bkv_jobs = reinterpret_cast<const BwdJob*>(base + o_kj);
+  plan->d_bkv_cta_off = reinterpret_cast<const int32_t*>(base + o_ko);
+  plan->d_bkv_cta_items = reinterpret_cast<const int32_t*>(base + o_kl);
+  plan->d_bmask_q = reinterpret_cast<const uint4*>(base + o_mq);
+  plan->d_bmask_k = reinterpret_cast<const uint4*>(base + o_mk);
+  plan->d_bdelta = reinterpret_cast<float*>(base + o_dl);
+  return ATTN_OK;
+}
+
 attn_status_t plan_impl(const attn_problem_t* problem, const attn_mask_desc_t* mask, cudaStream_t stream,
-                        attn_plan_t** out_plan) {
+                        attn_plan_t** out_plan, bool with_bwd = false) {
   if (!out_plan) return ATTN_ERR_INVALID_ARG;
   *out_plan = nullptr;
   Shape s;
@@ -775,6 +967,7 @@ attn_status_t plan_impl(const attn_problem_t* problem, const attn_mask_desc_t* m
   if (st != ATTN_OK) return st;
   st = validate_mask(mask, s);
   if (st != ATTN_OK) return st;
+  if (with_bwd && (s.paged || (s.d != 64 && s.d != 128))) return ATTN_ERR_UNSUPPORTED;
 
   int dev = 0, num_sms = 148;
   cudaError_t e = cudaGetDevice(&dev);
@@ -866,7 +1059,8 @@ attn_status_t plan_impl(const attn_problem_t* problem, const attn_mask_desc_t* m
   if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
   st = cuda_status(e);
   if (st == ATTN_OK && mask->kind == ATTN_MASK_CUSTOM)
-    st = custom_repack(mask, s, R, wl, reinterpret_cast<uint4*>(base + lay.off_tiles), stream);
+    st = custom_repack(mask, s, R, wl.mask_tiles, reinterpret_cast<uint4*>(base + lay.off_tiles), stream);
+  if (st == ATTN_OK && with_bwd) st = plan_backward(mask, s, src, num_sms, stream, plan);
   if (st != ATTN_OK) {
     cudaFree(plan->ws);
     delete plan;
@@ -989,6 +1183,25 @@ attn_status_t attn_plan(const attn_problem_t* problem, const attn_mask_desc_t* m
   }
 }
 
+attn_status_t attn_plan_bwd(const attn_problem_t* problem, const attn_mask_desc_t* mask, attn_stream_t stream,
+                            attn_plan_t** out_plan) {
+  try {
+    return plan_impl(problem, mask, reinterpret_cast<cudaStream_t>(stream), out_plan, /*with_bwd=*/true);
+  } catch (const std::bad_alloc&) {
+    return ATTN_ERR_OOM;
+  }
+}
+
+attn_status_t attn_masked_bwd(const attn_plan_t* plan, const void* q, const void* k, const void* v, const void* out,
+                              const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                              attn_stream_t stream) {
+  if (!plan || !plan->has_bwd) return ATTN_ERR_INVALID_ARG;
+  const void* ptrs[] = {q, k, v, out, lse, dout, dq, dk, dv};
+  for (const void* p : ptrs)
+    if (!p || (reinterpret_cast<uintptr_t>(p) & 15u)) return ATTN_ERR_INVALID_ARG;
+  return mfa_launch_backward(plan, q, k, v, out, lse, dout, dq, dk, dv, reinterpret_cast<cudaStream_t>(stream));
+}
+
 attn_status_t attn_masked_fwd(const attn_plan_t* plan, const void* q, const void* k, const void* v, void* out,
                               float* lse, attn_stream_t stream) {
   if (!plan) return ATTN_ERR_INVALID_ARG;
@@ -1037,6 +1250,10 @@ attn_status_t attn_plan_destroy(attn_plan_t* plan) {
   if (!plan) return ATTN_OK;
   cudaError_t e = cudaSuccess;
   if (plan->ws) e = cudaFree(plan->ws);
+  if (plan->bws) {
+    const cudaError_t e2 = cudaFree(plan->bws);
+    if (e == cudaSuccess) e = e2;
+  }
   delete plan;
   return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }

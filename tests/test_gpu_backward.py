@@ -1,0 +1,103 @@
+"""GPU parity of the backward pass (dQ, dK, dV) through the C ABI against the fp64 oracle
+gradients (oracle/backward.py), on ragged contiguous batches of every mask kind, head dims
+64 and 128, grouped-query heads, rows that see no key and keys no query sees.
+
+Tolerance: P and dS enter the tensor cores as bf16 (relative rounding 2^-9 each) with fp32
+accumulation, and the gradients are stored as bf16; with the forward's bf16 out in
+delta = dout . out the expected error is a few 1e-3 of the gradient scale. The bound
+used: max |err| <= 2e-2 * max |ref| and mean |err| <= 1e-2 * mean |ref|, per tensor."""
+import numpy as np
+import pytest
+import torch
+
+import workloads as W
+import oracle
+from tests import gpu_helpers as G
+
+pytestmark = pytest.mark.gpu
+
+KINDS = ["FULL", "CAUSAL", "SLIDING_WINDOW", "PREFIX_LM", "CHUNK_CAUSAL", "RANGES", "CUSTOM", "BLOCK_SPARSE"]
+REL_MAX, REL_MEAN = 2e-2, 1e-2
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib(attn_lib):
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    return attn_lib
+
+
+def _close(got, ref, what):
+    got = got.float().cpu().numpy().astype(np.float64)
+    assert np.isfinite(got).all(), f"{what}: non-finite"
+    err = np.abs(got - ref)
+    scale_max, scale_mean = max(np.abs(ref).max(), 1e-6), max(np.abs(ref).mean(), 1e-6)
+    assert err.max() <= REL_MAX * scale_max, f"{what}: max err {err.max():.3e} vs scale {scale_max:.3e}"
+    assert err.mean() <= REL_MEAN * scale_mean, f"{what}: mean err {err.mean():.3e} vs scale {scale_mean:.3e}"
+
+
+def check_backward(wl, spec, what, seed=0):
+    q, k, v = G.device_inputs(wl)
+    plan = G.M.attn_plan(hq=wl.hq, hkv=wl.hkv, head_dim=wl.d, cu_seqlens_q=wl.cu_seqlens_q,
+                         cu_seqlens_k=wl.cu_seqlens_k, mask=spec, scale=wl.scale, backward=True)
+    out, lse = G.M.forward(plan, q, k, v)
+    gen = torch.Generator().manual_seed(1000 + seed)
+    dout_h = W.randn_bf16(gen, q.shape[0], wl.hq, wl.d)
+    dq, dk, dv = G.M.backward(plan, q, k, v, out, lse, dout_h.cuda())
+    assert G.M.attn_plan_check_status(plan) == 0
+    rq, rk, rv = oracle.masked_attention_backward(wl, spec, dout_h)
+    _close(dq, rq, f"{what} dq")
+    _close(dk, rk, f"{what} dk")
+    _close(dv, rv, f"{what} dv")
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("kind", KINDS)
+def test_backward_all_kinds(kind, d):
+    wl = W.random_small(seed=500 + d + 3 * KINDS.index(kind), kind=kind, batch=3, hq=4, hkv=2, d=d,
+                        lmin=1, lmax=330)
+    check_backward(wl, wl.masks[0], f"bwd {kind} d={d}")
+
+
+@pytest.mark.parametrize("g", [1, 4])
+def test_backward_gqa_long(g):
+    wl = W.random_small(seed=70 + g, kind="CAUSAL", batch=2, hq=2 * g, hkv=2, d=128, lmin=200, lmax=700)
+    check_backward(wl, wl.masks[0], f"bwd gqa g={g}")
+
+
+def test_backward_rows_without_keys_and_unseen_keys():
+    # rows 0..9 see nothing (dq = 0); keys 600.. are seen by no query (dk = dv = 0)
+    rng = np.random.default_rng(12)
+    lq, lk = [190, 260], [700, 300]
+    dense = []
+    for a, b in zip(lq, lk):
+        m = rng.random((a, b)) < 0.4
+        m[:10] = False
+        m[:, 600:] = False
+        dense.append(m)
+    words, offs = [], [0]
+    for m in dense:
+        w = W.pack_rows(m)
+        words.append(w.reshape(-1))
+        offs.append(offs[-1] + w.size)
+    spec = W.MaskSpec("CUSTOM", bits=np.concatenate(words).astype(np.uint32), word_offsets=np.asarray(offs, np.int64))
+    gen = torch.Generator().manual_seed(5)
+    cq, ck = W.cu_from_lengths(lq), W.cu_from_lengths(lk)
+    wl = W.Workload(name="bwd_masked", hq=4, hkv=2, d=128, scale=0.09, cu_seqlens_q=cq,
+                    q=W.randn_bf16(gen, int(cq[-1]), 4, 128), masks=[spec], cu_seqlens_k=ck,
+                    k=W.randn_bf16(gen, int(ck[-1]), 2, 128), v=W.randn_bf16(gen, int(ck[-1]), 2, 128), seed=5)
+    check_backward(wl, spec, "bwd masked rows")
+
+
+def test_backward_plan_required_and_unsupported():
+    wl = W.random_small(seed=3, kind="CAUSAL", batch=2, hq=2, hkv=1, d=128, lmin=10, lmax=50)
+    q, k, v = G.device_inputs(wl)
+    plan = G.make_plan(wl, wl.masks[0])          # forward-only plan
+    out, lse = G.M.forward(plan, q, k, v)
+    with pytest.raises(G.M.AttnError) as e:
+        G.M.backward(plan, q, k, v, out, lse, torch.zeros_like(out))
+    assert e.value.status == 1
+    wl = W.random_small(seed=3, kind="CAUSAL", batch=2, hq=2, hkv=1, d=256, lmin=10, lmax=50)
+    with pytest.raises(G.M.AttnError) as e:
+        G.M.attn_plan(hq=2, hkv=1, head_dim=256, cu_seqlens_q=wl.cu_seqlens_q, cu_seqlens_k=wl.cu_seqlens_k,
+                      mask=wl.masks[0], backward=True)
+    assert e.value.status == 2
