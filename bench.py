@@ -33,6 +33,9 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "effective masked-attn TFLOP/s (unmasked pairs) and % of B200 bf16 tensor peak"
+# --pass bwd: the backward pass, counted as the usual 10 d FLOPs per unmasked pair and head
+# (S, dP, dV, dK, dQ: five 2 d products; the kernels recompute S and dP once more for dQ)
+METRIC_BWD = "effective masked-attn backward TFLOP/s (10 d FLOPs per unmasked pair) and % of B200 bf16 tensor peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_BYTES = 126 * 1024 * 1024
 
@@ -204,7 +207,7 @@ def config_of(wl, args, world):
             "lengths_q": [wl.lq(b) for b in range(wl.batch)][:64],
             "hq": wl.hq, "hkv": wl.hkv, "head_dim": wl.d,
             "masks": [m.kind + (f"({m.window})" if m.kind == "SLIDING_WINDOW" else "") for m in wl.masks],
-            "seed": wl.seed, "kv_splits": getattr(args, "kv_splits", 0),
+            "seed": wl.seed, "kv_splits": getattr(args, "kv_splits", 0), "pass": getattr(args, "pass_", "fwd"),
             "parallelism": f"dp{world} (independent batches, no collective)",
             "l2": f"inputs {in_bytes / 2**20:.0f} MiB vs 126 MiB L2; no flush" if in_bytes > L2_BYTES
             else "inputs fit L2; L2 flushed between steps"}
@@ -230,10 +233,10 @@ def device_inputs(wl, dev):
     return q, wl.k.to(dev), wl.v.to(dev)
 
 
-def make_plan(M, wl, spec, dev, kv_splits=0):
+def make_plan(M, wl, spec, dev, kv_splits=0, backward=False):
     import torch
     kw = dict(hq=wl.hq, hkv=wl.hkv, head_dim=wl.d, cu_seqlens_q=wl.cu_seqlens_q, mask=spec, scale=wl.scale,
-              kv_splits=kv_splits)
+              kv_splits=kv_splits, backward=backward)
     if wl.paged:
         kw.update(kv_lens=wl.kv_lens, page_table=torch.from_numpy(wl.page_table).to(dev),
                   page_size=wl.page_size, num_pages=wl.k_cache.shape[0])
@@ -254,14 +257,31 @@ def run_ours(args, rank, world, local_rank):
     wl = workload(args.config, rank)
     stream = torch.cuda.current_stream()
     q, k, v = device_inputs(wl, dev)
-    plans = [make_plan(M, wl, spec, dev, args.kv_splits) for spec in wl.masks]
+    bwd = args.pass_ == "bwd"
+    if bwd and (wl.paged or wl.d > 128):
+        raise SystemExit("--pass bwd: contiguous K/V and head_dim <= 128 only (workloads 1, 4, 5)")
+    plans = [make_plan(M, wl, spec, dev, args.kv_splits, backward=bwd) for spec in wl.masks]
     stats = [M.attn_plan_get_stats(p) for p in plans]
-    flops = [flops_of(s, wl) for s in stats]
+    flops = [flops_of(s, wl) * (2.5 if bwd else 1.0) for s in stats]
     tq = q.shape[0]
     outs = [torch.empty(tq, wl.hq, wl.d, dtype=torch.bfloat16, device=dev) for _ in plans]
     lses = [torch.empty(tq, wl.hq, dtype=torch.float32, device=dev) for _ in plans]
     in_bytes = q.numel() * 2 + k.numel() * 2 + v.numel() * 2
+    if bwd:
+        # the forward's out / lse are inputs of the backward; dout is seeded N(0,1)
+        for i, p in enumerate(plans):
+            M.attn_masked_fwd(p, q, k, v, outs[i], lses[i], stream)
+        gen = torch.Generator(device=dev).manual_seed(wl.seed + 101)
+        dout = torch.randn(tq, wl.hq, wl.d, generator=gen, device=dev).to(torch.bfloat16)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        in_bytes += sum(o.numel() * 2 + l.numel() * 4 for o, l in zip(outs, lses)) + dout.numel() * 2
     flush = torch.empty(256 * 2**20, dtype=torch.uint8, device=dev) if in_bytes <= L2_BYTES else None
+
+    def run_one(i, p):
+        if bwd:
+            M.attn_masked_bwd(p, q, k, v, outs[i], lses[i], dout, dq, dk, dv, stream)
+        else:
+            M.attn_masked_fwd(p, q, k, v, outs[i], lses[i], stream)
 
     def step(events=None):
         for i, p in enumerate(plans):
@@ -269,7 +289,7 @@ def run_ours(args, rank, world, local_rank):
                 flush.fill_(i)
             if events is not None:
                 events[i][0].record(stream)
-            M.attn_masked_fwd(p, q, k, v, outs[i], lses[i], stream)
+            run_one(i, p)
             if events is not None:
                 events[i][1].record(stream)
 
@@ -306,14 +326,32 @@ def run_ours(args, rank, world, local_rank):
     hl = [torch.empty(l.shape, dtype=l.dtype).pin_memory() for l in lses]
     e2e_steps = max(3, min(args.steps, 20))
 
+    if bwd:
+        hdo = dout.cpu().pin_memory()
+        hg = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (dq, dk, dv)]
+
     def e2e_step():
         q.copy_(hq_, non_blocking=True)
         k.copy_(hk_, non_blocking=True)
         v.copy_(hv_, non_blocking=True)
+        if bwd:
+            dout.copy_(hdo, non_blocking=True)
         for i, p in enumerate(plans):
-            M.attn_masked_fwd(p, q, k, v, outs[i], lses[i], stream)
-            ho[i].copy_(outs[i], non_blocking=True)
-            hl[i].copy_(lses[i], non_blocking=True)
+            if bwd:
+                outs[i].copy_(ho[i], non_blocking=True)
+                lses[i].copy_(hl[i], non_blocking=True)
+                M.attn_masked_bwd(p, q, k, v, outs[i], lses[i], dout, dq, dk, dv, stream)
+                for h, t in zip(hg, (dq, dk, dv)):
+                    h.copy_(t, non_blocking=True)
+            else:
+                M.attn_masked_fwd(p, q, k, v, outs[i], lses[i], stream)
+                ho[i].copy_(outs[i], non_blocking=True)
+                hl[i].copy_(lses[i], non_blocking=True)
+
+    if bwd:   # the host copies of out / lse hold the forward's results
+        for i in range(len(plans)):
+            ho[i].copy_(outs[i])
+            hl[i].copy_(lses[i])
 
     e2e_step()
     torch.cuda.synchronize()
@@ -328,6 +366,8 @@ def run_ours(args, rank, world, local_rank):
     e2e_ms = e0.elapsed_time(e1)
     h2d = in_bytes
     d2h = sum(o.numel() * 2 + l.numel() * 4 for o, l in zip(outs, lses))
+    if bwd:
+        d2h = len(plans) * sum(t.numel() * 2 for t in (dq, dk, dv))
 
     # ---- reduce over ranks (reporting only) ----
     (ms, e2e_ms), total_flops = reduce_over_ranks([ms, e2e_ms], sum(flops), dev)
@@ -347,10 +387,10 @@ def run_ours(args, rank, world, local_rank):
     pk_src += " bf16_tflops_sustained" if use_sustained else " bf16_tflops (burst)"
     avg_launch_ms = sum(sum(x) for x in launch_ms) / sum(len(x) for x in launch_ms)
     achieved = (sum(flops) / len(flops)) / (avg_launch_ms * 1e-3) / 1e12
-    tr = traffic_for(wl.name)
+    tr = None if bwd else traffic_for(wl.name)
     mask_bytes = sum(s["mask_tile_reads"] for s in stats) * 2048.0
     line = {
-        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "metric": METRIC_BWD if bwd else METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) bf16, lengths from seed)",
         "config": config_of(wl, args, world),
@@ -358,7 +398,8 @@ def run_ours(args, rank, world, local_rank):
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": tr,
                      "peak_source": pk_src,
-                     "kernel": f"masked_attn_fwd_kernel d={wl.d}",
+                     "kernel": (f"masked_attn_bwd_dq_kernel + masked_attn_bwd_dkv_kernel d={wl.d}" if bwd
+                                else f"masked_attn_fwd_kernel d={wl.d}"),
                      "algorithmic_flops_per_launch": sum(flops) / len(flops),
                      "avg_launch_ms": avg_launch_ms},
         "per_mask": [{"mask": m.kind, "unmasked_pairs_per_head": s["unmasked_pairs"], "tflops_per_s":
@@ -370,10 +411,11 @@ def run_ours(args, rank, world, local_rank):
         "e2e": {"value": e2e_val, "unit": "TFLOP/s", "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                 "steps": e2e_steps},
         # the forward kernel per plan and step, plus the split-KV merge kernel where a plan split
-        "gpu_launches": sum(1 + (s["merge_tiles"] > 0) for s in stats) * args.steps,
+        # backward: delta, dQ and dK/dV kernels per plan and step
+        "gpu_launches": (3 * len(plans) if bwd else sum(1 + (s["merge_tiles"] > 0) for s in stats)) * args.steps,
         "clocks": clocks,
     }
-    if world == 1 and not args.no_cpu_baseline:
+    if world == 1 and not args.no_cpu_baseline and not bwd:
         pairs, secs, desc = oracle_sample(wl, wl.masks, args.cpu_seconds)
         line["cpu_baseline"] = {"value": 4.0 * wl.d * pairs / secs / 1e12, "unit": "TFLOP/s",
                                 "cores": blas_threads(), "kind": "oracle", "sample": desc,
@@ -389,6 +431,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", type=int, default=2, choices=[1, 2, 3, 4, 5, 6],
                     help="1-5: the benchmark workloads; 6: long-context tree verify (split-KV case)")
+    ap.add_argument("--pass", dest="pass_", choices=["fwd", "bwd"], default="fwd",
+                    help="fwd: the forward (the benchmark metric); bwd: the backward pass (workloads 1, 4, 5)")
     ap.add_argument("--kv-splits", type=int, default=0,
                     help="split-KV: 0 automatic, 1 never, N >= 2 at most N key ranges per query tile")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
