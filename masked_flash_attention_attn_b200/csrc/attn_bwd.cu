@@ -18,9 +18,11 @@
 // forward: warp 0 TMA producer, warp 1 MMA issuer (one thread), warps 4-7 the elementwise
 // warpgroup, one TMEM lane (= one tile row) per thread. Tiles are 128 rows of one head,
 // 64-column boxes with the 128-byte swizzle; a ring of STAGES tile slots streams the
-// per-job operands (dQ: K and V tiles; dK/dV: Q and dO tiles). TMEM: S at column 0, dP at
-// 128, the accumulators from 256 (dQ: D columns; dK/dV: dV then dK). Every mbarrier wait is
-// bounded as in the forward.
+// per-job operands (dQ: K and V tiles; dK/dV: Q and dO tiles). Each job runs as two half
+// jobs of 64 columns (keys for dQ, query rows for dK/dV) with two S / dP slots in TMEM, so
+// the S / dP MMAs of the next half job overlap the elementwise work on the current one.
+// TMEM: S slots at columns 0 and 64, dP slots at 128 and 192, the accumulators from 256
+// (dQ: D columns; dK/dV: dV then dK). Every mbarrier wait is bounded as in the forward.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_bf16.h>
@@ -67,14 +69,16 @@ struct BwdCfg {
   static constexpr int OFF_ROWV = OFF_RING + STAGES * TILE_BYTES;  // dK/dV: per warp 128 lse2 + 128 delta
   static constexpr int OFF_BAR = OFF_ROWV + 4 * 2 * 128 * 4;
   static constexpr int B_AFULL = 0, B_AEMPTY = 1, B_RFULL = 2, B_REMPTY = B_RFULL + STAGES,
-                       B_SFULL = B_REMPTY + STAGES, B_PFULL = B_SFULL + 1, B_ACCFULL = B_PFULL + 1,
+                       B_SFULL = B_REMPTY + STAGES, B_PFULL = B_SFULL + 2, B_ACCFULL = B_PFULL + 2,
                        B_ACCEMPTY = B_ACCFULL + 1, B_DRAIN = B_ACCEMPTY + 1, NBAR = B_DRAIN + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;       // [0] TMEM base, [1] abort flag
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;   // + slack to align the base to 1 KiB
   static constexpr int THREADS = 256;
+  // TMEM: S half-job slots at 0 and 64, dP slots at 128 and 192, accumulators from 256
   static constexpr int TM_S = 0, TM_P = 128, TM_ACC = 256;
-  static constexpr uint32_t IDESC_SS =  // M=128, N=128, bf16 x bf16 -> fp32, both K-major
-      (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(128 >> 3) << 17) | (uint32_t(128 >> 4) << 24);
+  static constexpr int HALF_BYTES = 64 * 128;  // 64 rows of every 64-column box (8 swizzle atoms)
+  static constexpr uint32_t IDESC_SS =  // M=128, N=64 (a half job), bf16 x bf16 -> fp32, both K-major
+      (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(64 >> 3) << 17) | (uint32_t(128 >> 4) << 24);
   static constexpr uint32_t IDESC_TS =  // M=128, N=D, A from TMEM, B MN-major
       (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) | (uint32_t(D >> 3) << 17) | (uint32_t(128 >> 4) << 24);
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
@@ -86,23 +90,19 @@ enum : int32_t {
   kBwdWaitSFull, kBwdWaitAccFull
 };
 
-// C[128 x 128] (TMEM, fp32) = A[128 x D] . B[128 x D]^T, both tiles K-major in shared memory.
+// C[128 x 64] (TMEM, fp32) = A[128 x D] . B[64 x D]^T: A a whole tile, B 64 rows of a tile
+// (b_smem = tile + half * HALF_BYTES); both K-major in shared memory.
 template <int D>
-__device__ __forceinline__ void mma_tile_ss(uint32_t d, uint32_t a_smem, uint32_t b_smem, uint32_t idesc) {
+__device__ __forceinline__ void mma_half_ss(uint32_t d, uint32_t a_smem, uint32_t b_smem, uint32_t idesc) {
   if constexpr (D == 128) mma_ss_x8_k128(d, desc_of(desc_lo(a_smem, 16)), desc_of(desc_lo(b_smem, 16)), idesc, 0u);
   else mma_ss_x4_k64(d, desc_of(desc_lo(a_smem, 16)), desc_of(desc_lo(b_smem, 16)), idesc, 0u);
 }
 
-// C[128 x D] (+)= A[128 x 128] (bf16 in TMEM) . B[128 x D] (tile in shared memory, MN-major).
-template <int D>
-__device__ __forceinline__ void mma_tile_ts(uint32_t d, uint32_t a_tmem, uint32_t b_smem, uint32_t idesc,
+// C[128 x D] (+)= A[128 x 64] (bf16 in TMEM, 32 columns) . B[64 x D] (64 rows of a tile in
+// shared memory, MN-major).
+__device__ __forceinline__ void mma_half_ts(uint32_t d, uint32_t a_tmem, uint32_t b_smem, uint32_t idesc,
                                             uint32_t acc) {
-  mma_ts_x8(d, a_tmem, desc_of(desc_lo(b_smem, 128 * 128)), idesc, acc);
-}
-
-__device__ __forceinline__ bool mask_bit(const uint4& bits, int c) {
-  const uint32_t w = c < 64 ? (c < 32 ? bits.x : bits.y) : (c < 96 ? bits.z : bits.w);
-  return (w >> (c & 31)) & 1u;
+  mma_ts_x4(d, a_tmem, desc_of(desc_lo(b_smem, 128 * 128)), idesc, acc);
 }
 
 // One 128-row x D tile of bf16 gradients from TMEM (fp32, times `mul`) to global memory.
@@ -164,8 +164,10 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd_dq_kernel(const
       mbar_init(BAR(C::B_RFULL + s), 1);
       mbar_init(BAR(C::B_REMPTY + s), 1);
     }
-    mbar_init(BAR(C::B_SFULL), 1);
-    mbar_init(BAR(C::B_PFULL), 128);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(BAR(C::B_SFULL + b), 1);
+      mbar_init(BAR(C::B_PFULL + b), 128);
+    }
     mbar_init(BAR(C::B_ACCFULL), 1);
     mbar_init(BAR(C::B_ACCEMPTY), 128);
     mbar_init(BAR(C::B_DRAIN), 1);
@@ -224,45 +226,56 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd_dq_kernel(const
     }
     __syncwarp();
   } else if (warp == 1) {
-    // ---- MMA issuer ----
+    // ---- MMA issuer: half jobs u = 2 j + h (keys 64 h .. 64 h + 63 of job j's tiles) ----
+    // issued S(0), dP(0), S(1), dP(1), then dQ(u), S(u + 2), dP(u + 2): the MMAs of the next
+    // half job run while the warpgroup works on the current one (two S / dP slots).
     if (lane == 0) {
-      uint32_t rc = 0, gj = 0;
+      uint32_t rc = 0, gu = 0;
       int n = 0;
       bool ok = true;
       for (int ii = i_begin; ok && ii < i_end; ++ii, ++n) {
         const BwdItem it = p.items[p.cta_items[ii]];
         if (!wait_bounded(BAR(C::B_AFULL), n & 1, guard, kBwdWaitAFull)) break;
         tc_fence_after();
-        for (int j = 0; j < it.job_count; ++j, ++gj) {
-          const uint32_t rk = rc, rv = rc + 1;
-          rc += 2;
-          if (!wait_bounded(BAR(C::B_RFULL + rk % C::STAGES), (rk / C::STAGES) & 1, guard, kBwdWaitRFull) ||
-              !wait_bounded(BAR(C::B_RFULL + rv % C::STAGES), (rv / C::STAGES) & 1, guard, kBwdWaitRFull)) {
-            ok = false;
-            break;
+        const uint32_t base = rc;   // job j: K tile at ring index base + 2 j, V tile at base + 2 j + 1
+        rc += 2 * uint32_t(it.job_count);
+        const int U = 2 * it.job_count;
+        auto ring = [&](uint32_t r) { return sbase + C::OFF_RING + (r % C::STAGES) * C::TILE_BYTES; };
+        auto ss = [&](int u) -> bool {
+          const uint32_t slot = (gu + u) & 1, rk = base + 2 * (u >> 1), rv = rk + 1, h = u & 1;
+          if (h == 0) {
+            if (!wait_bounded(BAR(C::B_RFULL + rk % C::STAGES), (rk / C::STAGES) & 1, guard, kBwdWaitRFull) ||
+                !wait_bounded(BAR(C::B_RFULL + rv % C::STAGES), (rv / C::STAGES) & 1, guard, kBwdWaitRFull))
+              return false;
+            tc_fence_after();
           }
+          mma_half_ss<C::D>(tmem + C::TM_S + 64 * slot, sbase + C::OFF_A, ring(rk) + h * C::HALF_BYTES,
+                            C::IDESC_SS);   // S = Q K^T
+          mma_half_ss<C::D>(tmem + C::TM_P + 64 * slot, sbase + C::OFF_B, ring(rv) + h * C::HALF_BYTES,
+                            C::IDESC_SS);   // dP = dO V^T
+          if (h == 1) mma_commit(BAR(C::B_REMPTY + rv % C::STAGES));
+          mma_commit(BAR(C::B_SFULL + slot));
+          return true;
+        };
+        auto ts = [&](int u) -> bool {
+          const uint32_t g = gu + u, slot = g & 1, rk = base + 2 * (u >> 1), h = u & 1;
+          if (!wait_bounded(BAR(C::B_PFULL + slot), (g >> 1) & 1, guard, kBwdWaitPFull)) return false;
+          if (u == 0 && !wait_bounded(BAR(C::B_ACCEMPTY), (n & 1) ^ 1, guard, kBwdWaitAccEmpty)) return false;
           tc_fence_after();
-          const uint32_t k_tile = sbase + C::OFF_RING + (rk % C::STAGES) * C::TILE_BYTES;
-          const uint32_t v_tile = sbase + C::OFF_RING + (rv % C::STAGES) * C::TILE_BYTES;
-          mma_tile_ss<C::D>(tmem + C::TM_S, sbase + C::OFF_A, k_tile, C::IDESC_SS);   // S = Q K^T
-          mma_tile_ss<C::D>(tmem + C::TM_P, sbase + C::OFF_B, v_tile, C::IDESC_SS);   // dP = dO V^T
-          mma_commit(BAR(C::B_REMPTY + rv % C::STAGES));
-          mma_commit(BAR(C::B_SFULL));
-          if (!wait_bounded(BAR(C::B_PFULL), gj & 1, guard, kBwdWaitPFull)) {
-            ok = false;
-            break;
-          }
-          if (j == 0 && !wait_bounded(BAR(C::B_ACCEMPTY), (n & 1) ^ 1, guard, kBwdWaitAccEmpty)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          mma_tile_ts<C::D>(tmem + C::TM_ACC, tmem + C::TM_S, k_tile, C::IDESC_TS, j > 0 ? 1u : 0u);  // dQ += dS K
-          mma_commit(BAR(C::B_REMPTY + rk % C::STAGES));
+          mma_half_ts(tmem + C::TM_ACC, tmem + C::TM_S + 64 * slot, ring(rk) + h * C::HALF_BYTES, C::IDESC_TS,
+                      u > 0 ? 1u : 0u);     // dQ += dS K
+          if (h == 1) mma_commit(BAR(C::B_REMPTY + rk % C::STAGES));
+          return true;
+        };
+        ok = ss(0) && ss(1);
+        for (int u = 0; ok && u < U; ++u) {
+          ok = ts(u);
+          if (ok && u + 2 < U) ok = ss(u + 2);
         }
         if (!ok) break;
         mma_commit(BAR(C::B_ACCFULL));
         mma_commit(BAR(C::B_AEMPTY));
+        gu += U;
       }
       mma_commit(BAR(C::B_DRAIN));
       wait_drain(BAR(C::B_DRAIN), 0, p.timeout_ns);
@@ -273,7 +286,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd_dq_kernel(const
     const int r = tid - 128;
     const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
     const float sl2 = p.scale_log2;
-    uint32_t gj = 0;
+    uint32_t gu = 0;
     int n = 0;
     bool ok = true;
     for (int ii = i_begin; ok && ii < i_end; ++ii, ++n) {
@@ -286,41 +299,48 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd_dq_kernel(const
         lse2 = l == -INFINITY ? INFINITY : l * 1.4426950408889634f;
         dlt = p.delta[grow];
       }
-      for (int j = 0; j < it.job_count; ++j, ++gj) {
-        const int mi = p.jobs[it.job_start + j].mask;
-        uint4 bits = make_uint4(0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu);
-        if (mi >= 0) bits = __ldg(p.mask_tiles + int64_t(mi) * 128 + r);
-        else if (mi == kMaskNone) bits = make_uint4(0u, 0u, 0u, 0u);
-        if (!__all_sync(0xffffffffu, wait_bounded(BAR(C::B_SFULL), gj & 1, guard, kBwdWaitSFull))) {
+      for (int u = 0; ok && u < 2 * it.job_count; ++u) {
+        const int mi = p.jobs[it.job_start + (u >> 1)].mask;
+        const int h = u & 1;
+        uint2 bits = make_uint2(0xffffffffu, 0xffffffffu);   // this half job's 64 key bits
+        if (mi >= 0) {
+          const uint4 b4 = __ldg(p.mask_tiles + int64_t(mi) * 128 + r);
+          bits = h ? make_uint2(b4.z, b4.w) : make_uint2(b4.x, b4.y);
+        } else if (mi == kMaskNone) {
+          bits = make_uint2(0u, 0u);
+        }
+        const uint32_t g = gu + u, slot = g & 1;
+        if (!__all_sync(0xffffffffu, wait_bounded(BAR(C::B_SFULL + slot), (g >> 1) & 1, guard, kBwdWaitSFull))) {
           ok = false;
           break;
         }
         tc_fence_after();
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
           uint32_t sv[32], dv[32];
-          tmem_ld32x32(tmem + lane_base + C::TM_S + 32 * c, sv);
-          tmem_ld32x32(tmem + lane_base + C::TM_P + 32 * c, dv);
+          tmem_ld32x32(tmem + lane_base + C::TM_S + 64 * slot + 32 * c, sv);
+          tmem_ld32x32(tmem + lane_base + C::TM_P + 64 * slot + 32 * c, dv);
           tmem_wait_ld();
+          const uint32_t w = c ? bits.y : bits.x;
           uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
             float ds[2];
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const int col = 32 * c + 2 * e + h;
-              const float pr = mask_bit(bits, col) ? ex2(fmaf(__uint_as_float(sv[2 * e + h]), sl2, -lse2)) : 0.f;
-              ds[h] = pr * (__uint_as_float(dv[2 * e + h]) - dlt);
+            for (int q = 0; q < 2; ++q) {
+              const float pr = ((w >> (2 * e + q)) & 1u) ? ex2(fmaf(__uint_as_float(sv[2 * e + q]), sl2, -lse2)) : 0.f;
+              ds[q] = pr * (__uint_as_float(dv[2 * e + q]) - dlt);
             }
             pk[e] = pack_bf16(ds[0], ds[1]);
           }
-          // dS of columns 32c .. 32c+31 over S columns 16c .. 16c+15 (already read)
-          tmem_st32x16(tmem + lane_base + C::TM_S + 16 * c, pk);
+          // dS of the slot's columns 32c .. 32c+31 over its S columns 16c .. 16c+15 (already read)
+          tmem_st32x16(tmem + lane_base + C::TM_S + 64 * slot + 16 * c, pk);
         }
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(BAR(C::B_PFULL));
+        mbar_arrive(BAR(C::B_PFULL + slot));
       }
+      gu += 2 * it.job_count;
       if (!ok) break;
       if (!__all_sync(0xffffffffu, wait_bounded(BAR(C::B_ACCFULL), n & 1, guard, kBwdWaitAccFull))) break;
       tc_fence_after();
@@ -355,8 +375,10 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd_dkv_kernel(cons
       mbar_init(BAR(C::B_RFULL + s), 1);
       mbar_init(BAR(C::B_REMPTY + s), 1);
     }
-    mbar_init(BAR(C::B_SFULL), 1);
-    mbar_init(BAR(C::B_PFULL), 128);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(BAR(C::B_SFULL + b), 1);
+      mbar_init(BAR(C::B_PFULL + b), 128);
+    }
     mbar_init(BAR(C::B_ACCFULL), 1);
     mbar_init(BAR(C::B_ACCEMPTY), 128);
     mbar_init(BAR(C::B_DRAIN), 1);
@@ -415,47 +437,60 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd_dkv_kernel(cons
     }
     __syncwarp();
   } else if (warp == 1) {
-    // ---- MMA issuer ----
+    // ---- MMA issuer: half jobs u = 2 j + h (query rows 64 h .. 64 h + 63 of job j's tiles),
+    // issued as in the dQ kernel: S^T(0), dP^T(0), S^T(1), dP^T(1), then dV, dK (u), S^T, dP^T (u + 2)
     if (lane == 0) {
-      uint32_t rc = 0, gj = 0;
+      uint32_t rc = 0, gu = 0;
       int n = 0;
       bool ok = true;
       for (int ii = i_begin; ok && ii < i_end; ++ii, ++n) {
         const BwdItem it = p.items[p.cta_items[ii]];
         if (!wait_bounded(BAR(C::B_AFULL), n & 1, guard, kBwdWaitAFull)) break;
         tc_fence_after();
-        for (int j = 0; j < it.job_count; ++j, ++gj) {
-          const uint32_t rq = rc, rd = rc + 1;
-          rc += 2;
-          if (!wait_bounded(BAR(C::B_RFULL + rq % C::STAGES), (rq / C::STAGES) & 1, guard, kBwdWaitRFull) ||
-              !wait_bounded(BAR(C::B_RFULL + rd % C::STAGES), (rd / C::STAGES) & 1, guard, kBwdWaitRFull)) {
-            ok = false;
-            break;
+        const uint32_t base = rc;   // job j: Q tile at ring index base + 2 j, dO tile at base + 2 j + 1
+        rc += 2 * uint32_t(it.job_count);
+        const int U = 2 * it.job_count;
+        auto ring = [&](uint32_t r) { return sbase + C::OFF_RING + (r % C::STAGES) * C::TILE_BYTES; };
+        auto ss = [&](int u) -> bool {
+          const uint32_t slot = (gu + u) & 1, rq = base + 2 * (u >> 1), rd = rq + 1, h = u & 1;
+          if (h == 0) {
+            if (!wait_bounded(BAR(C::B_RFULL + rq % C::STAGES), (rq / C::STAGES) & 1, guard, kBwdWaitRFull) ||
+                !wait_bounded(BAR(C::B_RFULL + rd % C::STAGES), (rd / C::STAGES) & 1, guard, kBwdWaitRFull))
+              return false;
+            tc_fence_after();
           }
+          mma_half_ss<C::D>(tmem + C::TM_S + 64 * slot, sbase + C::OFF_A, ring(rq) + h * C::HALF_BYTES,
+                            C::IDESC_SS);   // S^T = K Q^T
+          mma_half_ss<C::D>(tmem + C::TM_P + 64 * slot, sbase + C::OFF_B, ring(rd) + h * C::HALF_BYTES,
+                            C::IDESC_SS);   // dP^T = V dO^T
+          mma_commit(BAR(C::B_SFULL + slot));
+          return true;
+        };
+        auto ts = [&](int u) -> bool {
+          const uint32_t g = gu + u, slot = g & 1, rq = base + 2 * (u >> 1), rd = rq + 1, h = u & 1;
+          if (!wait_bounded(BAR(C::B_PFULL + slot), (g >> 1) & 1, guard, kBwdWaitPFull)) return false;
+          if (u == 0 && !wait_bounded(BAR(C::B_ACCEMPTY), (n & 1) ^ 1, guard, kBwdWaitAccEmpty)) return false;
           tc_fence_after();
-          const uint32_t q_tile = sbase + C::OFF_RING + (rq % C::STAGES) * C::TILE_BYTES;
-          const uint32_t do_tile = sbase + C::OFF_RING + (rd % C::STAGES) * C::TILE_BYTES;
-          mma_tile_ss<C::D>(tmem + C::TM_S, sbase + C::OFF_A, q_tile, C::IDESC_SS);    // S^T = K Q^T
-          mma_tile_ss<C::D>(tmem + C::TM_P, sbase + C::OFF_B, do_tile, C::IDESC_SS);   // dP^T = V dO^T
-          mma_commit(BAR(C::B_SFULL));
-          if (!wait_bounded(BAR(C::B_PFULL), gj & 1, guard, kBwdWaitPFull)) {
-            ok = false;
-            break;
+          const uint32_t acc = u > 0 ? 1u : 0u;
+          mma_half_ts(tmem + C::TM_ACC, tmem + C::TM_S + 64 * slot, ring(rd) + h * C::HALF_BYTES, C::IDESC_TS,
+                      acc);                 // dV += P^T dO
+          mma_half_ts(tmem + C::TM_ACC + C::D, tmem + C::TM_P + 64 * slot, ring(rq) + h * C::HALF_BYTES,
+                      C::IDESC_TS, acc);    // dK += dS^T Q
+          if (h == 1) {
+            mma_commit(BAR(C::B_REMPTY + rq % C::STAGES));
+            mma_commit(BAR(C::B_REMPTY + rd % C::STAGES));
           }
-          if (j == 0 && !wait_bounded(BAR(C::B_ACCEMPTY), (n & 1) ^ 1, guard, kBwdWaitAccEmpty)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t acc = j > 0 ? 1u : 0u;
-          mma_tile_ts<C::D>(tmem + C::TM_ACC, tmem + C::TM_S, do_tile, C::IDESC_TS, acc);         // dV += P^T dO
-          mma_tile_ts<C::D>(tmem + C::TM_ACC + C::D, tmem + C::TM_P, q_tile, C::IDESC_TS, acc);   // dK += dS^T Q
-          mma_commit(BAR(C::B_REMPTY + rq % C::STAGES));
-          mma_commit(BAR(C::B_REMPTY + rd % C::STAGES));
+          return true;
+        };
+        ok = ss(0) && ss(1);
+        for (int u = 0; ok && u < U; ++u) {
+          ok = ts(u);
+          if (ok && u + 2 < U) ok = ss(u + 2);
         }
         if (!ok) break;
         mma_commit(BAR(C::B_ACCFULL));
         mma_commit(BAR(C::B_AEMPTY));
+        gu += U;
       }
       mma_commit(BAR(C::B_DRAIN));
       wait_drain(BAR(C::B_DRAIN), 0, p.timeout_ns);
@@ -469,63 +504,72 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd_dkv_kernel(cons
     // this warp's copy of the job's per-query-row terms (no barrier across warps)
     float* rl2 = reinterpret_cast<float*>(sgen + C::OFF_ROWV) + (warp - 4) * 256;
     float* rdl = rl2 + 128;
-    uint32_t gj = 0;
+    uint32_t gu = 0;
     int n = 0;
     bool ok = true;
     for (int ii = i_begin; ok && ii < i_end; ++ii, ++n) {
       const BwdItem it = p.items[p.cta_items[ii]];
-      for (int j = 0; j < it.job_count; ++j, ++gj) {
-        const BwdJob jb = p.jobs[it.job_start + j];
-        __syncwarp();   // the previous job's reads of rl2 / rdl are done
+      uint4 bits = make_uint4(0u, 0u, 0u, 0u);
+      for (int u = 0; ok && u < 2 * it.job_count; ++u) {
+        const int h = u & 1;
+        if (h == 0) {
+          // a new job: its query rows' lse (log2 e scaled) and delta into this warp's copy
+          const BwdJob jb = p.jobs[it.job_start + (u >> 1)];
+          __syncwarp();   // the previous job's reads of rl2 / rdl are done
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const int qr = 4 * lane + k;
-          float l2 = INFINITY, dl = 0.f;
-          if (qr < jb.rows) {
-            const int64_t g = int64_t(jb.tok + qr) * p.hq + jb.head;
-            const float l = p.lse[g];
-            l2 = l == -INFINITY ? INFINITY : l * 1.4426950408889634f;
-            dl = p.delta[g];
+          for (int k = 0; k < 4; ++k) {
+            const int qr = 4 * lane + k;
+            float l2 = INFINITY, dl = 0.f;
+            if (qr < jb.rows) {
+              const int64_t g = int64_t(jb.tok + qr) * p.hq + jb.head;
+              const float l = p.lse[g];
+              l2 = l == -INFINITY ? INFINITY : l * 1.4426950408889634f;
+              dl = p.delta[g];
+            }
+            rl2[qr] = l2;
+            rdl[qr] = dl;
           }
-          rl2[qr] = l2;
-          rdl[qr] = dl;
+          __syncwarp();
+          bits = make_uint4(0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu);
+          if (jb.mask >= 0) bits = __ldg(p.mask_tiles + int64_t(jb.mask) * 128 + r);
+          else if (jb.mask == kMaskNone) bits = make_uint4(0u, 0u, 0u, 0u);
         }
-        __syncwarp();
-        uint4 bits = make_uint4(0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu);
-        if (jb.mask >= 0) bits = __ldg(p.mask_tiles + int64_t(jb.mask) * 128 + r);
-        else if (jb.mask == kMaskNone) bits = make_uint4(0u, 0u, 0u, 0u);
-        if (!__all_sync(0xffffffffu, wait_bounded(BAR(C::B_SFULL), gj & 1, guard, kBwdWaitSFull))) {
+        const uint32_t g = gu + u, slot = g & 1;
+        if (!__all_sync(0xffffffffu, wait_bounded(BAR(C::B_SFULL + slot), (g >> 1) & 1, guard, kBwdWaitSFull))) {
           ok = false;
           break;
         }
         tc_fence_after();
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
           uint32_t sv[32], dv[32];
-          tmem_ld32x32(tmem + lane_base + C::TM_S + 32 * c, sv);
-          tmem_ld32x32(tmem + lane_base + C::TM_P + 32 * c, dv);
+          tmem_ld32x32(tmem + lane_base + C::TM_S + 64 * slot + 32 * c, sv);
+          tmem_ld32x32(tmem + lane_base + C::TM_P + 64 * slot + 32 * c, dv);
           tmem_wait_ld();
+          const int q0 = 64 * h + 32 * c;   // first query row of the chunk
+          const uint32_t w = h ? (c ? bits.w : bits.z) : (c ? bits.y : bits.x);
           uint32_t pp[16], pd[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
             float pr[2], ds[2];
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const int col = 32 * c + 2 * e + h;   // query row of the tile
-              pr[h] = mask_bit(bits, col) ? ex2(fmaf(__uint_as_float(sv[2 * e + h]), sl2, -rl2[col])) : 0.f;
-              ds[h] = pr[h] * (__uint_as_float(dv[2 * e + h]) - rdl[col]);
+            for (int q = 0; q < 2; ++q) {
+              const int qi = q0 + 2 * e + q;
+              pr[q] = ((w >> (2 * e + q)) & 1u) ? ex2(fmaf(__uint_as_float(sv[2 * e + q]), sl2, -rl2[qi])) : 0.f;
+              ds[q] = pr[q] * (__uint_as_float(dv[2 * e + q]) - rdl[qi]);
             }
             pp[e] = pack_bf16(pr[0], pr[1]);
             pd[e] = pack_bf16(ds[0], ds[1]);
           }
-          // P^T over S^T columns 16c.., dS^T over dP^T columns 16c.. (both already read)
-          tmem_st32x16(tmem + lane_base + C::TM_S + 16 * c, pp);
-          tmem_st32x16(tmem + lane_base + C::TM_P + 16 * c, pd);
+          // P^T over the slot's S^T columns 16c.., dS^T over its dP^T columns 16c.. (already read)
+          tmem_st32x16(tmem + lane_base + C::TM_S + 64 * slot + 16 * c, pp);
+          tmem_st32x16(tmem + lane_base + C::TM_P + 64 * slot + 16 * c, pd);
         }
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(BAR(C::B_PFULL));
+        mbar_arrive(BAR(C::B_PFULL + slot));
       }
+      gu += 2 * it.job_count;
       if (!ok) break;
       if (!__all_sync(0xffffffffu, wait_bounded(BAR(C::B_ACCFULL), n & 1, guard, kBwdWaitAccFull))) break;
       tc_fence_after();

@@ -25,6 +25,7 @@
 #include <new>
 #include <numeric>
 #include <queue>
+#include <unordered_map>
 #include <stdexcept>
 #include <utility>
 #include <vector>
@@ -768,13 +769,25 @@ void work_stats(const attn_plan_t& m, const WorkList& wl, attn_plan_stats_t& st)
 
 // ---- backward planning ----------------------------------------------------------------
 
-// Longest-first greedy assignment of items (costs) onto units: per-unit offsets and lists.
-void assign_lpt(const std::vector<int64_t>& cost, int units, std::vector<int32_t>& off, std::vector<int32_t>& list) {
+// Greedy least-loaded assignment of items (costs) onto units, group by group: groups (items
+// sharing the tiles they stream, i.e. one (sequence, key/value head)) go out largest first and
+// their items longest first, so that the units working on one group at a time find its
+// tiles in L2. Returns per-unit offsets and item lists.
+void assign_lpt(const std::vector<int64_t>& cost, const std::vector<int64_t>& group, int units,
+                std::vector<int32_t>& off, std::vector<int32_t>& list) {
   const int n = int(cost.size());
   const int C = std::max(1, std::min(units, n));
   std::vector<int32_t> order(n);
   std::iota(order.begin(), order.end(), 0);
-  std::stable_sort(order.begin(), order.end(), [&](int32_t x, int32_t y) { return cost[x] > cost[y]; });
+  std::unordered_map<int64_t, int64_t> gcost;
+  for (int i = 0; i < n; ++i) gcost[group[i]] += cost[i];
+  std::stable_sort(order.begin(), order.end(), [&](int32_t x, int32_t y) {
+    if (group[x] != group[y]) {
+      const int64_t cx = gcost[group[x]], cy = gcost[group[y]];
+      return cx != cy ? cx > cy : group[x] < group[y];
+    }
+    return cost[x] > cost[y];
+  });
   using Load = std::pair<int64_t, int32_t>;
   std::priority_queue<Load, std::vector<Load>, std::greater<Load>> heap;
   for (int c = 0; c < C; ++c) heap.push(Load{0, c});
@@ -807,7 +820,7 @@ struct BwdLists {
 
 void build_bwd(const Shape& s, const std::vector<std::vector<int32_t>>& cnts, int num_sms, BwdLists& bl) {
   const int g = s.hq / s.hkv;
-  std::vector<int64_t> q_cost, kv_cost;
+  std::vector<int64_t> q_cost, kv_cost, q_group, kv_group;
   for (int b = 0; b < s.B; ++b) {
     const int lq = s.lq[b], lk = s.lk[b];
     const int n_qt = (lq + kTile - 1) / kTile, n_kt = (lk + kTile - 1) / kTile;
@@ -838,6 +851,7 @@ void build_bwd(const Shape& s, const std::vector<std::vector<int32_t>>& cnts, in
             bl.q_jobs.push_back(BwdJob{s.koff[b], kMaskNone, h, 0});
           it.job_count = int32_t(bl.q_jobs.size()) - it.job_start;
           q_cost.push_back(it.job_count + 2);
+          q_group.push_back(int64_t(b) * s.hkv + kh);
           bl.q_items.push_back(it);
         }
       // dK/dV items
@@ -854,12 +868,13 @@ void build_bwd(const Shape& s, const std::vector<std::vector<int32_t>>& cnts, in
           bl.kv_jobs.push_back(BwdJob{s.qoff[b], kMaskNone, kh * g, 0});
         it.job_count = int32_t(bl.kv_jobs.size()) - it.job_start;
         kv_cost.push_back(it.job_count + 2);
+        kv_group.push_back(int64_t(b) * s.hkv + kh);
         bl.kv_items.push_back(it);
       }
     }
   }
-  assign_lpt(q_cost, num_sms, bl.q_off, bl.q_list);
-  assign_lpt(kv_cost, num_sms, bl.kv_off, bl.kv_list);
+  assign_lpt(q_cost, q_group, num_sms, bl.q_off, bl.q_list);
+  assign_lpt(kv_cost, kv_group, num_sms, bl.kv_off, bl.kv_list);
 }
 
 // Row-major 2 KiB tile (row r: 4 words, bit c = key c) -> the transposed tile (row c, bit r).
