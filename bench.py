@@ -258,8 +258,11 @@ def run_ours(args, rank, world, local_rank):
     stream = torch.cuda.current_stream()
     q, k, v = device_inputs(wl, dev)
     bwd = args.pass_ == "bwd"
+    fp8 = args.dtype == "e4m3"
     if bwd and (wl.paged or wl.d > 128):
         raise SystemExit("--pass bwd: contiguous K/V and head_dim <= 128 only (workloads 1, 4, 5)")
+    if fp8 and (bwd or wl.paged or wl.d != 128):
+        raise SystemExit("--dtype e4m3: the forward with contiguous K/V and head_dim 128 (workloads 4, 5)")
     plans = [make_plan(M, wl, spec, dev, args.kv_splits, backward=bwd) for spec in wl.masks]
     stats = [M.attn_plan_get_stats(p) for p in plans]
     flops = [flops_of(s, wl) * (2.5 if bwd else 1.0) for s in stats]
@@ -275,11 +278,23 @@ def run_ours(args, rank, world, local_rank):
         dout = torch.randn(tq, wl.hq, wl.d, generator=gen, device=dev).to(torch.bfloat16)
         dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
         in_bytes += sum(o.numel() * 2 + l.numel() * 4 for o, l in zip(outs, lses)) + dout.numel() * 2
+    if fp8:
+        # per-tensor e4m3 inputs; V transposed once per plan (a cache would keep it in that layout)
+        import workloads as W
+        (q8, qs), (k8, ks), (v8, vs) = (W.quantize_e4m3(t) for t in (wl.q, wl.k, wl.v))
+        q8, k8, v8 = q8.to(dev), k8.to(dev), v8.to(dev)
+        ldvs = [(st["vt_keys"] + 15) // 16 * 16 for st in stats]
+        vts = [torch.empty(wl.hkv, wl.d, ld, dtype=torch.uint8, device=dev) for ld in ldvs]
+        for p, vt, ld in zip(plans, vts, ldvs):
+            M.attn_fp8_transpose_v(p, v8, vt, ld, stream)
+        in_bytes = q8.numel() + k8.numel() + v8.numel()
     flush = torch.empty(256 * 2**20, dtype=torch.uint8, device=dev) if in_bytes <= L2_BYTES else None
 
     def run_one(i, p):
         if bwd:
             M.attn_masked_bwd(p, q, k, v, outs[i], lses[i], dout, dq, dk, dv, stream)
+        elif fp8:
+            M.attn_masked_fwd_fp8(p, q8, k8, vts[i], ldvs[i], qs, ks, vs, outs[i], lses[i], stream)
         else:
             M.attn_masked_fwd(p, q, k, v, outs[i], lses[i], stream)
 
@@ -330,7 +345,19 @@ def run_ours(args, rank, world, local_rank):
         hdo = dout.cpu().pin_memory()
         hg = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (dq, dk, dv)]
 
+    if fp8:
+        hq_, hk_, hv_ = (t.cpu().pin_memory() for t in (q8, k8, vts[0]))
+
     def e2e_step():
+        if fp8:   # host e4m3 q, k and transposed v in; out / lse back
+            q8.copy_(hq_, non_blocking=True)
+            k8.copy_(hk_, non_blocking=True)
+            vts[0].copy_(hv_, non_blocking=True)
+            for i, p in enumerate(plans):
+                run_one(i, p)
+                ho[i].copy_(outs[i], non_blocking=True)
+                hl[i].copy_(lses[i], non_blocking=True)
+            return
         q.copy_(hq_, non_blocking=True)
         k.copy_(hk_, non_blocking=True)
         v.copy_(hv_, non_blocking=True)
@@ -364,7 +391,7 @@ def run_ours(args, rank, world, local_rank):
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1)
-    h2d = in_bytes
+    h2d = in_bytes if not fp8 else q8.numel() + k8.numel() + vts[0].numel()
     d2h = sum(o.numel() * 2 + l.numel() * 4 for o, l in zip(outs, lses))
     if bwd:
         d2h = len(plans) * sum(t.numel() * 2 for t in (dq, dk, dv))
@@ -385,20 +412,25 @@ def run_ours(args, rank, world, local_rank):
     use_sustained = clocks is not None and clocks["sm_mhz"] < 0.9 * clocks["sm_max_mhz"]
     peak = sustained if use_sustained else burst
     pk_src += " bf16_tflops_sustained" if use_sustained else " bf16_tflops (burst)"
+    if fp8:   # e4m3 tensor rate: the measured bf16 figure x the nominal fp8 / bf16 ratio (4.5 / 2.25)
+        peak *= 2.0
+        pk_src += " x 2 (nominal e4m3 / bf16 ratio)"
     avg_launch_ms = sum(sum(x) for x in launch_ms) / sum(len(x) for x in launch_ms)
     achieved = (sum(flops) / len(flops)) / (avg_launch_ms * 1e-3) / 1e12
-    tr = None if bwd else traffic_for(wl.name)
+    tr = None if (bwd or fp8) else traffic_for(wl.name)
     mask_bytes = sum(s["mask_tile_reads"] for s in stats) * 2048.0
     line = {
         "metric": METRIC_BWD if bwd else METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) bf16, lengths from seed)",
+        "vs_baseline": None, "dtype": "e4m3" if fp8 else "bf16",
+        "data": "synthetic (seeded N(0,1) bf16, lengths from seed" + ("; per-tensor e4m3)" if fp8 else ")"),
         "config": config_of(wl, args, world),
         "pct_of_peak": 100.0 * value / world / peak,
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": tr,
                      "peak_source": pk_src,
                      "kernel": (f"masked_attn_bwd_dq_kernel + masked_attn_bwd_dkv_kernel d={wl.d}" if bwd
+                                else f"masked_attn_fwd_kernel e4m3 d={wl.d}" if fp8
                                 else f"masked_attn_fwd_kernel d={wl.d}"),
                      "algorithmic_flops_per_launch": sum(flops) / len(flops),
                      "avg_launch_ms": avg_launch_ms},
@@ -415,7 +447,7 @@ def run_ours(args, rank, world, local_rank):
         "gpu_launches": (3 * len(plans) if bwd else sum(1 + (s["merge_tiles"] > 0) for s in stats)) * args.steps,
         "clocks": clocks,
     }
-    if world == 1 and not args.no_cpu_baseline and not bwd:
+    if world == 1 and not args.no_cpu_baseline and not bwd and not fp8:
         pairs, secs, desc = oracle_sample(wl, wl.masks, args.cpu_seconds)
         line["cpu_baseline"] = {"value": 4.0 * wl.d * pairs / secs / 1e12, "unit": "TFLOP/s",
                                 "cores": blas_threads(), "kind": "oracle", "sample": desc,
@@ -433,6 +465,8 @@ def main():
                     help="1-5: the benchmark workloads; 6: long-context tree verify (split-KV case)")
     ap.add_argument("--pass", dest="pass_", choices=["fwd", "bwd"], default="fwd",
                     help="fwd: the forward (the benchmark metric); bwd: the backward pass (workloads 1, 4, 5)")
+    ap.add_argument("--dtype", choices=["bf16", "e4m3"], default="bf16",
+                    help="e4m3: the fp8 forward (head_dim 128, contiguous K/V: workloads 4, 5)")
     ap.add_argument("--kv-splits", type=int, default=0,
                     help="split-KV: 0 automatic, 1 never, N >= 2 at most N key ranges per query tile")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)

@@ -157,6 +157,8 @@ typedef struct {
   int32_t cluster_size;             /* CTAs that cooperate on one work item (2: a pair of SMs) */
   int32_t kv_splits_max;            /* largest number of key ranges any query tile was split into (1: none) */
   int32_t merge_tiles;              /* 128-row query tiles whose partial results the merge kernel combines */
+  int64_t vt_keys;                  /* contiguous K/V: columns of the transposed V that attn_fp8_transpose_v
+                                       writes (each sequence starts at a multiple of 128); 0 if paged */
 } attn_plan_stats_t;
 
 /* Validate and plan. `stream` orders the plan's device work (the CUSTOM mask scan and
@@ -203,6 +205,30 @@ attn_status_t attn_plan_bwd(const attn_problem_t* problem, const attn_mask_desc_
 attn_status_t attn_masked_bwd(const attn_plan_t* plan, const void* q, const void* k, const void* v,
                               const void* out, const float* lse, const void* dout, void* dq, void* dk, void* dv,
                               attn_stream_t stream);
+
+/* e4m3 (fp8) forward. No page names a layout for it; "Custom mask slows down attention."
+ * asks whether the custom-mask path supports fp8. Inputs are e4m3 bytes (1 sign, 4
+ * exponent bits with bias 7, 3 mantissa bits; no infinities) with per-tensor scales:
+ * the real values are q_scale * q8, k_scale * k8, v_scale * v8. The scores
+ * scale * q_scale * k_scale * (q8 . k8) are exact in fp32; P is rounded to e4m3 for the
+ * P V product (the row sums use P before rounding); out (bf16) and lse (fp32) as in
+ * attn_masked_fwd.
+ *   q   bytes [total_q][hq][128]        k bytes [total_k][hkv][128]
+ *   vt  bytes [hkv][128][ldv]           V transposed per head by attn_fp8_transpose_v
+ *   ldv >= stats.vt_keys, a multiple of 16
+ * head_dim 128 and contiguous K/V only (else UNSUPPORTED); the plan is an ordinary
+ * attn_plan() (split-KV applies). Pointers 16-byte aligned (lse: 4-byte, may be NULL).
+ * Allocates nothing. Errors: INVALID_ARG, UNSUPPORTED, CUDA. */
+attn_status_t attn_masked_fwd_fp8(const attn_plan_t* plan, const void* q, const void* k, const void* vt,
+                                  int64_t ldv, float q_scale, float k_scale, float v_scale, void* out,
+                                  float* lse, attn_stream_t stream);
+
+/* V bytes [total_k][hkv][head_dim] -> vt [hkv][head_dim][ldv]: sequence b's keys go to
+ * columns from the sum over earlier sequences of their key counts rounded up to 128, the
+ * gaps are zero. ldv >= stats.vt_keys and a multiple of 16. Asynchronous on `stream`.
+ * Errors: INVALID_ARG (paged plan, null pointer, ldv), UNSUPPORTED (head_dim % 32), CUDA. */
+attn_status_t attn_fp8_transpose_v(const attn_plan_t* plan, const void* v, void* vt, int64_t ldv,
+                                   attn_stream_t stream);
 
 /* Copy the 128 x 128 tile classes (0 empty, 1 full, 2 partial) in the order sequence,
  * query tile, key tile (row-major) into host_dst[0 .. n). *n_needed (may be NULL)

@@ -28,7 +28,7 @@ RANGE_FULL, RANGE_CAUSAL, RANGE_INV_CAUSAL, RANGE_BI_CAUSAL, RANGE_CHUNK_CAUSAL 
 EXPORTS = ("attn_plan", "attn_masked_fwd", "attn_plan_get_tile_classes", "attn_plan_get_stats",
            "attn_plan_check_status", "attn_plan_set_debug", "attn_plan_destroy", "attn_classify_host",
            "attn_status_string", "attn_masked_fwd_noalloc", "attn_test_exp2_poly", "attn_plan_dry_run",
-           "attn_plan_bwd", "attn_masked_bwd")
+           "attn_plan_bwd", "attn_masked_bwd", "attn_masked_fwd_fp8", "attn_fp8_transpose_v")
 
 
 class AttnError(RuntimeError):
@@ -63,7 +63,7 @@ class attn_plan_stats_t(ctypes.Structure):
                 ("tiles_partial", ctypes.c_int64), ("mask_tiles", ctypes.c_int64), ("work_items", ctypes.c_int64),
                 ("jobs", ctypes.c_int64), ("mask_tile_reads", ctypes.c_int64), ("ctas", ctypes.c_int32), ("heads_per_tile", ctypes.c_int32),
                 ("tiles_per_cta", ctypes.c_int32), ("cluster_size", ctypes.c_int32),
-                ("kv_splits_max", ctypes.c_int32), ("merge_tiles", ctypes.c_int32)]
+                ("kv_splits_max", ctypes.c_int32), ("merge_tiles", ctypes.c_int32), ("vt_keys", ctypes.c_int64)]
 
 
 _lib = None
@@ -94,6 +94,9 @@ def lib() -> ctypes.CDLL:
         L.attn_plan_bwd.argtypes = [ctypes.POINTER(attn_problem_t), ctypes.POINTER(attn_mask_desc_t), vp,
                                     ctypes.POINTER(vp)]
         L.attn_masked_bwd.argtypes = [vp] * 11
+        L.attn_masked_fwd_fp8.argtypes = [vp, vp, vp, vp, i64, ctypes.c_float, ctypes.c_float, ctypes.c_float, vp, vp,
+                                          vp]
+        L.attn_fp8_transpose_v.argtypes = [vp, vp, vp, i64, vp]
         L.attn_plan_dry_run.argtypes = [ctypes.POINTER(attn_problem_t), ctypes.POINTER(attn_mask_desc_t), i32,
                                         ctypes.POINTER(attn_plan_stats_t)]
         L.attn_masked_fwd_noalloc.argtypes = [ctypes.POINTER(attn_problem_t), ctypes.POINTER(attn_mask_desc_t),
@@ -357,3 +360,17 @@ def backward(plan: Plan, q, k, v, out, lse, dout, stream=None):
     dv = torch.empty_like(v)
     attn_masked_bwd(plan, q, k, v, out, lse, dout, dq, dk, dv, stream)
     return dq, dk, dv
+
+
+def attn_fp8_transpose_v(plan: Plan, v8, vt8, ldv: int, stream=None) -> None:
+    """attn_fp8_transpose_v(): e4m3 V [total_k, hkv, d] -> vt [hkv, d, ldv] (uint8 tensors)."""
+    _check(lib().attn_fp8_transpose_v(plan.handle, _ptr(v8), _ptr(vt8), int(ldv), _stream(stream)),
+           "attn_fp8_transpose_v")
+
+
+def attn_masked_fwd_fp8(plan: Plan, q8, k8, vt8, ldv: int, q_scale: float, k_scale: float, v_scale: float, out,
+                        lse=None, stream=None) -> None:
+    """attn_masked_fwd_fp8(): e4m3 q, k (uint8 tensors) and transposed v with per-tensor scales."""
+    _check(lib().attn_masked_fwd_fp8(plan.handle, _ptr(q8), _ptr(k8), _ptr(vt8), int(ldv), float(q_scale),
+                                     float(k_scale), float(v_scale), _ptr(out), _ptr(lse), _stream(stream)),
+           "attn_masked_fwd_fp8")

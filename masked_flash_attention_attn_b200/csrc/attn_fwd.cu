@@ -59,18 +59,23 @@ struct Params {
   int32_t* status;
   int32_t hq, R, hp, page_size, num_pages, debug_flags;
   float scale_log2;
+  float v_scale;       // e4m3 forward: the value tensor's scale (1 for bf16)
   int64_t timeout_ns;
 };
 
-template <int D_, int NQ_, int STAGES_, bool PAGED_, int EMU_ = 0>
+// FP8_: e4m3 Q, K and V (the latter transposed, [Hkv][d][keys]) with .kind::f8f6f4 MMAs and P
+// quantised to e4m3 in TMEM; head_dim 128 only.
+template <int D_, int NQ_, int STAGES_, bool PAGED_, int EMU_ = 0, bool FP8_ = false>
 struct Cfg {
   static constexpr int D = D_, NQ = NQ_, STAGES = STAGES_;
   static constexpr int EMU = EMU_;               // of every 8 column pairs, EMU use exp2_poly
   static constexpr bool PAGED = PAGED_;
+  static constexpr bool FP8 = FP8_;
+  static constexpr int BOX_COLS = FP8 ? 128 : 64;  // elements per 128-byte box row
   static constexpr int CH = D < 128 ? D : 128;   // columns of one ring chunk
   static constexpr int NCH = D / CH;             // ring chunks per K or V tile
-  static constexpr int NBOX = CH / 64;           // 64-column (128-byte) boxes per chunk
-  static constexpr int QBOX = D / 64;            // 64-column boxes per Q tile
+  static constexpr int NBOX = CH / BOX_COLS;     // 128-byte boxes per chunk
+  static constexpr int QBOX = D / BOX_COLS;      // 128-byte boxes per Q tile
   static constexpr int BOX_BYTES = 128 * 128;    // 128 rows x 128 bytes
   static constexpr int Q_BYTES = QBOX * BOX_BYTES;
   static constexpr int CHUNK_BYTES = NBOX * BOX_BYTES;
@@ -89,10 +94,14 @@ struct Cfg {
   static constexpr int REG_LOW = 64, REG_HIGH = 208;
   static constexpr int REG_SPLIT_TOTAL = 128 * REG_LOW + 128 * NQ * REG_HIGH;
   static constexpr int TM_O = 256;
-  static constexpr uint32_t IDESC_QK =  // M=128, N=128, bf16 x bf16 -> fp32, both K-major
-      (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(128 >> 3) << 17) | (uint32_t(128 >> 4) << 24);
-  static constexpr uint32_t IDESC_PV =  // M=128, N=CH, A (P) from TMEM K-major, B (V) MN-major
-      (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) | (uint32_t(CH >> 3) << 17) | (uint32_t(128 >> 4) << 24);
+  // instruction descriptors: fp32 accumulate (bit 4); A / B types bf16 (1 at bits 7 / 10) or
+  // e4m3 (0); B major-ness bit 16; N / 8 at bit 17; M / 16 at bit 24
+  static constexpr uint32_t AB_TYPES = FP8 ? 0u : (1u << 7) | (1u << 10);
+  static constexpr uint32_t IDESC_QK =  // M=128, N=128, both K-major
+      (1u << 4) | AB_TYPES | (uint32_t(128 >> 3) << 17) | (uint32_t(128 >> 4) << 24);
+  static constexpr uint32_t IDESC_PV =  // M=128, N=CH, A (P) from TMEM; B: V MN-major (bf16), V^T K-major (e4m3)
+      (1u << 4) | AB_TYPES | (FP8 ? 0u : (1u << 16)) | (uint32_t(CH >> 3) << 17) | (uint32_t(128 >> 4) << 24);
+  static_assert(!FP8 || (D == 128 && !PAGED && NCH == 1), "e4m3 forward: head_dim 128, contiguous K/V");
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
   static_assert(2 * 128 + NQ * D <= 512, "TMEM budget");
 };
@@ -111,7 +120,8 @@ struct RowState {
 // S row (128 fp32 columns at t_s) -> masked online-softmax step -> P (bf16, written over
 // the first 64 columns of t_s). Returns the factor alpha by which O and l must be
 // multiplied (1 when the reference did not move); `need` tells whether it moved.
-template <int EMU>
+// FP8: P is written as e4m3, four per TMEM column (columns 0 .. 31), instead of bf16 pairs.
+template <int EMU, bool FP8 = false>
 __device__ __forceinline__ float softmax_tile(uint32_t t_s, int mi, const uint4& bits, float sl2, RowState& st,
                                               bool& need) {
   float s[128];
@@ -152,9 +162,11 @@ __device__ __forceinline__ float softmax_tile(uint32_t t_s, int mi, const uint4&
   const float mref = st.m_run == -INFINITY ? 0.f : st.m_run;
   const uint64_t sl2x2 = pk2(sl2, sl2), nm2 = pk2(-mref, -mref);
   uint64_t lsum2[4] = {pk2(0.f, 0.f), pk2(0.f, 0.f), pk2(0.f, 0.f), pk2(0.f, 0.f)};  // 4 independent sums
+  uint32_t p8[FP8 ? 32 : 1];
 #pragma unroll
   for (int cc = 0; cc < 4; ++cc) {
     uint32_t pk[16];
+    float pf[FP8 ? 32 : 1];
 #pragma unroll
     for (int e = 0; e < 16; ++e) {
       float x0, x1;
@@ -168,10 +180,21 @@ __device__ __forceinline__ float softmax_tile(uint32_t t_s, int mi, const uint4&
       lsum2[e & 3] = fadd2(lsum2[e & 3], p01);
       float p0, p1;
       unpk2(p01, p0, p1);
-      pk[e] = pack_bf16(p0, p1);
+      if constexpr (FP8) {
+        pf[2 * e] = p0;
+        pf[2 * e + 1] = p1;
+      } else {
+        pk[e] = pack_bf16(p0, p1);
+      }
     }
-    tmem_st32x16(t_s + cc * 16, pk);
+    if constexpr (FP8) {
+#pragma unroll
+      for (int w = 0; w < 8; ++w) p8[cc * 8 + w] = pack_e4m3x4(pf[4 * w], pf[4 * w + 1], pf[4 * w + 2], pf[4 * w + 3]);
+    } else {
+      tmem_st32x16(t_s + cc * 16, pk);
+    }
   }
+  if constexpr (FP8) tmem_st32x32(t_s, p8);
   {
     float a, b;
     unpk2(fadd2(fadd2(lsum2[0], lsum2[1]), fadd2(lsum2[2], lsum2[3])), a, b);
@@ -202,9 +225,9 @@ __device__ __forceinline__ void rescale_o(uint32_t t_o, float alpha) {
 // the global stores are guarded by `valid`.
 template <int D>
 __device__ __forceinline__ void store_row(uint32_t t_o, const RowState& st, bool valid, int64_t row,
-                                          __nv_bfloat16* out, float* lse) {
+                                          __nv_bfloat16* out, float* lse, float oscale = 1.f) {
   const bool seen = st.m_run != -INFINITY;
-  const float inv = seen ? 1.f / st.l_run : 0.f;
+  const float inv = seen ? oscale / st.l_run : 0.f;
 #pragma unroll 1
   for (int cc = 0; cc < D / 32; ++cc) {
     uint32_t o[32];
@@ -229,9 +252,9 @@ __device__ __forceinline__ void store_row(uint32_t t_o, const RowState& st, bool
 // (natural log), into partial slot row `srow`; merged later by merge_partials_kernel.
 template <int D>
 __device__ __forceinline__ void store_partial(uint32_t t_o, const RowState& st, bool valid, int64_t srow, float* po,
-                                              float* plse) {
+                                              float* plse, float oscale = 1.f) {
   const bool seen = st.m_run != -INFINITY;
-  const float inv = seen ? 1.f / st.l_run : 0.f;
+  const float inv = seen ? oscale / st.l_run : 0.f;
 #pragma unroll 1
   for (int cc = 0; cc < D / 32; ++cc) {
     uint32_t o[32];
@@ -322,8 +345,8 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_fwd_kernel(const __
           for (int t = 0; t < C::NQ; ++t)
             for (int hh = 0; hh < p.hp; ++hh)
               for (int c = 0; c < C::QBOX; ++c)
-                tma_load_3d(sbase + C::OFF_Q + t * C::Q_BYTES + c * C::BOX_BYTES + hh * p.R * 128, &p.tm_q, c * 64,
-                            it.head[t] + hh, it.tok[t], BAR(C::B_QFULL));
+                tma_load_3d(sbase + C::OFF_Q + t * C::Q_BYTES + c * C::BOX_BYTES + hh * p.R * 128, &p.tm_q,
+                            c * C::BOX_COLS, it.head[t] + hh, it.tok[t], BAR(C::B_QFULL));
         }
         const int T = C::NQ * it.job_count;
         auto load_tile = [&](bool is_v, int j) -> bool {
@@ -335,9 +358,13 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_fwd_kernel(const __
               return false;
             mbar_expect_tx(BAR(C::B_KVFULL + slot), C::CHUNK_BYTES);
             const uint32_t dst = sbase + C::OFF_RING + slot * C::CHUNK_BYTES;
-            if constexpr (!C::PAGED) {
+            if constexpr (C::FP8) {
+              // K: 128 keys x 128 bytes; V^T ([Hkv][d][keys]): d = 128 rows x 128 keys
+              if (is_v) tma_load_3d(dst, tm, it.vt_base + kt * 128, 0, it.kv_head, BAR(C::B_KVFULL + slot));
+              else tma_load_3d(dst, tm, 0, it.kv_head, it.k_base + kt * 128, BAR(C::B_KVFULL + slot));
+            } else if constexpr (!C::PAGED) {
               for (int c = 0; c < C::NBOX; ++c)
-                tma_load_3d(dst + c * C::BOX_BYTES, tm, h * C::CH + c * 64, it.kv_head, it.k_base + kt * 128,
+                tma_load_3d(dst + c * C::BOX_BYTES, tm, h * C::CH + c * C::BOX_COLS, it.kv_head, it.k_base + kt * 128,
                             BAR(C::B_KVFULL + slot));
             } else {
               const int ps = p.page_size, ppt = 128 / ps;
@@ -360,7 +387,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_fwd_kernel(const __
                 int32_t row = p.num_pages * ps;  // fully out of bounds: the box reads zeros
                 if (page[pg] >= 0 && page[pg] < p.num_pages) row = page[pg] * ps;
                 for (int c = 0; c < C::NBOX; ++c)
-                  tma_load_3d(dst + c * C::BOX_BYTES + pg * ps * 128, tm, h * C::CH + c * 64, it.kv_head, row,
+                  tma_load_3d(dst + c * C::BOX_BYTES + pg * ps * 128, tm, h * C::CH + c * C::BOX_COLS, it.kv_head, row,
                               BAR(C::B_KVFULL + slot));
               }
             }
@@ -410,7 +437,8 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_fwd_kernel(const __
 #pragma unroll
           for (int h = 0; h < C::NCH; ++h) {
             const uint32_t klo = desc_lo(sbase + C::OFF_RING + ((rk + h) % C::STAGES) * C::CHUNK_BYTES, 16);
-            if constexpr (C::D == 128) mma_ss_x8_k128(d_s, desc_of(qlo), desc_of(klo), C::IDESC_QK, 0u);
+            if constexpr (C::FP8) mma8_ss_x4_k128(d_s, desc_of(qlo), desc_of(klo), C::IDESC_QK, 0u);
+            else if constexpr (C::D == 128) mma_ss_x8_k128(d_s, desc_of(qlo), desc_of(klo), C::IDESC_QK, 0u);
             else mma_ss_x4_k64(d_s, desc_of(qlo), desc_of(klo), C::IDESC_QK, 0u);
             // the chunk is free once these MMAs complete (commit tracks all earlier MMAs)
             if (q == C::NQ - 1) mma_commit(BAR(C::B_KVEMPTY + (rk + h) % C::STAGES));
@@ -434,9 +462,10 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_fwd_kernel(const __
           const uint32_t first = u < C::NQ ? 1u : 0u;
 #pragma unroll
           for (int h = 0; h < C::NCH; ++h) {
-            const uint32_t vlo = desc_lo(sbase + C::OFF_RING + ((rv + h) % C::STAGES) * C::CHUNK_BYTES, C::BOX_BYTES);
+            const uint32_t vbase = sbase + C::OFF_RING + ((rv + h) % C::STAGES) * C::CHUNK_BYTES;
             const uint32_t d_o = tmem + C::TM_O + q * C::D + h * 128, a_p = tmem + 128 * slot;
-            mma_ts_x8(d_o, a_p, desc_of(vlo), C::IDESC_PV, first ^ 1u);
+            if constexpr (C::FP8) mma8_ts_x4_k128(d_o, a_p, desc_of(desc_lo(vbase, 16)), C::IDESC_PV, first ^ 1u);
+            else mma_ts_x8(d_o, a_p, desc_of(desc_lo(vbase, C::BOX_BYTES)), C::IDESC_PV, first ^ 1u);
             if (q == C::NQ - 1) mma_commit(BAR(C::B_KVEMPTY + (rv + h) % C::STAGES));
           }
           mma_commit(BAR(C::B_PVDONE + q));
@@ -483,7 +512,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_fwd_kernel(const __
         }
         tc_fence_after();
         bool need;
-        const float alpha = softmax_tile<C::EMU>(tmem + lane_base + 128 * slot, mi, bits, sl2, st, need);
+        const float alpha = softmax_tile<C::EMU, C::FP8>(tmem + lane_base + 128 * slot, mi, bits, sl2, st, need);
         if (t >= C::NQ) {
           // the previous P V of this tile must be done before O is touched or P is published
           if (!__all_sync(0xffffffffu, wait_bounded(BAR(C::B_PVDONE + q), pvc & 1, guard, kWaitPvDone))) {
@@ -504,9 +533,11 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_fwd_kernel(const __
       tc_fence_after();
       const int lr = r % p.R, hh = r / p.R;
       if (it.part < 0)
-        store_row<C::D>(t_o, st, lr < it.rows[q], int64_t(it.tok[q] + lr) * p.hq + it.head[q] + hh, p.out, p.lse);
+        store_row<C::D>(t_o, st, lr < it.rows[q], int64_t(it.tok[q] + lr) * p.hq + it.head[q] + hh, p.out, p.lse,
+                        p.v_scale);
       else
-        store_partial<C::D>(t_o, st, lr < it.rows[q], int64_t(it.part + q) * kSlotRows + r, p.part_o, p.part_lse);
+        store_partial<C::D>(t_o, st, lr < it.rows[q], int64_t(it.part + q) * kSlotRows + r, p.part_o, p.part_lse,
+                            p.v_scale);
       tc_fence_before();
       mbar_arrive(BAR(C::B_OEMPTY + q));
       sj += T;
@@ -907,28 +938,20 @@ attn_status_t launch_pair(const attn_plan_t* plan, Params& p, cudaStream_t strea
 }  // namespace
 }  // namespace mfa
 
-attn_status_t mfa_launch_forward(const attn_plan_t* plan, const void* q, const void* k, const void* v, void* out,
-                                 float* lse, cudaStream_t stream) {
-  using namespace mfa;
-  const int D = plan->d;
-  if (plan->total_kv_rows == 0) {
-    // no key anywhere: every row is fully masked
-    cudaError_t e = cudaMemsetAsync(out, 0, size_t(plan->total_q) * plan->hq * D * 2, stream);
-    if (e == cudaSuccess && lse) {
-      fill_empty_kernel<<<148, 256, 0, stream>>>(lse, plan->total_q * plan->hq);
-      e = cudaGetLastError();
-    }
-    return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+namespace {
+
+// out = 0 and lse = -inf everywhere: a problem without any key.
+attn_status_t forward_no_keys(const attn_plan_t* plan, void* out, float* lse, cudaStream_t stream) {
+  cudaError_t e = cudaMemsetAsync(out, 0, size_t(plan->total_q) * plan->hq * plan->d * 2, stream);
+  if (e == cudaSuccess && lse) {
+    mfa::fill_empty_kernel<<<148, 256, 0, stream>>>(lse, plan->total_q * plan->hq);
+    e = cudaGetLastError();
   }
-  Params p{};
-  // rows per K / V box: a page, a whole 128-key tile, or (pair kernel) a 64-key half tile
-  const uint32_t ps = uint32_t(plan->page_size);
-  uint32_t k_box = plan->paged ? ps : 128u, v_box = k_box;
-  if (plan->cluster == 2) k_box = k_box < 64u ? k_box : 64u;
-  if (!encode3d(&p.tm_q, q, D, plan->hq, plan->total_q, uint32_t(plan->R)) ||
-      !encode3d(&p.tm_k, k, D, plan->hkv, plan->total_kv_rows, k_box) ||
-      !encode3d(&p.tm_v, v, D, plan->hkv, plan->total_kv_rows, v_box))
-    return ATTN_ERR_CUDA;
+  return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+// The plan's work list, masks and partial slots, the outputs and the scalars into Params.
+void plan_params(const attn_plan_t* plan, void* out, float* lse, mfa::Params& p) {
   p.items = plan->d_items;
   p.jobs = plan->d_jobs;
   p.cta_off = plan->d_cta_off;
@@ -947,7 +970,38 @@ attn_status_t mfa_launch_forward(const attn_plan_t* plan, const void* q, const v
   p.num_pages = plan->num_pages;
   p.debug_flags = plan->debug_flags;
   p.scale_log2 = plan->scale * 1.4426950408889634f;
+  p.v_scale = 1.f;
   p.timeout_ns = plan->timeout_ns;
+}
+
+// Split-KV: merge the partial results of the split query tiles (after the forward kernel).
+attn_status_t merge_if_split(const attn_plan_t* plan, void* out, float* lse, cudaStream_t stream) {
+  using namespace mfa;
+  if (plan->n_merge == 0) return ATTN_OK;
+  const dim3 grid(plan->n_merge, kSlotRows / kMergeRowsPerBlock);
+  merge_partials_kernel<<<grid, 32 * kMergeRowsPerBlock, 0, stream>>>(plan->d_merge, plan->d_part_o, plan->d_part_lse,
+                                                                     plan->d, plan->R, plan->hq,
+                                                                     static_cast<__nv_bfloat16*>(out), lse);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+}  // namespace
+
+attn_status_t mfa_launch_forward(const attn_plan_t* plan, const void* q, const void* k, const void* v, void* out,
+                                 float* lse, cudaStream_t stream) {
+  using namespace mfa;
+  const int D = plan->d;
+  if (plan->total_kv_rows == 0) return forward_no_keys(plan, out, lse, stream);
+  Params p{};
+  // rows per K / V box: a page, a whole 128-key tile, or (pair kernel) a 64-key half tile
+  const uint32_t ps = uint32_t(plan->page_size);
+  uint32_t k_box = plan->paged ? ps : 128u, v_box = k_box;
+  if (plan->cluster == 2) k_box = k_box < 64u ? k_box : 64u;
+  if (!encode3d(&p.tm_q, q, D, plan->hq, plan->total_q, uint32_t(plan->R)) ||
+      !encode3d(&p.tm_k, k, D, plan->hkv, plan->total_kv_rows, k_box) ||
+      !encode3d(&p.tm_v, v, D, plan->hkv, plan->total_kv_rows, v_box))
+    return ATTN_ERR_CUDA;
+  plan_params(plan, out, lse, p);
   attn_status_t st;
   if (D == 64) {
     st = plan->paged ? launch<Cfg<64, 2, 10, true, MFA_EMU_D128>>(plan, p, stream)
@@ -959,10 +1013,70 @@ attn_status_t mfa_launch_forward(const attn_plan_t* plan, const void* q, const v
     st = plan->paged ? launch_pair<PairCfg<256, 5, true>>(plan, p, stream)
                      : launch_pair<PairCfg<256, 5, false>>(plan, p, stream);
   }
-  if (st != ATTN_OK || plan->n_merge == 0) return st;
-  const dim3 grid(plan->n_merge, kSlotRows / kMergeRowsPerBlock);
-  merge_partials_kernel<<<grid, 32 * kMergeRowsPerBlock, 0, stream>>>(plan->d_merge, plan->d_part_o, plan->d_part_lse,
-                                                                     D, plan->R, plan->hq, p.out, lse);
+  return st != ATTN_OK ? st : merge_if_split(plan, out, lse, stream);
+}
+
+// e4m3 forward (head_dim 128, contiguous K/V, single-CTA kernel): q, k bytes
+// [rows][heads][128]; vt bytes [Hkv][128][ldv] (V transposed per head); the scores are
+// scale * q_scale * k_scale * (q8 . k8), the output v_scale * (P8 . vt8) / l.
+attn_status_t mfa_launch_forward_fp8(const attn_plan_t* plan, const void* q, const void* k, const void* vt,
+                                     int64_t ldv, float q_scale, float k_scale, float v_scale, void* out, float* lse,
+                                     cudaStream_t stream) {
+  using namespace mfa;
+  if (plan->d != 128 || plan->paged || plan->cluster != 1) return ATTN_ERR_UNSUPPORTED;
+  if (plan->total_kv_rows == 0) return forward_no_keys(plan, out, lse, stream);
+  Params p{};
+  const uint64_t D = 128;
+  if (!encode3d_u8(&p.tm_q, q, D, plan->hq, plan->total_q, D, D * plan->hq, 128, 1, uint32_t(plan->R)) ||
+      !encode3d_u8(&p.tm_k, k, D, plan->hkv, plan->total_kv_rows, D, D * plan->hkv, 128, 1, 128) ||
+      !encode3d_u8(&p.tm_v, vt, uint64_t(plan->vt_keys), D, plan->hkv, uint64_t(ldv), uint64_t(ldv) * D, 128, 128, 1))
+    return ATTN_ERR_CUDA;
+  plan_params(plan, out, lse, p);
+  p.scale_log2 = plan->scale * q_scale * k_scale * 1.4426950408889634f;
+  p.v_scale = v_scale;
+  const attn_status_t st = launch<Cfg<128, 2, 10, false, 0, true>>(plan, p, stream);
+  return st != ATTN_OK ? st : merge_if_split(plan, out, lse, stream);
+}
+
+namespace mfa {
+namespace {
+// V [rows][Hkv][d] (bytes) -> V^T [Hkv][d][ldv] with sequence b's keys at columns
+// vt_off[b] .. (128-aligned starts) and zeros in the gaps; 32 x 32 byte tiles through
+// shared memory, one 32-column tile of one head per block.
+__global__ void transpose_v_kernel(const uint8_t* __restrict__ v, uint8_t* __restrict__ vt,
+                                   const int32_t* __restrict__ cu_k, const int32_t* __restrict__ vt_off, int batch,
+                                   int hkv, int d, int64_t ldv) {
+  __shared__ uint8_t tile[32][33];
+  const int c0 = blockIdx.x * 32;   // transposed column (padded key index)
+  const int d0 = blockIdx.y * 32, h = blockIdx.z;
+  const int tx = threadIdx.x, ty = threadIdx.y;
+  for (int i = ty; i < 32; i += 8) {
+    const int c = c0 + i;
+    int lo = 0, hi = batch;   // the sequence b with vt_off[b] <= c < vt_off[b + 1]
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) / 2;
+      if (vt_off[mid] <= c) lo = mid;
+      else hi = mid;
+    }
+    const int local = c - vt_off[lo];
+    const int64_t row = int64_t(cu_k[lo]) + local;
+    tile[i][tx] = (c < vt_off[batch] && row < cu_k[lo + 1]) ? v[(row * hkv + h) * d + d0 + tx] : uint8_t(0);
+  }
+  __syncthreads();
+  for (int i = ty; i < 32; i += 8) {
+    const int c = c0 + tx;
+    if (c < vt_off[batch]) vt[(int64_t(h) * d + d0 + i) * ldv + c] = tile[tx][i];
+  }
+}
+}  // namespace
+}  // namespace mfa
+
+attn_status_t mfa_transpose_v(const attn_plan_t* plan, const void* v, void* vt, int64_t ldv, cudaStream_t stream) {
+  if (plan->vt_keys == 0 || plan->batch == 0) return ATTN_OK;
+  const dim3 grid(uint32_t((plan->vt_keys + 31) / 32), uint32_t(plan->d / 32), uint32_t(plan->hkv)), block(32, 8);
+  mfa::transpose_v_kernel<<<grid, block, 0, stream>>>(static_cast<const uint8_t*>(v), static_cast<uint8_t*>(vt),
+                                                      plan->d_cu_k, plan->d_vt_off, plan->batch, plan->hkv, plan->d,
+                                                      ldv);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 

@@ -34,6 +34,8 @@ struct alignas(16) WorkItem {
   int32_t job_count;
   int32_t npages;      // paged: pages that hold the sequence's keys
   int32_t part;        // -1: write out / lse; else query tile t writes partial slot part + t
+  int32_t vt_base;     // contiguous: first column of the sequence in a transposed V (128-aligned)
+  int32_t pad;
 };
 static_assert(sizeof(WorkItem) == 64, "WorkItem layout");
 
@@ -126,6 +128,10 @@ struct attn_plan {
   const int32_t* d_cta_off = nullptr;
   const int32_t* d_cta_items = nullptr;
   const uint4* d_mask_tiles = nullptr;
+  // contiguous K/V: per sequence [B + 1] key offsets and 128-aligned transposed-V column offsets
+  const int32_t* d_cu_k = nullptr;
+  const int32_t* d_vt_off = nullptr;
+  int64_t vt_keys = 0;
   // split-KV: partial slots and the tiles to merge (none when nothing was split)
   float* d_part_o = nullptr;
   float* d_part_lse = nullptr;
@@ -165,6 +171,12 @@ attn_status_t mfa_plan_host(const attn_problem_t* problem, const attn_mask_desc_
 // forward launcher (attn_fwd.cu)
 attn_status_t mfa_launch_forward(const attn_plan_t* plan, const void* q, const void* k, const void* v,
                                  void* out, float* lse, cudaStream_t stream);
+
+// e4m3 forward and the V transpose it reads (attn_fwd.cu)
+attn_status_t mfa_launch_forward_fp8(const attn_plan_t* plan, const void* q, const void* k, const void* vt,
+                                     int64_t ldv, float q_scale, float k_scale, float v_scale, void* out, float* lse,
+                                     cudaStream_t stream);
+attn_status_t mfa_transpose_v(const attn_plan_t* plan, const void* v, void* vt, int64_t ldv, cudaStream_t stream);
 
 // backward launcher (attn_bwd.cu)
 attn_status_t mfa_launch_backward(const attn_plan_t* plan, const void* q, const void* k, const void* v,

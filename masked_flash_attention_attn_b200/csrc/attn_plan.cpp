@@ -494,10 +494,19 @@ void split_items(const Shape& s, int units, int nq, WorkList& wl) {
   wl.items.swap(out);
 }
 
+// Column of sequence b in a transposed V whose sequences start at multiples of 128 keys
+// (the e4m3 forward's TMA needs 16-byte aligned starts): offsets[B + 1].
+std::vector<int32_t> vt_offsets(const Shape& s) {
+  std::vector<int32_t> off(size_t(s.B) + 1, 0);
+  for (int b = 0; b < s.B; ++b) off[b + 1] = off[b] + (s.lk[b] + kTile - 1) / kTile * kTile;
+  return off;
+}
+
 void build_work(const Shape& s, int R, int hp, int nq, const std::vector<std::vector<int32_t>>& cnts,
                 int num_sms, WorkList& wl, bool allow_split = true) {
   const int g = s.hq / s.hkv;
   const int G = g / hp;  // head groups per kv head
+  const std::vector<int32_t> vt_off = vt_offsets(s);
   for (int b = 0; b < s.B; ++b) {
     const int lq = s.lq[b], lk = s.lk[b];
     if (lq == 0) continue;
@@ -524,6 +533,7 @@ void build_work(const Shape& s, int R, int hp, int nq, const std::vector<std::ve
     auto add_item = [&](int kh, int rb0, int hg0, int rb1, int hg1) {
       WorkItem it{};
       it.part = -1;
+      it.vt_base = s.paged ? 0 : vt_off[b];
       it.seq = b;
       it.kv_head = kh;
       it.k_base = s.koff[b];
@@ -626,17 +636,20 @@ void write_mask_tile(RowSource& src, const Shape& s, int R, const TileRef& t, ui
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 struct Staging {
-  size_t off_items, off_jobs, off_cta_off, off_cta_items, off_tiles, off_merge, off_part_lse, off_part_o, total;
+  size_t off_items, off_jobs, off_cta_off, off_cta_items, off_seq, off_tiles, off_merge, off_part_lse, off_part_o,
+      total;
 };
 
-// [status | items | jobs | cta_off | cta_items | mask tiles | merge tiles | partial lse | partial out]
-Staging layout(const WorkList& wl, int d) {
+// [status | items | jobs | cta_off | cta_items | cu_k, vt_off | mask tiles | merge tiles |
+//  partial lse | partial out]
+Staging layout(const WorkList& wl, int d, int batch) {
   Staging st{};
   st.off_items = 256;
   st.off_jobs = align256(st.off_items + wl.items.size() * sizeof(WorkItem));
   st.off_cta_off = align256(st.off_jobs + wl.jobs.size() * sizeof(Job));
   st.off_cta_items = align256(st.off_cta_off + wl.cta_off.size() * sizeof(int32_t));
-  st.off_tiles = align256(st.off_cta_items + wl.cta_items.size() * sizeof(int32_t));
+  st.off_seq = align256(st.off_cta_items + wl.cta_items.size() * sizeof(int32_t));
+  st.off_tiles = align256(st.off_seq + 2 * (size_t(batch) + 1) * sizeof(int32_t));
   st.off_merge = align256(st.off_tiles + wl.mask_tiles.size() * size_t(kMaskTileBytes));
   st.off_part_lse = align256(st.off_merge + wl.merge.size() * sizeof(MergeTile));
   st.off_part_o = align256(st.off_part_lse + size_t(wl.slots) * kSlotRows * sizeof(float));
@@ -765,6 +778,7 @@ void work_stats(const attn_plan_t& m, const WorkList& wl, attn_plan_stats_t& st)
   st.cluster_size = m.cluster;
   st.kv_splits_max = wl.splits_max;
   st.merge_tiles = int32_t(wl.merge.size());
+  st.vt_keys = m.vt_keys;
 }
 
 // ---- backward planning ----------------------------------------------------------------
@@ -1025,14 +1039,23 @@ attn_status_t plan_impl(const attn_problem_t* problem, const attn_mask_desc_t* m
   WorkList wl;
   build_work(s, R, plan->hp, plan->nq, cnts, num_sms / plan->cluster, wl);
   plan->ctas = int32_t(wl.cta_off.size()) - 1;   // work units: CTAs, or CTA pairs
+  plan->vt_keys = s.paged ? 0 : vt_offsets(s)[s.B];
   work_stats(*plan, wl, plan->stats);
 
-  const Staging lay = layout(wl, s.d);
+  const Staging lay = layout(wl, s.d, s.B);
   std::vector<char> host(lay.off_tiles, 0);
   std::memcpy(host.data() + lay.off_items, wl.items.data(), wl.items.size() * sizeof(WorkItem));
   std::memcpy(host.data() + lay.off_jobs, wl.jobs.data(), wl.jobs.size() * sizeof(Job));
   std::memcpy(host.data() + lay.off_cta_off, wl.cta_off.data(), wl.cta_off.size() * sizeof(int32_t));
   std::memcpy(host.data() + lay.off_cta_items, wl.cta_items.data(), wl.cta_items.size() * sizeof(int32_t));
+  {
+    const std::vector<int32_t> vt_off = vt_offsets(s);
+    std::vector<int32_t> cu_k(size_t(s.B) + 1, 0);
+    for (int b = 0; b < s.B; ++b) cu_k[b + 1] = s.paged ? 0 : s.koff[b] + s.lk[b];
+    if (!s.paged && s.B > 0) cu_k[0] = s.koff[0];
+    std::memcpy(host.data() + lay.off_seq, cu_k.data(), cu_k.size() * sizeof(int32_t));
+    std::memcpy(host.data() + lay.off_seq + cu_k.size() * sizeof(int32_t), vt_off.data(), vt_off.size() * sizeof(int32_t));
+  }
   std::vector<uint32_t> tiles;
   if (mask->kind != ATTN_MASK_CUSTOM && !wl.mask_tiles.empty()) {
     tiles.resize(wl.mask_tiles.size() * (kMaskTileBytes / 4));
@@ -1059,6 +1082,8 @@ attn_status_t plan_impl(const attn_problem_t* problem, const attn_mask_desc_t* m
   plan->d_cta_off = reinterpret_cast<const int32_t*>(base + lay.off_cta_off);
   plan->d_cta_items = reinterpret_cast<const int32_t*>(base + lay.off_cta_items);
   plan->d_mask_tiles = reinterpret_cast<const uint4*>(base + lay.off_tiles);
+  plan->d_cu_k = reinterpret_cast<const int32_t*>(base + lay.off_seq);
+  plan->d_vt_off = plan->d_cu_k + (s.B + 1);
   if (!wl.merge.empty()) {
     plan->d_merge = reinterpret_cast<const MergeTile*>(base + lay.off_merge);
     plan->n_merge = int32_t(wl.merge.size());
@@ -1123,7 +1148,7 @@ attn_status_t mfa_plan_host(const attn_problem_t* problem, const attn_mask_desc_
     WorkList wl;
     build_work(s, R, m.hp, m.nq, cnts, num_sms / m.cluster, wl, /*allow_split=*/false);
     m.ctas = int32_t(wl.cta_off.size()) - 1;
-    const Staging lay = layout(wl, s.d);
+    const Staging lay = layout(wl, s.d, s.B);
     out->off_items = lay.off_items;
     out->off_jobs = lay.off_jobs;
     out->off_cta_off = lay.off_cta_off;
@@ -1179,6 +1204,7 @@ attn_status_t attn_plan_dry_run(const attn_problem_t* problem, const attn_mask_d
     WorkList wl;
     build_work(s, m.R, m.hp, m.nq, cnts, num_sms / m.cluster, wl);
     m.ctas = int32_t(wl.cta_off.size()) - 1;
+    m.vt_keys = s.paged ? 0 : vt_offsets(s)[s.B];
     work_stats(m, wl, out);
     *stats = out;
     return ATTN_OK;
@@ -1215,6 +1241,29 @@ attn_status_t attn_masked_bwd(const attn_plan_t* plan, const void* q, const void
   for (const void* p : ptrs)
     if (!p || (reinterpret_cast<uintptr_t>(p) & 15u)) return ATTN_ERR_INVALID_ARG;
   return mfa_launch_backward(plan, q, k, v, out, lse, dout, dq, dk, dv, reinterpret_cast<cudaStream_t>(stream));
+}
+
+attn_status_t attn_fp8_transpose_v(const attn_plan_t* plan, const void* v, void* vt, int64_t ldv,
+                                   attn_stream_t stream) {
+  if (!plan || plan->paged || !v || !vt || ldv < plan->vt_keys || ldv % 16 != 0) return ATTN_ERR_INVALID_ARG;
+  if (plan->d % 32 != 0) return ATTN_ERR_UNSUPPORTED;
+  return mfa_transpose_v(plan, v, vt, ldv, reinterpret_cast<cudaStream_t>(stream));
+}
+
+attn_status_t attn_masked_fwd_fp8(const attn_plan_t* plan, const void* q, const void* k, const void* vt, int64_t ldv,
+                                  float q_scale, float k_scale, float v_scale, void* out, float* lse,
+                                  attn_stream_t stream) {
+  if (!plan) return ATTN_ERR_INVALID_ARG;
+  if (plan->d != 128 || plan->paged || plan->cluster != 1) return ATTN_ERR_UNSUPPORTED;
+  const void* ptrs[] = {q, k, vt, out};
+  for (const void* p : ptrs)
+    if (!p || (reinterpret_cast<uintptr_t>(p) & 15u)) return ATTN_ERR_INVALID_ARG;
+  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return ATTN_ERR_INVALID_ARG;
+  if (ldv < plan->vt_keys || ldv % 16 != 0) return ATTN_ERR_INVALID_ARG;
+  for (float x : {q_scale, k_scale, v_scale})
+    if (!(x > 0.f) || std::isinf(x)) return ATTN_ERR_INVALID_ARG;
+  return mfa_launch_forward_fp8(plan, q, k, vt, ldv, q_scale, k_scale, v_scale, out, lse,
+                                reinterpret_cast<cudaStream_t>(stream));
 }
 
 attn_status_t attn_masked_fwd(const attn_plan_t* plan, const void* q, const void* k, const void* v, void* out,

@@ -291,6 +291,15 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
   return d;
 }
 
+// Four fp32 -> four e4m3 in one word (round to nearest even, saturating at +-448); `a0` in
+// the lowest byte (the lowest key index). cvt's first source lands in the upper byte.
+__device__ __forceinline__ uint32_t pack_e4m3x4(float a0, float a1, float a2, float a3) {
+  uint16_t lo, hi;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(lo) : "f"(a1), "f"(a0));
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(hi) : "f"(a3), "f"(a2));
+  return uint32_t(lo) | (uint32_t(hi) << 16);
+}
+
 // Two fp32 -> one bf16x2 word (round to nearest even); `lo` lands in the low half, which
 // is the lower column / key index in every layout used here.
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
@@ -313,6 +322,21 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
       fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
   });
   return fn;
+}
+
+// 3-D byte (e4m3) tensor map: dims d0 (contiguous) x d1 x d2, row strides s1 / s2 bytes
+// (multiples of 16), boxes {b0, b1, b2} with the 128-byte swizzle (b0 = 128).
+bool encode3d_u8(CUtensorMap* tm, const void* ptr, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t s1, uint64_t s2,
+                 uint32_t b0, uint32_t b1, uint32_t b2) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {d0, d1, d2};
+  const cuuint64_t strides[2] = {s1, s2};
+  const cuuint32_t box[3] = {b0, b1, b2};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 bool encode3d(CUtensorMap* tm, const void* ptr, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t box2) {

@@ -11,6 +11,7 @@ Contents
   attention.py  O = softmax(scale * Q K^T + mask) V and the row log-sum-exp, fp64
   backward.py   dQ, dK, dV of that forward for a given dO (chain rule through the row
                 softmax), fp64
+  fp8.py        e4m3 byte decoding (inputs of the fp8 forward)
 
 Every function is pinned by the CPU tests (tests/test_oracle_*.py) to facts
 the pages or the mathematics fix: the pages' worked chunk-causal example,
@@ -21,8 +22,9 @@ from .masks import (dense_mask_rows, dense_mask, unpack_rows, tile_classes, unma
                     CLASS_EMPTY, CLASS_FULL, CLASS_PARTIAL)
 from .attention import attention_one_head, masked_attention, sampled_attention
 from .backward import attention_backward_one_head, masked_attention_backward
+from .fp8 import decode_e4m3
 
 __all__ = ["dense_mask_rows", "dense_mask", "unpack_rows", "tile_classes", "unmasked_pairs",
            "CLASS_EMPTY", "CLASS_FULL", "CLASS_PARTIAL",
            "attention_one_head", "masked_attention", "sampled_attention",
-           "attention_backward_one_head", "masked_attention_backward"]
+           "attention_backward_one_head", "masked_attention_backward", "decode_e4m3"]

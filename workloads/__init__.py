@@ -132,6 +132,14 @@ def randn_bf16(gen: torch.Generator, *shape) -> torch.Tensor:
     return torch.randn(*shape, generator=gen, dtype=torch.float32).to(torch.bfloat16)
 
 
+def quantize_e4m3(t: torch.Tensor):
+    """Per-tensor e4m3 quantisation of an input: scale = max |t| / 448 and the e4m3 bytes of
+    t / scale (the library's round-to-nearest-even conversion), as a uint8 tensor."""
+    amax = float(t.float().abs().max()) if t.numel() else 0.0
+    scale = amax / 448.0 if amax > 0 else 1.0
+    return (t.float() / scale).to(torch.float8_e4m3fn).view(torch.uint8), scale
+
+
 def pack_rows(dense: np.ndarray) -> np.ndarray:
     """Pack a bool [rows, L_k] array into uint32 words, LSB = lowest key."""
     rows, lk = dense.shape
