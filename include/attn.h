@@ -141,6 +141,13 @@ typedef struct {
                                        per-CTA share of the work (few long items: short queries over
                                        long keys, the tree-verify case of "Custom mask slows down
                                        attention."). Must be >= 0. */
+  int32_t q_begin, q_end;           /* query-row shard: this plan computes only the 128 / heads_per_tile row
+                                       blocks of every sequence that overlap sequence-local rows
+                                       [q_begin, q_end) (q_end <= 0: to the end). Rows of those blocks are
+                                       written in full; other rows are left untouched. Masks keep their
+                                       sequence-local row indices. For one long sequence split over GPUs:
+                                       every rank holds all K/V (one all-gather) and its query rows.
+                                       0 / 0 = all rows. */
 } attn_problem_t;
 
 typedef struct attn_plan attn_plan_t; /* opaque */

@@ -55,7 +55,7 @@ class attn_problem_t(ctypes.Structure):
                 ("head_dim", ctypes.c_int32), ("scale", ctypes.c_float), ("cu_seqlens_q", ctypes.c_void_p),
                 ("cu_seqlens_k", ctypes.c_void_p), ("kv_lens", ctypes.c_void_p), ("page_table", ctypes.c_void_p),
                 ("page_size", ctypes.c_int32), ("max_pages_per_seq", ctypes.c_int32), ("num_pages", ctypes.c_int32),
-                ("kv_splits", ctypes.c_int32)]
+                ("kv_splits", ctypes.c_int32), ("q_begin", ctypes.c_int32), ("q_end", ctypes.c_int32)]
 
 
 class attn_plan_stats_t(ctypes.Structure):
@@ -143,12 +143,14 @@ class _Marshal:
 
 
 def _problem(m: _Marshal, *, hq, hkv, head_dim, cu_seqlens_q, cu_seqlens_k=None, kv_lens=None, page_table=None,
-             page_size=0, num_pages=0, scale=0.0, kv_splits=0):
+             page_size=0, num_pages=0, scale=0.0, kv_splits=0, q_rows=None):
     cq = np.asarray(cu_seqlens_q, dtype=np.int32)
     pr = attn_problem_t()
     pr.batch = len(cq) - 1
     pr.hq, pr.hkv, pr.head_dim, pr.scale = hq, hkv, head_dim, float(scale)
     pr.kv_splits = int(kv_splits)
+    if q_rows is not None:
+        pr.q_begin, pr.q_end = int(q_rows[0]), int(q_rows[1])
     pr.cu_seqlens_q = m.arr(cq, np.int32)
     pr.cu_seqlens_k = m.arr(cu_seqlens_k, np.int32)
     pr.kv_lens = m.arr(kv_lens, np.int32)
@@ -213,7 +215,7 @@ class Plan:
 
 def attn_plan(*, hq: int, hkv: int, head_dim: int, cu_seqlens_q, mask, cu_seqlens_k=None, kv_lens=None,
               page_table=None, page_size: int = 0, num_pages: int = 0, scale: float = 0.0, kv_splits: int = 0,
-              stream=None, backward: bool = False) -> Plan:
+              stream=None, backward: bool = False, q_rows=None) -> Plan:
     """attn_plan(): validate, classify tiles, build the work list. ``page_table`` is a device
     int32 tensor [batch, max_pages]; CUSTOM ``mask.bits`` may be host (numpy) or device words;
     ``kv_splits``: 0 automatic, 1 never, N >= 2 at most N key ranges per query tile."""
@@ -221,7 +223,7 @@ def attn_plan(*, hq: int, hkv: int, head_dim: int, cu_seqlens_q, mask, cu_seqlen
     m = _Marshal()
     pr = _problem(m, hq=hq, hkv=hkv, head_dim=head_dim, cu_seqlens_q=cu_seqlens_q, cu_seqlens_k=cu_seqlens_k,
                   kv_lens=kv_lens, page_table=page_table, page_size=page_size, num_pages=num_pages, scale=scale,
-                  kv_splits=kv_splits)
+                  kv_splits=kv_splits, q_rows=q_rows)
     dev_bits = None
     if mask.kind == "CUSTOM":
         b = mask.bits
@@ -285,11 +287,11 @@ def attn_plan_destroy(plan: Plan) -> None:
 
 def attn_plan_dry_run(*, hq: int, hkv: int, head_dim: int, cu_seqlens_q, mask, num_sms: int = 148,
                       cu_seqlens_k=None, kv_lens=None, page_size: int = 0, max_pages_per_seq: int = 0,
-                      num_pages: int = 0, kv_splits: int = 0) -> dict:
+                      num_pages: int = 0, kv_splits: int = 0, q_rows=None) -> dict:
     """Host-only attn_plan() (analytic kinds) for a GPU of ``num_sms`` SMs: the plan statistics."""
     m = _Marshal()
     pr = _problem(m, hq=hq, hkv=hkv, head_dim=head_dim, cu_seqlens_q=cu_seqlens_q, cu_seqlens_k=cu_seqlens_k,
-                  kv_lens=kv_lens, kv_splits=kv_splits)
+                  kv_lens=kv_lens, kv_splits=kv_splits, q_rows=q_rows)
     if kv_lens is not None:
         pr.page_size, pr.max_pages_per_seq, pr.num_pages = page_size, max_pages_per_seq, num_pages
     d = _mask_desc(m, mask)

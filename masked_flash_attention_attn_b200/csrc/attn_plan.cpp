@@ -56,6 +56,7 @@ struct Shape {
   std::vector<int32_t> lq, lk, qoff, koff;
   int64_t total_q = 0, total_kv_rows = 0;
   int kv_splits = 0;   // 0 automatic, 1 never, N >= 2 at most N key ranges per query tile
+  int q_begin = 0, q_end = INT32_MAX;   // query-row shard (sequence-local rows)
 };
 
 attn_status_t validate_problem(const attn_problem_t* p, Shape& s, bool need_device_ptrs = true) {
@@ -66,6 +67,9 @@ attn_status_t validate_problem(const attn_problem_t* p, Shape& s, bool need_devi
   if (std::isnan(p->scale) || std::isinf(p->scale)) return ATTN_ERR_INVALID_ARG;
   if (p->kv_splits < 0) return ATTN_ERR_INVALID_ARG;
   s.kv_splits = p->kv_splits;
+  if (p->q_begin < 0 || (p->q_end > 0 && p->q_end < p->q_begin)) return ATTN_ERR_INVALID_ARG;
+  s.q_begin = p->q_begin;
+  s.q_end = p->q_end > 0 ? p->q_end : INT32_MAX;
   s.B = p->batch;
   s.hq = p->hq;
   s.hkv = p->hkv;
@@ -562,14 +566,17 @@ void build_work(const Shape& s, int R, int hp, int nq, const std::vector<std::ve
       it.job_count = int32_t(wl.jobs.size()) - it.job_start;
       wl.items.push_back(it);
     };
+    // the row blocks this plan computes: those overlapping the query-row shard
+    const int rb0 = std::min(n_rb, s.q_begin / R);
+    const int rb1 = std::min<int64_t>(n_rb, (std::min<int64_t>(s.q_end, lq) + R - 1) / R);
     for (int kh = 0; kh < s.hkv; ++kh) {
       if (nq == 2 && G >= 2) {
-        for (int rb = 0; rb < n_rb; ++rb)
+        for (int rb = rb0; rb < rb1; ++rb)
           for (int hg = 0; hg < G; hg += 2) add_item(kh, rb, hg, hg + 1 < G ? rb : -1, hg + 1);
       } else if (nq == 2) {
-        for (int rb = 0; rb < n_rb; rb += 2) add_item(kh, rb, 0, rb + 1 < n_rb ? rb + 1 : -1, 0);
+        for (int rb = rb0; rb < rb1; rb += 2) add_item(kh, rb, 0, rb + 1 < rb1 ? rb + 1 : -1, 0);
       } else {
-        for (int rb = 0; rb < n_rb; ++rb)
+        for (int rb = rb0; rb < rb1; ++rb)
           for (int hg = 0; hg < G; ++hg) add_item(kh, rb, hg, -1, 0);
       }
     }

@@ -1,0 +1,42 @@
+"""One long sequence over several GPUs: query-row shards plus one K/V all-gather.
+
+Every rank computes a contiguous range of query rows of every sequence (attn_problem_t
+q_begin / q_end, whole row blocks) against all keys; K and V are sharded by rows across
+the ranks beforehand, so the exchange step is one all-gather that lands every rank's K/V
+rows in every GPU's own memory (NCCL over NVLink; no peer memory is read by a kernel).
+Outputs stay sharded by query rows. This module holds only the shard arithmetic and the
+torch.distributed plumbing; the attention itself runs in the library's kernels.
+"""
+from __future__ import annotations
+
+
+def query_shard(lq_max: int, rank: int, world: int, block: int = 128):
+    """Sequence-local rows [begin, end) of `rank`: equal whole blocks of `block` rows."""
+    if world <= 0 or not 0 <= rank < world:
+        raise ValueError("bad rank / world")
+    blocks = (lq_max + block - 1) // block
+    per = (blocks + world - 1) // world
+    begin = min(lq_max, rank * per * block)
+    end = min(lq_max, (rank + 1) * per * block)
+    return begin, end
+
+
+def row_shard(rows: int, rank: int, world: int):
+    """Rows [begin, end) of a row-sharded tensor (K or V) owned by `rank`: equal parts, the
+    last one shorter."""
+    per = (rows + world - 1) // world
+    return min(rows, rank * per), min(rows, (rank + 1) * per)
+
+
+def all_gather_rows(local, rows: int, group=None):
+    """All-gather a row-sharded tensor (this rank's rows from row_shard) into the full
+    [rows, ...] tensor on every rank: one all_gather_into_tensor over equal padded parts."""
+    import torch
+    import torch.distributed as dist
+    world = dist.get_world_size(group)
+    per = (rows + world - 1) // world
+    buf = torch.zeros((per,) + tuple(local.shape[1:]), dtype=local.dtype, device=local.device)
+    buf[:local.shape[0]] = local
+    out = torch.empty((per * world,) + tuple(local.shape[1:]), dtype=local.dtype, device=local.device)
+    dist.all_gather_into_tensor(out, buf, group=group)
+    return out[:rows]

@@ -1,0 +1,59 @@
+"""Host side of the long-sequence multi-GPU path: query shards partition the work exactly
+(attn_plan_dry_run), and the K/V all-gather of row shards over a world-size-2 gloo group
+rebuilds the full tensors on every rank."""
+import multiprocessing as mp
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import workloads as W
+from masked_flash_attention_attn_b200 import sharding as S
+
+
+def test_query_shards_partition_the_work(attn_lib):
+    M = attn_lib
+    wl = W.config(5)
+    spec = wl.masks[1]   # the range form (analytic: plannable on the host)
+    kw = dict(hq=wl.hq, hkv=wl.hkv, head_dim=wl.d, cu_seqlens_q=wl.cu_seqlens_q, cu_seqlens_k=wl.cu_seqlens_k,
+              mask=spec)
+    full = M.attn_plan_dry_run(**kw)
+    L = wl.lq(0)
+    for world in (2, 3, 8):
+        shards = [S.query_shard(L, r, world) for r in range(world)]
+        assert shards[0][0] == 0 and shards[-1][1] == L
+        assert all(a[1] == b[0] for a, b in zip(shards, shards[1:]))
+        st = [M.attn_plan_dry_run(q_rows=sh, **kw) for sh in shards]
+        assert sum(x["work_items"] for x in st) == full["work_items"]
+        assert sum(x["jobs"] for x in st) == full["jobs"]
+        jobs = [x["jobs"] for x in st]
+        assert max(jobs) <= 1.25 * (sum(jobs) / world)     # balanced for this mask
+
+
+def _gather_worker(rank, world, port, rows, q):
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        full = torch.arange(rows * 6, dtype=torch.float32).reshape(rows, 2, 3)
+        a, b = S.row_shard(rows, rank, world)
+        got = S.all_gather_rows(full[a:b].clone(), rows)
+        q.put((rank, bool(torch.equal(got, full))))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("rows", [10, 7])
+def test_all_gather_rows_gloo(rows):
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = 29650 + rows
+    procs = [ctx.Process(target=_gather_worker, args=(r, 2, port, rows, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = [q.get(timeout=120) for _ in procs]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert all(ok for _, ok in res)
