@@ -261,8 +261,8 @@ def run_ours(args, rank, world, local_rank):
     fp8 = args.dtype == "e4m3"
     if bwd and (wl.paged or wl.d > 128):
         raise SystemExit("--pass bwd: contiguous K/V and head_dim <= 128 only (workloads 1, 4, 5)")
-    if fp8 and (bwd or wl.paged or wl.d != 128):
-        raise SystemExit("--dtype e4m3: the forward with contiguous K/V and head_dim 128 (workloads 4, 5)")
+    if fp8 and (bwd or wl.paged or wl.d not in (128, 256)):
+        raise SystemExit("--dtype e4m3: the forward with contiguous K/V, head_dim 128 or 256 (workloads 2, 4, 5)")
     plans = [make_plan(M, wl, spec, dev, args.kv_splits, backward=bwd) for spec in wl.masks]
     stats = [M.attn_plan_get_stats(p) for p in plans]
     flops = [flops_of(s, wl) * (2.5 if bwd else 1.0) for s in stats]
@@ -466,7 +466,7 @@ def main():
     ap.add_argument("--pass", dest="pass_", choices=["fwd", "bwd"], default="fwd",
                     help="fwd: the forward (the benchmark metric); bwd: the backward pass (workloads 1, 4, 5)")
     ap.add_argument("--dtype", choices=["bf16", "e4m3"], default="bf16",
-                    help="e4m3: the fp8 forward (head_dim 128, contiguous K/V: workloads 4, 5)")
+                    help="e4m3: the fp8 forward (contiguous K/V, head_dim 128 or 256: workloads 2, 4, 5)")
     ap.add_argument("--kv-splits", type=int, default=0,
                     help="split-KV: 0 automatic, 1 never, N >= 2 at most N key ranges per query tile")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)

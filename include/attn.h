@@ -220,11 +220,11 @@ attn_status_t attn_masked_bwd(const attn_plan_t* plan, const void* q, const void
  * scale * q_scale * k_scale * (q8 . k8) are exact in fp32; P is rounded to e4m3 for the
  * P V product (the row sums use P before rounding); out (bf16) and lse (fp32) as in
  * attn_masked_fwd.
- *   q   bytes [total_q][hq][128]        k bytes [total_k][hkv][128]
- *   vt  bytes [hkv][128][ldv]           V transposed per head by attn_fp8_transpose_v
+ *   q   bytes [total_q][hq][d]          k bytes [total_k][hkv][d]      (d = head_dim)
+ *   vt  bytes [hkv][d][ldv]             V transposed per head by attn_fp8_transpose_v
  *   ldv >= stats.vt_keys, a multiple of 16
- * head_dim 128 and contiguous K/V only (else UNSUPPORTED); the plan is an ordinary
- * attn_plan() (split-KV applies). Pointers 16-byte aligned (lse: 4-byte, may be NULL).
+ * head_dim 128 (single-SM kernel) or 256 (2-SM kernel) and contiguous K/V only (else
+ * UNSUPPORTED); the plan is an ordinary attn_plan() (split-KV applies). Pointers 16-byte aligned (lse: 4-byte, may be NULL).
  * Allocates nothing. Errors: INVALID_ARG, UNSUPPORTED, CUDA. */
 attn_status_t attn_masked_fwd_fp8(const attn_plan_t* plan, const void* q, const void* k, const void* vt,
                                   int64_t ldv, float q_scale, float k_scale, float v_scale, void* out,

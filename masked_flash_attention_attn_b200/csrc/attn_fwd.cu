@@ -560,12 +560,18 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_fwd_kernel(const __
 // Both CTAs' TMA loads count on the leader's "full" barriers; the leader's commits arrive
 // on both CTAs' barriers; the softmax warpgroups of both CTAs arrive on the leader's "P
 // ready" and "O free" barriers. No TMA load multicasts.
-template <int D_, int STAGES_, bool PAGED_, int EMU_ = 0>
+// FP8_: e4m3 Q, K and V^T ([Hkv][d][keys]; each CTA reads the d / 2 rows of its V half),
+// .kind::f8f6f4 2-SM MMAs, P in e4m3.
+template <int D_, int STAGES_, bool PAGED_, int EMU_ = 0, bool FP8_ = false>
 struct PairCfg {
   static constexpr int D = D_, STAGES = STAGES_, EMU = EMU_;
   static constexpr bool PAGED = PAGED_;
-  static constexpr int QBOX = D / 64;              // 64-column boxes of a Q tile and of a K half
-  static constexpr int VBOX = D / 128;             // 64-column boxes of a V half (D / 2 columns)
+  static constexpr bool FP8 = FP8_;
+  static constexpr int BOX_COLS = FP8 ? 128 : 64;  // elements per 128-byte box row
+  static constexpr int QBOX = D / BOX_COLS;        // 128-byte boxes of a Q tile and of a K half
+  // boxes of a V half: bf16 d / 2 columns in 64-column boxes (MN-major); e4m3 one box of d / 2
+  // V^T rows x 128 keys (K-major)
+  static constexpr int VBOX = FP8 ? 1 : D / 128;
   static constexpr int Q_BYTES = QBOX * 128 * 128;
   static constexpr int KH_BOX = 64 * 128;          // 64 keys x 128 bytes
   static constexpr int VH_BOX = 128 * 128;         // 128 keys x 128 bytes
@@ -581,10 +587,12 @@ struct PairCfg {
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
   static constexpr int THREADS = 256;
   static constexpr int TM_O = 256;
-  static constexpr uint32_t IDESC_QK =  // M=256 (pair), N=128, bf16 -> fp32, both K-major
-      (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(128 >> 3) << 17) | (uint32_t(256 >> 4) << 24);
-  static constexpr uint32_t IDESC_PV =  // M=256, N=D, A (P) from TMEM, B (V) MN-major
-      (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) | (uint32_t(D >> 3) << 17) | (uint32_t(256 >> 4) << 24);
+  static constexpr uint32_t AB_TYPES = FP8 ? 0u : (1u << 7) | (1u << 10);   // bf16 (1) or e4m3 (0)
+  static constexpr uint32_t IDESC_QK =  // M=256 (pair), N=128, fp32 accumulate, both K-major
+      (1u << 4) | AB_TYPES | (uint32_t(128 >> 3) << 17) | (uint32_t(256 >> 4) << 24);
+  static constexpr uint32_t IDESC_PV =  // M=256, N=D, A (P) from TMEM; B: V MN-major (bf16), V^T K-major (e4m3)
+      (1u << 4) | AB_TYPES | (FP8 ? 0u : (1u << 16)) | (uint32_t(D >> 3) << 17) | (uint32_t(256 >> 4) << 24);
+  static_assert(!FP8 || (D == 256 && !PAGED), "e4m3 pair kernel: head_dim 256, contiguous K/V");
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
   static_assert(256 + D <= 512, "TMEM budget");
 };
@@ -651,8 +659,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::THREADS, 1)
           q_last = n;
           for (int hh = 0; hh < p.hp; ++hh)
             for (int c = 0; c < C::QBOX; ++c)
-              tma2_load_3d_hint(sbase + C::OFF_Q + c * 16384 + hh * p.R * 128, &p.tm_q, c * 64, it.head[rank] + hh,
-                                it.tok[rank], LBAR(C::B_QFULL), pol_q);
+              tma2_load_3d_hint(sbase + C::OFF_Q + c * 16384 + hh * p.R * 128, &p.tm_q, c * C::BOX_COLS,
+                                it.head[rank] + hh, it.tok[rank], LBAR(C::B_QFULL), pol_q);
         }
         const int T = it.job_count;
         auto load_half = [&](bool is_v, int j) -> bool {
@@ -670,9 +678,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::THREADS, 1)
           const int box_bytes = is_v ? C::VH_BOX : C::KH_BOX;
           const int col0 = is_v ? int(rank) * (C::D / 2) : 0;
           const CUtensorMap* tm = is_v ? &p.tm_v : &p.tm_k;
-          if constexpr (!C::PAGED) {
+          if constexpr (C::FP8) {
+            // K half: 64 keys x two 128-byte boxes; V^T half: d / 2 rows x 128 keys
+            if (is_v)
+              tma2_load_3d_hint(dst, tm, it.vt_base + kt * 128, int(rank) * (C::D / 2), it.kv_head, fb, pol_kv);
+            else
+              for (int c = 0; c < nbox; ++c)
+                tma2_load_3d_hint(dst + c * box_bytes, tm, c * C::BOX_COLS, it.kv_head, it.k_base + key0, fb, pol_kv);
+          } else if constexpr (!C::PAGED) {
             for (int c = 0; c < nbox; ++c)
-              tma2_load_3d_hint(dst + c * box_bytes, tm, col0 + c * 64, it.kv_head, it.k_base + key0, fb, pol_kv);
+              tma2_load_3d_hint(dst + c * box_bytes, tm, col0 + c * C::BOX_COLS, it.kv_head, it.k_base + key0, fb,
+                                pol_kv);
           } else {
             const int ps = p.page_size;
             const int rows = ps < nkeys ? ps : nkeys;  // rows per box
@@ -693,8 +709,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::THREADS, 1)
               int32_t row = p.num_pages * ps;  // fully out of bounds: the box reads zeros
               if (page[pg] >= 0 && page[pg] < p.num_pages) row = page[pg] * ps + (key0 + pg * rows) % ps;
               for (int c = 0; c < nbox; ++c)
-                tma2_load_3d_hint(dst + c * box_bytes + pg * rows * 128, tm, col0 + c * 64, it.kv_head, row, fb,
-                                  pol_kv);
+                tma2_load_3d_hint(dst + c * box_bytes + pg * rows * 128, tm, col0 + c * C::BOX_COLS, it.kv_head, row,
+                                  fb, pol_kv);
             }
           }
           ++rc;
@@ -736,7 +752,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::THREADS, 1)
           const uint32_t klo = desc_lo(sbase + C::OFF_RING + (rk % C::STAGES) * C::SLOT_BYTES, 16);
           const uint32_t d_s = tmem + 128 * slot;
           static_assert(C::D == 256, "pair kernel issue groups are laid out for head_dim 256");
-          mma2_ss_x16_k256(d_s, desc_of(qlo), desc_of(klo), C::IDESC_QK, 0u);
+          if constexpr (C::FP8) mma2_8_ss_x8_k256(d_s, desc_of(qlo), desc_of(klo), C::IDESC_QK, 0u);
+          else mma2_ss_x16_k256(d_s, desc_of(qlo), desc_of(klo), C::IDESC_QK, 0u);
           mma2_commit_both(BAR(C::B_KVEMPTY + rk % C::STAGES));
           mma2_commit_both(BAR(C::B_SFULL + slot));
           if (t == T - 1) mma2_commit_both(BAR(C::B_QEMPTY));
@@ -750,9 +767,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::THREADS, 1)
             return false;
           ++rc;
           tc_fence_after();
-          const uint32_t vlo = desc_lo(sbase + C::OFF_RING + (rv % C::STAGES) * C::SLOT_BYTES, C::VH_BOX);
+          const uint32_t vbase = sbase + C::OFF_RING + (rv % C::STAGES) * C::SLOT_BYTES;
           const uint32_t a_p = tmem + 128 * slot, acc0 = u == 0 ? 0u : 1u;
-          mma2_ts_x8(tmem + C::TM_O, a_p, desc_of(vlo), C::IDESC_PV, acc0);
+          if constexpr (C::FP8) mma2_8_ts_x4(tmem + C::TM_O, a_p, desc_of(desc_lo(vbase, 16)), C::IDESC_PV, acc0);
+          else mma2_ts_x8(tmem + C::TM_O, a_p, desc_of(desc_lo(vbase, C::VH_BOX)), C::IDESC_PV, acc0);
           mma2_commit_both(BAR(C::B_KVEMPTY + rv % C::STAGES));
           mma2_commit_both(BAR(C::B_PVDONE));
           return true;
@@ -794,7 +812,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::THREADS, 1)
         }
         tc_fence_after();
         bool need;
-        const float alpha = softmax_tile<C::EMU>(tmem + lane_base + 128 * slot, mi, bits, sl2, st, need);
+        const float alpha = softmax_tile<C::EMU, C::FP8>(tmem + lane_base + 128 * slot, mi, bits, sl2, st, need);
         if (t >= 1) {
           if (!__all_sync(0xffffffffu, wait_bounded(BAR(C::B_PVDONE), pvc & 1, guard, kWaitPvDone))) {
             ok = false;
@@ -814,10 +832,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::THREADS, 1)
       const int lr = r % p.R, hh = r / p.R;
       if (it.part < 0)
         store_row<C::D>(t_o, st, lr < it.rows[rank], int64_t(it.tok[rank] + lr) * p.hq + it.head[rank] + hh, p.out,
-                        p.lse);
+                        p.lse, p.v_scale);
       else
         store_partial<C::D>(t_o, st, lr < it.rows[rank], int64_t(it.part + int(rank)) * kSlotRows + r, p.part_o,
-                            p.part_lse);
+                            p.part_lse, p.v_scale);
       tc_fence_before();
       warp_arrive_leader(LBAR(C::B_OEMPTY));
       sj += T;
@@ -1023,18 +1041,23 @@ attn_status_t mfa_launch_forward_fp8(const attn_plan_t* plan, const void* q, con
                                      int64_t ldv, float q_scale, float k_scale, float v_scale, void* out, float* lse,
                                      cudaStream_t stream) {
   using namespace mfa;
-  if (plan->d != 128 || plan->paged || plan->cluster != 1) return ATTN_ERR_UNSUPPORTED;
+  const bool pair = plan->d == 256;
+  if ((plan->d != 128 && !pair) || plan->paged || plan->cluster != (pair ? 2 : 1)) return ATTN_ERR_UNSUPPORTED;
   if (plan->total_kv_rows == 0) return forward_no_keys(plan, out, lse, stream);
   Params p{};
-  const uint64_t D = 128;
+  const uint64_t D = uint64_t(plan->d);
+  // K boxes: a 128-key tile (single-CTA kernel) or a 64-key half (pair); V^T boxes: d or d / 2 rows
+  const uint32_t k_rows = pair ? 64u : 128u, vt_rows = uint32_t(pair ? D / 2 : D);
   if (!encode3d_u8(&p.tm_q, q, D, plan->hq, plan->total_q, D, D * plan->hq, 128, 1, uint32_t(plan->R)) ||
-      !encode3d_u8(&p.tm_k, k, D, plan->hkv, plan->total_kv_rows, D, D * plan->hkv, 128, 1, 128) ||
-      !encode3d_u8(&p.tm_v, vt, uint64_t(plan->vt_keys), D, plan->hkv, uint64_t(ldv), uint64_t(ldv) * D, 128, 128, 1))
+      !encode3d_u8(&p.tm_k, k, D, plan->hkv, plan->total_kv_rows, D, D * plan->hkv, 128, 1, k_rows) ||
+      !encode3d_u8(&p.tm_v, vt, uint64_t(plan->vt_keys), D, plan->hkv, uint64_t(ldv), uint64_t(ldv) * D, 128, vt_rows,
+                   1))
     return ATTN_ERR_CUDA;
   plan_params(plan, out, lse, p);
   p.scale_log2 = plan->scale * q_scale * k_scale * 1.4426950408889634f;
   p.v_scale = v_scale;
-  const attn_status_t st = launch<Cfg<128, 2, 10, false, 0, true>>(plan, p, stream);
+  const attn_status_t st = pair ? launch_pair<PairCfg<256, 10, false, 0, true>>(plan, p, stream)
+                                : launch<Cfg<128, 2, 10, false, 0, true>>(plan, p, stream);
   return st != ATTN_OK ? st : merge_if_split(plan, out, lse, stream);
 }
 

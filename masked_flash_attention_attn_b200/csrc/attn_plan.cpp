@@ -1261,7 +1261,7 @@ attn_status_t attn_masked_fwd_fp8(const attn_plan_t* plan, const void* q, const 
                                   float q_scale, float k_scale, float v_scale, void* out, float* lse,
                                   attn_stream_t stream) {
   if (!plan) return ATTN_ERR_INVALID_ARG;
-  if (plan->d != 128 || plan->paged || plan->cluster != 1) return ATTN_ERR_UNSUPPORTED;
+  if ((plan->d != 128 && plan->d != 256) || plan->paged) return ATTN_ERR_UNSUPPORTED;
   const void* ptrs[] = {q, k, vt, out};
   for (const void* p : ptrs)
     if (!p || (reinterpret_cast<uintptr_t>(p) & 15u)) return ATTN_ERR_INVALID_ARG;

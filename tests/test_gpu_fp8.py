@@ -87,23 +87,25 @@ def check_fp8(wl, spec, what, kv_splits=0):
     return float(err.max()), float(worst)
 
 
+@pytest.mark.parametrize("d", [128, 256])
 @pytest.mark.parametrize("kind", ["FULL", "CAUSAL", "SLIDING_WINDOW", "PREFIX_LM", "CHUNK_CAUSAL", "RANGES",
                                   "CUSTOM", "BLOCK_SPARSE"])
-def test_fp8_all_kinds(kind):
-    wl = W.random_small(seed=900 + len(kind), kind=kind, batch=3, hq=4, hkv=2, d=128, lmin=1, lmax=400)
-    check_fp8(wl, wl.masks[0], f"fp8 {kind}")
+def test_fp8_all_kinds(kind, d):
+    wl = W.random_small(seed=900 + len(kind) + d, kind=kind, batch=3, hq=4, hkv=2, d=d, lmin=1, lmax=400)
+    check_fp8(wl, wl.masks[0], f"fp8 {kind} d={d}")
 
 
-def test_fp8_short_queries_and_split():
-    # head packing (short queries) and split-KV partials go through the same e4m3 kernel
+@pytest.mark.parametrize("d", [128, 256])
+def test_fp8_short_queries_and_split(d):
+    # head packing (short queries) and split-KV partials go through the same e4m3 kernels
     rng = np.random.default_rng(8)
     lq = rng.integers(1, 33, size=4)
     lk = lq + rng.integers(500, 1500, size=4)
     gen = torch.Generator().manual_seed(8)
     cq, ck = W.cu_from_lengths(lq), W.cu_from_lengths(lk)
-    wl = W.Workload(name="fp8_short", hq=8, hkv=2, d=128, scale=0.088, cu_seqlens_q=cq,
-                    q=W.randn_bf16(gen, int(cq[-1]), 8, 128), masks=[W.MaskSpec("CAUSAL")], cu_seqlens_k=ck,
-                    k=W.randn_bf16(gen, int(ck[-1]), 2, 128), v=W.randn_bf16(gen, int(ck[-1]), 2, 128), seed=8)
+    wl = W.Workload(name="fp8_short", hq=8, hkv=2, d=d, scale=d ** -0.5, cu_seqlens_q=cq,
+                    q=W.randn_bf16(gen, int(cq[-1]), 8, d), masks=[W.MaskSpec("CAUSAL")], cu_seqlens_k=ck,
+                    k=W.randn_bf16(gen, int(ck[-1]), 2, d), v=W.randn_bf16(gen, int(ck[-1]), 2, d), seed=8)
     check_fp8(wl, wl.masks[0], "fp8 short q")
     check_fp8(wl, wl.masks[0], "fp8 short q split", kv_splits=4)
 
