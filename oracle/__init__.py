@@ -21,10 +21,10 @@ tiny inputs and the library softmax on unmasked rows.
 from .masks import (dense_mask_rows, dense_mask, unpack_rows, tile_classes, unmasked_pairs,
                     CLASS_EMPTY, CLASS_FULL, CLASS_PARTIAL)
 from .attention import attention_one_head, masked_attention, sampled_attention
-from .backward import attention_backward_one_head, masked_attention_backward
+from .backward import attention_backward_one_head, masked_attention_backward, sampled_backward
 from .fp8 import decode_e4m3
 
 __all__ = ["dense_mask_rows", "dense_mask", "unpack_rows", "tile_classes", "unmasked_pairs",
            "CLASS_EMPTY", "CLASS_FULL", "CLASS_PARTIAL",
            "attention_one_head", "masked_attention", "sampled_attention",
-           "attention_backward_one_head", "masked_attention_backward", "decode_e4m3"]
+           "attention_backward_one_head", "masked_attention_backward", "sampled_backward", "decode_e4m3"]

@@ -25,7 +25,7 @@ from __future__ import annotations
 import numpy as np
 
 from .attention import attention_one_head, _f64
-from .masks import dense_mask
+from .masks import dense_mask, dense_mask_rows
 
 
 def attention_backward_one_head(q, k, v, mask, scale, dout):
@@ -70,4 +70,54 @@ def masked_attention_backward(wl, spec, dout):
             dq[q0:q0 + lq, h] = a
             dk[k0:k0 + lk, kh] += bk
             dv[k0:k0 + lk, kh] += bv
+    return dq, dk, dv
+
+
+def sampled_backward(wl, spec, dout, q_samples, k_samples, row_block: int = 1024):
+    """Gradients at sampled places of a contiguous workload, for full-size problems.
+
+    q_samples: (b, h, i) -> dq[token of row i of sequence b, h]
+    k_samples: (b, kh, j) -> dk, dv[key j of sequence b, kh] (summed over kh's query heads)
+    Every value follows the definitions of this module; a dq row needs its own row of p and
+    dp, a dk / dv row needs column j of p and ds over every query row of every query head
+    of kh (computed in blocks of rows). Returns (dq [n_q, d], dk [n_k, d], dv [n_k, d])."""
+    import torch
+    dout = dout.to(torch.float64).numpy() if hasattr(dout, "numpy") else np.asarray(dout, np.float64)
+    g = wl.hq // wl.hkv
+    dq = np.zeros((len(q_samples), wl.d))
+    for n, (b, h, i) in enumerate(q_samples):
+        lq, lk = wl.lq(b), wl.lk(b)
+        q0, k0 = int(wl.cu_seqlens_q[b]), int(wl.cu_seqlens_k[b])
+        kk, vv = (_f64(t) for t in wl.kv_of_seq(b))
+        m = dense_mask_rows(spec, b, lq, lk, i, i + 1)
+        a, _, _ = attention_backward_one_head(_f64(wl.q[q0 + i:q0 + i + 1, h]), kk[:, h // g], vv[:, h // g], m,
+                                              wl.scale, dout[q0 + i:q0 + i + 1, h])
+        dq[n] = a[0]
+    dk = np.zeros((len(k_samples), wl.d))
+    dv = np.zeros((len(k_samples), wl.d))
+    by_seq_head = {}
+    for n, (b, kh, j) in enumerate(k_samples):
+        by_seq_head.setdefault((b, kh), []).append((n, j))
+    for (b, kh), lst in by_seq_head.items():
+        lq, lk = wl.lq(b), wl.lk(b)
+        q0 = int(wl.cu_seqlens_q[b])
+        kk, vv = (_f64(t) for t in wl.kv_of_seq(b))
+        kk, vv = kk[:, kh], vv[:, kh]
+        cols = np.array([j for _, j in lst])
+        for h in range(kh * g, (kh + 1) * g):
+            for r0 in range(0, lq, row_block):
+                r1 = min(lq, r0 + row_block)
+                m = dense_mask_rows(spec, b, lq, lk, r0, r1)
+                q = _f64(wl.q[q0 + r0:q0 + r1, h])
+                do = dout[q0 + r0:q0 + r1, h]
+                out, lse = attention_one_head(q, kk, vv, m, wl.scale)
+                has = np.isfinite(lse)
+                s = wl.scale * (q @ kk[cols].T)                       # rows x sampled keys
+                mc = m[:, cols] & has[:, None]
+                p = np.where(mc, np.exp(np.where(mc, s, 0.0) - np.where(has, lse, 0.0)[:, None]), 0.0)
+                big_d = np.sum(do * out, axis=1)                      # D_i = dout_i . out_i
+                ds = p * (do @ vv[cols].T - big_d[:, None])
+                for c, (n, _) in enumerate(lst):
+                    dk[n] += wl.scale * ds[:, c] @ q
+                    dv[n] += p[:, c] @ do
     return dq, dk, dv

@@ -101,3 +101,37 @@ def test_backward_plan_required_and_unsupported():
         G.M.attn_plan(hq=2, hkv=1, head_dim=256, cu_seqlens_q=wl.cu_seqlens_q, cu_seqlens_k=wl.cu_seqlens_k,
                       mask=wl.masks[0], backward=True)
     assert e.value.status == 2
+
+
+def test_backward_full_size_chunk_causal_sampled():
+    """The chunk-causal workload at full size (8 x 8192 tokens, 16 heads, d=128), both
+    descriptor forms: dq on sampled rows (first / middle / last rows of every sequence and
+    random ones) and dk, dv on sampled keys of two (sequence, head) pairs, against the oracle
+    evaluated at those places; the two descriptor forms give identical gradients."""
+    wl = W.config(4)
+    q, k, v = G.device_inputs(wl)
+    gen = torch.Generator().manual_seed(44)
+    dout_h = W.randn_bf16(gen, q.shape[0], wl.hq, wl.d)
+    dout = dout_h.cuda()
+    rng = np.random.default_rng(44)
+    qs = G.sample_rows(wl, 40, seed=44)
+    ks = [(b, int(rng.integers(0, wl.hkv)), int(j)) for b in (0, 5) for j in
+          list(rng.integers(0, wl.lk(b), size=6)) + [0, wl.lk(b) - 1, 4095, 4096]]
+    grads = []
+    for spec in wl.masks:
+        plan = G.M.attn_plan(hq=wl.hq, hkv=wl.hkv, head_dim=wl.d, cu_seqlens_q=wl.cu_seqlens_q,
+                             cu_seqlens_k=wl.cu_seqlens_k, mask=spec, scale=wl.scale, backward=True)
+        out, lse = G.M.forward(plan, q, k, v)
+        dq, dk, dv = G.M.backward(plan, q, k, v, out, lse, dout)
+        assert G.M.attn_plan_check_status(plan) == 0
+        grads.append((dq.cpu(), dk.cpu(), dv.cpu()))
+    for a, b in zip(grads[0], grads[1]):
+        assert torch.equal(a, b)
+    dq, dk, dv = grads[0]
+    rq, rk, rv = oracle.sampled_backward(wl, wl.masks[0], dout_h, qs, ks)
+    got_q = torch.stack([dq[int(wl.cu_seqlens_q[b]) + i, h] for b, h, i in qs])
+    got_k = torch.stack([dk[int(wl.cu_seqlens_k[b]) + j, kh] for b, kh, j in ks])
+    got_v = torch.stack([dv[int(wl.cu_seqlens_k[b]) + j, kh] for b, kh, j in ks])
+    _close(got_q, rq, "full-size dq")
+    _close(got_k, rk, "full-size dk")
+    _close(got_v, rv, "full-size dv")

@@ -119,3 +119,18 @@ def test_planted_mistakes_are_caught(monkeypatch):
             caught += 1
         monkeypatch.setattr(OB, "attention_backward_one_head", good)
     assert caught == 3
+
+
+def test_sampled_backward_matches_full():
+    wl = W.random_small(seed=9, kind="SLIDING_WINDOW", batch=2, hq=4, hkv=2, d=16, lmin=40, lmax=90)
+    rng = np.random.default_rng(9)
+    do = rng.standard_normal((int(wl.cu_seqlens_q[-1]), wl.hq, wl.d))
+    dq, dk, dv = oracle.masked_attention_backward(wl, wl.masks[0], do)
+    qs = [(b, int(rng.integers(0, wl.hq)), int(rng.integers(0, wl.lq(b)))) for b in (0, 1) for _ in range(4)]
+    ks = [(b, int(rng.integers(0, wl.hkv)), int(rng.integers(0, wl.lk(b)))) for b in (0, 1) for _ in range(4)]
+    sq, sk, sv = OB.sampled_backward(wl, wl.masks[0], do, qs, ks, row_block=16)
+    for n, (b, h, i) in enumerate(qs):
+        assert np.allclose(sq[n], dq[int(wl.cu_seqlens_q[b]) + i, h], atol=1e-12)
+    for n, (b, kh, j) in enumerate(ks):
+        assert np.allclose(sk[n], dk[int(wl.cu_seqlens_k[b]) + j, kh], atol=1e-12)
+        assert np.allclose(sv[n], dv[int(wl.cu_seqlens_k[b]) + j, kh], atol=1e-12)
