@@ -29,7 +29,15 @@
  * masks of the partial tiles and a balanced work list into a device workspace that the
  * plan owns. attn_masked_fwd() then runs the forward on a stream; it allocates nothing
  * and may be called any number of times with the same plan (e.g. the same lengths and
- * mask for every layer). attn_plan_destroy() frees the plan.
+ * mask for every layer). attn_plan_destroy() frees the plan. Beyond that:
+ *   - split-KV (attn_problem_t.kv_splits): few long work items are cut into key ranges
+ *     whose partial results a second kernel merges;
+ *   - query-row shards (attn_problem_t.q_begin / q_end): one long sequence over several
+ *     GPUs, each computing its rows against all (all-gathered) keys;
+ *   - attn_plan_bwd() + attn_masked_bwd(): dq, dk, dv;
+ *   - attn_fp8_transpose_v() + attn_masked_fwd_fp8(): the forward on e4m3 inputs;
+ *   - attn_plan_dry_run(): the plan statistics on the host, without a GPU;
+ *   - attn_masked_fwd_noalloc(): plan + forward without any device allocation.
  *
  * Errors. Every call returns an attn_status_t; nothing is thrown across the ABI and
  * nothing exits the process. attn_status_string() names a status.
