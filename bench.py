@@ -199,6 +199,11 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def custom_bytes(spec):
+    """Bytes of a CUSTOM mask's packed bits (what attn_plan scans on the device)."""
+    return int(np.asarray(spec.bits).nbytes) if getattr(spec, "bits", None) is not None else 0
+
+
 def config_of(wl, args, world):
     tq = int(wl.cu_seqlens_q[-1])
     tk = int(wl.cu_seqlens_k[-1]) if not wl.paged else int(wl.k_cache.shape[0] * wl.page_size)
@@ -263,7 +268,11 @@ def run_ours(args, rank, world, local_rank):
         raise SystemExit("--pass bwd: contiguous K/V and head_dim <= 128 only (workloads 1, 4, 5)")
     if fp8 and (bwd or wl.paged or wl.d not in (128, 256)):
         raise SystemExit("--dtype e4m3: the forward with contiguous K/V, head_dim 128 or 256 (workloads 2, 4, 5)")
-    plans = [make_plan(M, wl, spec, dev, args.kv_splits, backward=bwd) for spec in wl.masks]
+    plans, plan_ms = [], []
+    for spec in wl.masks:   # attn_plan is timed on its own (host wall clock; it synchronises its stream)
+        t0 = time.perf_counter()
+        plans.append(make_plan(M, wl, spec, dev, args.kv_splits, backward=bwd))
+        plan_ms.append((time.perf_counter() - t0) * 1e3)
     stats = [M.attn_plan_get_stats(p) for p in plans]
     flops = [flops_of(s, wl) * (2.5 if bwd else 1.0) for s in stats]
     tq = q.shape[0]
@@ -433,12 +442,17 @@ def run_ours(args, rank, world, local_rank):
                                 else f"masked_attn_fwd_kernel e4m3 d={wl.d}" if fp8
                                 else f"masked_attn_fwd_kernel d={wl.d}"),
                      "algorithmic_flops_per_launch": sum(flops) / len(flops),
-                     "avg_launch_ms": avg_launch_ms},
+                     "avg_launch_ms": avg_launch_ms,
+                     # DRAM GB/s of the captured launch (ncu bytes over this run's mean launch time)
+                     "dram_gbs": (tr / (avg_launch_ms * 1e-3) / 1e9) if tr else None},
         "per_mask": [{"mask": m.kind, "unmasked_pairs_per_head": s["unmasked_pairs"], "tflops_per_s":
                       f / (statistics.mean(x) * 1e-3) / 1e12, "ms": statistics.mean(x),
                       "tiles_e_f_p": [s["tiles_empty"], s["tiles_full"], s["tiles_partial"]],
-                      "kv_splits_max": s["kv_splits_max"], "merge_tiles": s["merge_tiles"]}
-                     for m, s, f, x in zip(wl.masks, stats, flops, launch_ms)],
+                      "kv_splits_max": s["kv_splits_max"], "merge_tiles": s["merge_tiles"],
+                      "plan_ms": pm,
+                      # CUSTOM: the device scan of the packed bits happens inside attn_plan
+                      "custom_scan_gbs": (custom_bytes(m) / (pm * 1e-3) / 1e9) if m.kind == "CUSTOM" else None}
+                     for m, s, f, x, pm in zip(wl.masks, stats, flops, launch_ms, plan_ms)],
         "mask_gbs": mask_bytes / (sum(statistics.mean(x) for x in launch_ms) * 1e-3) / 1e9,
         "e2e": {"value": e2e_val, "unit": "TFLOP/s", "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                 "steps": e2e_steps},

@@ -994,6 +994,23 @@ attn_status_t plan_backward(const attn_mask_desc_t* mask, const Shape& s, RowSou
   return ATTN_OK;
 }
 
+// Problem shape and kernel shape of a plan from the validated problem.
+void fill_meta(const Shape& s, const attn_problem_t* problem, attn_plan_t& m) {
+  m.batch = s.B;
+  m.hq = s.hq;
+  m.hkv = s.hkv;
+  m.d = s.d;
+  m.scale = s.scale;
+  m.paged = s.paged;
+  m.page_size = s.ps;
+  m.max_pages = s.maxp;
+  m.num_pages = s.npages;
+  m.page_table = s.paged ? problem->page_table : nullptr;
+  m.total_q = s.total_q;
+  m.total_kv_rows = s.total_kv_rows;
+  choose_shape(s, m);
+}
+
 attn_status_t plan_impl(const attn_problem_t* problem, const attn_mask_desc_t* mask, cudaStream_t stream,
                         attn_plan_t** out_plan, bool with_bwd = false) {
   if (!out_plan) return ATTN_ERR_INVALID_ARG;
@@ -1012,19 +1029,7 @@ attn_status_t plan_impl(const attn_problem_t* problem, const attn_mask_desc_t* m
 
   auto plan = new attn_plan_t();
   plan->device = dev;
-  plan->batch = s.B;
-  plan->hq = s.hq;
-  plan->hkv = s.hkv;
-  plan->d = s.d;
-  plan->scale = s.scale;
-  plan->paged = s.paged;
-  plan->page_size = s.ps;
-  plan->max_pages = s.maxp;
-  plan->num_pages = s.npages;
-  plan->page_table = s.paged ? problem->page_table : nullptr;
-  plan->total_q = s.total_q;
-  plan->total_kv_rows = s.total_kv_rows;
-  choose_shape(s, *plan);
+  fill_meta(s, problem, *plan);
   const int R = plan->R;
 
   std::vector<std::vector<int32_t>> cnts(s.B);
@@ -1132,19 +1137,7 @@ attn_status_t mfa_plan_host(const attn_problem_t* problem, const attn_mask_desc_
     st = validate_mask(mask, s);
     if (st != ATTN_OK) return st;
     attn_plan_t& m = out->meta;
-    m.batch = s.B;
-    m.hq = s.hq;
-    m.hkv = s.hkv;
-    m.d = s.d;
-    m.scale = s.scale;
-    m.paged = s.paged;
-    m.page_size = s.ps;
-    m.max_pages = s.maxp;
-    m.num_pages = s.npages;
-    m.page_table = s.paged ? problem->page_table : nullptr;
-    m.total_q = s.total_q;
-    m.total_kv_rows = s.total_kv_rows;
-    choose_shape(s, m);
+    fill_meta(s, problem, m);
     const int R = m.R;
     std::vector<std::vector<int32_t>> cnts(s.B);
     RowSource src(mask, s);
@@ -1195,11 +1188,7 @@ attn_status_t attn_plan_dry_run(const attn_problem_t* problem, const attn_mask_d
     st = validate_mask(mask, s);
     if (st != ATTN_OK) return st;
     attn_plan_t m;
-    m.batch = s.B;
-    m.hq = s.hq;
-    m.hkv = s.hkv;
-    m.d = s.d;
-    choose_shape(s, m);
+    fill_meta(s, problem, m);
     attn_plan_stats_t out{};
     std::vector<std::vector<int32_t>> cnts(s.B);
     RowSource src(mask, s);
