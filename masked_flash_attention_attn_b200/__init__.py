@@ -1,10 +1,27 @@
-"""B200 (sm_100a) masked attention forward.
+"""B200 (sm_100a) masked attention: forward, backward and e4m3 forward.
 
 Thin Python binding over the C ABI declared in ``include/attn.h``: every function
 here only marshals arguments (torch tensors supply device memory and streams);
 all of the computation happens in ``libattn_b200.so``. Importing succeeds without a
 GPU; calls that need one fail with a RuntimeError. If the library has not been
 built, every call raises instead of falling back to anything else.
+
+Typical use (q [total_q, hq, d], k / v [total_k, hkv, d] bf16 CUDA tensors)::
+
+    plan = attn_plan(hq=16, hkv=8, head_dim=256, cu_seqlens_q=cu, cu_seqlens_k=cu,
+                     mask=spec)                      # spec.kind: "CAUSAL", "RANGES", ...
+    out, lse = forward(plan, q, k, v)                # every layer can reuse the plan
+
+    plan = attn_plan(..., backward=True)             # also the dQ / dK / dV work lists
+    out, lse = forward(plan, q, k, v)
+    dq, dk, dv = backward(plan, q, k, v, out, lse, dout)
+
+    attn_fp8_transpose_v(plan, v8, vt8, ldv)         # e4m3 inputs (uint8 tensors)
+    attn_masked_fwd_fp8(plan, q8, k8, vt8, ldv, q_scale, k_scale, v_scale, out, lse)
+
+``kv_splits`` (split-KV) and ``q_rows`` (a query-row shard, see ``sharding``) are
+further attn_plan() arguments; attn_plan_dry_run() gives the plan statistics without
+a GPU.
 """
 from __future__ import annotations
 
