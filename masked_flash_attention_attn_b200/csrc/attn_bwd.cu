@@ -54,6 +54,7 @@ struct BwdParams {
   __nv_bfloat16* g1;    // dK/dV: dv
   int32_t* status;
   int32_t hq, hkv;
+  int32_t debug_flags;   // bit 0: skip the first item's per-item loads (testing the timeout path)
   float scale, scale_log2;
   int64_t timeout_ns;
 };
@@ -198,11 +199,13 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd_dq_kernel(const
       for (int ii = i_begin; ok && ii < i_end; ++ii, ++n) {
         const BwdItem it = p.items[p.cta_items[ii]];
         if (!wait_bounded(BAR(C::B_AEMPTY), (n & 1) ^ 1, guard, kBwdWaitAEmpty)) break;
-        mbar_expect_tx(BAR(C::B_AFULL), 2 * C::TILE_BYTES);
-        a_last = n;
-        for (int c = 0; c < C::NBOX; ++c) {
-          tma_load_3d(sbase + C::OFF_A + c * C::BOX_BYTES, &p.tm_a, c * 64, it.head, it.tok, BAR(C::B_AFULL));
-          tma_load_3d(sbase + C::OFF_B + c * C::BOX_BYTES, &p.tm_b, c * 64, it.head, it.tok, BAR(C::B_AFULL));
+        if (!((p.debug_flags & 1) && n == 0)) {
+          mbar_expect_tx(BAR(C::B_AFULL), 2 * C::TILE_BYTES);
+          a_last = n;
+          for (int c = 0; c < C::NBOX; ++c) {
+            tma_load_3d(sbase + C::OFF_A + c * C::BOX_BYTES, &p.tm_a, c * 64, it.head, it.tok, BAR(C::B_AFULL));
+            tma_load_3d(sbase + C::OFF_B + c * C::BOX_BYTES, &p.tm_b, c * 64, it.head, it.tok, BAR(C::B_AFULL));
+          }
         }
         for (int j = 0; ok && j < it.job_count; ++j) {
           const BwdJob jb = p.jobs[it.job_start + j];
@@ -409,11 +412,13 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd_dkv_kernel(cons
       for (int ii = i_begin; ok && ii < i_end; ++ii, ++n) {
         const BwdItem it = p.items[p.cta_items[ii]];
         if (!wait_bounded(BAR(C::B_AEMPTY), (n & 1) ^ 1, guard, kBwdWaitAEmpty)) break;
-        mbar_expect_tx(BAR(C::B_AFULL), 2 * C::TILE_BYTES);
-        a_last = n;
-        for (int c = 0; c < C::NBOX; ++c) {
-          tma_load_3d(sbase + C::OFF_A + c * C::BOX_BYTES, &p.tm_a, c * 64, it.kv_head, it.tok, BAR(C::B_AFULL));
-          tma_load_3d(sbase + C::OFF_B + c * C::BOX_BYTES, &p.tm_b, c * 64, it.kv_head, it.tok, BAR(C::B_AFULL));
+        if (!((p.debug_flags & 1) && n == 0)) {
+          mbar_expect_tx(BAR(C::B_AFULL), 2 * C::TILE_BYTES);
+          a_last = n;
+          for (int c = 0; c < C::NBOX; ++c) {
+            tma_load_3d(sbase + C::OFF_A + c * C::BOX_BYTES, &p.tm_a, c * 64, it.kv_head, it.tok, BAR(C::B_AFULL));
+            tma_load_3d(sbase + C::OFF_B + c * C::BOX_BYTES, &p.tm_b, c * 64, it.kv_head, it.tok, BAR(C::B_AFULL));
+          }
         }
         for (int j = 0; ok && j < it.job_count; ++j) {
           const BwdJob jb = p.jobs[it.job_start + j];
@@ -639,6 +644,7 @@ attn_status_t mfa_launch_backward(const attn_plan_t* plan, const void* q, const 
     p->status = plan->d_status;
     p->hq = plan->hq;
     p->hkv = plan->hkv;
+    p->debug_flags = plan->debug_flags;
     p->scale = plan->scale;
     p->scale_log2 = plan->scale * 1.4426950408889634f;
     p->timeout_ns = plan->timeout_ns;

@@ -135,3 +135,26 @@ def test_backward_full_size_chunk_causal_sampled():
     _close(got_q, rq, "full-size dq")
     _close(got_k, rk, "full-size dk")
     _close(got_v, rv, "full-size dv")
+
+
+def test_backward_timeout_reports_and_context_survives():
+    """The forced missing arrival of the debug hook in both backward kernels: a bounded wait
+    expires, the status word reports ATTN_ERR_TIMEOUT, the kernels return through their abort
+    paths, and the next backward on the same plan is correct."""
+    wl = W.random_small(seed=6, kind="CAUSAL", batch=2, hq=4, hkv=2, d=128, lmin=100, lmax=300)
+    q, k, v = G.device_inputs(wl)
+    plan = G.M.attn_plan(hq=wl.hq, hkv=wl.hkv, head_dim=wl.d, cu_seqlens_q=wl.cu_seqlens_q,
+                         cu_seqlens_k=wl.cu_seqlens_k, mask=wl.masks[0], scale=wl.scale, backward=True)
+    out, lse = G.M.forward(plan, q, k, v)
+    gen = torch.Generator().manual_seed(6)
+    dout_h = W.randn_bf16(gen, q.shape[0], wl.hq, wl.d)
+    G.M.attn_plan_set_debug(plan, 1, 50_000_000)   # 50 ms per wait
+    G.M.backward(plan, q, k, v, out, lse, dout_h.cuda())
+    assert G.M.attn_plan_check_status(plan) == 6
+    G.M.attn_plan_set_debug(plan, 0, 0)
+    dq, dk, dv = G.M.backward(plan, q, k, v, out, lse, dout_h.cuda())
+    assert G.M.attn_plan_check_status(plan) == 0
+    rq, rk, rv = oracle.masked_attention_backward(wl, wl.masks[0], dout_h)
+    _close(dq, rq, "after timeout dq")
+    _close(dk, rk, "after timeout dk")
+    _close(dv, rv, "after timeout dv")
