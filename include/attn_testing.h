@@ -2,9 +2,9 @@
  * attn_testing.h - test hooks of the B200 masked attention library (not needed to use it).
  *
  * These entry points expose internal device routines so that tests can check them in
- * isolation. No page of the masked-attention pages has a counterpart; the routine below
- * is the share of the softmax exponentials the forward kernel evaluates on the FMA pipes
- * instead of the MUFU unit.
+ * isolation. No page of the masked-attention pages has a counterpart: the first routine
+ * is the share of the softmax exponentials the forward kernel can evaluate on the FMA pipes
+ * instead of the MUFU unit, the second the backward planner's mask-tile transposition.
  */
 #ifndef MASKED_ATTN_B200_ATTN_TESTING_H
 #define MASKED_ATTN_B200_ATTN_TESTING_H
@@ -22,6 +22,11 @@ extern "C" {
  * below -125 are clamped to -125). x and y are DEVICE fp32 arrays of n elements; the work
  * is enqueued on `stream`. Errors: INVALID_ARG (null pointer with n > 0), CUDA. */
 attn_status_t attn_test_exp2_poly(const float* x, float* y, int64_t n, attn_stream_t stream);
+
+/* The planner's transposition of a 2 KiB mask tile (host memory): src row r (four 32-bit
+ * words, bit c of word c / 32 = key c, LSB first) becomes dst row c (bit r = query r), the
+ * layout the dK/dV kernel reads. No GPU involved. Errors: INVALID_ARG (null pointer). */
+attn_status_t attn_test_transpose_mask_tile(const uint32_t* src, uint32_t* dst);
 
 #ifdef __cplusplus
 }

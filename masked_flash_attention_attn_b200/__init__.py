@@ -45,7 +45,8 @@ RANGE_FULL, RANGE_CAUSAL, RANGE_INV_CAUSAL, RANGE_BI_CAUSAL, RANGE_CHUNK_CAUSAL 
 EXPORTS = ("attn_plan", "attn_masked_fwd", "attn_plan_get_tile_classes", "attn_plan_get_stats",
            "attn_plan_check_status", "attn_plan_set_debug", "attn_plan_destroy", "attn_classify_host",
            "attn_status_string", "attn_masked_fwd_noalloc", "attn_test_exp2_poly", "attn_plan_dry_run",
-           "attn_plan_bwd", "attn_masked_bwd", "attn_masked_fwd_fp8", "attn_fp8_transpose_v")
+           "attn_plan_bwd", "attn_masked_bwd", "attn_masked_fwd_fp8", "attn_fp8_transpose_v",
+           "attn_test_transpose_mask_tile")
 
 
 class AttnError(RuntimeError):
@@ -114,6 +115,7 @@ def lib() -> ctypes.CDLL:
         L.attn_masked_fwd_fp8.argtypes = [vp, vp, vp, vp, i64, ctypes.c_float, ctypes.c_float, ctypes.c_float, vp, vp,
                                           vp]
         L.attn_fp8_transpose_v.argtypes = [vp, vp, vp, i64, vp]
+        L.attn_test_transpose_mask_tile.argtypes = [vp, vp]
         L.attn_plan_dry_run.argtypes = [ctypes.POINTER(attn_problem_t), ctypes.POINTER(attn_mask_desc_t), i32,
                                         ctypes.POINTER(attn_plan_stats_t)]
         L.attn_masked_fwd_noalloc.argtypes = [ctypes.POINTER(attn_problem_t), ctypes.POINTER(attn_mask_desc_t),
@@ -393,3 +395,11 @@ def attn_masked_fwd_fp8(plan: Plan, q8, k8, vt8, ldv: int, q_scale: float, k_sca
     _check(lib().attn_masked_fwd_fp8(plan.handle, _ptr(q8), _ptr(k8), _ptr(vt8), int(ldv), float(q_scale),
                                      float(k_scale), float(v_scale), _ptr(out), _ptr(lse), _stream(stream)),
            "attn_masked_fwd_fp8")
+
+
+def attn_test_transpose_mask_tile(tile_words: np.ndarray) -> np.ndarray:
+    """Test hook: the planner's transposition of one 2 KiB mask tile (512 uint32 words)."""
+    src = np.ascontiguousarray(tile_words, dtype=np.uint32).reshape(512)
+    dst = np.zeros(512, dtype=np.uint32)
+    _check(lib().attn_test_transpose_mask_tile(src.ctypes.data, dst.ctypes.data), "attn_test_transpose_mask_tile")
+    return dst

@@ -31,6 +31,7 @@
 #include <vector>
 
 #include "attn_internal.h"
+#include "attn_testing.h"
 
 // 1: balance items group by group (see build_work); 0: plain longest-processing-time-first
 #ifndef MFA_SCHED_GROUPED
@@ -898,12 +899,29 @@ void build_bwd(const Shape& s, const std::vector<std::vector<int32_t>>& cnts, in
   assign_lpt(kv_cost, kv_group, num_sms, bl.kv_off, bl.kv_list);
 }
 
-// Row-major 2 KiB tile (row r: 4 words, bit c = key c) -> the transposed tile (row c, bit r).
+// 32 x 32 bit matrix (word i = row i, bit k = column k) transposed in place: the off-diagonal
+// halves, quarters, ... of the rows are swapped in five rounds of masked shifts.
+void transpose32(uint32_t a[32]) {
+  uint32_t m = 0x0000FFFFu;
+  for (int j = 16; j != 0; j >>= 1, m ^= (m << j)) {
+    for (int k = 0; k < 32; k = (k + j + 1) & ~j) {
+      const uint32_t t = ((a[k] >> j) ^ a[k + j]) & m;
+      a[k] ^= t << j;
+      a[k + j] ^= t;
+    }
+  }
+}
+
+// Row-major 2 KiB tile (row r: 4 words, bit c = key c) -> the transposed tile (row c, bit r),
+// as 4 x 4 blocks of 32 x 32 bits.
 void transpose_tile(const uint32_t* src, uint32_t* dst) {
-  std::memset(dst, 0, kMaskTileBytes);
-  for (int r = 0; r < kTile; ++r)
-    for (int c = 0; c < kTile; ++c)
-      if ((src[4 * r + (c >> 5)] >> (c & 31)) & 1u) dst[4 * c + (r >> 5)] |= 1u << (r & 31);
+  for (int rb = 0; rb < 4; ++rb)
+    for (int cb = 0; cb < 4; ++cb) {
+      uint32_t a[32];
+      for (int i = 0; i < 32; ++i) a[i] = src[4 * (32 * rb + i) + cb];
+      transpose32(a);
+      for (int j = 0; j < 32; ++j) dst[4 * (32 * cb + j) + rb] = a[j];
+    }
 }
 
 attn_status_t plan_backward(const attn_mask_desc_t* mask, const Shape& s, RowSource& src, int num_sms,
@@ -1176,6 +1194,12 @@ attn_status_t mfa_plan_host(const attn_problem_t* problem, const attn_mask_desc_
 }
 
 extern "C" {
+
+attn_status_t attn_test_transpose_mask_tile(const uint32_t* src, uint32_t* dst) {
+  if (!src || !dst) return ATTN_ERR_INVALID_ARG;
+  transpose_tile(src, dst);
+  return ATTN_OK;
+}
 
 attn_status_t attn_plan_dry_run(const attn_problem_t* problem, const attn_mask_desc_t* mask, int32_t num_sms,
                                 attn_plan_stats_t* stats) {

@@ -200,3 +200,18 @@ def _err_dry(M, **kw):
     with pytest.raises(M.AttnError) as e:
         M.attn_plan_dry_run(**kw)
     return e.value.status
+
+
+def test_mask_tile_transposition(attn_lib):
+    """The planner's tile transposition (what the dK/dV kernel reads) against a plain bit
+    transpose of random, full, empty and single-bit tiles."""
+    rng = np.random.default_rng(17)
+    cases = [rng.integers(0, 2**32, size=512, dtype=np.uint64).astype(np.uint32),
+             np.full(512, 0xFFFFFFFF, np.uint32), np.zeros(512, np.uint32)]
+    one = np.zeros(512, np.uint32)
+    one[4 * 5 + 2] = 1 << 7                      # row 5, key 64 + 7
+    cases.append(one)
+    for t in cases:
+        bits = np.unpackbits(t.view(np.uint8), bitorder="little").reshape(128, 128)   # [row][key]
+        want = np.packbits(bits.T.reshape(-1), bitorder="little").view(np.uint32)
+        assert np.array_equal(attn_lib.attn_test_transpose_mask_tile(t), want)
