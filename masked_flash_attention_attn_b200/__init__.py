@@ -194,12 +194,15 @@ def _mask_desc(m: _Marshal, mask, device_bits=None):
         d.chunk = attn_range_t(*[int(x) for x in ch])
     rs = getattr(mask, "ranges", None)
     if rs is not None:
-        flat = [tuple(int(x) for x in r) for per in rs for r in per]
+        # attn_range_t is six int32 fields: an [n, 6] int32 array has its layout
+        counts = [len(per) for per in rs]
+        flat = np.zeros((max(1, sum(counts)), 6), np.int32)
+        if sum(counts):
+            flat[:sum(counts)] = np.concatenate([np.asarray(per, dtype=np.int64).reshape(-1, 6)
+                                                 for per in rs if len(per)])
         cu = np.zeros(len(rs) + 1, np.int32)
-        cu[1:] = np.cumsum([len(per) for per in rs])
-        arr = (attn_range_t * max(1, len(flat)))(*[attn_range_t(*r) for r in flat])
-        m.keep.append(arr)
-        d.ranges = ctypes.addressof(arr)
+        cu[1:] = np.cumsum(counts)
+        d.ranges = m.arr(flat, np.int32)
         d.cu_ranges = m.arr(cu, np.int32)
     if mask.kind == "BLOCK_SPARSE":
         d.block_q, d.block_k = int(mask.block_q), int(mask.block_k)
