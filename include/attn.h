@@ -205,21 +205,22 @@ attn_status_t attn_masked_fwd(const attn_plan_t* plan, const void* q, const void
 attn_status_t attn_plan_bwd(const attn_problem_t* problem, const attn_mask_desc_t* mask,
                             attn_stream_t stream, attn_plan_t** out_plan);
 
-/* Backward of attn_masked_fwd for a loss with gradient dout on out (lse has no gradient
- * of its own):
- *     dv_j = sum_i p_ij dout_i,  ds_ij = p_ij (dout_i . v_j - dout_i . out_i),
+/* Backward of attn_masked_fwd for a loss with gradient dout on out and, optionally, dlse on
+ * lse (d lse_i / d s_ij = p_ij):
+ *     dv_j = sum_i p_ij dout_i,  ds_ij = p_ij (dout_i . v_j - dout_i . out_i + dlse_i),
  *     dq_i = scale sum_j ds_ij k_j,  dk_j = scale sum_i ds_ij q_i,
  * p_ij = exp(scale q_i . k_j - lse_i) on visible pairs; dk, dv of a key/value head sum over
  * its query heads. Asynchronous on `stream`; all DEVICE pointers, 16-byte aligned:
  *   q, out, dout  bf16 [total_q][hq][head_dim]; lse fp32 [total_q][hq] as attn_masked_fwd wrote it
+ *   dlse          fp32 [total_q][hq], or NULL (no gradient on lse)
  *   k, v          bf16 [total_k][hkv][head_dim]
  *   dq            bf16 [total_q][hq][head_dim]  (0 on rows that see no key)
  *   dk, dv        bf16 [total_k][hkv][head_dim] (0 on keys that no query sees)
  * The plan must come from attn_plan_bwd(). Allocates nothing. Errors: INVALID_ARG (plan
  * without backward lists, null or misaligned pointer), CUDA. */
 attn_status_t attn_masked_bwd(const attn_plan_t* plan, const void* q, const void* k, const void* v,
-                              const void* out, const float* lse, const void* dout, void* dq, void* dk, void* dv,
-                              attn_stream_t stream);
+                              const void* out, const float* lse, const void* dout, const float* dlse, void* dq,
+                              void* dk, void* dv, attn_stream_t stream);
 
 /* e4m3 (fp8) forward. No page names a layout for it; "Custom mask slows down attention."
  * asks whether the custom-mask path supports fp8. Inputs are e4m3 bytes (1 sign, 4

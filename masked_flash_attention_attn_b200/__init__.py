@@ -111,7 +111,7 @@ def lib() -> ctypes.CDLL:
         L.attn_test_exp2_poly.argtypes = [vp, vp, i64, vp]
         L.attn_plan_bwd.argtypes = [ctypes.POINTER(attn_problem_t), ctypes.POINTER(attn_mask_desc_t), vp,
                                     ctypes.POINTER(vp)]
-        L.attn_masked_bwd.argtypes = [vp] * 11
+        L.attn_masked_bwd.argtypes = [vp] * 12
         L.attn_masked_fwd_fp8.argtypes = [vp, vp, vp, vp, i64, ctypes.c_float, ctypes.c_float, ctypes.c_float, vp, vp,
                                           vp]
         L.attn_fp8_transpose_v.argtypes = [vp, vp, vp, i64, vp]
@@ -270,11 +270,11 @@ def attn_masked_fwd(plan: Plan, q, k, v, out, lse=None, stream=None) -> None:
            "attn_masked_fwd")
 
 
-def attn_masked_bwd(plan: Plan, q, k, v, out, lse, dout, dq, dk, dv, stream=None) -> None:
-    """attn_masked_bwd(): enqueue dq, dk, dv for the gradient dout of out (plan from
-    attn_plan(..., backward=True))."""
-    _check(lib().attn_masked_bwd(plan.handle, _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dout), _ptr(dq),
-                                 _ptr(dk), _ptr(dv), _stream(stream)), "attn_masked_bwd")
+def attn_masked_bwd(plan: Plan, q, k, v, out, lse, dout, dq, dk, dv, stream=None, dlse=None) -> None:
+    """attn_masked_bwd(): enqueue dq, dk, dv for the gradient dout of out and, optionally,
+    dlse of lse (plan from attn_plan(..., backward=True))."""
+    _check(lib().attn_masked_bwd(plan.handle, _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dout),
+                                 _ptr(dlse), _ptr(dq), _ptr(dk), _ptr(dv), _stream(stream)), "attn_masked_bwd")
 
 
 def attn_plan_get_tile_classes(plan: Plan) -> np.ndarray:
@@ -376,13 +376,13 @@ def forward(plan: Plan, q, k, v, stream=None):
     return out, lse
 
 
-def backward(plan: Plan, q, k, v, out, lse, dout, stream=None):
+def backward(plan: Plan, q, k, v, out, lse, dout, stream=None, dlse=None):
     """Allocate dq / dk / dv with torch and run attn_masked_bwd (convenience)."""
     import torch
     dq = torch.empty_like(q)
     dk = torch.empty_like(k)
     dv = torch.empty_like(v)
-    attn_masked_bwd(plan, q, k, v, out, lse, dout, dq, dk, dv, stream)
+    attn_masked_bwd(plan, q, k, v, out, lse, dout, dq, dk, dv, stream, dlse=dlse)
     return dq, dk, dv
 
 

@@ -128,9 +128,10 @@ __device__ __forceinline__ void store_grad_row(uint32_t t_acc, float mul, bool v
   }
 }
 
-// delta[r][h] = dout[r][h] . out[r][h] (fp32), one warp per (row, head).
+// delta[r][h] = dout[r][h] . out[r][h] - dlse[r][h] (fp32; dlse may be null), one warp per
+// (row, head). With a gradient on lse, ds = p (dp - delta) picks up + p dlse.
 __global__ void bwd_delta_kernel(const __nv_bfloat16* __restrict__ out, const __nv_bfloat16* __restrict__ dout,
-                                 float* __restrict__ delta, int64_t rows, int D) {
+                                 const float* __restrict__ dlse, float* __restrict__ delta, int64_t rows, int D) {
   const int lane = threadIdx.x & 31;
   const int64_t warps = int64_t(gridDim.x) * (blockDim.x >> 5);
   for (int64_t r = int64_t(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); r < rows; r += warps) {
@@ -143,7 +144,7 @@ __global__ void bwd_delta_kernel(const __nv_bfloat16* __restrict__ out, const __
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-    if (lane == 0) delta[r] = acc;
+    if (lane == 0) delta[r] = dlse ? acc - dlse[r] : acc;
   }
 }
 
@@ -613,8 +614,8 @@ attn_status_t launch_bwd(int ctas, const BwdParams& p, cudaStream_t stream) {
 }  // namespace mfa
 
 attn_status_t mfa_launch_backward(const attn_plan_t* plan, const void* q, const void* k, const void* v,
-                                  const void* out, const float* lse, const void* dout, void* dq, void* dk, void* dv,
-                                  cudaStream_t stream) {
+                                  const void* out, const float* lse, const void* dout, const float* dlse, void* dq,
+                                  void* dk, void* dv, cudaStream_t stream) {
   using namespace mfa;
   const int D = plan->d;
   const int64_t qrows = plan->total_q * plan->hq, krows = plan->total_kv_rows * plan->hkv;
@@ -626,7 +627,7 @@ attn_status_t mfa_launch_backward(const attn_plan_t* plan, const void* q, const 
     return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
   }
   bwd_delta_kernel<<<4 * 148, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(out),
-                                                static_cast<const __nv_bfloat16*>(dout), plan->d_bdelta, qrows, D);
+                                                static_cast<const __nv_bfloat16*>(dout), dlse, plan->d_bdelta, qrows, D);
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
   BwdParams pq{}, pk{};
   if (!encode3d(&pq.tm_a, q, D, plan->hq, plan->total_q, 128) ||

@@ -180,5 +180,5 @@ attn_status_t mfa_transpose_v(const attn_plan_t* plan, const void* v, void* vt, 
 
 // backward launcher (attn_bwd.cu)
 attn_status_t mfa_launch_backward(const attn_plan_t* plan, const void* q, const void* k, const void* v,
-                                  const void* out, const float* lse, const void* dout, void* dq, void* dk,
-                                  void* dv, cudaStream_t stream);
+                                  const void* out, const float* lse, const void* dout, const float* dlse,
+                                  void* dq, void* dk, void* dv, cudaStream_t stream);

@@ -1254,13 +1254,14 @@ attn_status_t attn_plan_bwd(const attn_problem_t* problem, const attn_mask_desc_
 }
 
 attn_status_t attn_masked_bwd(const attn_plan_t* plan, const void* q, const void* k, const void* v, const void* out,
-                              const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                              const float* lse, const void* dout, const float* dlse, void* dq, void* dk, void* dv,
                               attn_stream_t stream) {
   if (!plan || !plan->has_bwd) return ATTN_ERR_INVALID_ARG;
   const void* ptrs[] = {q, k, v, out, lse, dout, dq, dk, dv};
   for (const void* p : ptrs)
     if (!p || (reinterpret_cast<uintptr_t>(p) & 15u)) return ATTN_ERR_INVALID_ARG;
-  return mfa_launch_backward(plan, q, k, v, out, lse, dout, dq, dk, dv, reinterpret_cast<cudaStream_t>(stream));
+  if (dlse && (reinterpret_cast<uintptr_t>(dlse) & 3u)) return ATTN_ERR_INVALID_ARG;
+  return mfa_launch_backward(plan, q, k, v, out, lse, dout, dlse, dq, dk, dv, reinterpret_cast<cudaStream_t>(stream));
 }
 
 attn_status_t attn_fp8_transpose_v(const attn_plan_t* plan, const void* v, void* vt, int64_t ldv,

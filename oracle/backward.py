@@ -17,7 +17,9 @@ a gradient of its own), the chain rule through the row softmax gives
     dk_j  = scale * sum_i ds_ij q_i
 
 and dk, dv of a key/value head are the sums over the g query heads that read it. A row
-that sees no key has p = 0 and contributes nothing. These are the textbook derivatives of
+that sees no key has p = 0 and contributes nothing. When the loss also depends on lse
+with gradient dlse_i, d lse_i / d s_ij = p_ij adds p_ij dlse_i to ds_ij, i.e. D_i becomes
+D_i - dlse_i. These are the textbook derivatives of
 softmax(scale Q K^T + mask) V; nothing here is taken from the CUDA path.
 """
 from __future__ import annotations
@@ -28,8 +30,8 @@ from .attention import attention_one_head, _f64
 from .masks import dense_mask, dense_mask_rows
 
 
-def attention_backward_one_head(q, k, v, mask, scale, dout):
-    """q [n, d], k, v [L_k, d], mask bool [n, L_k], dout [n, d]; fp64.
+def attention_backward_one_head(q, k, v, mask, scale, dout, dlse=None):
+    """q [n, d], k, v [L_k, d], mask bool [n, L_k], dout [n, d], dlse [n] or None; fp64.
     Returns (dq [n, d], dk [L_k, d], dv [L_k, d])."""
     out, lse = attention_one_head(q, k, v, mask, scale)
     has = np.isfinite(lse)
@@ -38,18 +40,22 @@ def attention_backward_one_head(q, k, v, mask, scale, dout):
     dv = p.T @ dout
     dp = dout @ v.T
     big_d = np.sum(p * dp, axis=1)
+    if dlse is not None:
+        big_d = big_d - np.asarray(dlse, np.float64)
     ds = p * (dp - big_d[:, None])
     dq = scale * (ds @ k)
     dk = scale * (ds.T @ q)
     return dq, dk, dv
 
 
-def masked_attention_backward(wl, spec, dout):
-    """Gradients over a contiguous workload: dout [total_q, Hq, d] (torch or numpy).
-    Returns (dq fp64 [total_q, Hq, d], dk, dv fp64 [total_k, Hkv, d])."""
+def masked_attention_backward(wl, spec, dout, dlse=None):
+    """Gradients over a contiguous workload: dout [total_q, Hq, d], dlse [total_q, Hq] or None
+    (torch or numpy). Returns (dq fp64 [total_q, Hq, d], dk, dv fp64 [total_k, Hkv, d])."""
     if wl.paged:
         raise ValueError("backward oracle: contiguous K/V only")
     dout = dout.to(__import__("torch").float64).numpy() if hasattr(dout, "numpy") else np.asarray(dout, np.float64)
+    if dlse is not None:
+        dlse = dlse.to(__import__("torch").float64).numpy() if hasattr(dlse, "numpy") else np.asarray(dlse, np.float64)
     g = wl.hq // wl.hkv
     total_q, total_k = int(wl.cu_seqlens_q[-1]), int(wl.cu_seqlens_k[-1])
     dq = np.zeros((total_q, wl.hq, wl.d))
@@ -66,7 +72,8 @@ def masked_attention_backward(wl, spec, dout):
         for h in range(wl.hq):
             kh = h // g
             a, bk, bv = attention_backward_one_head(_f64(wl.q[q0:q0 + lq, h]), kk[:, kh], vv[:, kh], m, wl.scale,
-                                                    dout[q0:q0 + lq, h])
+                                                    dout[q0:q0 + lq, h],
+                                                    None if dlse is None else dlse[q0:q0 + lq, h])
             dq[q0:q0 + lq, h] = a
             dk[k0:k0 + lk, kh] += bk
             dv[k0:k0 + lk, kh] += bv

@@ -35,16 +35,18 @@ def _close(got, ref, what):
     assert err.mean() <= REL_MEAN * scale_mean, f"{what}: mean err {err.mean():.3e} vs scale {scale_mean:.3e}"
 
 
-def check_backward(wl, spec, what, seed=0):
+def check_backward(wl, spec, what, seed=0, with_dlse=False):
     q, k, v = G.device_inputs(wl)
     plan = G.M.attn_plan(hq=wl.hq, hkv=wl.hkv, head_dim=wl.d, cu_seqlens_q=wl.cu_seqlens_q,
                          cu_seqlens_k=wl.cu_seqlens_k, mask=spec, scale=wl.scale, backward=True)
     out, lse = G.M.forward(plan, q, k, v)
     gen = torch.Generator().manual_seed(1000 + seed)
     dout_h = W.randn_bf16(gen, q.shape[0], wl.hq, wl.d)
-    dq, dk, dv = G.M.backward(plan, q, k, v, out, lse, dout_h.cuda())
+    dlse_h = torch.randn(q.shape[0], wl.hq, generator=gen) if with_dlse else None
+    dq, dk, dv = G.M.backward(plan, q, k, v, out, lse, dout_h.cuda(),
+                              dlse=None if dlse_h is None else dlse_h.cuda())
     assert G.M.attn_plan_check_status(plan) == 0
-    rq, rk, rv = oracle.masked_attention_backward(wl, spec, dout_h)
+    rq, rk, rv = oracle.masked_attention_backward(wl, spec, dout_h, dlse_h)
     _close(dq, rq, f"{what} dq")
     _close(dk, rk, f"{what} dk")
     _close(dv, rv, f"{what} dv")
@@ -56,6 +58,13 @@ def test_backward_all_kinds(kind, d):
     wl = W.random_small(seed=500 + d + 3 * KINDS.index(kind), kind=kind, batch=3, hq=4, hkv=2, d=d,
                         lmin=1, lmax=330)
     check_backward(wl, wl.masks[0], f"bwd {kind} d={d}")
+
+
+@pytest.mark.parametrize("kind", ["CAUSAL", "CUSTOM"])
+def test_backward_with_lse_gradient(kind):
+    # a loss on lse as well: ds picks up p dlse (delta becomes dout . out - dlse)
+    wl = W.random_small(seed=60 + len(kind), kind=kind, batch=2, hq=4, hkv=2, d=128, lmin=50, lmax=400)
+    check_backward(wl, wl.masks[0], f"bwd dlse {kind}", seed=3, with_dlse=True)
 
 
 @pytest.mark.parametrize("g", [1, 4])

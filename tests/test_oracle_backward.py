@@ -134,3 +134,22 @@ def test_sampled_backward_matches_full():
     for n, (b, kh, j) in enumerate(ks):
         assert np.allclose(sk[n], dk[int(wl.cu_seqlens_k[b]) + j, kh], atol=1e-12)
         assert np.allclose(sv[n], dv[int(wl.cu_seqlens_k[b]) + j, kh], atol=1e-12)
+
+
+@pytest.mark.parametrize("seed", [0, 4])
+def test_finite_differences_with_lse_gradient(seed):
+    # loss = sum dout . out + sum over rows with keys of dlse . lse
+    q, k, v, do, mask = _case(seed)
+    rng = np.random.default_rng(seed + 100)
+    dl = rng.standard_normal(q.shape[0])
+    scale = 0.6
+
+    def loss(qq, kk, vv):
+        out, lse = oracle.attention_one_head(qq, kk, vv, mask, scale)
+        fin = np.isfinite(lse)
+        return float(np.sum(out * do) + np.sum(dl[fin] * lse[fin]))
+
+    dq, dk, dv = OB.attention_backward_one_head(q, k, v, mask, scale, do, dl)
+    assert np.allclose(dq, _fd(lambda x: loss(x, k, v), q), rtol=1e-6, atol=1e-8)
+    assert np.allclose(dk, _fd(lambda x: loss(q, x, v), k), rtol=1e-6, atol=1e-8)
+    assert np.allclose(dv, _fd(lambda x: loss(q, k, x), v), rtol=1e-6, atol=1e-8)
