@@ -40,3 +40,35 @@ def all_gather_rows(local, rows: int, group=None):
     out = torch.empty((per * world,) + tuple(local.shape[1:]), dtype=local.dtype, device=local.device)
     dist.all_gather_into_tensor(out, buf, group=group)
     return out[:rows]
+
+
+def balanced_query_shards(tile_classes, lengths, world: int, block: int = 128):
+    """Row shards [begin, end) for every rank (sequence-local rows, whole `block`-row tiles)
+    that give each rank about the same number of non-empty 128 x 128 tiles, summed over the
+    sequences of the batch (causal masks put more work in later rows than equal row counts
+    would). tile_classes: the classes attn_classify_host returns (sequence, query tile, key
+    tile order; 0 = empty); lengths: [(L_q, L_k)] per sequence. Returns `world` pairs; ranks
+    past the last row get empty shards."""
+    import numpy as np
+    if world <= 0:
+        raise ValueError("bad world")
+    n_qt_max = max(((lq + block - 1) // block for lq, _ in lengths), default=0)
+    work = np.zeros(n_qt_max, np.int64)
+    pos = 0
+    for lq, lk in lengths:
+        n_qt, n_kt = (lq + block - 1) // block, (lk + block - 1) // block
+        cls = np.asarray(tile_classes[pos:pos + n_qt * n_kt]).reshape(n_qt, n_kt) if n_qt * n_kt else None
+        if cls is not None:
+            work[:n_qt] += (cls != 0).sum(axis=1) + 1     # + 1: per-tile fixed cost
+        pos += n_qt * n_kt
+    if pos != len(tile_classes):
+        raise ValueError("tile_classes do not match lengths")
+    cum = np.concatenate([[0], np.cumsum(work)])
+    total = cum[-1]
+    bounds = [0]
+    for r in range(1, world):
+        bounds.append(int(np.searchsorted(cum, total * r / world, side="left")))
+    bounds.append(n_qt_max)
+    bounds = np.maximum.accumulate(np.clip(bounds, 0, n_qt_max))
+    lq_max = max((lq for lq, _ in lengths), default=0)
+    return [(min(lq_max, int(a) * block), min(lq_max, int(b) * block)) for a, b in zip(bounds[:-1], bounds[1:])]

@@ -57,3 +57,25 @@ def test_all_gather_rows_gloo(rows):
         p.join(timeout=60)
         assert p.exitcode == 0
     assert all(ok for _, ok in res)
+
+
+def test_balanced_shards_even_out_causal_work(attn_lib):
+    """For a causal batch, equal row counts give the last rank most of the tiles; the
+    work-balanced shards (from the host tile classes) give every rank about the same number
+    of jobs, and the shards still partition the work list exactly."""
+    M = attn_lib
+    L = 16384
+    cq = W.cu_from_lengths([L, L // 2])
+    kw = dict(hq=8, hkv=2, head_dim=128, cu_seqlens_q=cq, cu_seqlens_k=cq, mask=W.MaskSpec("CAUSAL"))
+    cls, _ = M.attn_classify_host(**kw)
+    lengths = [(L, L), (L // 2, L // 2)]
+    full = M.attn_plan_dry_run(kv_splits=1, **kw)
+    world = 4
+    equal = [S.query_shard(L, r, world) for r in range(world)]
+    bal = S.balanced_query_shards(cls, lengths, world)
+    assert bal[0][0] == 0 and bal[-1][1] == L and all(a[1] == b[0] for a, b in zip(bal, bal[1:]))
+    jobs_eq = [M.attn_plan_dry_run(kv_splits=1, q_rows=sh, **kw)["jobs"] for sh in equal]
+    jobs_bal = [M.attn_plan_dry_run(kv_splits=1, q_rows=sh, **kw)["jobs"] for sh in bal]
+    assert sum(jobs_bal) == full["jobs"] == sum(jobs_eq)
+    assert max(jobs_eq) > 1.3 * (full["jobs"] / world)         # equal rows: imbalanced
+    assert max(jobs_bal) < 1.15 * (full["jobs"] / world)       # balanced within 15 %
