@@ -14,7 +14,7 @@ same workload (seed offset by rank); there is no collective on the data path. Ti
 the max over ranks of CUDA-event time; the value is the work of all ranks / that time.
 
 --impl reference times the fp64 CPU oracle on a bounded row sample of the same workload
-(rank 0 only), the baseline arm of this build.
+(rank 0 only): the CPU baseline arm.
 """
 from __future__ import annotations
 
@@ -24,6 +24,7 @@ import json
 import os
 import statistics
 import subprocess
+import tempfile
 import sys
 import time
 
@@ -86,9 +87,9 @@ class ClockSampler:
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, device_index):
+    def __init__(self, device_index, log_dir=None):
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{device_index}.csv")
+        self.path = os.path.join(log_dir or tempfile.gettempdir(), f"clocks_rank{device_index}.csv")
         try:
             import torch
             uuid = "GPU-" + str(torch.cuda.get_device_properties(device_index).uuid)
@@ -327,7 +328,7 @@ def run_ours(args, rank, world, local_rank):
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    sampler = ClockSampler(local_rank)
+    sampler = ClockSampler(local_rank, args.clock_log)
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     t_start.record(stream)
     for s in range(args.steps):
@@ -537,6 +538,8 @@ def main():
     ap.add_argument("--kv-splits", type=int, default=0,
                     help="split-KV: 0 automatic, 1 never, N >= 2 at most N key ranges per query tile")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--clock-log", default=None,
+                    help="folder for the raw nvidia-smi clock samples (default: the temp folder)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
