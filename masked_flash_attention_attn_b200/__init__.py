@@ -8,8 +8,9 @@ built, every call raises instead of falling back to anything else.
 
 Typical use (q [total_q, hq, d], k / v [total_k, hkv, d] bf16 CUDA tensors)::
 
+    from masked_flash_attention_attn_b200 import mask as masks
     plan = attn_plan(hq=16, hkv=8, head_dim=256, cu_seqlens_q=cu, cu_seqlens_k=cu,
-                     mask=spec)                      # spec.kind: "CAUSAL", "RANGES", ...
+                     mask=masks.sliding_window(4096))  # masks.causal(), .ranges(...), .custom(...)
     out, lse = forward(plan, q, k, v)                # every layer can reuse the plan
 
     plan = attn_plan(..., backward=True)             # also the dQ / dK / dV work lists
