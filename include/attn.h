@@ -192,7 +192,12 @@ attn_status_t attn_plan(const attn_problem_t* problem, const attn_mask_desc_t* m
  *       bf16 [num_pages][page_size][hkv][head_dim] paged caches
  *   out bf16 [total_q][hq][head_dim]             written for every valid row
  *   lse fp32 [total_q][hq]                       natural log, scale included; may be NULL
- * Allocates nothing. Errors: INVALID_ARG (null/misaligned pointer), CUDA (launch). */
+ * Allocates nothing. Errors: INVALID_ARG (null/misaligned pointer), CUDA (launch).
+ * Concurrency: the forward only reads the plan, except that a split plan (stats
+ * kv_splits_max > 1) keeps the partial results of its key ranges in the plan's workspace.
+ * Unsplit plans may therefore serve forwards on several streams at once; forwards of a
+ * split plan, and backwards (attn_masked_bwd keeps its per-row dout . out there too), must
+ * be ordered one after another (one stream, or events between the streams). */
 attn_status_t attn_masked_fwd(const attn_plan_t* plan, const void* q, const void* k, const void* v,
                               void* out, float* lse, attn_stream_t stream);
 
