@@ -1230,6 +1230,8 @@ attn_status_t attn_plan_dry_run(const attn_problem_t* problem, const attn_mask_d
     return ATTN_OK;
   } catch (const std::bad_alloc&) {
     return ATTN_ERR_OOM;
+  } catch (...) {
+    return ATTN_ERR_INVALID_ARG;
   }
 }
 
@@ -1250,6 +1252,8 @@ attn_status_t attn_plan_bwd(const attn_problem_t* problem, const attn_mask_desc_
     return plan_impl(problem, mask, reinterpret_cast<cudaStream_t>(stream), out_plan, /*with_bwd=*/true);
   } catch (const std::bad_alloc&) {
     return ATTN_ERR_OOM;
+  } catch (...) {
+    return ATTN_ERR_INVALID_ARG;
   }
 }
 
@@ -1367,6 +1371,8 @@ attn_status_t attn_classify_host(const attn_problem_t* problem, const attn_mask_
     return ATTN_OK;
   } catch (const std::bad_alloc&) {
     return ATTN_ERR_OOM;
+  } catch (...) {
+    return ATTN_ERR_INVALID_ARG;
   }
 }
 
