@@ -19,6 +19,7 @@ the max over ranks of CUDA-event time; the value is the work of all ranks / that
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import hashlib
 import json
 import os
@@ -271,6 +272,12 @@ def run_ours(args, rank, world, local_rank):
         raise SystemExit("--dtype e4m3: the forward with contiguous K/V, head_dim 128 or 256 (workloads 2, 4, 5)")
     plans, plan_ms = [], []
     for spec in wl.masks:   # attn_plan is timed on its own (host wall clock; it synchronises its stream)
+        if spec.kind == "CUSTOM" and isinstance(spec.bits, np.ndarray):
+            # attn_mask_desc_t.mask_bits is a device pointer: the packed bits are staged in HBM
+            # first, so plan_ms (and custom_scan_gbs) cover the device scan, not a host upload
+            spec = dataclasses.replace(spec, bits=torch.from_numpy(
+                np.ascontiguousarray(spec.bits.astype(np.uint32).view(np.int32))).to(dev))
+            torch.cuda.synchronize()
         t0 = time.perf_counter()
         plans.append(make_plan(M, wl, spec, dev, args.kv_splits, backward=bwd))
         plan_ms.append((time.perf_counter() - t0) * 1e3)
