@@ -278,6 +278,9 @@ def run_ours(args, rank, world, local_rank):
             spec = dataclasses.replace(spec, bits=torch.from_numpy(
                 np.ascontiguousarray(spec.bits.astype(np.uint32).view(np.int32))).to(dev))
             torch.cuda.synchronize()
+        # the first plan of a kind also pays one-off costs (context set-up, module loading):
+        # plan once untimed, then time the plan that is kept
+        make_plan(M, wl, spec, dev, args.kv_splits, backward=bwd)
         t0 = time.perf_counter()
         plans.append(make_plan(M, wl, spec, dev, args.kv_splits, backward=bwd))
         plan_ms.append((time.perf_counter() - t0) * 1e3)
