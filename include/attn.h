@@ -174,6 +174,8 @@ typedef struct {
   int32_t merge_tiles;              /* 128-row query tiles whose partial results the merge kernel combines */
   int64_t vt_keys;                  /* contiguous K/V: columns of the transposed V that attn_fp8_transpose_v
                                        writes (each sequence starts at a multiple of 128); 0 if paged */
+  int64_t workspace_bytes;          /* device workspace of the forward plan: work list, mask tiles, split-KV
+                                       slots (attn_plan_bwd allocates the backward's on top) */
 } attn_plan_stats_t;
 
 /* Validate and plan. `stream` orders the plan's device work (the CUSTOM mask scan and

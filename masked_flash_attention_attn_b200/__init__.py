@@ -82,7 +82,8 @@ class attn_plan_stats_t(ctypes.Structure):
                 ("tiles_partial", ctypes.c_int64), ("mask_tiles", ctypes.c_int64), ("work_items", ctypes.c_int64),
                 ("jobs", ctypes.c_int64), ("mask_tile_reads", ctypes.c_int64), ("ctas", ctypes.c_int32), ("heads_per_tile", ctypes.c_int32),
                 ("tiles_per_cta", ctypes.c_int32), ("cluster_size", ctypes.c_int32),
-                ("kv_splits_max", ctypes.c_int32), ("merge_tiles", ctypes.c_int32), ("vt_keys", ctypes.c_int64)]
+                ("kv_splits_max", ctypes.c_int32), ("merge_tiles", ctypes.c_int32), ("vt_keys", ctypes.c_int64),
+                ("workspace_bytes", ctypes.c_int64)]
 
 
 _lib = None

@@ -518,6 +518,7 @@ void build_work(const Shape& s, int R, int hp, int nq, const std::vector<std::ve
     const int n_rb = (lq + R - 1) / R, n_kt = (lk + kTile - 1) / kTile;
     const std::vector<int32_t>& cnt = cnts[b];
     std::vector<int32_t> tidx(size_t(n_rb) * n_kt, -1);
+    std::unordered_map<int64_t, std::pair<int32_t, int32_t>> lists;   // (row blocks) -> jobs
     auto kclass = [&](int rb, int kt) -> int32_t {
       const int64_t rows = std::min(R, lq - rb * R), cols = std::min(kTile, lk - kt * kTile);
       return classify(cnt[size_t(rb) * n_kt + kt], rows * cols);
@@ -551,6 +552,16 @@ void build_work(const Shape& s, int R, int hp, int nq, const std::vector<std::ve
         it.rows[t] = rbs[t] >= 0 ? std::min(R, lq - rb * R) : 0;
         it.head[t] = kh * g + hg * hp;
       }
+      // The jobs depend on the row blocks only, not on the heads: items of other KV heads
+      // and head groups over the same row blocks share one list (read-only on the device).
+      const int64_t key = int64_t(rb0) * (int64_t(n_rb) + 1) + (rb1 + 1);
+      auto hit = lists.find(key);
+      if (hit != lists.end()) {
+        it.job_start = hit->second.first;
+        it.job_count = hit->second.second;
+        wl.items.push_back(it);
+        return;
+      }
       it.job_start = int32_t(wl.jobs.size());
       for (int kt = 0; kt < n_kt; ++kt) {
         Job j{};
@@ -565,6 +576,7 @@ void build_work(const Shape& s, int R, int hp, int nq, const std::vector<std::ve
         wl.jobs.push_back(Job{0, {kMaskNone, kMaskNone}, 0});
       }
       it.job_count = int32_t(wl.jobs.size()) - it.job_start;
+      lists.emplace(key, std::make_pair(it.job_start, it.job_count));
       wl.items.push_back(it);
     };
     // the row blocks this plan computes: those overlapping the query-row shard
@@ -1073,6 +1085,7 @@ attn_status_t plan_impl(const attn_problem_t* problem, const attn_mask_desc_t* m
   work_stats(*plan, wl, plan->stats);
 
   const Staging lay = layout(wl, s.d, s.B);
+  plan->stats.workspace_bytes = int64_t(lay.total);
   std::vector<char> host(lay.off_tiles, 0);
   std::memcpy(host.data() + lay.off_items, wl.items.data(), wl.items.size() * sizeof(WorkItem));
   std::memcpy(host.data() + lay.off_jobs, wl.jobs.data(), wl.jobs.size() * sizeof(Job));
@@ -1226,6 +1239,7 @@ attn_status_t attn_plan_dry_run(const attn_problem_t* problem, const attn_mask_d
     m.ctas = int32_t(wl.cta_off.size()) - 1;
     m.vt_keys = s.paged ? 0 : vt_offsets(s)[s.B];
     work_stats(m, wl, out);
+    out.workspace_bytes = int64_t(layout(wl, s.d, s.B).total);
     *stats = out;
     return ATTN_OK;
   } catch (const std::bad_alloc&) {

@@ -66,3 +66,21 @@ def test_shard_validation_and_empty_shard(attn_lib):
     assert e.value.status == 1
     st = M.attn_plan_dry_run(q_rows=(10000, 20000), **kw)          # past every sequence
     assert st["work_items"] == 0 and st["jobs"] == 0
+
+
+@pytest.mark.parametrize("kind", ["CAUSAL", "RANGES", "BLOCK_SPARSE"])
+def test_job_lists_are_shared_across_heads(attn_lib, kind):
+    """Items over the same row blocks read one job list whatever their KV head: going from
+    1 to 8 KV heads (same group size) multiplies the items and jobs by 8 but adds to the
+    workspace only the items and per-CTA lists, never another copy of the job lists."""
+    wl = W.random_small(seed=31, kind=kind, batch=3, hq=2, hkv=1, d=128, lmin=200, lmax=1500)
+    kw = _kw(wl, wl.masks[0])
+    one = attn_lib.attn_plan_dry_run(kv_splits=1, **kw)
+    kw.update(hq=16, hkv=8)
+    eight = attn_lib.attn_plan_dry_run(kv_splits=1, **kw)
+    assert eight["work_items"] == 8 * one["work_items"] and eight["jobs"] == 8 * one["jobs"]
+    grown = eight["workspace_bytes"] - one["workspace_bytes"]
+    # 64-byte items, one int32 per listed item and per CTA offset, plus alignment of the parts
+    assert grown <= (eight["work_items"] - one["work_items"]) * (64 + 4) + 4 * (eight["ctas"] + 1) + 8 * 256
+    # copies of the 16-byte jobs per head would exceed that bound by more than its slack
+    assert 16 * (eight["jobs"] - one["jobs"]) > 8 * 256
