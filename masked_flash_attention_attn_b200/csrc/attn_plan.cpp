@@ -646,8 +646,13 @@ void write_mask_tile(RowSource& src, const Shape& s, int R, const TileRef& t, ui
     const Iv* iv;
     const int n = src.row(t.seq, i, &iv);
     for (int k = 0; k < n; ++k) {
-      const int a = std::max(iv[k].a, c0), e = std::min(iv[k].b, c1);
-      for (int j = a; j < e; ++j) w[(j - c0) >> 5] |= 1u << ((j - c0) & 31);
+      // bits [lo, hi) of the tile row, a word at a time
+      const int lo = std::max(iv[k].a, c0) - c0, hi = std::min(iv[k].b, c1) - c0;
+      for (int x = lo; x < hi;) {
+        const int word = x >> 5, end = std::min(hi, (word + 1) * 32), len = end - x;
+        w[word] |= (len == 32 ? ~0u : ((1u << len) - 1u)) << (x & 31);
+        x = end;
+      }
     }
     for (int r = lr; r < kTile; r += R) std::memcpy(dst + 4 * r, w, 16);
   }
