@@ -864,27 +864,50 @@ void build_bwd(const Shape& s, const std::vector<std::vector<int32_t>>& cnts, in
     const int lq = s.lq[b], lk = s.lk[b];
     const int n_qt = (lq + kTile - 1) / kTile, n_kt = (lk + kTile - 1) / kTile;
     const std::vector<int32_t>& cnt = cnts[b];
-    std::vector<int32_t> tidx(size_t(n_qt) * n_kt, -1);
-    auto mask_of = [&](int qt, int kt) -> int32_t {
-      const int64_t rows = std::min(kTile, lq - qt * kTile), cols = std::min(kTile, lk - kt * kTile);
-      const int32_t k = classify(cnt[size_t(qt) * n_kt + kt], rows * cols);
-      if (k == kClassEmpty) return kMaskNone;
-      if (k == kClassFull && (kt + 1) * kTile <= lk && (qt + 1) * kTile <= lq) return kMaskFull;
-      int32_t& t = tidx[size_t(qt) * n_kt + kt];
-      if (t < 0) {
-        t = int32_t(bl.tiles.size());
-        bl.tiles.push_back(TileRef{b, qt, kt, t});
+    // How every (query tile, key tile) is masked, the same for all heads; partial tiles are
+    // numbered in row-major order. Row lists serve the dQ items, column lists the dK/dV items.
+    std::vector<int32_t> row_off(size_t(n_qt) + 1, 0), col_off(size_t(n_kt) + 1, 0);
+    std::vector<int32_t> tab(size_t(n_qt) * n_kt, kMaskNone);
+    for (int qt = 0; qt < n_qt; ++qt)
+      for (int kt = 0; kt < n_kt; ++kt) {
+        const int64_t rows = std::min(kTile, lq - qt * kTile), cols = std::min(kTile, lk - kt * kTile);
+        const int32_t k = classify(cnt[size_t(qt) * n_kt + kt], rows * cols);
+        int32_t m = kMaskNone;
+        if (k == kClassFull && (kt + 1) * kTile <= lk && (qt + 1) * kTile <= lq) {
+          m = kMaskFull;
+        } else if (k != kClassEmpty) {
+          m = int32_t(bl.tiles.size());
+          bl.tiles.push_back(TileRef{b, qt, kt, m});
+        }
+        tab[size_t(qt) * n_kt + kt] = m;
+        if (m != kMaskNone) {
+          row_off[qt + 1]++;
+          col_off[kt + 1]++;
+        }
       }
-      return t;
-    };
+    for (int qt = 0; qt < n_qt; ++qt) row_off[qt + 1] += row_off[qt];
+    for (int kt = 0; kt < n_kt; ++kt) col_off[kt + 1] += col_off[kt];
+    std::vector<int32_t> row_kt(row_off[n_qt]), col_qt(col_off[n_kt]);
+    {
+      std::vector<int32_t> rf(row_off.begin(), row_off.end() - 1), cf(col_off.begin(), col_off.end() - 1);
+      for (int qt = 0; qt < n_qt; ++qt)
+        for (int kt = 0; kt < n_kt; ++kt)
+          if (tab[size_t(qt) * n_kt + kt] != kMaskNone) {
+            row_kt[rf[qt]++] = kt;
+            col_qt[cf[kt]++] = qt;
+          }
+    }
+    const size_t nnz = row_kt.size();
+    bl.q_jobs.reserve(bl.q_jobs.size() + size_t(s.hq) * (nnz + n_qt));
+    bl.kv_jobs.reserve(bl.kv_jobs.size() + size_t(s.hq) * nnz + size_t(s.hkv) * n_kt);
     for (int kh = 0; kh < s.hkv; ++kh) {
       // dQ items
       for (int h = kh * g; h < (kh + 1) * g; ++h)
         for (int qt = 0; qt < n_qt; ++qt) {
           BwdItem it{b, kh, h, s.qoff[b] + qt * kTile, std::min(kTile, lq - qt * kTile), int32_t(bl.q_jobs.size()), 0, 0};
-          for (int kt = 0; kt < n_kt; ++kt) {
-            const int32_t m = mask_of(qt, kt);
-            if (m != kMaskNone) bl.q_jobs.push_back(BwdJob{s.koff[b] + kt * kTile, m, h, 0});
+          for (int32_t e = row_off[qt]; e < row_off[qt + 1]; ++e) {
+            const int kt = row_kt[e];
+            bl.q_jobs.push_back(BwdJob{s.koff[b] + kt * kTile, tab[size_t(qt) * n_kt + kt], h, 0});
           }
           if (bl.q_jobs.size() == size_t(it.job_start))   // no key anywhere: one hidden job writes dq = 0
             bl.q_jobs.push_back(BwdJob{s.koff[b], kMaskNone, h, 0});
@@ -898,10 +921,10 @@ void build_bwd(const Shape& s, const std::vector<std::vector<int32_t>>& cnts, in
         BwdItem it{b, kh, kh * g, s.koff[b] + kt * kTile, std::min(kTile, lk - kt * kTile),
                    int32_t(bl.kv_jobs.size()), 0, 0};
         for (int h = kh * g; h < (kh + 1) * g; ++h)
-          for (int qt = 0; qt < n_qt; ++qt) {
-            const int32_t m = mask_of(qt, kt);
-            if (m != kMaskNone)
-              bl.kv_jobs.push_back(BwdJob{s.qoff[b] + qt * kTile, m, h, std::min(kTile, lq - qt * kTile)});
+          for (int32_t e = col_off[kt]; e < col_off[kt + 1]; ++e) {
+            const int qt = col_qt[e];
+            bl.kv_jobs.push_back(BwdJob{s.qoff[b] + qt * kTile, tab[size_t(qt) * n_kt + kt], h,
+                                        std::min(kTile, lq - qt * kTile)});
           }
         if (bl.kv_jobs.size() == size_t(it.job_start))   // no query sees the tile: dk = dv = 0
           bl.kv_jobs.push_back(BwdJob{s.qoff[b], kMaskNone, kh * g, 0});
