@@ -992,21 +992,30 @@ attn_status_t plan_backward(const attn_mask_desc_t* mask, const Shape& s, RowSou
                o_ko = take(bl.kv_off.size() * 4), o_kl = take(bl.kv_list.size() * 4),
                o_mq = take(nt * kMaskTileBytes), o_mk = take(nt * kMaskTileBytes),
                o_dl = take(size_t(std::max<int64_t>(1, s.total_q)) * s.hq * sizeof(float));
-  std::vector<char> host(o_mq, 0);
-  std::memcpy(host.data() + o_qi, bl.q_items.data(), bl.q_items.size() * sizeof(BwdItem));
-  std::memcpy(host.data() + o_qj, bl.q_jobs.data(), bl.q_jobs.size() * sizeof(BwdJob));
-  std::memcpy(host.data() + o_qo, bl.q_off.data(), bl.q_off.size() * 4);
-  std::memcpy(host.data() + o_ql, bl.q_list.data(), bl.q_list.size() * 4);
-  std::memcpy(host.data() + o_ki, bl.kv_items.data(), bl.kv_items.size() * sizeof(BwdItem));
-  std::memcpy(host.data() + o_kj, bl.kv_jobs.data(), bl.kv_jobs.size() * sizeof(BwdJob));
-  std::memcpy(host.data() + o_ko, bl.kv_off.data(), bl.kv_off.size() * 4);
-  std::memcpy(host.data() + o_kl, bl.kv_list.data(), bl.kv_list.size() * 4);
   void* ws = nullptr;
   cudaError_t e = cudaMalloc(&ws, off);
   if (e != cudaSuccess) return cuda_status(e);
   char* base = static_cast<char*>(ws);
   std::vector<uint32_t> qmaj(nt * (kMaskTileBytes / 4)), kmaj(nt * (kMaskTileBytes / 4));
-  e = cudaMemcpyAsync(base, host.data(), host.size(), cudaMemcpyHostToDevice, stream);
+  // the lists go up straight from their vectors (the block-dense lists are ~46 MB: a host
+  // staging copy would double the host traffic); the padding between them is zeroed on the
+  // device
+  e = cudaMemsetAsync(base, 0, o_mq, stream);
+  const struct {
+    size_t dst;
+    const void* src;
+    size_t bytes;
+  } parts[] = {{o_qi, bl.q_items.data(), bl.q_items.size() * sizeof(BwdItem)},
+               {o_qj, bl.q_jobs.data(), bl.q_jobs.size() * sizeof(BwdJob)},
+               {o_qo, bl.q_off.data(), bl.q_off.size() * 4},
+               {o_ql, bl.q_list.data(), bl.q_list.size() * 4},
+               {o_ki, bl.kv_items.data(), bl.kv_items.size() * sizeof(BwdItem)},
+               {o_kj, bl.kv_jobs.data(), bl.kv_jobs.size() * sizeof(BwdJob)},
+               {o_ko, bl.kv_off.data(), bl.kv_off.size() * 4},
+               {o_kl, bl.kv_list.data(), bl.kv_list.size() * 4}};
+  for (const auto& pt : parts)
+    if (e == cudaSuccess && pt.bytes)
+      e = cudaMemcpyAsync(base + pt.dst, pt.src, pt.bytes, cudaMemcpyHostToDevice, stream);
   attn_status_t st = cuda_status(e);
   if (st == ATTN_OK && nt) {
     if (mask->kind == ATTN_MASK_CUSTOM) {
