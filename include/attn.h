@@ -273,7 +273,11 @@ attn_status_t attn_plan_check_status(const attn_plan_t* plan, attn_stream_t stre
  * (default 2 s). 0 / 0 restores the defaults. */
 attn_status_t attn_plan_set_debug(attn_plan_t* plan, int32_t flags, int64_t timeout_ns);
 
-/* Free the plan and its device workspace (after the forwards that use it finished). */
+/* Free the plan and its device workspace (after the forwards that use it finished).
+ * The workspace is freed with cudaFree, which waits for the work in flight on the device;
+ * attn_plan() likewise allocates with cudaMalloc and waits for `stream`. A runtime that
+ * re-plans every step beside other streams' kernels keeps plans alive across steps or
+ * uses attn_masked_fwd_noalloc(), which allocates and frees nothing. */
 attn_status_t attn_plan_destroy(attn_plan_t* plan);
 
 /* Host-only classification for the analytic kinds (everything but CUSTOM): the same
