@@ -13,6 +13,14 @@ OUT_MEAN_ABS = 2e-3
 LSE_ABS = 1e-3
 
 
+def noalloc_too_large_problem():
+    """A problem whose plan exceeds the allocation-free entry's 32 MiB array: 16384 sequences
+    of 128 tokens, 64 query and KV heads, FULL mask -- about a million 64-byte work items.
+    Returns (cu_seqlens, keyword arguments)."""
+    cq = (np.arange(16384 + 1) * 128).astype(np.int32)
+    return cq, dict(hq=64, hkv=64, head_dim=128)
+
+
 def device_inputs(wl, dev="cuda"):
     q = wl.q.to(dev)
     if wl.paged:

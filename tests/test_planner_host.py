@@ -84,3 +84,12 @@ def test_job_lists_are_shared_across_heads(attn_lib, kind):
     assert grown <= (eight["work_items"] - one["work_items"]) * (64 + 4) + 4 * (eight["ctas"] + 1) + 8 * 256
     # copies of the 16-byte jobs per head would exceed that bound by more than its slack
     assert 16 * (eight["jobs"] - one["jobs"]) > 8 * 256
+
+
+def test_noalloc_size_limit_premise(attn_lib):
+    """The GPU test of the allocation-free entry's size limit relies on this problem needing
+    more than its 32 MiB array (the limit is checked on the same host plan)."""
+    from tests import gpu_helpers as G
+    cq, kw = G.noalloc_too_large_problem()
+    st = attn_lib.attn_plan_dry_run(cu_seqlens_q=cq, cu_seqlens_k=cq, mask=W.MaskSpec("FULL"), kv_splits=1, **kw)
+    assert st["workspace_bytes"] > 1.5 * attn_lib.NOALLOC_SCRATCH_BYTES

@@ -45,12 +45,12 @@ def test_noalloc_matches_regular_entry_two_calls_in_a_row(attn_lib):
 
 
 def test_noalloc_rejects_plans_beyond_its_scratch(attn_lib):
-    # FULL attention over 65536 tokens x 32 heads needs a ~67 MB work list: rejected before
-    # any device work (no tensors are touched)
-    cq = np.array([0, 65536], np.int32)
+    # 16384 sequences of 128 tokens x 64 heads: about a million 64-byte work items (68 MiB,
+    # see the CPU test of this premise), rejected before any device work (no tensors are touched)
+    cq, kw = G.noalloc_too_large_problem()
     with pytest.raises(M.AttnError) as e:
-        M.attn_masked_fwd_noalloc(hq=32, hkv=32, head_dim=128, cu_seqlens_q=cq, cu_seqlens_k=cq,
-                                  mask=W.MaskSpec("FULL"), q=None, k=None, v=None, out=None)
+        M.attn_masked_fwd_noalloc(cu_seqlens_q=cq, cu_seqlens_k=cq, mask=W.MaskSpec("FULL"), q=None, k=None,
+                                  v=None, out=None, **kw)
     assert e.value.status == 7
     with pytest.raises(M.AttnError) as e:
         wl = W.random_small(seed=3, kind="CUSTOM", batch=2)
