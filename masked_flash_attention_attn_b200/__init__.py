@@ -218,12 +218,14 @@ def _mask_desc(m: _Marshal, mask, device_bits=None):
 
 
 class Plan:
-    """Owns an attn_plan_t. Keeps the device page table (read by every forward) alive."""
+    """Owns an attn_plan_t. Keeps the device page table (read by every forward) alive and
+    remembers the sizes the tensors of its calls must have."""
 
-    def __init__(self, handle, page_table, hq, head_dim, total_q):
+    def __init__(self, handle, page_table, hq, head_dim, total_q, hkv=None, kv_rows=None):
         self.handle = handle
         self._page_table = page_table
         self.hq, self.head_dim, self.total_q = hq, head_dim, total_q
+        self.hkv, self.kv_rows = hkv, kv_rows   # kv_rows: total keys, or pages x page size
 
     def __del__(self):
         if getattr(self, "handle", None):
@@ -263,20 +265,80 @@ def attn_plan(*, hq: int, hkv: int, head_dim: int, cu_seqlens_q, mask, cu_seqlen
     else:
         _check(lib().attn_plan(ctypes.byref(pr), ctypes.byref(d), _stream(stream), ctypes.byref(h)), "attn_plan")
     total_q = int(np.asarray(cu_seqlens_q)[-1])
-    return Plan(h.value, page_table, hq, head_dim, total_q)
+    kv_rows = int(np.asarray(cu_seqlens_k)[-1]) if cu_seqlens_k is not None else int(num_pages) * int(page_size)
+    return Plan(h.value, page_table, hq, head_dim, total_q, hkv=hkv, kv_rows=kv_rows)
+
+
+def _tensors(*specs):
+    """Device pointers of tensor arguments after checking them. Each spec is (tensor, name,
+    dtypes, least numel or None, optional): a torch tensor of one of ``dtypes``, contiguous,
+    with at least that many elements; then every one must be on a CUDA device. The C ABI
+    takes bare pointers and cannot see sizes; a wrong tensor would be read or written out
+    of bounds, so it is refused here."""
+    import torch
+    for t, name, dtypes, numel, optional in specs:
+        if t is None:
+            if optional:
+                continue
+            raise ValueError(f"{name} is required")
+        if not isinstance(t, torch.Tensor):
+            raise TypeError(f"{name} must be a torch tensor")
+        if t.dtype not in dtypes:
+            raise TypeError(f"{name} must be {' or '.join(str(d) for d in dtypes)}, not {t.dtype}")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+        if numel is not None and t.numel() < numel:
+            raise ValueError(f"{name} has {t.numel()} elements; the plan needs {numel}")
+    for t, name, *_ in specs:
+        if t is not None and not t.is_cuda:
+            raise ValueError(f"{name} must be a CUDA tensor")
+    return [None if t is None else t.data_ptr() for t, *_ in specs]
+
+
+def _bf16():
+    import torch
+    return (torch.bfloat16,)
+
+
+def _f32():
+    import torch
+    return (torch.float32,)
+
+
+def _bytes():
+    import torch
+    return (torch.uint8, torch.float8_e4m3fn)
+
+
+def _sizes(plan: Plan):
+    """(q / out elements, k / v elements, lse elements) of a plan; None where unknown."""
+    qn = plan.total_q * plan.hq * plan.head_dim
+    kn = plan.kv_rows * plan.hkv * plan.head_dim if plan.kv_rows is not None and plan.hkv else None
+    return qn, kn, plan.total_q * plan.hq
 
 
 def attn_masked_fwd(plan: Plan, q, k, v, out, lse=None, stream=None) -> None:
-    """attn_masked_fwd(): enqueue the forward on ``stream`` (default: torch's current stream)."""
-    _check(lib().attn_masked_fwd(plan.handle, _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _stream(stream)),
-           "attn_masked_fwd")
+    """attn_masked_fwd(): enqueue the forward on ``stream`` (default: torch's current stream).
+    q, out: bf16 [total_q, hq, d]; k, v: bf16 [total_k, hkv, d] or paged caches; lse: fp32
+    [total_q, hq] or None."""
+    qn, kn, ln = _sizes(plan)
+    b, f = _bf16(), _f32()
+    args = _tensors((q, "q", b, qn, False), (k, "k", b, kn, False), (v, "v", b, kn, False),
+                    (out, "out", b, qn, False), (lse, "lse", f, ln, True))
+    _check(lib().attn_masked_fwd(plan.handle, *args, _stream(stream)), "attn_masked_fwd")
 
 
 def attn_masked_bwd(plan: Plan, q, k, v, out, lse, dout, dq, dk, dv, stream=None, dlse=None) -> None:
     """attn_masked_bwd(): enqueue dq, dk, dv for the gradient dout of out and, optionally,
-    dlse of lse (plan from attn_plan(..., backward=True))."""
-    _check(lib().attn_masked_bwd(plan.handle, _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dout),
-                                 _ptr(dlse), _ptr(dq), _ptr(dk), _ptr(dv), _stream(stream)), "attn_masked_bwd")
+    dlse of lse (plan from attn_plan(..., backward=True)). Shapes as in attn_masked_fwd;
+    dq like q, dk / dv like k / v, dout like out, dlse like lse."""
+    qn, kn, ln = _sizes(plan)
+    b, f = _bf16(), _f32()
+    args = _tensors((q, "q", b, qn, False), (k, "k", b, kn, False), (v, "v", b, kn, False),
+                    (out, "out", b, qn, False), (lse, "lse", f, ln, False), (dout, "dout", b, qn, False),
+                    (dlse, "dlse", f, ln, True), (dq, "dq", b, qn, False), (dk, "dk", b, kn, False),
+                    (dv, "dv", b, kn, False))
+    _check(lib().attn_masked_bwd(plan.handle, *args, _stream(stream)), "attn_masked_bwd")
 
 
 def attn_plan_get_tile_classes(plan: Plan) -> np.ndarray:
@@ -390,16 +452,20 @@ def backward(plan: Plan, q, k, v, out, lse, dout, stream=None, dlse=None):
 
 def attn_fp8_transpose_v(plan: Plan, v8, vt8, ldv: int, stream=None) -> None:
     """attn_fp8_transpose_v(): e4m3 V [total_k, hkv, d] -> vt [hkv, d, ldv] (uint8 tensors)."""
-    _check(lib().attn_fp8_transpose_v(plan.handle, _ptr(v8), _ptr(vt8), int(ldv), _stream(stream)),
-           "attn_fp8_transpose_v")
+    by = _bytes()
+    pv, pvt = _tensors((v8, "v8", by, None, False), (vt8, "vt8", by, None, False))
+    _check(lib().attn_fp8_transpose_v(plan.handle, pv, pvt, int(ldv), _stream(stream)), "attn_fp8_transpose_v")
 
 
 def attn_masked_fwd_fp8(plan: Plan, q8, k8, vt8, ldv: int, q_scale: float, k_scale: float, v_scale: float, out,
                         lse=None, stream=None) -> None:
     """attn_masked_fwd_fp8(): e4m3 q, k (uint8 tensors) and transposed v with per-tensor scales."""
-    _check(lib().attn_masked_fwd_fp8(plan.handle, _ptr(q8), _ptr(k8), _ptr(vt8), int(ldv), float(q_scale),
-                                     float(k_scale), float(v_scale), _ptr(out), _ptr(lse), _stream(stream)),
-           "attn_masked_fwd_fp8")
+    by = _bytes()
+    pq, pk, pvt, po, pl = _tensors((q8, "q8", by, None, False), (k8, "k8", by, None, False),
+                                   (vt8, "vt8", by, None, False), (out, "out", _bf16(), None, False),
+                                   (lse, "lse", _f32(), None, True))
+    _check(lib().attn_masked_fwd_fp8(plan.handle, pq, pk, pvt, int(ldv), float(q_scale), float(k_scale),
+                                     float(v_scale), po, pl, _stream(stream)), "attn_masked_fwd_fp8")
 
 
 def attn_test_transpose_mask_tile(tile_words: np.ndarray) -> np.ndarray:

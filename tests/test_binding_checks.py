@@ -1,0 +1,85 @@
+"""CPU tests of the binding's tensor checks: the C ABI takes bare pointers, so the binding
+refuses, before any library call, tensors of the wrong type, layout or size and tensors
+that are not on a CUDA device."""
+import pytest
+import torch
+
+import masked_flash_attention_attn_b200 as M
+
+
+def _plan():
+    # a plan object without a library handle: only its sizes are used by the checks
+    return M.Plan(None, None, hq=4, head_dim=64, total_q=10, hkv=2, kv_rows=12)
+
+
+def _good():
+    bf = torch.bfloat16
+    return dict(q=torch.zeros(10, 4, 64, dtype=bf), k=torch.zeros(12, 2, 64, dtype=bf),
+                v=torch.zeros(12, 2, 64, dtype=bf), out=torch.zeros(10, 4, 64, dtype=bf),
+                lse=torch.zeros(10, 4, dtype=torch.float32))
+
+
+def _fwd(**kw):
+    a = _good()
+    a.update(kw)
+    M.attn_masked_fwd(_plan(), a["q"], a["k"], a["v"], a["out"], a["lse"])
+
+
+def test_right_tensors_fail_only_for_not_being_on_a_gpu():
+    with pytest.raises(ValueError, match="CUDA"):
+        _fwd()
+
+
+@pytest.mark.parametrize("name", ["q", "k", "v", "out"])
+def test_wrong_dtype(name):
+    t = _good()[name].float()
+    with pytest.raises(TypeError, match=name):
+        _fwd(**{name: t})
+
+
+def test_lse_dtype_and_optional():
+    with pytest.raises(TypeError, match="lse"):
+        _fwd(lse=torch.zeros(10, 4, dtype=torch.bfloat16))
+    with pytest.raises(ValueError, match="CUDA"):   # lse may be omitted
+        _fwd(lse=None)
+
+
+@pytest.mark.parametrize("name,shape", [("q", (9, 4, 64)), ("k", (11, 2, 64)), ("v", (12, 2, 32)),
+                                        ("out", (10, 3, 64)), ("lse", (10, 3))])
+def test_too_small(name, shape):
+    dt = torch.float32 if name == "lse" else torch.bfloat16
+    with pytest.raises(ValueError, match=name):
+        _fwd(**{name: torch.zeros(*shape, dtype=dt)})
+
+
+def test_not_contiguous_and_not_a_tensor():
+    with pytest.raises(ValueError, match="contiguous"):
+        _fwd(q=torch.zeros(64, 4, 10, dtype=torch.bfloat16).transpose(0, 2))
+    with pytest.raises(TypeError, match="torch tensor"):
+        _fwd(k=[0.0] * 10)
+    with pytest.raises(ValueError, match="required"):
+        _fwd(out=None)
+
+
+def test_backward_checks_every_tensor():
+    a = _good()
+    g = dict(dout=a["out"].clone(), dq=a["q"].clone(), dk=a["k"].clone(), dv=a["v"].clone())
+    with pytest.raises(ValueError, match="CUDA"):
+        M.attn_masked_bwd(_plan(), a["q"], a["k"], a["v"], a["out"], a["lse"], g["dout"], g["dq"], g["dk"], g["dv"])
+    with pytest.raises(ValueError, match="dk"):
+        M.attn_masked_bwd(_plan(), a["q"], a["k"], a["v"], a["out"], a["lse"], g["dout"], g["dq"],
+                          a["k"][:5].clone(), g["dv"])
+    with pytest.raises(ValueError, match="lse is required"):
+        M.attn_masked_bwd(_plan(), a["q"], a["k"], a["v"], a["out"], None, g["dout"], g["dq"], g["dk"], g["dv"])
+    with pytest.raises(TypeError, match="dlse"):
+        M.attn_masked_bwd(_plan(), a["q"], a["k"], a["v"], a["out"], a["lse"], g["dout"], g["dq"], g["dk"], g["dv"],
+                          dlse=a["lse"].double())
+
+
+def test_e4m3_inputs_are_bytes():
+    z = torch.zeros(64, dtype=torch.uint8)
+    out = torch.zeros(10, 4, 64, dtype=torch.bfloat16)
+    with pytest.raises(TypeError, match="q8"):
+        M.attn_masked_fwd_fp8(_plan(), z.float(), z, z, 16, 1.0, 1.0, 1.0, out)
+    with pytest.raises(ValueError, match="CUDA"):
+        M.attn_masked_fwd_fp8(_plan(), z, z.view(torch.float8_e4m3fn), z, 16, 1.0, 1.0, 1.0, out)
