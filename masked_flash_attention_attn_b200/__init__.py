@@ -418,8 +418,15 @@ def attn_masked_fwd_noalloc(*, hq: int, hkv: int, head_dim: int, cu_seqlens_q, m
     pr = _problem(m, hq=hq, hkv=hkv, head_dim=head_dim, cu_seqlens_q=cu_seqlens_q, cu_seqlens_k=cu_seqlens_k,
                   kv_lens=kv_lens, page_table=page_table, page_size=page_size, num_pages=num_pages, scale=scale)
     d = _mask_desc(m, mask)
-    _check(lib().attn_masked_fwd_noalloc(ctypes.byref(pr), ctypes.byref(d), _ptr(q), _ptr(k), _ptr(v), _ptr(out),
-                                         _ptr(lse), _stream(stream)), "attn_masked_fwd_noalloc")
+    total_q = int(np.asarray(cu_seqlens_q)[-1])
+    kv_rows = int(np.asarray(cu_seqlens_k)[-1]) if cu_seqlens_k is not None else int(num_pages) * int(page_size)
+    qn, kn = total_q * hq * head_dim, kv_rows * hkv * head_dim
+    b = _bf16()
+    # a missing tensor is left to the C side, which reports it after its own size limit
+    args = _tensors((q, "q", b, qn, True), (k, "k", b, kn, True), (v, "v", b, kn, True), (out, "out", b, qn, True),
+                    (lse, "lse", _f32(), total_q * hq, True))
+    _check(lib().attn_masked_fwd_noalloc(ctypes.byref(pr), ctypes.byref(d), *args, _stream(stream)),
+           "attn_masked_fwd_noalloc")
 
 
 def attn_test_exp2_poly(x, y, stream=None) -> None:

@@ -83,3 +83,15 @@ def test_e4m3_inputs_are_bytes():
         M.attn_masked_fwd_fp8(_plan(), z.float(), z, z, 16, 1.0, 1.0, 1.0, out)
     with pytest.raises(ValueError, match="CUDA"):
         M.attn_masked_fwd_fp8(_plan(), z, z.view(torch.float8_e4m3fn), z, 16, 1.0, 1.0, 1.0, out)
+
+
+def test_noalloc_checks_the_tensors_it_is_given():
+    import numpy as np
+    import workloads as W
+    a = _good()
+    cq, ck = np.array([0, 10], np.int32), np.array([0, 12], np.int32)
+    kw = dict(hq=4, hkv=2, head_dim=64, cu_seqlens_q=cq, cu_seqlens_k=ck, mask=W.MaskSpec("CAUSAL"))
+    with pytest.raises(ValueError, match="CUDA"):
+        M.attn_masked_fwd_noalloc(**kw, **a)
+    with pytest.raises(ValueError, match="v has"):
+        M.attn_masked_fwd_noalloc(**kw, **dict(a, v=a["v"][:3].clone()))
