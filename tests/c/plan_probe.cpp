@@ -1,8 +1,8 @@
 // The host planner (attn_plan.cpp) built against host-memory stand-ins for the CUDA runtime
 // calls it makes, so that a test can run attn_plan() without a GPU and read the workspace it
-// would upload: the work items, their jobs and the 2 KiB partial-tile masks. The kernel
-// launchers are stubs that report "unsupported"; CUSTOM masks (scanned by a device kernel)
-// therefore fail to plan here. Test infrastructure only.
+// would upload: the work items, their jobs and the 2 KiB partial-tile masks. The attention
+// launchers are stubs that report "unsupported"; the CUSTOM mask scan runs as host code
+// written from the scan kernels' contracts. Test infrastructure only.
 #include <cstdlib>
 #include <cstring>
 
@@ -63,14 +63,47 @@ attn_status_t mfa_launch_backward(const attn_plan_t*, const void*, const void*, 
                                   const void*, const float*, void*, void*, void*, cudaStream_t) {
   return ATTN_ERR_UNSUPPORTED;
 }
+// Host versions of the two CUSTOM-mask kernels, from their stated contracts (the device
+// kernels themselves are checked on the GPU): count = visible keys of every (R-row block,
+// 128-key tile) of a task's 32 key tiles; repack = 128 rows x 4 words per tile, query row
+// rb * R + r % R, bits past L_k or past the sequence's rows cleared.
 namespace mfa {
-cudaError_t launch_custom_count(const uint32_t*, const CustomSeq*, const CountTask*, int, int, int32_t*,
-                                cudaStream_t) {
-  return cudaErrorNotSupported;
+namespace {
+uint32_t row_word(const uint32_t* bits, const CustomSeq& s, int64_t i, int64_t w) {
+  const int64_t W = (int64_t(s.lk) + 31) / 32;
+  if (i >= s.lq || w >= W) return 0u;
+  const int64_t rem = int64_t(s.lk) - 32 * w;
+  const uint32_t valid = rem >= 32 ? 0xffffffffu : ((1u << rem) - 1u);
+  return bits[s.word_off + i * W + w] & valid;
 }
-cudaError_t launch_custom_repack(const uint32_t*, const CustomSeq*, const RepackTask*, int, int, uint4*,
-                                 cudaStream_t) {
-  return cudaErrorNotSupported;
+}  // namespace
+cudaError_t launch_custom_count(const uint32_t* bits, const CustomSeq* seqs, const CountTask* tasks, int ntasks,
+                                int R, int32_t* counts, cudaStream_t) {
+  for (int n = 0; n < ntasks; ++n) {
+    const CountTask& t = tasks[n];
+    const CustomSeq& s = seqs[t.seq];
+    for (int kt = t.kt0; kt < std::min(s.n_kt, t.kt0 + 32); ++kt) {
+      int32_t c = 0;
+      for (int64_t i = int64_t(t.rb) * R; i < std::min<int64_t>(s.lq, int64_t(t.rb + 1) * R); ++i)
+        for (int j = 0; j < 4; ++j) c += __builtin_popcount(row_word(bits, s, i, int64_t(kt) * 4 + j));
+      counts[s.cnt_off + int64_t(t.rb) * s.n_kt + kt] = c;
+    }
+  }
+  return cudaSuccess;
+}
+cudaError_t launch_custom_repack(const uint32_t* bits, const CustomSeq* seqs, const RepackTask* tasks, int ntasks,
+                                 int R, uint4* tiles, cudaStream_t) {
+  for (int n = 0; n < ntasks; ++n) {
+    const RepackTask& t = tasks[n];
+    const CustomSeq& s = seqs[t.seq];
+    for (int r = 0; r < 128; ++r) {
+      const int64_t i = int64_t(t.rb) * R + r % R;
+      uint32_t w[4];
+      for (int j = 0; j < 4; ++j) w[j] = row_word(bits, s, i, int64_t(t.kt) * 4 + j);
+      tiles[int64_t(t.idx) * 128 + r] = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+  }
+  return cudaSuccess;
 }
 }  // namespace mfa
 

@@ -2,7 +2,7 @@
 
 tests/c/plan_probe.cpp builds the host planner with host-memory stand-ins for the CUDA
 runtime, so attn_plan() / attn_plan_bwd() run here and their workspace (what the kernels
-would read) can be inspected. For random problems of every analytic kind:
+would read) can be inspected. For random problems of every kind:
   * every (sequence, query head, query row) is covered by exactly one forward work item
     (or, split, by ranges of one), and an item's jobs are exactly the key tiles where the
     oracle's dense mask has a visible pair for that query tile;
@@ -12,7 +12,8 @@ would read) can be inspected. For random problems of every analytic kind:
     zero elsewhere;
   * the backward lists (dQ items by query tile, dK/dV items by key tile) satisfy the same,
     with the key-major tiles the exact transposes of the query-major ones.
-CUSTOM masks are scanned by a device kernel and are not planned here.
+CUSTOM masks go through host versions of the two scan kernels written from their contracts
+(tests/c/plan_probe.cpp), so their host-side planning is covered as well.
 """
 import ctypes
 import os
@@ -28,7 +29,7 @@ from oracle import masks as OM
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 CSRC = os.path.join(ROOT, "masked_flash_attention_attn_b200", "csrc")
 FULL, NONE = -1, -2
-KINDS = ["FULL", "CAUSAL", "SLIDING_WINDOW", "PREFIX_LM", "CHUNK_CAUSAL", "RANGES", "BLOCK_SPARSE"]
+KINDS = ["FULL", "CAUSAL", "SLIDING_WINDOW", "PREFIX_LM", "CHUNK_CAUSAL", "RANGES", "BLOCK_SPARSE", "CUSTOM"]
 
 
 @pytest.fixture(scope="module")
@@ -61,11 +62,16 @@ def _plan(probe, M, wl, spec, kv_splits=1, backward=False):
     else:
         kw.update(cu_seqlens_k=wl.cu_seqlens_k)
     pr = M._problem(m, **kw)
-    d = M._mask_desc(m, spec)
+    bits = None
+    if spec.kind == "CUSTOM":   # "device" words: host memory under the probe's stand-ins
+        import torch
+        bits = torch.from_numpy(np.ascontiguousarray(spec.bits.astype(np.uint32).view(np.int32)))
+    d = M._mask_desc(m, spec, bits)
     h = ctypes.c_void_p()
     fn = probe.attn_plan_bwd if backward else probe.attn_plan
     st = fn(ctypes.addressof(pr), ctypes.addressof(d), None, ctypes.addressof(h))
     assert st == 0, M.STATUS.get(st, st)
+    h.keep = bits
     return h
 
 
@@ -168,14 +174,14 @@ def test_forward_workspace_matches_oracle(attn_lib, probe, kind, seed):
     _forward_check(probe, attn_lib, wl, wl.masks[0], kv_splits=1)
 
 
-@pytest.mark.parametrize("kind", ["CAUSAL", "PREFIX_LM", "RANGES", "BLOCK_SPARSE"])
+@pytest.mark.parametrize("kind", ["CAUSAL", "PREFIX_LM", "RANGES", "BLOCK_SPARSE", "CUSTOM"])
 def test_forward_workspace_short_queries_packed_heads(attn_lib, probe, kind):
     """Queries of at most 60 rows: several heads share one 128-row tile."""
     wl = W.random_small(seed=41, kind=kind, batch=4, hq=8, hkv=1, d=64, lmin=1, lmax=60)
     _forward_check(probe, attn_lib, wl, wl.masks[0], kv_splits=1)
 
 
-@pytest.mark.parametrize("kind", ["CAUSAL", "SLIDING_WINDOW", "RANGES"])
+@pytest.mark.parametrize("kind", ["CAUSAL", "SLIDING_WINDOW", "RANGES", "CUSTOM"])
 def test_forward_workspace_split_and_paged(attn_lib, probe, kind):
     """Forced split-KV ranges still cover every visible key tile once; paged lengths."""
     wl = W.random_small(seed=57, kind=kind, batch=3, hq=4, hkv=2, d=128, lmin=200, lmax=900)
