@@ -125,6 +125,28 @@ int probe_forward(const attn_plan_t* p, const void** items, const void** jobs, c
   return 0;
 }
 
+// The host plan of the allocation-free entry (the bytes it copies into its fixed array):
+// the same pointers as probe_forward, into a plan object the caller frees with
+// probe_host_plan_free.
+void* probe_host_plan(const attn_problem_t* problem, const attn_mask_desc_t* mask, int* status, const void** items,
+                      const void** jobs, const void** tiles, int64_t* n_items, int64_t* n_tiles, int64_t* bytes) {
+  auto* hp = new mfa_host_plan();
+  *status = int(mfa_plan_host(problem, mask, 148, hp));
+  if (*status != ATTN_OK) {
+    delete hp;
+    return nullptr;
+  }
+  const char* b = hp->bytes.data();
+  *items = b + hp->off_items;
+  *jobs = b + hp->off_jobs;
+  *tiles = b + hp->off_tiles;
+  *n_items = reinterpret_cast<const int32_t*>(b + hp->off_cta_off)[hp->meta.ctas];   // every item listed once
+  *n_tiles = (hp->bytes.size() - hp->off_tiles) / kMaskTileBytes;
+  *bytes = int64_t(hp->bytes.size());
+  return hp;
+}
+void probe_host_plan_free(void* hp) { delete static_cast<mfa_host_plan*>(hp); }
+
 // The backward lists of an attn_plan_bwd() plan: dQ and dK/dV items (32-byte BwdItem), their
 // jobs (16-byte BwdJob) and the query-major / key-major mask tiles.
 int probe_backward(const attn_plan_t* p, const void** q_items, const void** q_jobs, const void** kv_items,

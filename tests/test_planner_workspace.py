@@ -50,6 +50,10 @@ def probe(tmp_path_factory):
     lib.probe_forward.argtypes = [vp] + [ctypes.POINTER(vp)] * 3 + [ctypes.POINTER(ctypes.c_int64)] * 2 + \
         [ctypes.POINTER(ctypes.c_int32)] * 3
     lib.probe_backward.argtypes = [vp] + [ctypes.POINTER(vp)] * 6 + [ctypes.POINTER(ctypes.c_int64)] * 2
+    lib.probe_host_plan.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_int)] + [ctypes.POINTER(vp)] * 3 + \
+        [ctypes.POINTER(ctypes.c_int64)] * 3
+    lib.probe_host_plan.restype = vp
+    lib.probe_host_plan_free.argtypes = [vp]
     return lib
 
 
@@ -260,3 +264,42 @@ def test_backward_workspace_matches_oracle(attn_lib, probe, kind):
                 if dense[seq][q0:q0 + 128, k0:k0 + krows].any()}
         assert pairs == need, (kind, "dkv", seq, kvh, k0)
     assert seen_k == {(b, kh, k0) for b in range(wl.batch) for kh in range(wl.hkv) for k0 in range(0, wl.lk(b), 128)}
+
+
+@pytest.mark.parametrize("kind", ["CAUSAL", "SLIDING_WINDOW", "CHUNK_CAUSAL", "RANGES", "BLOCK_SPARSE"])
+def test_allocation_free_host_plan_equals_the_plan_workspace(attn_lib, probe, kind):
+    """attn_masked_fwd_noalloc copies a host plan into its fixed array; that plan's items,
+    jobs and mask tiles equal those attn_plan (never splitting) uploads."""
+    M = attn_lib
+    wl = W.random_small(seed=90 + len(kind), kind=kind, batch=3, hq=8, hkv=2, d=128, lmin=1, lmax=700)
+    spec = wl.masks[0]
+    h = _plan(probe, M, wl, spec, kv_splits=1)
+    vp, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32
+    try:
+        pi, pj, pt, ni, nt, R, hp, nq = vp(), vp(), vp(), i64(), i64(), i32(), i32(), i32()
+        assert probe.probe_forward(h, ctypes.byref(pi), ctypes.byref(pj), ctypes.byref(pt), ctypes.byref(ni),
+                                   ctypes.byref(nt), ctypes.byref(R), ctypes.byref(hp), ctypes.byref(nq)) == 0
+        items = _array(pi.value, ni.value, 16)
+        n_jobs = int((items[:, 10] + items[:, 11]).max())
+        jobs = _array(pj.value, n_jobs, 4)
+        tiles = _tile_bits(pt.value, nt.value)
+    finally:
+        probe.attn_plan_destroy(h)
+    m = M._Marshal()
+    pr = M._problem(m, hq=wl.hq, hkv=wl.hkv, head_dim=wl.d, cu_seqlens_q=wl.cu_seqlens_q,
+                    cu_seqlens_k=wl.cu_seqlens_k)
+    d = M._mask_desc(m, spec)
+    st = ctypes.c_int()
+    hi, hj, ht, hni, hnt, nbytes = vp(), vp(), vp(), i64(), i64(), i64()
+    hplan = probe.probe_host_plan(ctypes.addressof(pr), ctypes.addressof(d), ctypes.byref(st), ctypes.byref(hi),
+                                  ctypes.byref(hj), ctypes.byref(ht), ctypes.byref(hni), ctypes.byref(hnt),
+                                  ctypes.byref(nbytes))
+    assert st.value == 0 and hplan
+    try:
+        h_items = _array(hi.value, hni.value, 16)
+        h_jobs = _array(hj.value, n_jobs, 4)
+        h_tiles = _tile_bits(ht.value, hnt.value)
+    finally:
+        probe.probe_host_plan_free(hplan)
+    assert np.array_equal(h_items, items) and np.array_equal(h_jobs, jobs) and np.array_equal(h_tiles, tiles)
+    assert nbytes.value <= M.NOALLOC_SCRATCH_BYTES
