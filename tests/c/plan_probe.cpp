@@ -125,6 +125,14 @@ int probe_forward(const attn_plan_t* p, const void** items, const void** jobs, c
   return 0;
 }
 
+// Split-KV: the merge list (32-byte MergeTile: tok, head, rows, slot0, nsplit, stride).
+int probe_merge(const attn_plan_t* p, const void** merge, int64_t* n) {
+  if (!p) return 1;
+  *merge = p->d_merge;
+  *n = p->n_merge;
+  return 0;
+}
+
 // The host plan of the allocation-free entry (the bytes it copies into its fixed array):
 // the same pointers as probe_forward, into a plan object the caller frees with
 // probe_host_plan_free.

@@ -54,6 +54,7 @@ def probe(tmp_path_factory):
         [ctypes.POINTER(ctypes.c_int64)] * 3
     lib.probe_host_plan.restype = vp
     lib.probe_host_plan_free.argtypes = [vp]
+    lib.probe_merge.argtypes = [vp, ctypes.POINTER(vp), ctypes.POINTER(ctypes.c_int64)]
     return lib
 
 
@@ -113,6 +114,28 @@ def _check_block(dense, r0, nrows, k0, lk, mask, what):
     return bool(blk.any())
 
 
+def _check_merge(items, merge, nq):
+    """Split-KV bookkeeping: every partial slot is written by exactly one key range, and the
+    merge list names, for each split query tile, exactly the slots of its ranges."""
+    slots = {}
+    for it in items:
+        if it[13] < 0:
+            continue
+        for t in range(nq):
+            if it[6 + t] > 0:
+                slot = int(it[13]) + t
+                assert slot not in slots, "a partial slot written twice"
+                slots[slot] = (int(it[4 + t]), int(it[8 + t]), int(it[6 + t]))
+    listed = set()
+    for tok, head, rows, slot0, nsplit, stride, _, _ in merge:
+        assert nsplit >= 2
+        mine = {int(slot0) + c * int(stride) for c in range(nsplit)}
+        assert all(slots.get(x) == (tok, head, rows) for x in mine), "merge tile and its ranges disagree"
+        assert not (mine & listed)
+        listed |= mine
+    assert listed == set(slots), "every partial slot is merged once"
+
+
 def _forward_check(probe, M, wl, spec, kv_splits):
     h = _plan(probe, M, wl, spec, kv_splits=kv_splits)
     try:
@@ -124,9 +147,13 @@ def _forward_check(probe, M, wl, spec, kv_splits):
         n_jobs = int((items[:, 10] + items[:, 11]).max()) if len(items) else 0
         jobs = _array(pj.value, n_jobs, 4)
         tiles = _tile_bits(pt.value, nt.value)
+        pm, nm = vp(), i64()
+        assert probe.probe_merge(h, ctypes.byref(pm), ctypes.byref(nm)) == 0
+        merge = _array(pm.value, nm.value, 8)
     finally:
         probe.attn_plan_destroy(h)
     R, hp, nq = R.value, hp.value, nq.value
+    _check_merge(items, merge, nq)
     dense = _dense(wl, spec)
     cq = wl.cu_seqlens_q
     covered = np.zeros((int(cq[-1]), wl.hq), np.int32)
@@ -168,6 +195,7 @@ def _forward_check(probe, M, wl, spec, kv_splits):
         need = {kt for kt in range(-(-lk // 128)) if dense[seq][r0:r0 + rows, kt * 128:kt * 128 + 128].any()}
         assert vis == need, (spec.kind, seq, head, r0)
     assert used_tiles.all()
+    return len(merge)
 
 
 @pytest.mark.parametrize("kind", KINDS)
@@ -189,7 +217,7 @@ def test_forward_workspace_short_queries_packed_heads(attn_lib, probe, kind):
 def test_forward_workspace_split_and_paged(attn_lib, probe, kind):
     """Forced split-KV ranges still cover every visible key tile once; paged lengths."""
     wl = W.random_small(seed=57, kind=kind, batch=3, hq=4, hkv=2, d=128, lmin=200, lmax=900)
-    _forward_check(probe, attn_lib, wl, wl.masks[0], kv_splits=3)
+    assert _forward_check(probe, attn_lib, wl, wl.masks[0], kv_splits=3) > 0
     wp = W.random_small(seed=58, kind=kind, batch=3, hq=4, hkv=2, d=128, lmin=1, lmax=500, paged=True)
     _forward_check(probe, attn_lib, wp, wp.masks[0], kv_splits=1)
 
