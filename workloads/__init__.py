@@ -308,7 +308,7 @@ def tree_verify_long_paged(seed: int = 6, requests: int = 4) -> Workload:
     return wl
 
 
-CONFIGS = {
+WORKLOADS_BY_NUMBER = {
     1: prefix_lm_small,
     2: gemma2_local_global,
     3: tree_verify_paged,
@@ -319,7 +319,7 @@ CONFIGS = {
 
 
 def config(n: int, **kw) -> Workload:
-    return CONFIGS[n](**kw)
+    return WORKLOADS_BY_NUMBER[n](**kw)
 
 
 def random_small(seed: int, kind: str, batch: int = 3, hq: int = 4, hkv: int = 2, d: int = 64,
