@@ -1240,6 +1240,8 @@ attn_status_t mfa_plan_host(const attn_problem_t* problem, const attn_mask_desc_
     return ATTN_OK;
   } catch (const std::bad_alloc&) {
     return ATTN_ERR_OOM;
+  } catch (...) {
+    return ATTN_ERR_INVALID_ARG;
   }
 }
 
