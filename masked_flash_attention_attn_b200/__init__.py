@@ -199,9 +199,11 @@ def _mask_desc(m: _Marshal, mask, device_bits=None):
         # attn_range_t is six int32 fields: an [n, 6] int32 array has its layout
         counts = [len(per) for per in rs]
         flat = np.zeros((max(1, sum(counts)), 6), np.int32)
-        if sum(counts):
-            flat[:sum(counts)] = np.concatenate([np.asarray(per, dtype=np.int64).reshape(-1, 6)
-                                                 for per in rs if len(per)])
+        parts = [np.asarray(per, dtype=np.int64) for per in rs if len(per)]
+        if any(a.ndim != 2 or a.shape[1] != 6 for a in parts):
+            raise ValueError("each range has six fields (q_start, q_end, k_start, k_end, type, chunk_size)")
+        if parts:
+            flat[:sum(counts)] = np.concatenate(parts)
         cu = np.zeros(len(rs) + 1, np.int32)
         cu[1:] = np.cumsum(counts)
         d.ranges = m.arr(flat, np.int32)

@@ -95,3 +95,12 @@ def test_noalloc_checks_the_tensors_it_is_given():
         M.attn_masked_fwd_noalloc(**kw, **a)
     with pytest.raises(ValueError, match="v has"):
         M.attn_masked_fwd_noalloc(**kw, **dict(a, v=a["v"][:3].clone()))
+
+
+def test_ranges_with_the_wrong_number_of_fields_are_refused(attn_lib):
+    import numpy as np
+    import workloads as W
+    cq = np.array([0, 12], np.int32)
+    bad = W.MaskSpec("RANGES", ranges=[[(0, 12, 0, 12, 1)] * 6])   # five fields: 30 numbers = 5 x 6
+    with pytest.raises(ValueError, match="six fields"):
+        attn_lib.attn_classify_host(hq=1, hkv=1, head_dim=64, cu_seqlens_q=cq, cu_seqlens_k=cq, mask=bad)
