@@ -182,10 +182,37 @@ def _problem(m: _Marshal, *, hq, hkv, head_dim, cu_seqlens_q, cu_seqlens_k=None,
     return pr
 
 
-def _mask_desc(m: _Marshal, mask, device_bits=None):
+def _check_mask_arrays(mask, cu_seqlens_q):
+    """The C side reads the mask's host arrays at indices the lengths imply and cannot see
+    their sizes: check them here."""
+    lq = np.diff(np.asarray(cu_seqlens_q, dtype=np.int64))
+    batch = len(lq)
+    pl = getattr(mask, "prefix_lens", None)
+    if mask.kind == "PREFIX_LM" and pl is not None and len(pl) < batch:
+        raise ValueError(f"prefix_lens has {len(pl)} entries for {batch} sequences")
+    if mask.kind == "RANGES" and len(mask.ranges) < batch:
+        raise ValueError(f"ranges has {len(mask.ranges)} sequences for {batch}")
+    if mask.kind == "CUSTOM" and len(mask.word_offsets) < batch + 1:
+        raise ValueError(f"word_offsets has {len(mask.word_offsets)} entries for {batch} sequences (needs B + 1)")
+    if mask.kind == "BLOCK_SPARSE":
+        bq = int(mask.block_q)
+        if bq < 1:
+            raise ValueError("block_q must be >= 1")
+        rows = int(((lq + bq - 1) // bq).sum())
+        ptr = np.asarray(mask.bsr_row_ptr, dtype=np.int64)
+        if len(ptr) < rows + 1:
+            raise ValueError(f"bsr_row_ptr has {len(ptr)} entries for {rows} block rows (needs rows + 1)")
+        if len(mask.bsr_col_idx) < ptr[rows]:
+            raise ValueError(f"bsr_col_idx has {len(mask.bsr_col_idx)} entries; bsr_row_ptr needs {ptr[rows]}")
+
+
+def _mask_desc(m: _Marshal, mask, device_bits=None, cu_seqlens_q=None):
     """``mask``: an object with the attributes kind, window, prefix_len, prefix_lens, chunk,
     ranges (per-sequence lists of 6-tuples), bits, word_offsets, block_q, block_k,
-    bsr_row_ptr, bsr_col_idx (see include/attn.h)."""
+    bsr_row_ptr, bsr_col_idx (see include/attn.h). With ``cu_seqlens_q`` the host arrays
+    are checked against the batch first."""
+    if cu_seqlens_q is not None:
+        _check_mask_arrays(mask, cu_seqlens_q)
     d = attn_mask_desc_t()
     d.kind = MASK_KIND[mask.kind]
     d.window = int(getattr(mask, "window", 0) or 0)
@@ -259,7 +286,7 @@ def attn_plan(*, hq: int, hkv: int, head_dim: int, cu_seqlens_q, mask, cu_seqlen
             dev_bits = torch.from_numpy(np.ascontiguousarray(b.astype(np.uint32).view(np.int32))).cuda()
         else:
             dev_bits = b
-    d = _mask_desc(m, mask, dev_bits)
+    d = _mask_desc(m, mask, dev_bits, cu_seqlens_q)
     h = ctypes.c_void_p()
     if backward:   # attn_plan_bwd(): forward and backward work lists
         _check(lib().attn_plan_bwd(ctypes.byref(pr), ctypes.byref(d), _stream(stream), ctypes.byref(h)),
@@ -382,7 +409,7 @@ def attn_plan_dry_run(*, hq: int, hkv: int, head_dim: int, cu_seqlens_q, mask, n
                   kv_lens=kv_lens, kv_splits=kv_splits, q_rows=q_rows)
     if kv_lens is not None:
         pr.page_size, pr.max_pages_per_seq, pr.num_pages = page_size, max_pages_per_seq, num_pages
-    d = _mask_desc(m, mask)
+    d = _mask_desc(m, mask, cu_seqlens_q=cu_seqlens_q)
     st = attn_plan_stats_t()
     _check(lib().attn_plan_dry_run(ctypes.byref(pr), ctypes.byref(d), int(num_sms), ctypes.byref(st)),
            "attn_plan_dry_run")
@@ -397,7 +424,7 @@ def attn_classify_host(*, hq: int, hkv: int, head_dim: int, cu_seqlens_q, mask, 
                   kv_lens=kv_lens, kv_splits=kv_splits)
     if kv_lens is not None:
         pr.page_size, pr.max_pages_per_seq, pr.num_pages = page_size, max_pages_per_seq, num_pages
-    d = _mask_desc(m, mask)
+    d = _mask_desc(m, mask, cu_seqlens_q=cu_seqlens_q)
     n, pairs = ctypes.c_size_t(), ctypes.c_int64()
     _check(lib().attn_classify_host(ctypes.byref(pr), ctypes.byref(d), None, 0, ctypes.byref(n), ctypes.byref(pairs)),
            "attn_classify_host")
@@ -419,7 +446,7 @@ def attn_masked_fwd_noalloc(*, hq: int, hkv: int, head_dim: int, cu_seqlens_q, m
     m = _Marshal()
     pr = _problem(m, hq=hq, hkv=hkv, head_dim=head_dim, cu_seqlens_q=cu_seqlens_q, cu_seqlens_k=cu_seqlens_k,
                   kv_lens=kv_lens, page_table=page_table, page_size=page_size, num_pages=num_pages, scale=scale)
-    d = _mask_desc(m, mask)
+    d = _mask_desc(m, mask, cu_seqlens_q=cu_seqlens_q)
     total_q = int(np.asarray(cu_seqlens_q)[-1])
     kv_rows = int(np.asarray(cu_seqlens_k)[-1]) if cu_seqlens_k is not None else int(num_pages) * int(page_size)
     qn, kn = total_q * hq * head_dim, kv_rows * hkv * head_dim

@@ -104,3 +104,21 @@ def test_ranges_with_the_wrong_number_of_fields_are_refused(attn_lib):
     bad = W.MaskSpec("RANGES", ranges=[[(0, 12, 0, 12, 1)] * 6])   # five fields: 30 numbers = 5 x 6
     with pytest.raises(ValueError, match="six fields"):
         attn_lib.attn_classify_host(hq=1, hkv=1, head_dim=64, cu_seqlens_q=cq, cu_seqlens_k=cq, mask=bad)
+
+
+def test_mask_host_arrays_checked_against_the_batch(attn_lib):
+    import numpy as np
+    import workloads as W
+    cq = np.array([0, 100, 300], np.int32)
+    kw = dict(hq=1, hkv=1, head_dim=64, cu_seqlens_q=cq, cu_seqlens_k=cq)
+    cases = [W.MaskSpec("PREFIX_LM", prefix_lens=np.array([4], np.int32)),
+             W.MaskSpec("RANGES", ranges=[[(0, 10, 0, 10, 0, 0)]]),
+             W.MaskSpec("BLOCK_SPARSE", block_q=64, block_k=64, bsr_row_ptr=np.zeros(5, np.int32),
+                        bsr_col_idx=np.zeros(0, np.int32)),   # 2 + 4 block rows need 7 entries
+             W.MaskSpec("BLOCK_SPARSE", block_q=64, block_k=64, bsr_row_ptr=np.full(7, 3, np.int32),
+                        bsr_col_idx=np.zeros(2, np.int32))]
+    for spec in cases:
+        with pytest.raises(ValueError):
+            attn_lib.attn_classify_host(mask=spec, **kw)
+        with pytest.raises(ValueError):
+            attn_lib.attn_plan_dry_run(mask=spec, **kw)
