@@ -182,6 +182,18 @@ def _problem(m: _Marshal, *, hq, hkv, head_dim, cu_seqlens_q, cu_seqlens_k=None,
     return pr
 
 
+def _check_page_table(page_table, cu_seqlens_q):
+    """The kernels read page_table[b][p] for every sequence b: a device int32 [batch,
+    max_pages] tensor with a row per sequence."""
+    if page_table is None:
+        return
+    import torch
+    batch = len(np.asarray(cu_seqlens_q)) - 1
+    if isinstance(page_table, torch.Tensor) and (page_table.dim() != 2 or page_table.shape[0] < batch):
+        raise ValueError(f"page_table must be [batch, max_pages] with at least {batch} rows")
+    _tensors((page_table, "page_table", (torch.int32,), None, False))
+
+
 def _check_mask_arrays(mask, cu_seqlens_q):
     """The C side reads the mask's host arrays at indices the lengths imply and cannot see
     their sizes: check them here."""
@@ -275,6 +287,7 @@ def attn_plan(*, hq: int, hkv: int, head_dim: int, cu_seqlens_q, mask, cu_seqlen
     int32 tensor [batch, max_pages]; CUSTOM ``mask.bits`` may be host (numpy) or device words;
     ``kv_splits``: 0 automatic, 1 never, N >= 2 at most N key ranges per query tile."""
     import torch
+    _check_page_table(page_table, cu_seqlens_q)
     m = _Marshal()
     pr = _problem(m, hq=hq, hkv=hkv, head_dim=head_dim, cu_seqlens_q=cu_seqlens_q, cu_seqlens_k=cu_seqlens_k,
                   kv_lens=kv_lens, page_table=page_table, page_size=page_size, num_pages=num_pages, scale=scale,
@@ -443,6 +456,7 @@ def attn_masked_fwd_noalloc(*, hq: int, hkv: int, head_dim: int, cu_seqlens_q, m
     allocation through its own pool): the plan goes into a fixed 32 MiB array inside the
     library instead of a cudaMalloc'd workspace. Calls that overlap on the GPU race on that
     array; keep them on one stream. CUSTOM masks are not accepted here."""
+    _check_page_table(page_table, cu_seqlens_q)
     m = _Marshal()
     pr = _problem(m, hq=hq, hkv=hkv, head_dim=head_dim, cu_seqlens_q=cu_seqlens_q, cu_seqlens_k=cu_seqlens_k,
                   kv_lens=kv_lens, page_table=page_table, page_size=page_size, num_pages=num_pages, scale=scale)

@@ -122,3 +122,17 @@ def test_mask_host_arrays_checked_against_the_batch(attn_lib):
             attn_lib.attn_classify_host(mask=spec, **kw)
         with pytest.raises(ValueError):
             attn_lib.attn_plan_dry_run(mask=spec, **kw)
+
+
+def test_page_table_checked():
+    import numpy as np
+    import workloads as W
+    cq = np.array([0, 10, 20], np.int32)
+    kw = dict(hq=1, hkv=1, head_dim=64, cu_seqlens_q=cq, kv_lens=np.array([10, 10], np.int32), page_size=16,
+              num_pages=4, mask=W.MaskSpec("CAUSAL"))
+    with pytest.raises(TypeError, match="page_table"):
+        M.attn_plan(page_table=torch.zeros(2, 1, dtype=torch.int64), **kw)
+    with pytest.raises(ValueError, match="rows"):
+        M.attn_plan(page_table=torch.zeros(1, 1, dtype=torch.int32), **kw)
+    with pytest.raises(ValueError, match="CUDA"):
+        M.attn_plan(page_table=torch.zeros(2, 1, dtype=torch.int32), **kw)
