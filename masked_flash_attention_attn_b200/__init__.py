@@ -297,7 +297,8 @@ def attn_plan(*, hq: int, hkv: int, head_dim: int, cu_seqlens_q, mask, cu_seqlen
         b = mask.bits
         if isinstance(b, np.ndarray):
             dev_bits = torch.from_numpy(np.ascontiguousarray(b.astype(np.uint32).view(np.int32))).cuda()
-        else:
+        else:   # device words: 32-bit, contiguous, on the GPU
+            _tensors((b, "mask.bits", (torch.int32, torch.uint32), None, False))
             dev_bits = b
     d = _mask_desc(m, mask, dev_bits, cu_seqlens_q)
     h = ctypes.c_void_p()

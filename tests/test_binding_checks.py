@@ -136,3 +136,15 @@ def test_page_table_checked():
         M.attn_plan(page_table=torch.zeros(1, 1, dtype=torch.int32), **kw)
     with pytest.raises(ValueError, match="CUDA"):
         M.attn_plan(page_table=torch.zeros(2, 1, dtype=torch.int32), **kw)
+
+
+def test_device_mask_bits_checked():
+    import numpy as np
+    import workloads as W
+    cq = np.array([0, 40], np.int32)
+    off = np.array([0, 80], np.int64)
+    kw = dict(hq=1, hkv=1, head_dim=64, cu_seqlens_q=cq, cu_seqlens_k=cq)
+    with pytest.raises(TypeError, match="mask.bits"):
+        M.attn_plan(mask=W.MaskSpec("CUSTOM", bits=torch.zeros(80, dtype=torch.int64), word_offsets=off), **kw)
+    with pytest.raises(ValueError, match="CUDA"):
+        M.attn_plan(mask=W.MaskSpec("CUSTOM", bits=torch.zeros(80, dtype=torch.int32), word_offsets=off), **kw)
