@@ -1095,6 +1095,16 @@ attn_status_t plan_impl(const attn_problem_t* problem, const attn_mask_desc_t* m
   if (e != cudaSuccess) return ATTN_ERR_CUDA;
 
   auto plan = new attn_plan_t();
+  // frees the plan and what it holds on every early return and on an exception
+  struct Guard {
+    attn_plan_t* p;
+    ~Guard() {
+      if (!p) return;
+      if (p->ws) cudaFree(p->ws);
+      if (p->bws) cudaFree(p->bws);
+      delete p;
+    }
+  } guard{plan};
   plan->device = dev;
   fill_meta(s, problem, *plan);
   const int R = plan->R;
@@ -1103,10 +1113,7 @@ attn_status_t plan_impl(const attn_problem_t* problem, const attn_mask_desc_t* m
   RowSource src(mask, s);
   if (mask->kind == ATTN_MASK_CUSTOM) {
     st = custom_counts(mask, s, R, stream, cnts);
-    if (st != ATTN_OK) {
-      delete plan;
-      return st;
-    }
+    if (st != ATTN_OK) return st;
   } else {
     for (int b = 0; b < s.B; ++b) {
       src.prepare(b);
@@ -1151,7 +1158,7 @@ attn_status_t plan_impl(const attn_problem_t* problem, const attn_mask_desc_t* m
 
   e = cudaMalloc(&plan->ws, lay.total);
   if (e != cudaSuccess) {
-    delete plan;
+    plan->ws = nullptr;
     return cuda_status(e);
   }
   plan->ws_bytes = lay.total;
@@ -1181,11 +1188,8 @@ attn_status_t plan_impl(const attn_problem_t* problem, const attn_mask_desc_t* m
   if (st == ATTN_OK && mask->kind == ATTN_MASK_CUSTOM)
     st = custom_repack(mask, s, R, wl.mask_tiles, reinterpret_cast<uint4*>(base + lay.off_tiles), stream);
   if (st == ATTN_OK && with_bwd) st = plan_backward(mask, s, src, num_sms, stream, plan);
-  if (st != ATTN_OK) {
-    cudaFree(plan->ws);
-    delete plan;
-    return st;
-  }
+  if (st != ATTN_OK) return st;
+  guard.p = nullptr;
   *out_plan = plan;
   return ATTN_OK;
 }

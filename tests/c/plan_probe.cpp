@@ -8,14 +8,26 @@
 
 #include <cuda_runtime.h>
 
+static int g_mallocs_left = -1;   // >= 0: that many more allocations succeed, then they fail
+static int g_live = 0;            // device allocations not freed yet
+
 extern "C" {
+void probe_fail_malloc_after(int n) { g_mallocs_left = n; }
+int probe_live_allocations() { return g_live; }
 cudaError_t cudaMalloc(void** p, size_t n) {
+  if (g_mallocs_left == 0) {
+    *p = nullptr;
+    return cudaErrorMemoryAllocation;
+  }
+  if (g_mallocs_left > 0) --g_mallocs_left;
   *p = std::malloc(n ? n : 1);
   if (!*p) return cudaErrorMemoryAllocation;
+  ++g_live;
   std::memset(*p, 0xCD, n);   // "uninitialised device memory": nothing may rely on its value
   return cudaSuccess;
 }
 cudaError_t cudaFree(void* p) {
+  if (p) --g_live;
   std::free(p);
   return cudaSuccess;
 }

@@ -55,6 +55,8 @@ def probe(tmp_path_factory):
     lib.probe_host_plan.restype = vp
     lib.probe_host_plan_free.argtypes = [vp]
     lib.probe_merge.argtypes = [vp, ctypes.POINTER(vp), ctypes.POINTER(ctypes.c_int64)]
+    lib.probe_fail_malloc_after.argtypes = [ctypes.c_int]
+    lib.probe_live_allocations.restype = ctypes.c_int
     return lib
 
 
@@ -331,3 +333,38 @@ def test_allocation_free_host_plan_equals_the_plan_workspace(attn_lib, probe, ki
         probe.probe_host_plan_free(hplan)
     assert np.array_equal(h_items, items) and np.array_equal(h_jobs, jobs) and np.array_equal(h_tiles, tiles)
     assert nbytes.value <= M.NOALLOC_SCRATCH_BYTES
+
+
+@pytest.mark.parametrize("kind", ["CAUSAL", "CUSTOM"])
+def test_failed_device_allocations_are_reported_and_cleaned_up(attn_lib, probe, kind):
+    """Every device allocation of a backward plan failing in turn: attn_plan_bwd reports
+    ATTN_ERR_OOM, returns no plan and frees every device allocation it had made (counted by
+    the probe; a double free would abort this process); afterwards planning works again."""
+    M = attn_lib
+    wl = W.random_small(seed=5, kind=kind, batch=2, hq=4, hkv=2, d=64, lmin=100, lmax=400)
+    spec = wl.masks[0]
+    m = M._Marshal()
+    pr = M._problem(m, hq=wl.hq, hkv=wl.hkv, head_dim=wl.d, cu_seqlens_q=wl.cu_seqlens_q,
+                    cu_seqlens_k=wl.cu_seqlens_k)
+    bits = None
+    if kind == "CUSTOM":
+        import torch
+        bits = torch.from_numpy(np.ascontiguousarray(spec.bits.astype(np.uint32).view(np.int32)))
+    d = M._mask_desc(m, spec, bits)
+    live = probe.probe_live_allocations()
+    try:
+        for n in range(12):
+            probe.probe_fail_malloc_after(n)
+            h = ctypes.c_void_p()
+            st = probe.attn_plan_bwd(ctypes.addressof(pr), ctypes.addressof(d), None, ctypes.addressof(h))
+            if st == 0:
+                probe.attn_plan_destroy(h)
+                assert probe.probe_live_allocations() == live
+                break
+            assert st == 4 and not h.value, (n, st)   # ATTN_ERR_OOM
+            assert probe.probe_live_allocations() == live, f"allocation {n} failed: device memory leaked"
+        else:
+            pytest.fail("a backward plan needs more than 11 allocations")
+        assert n >= 2   # forward workspace and backward workspace at least
+    finally:
+        probe.probe_fail_malloc_after(-1)
