@@ -95,6 +95,22 @@ def test_full_mask_equals_library_softmax():
     np.testing.assert_allclose(lse, torch.logsumexp(s, -1).numpy(), atol=1e-13)
 
 
+def test_masked_rows_equal_library_attention():
+    """With a random boolean mask (every row keeps at least one key) the oracle equals
+    torch's scaled_dot_product_attention in fp64 given the same boolean mask."""
+    g = torch.Generator().manual_seed(12)
+    n, L, d = 29, 53, 32
+    q = torch.randn(n, d, generator=g, dtype=torch.float64)
+    k = torch.randn(L, d, generator=g, dtype=torch.float64)
+    v = torch.randn(L, d, generator=g, dtype=torch.float64)
+    mask = torch.rand(n, L, generator=g) < 0.3
+    mask[torch.arange(n), torch.randint(0, L, (n,), generator=g)] = True
+    ref = torch.nn.functional.scaled_dot_product_attention(q[None, None], k[None, None], v[None, None],
+                                                           attn_mask=mask[None, None], scale=0.3)[0, 0]
+    out, _ = OA.attention_one_head(q.numpy(), k.numpy(), v.numpy(), mask.numpy(), 0.3)
+    np.testing.assert_allclose(out, ref.numpy(), atol=1e-12)
+
+
 def test_lse_merge_over_disjoint_key_sets():
     rng = np.random.default_rng(3)
     n, L, d = 7, 40, 8
