@@ -56,3 +56,24 @@ def test_reference_arm_runs_on_rank0_only(capsys):
 def test_single_process_reduction_is_identity():
     import bench
     assert bench.reduce_over_ranks([3.0, 4.0], 7.0, "cpu") == ([3.0, 4.0], 7.0)
+
+
+def test_reference_arm_prints_the_contract_line():
+    """One step of the reference arm (the fp64 oracle on a bounded row sample) prints one
+    JSON line with every key the benchmark contract names."""
+    import json
+    import subprocess
+    import sys
+    r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--config", "1", "--steps", "1",
+                        "--warmup", "3", "--cpu-seconds", "0.5"], capture_output=True, text=True, timeout=600,
+                       cwd=os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    j = json.loads(lines[0])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "impl", "cpu_baseline", "e2e"):
+        assert key in j, key
+    assert j["impl"] == "reference" and j["value"] > 0 and j["steps"] == 1
+    assert j["e2e"]["h2d_bytes_per_step"] == 0 and j["e2e"]["value"] == j["value"]
+    assert j["cpu_baseline"]["kind"] == "oracle" and j["cpu_baseline"]["cores"] >= 1
