@@ -898,20 +898,30 @@ void build_bwd(const Shape& s, const std::vector<std::vector<int32_t>>& cnts, in
           }
     }
     const size_t nnz = row_kt.size();
-    bl.q_jobs.reserve(bl.q_jobs.size() + size_t(s.hq) * (nnz + n_qt));
+    bl.q_jobs.reserve(bl.q_jobs.size() + nnz + n_qt);
     bl.kv_jobs.reserve(bl.kv_jobs.size() + size_t(s.hq) * nnz + size_t(s.hkv) * n_kt);
+    // A dQ job names a key tile and its mask only (the dQ kernel takes the head from the
+    // item), so the query heads of one query tile share one list.
+    std::vector<int32_t> q_start(size_t(n_qt), -1), q_count(size_t(n_qt), 0);
     for (int kh = 0; kh < s.hkv; ++kh) {
       // dQ items
       for (int h = kh * g; h < (kh + 1) * g; ++h)
         for (int qt = 0; qt < n_qt; ++qt) {
           BwdItem it{b, kh, h, s.qoff[b] + qt * kTile, std::min(kTile, lq - qt * kTile), int32_t(bl.q_jobs.size()), 0, 0};
-          for (int32_t e = row_off[qt]; e < row_off[qt + 1]; ++e) {
-            const int kt = row_kt[e];
-            bl.q_jobs.push_back(BwdJob{s.koff[b] + kt * kTile, tab[size_t(qt) * n_kt + kt], h, 0});
+          if (q_start[qt] >= 0) {
+            it.job_start = q_start[qt];
+            it.job_count = q_count[qt];
+          } else {
+            for (int32_t e = row_off[qt]; e < row_off[qt + 1]; ++e) {
+              const int kt = row_kt[e];
+              bl.q_jobs.push_back(BwdJob{s.koff[b] + kt * kTile, tab[size_t(qt) * n_kt + kt], h, 0});
+            }
+            if (bl.q_jobs.size() == size_t(it.job_start))   // no key anywhere: one hidden job writes dq = 0
+              bl.q_jobs.push_back(BwdJob{s.koff[b], kMaskNone, h, 0});
+            it.job_count = int32_t(bl.q_jobs.size()) - it.job_start;
+            q_start[qt] = it.job_start;
+            q_count[qt] = it.job_count;
           }
-          if (bl.q_jobs.size() == size_t(it.job_start))   // no key anywhere: one hidden job writes dq = 0
-            bl.q_jobs.push_back(BwdJob{s.koff[b], kMaskNone, h, 0});
-          it.job_count = int32_t(bl.q_jobs.size()) - it.job_start;
           q_cost.push_back(it.job_count + 2);
           q_group.push_back(int64_t(b) * s.hkv + kh);
           bl.q_items.push_back(it);
