@@ -511,6 +511,7 @@ def run_ours(args, rank, world, local_rank):
                      "dram_gbs": (tr / (avg_launch_ms * 1e-3) / 1e9) if tr else None},
         "per_mask": [{"mask": m.kind, "unmasked_pairs_per_head": s["unmasked_pairs"], "tflops_per_s":
                       f / (statistics.mean(x) * 1e-3) / 1e12, "ms": statistics.mean(x),
+                      "ms_median": statistics.median(x),
                       "tiles_e_f_p": [s["tiles_empty"], s["tiles_full"], s["tiles_partial"]],
                       "kv_splits_max": s["kv_splits_max"], "merge_tiles": s["merge_tiles"],
                       "plan_ms": pm,
