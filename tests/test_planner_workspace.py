@@ -368,3 +368,30 @@ def test_failed_device_allocations_are_reported_and_cleaned_up(attn_lib, probe, 
         assert n >= 2   # forward workspace and backward workspace at least
     finally:
         probe.probe_fail_malloc_after(-1)
+
+
+@pytest.mark.parametrize("kind", KINDS)
+def test_plan_tile_classes_and_stats_match_the_oracle(attn_lib, probe, kind):
+    """attn_plan_get_tile_classes / attn_plan_get_stats of a plan built by attn_plan (CUSTOM
+    through the scan's host versions) against the oracle's classes and pair count."""
+    M = attn_lib
+    wl = W.random_small(seed=120 + len(kind), kind=kind, batch=3, hq=4, hkv=2, d=128, lmin=1, lmax=700)
+    spec = wl.masks[0]
+    h = _plan(probe, M, wl, spec)
+    try:
+        n = ctypes.c_size_t()
+        probe.attn_plan_get_tile_classes.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
+                                                     ctypes.c_void_p]
+        assert probe.attn_plan_get_tile_classes(h, None, 0, ctypes.addressof(n)) == 0
+        cls = np.zeros(n.value, np.uint8)
+        assert probe.attn_plan_get_tile_classes(h, cls.ctypes.data, n.value, None) == 0
+        st = M.attn_plan_stats_t()
+        probe.attn_plan_get_stats.argtypes = [ctypes.c_void_p, ctypes.c_void_p]
+        assert probe.attn_plan_get_stats(h, ctypes.addressof(st)) == 0
+    finally:
+        probe.attn_plan_destroy(h)
+    lengths = [(wl.lq(b), wl.lk(b)) for b in range(wl.batch)]
+    ref = OM.tile_classes(spec, lengths)
+    assert np.array_equal(cls, ref)
+    assert st.unmasked_pairs == OM.unmasked_pairs(spec, lengths)
+    assert (st.tiles_empty, st.tiles_full, st.tiles_partial) == tuple(int((ref == c).sum()) for c in (0, 1, 2))
