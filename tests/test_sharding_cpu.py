@@ -1,5 +1,5 @@
 """Host side of the long-sequence multi-GPU path: query shards partition the work exactly
-(attn_plan_dry_run), and the K/V all-gather of row shards over a world-size-2 gloo group
+(attn_plan_dry_run), and the K/V all-gather of row shards over gloo groups of 2 and 3 ranks
 rebuilds the full tensors on every rank."""
 import multiprocessing as mp
 import os
@@ -44,12 +44,12 @@ def _gather_worker(rank, world, port, rows, q):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("rows", [10, 7])
-def test_all_gather_rows_gloo(rows):
+@pytest.mark.parametrize("rows,world", [(10, 2), (7, 2), (7, 3), (2, 3)])   # (2, 3): a rank holds no rows
+def test_all_gather_rows_gloo(rows, world):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
-    port = 29650 + rows
-    procs = [ctx.Process(target=_gather_worker, args=(r, 2, port, rows, q)) for r in range(2)]
+    port = 29650 + 10 * world + rows
+    procs = [ctx.Process(target=_gather_worker, args=(r, world, port, rows, q)) for r in range(world)]
     for p in procs:
         p.start()
     res = [q.get(timeout=120) for _ in procs]
