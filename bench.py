@@ -514,6 +514,7 @@ def run_ours(args, rank, world, local_rank):
                       "ms_median": statistics.median(x),
                       "tiles_e_f_p": [s["tiles_empty"], s["tiles_full"], s["tiles_partial"]],
                       "kv_splits_max": s["kv_splits_max"], "merge_tiles": s["merge_tiles"],
+                      "workspace_bytes": s["workspace_bytes"],
                       "plan_ms": pm,
                       # CUSTOM: the device scan of the packed bits happens inside attn_plan
                       "custom_scan_gbs": (custom_bytes(m) / (pm * 1e-3) / 1e9) if m.kind == "CUSTOM" else None}
