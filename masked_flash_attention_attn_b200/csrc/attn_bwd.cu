@@ -596,10 +596,8 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd_dkv_kernel(cons
 
 template <class C, bool DKV>
 attn_status_t launch_bwd(int ctas, const BwdParams& p, cudaStream_t stream) {
-  static std::once_flag once;
-  static cudaError_t attr = cudaSuccess;
-  std::call_once(once, [] {
-    attr = DKV ? cudaFuncSetAttribute(masked_attn_bwd_dkv_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  const cudaError_t attr = once_per_device([] {
+    return DKV ? cudaFuncSetAttribute(masked_attn_bwd_dkv_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       C::SMEM_BYTES)
                : cudaFuncSetAttribute(masked_attn_bwd_dq_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       C::SMEM_BYTES);

@@ -921,30 +921,26 @@ __global__ void fill_empty_kernel(float* lse, int64_t n) {
 
 template <class C>
 attn_status_t launch(const attn_plan_t* plan, Params& p, cudaStream_t stream) {
-  static std::once_flag once;
-  static cudaError_t attr = cudaSuccess;
-  static bool regs_ok = true;
-  std::call_once(once, [] {
-    attr = cudaFuncSetAttribute(masked_attn_fwd_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                C::SMEM_BYTES);
-    if (attr == cudaSuccess && C::REG_SPLIT) {
+  const cudaError_t attr = once_per_device([] {
+    cudaError_t e = cudaFuncSetAttribute(masked_attn_fwd_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         C::SMEM_BYTES);
+    if (e == cudaSuccess && C::REG_SPLIT) {
       // setmaxnreg.inc draws on the registers the block was launched with: the split must fit
       cudaFuncAttributes fa{};
-      attr = cudaFuncGetAttributes(&fa, masked_attn_fwd_kernel<C>);
-      regs_ok = attr == cudaSuccess && fa.numRegs * C::THREADS >= C::REG_SPLIT_TOTAL;
+      e = cudaFuncGetAttributes(&fa, masked_attn_fwd_kernel<C>);
+      if (e == cudaSuccess && fa.numRegs * C::THREADS < C::REG_SPLIT_TOTAL) e = cudaErrorInvalidConfiguration;
     }
+    return e;
   });
-  if (attr != cudaSuccess || !regs_ok) return ATTN_ERR_CUDA;
+  if (attr != cudaSuccess) return ATTN_ERR_CUDA;
   masked_attn_fwd_kernel<C><<<plan->ctas, C::THREADS, C::SMEM_BYTES, stream>>>(p);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
 template <class C>
 attn_status_t launch_pair(const attn_plan_t* plan, Params& p, cudaStream_t stream) {
-  static std::once_flag once;
-  static cudaError_t attr = cudaSuccess;
-  std::call_once(once, [] {
-    attr = cudaFuncSetAttribute(masked_attn_fwd_pair_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  const cudaError_t attr = once_per_device([] {
+    return cudaFuncSetAttribute(masked_attn_fwd_pair_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 C::SMEM_BYTES);
   });
   if (attr != cudaSuccess) return ATTN_ERR_CUDA;

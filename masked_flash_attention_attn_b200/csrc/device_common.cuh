@@ -350,3 +350,19 @@ bool encode3d(CUtensorMap* tm, const void* ptr, uint64_t d0, uint64_t d1, uint64
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
+
+// Runs `set` (a kernel's launch attributes) once per device and returns its result on every
+// later call from that device: the attributes belong to one device's context, and a process
+// may drive several GPUs. Each call site's lambda type gives it its own flags.
+template <class F>
+cudaError_t once_per_device(F set) {
+  constexpr int kDevices = 64;
+  static std::once_flag flags[kDevices];
+  static cudaError_t result[kDevices];
+  int dev = 0;
+  const cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kDevices) return cudaErrorInvalidDevice;
+  std::call_once(flags[dev], [&] { result[dev] = set(); });
+  return result[dev];
+}
