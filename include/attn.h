@@ -194,7 +194,9 @@ attn_status_t attn_plan(const attn_problem_t* problem, const attn_mask_desc_t* m
  *       bf16 [num_pages][page_size][hkv][head_dim] paged caches
  *   out bf16 [total_q][hq][head_dim]             written for every valid row
  *   lse fp32 [total_q][hq]                       natural log, scale included; may be NULL
- * Allocates nothing. Errors: INVALID_ARG (null/misaligned pointer), CUDA (launch).
+ * Runs on the device the plan was made on, which must be the current device.
+ * Allocates nothing. Errors: INVALID_ARG (null/misaligned pointer, or another current
+ * device), CUDA (launch).
  * Concurrency: the forward only reads the plan, except that a split plan (stats
  * kv_splits_max > 1) keeps the partial results of its key ranges in the plan's workspace.
  * Unsplit plans may therefore serve forwards on several streams at once; forwards of a
@@ -224,7 +226,8 @@ attn_status_t attn_plan_bwd(const attn_problem_t* problem, const attn_mask_desc_
  *   dq            bf16 [total_q][hq][head_dim]  (0 on rows that see no key)
  *   dk, dv        bf16 [total_k][hkv][head_dim] (0 on keys that no query sees)
  * The plan must come from attn_plan_bwd(). Allocates nothing. Errors: INVALID_ARG (plan
- * without backward lists, null or misaligned pointer), CUDA. */
+ * without backward lists, null or misaligned pointer, another current device than the
+ * plan's), CUDA. */
 attn_status_t attn_masked_bwd(const attn_plan_t* plan, const void* q, const void* k, const void* v,
                               const void* out, const float* lse, const void* dout, const float* dlse, void* dq,
                               void* dk, void* dv, attn_stream_t stream);
@@ -241,7 +244,8 @@ attn_status_t attn_masked_bwd(const attn_plan_t* plan, const void* q, const void
  *   ldv >= stats.vt_keys, a multiple of 16
  * head_dim 128 (single-SM kernel) or 256 (2-SM kernel) and contiguous K/V only (else
  * UNSUPPORTED); the plan is an ordinary attn_plan() (split-KV applies). Pointers 16-byte aligned (lse: 4-byte, may be NULL).
- * Allocates nothing. Errors: INVALID_ARG, UNSUPPORTED, CUDA. */
+ * Allocates nothing. Errors: INVALID_ARG (as attn_masked_fwd, or ldv / a scale out of
+ * range), UNSUPPORTED, CUDA. */
 attn_status_t attn_masked_fwd_fp8(const attn_plan_t* plan, const void* q, const void* k, const void* vt,
                                   int64_t ldv, float q_scale, float k_scale, float v_scale, void* out,
                                   float* lse, attn_stream_t stream);
@@ -249,7 +253,8 @@ attn_status_t attn_masked_fwd_fp8(const attn_plan_t* plan, const void* q, const 
 /* V bytes [total_k][hkv][head_dim] -> vt [hkv][head_dim][ldv]: sequence b's keys go to
  * columns from the sum over earlier sequences of their key counts rounded up to 128, the
  * gaps are zero. ldv >= stats.vt_keys and a multiple of 16. Asynchronous on `stream`.
- * Errors: INVALID_ARG (paged plan, null pointer, ldv), UNSUPPORTED (head_dim % 32), CUDA. */
+ * Errors: INVALID_ARG (paged plan, null pointer, ldv, another current device than the
+ * plan's), UNSUPPORTED (head_dim % 32), CUDA. */
 attn_status_t attn_fp8_transpose_v(const attn_plan_t* plan, const void* v, void* vt, int64_t ldv,
                                    attn_stream_t stream);
 

@@ -1324,10 +1324,16 @@ attn_status_t attn_plan_bwd(const attn_problem_t* problem, const attn_mask_desc_
   }
 }
 
+// The plan's workspace lives on the device it was made on: its kernels run there only.
+static bool on_plan_device(const attn_plan_t* plan) {
+  int dev = -1;
+  return cudaGetDevice(&dev) == cudaSuccess && dev == plan->device;
+}
+
 attn_status_t attn_masked_bwd(const attn_plan_t* plan, const void* q, const void* k, const void* v, const void* out,
                               const float* lse, const void* dout, const float* dlse, void* dq, void* dk, void* dv,
                               attn_stream_t stream) {
-  if (!plan || !plan->has_bwd) return ATTN_ERR_INVALID_ARG;
+  if (!plan || !plan->has_bwd || !on_plan_device(plan)) return ATTN_ERR_INVALID_ARG;
   const void* ptrs[] = {q, k, v, out, lse, dout, dq, dk, dv};
   for (const void* p : ptrs)
     if (!p || (reinterpret_cast<uintptr_t>(p) & 15u)) return ATTN_ERR_INVALID_ARG;
@@ -1337,7 +1343,8 @@ attn_status_t attn_masked_bwd(const attn_plan_t* plan, const void* q, const void
 
 attn_status_t attn_fp8_transpose_v(const attn_plan_t* plan, const void* v, void* vt, int64_t ldv,
                                    attn_stream_t stream) {
-  if (!plan || plan->paged || !v || !vt || ldv < plan->vt_keys || ldv % 16 != 0) return ATTN_ERR_INVALID_ARG;
+  if (!plan || plan->paged || !v || !vt || ldv < plan->vt_keys || ldv % 16 != 0 || !on_plan_device(plan))
+    return ATTN_ERR_INVALID_ARG;
   if (plan->d % 32 != 0) return ATTN_ERR_UNSUPPORTED;
   return mfa_transpose_v(plan, v, vt, ldv, reinterpret_cast<cudaStream_t>(stream));
 }
@@ -1345,7 +1352,7 @@ attn_status_t attn_fp8_transpose_v(const attn_plan_t* plan, const void* v, void*
 attn_status_t attn_masked_fwd_fp8(const attn_plan_t* plan, const void* q, const void* k, const void* vt, int64_t ldv,
                                   float q_scale, float k_scale, float v_scale, void* out, float* lse,
                                   attn_stream_t stream) {
-  if (!plan) return ATTN_ERR_INVALID_ARG;
+  if (!plan || !on_plan_device(plan)) return ATTN_ERR_INVALID_ARG;
   if ((plan->d != 128 && plan->d != 256) || plan->paged) return ATTN_ERR_UNSUPPORTED;
   const void* ptrs[] = {q, k, vt, out};
   for (const void* p : ptrs)
@@ -1360,7 +1367,7 @@ attn_status_t attn_masked_fwd_fp8(const attn_plan_t* plan, const void* q, const 
 
 attn_status_t attn_masked_fwd(const attn_plan_t* plan, const void* q, const void* k, const void* v, void* out,
                               float* lse, attn_stream_t stream) {
-  if (!plan) return ATTN_ERR_INVALID_ARG;
+  if (!plan || !on_plan_device(plan)) return ATTN_ERR_INVALID_ARG;
   if (plan->total_q == 0) return ATTN_OK;
   if (!q || !k || !v || !out) return ATTN_ERR_INVALID_ARG;
   auto mis = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) != 0; };

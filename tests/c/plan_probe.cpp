@@ -10,9 +10,11 @@
 
 static int g_mallocs_left = -1;   // >= 0: that many more allocations succeed, then they fail
 static int g_live = 0;            // device allocations not freed yet
+static int g_device = 0;          // the "current device"
 
 extern "C" {
 void probe_fail_malloc_after(int n) { g_mallocs_left = n; }
+void probe_set_device(int d) { g_device = d; }
 int probe_live_allocations() { return g_live; }
 cudaError_t cudaMalloc(void** p, size_t n) {
   if (g_mallocs_left == 0) {
@@ -49,7 +51,7 @@ cudaError_t cudaMemset(void* d, int v, size_t n) {
 }
 cudaError_t cudaStreamSynchronize(cudaStream_t) { return cudaSuccess; }
 cudaError_t cudaGetDevice(int* d) {
-  *d = 0;
+  *d = g_device;
   return cudaSuccess;
 }
 cudaError_t cudaDeviceGetAttribute(int* v, cudaDeviceAttr, int) {

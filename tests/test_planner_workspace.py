@@ -57,6 +57,8 @@ def probe(tmp_path_factory):
     lib.probe_merge.argtypes = [vp, ctypes.POINTER(vp), ctypes.POINTER(ctypes.c_int64)]
     lib.probe_fail_malloc_after.argtypes = [ctypes.c_int]
     lib.probe_live_allocations.restype = ctypes.c_int
+    lib.probe_set_device.argtypes = [ctypes.c_int]
+    lib.attn_masked_fwd.argtypes = [vp] * 7
     return lib
 
 
@@ -395,3 +397,19 @@ def test_plan_tile_classes_and_stats_match_the_oracle(attn_lib, probe, kind):
     assert np.array_equal(cls, ref)
     assert st.unmasked_pairs == OM.unmasked_pairs(spec, lengths)
     assert (st.tiles_empty, st.tiles_full, st.tiles_partial) == tuple(int((ref == c).sum()) for c in (0, 1, 2))
+
+
+def test_calls_on_another_device_than_the_plans_are_refused(attn_lib, probe):
+    """A plan's workspace lives on the device it was made on: attn_masked_fwd with another
+    current device returns INVALID_ARG before any launch (the probe's launcher stub answers
+    UNSUPPORTED when the call gets that far)."""
+    wl = W.random_small(seed=4, kind="CAUSAL", batch=2, hq=2, hkv=1, d=128, lmin=10, lmax=100)
+    h = _plan(probe, attn_lib, wl, wl.masks[0])
+    try:
+        fake = [4096, 8192, 12288, 16384, 20480]   # aligned addresses, never dereferenced here
+        assert probe.attn_masked_fwd(h, *fake, None) == 2
+        probe.probe_set_device(1)
+        assert probe.attn_masked_fwd(h, *fake, None) == 1
+    finally:
+        probe.probe_set_device(0)
+        probe.attn_plan_destroy(h)
