@@ -7,8 +7,6 @@ import multiprocessing as mp
 import os
 import socket
 
-import pytest
-
 
 def _free_port():
     with socket.socket() as s:

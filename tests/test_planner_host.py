@@ -2,7 +2,6 @@
 pair counts match attn_classify_host, query-row shards partition the work list for every
 kind (with and without head packing), forced splits keep every job exactly once, and the
 shard arguments are validated."""
-import numpy as np
 import pytest
 
 import workloads as W

@@ -4,7 +4,6 @@ rebuilds the full tensors on every rank."""
 import multiprocessing as mp
 import os
 
-import numpy as np
 import pytest
 import torch
 
