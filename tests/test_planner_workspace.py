@@ -164,10 +164,18 @@ def _forward_check(probe, M, wl, spec, kv_splits):
     # (seq, head, first row) -> key tiles with a visible pair, gathered over split ranges
     seen = {}
     used_tiles = np.zeros(len(tiles), bool)
+    g = wl.hq // wl.hkv
+    vt0 = np.concatenate([[0], np.cumsum([-(-wl.lk(b) // 128) * 128 for b in range(wl.batch)])])
     for it in items:
         seq, tok, rows, head = it[0], it[4:6], it[6:8], it[8:10]
         js = jobs[it[10]:it[10] + it[11]]
         lq, lk = wl.lq(seq), wl.lk(seq)
+        # the fields the kernels address K / V with
+        assert it[3] == lk and all(head[t] // g == it[1] for t in range(nq) if rows[t] > 0)
+        if wl.paged:
+            assert it[2] == seq * wl.page_table.shape[1] and it[12] == -(-lk // wl.page_size) and it[14] == 0
+        else:
+            assert it[2] == wl.cu_seqlens_k[seq] and it[12] == 0 and it[14] == vt0[seq]
         for t in range(nq):
             if rows[t] == 0:
                 continue
