@@ -75,3 +75,17 @@ def test_reference_arm_prints_the_contract_line():
     assert j["impl"] == "reference" and j["value"] > 0 and j["steps"] == 1
     assert j["e2e"]["h2d_bytes_per_step"] == 0 and j["e2e"]["value"] == j["value"]
     assert j["cpu_baseline"]["kind"] == "oracle" and j["cpu_baseline"]["cores"] >= 1
+
+
+def test_traffic_figures_are_keyed_to_the_current_kernel_sources():
+    """bench.py reports the ncu DRAM traffic of a workload only while the forward kernels'
+    sources hash to the value the figure was recorded under. An entry left behind by a
+    kernel edit is stale: recapture it, or remove it (the bench line then reports null)."""
+    import json
+    import bench
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    with open(os.path.join(root, "profiles", "fwd_traffic.json")) as f:
+        table = json.load(f)
+    for name, entry in table.items():
+        assert entry["kernel_source_hash"] == bench.kernel_source_hash(), f"stale traffic entry {name}"
+        assert bench.traffic_for(name) == entry["dram_bytes_per_launch"]
