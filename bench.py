@@ -1,13 +1,17 @@
 """Benchmark of the masked attention forward on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config 1..5]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config 1..6]
 
-Default workload: the Gemma2-style local/global pair -- 4 ragged sequences with lengths
-uniform in [1024, 8192] (seed 2), Hq=16, Hkv=8, d=256, bf16 N(0,1) inputs -- run with
-SLIDING_WINDOW(4096) and with CAUSAL on the same tensors. One step = both forwards.
+Default (headline) workload: the long block-dense custom mask -- one sequence of 29576
+queries / keys, rows < 24576 see keys [0, 24576), the last 5000 rows add causal attention
+inside their own 100-row block; Hq=32, Hkv=8, d=128, bf16 N(0,1) inputs -- given once as
+packed CUSTOM bits and once as typed ranges. One step = both forwards. It is the largest
+of the five benchmark workloads that fit one GPU.
 
 Metric: effective TFLOP/s = 4 * d * (unmasked pairs) * Hq / time, summed over the masks of
-the step (masked pairs are not counted). Prints ONE JSON line on rank 0.
+the step (masked pairs are not counted). Prints ONE JSON line on rank 0. After the
+headline, the other four benchmark workloads are timed one by one and reported in the same
+line under "per_config" (--no-per-config skips them).
 
 Multi-GPU (torchrun, one rank per GPU): every rank runs its own independent batch of the
 same workload (seed offset by rank); there is no collective on the data path. Timing is
@@ -83,50 +87,131 @@ def traffic_for(workload_name):
 
 
 class ClockSampler:
-    """nvidia-smi clocks / throttle reasons sampled every 200 ms during the timed region."""
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """SM clock and clock-event (throttle) reasons of one GPU, sampled through NVML every
+    `period_s` seconds on a background thread while the timed region runs; falls back to an
+    `nvidia-smi -lms` subprocess when NVML cannot be used. `stop()` returns the summary of
+    the samples taken inside [mark_start(), mark_end()] -- or, when NVML and nvidia-smi both
+    fail, {"error": why} instead of a silent null."""
+    REASON_BITS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
+                   "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80}
+    SMI_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                  "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                  "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, device_index, log_dir=None):
-        self.proc = None
-        self.path = os.path.join(log_dir or tempfile.gettempdir(), f"clocks_rank{device_index}.csv")
+    def __init__(self, device_index, log_dir=None, period_s=0.01):
+        import threading
+        self.samples = []          # (host time, sm MHz, max sm MHz, reason names)
+        self.errors = []
+        self.t0 = self.t1 = None
+        self.source = None
+        self._stop = threading.Event()
+        self._thread = None
+        self._proc = None
+        self.log_path = os.path.join(log_dir or tempfile.gettempdir(), f"clocks_dev{device_index}.csv")
         try:
             import torch
             uuid = "GPU-" + str(torch.cuda.get_device_properties(device_index).uuid)
-            os.makedirs(os.path.dirname(self.path), exist_ok=True)
-            self.fh = open(self.path, "w")
-            self.proc = subprocess.Popen(["nvidia-smi", "-i", uuid, f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
-                                         stdout=self.fh, stderr=subprocess.DEVNULL)
-        except Exception:
-            self.proc = None
-
-    def stop(self):
-        if self.proc is None:
-            return None
-        self.proc.terminate()
+        except Exception as e:          # pragma: no cover - needs a GPU
+            self.errors.append(f"device uuid: {type(e).__name__}: {e}")
+            return
         try:
-            self.proc.wait(timeout=5)
+            import pynvml
+            pynvml.nvmlInit()
+            try:
+                h = pynvml.nvmlDeviceGetHandleByUUID(uuid)
+            except Exception:
+                h = pynvml.nvmlDeviceGetHandleByUUID(uuid.encode())
+            smax = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
+            get_reasons = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
+
+            def sample():
+                sm = float(pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM))
+                bits = int(get_reasons(h))
+                return (time.perf_counter(), sm, smax, [n for n, b in self.REASON_BITS.items() if bits & b])
+
+            self.samples.append(sample())    # fails here, not on the thread, if NVML is unusable
+
+            def loop():
+                while not self._stop.wait(period_s):
+                    try:
+                        self.samples.append(sample())
+                    except Exception as e:   # pragma: no cover
+                        self.errors.append(f"nvml sample: {type(e).__name__}: {e}")
+                        return
+
+            self._thread = threading.Thread(target=loop, daemon=True)
+            self._thread.start()
+            self.source = f"nvml every {period_s * 1e3:.0f} ms"
+            return
+        except Exception as e:
+            self.errors.append(f"nvml: {type(e).__name__}: {e}")
+        try:
+            os.makedirs(os.path.dirname(self.log_path), exist_ok=True)
+            self._fh = open(self.log_path, "w")
+            self._proc = subprocess.Popen(["nvidia-smi", "-i", uuid, f"--query-gpu={self.SMI_FIELDS}",
+                                           "--format=csv,noheader,nounits", "-lms", "50"],
+                                          stdout=self._fh, stderr=subprocess.PIPE)
+            self.source = "nvidia-smi -lms 50"
+            # wait (up to 3 s) for its first sample so the timed region is covered
+            t_wait = time.perf_counter()
+            while time.perf_counter() - t_wait < 3.0 and os.path.getsize(self.log_path) == 0:
+                if self._proc.poll() is not None:
+                    break
+                time.sleep(0.02)
+        except Exception as e:
+            self.errors.append(f"nvidia-smi: {type(e).__name__}: {e}")
+            self._proc = None
+
+    def mark_start(self):
+        self.t0 = time.perf_counter()
+
+    def mark_end(self):
+        self.t1 = time.perf_counter()
+
+    def _smi_rows(self):
+        self._proc.terminate()
+        try:
+            _, err = self._proc.communicate(timeout=5)
         except Exception:
-            self.proc.kill()
-        self.fh.close()
+            self._proc.kill()
+            err = b""
+        self._fh.close()
         rows = []
-        with open(self.path) as f:
+        with open(self.log_path) as f:
             for line in f:
                 p = [x.strip() for x in line.split(",")]
                 if len(p) < 9:
                     continue
                 try:
-                    rows.append((float(p[1]), float(p[2]), p[5:9]))
+                    rows.append((None, float(p[1]), float(p[2]),
+                                 [n for n, v in zip(("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
+                                                     "sw_power_cap"), p[5:9]) if v.lower().startswith("active")]))
                 except ValueError:
                     continue
-        if not rows:
-            return None
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for _, _, r in rows for i in range(4) if r[i].lower().startswith("active")})
-        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
-                "reasons": reasons, "samples": len(rows)}
+        if not rows and err:
+            self.errors.append("nvidia-smi: " + err.decode(errors="replace").strip()[:200])
+        return rows
+
+    def stop(self):
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join(timeout=2)
+            rows = self.samples
+            inside = [r for r in rows if self.t0 is not None and self.t1 is not None and self.t0 <= r[0] <= self.t1]
+            # a timed region shorter than the sampling period still gets its nearest samples
+            if not inside and rows and self.t0 is not None:
+                inside = sorted(rows, key=lambda r: abs(r[0] - self.t0))[:2]
+        elif self._proc is not None:
+            inside = self._smi_rows()      # nvidia-smi rows carry no host time: all of them
+        else:
+            inside = []
+        if not inside:
+            return {"error": "; ".join(self.errors) or "no clock samples"}
+        reasons = sorted({n for r in inside for n in r[3]})
+        return {"sm_mhz": statistics.median(r[1] for r in inside), "sm_min_mhz": min(r[1] for r in inside),
+                "sm_max_mhz": max(r[2] for r in inside), "reasons": reasons, "samples": len(inside),
+                "source": self.source}
 
 
 def oracle_sample(wl, specs, budget_s, rows_per_block=128):
@@ -252,6 +337,118 @@ def make_plan(M, wl, spec, dev, kv_splits=0, backward=False):
     return M.attn_plan(**kw)
 
 
+def kernel_name(wl, fp8=False, bwd=False):
+    """The kernel a forward (or backward) of this workload launches."""
+    if bwd:
+        return f"masked_attn_bwd_dq_kernel + masked_attn_bwd_dkv_kernel d={wl.d}"
+    base = "masked_attn_fwd_pair_kernel (2-SM)" if wl.d == 256 else "masked_attn_fwd_kernel"
+    return f"{base}{' e4m3' if fp8 else ''} d={wl.d}{' paged' if wl.paged else ''}"
+
+
+def stage_mask(spec, dev):
+    """attn_mask_desc_t.mask_bits is a device pointer: CUSTOM bits are staged in HBM before
+    planning, so a timed attn_plan covers the device scan, not a host upload."""
+    import torch
+    if spec.kind == "CUSTOM" and isinstance(spec.bits, np.ndarray):
+        spec = dataclasses.replace(spec, bits=torch.from_numpy(
+            np.ascontiguousarray(spec.bits.astype(np.uint32).view(np.int32))).to(dev))
+        torch.cuda.synchronize()
+    return spec
+
+
+def build_plans(M, wl, dev, kv_splits=0, backward=False):
+    """One plan per mask of the workload; attn_plan is timed on its own (host wall clock; it
+    synchronises its stream). The first plan of a kind also pays one-off costs (context
+    set-up, module loading): each mask is planned once untimed, then the kept plan is timed."""
+    plans, plan_ms = [], []
+    for spec in wl.masks:
+        spec = stage_mask(spec, dev)
+        make_plan(M, wl, spec, dev, kv_splits, backward=backward)
+        t0 = time.perf_counter()
+        plans.append(make_plan(M, wl, spec, dev, kv_splits, backward=backward))
+        plan_ms.append((time.perf_counter() - t0) * 1e3)
+    return plans, plan_ms
+
+
+def kv_bytes_read(wl):
+    """K and V bytes one forward must read at least once (bf16): the keys of every sequence."""
+    return sum(wl.lk(b) for b in range(wl.batch)) * wl.hkv * wl.d * 2 * 2
+
+
+def choose_peak(clocks, fp8=False):
+    """Tensor peak for the roofline: the measured burst cuBLAS bf16 figure, or the sustained
+    one when the sampled SM clock fell below 90 % of its maximum (a long run at the power cap)."""
+    pk, pk_src = peaks()
+    burst = float(pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    sustained = float(pk.get("bf16_tflops_sustained", burst))
+    use_sustained = isinstance(clocks, dict) and "sm_mhz" in clocks and \
+        clocks["sm_mhz"] < 0.9 * clocks["sm_max_mhz"]
+    peak = sustained if use_sustained else burst
+    pk_src += " bf16_tflops_sustained" if use_sustained else " bf16_tflops (burst)"
+    if fp8:   # e4m3 tensor rate: the measured bf16 figure x the nominal fp8 / bf16 ratio (4.5 / 2.25)
+        peak *= 2.0
+        pk_src += " x 2 (nominal e4m3 / bf16 ratio)"
+    hbm = float(pk.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    return peak, pk_src, hbm
+
+
+def time_config(M, cfg, dev, stream, steps, warmup, peak, hbm_peak):
+    """Forward of one benchmark workload (every mask of it) on this GPU: CUDA-event time of
+    each launch over `steps` steps after `warmup`, L2 flushed between launches when the
+    inputs fit in it. Returns the per-config entry of the bench line."""
+    import torch
+    wl = workload(cfg, 0)
+    q, k, v = device_inputs(wl, dev)
+    plans, plan_ms = build_plans(M, wl, dev)
+    stats = [M.attn_plan_get_stats(p) for p in plans]
+    flops = [flops_of(s, wl) for s in stats]
+    tq = q.shape[0]
+    outs = [torch.empty(tq, wl.hq, wl.d, dtype=torch.bfloat16, device=dev) for _ in plans]
+    lses = [torch.empty(tq, wl.hq, dtype=torch.float32, device=dev) for _ in plans]
+    in_bytes = (q.numel() + k.numel() + v.numel()) * 2
+    flush = torch.empty(256 * 2**20, dtype=torch.uint8, device=dev) if in_bytes <= L2_BYTES else None
+    ev = [[[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in plans] for _ in range(steps)]
+    for s in range(warmup + steps):
+        for i, p in enumerate(plans):
+            if flush is not None:
+                flush.fill_(s & 255)
+            if s >= warmup:
+                ev[s - warmup][i][0].record(stream)
+            M.attn_masked_fwd(p, q, k, v, outs[i], lses[i], stream)
+            if s >= warmup:
+                ev[s - warmup][i][1].record(stream)
+    torch.cuda.synchronize()
+    for p in plans:
+        st = M.attn_plan_check_status(p)
+        if st != 0:
+            raise RuntimeError(f"workload {cfg}: forward reported {M.STATUS.get(st, st)}")
+    launch_ms = [[ev[s][i][0].elapsed_time(ev[s][i][1]) for s in range(steps)] for i in range(len(plans))]
+    mean_ms = [statistics.mean(x) for x in launch_ms]
+    step_ms = sum(mean_ms)
+    tflops = sum(flops) / (step_ms * 1e-3) / 1e12
+    entry = {"config": cfg, "workload": wl.name, "kernel": kernel_name(wl), "steps": steps,
+             "ms_per_step": step_ms, "tflops_per_s": tflops, "frac": tflops / peak,
+             "per_mask": [{"mask": m.kind, "ms": mm, "ms_median": statistics.median(x),
+                           "tflops_per_s": f / (mm * 1e-3) / 1e12, "frac": f / (mm * 1e-3) / 1e12 / peak,
+                           "unmasked_pairs_per_head": s["unmasked_pairs"],
+                           "tiles_e_f_p": [s["tiles_empty"], s["tiles_full"], s["tiles_partial"]],
+                           "kv_splits_max": s["kv_splits_max"], "plan_ms": pm}
+                          for m, s, f, x, mm, pm in zip(wl.masks, stats, flops, launch_ms, mean_ms, plan_ms)],
+             "l2": "L2 flushed between launches" if flush is not None else
+                   f"inputs {in_bytes / 2**20:.0f} MiB vs 126 MiB L2; no flush"}
+    if wl.paged:
+        # the K/V stream: bytes of the keys every request holds, read once per launch at least
+        kvb = kv_bytes_read(wl)
+        gbs = kvb / (step_ms / len(plans) * 1e-3) / 1e9
+        entry["kv_stream"] = {"bytes_per_launch": kvb, "gbs": gbs, "hbm_peak_gbs": hbm_peak,
+                              "frac_of_hbm": gbs / hbm_peak}
+    mask_bytes = sum(s["mask_tile_reads"] for s in stats) * 2048.0
+    entry["mask_gbs"] = mask_bytes / (step_ms * 1e-3) / 1e9
+    del q, k, v, outs, lses, flush, plans
+    torch.cuda.empty_cache()
+    return entry
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -270,20 +467,7 @@ def run_ours(args, rank, world, local_rank):
         raise SystemExit("--pass bwd: contiguous K/V and head_dim <= 128 only (workloads 1, 4, 5)")
     if fp8 and (bwd or wl.paged or wl.d not in (128, 256)):
         raise SystemExit("--dtype e4m3: the forward with contiguous K/V, head_dim 128 or 256 (workloads 2, 4, 5)")
-    plans, plan_ms = [], []
-    for spec in wl.masks:   # attn_plan is timed on its own (host wall clock; it synchronises its stream)
-        if spec.kind == "CUSTOM" and isinstance(spec.bits, np.ndarray):
-            # attn_mask_desc_t.mask_bits is a device pointer: the packed bits are staged in HBM
-            # first, so plan_ms (and custom_scan_gbs) cover the device scan, not a host upload
-            spec = dataclasses.replace(spec, bits=torch.from_numpy(
-                np.ascontiguousarray(spec.bits.astype(np.uint32).view(np.int32))).to(dev))
-            torch.cuda.synchronize()
-        # the first plan of a kind also pays one-off costs (context set-up, module loading):
-        # plan once untimed, then time the plan that is kept
-        make_plan(M, wl, spec, dev, args.kv_splits, backward=bwd)
-        t0 = time.perf_counter()
-        plans.append(make_plan(M, wl, spec, dev, args.kv_splits, backward=bwd))
-        plan_ms.append((time.perf_counter() - t0) * 1e3)
+    plans, plan_ms = build_plans(M, wl, dev, args.kv_splits, backward=bwd)
     stats = [M.attn_plan_get_stats(p) for p in plans]
     flops = [flops_of(s, wl) * (2.5 if bwd else 1.0) for s in stats]
     tq = q.shape[0]
@@ -340,10 +524,14 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     sampler = ClockSampler(local_rank, args.clock_log)
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler.mark_start()
     t_start.record(stream)
     for s in range(args.steps):
         step(ev[s])
     t_end.record(stream)
+    while not t_end.query():     # poll (GIL released) so the sampler thread runs meanwhile
+        time.sleep(2e-4)
+    sampler.mark_end()
     torch.cuda.synchronize()
     clocks = sampler.stop()
     if world > 1:
@@ -475,19 +663,11 @@ def run_ours(args, rank, world, local_rank):
         return
     value = total_flops * args.steps / (ms * 1e-3) / 1e12
     e2e_val = total_flops * e2e_steps / (e2e_ms * 1e-3) / 1e12
-    pk, pk_src = peaks()
     # The timed regions here are short (well under the seconds a GEMM needs to settle at the
     # power cap) and the SM clock stays near its maximum (see "clocks"), so the burst cuBLAS
     # figure is the denominator; the sustained one is used only when the sampled clock fell
     # below 90 % of the maximum.
-    burst = float(pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
-    sustained = float(pk.get("bf16_tflops_sustained", burst))
-    use_sustained = clocks is not None and clocks["sm_mhz"] < 0.9 * clocks["sm_max_mhz"]
-    peak = sustained if use_sustained else burst
-    pk_src += " bf16_tflops_sustained" if use_sustained else " bf16_tflops (burst)"
-    if fp8:   # e4m3 tensor rate: the measured bf16 figure x the nominal fp8 / bf16 ratio (4.5 / 2.25)
-        peak *= 2.0
-        pk_src += " x 2 (nominal e4m3 / bf16 ratio)"
+    peak, pk_src, hbm_peak = choose_peak(clocks, fp8)
     avg_launch_ms = sum(sum(x) for x in launch_ms) / sum(len(x) for x in launch_ms)
     achieved = (sum(flops) / len(flops)) / (avg_launch_ms * 1e-3) / 1e12
     tr = None if (bwd or fp8) else traffic_for(wl.name)
@@ -502,9 +682,7 @@ def run_ours(args, rank, world, local_rank):
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": tr,
                      "peak_source": pk_src,
-                     "kernel": (f"masked_attn_bwd_dq_kernel + masked_attn_bwd_dkv_kernel d={wl.d}" if bwd
-                                else f"masked_attn_fwd_kernel e4m3 d={wl.d}" if fp8
-                                else f"masked_attn_fwd_kernel d={wl.d}"),
+                     "kernel": kernel_name(wl, fp8, bwd),
                      "algorithmic_flops_per_launch": sum(flops) / len(flops),
                      "avg_launch_ms": avg_launch_ms,
                      # DRAM GB/s of the captured launch (ncu bytes over this run's mean launch time)
@@ -527,6 +705,18 @@ def run_ours(args, rank, world, local_rank):
         "gpu_launches": (3 * len(plans) if bwd else sum(1 + (s["merge_tiles"] > 0) for s in stats)) * args.steps,
         "clocks": clocks,
     }
+    if wl.paged and not bwd:
+        kvb = kv_bytes_read(wl)
+        gbs = kvb / (avg_launch_ms * 1e-3) / 1e9
+        line["kv_stream"] = {"bytes_per_launch": kvb, "gbs": gbs, "hbm_peak_gbs": hbm_peak,
+                             "frac_of_hbm": gbs / hbm_peak}
+    if world == 1 and not args.no_per_config and not bwd and not fp8:
+        # the other benchmark workloads, each timed on its own after the headline (outside
+        # its timed region): every configuration's throughput in the same line
+        del q, k, v, outs, lses
+        torch.cuda.empty_cache()
+        line["per_config"] = [time_config(M, c, dev, stream, max(3, min(args.steps, 30)), 3, peak, hbm_peak)
+                              for c in (1, 2, 3, 4, 5) if c != args.config]
     if world == 1 and not args.no_cpu_baseline and not bwd and not fp8:
         pairs, secs, desc = oracle_sample(wl, wl.masks, args.cpu_seconds)
         line["cpu_baseline"] = {"value": 4.0 * wl.d * pairs / secs / 1e12, "unit": "TFLOP/s",
@@ -538,11 +728,12 @@ def run_ours(args, rank, world, local_rank):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--config", type=int, default=2, choices=[1, 2, 3, 4, 5, 6],
-                    help="1-5: the benchmark workloads; 6: long-context tree verify (split-KV case)")
+    ap.add_argument("--config", type=int, default=5, choices=[1, 2, 3, 4, 5, 6],
+                    help="1-5: the benchmark workloads (5, the long block-dense CUSTOM mask, is the "
+                         "headline: the largest single-GPU one); 6: long-context tree verify (split-KV case)")
     ap.add_argument("--pass", dest="pass_", choices=["fwd", "bwd"], default="fwd",
                     help="fwd: the forward (the benchmark metric); bwd: the backward pass (workloads 1, 4, 5)")
     ap.add_argument("--dtype", choices=["bf16", "e4m3"], default="bf16",
@@ -553,6 +744,8 @@ def main():
     ap.add_argument("--clock-log", default=None,
                     help="folder for the raw nvidia-smi clock samples (default: the temp folder)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="skip timing the other benchmark workloads after the headline")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
