@@ -1,28 +1,17 @@
 // Masked attention forward for sm_100a (B200).
 //
-// One persistent CTA per SM walks its list of work items (built by the planner). A work
-// item is NQ 128-row query tiles (NQ = 2 for head_dim <= 128, 1 for head_dim 256) that
-// share one key/value head and one run of key tiles; empty key tiles never appear in the
-// run, full key tiles carry no mask, partial ones carry the index of a 2 KiB
-// tile-transposed bit mask.
+// One persistent CTA (or CTA pair) per SM walks its list of work items (built by the
+// planner). A work item is two 128-row query tiles that share one key/value head and one
+// run of key tiles; empty key tiles never appear in the run, full key tiles carry no mask,
+// partial ones carry the index of a 2 KiB tile-transposed bit mask. Three kernels:
 //
-// Warp roles (128 * (1 + NQ) threads):
-//   warp 0      TMA producer: Q tiles once per item, K and V tiles through a ring of
-//               STAGES shared-memory chunks (128 keys x 128 columns, 128-byte swizzle);
-//               paged K/V arrive as one box per page.
-//   warp 1      MMA issuer (one thread): S = Q K^T into TMEM (tcgen05.mma, bf16 inputs,
-//               fp32 accumulators) and O += P V with P read from TMEM.
-//   warps 2-3   idle (they hold the warpgroup's TMEM lane quarters for the allocator).
-//   warpgroup 1+t  softmax of query tile t: one thread per row reads its S row from TMEM
-//               (tcgen05.ld), applies the row's 128 mask bits (one 16-byte load) on partial
-//               tiles, keeps the online max / sum, writes P as bf16 back into the S
-//               columns, rescales O in TMEM when the running max grows by more than 2^8,
-//               and finally normalises O, writes out (bf16) and the row lse (fp32).
-//
-// The S accumulators are double buffered: the stream of (key tile, query tile) jobs of an
-// item is issued as S(0), S(1), then P V(u), S(u + 2) for u = 0, 1, ..., so the tensor
-// core works on the next job while the softmax warpgroup(s) work on the current one.
-// TMEM (512 columns): S slot 0 at column 0, S slot 1 at 128, O of tile t at 256 + t D.
+//   masked_attn_fwd_kernel       (bf16, head_dim 64 / 128): the two query tiles take turns
+//       in one S accumulator in TMEM, P has a TMEM slot of its own per tile, Q K^T and P V
+//       are issued by two different threads (see the kernel's comment).
+//   masked_attn_fwd_e4m3_kernel  (e4m3, head_dim 128): S double buffered, P written over S,
+//       one issuing thread; Q, K and V^T in e4m3 with .kind::f8f6f4 MMAs.
+//   masked_attn_fwd_pair_kernel  (head_dim 256, bf16 or e4m3): a CTA pair, one query tile per
+//       CTA, 2-SM MMAs (cta_group::2) so each SM streams half of every K and V tile.
 //
 // Every wait on an mbarrier is bounded (globaltimer). When a wait expires the thread
 // records ATTN_ERR_TIMEOUT in the plan's status word, raises a shared abort flag that
@@ -63,8 +52,14 @@ struct Params {
   int64_t timeout_ns;
 };
 
-// FP8_: e4m3 Q, K and V (the latter transposed, [Hkv][d][keys]) with .kind::f8f6f4 MMAs and P
-// quantised to e4m3 in TMEM; head_dim 128 only.
+// Configuration of masked_attn_fwd_e4m3_kernel (FP8_ = true: e4m3 Q, K and V, the latter
+// transposed, [Hkv][d][keys], .kind::f8f6f4 MMAs, P quantised to e4m3 in TMEM; head_dim 128).
+// Warp roles (128 * (1 + NQ) threads): warp 0 TMA producer (Q tiles once per item, K and V
+// tiles through a ring of STAGES chunks); warp 1 MMA issuer (one thread: S = Q K^T into one
+// of two TMEM S slots, O += P V with P read from TMEM); warpgroup 1 + t the softmax of query
+// tile t, one thread per row, P written back over the S columns. The jobs of an item are
+// issued as S(0), S(1), then P V(u), S(u + 2) for u = 0, 1, ...; TMEM: S slot 0 at column 0,
+// S slot 1 at 128, O of tile t at 256 + t D.
 template <int D_, int NQ_, int STAGES_, bool PAGED_, int EMU_ = 0, bool FP8_ = false>
 struct Cfg {
   static constexpr int D = D_, NQ = NQ_, STAGES = STAGES_;
@@ -271,6 +266,36 @@ __device__ __forceinline__ void store_partial(uint32_t t_o, const RowState& st, 
   if (valid) plse[srow] = seen ? (st.m_run + log2f(st.l_run)) * 0.69314718055994531f : -INFINITY;
 }
 
+// Paged K/V: the slots of a sequence's last page past its last key hold whatever the cache
+// holds there, possibly NaN or Inf. Their scores are masked (P = 0), but 0 x NaN is NaN in
+// P V, so before the P V of a key tile that reaches past the keys, the V rows of those
+// slots are zeroed in shared memory: rows [r0, r1) of a V chunk (nbox 128-byte boxes of
+// 128 rows, 16 KiB apart; the 128-byte swizzle permutes 16-byte pieces inside a row, so a
+// whole row is the same 128 bytes). `lanes` threads starting at `lane` share the stores;
+// `remote` (a cluster peer's shared::cluster address of the chunk) is zeroed as well when
+// not 0. The stores are made visible to the tensor core's async proxy before returning.
+__device__ __forceinline__ void zero_v_rows(uint32_t chunk, uint32_t remote, int nbox, int r0, int r1, int lane,
+                                            int lanes) {
+  const int n = (r1 - r0) * nbox * 8;   // 16-byte pieces
+  for (int i = lane; i < n; i += lanes) {
+    const int row = r0 + i / (nbox * 8), rem = i % (nbox * 8);
+    const uint32_t off = uint32_t((rem >> 3) * 16384 + row * 128 + (rem & 7) * 16);
+    asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(chunk + off), "r"(0u) : "memory");
+    if (remote) asm volatile("st.shared::cluster.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(remote + off), "r"(0u) : "memory");
+  }
+  asm volatile("fence.proxy.async;" ::: "memory");
+}
+
+// Rows [r0, r1) of key tile kt to zero: the tail of the sequence's last page, when the tile
+// reaches past the last key (rows from the page count on come from out-of-bounds boxes and
+// are zeros already). r0 >= r1 when there is nothing to zero.
+__device__ __forceinline__ void v_tail_rows(int kt, int kv_len, int npages, int page_size, int& r0, int& r1) {
+  r0 = kv_len - kt * 128;
+  r1 = npages * page_size - kt * 128;
+  r1 = r1 < 128 ? r1 : 128;
+  if (r0 < 0) r0 = r1;
+}
+
 // ---- the kernel ----------------------------------------------------------------------------
 
 enum : int32_t {
@@ -278,7 +303,7 @@ enum : int32_t {
 };
 
 template <class C>
-__global__ void __launch_bounds__(C::THREADS, 1) masked_attn_fwd_kernel(const __grid_constant__ Params p) {
+__global__ void __launch_bounds__(C::THREADS, 1) masked_attn_fwd_e4m3_kernel(const __grid_constant__ Params p) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t sbase = (raw + 1023u) & ~1023u;
@@ -550,6 +575,404 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_fwd_kernel(const __
   if (warp == 1) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem) : "memory");
 }
 
+// ================================ shared-S kernel (head_dim 64 / 128, bf16) ================================
+// One persistent CTA per SM, two 128-row query tiles per work item. The two query tiles take
+// turns in ONE S accumulator (TMEM columns 0-127): a softmax warpgroup frees it as soon as it
+// has read its scores into registers, so the next Q K^T (of the other tile) runs while it
+// computes; P goes to a slot of its own per tile (columns 128 + 64 t, bf16 pairs), O of tile t
+// sits at 256 + t D. Q K^T and P V are issued by two different threads, so a wait of one
+// never idles the tensor core while the other has work:
+//   warp 0       TMA producer: Q tiles once per item, then K(0), [K(1), V(0)], [K(2), V(1)],
+//                ..., V(J-1) through a ring of STAGES chunks (a chunk = a 128-key K or V tile).
+//   warp 1       Q K^T issuer: for key tile j, S = Q0 K(j)^T, then (once softmax 0 has read
+//                S) S = Q1 K(j)^T; releases K(j).
+//   warp 2       P V issuer: O_t += P_t V(j) for t = 0, 1 once P_t is published; releases V(j).
+//   warp 3       idle (holds its warpgroup's TMEM lane quarter).
+//   warpgroup 1+t  softmax of query tile t: one thread per row reads S, frees it, applies the
+//                row's mask bits (partial tiles), updates the online max / sum, writes P into
+//                its slot once the previous P V of the tile is done, rescales O when the
+//                running maximum grows by more than 2^8, and finally writes out / lse.
+template <int D_, bool PAGED_, int EMU_ = 0>
+struct SCfg {
+  static constexpr int D = D_, EMU = EMU_;
+  static constexpr bool PAGED = PAGED_;
+  static constexpr int NBOX = D / 64;                 // 128-byte boxes per Q tile and per K / V chunk
+  static constexpr int BOX_BYTES = 128 * 128;         // 128 rows x 128 bytes
+  static constexpr int Q_BYTES = NBOX * BOX_BYTES;
+  static constexpr int CHUNK_BYTES = NBOX * BOX_BYTES;
+  static constexpr int STAGES = D == 128 ? 5 : 10;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_RING = 2 * Q_BYTES;
+  static constexpr int OFF_BAR = OFF_RING + STAGES * CHUNK_BYTES;
+  static constexpr int B_QFULL = 0, B_QEMPTY = 1, B_KVFULL = 2, B_KVEMPTY = B_KVFULL + STAGES,
+                       B_SFULL = B_KVEMPTY + STAGES, B_SFREE = B_SFULL + 2, B_PFULL = B_SFREE + 2,
+                       B_PVDONE = B_PFULL + 2, B_OEMPTY = B_PVDONE + 2, B_DRAIN = B_OEMPTY + 2, NBAR = B_DRAIN + 2;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;  // [0] TMEM base, [1] abort flag
+  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
+  static constexpr int THREADS = 384;
+  static constexpr int REG_LOW = 64, REG_HIGH = 208;
+  static constexpr int REG_SPLIT_TOTAL = 128 * REG_LOW + 256 * REG_HIGH;
+  static constexpr int TM_S = 0, TM_P = 128, TM_O = 256;
+  static constexpr uint32_t AB_TYPES = (1u << 7) | (1u << 10);   // bf16 A and B
+  static constexpr uint32_t IDESC_QK =  // M=128, N=128, both K-major, fp32 accumulate
+      (1u << 4) | AB_TYPES | (uint32_t(128 >> 3) << 17) | (uint32_t(128 >> 4) << 24);
+  static constexpr uint32_t IDESC_PV =  // M=128, N=D, A (P) from TMEM, B (V) MN-major
+      (1u << 4) | AB_TYPES | (1u << 16) | (uint32_t(D >> 3) << 17) | (uint32_t(128 >> 4) << 24);
+  static_assert(D == 64 || D == 128, "shared-S kernel: head_dim 64 or 128");
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+  static_assert(TM_O + 2 * D <= 512, "TMEM budget");
+};
+
+// Position of K(j) / V(j) of an item with J key tiles in the producer's order
+// K(0), [K(1), V(0)], [K(2), V(1)], ..., [K(J-1), V(J-2)], V(J-1) (2 J chunks).
+__device__ __forceinline__ int k_pos(int j) { return j == 0 ? 0 : 2 * j - 1; }
+__device__ __forceinline__ int v_pos(int j, int J) { return j == J - 1 ? 2 * J - 1 : 2 * j + 2; }
+
+// Softmax step of a shared-S tile: the row's 128 scores at t_s (fp32) into registers, then
+// `freed()` (the S accumulator may be overwritten), mask / max / exponentials / row sum, and
+// P (bf16 pairs) into pk[64]. Returns the factor by which O and l must be multiplied.
+template <int EMU, class Freed>
+__device__ __forceinline__ float softmax_regs(uint32_t t_s, int mi, const uint4& bits, float sl2, RowState& st,
+                                              bool& need, uint32_t (&pk)[64], Freed freed) {
+  float s[128];
+  {
+    uint32_t su[128];
+    tmem_ld32x32(t_s + 0, su + 0);
+    tmem_ld32x32(t_s + 32, su + 32);
+    tmem_ld32x32(t_s + 64, su + 64);
+    tmem_ld32x32(t_s + 96, su + 96);
+    tmem_wait_ld();
+#pragma unroll
+    for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(su[c]);
+  }
+  freed();
+  if (mi != kMaskFull) {
+    const uint32_t wv[4] = {bits.x, bits.y, bits.z, bits.w};
+#pragma unroll
+    for (int c = 0; c < 128; ++c)
+      if (!((wv[c >> 5] >> (c & 31)) & 1u)) s[c] = -INFINITY;
+  }
+  float m8[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) m8[k] = fmaxf(s[k], s[k + 8]);
+#pragma unroll
+  for (int j = 1; j < 8; ++j)
+#pragma unroll
+    for (int k = 0; k < 8; ++k) m8[k] = max3f(m8[k], s[16 * j + k], s[16 * j + 8 + k]);
+  const float mx = max3f(max3f(m8[0], m8[1], m8[2]), max3f(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
+  const float m_new = mx * sl2;
+  need = m_new > st.m_run + 8.0f;
+  float alpha = 1.f;
+  if (need) {
+    alpha = ex2(st.m_run - m_new);
+    st.m_run = m_new;
+    st.l_run *= alpha;
+  }
+  const float mref = st.m_run == -INFINITY ? 0.f : st.m_run;
+  const uint64_t sl2x2 = pk2(sl2, sl2), nm2 = pk2(-mref, -mref);
+  uint64_t lsum2[4] = {pk2(0.f, 0.f), pk2(0.f, 0.f), pk2(0.f, 0.f), pk2(0.f, 0.f)};
+#pragma unroll
+  for (int e = 0; e < 64; ++e) {
+    float x0, x1;
+    unpk2(ffma2(pk2(s[2 * e], s[2 * e + 1]), sl2x2, nm2), x0, x1);
+    uint64_t p01;
+    if ((e & 7) < EMU) p01 = exp2_poly2(x0, x1);
+    else p01 = pk2(ex2(x0), ex2(x1));
+    lsum2[e & 3] = fadd2(lsum2[e & 3], p01);
+    float p0, p1;
+    unpk2(p01, p0, p1);
+    pk[e] = pack_bf16(p0, p1);
+  }
+  float a, b;
+  unpk2(fadd2(fadd2(lsum2[0], lsum2[1]), fadd2(lsum2[2], lsum2[3])), a, b);
+  st.l_run += a + b;
+  return alpha;
+}
+
+template <class C>
+__global__ void __launch_bounds__(C::THREADS, 1) masked_attn_fwd_kernel(const __grid_constant__ Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t sbase = (raw + 1023u) & ~1023u;
+  uint32_t* misc = reinterpret_cast<uint32_t*>(smem_raw + (sbase - raw) + C::OFF_MISC);
+  const uint32_t bar0 = sbase + C::OFF_BAR;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const Guard guard{smem_u32(misc + 1), 0u, p.status, p.timeout_ns};
+#define BAR(i) (bar0 + 8u * uint32_t(i))
+
+  if (tid == 0) {
+    mbar_init(BAR(C::B_QFULL), 1);
+    mbar_init(BAR(C::B_QEMPTY), 1);
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(BAR(C::B_KVFULL + s), 1);
+      mbar_init(BAR(C::B_KVEMPTY + s), 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(BAR(C::B_SFULL + t), 1);
+      mbar_init(BAR(C::B_SFREE + t), 4);      // one arrival per softmax warp
+      mbar_init(BAR(C::B_PFULL + t), 4);
+      mbar_init(BAR(C::B_PVDONE + t), 1);
+      mbar_init(BAR(C::B_OEMPTY + t), 4);
+      mbar_init(BAR(C::B_DRAIN + t), 1);
+    }
+    misc[1] = 0u;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    prefetch_tmap(&p.tm_q);
+    prefetch_tmap(&p.tm_k);
+    prefetch_tmap(&p.tm_v);
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(smem_u32(misc))
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = misc[0];
+  const int i_begin = p.cta_off[blockIdx.x], i_end = p.cta_off[blockIdx.x + 1];
+
+  if (warp < 4) {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::REG_LOW));
+  if (warp == 0) {
+    // ================================ TMA producer ================================
+    if (lane == 0) {
+      uint32_t rc = 0;
+      int n = 0, q_last = -1;
+      for (int ii = i_begin; ii < i_end; ++ii, ++n) {
+        const WorkItem it = p.items[p.cta_items[ii]];
+        if constexpr (C::PAGED) {
+          prefetch_l1(p.page_table + it.k_base);
+          if (ii + 1 < i_end) prefetch_l1(p.page_table + p.items[p.cta_items[ii + 1]].k_base);
+        }
+        if (!wait_bounded(BAR(C::B_QEMPTY), (n & 1) ^ 1, guard, kWaitQEmpty)) break;
+        if (!((p.debug_flags & 1) && n == 0)) {
+          mbar_expect_tx(BAR(C::B_QFULL), 2 * C::Q_BYTES);
+          q_last = n;
+          for (int t = 0; t < 2; ++t)
+            for (int hh = 0; hh < p.hp; ++hh)
+              for (int c = 0; c < C::NBOX; ++c)
+                tma_load_3d(sbase + C::OFF_Q + t * C::Q_BYTES + c * C::BOX_BYTES + hh * p.R * 128, &p.tm_q, c * 64,
+                            it.head[t] + hh, it.tok[t], BAR(C::B_QFULL));
+        }
+        auto load_tile = [&](bool is_v, int j) -> bool {
+          const int kt = p.jobs[it.job_start + j].k_tile;
+          const CUtensorMap* tm = is_v ? &p.tm_v : &p.tm_k;
+          const uint32_t slot = rc % C::STAGES;
+          if (!wait_bounded(BAR(C::B_KVEMPTY + slot), ((rc / C::STAGES) & 1) ^ 1, guard, kWaitKvEmpty)) return false;
+          mbar_expect_tx(BAR(C::B_KVFULL + slot), C::CHUNK_BYTES);
+          const uint32_t dst = sbase + C::OFF_RING + slot * C::CHUNK_BYTES;
+          if constexpr (!C::PAGED) {
+            for (int c = 0; c < C::NBOX; ++c)
+              tma_load_3d(dst + c * C::BOX_BYTES, tm, c * 64, it.kv_head, it.k_base + kt * 128, BAR(C::B_KVFULL + slot));
+          } else {
+            const int ps = p.page_size, ppt = 128 / ps;
+            if (!is_v) {
+              const int ahead = (kt + 2) * ppt;
+              if (ahead < it.npages) prefetch_l1(p.page_table + it.k_base + ahead);
+            }
+            int32_t page[8];
+#pragma unroll
+            for (int pg = 0; pg < 8; ++pg) {
+              const int idx = kt * ppt + pg;
+              page[pg] = (pg < ppt && idx < it.npages) ? __ldg(p.page_table + it.k_base + idx) : -1;
+            }
+#pragma unroll
+            for (int pg = 0; pg < 8; ++pg) {
+              if (pg >= ppt) break;
+              int32_t row = p.num_pages * ps;  // fully out of bounds: the box reads zeros
+              if (page[pg] >= 0 && page[pg] < p.num_pages) row = page[pg] * ps;
+              for (int c = 0; c < C::NBOX; ++c)
+                tma_load_3d(dst + c * C::BOX_BYTES + pg * ps * 128, tm, c * 64, it.kv_head, row, BAR(C::B_KVFULL + slot));
+            }
+          }
+          ++rc;
+          return true;
+        };
+        const int J = it.job_count;
+        bool ok = load_tile(false, 0);
+        for (int j = 1; ok && j < J; ++j) {
+          ok = load_tile(false, j);
+          if (ok) ok = load_tile(true, j - 1);
+        }
+        if (ok) ok = load_tile(true, J - 1);
+        if (!ok) break;
+      }
+      for (uint32_t r = rc > uint32_t(C::STAGES) ? rc - C::STAGES : 0u; r < rc; ++r)
+        wait_drain(BAR(C::B_KVFULL + r % C::STAGES), (r / C::STAGES) & 1, p.timeout_ns);
+      if (q_last >= 0) wait_drain(BAR(C::B_QFULL), q_last & 1, p.timeout_ns);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ================================ Q K^T issuer ================================
+    if (lane == 0) {
+      uint32_t base = 0;              // ring position of the item's first chunk
+      uint32_t nfree[2] = {0u, 0u};   // S-free phases consumed per tile
+      uint32_t produced = 0;          // Q K^T groups issued so far
+      int n = 0;
+      for (int ii = i_begin; ii < i_end; ++ii, ++n) {
+        const int J = p.items[p.cta_items[ii]].job_count;
+        if (!wait_bounded(BAR(C::B_QFULL), n & 1, guard, kWaitQFull)) break;
+        bool ok = true;
+        for (int j = 0; ok && j < J; ++j) {
+          const uint32_t rk = base + uint32_t(k_pos(j));
+          if (!wait_bounded(BAR(C::B_KVFULL + rk % C::STAGES), (rk / C::STAGES) & 1, guard, kWaitKvFull)) {
+            ok = false;
+            break;
+          }
+          const uint32_t klo = desc_lo(sbase + C::OFF_RING + (rk % C::STAGES) * C::CHUNK_BYTES, 16);
+          for (int t = 0; t < 2; ++t) {
+            // the previous scores in S (the other tile's) have been read
+            if (produced > 0) {
+              const int prev = t ^ 1;
+              if (!wait_bounded(BAR(C::B_SFREE + prev), nfree[prev] & 1, guard, kWaitSFull)) {
+                ok = false;
+                break;
+              }
+              ++nfree[prev];
+            }
+            tc_fence_after();
+            const uint32_t qlo = desc_lo(sbase + C::OFF_Q + t * C::Q_BYTES, 16);
+            if constexpr (C::D == 128) mma_ss_x8_k128(tmem + C::TM_S, desc_of(qlo), desc_of(klo), C::IDESC_QK, 0u);
+            else mma_ss_x4_k64(tmem + C::TM_S, desc_of(qlo), desc_of(klo), C::IDESC_QK, 0u);
+            mma_commit(BAR(C::B_SFULL + t));
+            ++produced;
+          }
+          if (!ok) break;
+          mma_commit(BAR(C::B_KVEMPTY + rk % C::STAGES));
+        }
+        if (!ok) break;
+        mma_commit(BAR(C::B_QEMPTY));
+        base += 2u * uint32_t(J);
+      }
+      mma_commit(BAR(C::B_DRAIN + 0));
+      wait_drain(BAR(C::B_DRAIN + 0), 0, p.timeout_ns);
+    }
+    __syncwarp();
+  } else if (warp == 2) {
+    // ================================ P V issuer ================================
+    if (lane == 0) {
+      uint32_t base = 0;
+      uint32_t pc[2] = {0u, 0u};      // P phases consumed per tile
+      int n = 0;
+      for (int ii = i_begin; ii < i_end; ++ii, ++n) {
+        const WorkItem* itp = p.items + p.cta_items[ii];
+        const int J = itp->job_count, job_start = itp->job_start;
+        const int kv_len = C::PAGED ? itp->kv_len : 0, npages = C::PAGED ? itp->npages : 0;
+        bool ok = true;
+        for (int j = 0; ok && j < J; ++j) {
+          const uint32_t rv = base + uint32_t(v_pos(j, J));
+          if (!wait_bounded(BAR(C::B_KVFULL + rv % C::STAGES), (rv / C::STAGES) & 1, guard, kWaitKvFull)) {
+            ok = false;
+            break;
+          }
+          const uint32_t vbase = sbase + C::OFF_RING + (rv % C::STAGES) * C::CHUNK_BYTES;
+          if constexpr (C::PAGED) {
+            int r0, r1;
+            v_tail_rows(p.jobs[job_start + j].k_tile, kv_len, npages, p.page_size, r0, r1);
+            if (r0 < r1) zero_v_rows(vbase, 0u, C::NBOX, r0, r1, 0, 1);
+          }
+          for (int t = 0; t < 2; ++t) {
+            if (!wait_bounded(BAR(C::B_PFULL + t), pc[t] & 1, guard, kWaitPFull)) {
+              ok = false;
+              break;
+            }
+            ++pc[t];
+            if (j == 0 && !wait_bounded(BAR(C::B_OEMPTY + t), (n & 1) ^ 1, guard, kWaitOEmpty)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            mma_ts_x8(tmem + C::TM_O + t * C::D, tmem + C::TM_P + 64 * t, desc_of(desc_lo(vbase, C::BOX_BYTES)),
+                      C::IDESC_PV, j == 0 ? 0u : 1u);
+            mma_commit(BAR(C::B_PVDONE + t));
+          }
+          if (!ok) break;
+          mma_commit(BAR(C::B_KVEMPTY + rv % C::STAGES));
+        }
+        if (!ok) break;
+        base += 2u * uint32_t(J);
+      }
+      mma_commit(BAR(C::B_DRAIN + 1));
+      wait_drain(BAR(C::B_DRAIN + 1), 0, p.timeout_ns);
+    }
+    __syncwarp();
+  }
+  } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(C::REG_HIGH));
+    // ================================ softmax warpgroup of query tile q ================================
+    const int q = warp / 4 - 1;
+    const int r = tid - 128 * (1 + q);                // row of the tile = TMEM lane
+    const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
+    const uint32_t t_o = tmem + lane_base + C::TM_O + q * C::D;
+    const uint32_t t_p = tmem + lane_base + C::TM_P + 64 * q;
+    const float sl2 = p.scale_log2;
+    uint32_t sc = 0, pc = 0;   // S phases consumed, P published
+    bool ok = true;
+    auto wait_pv = [&]() -> bool {   // the P V of the last P published is done
+      if (pc == 0) return true;
+      return __all_sync(0xffffffffu, wait_bounded(BAR(C::B_PVDONE + q), (pc - 1) & 1, guard, kWaitPvDone));
+    };
+    for (int ii = i_begin; ok && ii < i_end; ++ii) {
+      const WorkItem it = p.items[p.cta_items[ii]];
+      const int J = it.job_count;
+      RowState st{-INFINITY, 0.f};
+      for (int j = 0; j < J; ++j) {
+        const int mi = p.jobs[it.job_start + j].mask[q];
+        uint4 bits = make_uint4(0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu);
+        if (mi >= 0) bits = __ldg(p.mask_tiles + int64_t(mi) * 128 + r);
+        else if (mi == kMaskNone) bits = make_uint4(0u, 0u, 0u, 0u);
+        if (!__all_sync(0xffffffffu, wait_bounded(BAR(C::B_SFULL + q), sc & 1, guard, kWaitSFull))) {
+          ok = false;
+          break;
+        }
+        ++sc;
+        tc_fence_after();
+        bool need;
+        uint32_t pk[64];
+        const float alpha = softmax_regs<C::EMU>(tmem + lane_base + C::TM_S, mi, bits, sl2, st, need, pk, [&] {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(BAR(C::B_SFREE + q));
+        });
+        // the previous P V of this tile has read its P and added into O
+        if (!wait_pv()) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (j > 0 && __any_sync(0xffffffffu, need)) rescale_o<C::D>(t_o, alpha);
+        tmem_st32x16(t_p + 0, pk + 0);
+        tmem_st32x16(t_p + 16, pk + 16);
+        tmem_st32x16(t_p + 32, pk + 32);
+        tmem_st32x16(t_p + 48, pk + 48);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(BAR(C::B_PFULL + q));
+        ++pc;
+      }
+      if (!ok) break;
+      // ---- epilogue ----
+      if (!wait_pv()) break;
+      tc_fence_after();
+      const int lr = r % p.R, hh = r / p.R;
+      if (it.part < 0)
+        store_row<C::D>(t_o, st, lr < it.rows[q], int64_t(it.tok[q] + lr) * p.hq + it.head[q] + hh, p.out, p.lse);
+      else
+        store_partial<C::D>(t_o, st, lr < it.rows[q], int64_t(it.part + q) * kSlotRows + r, p.part_o, p.part_lse);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(BAR(C::B_OEMPTY + q));
+    }
+  }
+#undef BAR
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem) : "memory");
+}
+
 // ================================ cluster-pair kernel (head_dim 256) ================================
 // Two CTAs on the two SMs of a pair cooperate on one work item: CTA r owns query tile r
 // (128 rows) and its TMEM rows; the pair's leader (r = 0) issues 2-SM MMAs of M = 256:
@@ -768,6 +1191,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::THREADS, 1)
           ++rc;
           tc_fence_after();
           const uint32_t vbase = sbase + C::OFF_RING + (rv % C::STAGES) * C::SLOT_BYTES;
+          if constexpr (C::PAGED) {
+            // both CTAs' V halves: the leader writes the peer's through its cluster address
+            int r0, r1;
+            v_tail_rows(p.jobs[it.job_start + u].k_tile, it.kv_len, it.npages, p.page_size, r0, r1);
+            if (r0 < r1) zero_v_rows(vbase, mapa_shared(vbase, 1), C::VBOX, r0, r1, 0, 1);
+          }
           const uint32_t a_p = tmem + 128 * slot, acc0 = u == 0 ? 0u : 1u;
           if constexpr (C::FP8) mma2_8_ts_x4(tmem + C::TM_O, a_p, desc_of(desc_lo(vbase, 16)), C::IDESC_PV, acc0);
           else mma2_ts_x8(tmem + C::TM_O, a_p, desc_of(desc_lo(vbase, C::VH_BOX)), C::IDESC_PV, acc0);
@@ -919,12 +1348,31 @@ __global__ void fill_empty_kernel(float* lse, int64_t n) {
 #define MFA_EMU_D128 0
 #endif
 
+
 template <class C>
 attn_status_t launch(const attn_plan_t* plan, Params& p, cudaStream_t stream) {
   const cudaError_t attr = once_per_device([] {
-    cudaError_t e = cudaFuncSetAttribute(masked_attn_fwd_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(masked_attn_fwd_e4m3_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          C::SMEM_BYTES);
     if (e == cudaSuccess && C::REG_SPLIT) {
+      // setmaxnreg.inc draws on the registers the block was launched with: the split must fit
+      cudaFuncAttributes fa{};
+      e = cudaFuncGetAttributes(&fa, masked_attn_fwd_e4m3_kernel<C>);
+      if (e == cudaSuccess && fa.numRegs * C::THREADS < C::REG_SPLIT_TOTAL) e = cudaErrorInvalidConfiguration;
+    }
+    return e;
+  });
+  if (attr != cudaSuccess) return ATTN_ERR_CUDA;
+  masked_attn_fwd_e4m3_kernel<C><<<plan->ctas, C::THREADS, C::SMEM_BYTES, stream>>>(p);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+template <class C>
+attn_status_t launch_sharedS(const attn_plan_t* plan, Params& p, cudaStream_t stream) {
+  const cudaError_t attr = once_per_device([] {
+    cudaError_t e = cudaFuncSetAttribute(masked_attn_fwd_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         C::SMEM_BYTES);
+    if (e == cudaSuccess) {
       // setmaxnreg.inc draws on the registers the block was launched with: the split must fit
       cudaFuncAttributes fa{};
       e = cudaFuncGetAttributes(&fa, masked_attn_fwd_kernel<C>);
@@ -1018,11 +1466,11 @@ attn_status_t mfa_launch_forward(const attn_plan_t* plan, const void* q, const v
   plan_params(plan, out, lse, p);
   attn_status_t st;
   if (D == 64) {
-    st = plan->paged ? launch<Cfg<64, 2, 10, true, MFA_EMU_D128>>(plan, p, stream)
-                     : launch<Cfg<64, 2, 10, false, MFA_EMU_D128>>(plan, p, stream);
+    st = plan->paged ? launch_sharedS<SCfg<64, true, MFA_EMU_D128>>(plan, p, stream)
+                     : launch_sharedS<SCfg<64, false, MFA_EMU_D128>>(plan, p, stream);
   } else if (D == 128) {
-    st = plan->paged ? launch<Cfg<128, 2, 5, true, MFA_EMU_D128>>(plan, p, stream)
-                     : launch<Cfg<128, 2, 5, false, MFA_EMU_D128>>(plan, p, stream);
+    st = plan->paged ? launch_sharedS<SCfg<128, true, MFA_EMU_D128>>(plan, p, stream)
+                     : launch_sharedS<SCfg<128, false, MFA_EMU_D128>>(plan, p, stream);
   } else {
     st = plan->paged ? launch_pair<PairCfg<256, 5, true>>(plan, p, stream)
                      : launch_pair<PairCfg<256, 5, false>>(plan, p, stream);

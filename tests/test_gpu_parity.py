@@ -99,9 +99,14 @@ def test_canary_rows_untouched_and_outputs_deterministic():
     assert torch.equal(out[:tq], out2) and torch.equal(lse[:tq], lse2)
 
 
-def test_paged_poison_in_unused_slots():
-    # keys past kv_len in the last page and unreferenced pages hold a large finite value
-    wl = W.random_small(seed=21, kind="CUSTOM", batch=4, hq=4, hkv=2, d=128, lmin=20, lmax=400, paged=True)
+@pytest.mark.parametrize("poison", ["finite", "nan", "inf"])
+@pytest.mark.parametrize("d", [64, 128, 256])
+@pytest.mark.parametrize("kind", ["CUSTOM", "CAUSAL"])
+def test_paged_poison_in_unused_slots(kind, d, poison):
+    # Cache slots no sequence owns -- keys past kv_len in a sequence's last page and pages
+    # no page table names -- hold whatever a serving cache left there: a large finite value,
+    # NaN or Inf. The output must be bit-identical to the one with clean slots.
+    wl = W.random_small(seed=21 + d, kind=kind, batch=4, hq=4, hkv=2, d=d, lmin=20, lmax=400, paged=True)
     ref = G.run(wl, wl.masks[0])
     kc, vc = wl.k_cache.clone(), wl.v_cache.clone()
     used = np.zeros((kc.shape[0], wl.page_size), bool)
@@ -110,8 +115,10 @@ def test_paged_poison_in_unused_slots():
         for j in range(n):
             used[wl.page_table[b, j // wl.page_size], j % wl.page_size] = True
     mask = torch.from_numpy(~used)
-    kc[mask] = 3.0e4
-    vc[mask] = -3.0e4
+    assert mask.any() and bool(mask[np.unique(wl.page_table[wl.page_table >= 0])].any()), \
+        "some last page must be partly unused"
+    kv = {"finite": (3.0e4, -3.0e4), "nan": (float("nan"), float("nan")), "inf": (float("inf"), -float("inf"))}
+    kc[mask], vc[mask] = kv[poison]
     wl.k_cache, wl.v_cache = kc, vc
     out, lse, _ = G.run(wl, wl.masks[0])
     assert torch.equal(out, ref[0]) and torch.equal(lse, ref[1])

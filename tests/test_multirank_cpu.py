@@ -89,3 +89,7 @@ def test_traffic_figures_are_keyed_to_the_current_kernel_sources():
     for name, entry in table.items():
         assert entry["kernel_source_hash"] == bench.kernel_source_hash(), f"stale traffic entry {name}"
         assert bench.traffic_for(name) == entry["dram_bytes_per_launch"]
+        # a figure is measured on the source it is keyed to: a capture taken on other source
+        # and relabelled afterwards is not a measurement of this kernel
+        assert entry.get("captured_at_hash", entry["kernel_source_hash"]) == entry["kernel_source_hash"], name
+        assert "re-key" not in entry.get("note", "") and "rekey" not in entry.get("note", ""), name
