@@ -325,7 +325,16 @@ const char* attn_status_string(attn_status_t status);
  *   - Every call reuses the same array and overwrites what the previous call left there
  *     (the status word is cleared each time), so calls whose work overlaps on the GPU --
  *     different streams, or another host thread -- race; serialise them on one stream.
- * Errors: INVALID_ARG, UNSUPPORTED, TOO_LARGE, CUDA. */
+ *     Calls queued back to back on one stream are fine: each copy into the array waits
+ *     for the previous forward on that stream.
+ *   - In-kernel waits are bounded like those of attn_masked_fwd(), but no plan outlives the
+ *     call, so an expired wait cannot be queried afterwards. It shows in the output instead:
+ *     when lse is given, the call first fills it with NaN (on `stream`, before the forward),
+ *     and every row the kernel completes overwrites its lse with a finite value or -inf
+ *     (a row that sees no key). A row whose lse is still NaN after the stream has finished
+ *     was not computed; its out holds whatever the buffer held. With lse == NULL there is
+ *     no such signal.
+ * Errors: INVALID_ARG, UNSUPPORTED, TOO_LARGE, CUDA (launch or enqueue failures only). */
 #define ATTN_NOALLOC_SCRATCH_BYTES (32u << 20)
 attn_status_t attn_masked_fwd_noalloc(const attn_problem_t* problem, const attn_mask_desc_t* mask,
                                       const void* q, const void* k, const void* v, void* out, float* lse,

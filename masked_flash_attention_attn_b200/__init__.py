@@ -47,7 +47,7 @@ EXPORTS = ("attn_plan", "attn_masked_fwd", "attn_plan_get_tile_classes", "attn_p
            "attn_plan_check_status", "attn_plan_set_debug", "attn_plan_destroy", "attn_classify_host",
            "attn_status_string", "attn_masked_fwd_noalloc", "attn_test_exp2_poly", "attn_plan_dry_run",
            "attn_plan_bwd", "attn_masked_bwd", "attn_masked_fwd_fp8", "attn_fp8_transpose_v",
-           "attn_test_transpose_mask_tile")
+           "attn_test_transpose_mask_tile", "attn_test_noalloc_debug")
 
 
 class AttnError(RuntimeError):
@@ -122,6 +122,7 @@ def lib() -> ctypes.CDLL:
                                         ctypes.POINTER(attn_plan_stats_t)]
         L.attn_masked_fwd_noalloc.argtypes = [ctypes.POINTER(attn_problem_t), ctypes.POINTER(attn_mask_desc_t),
                                               vp, vp, vp, vp, vp, vp]
+        L.attn_test_noalloc_debug.argtypes = [i32, i64]
         for n in EXPORTS:
             if n != "attn_status_string":
                 getattr(L, n).restype = i32
@@ -456,7 +457,9 @@ def attn_masked_fwd_noalloc(*, hq: int, hkv: int, head_dim: int, cu_seqlens_q, m
     For callers that may not allocate device memory (e.g. a runtime that owns every device
     allocation through its own pool): the plan goes into a fixed 32 MiB array inside the
     library instead of a cudaMalloc'd workspace. Calls that overlap on the GPU race on that
-    array; keep them on one stream. CUSTOM masks are not accepted here."""
+    array; keep them on one stream. CUSTOM masks are not accepted here. An in-kernel wait
+    that expires leaves the rows it did not compute with lse = NaN (lse is filled with NaN
+    first); pass lse to see it."""
     _check_page_table(page_table, cu_seqlens_q)
     m = _Marshal()
     pr = _problem(m, hq=hq, hkv=hkv, head_dim=head_dim, cu_seqlens_q=cu_seqlens_q, cu_seqlens_k=cu_seqlens_k,
@@ -471,6 +474,11 @@ def attn_masked_fwd_noalloc(*, hq: int, hkv: int, head_dim: int, cu_seqlens_q, m
                     (lse, "lse", _f32(), total_q * hq, True))
     _check(lib().attn_masked_fwd_noalloc(ctypes.byref(pr), ctypes.byref(d), *args, _stream(stream)),
            "attn_masked_fwd_noalloc")
+
+
+def attn_test_noalloc_debug(flags: int, timeout_ns: int) -> None:
+    """Test hook: debug flags / wait limit of the following attn_masked_fwd_noalloc() calls."""
+    _check(lib().attn_test_noalloc_debug(int(flags), int(timeout_ns)), "attn_test_noalloc_debug")
 
 
 def attn_test_exp2_poly(x, y, stream=None) -> None:

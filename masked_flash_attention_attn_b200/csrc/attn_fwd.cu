@@ -21,6 +21,7 @@
 #include <cudaTypedefs.h>
 #include <cuda_bf16.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <mutex>
@@ -1564,6 +1565,9 @@ namespace {
 constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mu;
 void* g_noalloc_addr[kMaxDevices] = {};
+// test hook (attn_test_noalloc_debug): debug flags and wait limit of the following calls
+std::atomic<int32_t> g_noalloc_debug_flags{0};
+std::atomic<int64_t> g_noalloc_timeout_ns{2000000000LL};
 
 // Device address of g_noalloc_scratch on the current device, looked up once per device.
 attn_status_t noalloc_scratch(int dev, void** out) {
@@ -1602,6 +1606,12 @@ extern "C" attn_status_t attn_masked_fwd_noalloc(const attn_problem_t* problem, 
   // the bytes start with a zeroed status word: each call clears what the previous one left
   if (cudaMemcpyAsync(scratch, hp.bytes.data(), hp.bytes.size(), cudaMemcpyHostToDevice, stream) != cudaSuccess)
     return ATTN_ERR_CUDA;
+  // No plan survives this call, so an in-kernel wait that expires cannot be reported through a
+  // status query. Instead lse starts as NaN: every row the kernel completes overwrites it with
+  // a finite value or -inf, so rows still NaN afterwards are the ones that were not computed.
+  if (lse && cudaMemsetAsync(lse, 0xFF, size_t(hp.meta.total_q) * size_t(hp.meta.hq) * sizeof(float), stream) !=
+                 cudaSuccess)
+    return ATTN_ERR_CUDA;
   char* base = static_cast<char*>(scratch);
   attn_plan_t& plan = hp.meta;
   plan.d_status = reinterpret_cast<int32_t*>(base);
@@ -1610,7 +1620,16 @@ extern "C" attn_status_t attn_masked_fwd_noalloc(const attn_problem_t* problem, 
   plan.d_cta_off = reinterpret_cast<const int32_t*>(base + hp.off_cta_off);
   plan.d_cta_items = reinterpret_cast<const int32_t*>(base + hp.off_cta_items);
   plan.d_mask_tiles = reinterpret_cast<const uint4*>(base + hp.off_tiles);
+  plan.debug_flags = g_noalloc_debug_flags.load();
+  plan.timeout_ns = g_noalloc_timeout_ns.load();
   // (a copy from pageable host memory returns once the source has been staged, so the host
   // bytes may go away when this function returns)
   return mfa_launch_forward(&plan, q, k, v, out, lse, stream);
+}
+
+extern "C" attn_status_t attn_test_noalloc_debug(int32_t flags, int64_t timeout_ns) {
+  if (flags < 0 || timeout_ns <= 0) return ATTN_ERR_INVALID_ARG;
+  g_noalloc_debug_flags.store(flags);
+  g_noalloc_timeout_ns.store(timeout_ns);
+  return ATTN_OK;
 }

@@ -103,11 +103,12 @@ def test_chunk_clipped_at_q_end_and_k_range():
 
 def test_sliding_window_inert_equals_causal_and_biting_differs():
     g = dict((r[0], int(r[1])) for r in _read_golden("sliding_window_inert.txt"))
-    L, w = g["max_seq"], g["window_default"]
+    L, w, w_min = g["max_seq"], g["window_default"], g["window_inert_min"]
+    assert w >= w_min == L
     ca = OM.dense_mask(W.MaskSpec("CAUSAL"), 0, L, L)
     assert np.array_equal(OM.dense_mask(W.MaskSpec("SLIDING_WINDOW", window=w), 0, L, L), ca)
-    assert np.array_equal(OM.dense_mask(W.MaskSpec("SLIDING_WINDOW", window=L), 0, L, L), ca)
-    bite = OM.dense_mask(W.MaskSpec("SLIDING_WINDOW", window=L - 1), 0, L, L)
+    assert np.array_equal(OM.dense_mask(W.MaskSpec("SLIDING_WINDOW", window=w_min), 0, L, L), ca)
+    bite = OM.dense_mask(W.MaskSpec("SLIDING_WINDOW", window=w_min - 1), 0, L, L)
     assert not np.array_equal(bite, ca)
     # the local mask is the causal mask AND the window: never more keys than causal
     assert not (bite & ~ca).any()
