@@ -325,10 +325,10 @@ def device_inputs(wl, dev):
     return q, wl.k.to(dev), wl.v.to(dev)
 
 
-def make_plan(M, wl, spec, dev, kv_splits=0, backward=False):
+def make_plan(M, wl, spec, dev, kv_splits=0, backward=False, q_rows=None):
     import torch
     kw = dict(hq=wl.hq, hkv=wl.hkv, head_dim=wl.d, cu_seqlens_q=wl.cu_seqlens_q, mask=spec, scale=wl.scale,
-              kv_splits=kv_splits, backward=backward)
+              kv_splits=kv_splits, backward=backward, q_rows=q_rows)
     if wl.paged:
         kw.update(kv_lens=wl.kv_lens, page_table=torch.from_numpy(wl.page_table).to(dev),
                   page_size=wl.page_size, num_pages=wl.k_cache.shape[0])
@@ -447,6 +447,120 @@ def time_config(M, cfg, dev, stream, steps, warmup, peak, hbm_peak):
     del q, k, v, outs, lses, flush, plans
     torch.cuda.empty_cache()
     return entry
+
+
+def shard_rows_plan(M, wl, world):
+    """Query-row shards of one problem for `world` ranks: work-balanced by the host tile
+    classes of the workload's analytic mask form (a CUSTOM-only workload gets equal row
+    blocks). Returns [(begin, end)] sequence-local rows per rank."""
+    from masked_flash_attention_attn_b200 import sharding as S
+    lengths = [(wl.lq(b), wl.lk(b)) for b in range(wl.batch)]
+    analytic = next((m for m in wl.masks if m.kind != "CUSTOM"), None)
+    if analytic is None:
+        lq_max = max(lq for lq, _ in lengths)
+        return [S.query_shard(lq_max, r, world) for r in range(world)]
+    cls, _ = M.attn_classify_host(hq=wl.hq, hkv=wl.hkv, head_dim=wl.d, cu_seqlens_q=wl.cu_seqlens_q,
+                                  cu_seqlens_k=wl.cu_seqlens_k, mask=analytic)
+    return S.balanced_query_shards(cls, lengths, world)
+
+
+def run_shard_rows(args, rank, world, local_rank):
+    """One problem split over the ranks by query rows (--shard-rows): every rank plans its
+    own rows of every sequence against all keys; K and V start sharded by rows across the
+    ranks and each step first all-gathers them (NCCL all_gather_into_tensor into every GPU's
+    own memory), then runs the forward of every mask of the workload on this rank's rows.
+    The timed step is gather + forward; the value is the whole problem's work over the
+    slowest rank's time (strong scaling: the total work is fixed)."""
+    import torch
+    import torch.distributed as dist
+    import masked_flash_attention_attn_b200 as M
+    from masked_flash_attention_attn_b200 import sharding as S
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    wl = workload(args.config, 0)            # the same problem on every rank
+    if wl.paged:
+        raise SystemExit("--shard-rows: a workload with contiguous K/V (1, 2, 4 or 5)")
+    stream = torch.cuda.current_stream()
+    shards = shard_rows_plan(M, wl, world)
+    q_rows = shards[rank]
+    total_k = int(wl.cu_seqlens_k[-1])
+    a, b = S.row_shard(total_k, rank, world)
+    k_local, v_local = wl.k[a:b].to(dev), wl.v[a:b].to(dev)
+    q = wl.q.to(dev)
+    gk = S.RowGather(total_k, (wl.hkv, wl.d), torch.bfloat16, dev)
+    gv = S.RowGather(total_k, (wl.hkv, wl.d), torch.bfloat16, dev)
+    plans = [make_plan(M, wl, stage_mask(spec, dev), dev, q_rows=q_rows) for spec in wl.masks]
+    stats = [M.attn_plan_get_stats(p) for p in plans]
+    full_flops = 0.0
+    for spec in wl.masks:   # the whole problem's work (every rank's shard together)
+        full_flops += flops_of(M.attn_plan_get_stats(make_plan(M, wl, stage_mask(spec, dev), dev)), wl)
+    tq = q.shape[0]
+    outs = [torch.empty(tq, wl.hq, wl.d, dtype=torch.bfloat16, device=dev) for _ in plans]
+    lses = [torch.empty(tq, wl.hq, dtype=torch.float32, device=dev) for _ in plans]
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        k, v = gk.gather(k_local), gv.gather(v_local)
+        if ev is not None:
+            ev[1].record(stream)
+        for i, p in enumerate(plans):
+            M.attn_masked_fwd(p, q, k, v, outs[i], lses[i], stream)
+        if ev is not None:
+            ev[2].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local_rank, args.clock_log)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler.mark_start()
+    t0.record(stream)
+    for s_ in range(args.steps):
+        step(ev[s_])
+    t1.record(stream)
+    while not t1.query():
+        time.sleep(2e-4)
+    sampler.mark_end()
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    if world > 1:
+        dist.barrier()
+    for p in plans:
+        st = M.attn_plan_check_status(p)
+        if st != 0:
+            raise RuntimeError(f"forward reported {M.STATUS.get(st, st)}")
+    ms = t0.elapsed_time(t1)
+    gather_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
+    fwd_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
+    jobs = sum(s["jobs"] for s in stats)
+    (ms, gather_ms, fwd_ms), _ = reduce_over_ranks([ms, gather_ms, fwd_ms], 0.0, dev)
+    if rank != 0:
+        return
+    value = full_flops * args.steps / (ms * 1e-3) / 1e12
+    kv_bytes = 2 * total_k * wl.hkv * wl.d * 2
+    peak, pk_src, _ = choose_peak(clocks)
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "strong",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) bf16, lengths from seed)",
+        "config": dict(config_of(wl, args, world),
+                       parallelism=f"query-row shards x{world} + NCCL K/V all-gather (one problem, no batch split)",
+                       shards=shards),
+        "pct_of_peak": 100.0 * value / world / peak, "peak_source": pk_src,
+        "gather": {"kv_bytes": kv_bytes, "bytes_received_per_rank": gk.bytes_received + gv.bytes_received,
+                   "ms": gather_ms,
+                   "gbs_per_rank": (gk.bytes_received + gv.bytes_received) / (gather_ms * 1e-3) / 1e9
+                   if world > 1 and gather_ms > 0 else None},
+        "forward_ms": fwd_ms, "jobs_rank0": jobs,
+        "gpu_launches": len(plans) * args.steps,
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
 
 
 def run_ours(args, rank, world, local_rank):
@@ -746,6 +860,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-per-config", action="store_true",
                     help="skip timing the other benchmark workloads after the headline")
+    ap.add_argument("--shard-rows", action="store_true",
+                    help="split ONE problem over the ranks by query rows, with a K/V all-gather per step "
+                         "(strong scaling; contiguous K/V workloads)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -763,7 +880,10 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
     try:
-        run_ours(args, rank, world, local_rank)
+        if args.shard_rows:
+            run_shard_rows(args, rank, world, local_rank)
+        else:
+            run_ours(args, rank, world, local_rank)
     finally:
         if world > 1:
             import torch.distributed as dist

@@ -42,6 +42,42 @@ def all_gather_rows(local, rows: int, group=None):
     return out[:rows]
 
 
+class RowGather:
+    """all_gather_rows with buffers allocated once: every call sends this rank's rows of a
+    row-sharded [rows, ...] tensor and receives the full tensor (one all_gather_into_tensor
+    over equal padded parts; with one rank, a copy). For a step that repeats the gather (a
+    timed loop, every layer of a model), so that no allocation happens per call."""
+
+    def __init__(self, rows: int, feature_shape, dtype, device, group=None):
+        import torch
+        import torch.distributed as dist
+        self.group = group
+        self.world = dist.get_world_size(group) if dist.is_available() and dist.is_initialized() else 1
+        self.rows = rows
+        self.per = (rows + self.world - 1) // self.world
+        self.send = torch.zeros((self.per,) + tuple(feature_shape), dtype=dtype, device=device)
+        self.full = torch.empty((self.per * self.world,) + tuple(feature_shape), dtype=dtype, device=device)
+
+    def gather(self, local):
+        """local: this rank's rows (row_shard(rows, rank, world)); returns the full [rows, ...]
+        tensor (a view of the receive buffer, valid until the next call)."""
+        import torch.distributed as dist
+        n = local.shape[0]
+        if n > self.per:
+            raise ValueError("local rows exceed this rank's share")
+        self.send[:n].copy_(local)
+        if self.world == 1:
+            self.full[:self.per].copy_(self.send)
+        else:
+            dist.all_gather_into_tensor(self.full, self.send, group=self.group)
+        return self.full[:self.rows]
+
+    @property
+    def bytes_received(self) -> int:
+        """Bytes that land on this rank per call (the other ranks' parts)."""
+        return (self.world - 1) * self.send.numel() * self.send.element_size()
+
+
 def balanced_query_shards(tile_classes, lengths, world: int, block: int = 128):
     """Row shards [begin, end) for every rank (sequence-local rows, whole `block`-row tiles)
     that give each rank about the same number of non-empty 128 x 128 tiles, summed over the

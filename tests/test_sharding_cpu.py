@@ -43,6 +43,39 @@ def _gather_worker(rank, world, port, rows, q):
         dist.destroy_process_group()
 
 
+def _row_gather_worker(rank, world, port, rows, q):
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        g = S.RowGather(rows, (2, 3), torch.float32, "cpu")
+        ok = True
+        for step in range(3):   # the same buffers serve every call
+            full = (torch.arange(rows * 6, dtype=torch.float32) + 1000 * step).reshape(rows, 2, 3)
+            a, b = S.row_shard(rows, rank, world)
+            got = g.gather(full[a:b].clone())
+            ok = ok and bool(torch.equal(got, full)) and got.shape[0] == rows
+        ok = ok and g.bytes_received == (world - 1) * ((rows + world - 1) // world) * 6 * 4
+        q.put((rank, ok))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("rows,world", [(10, 2), (7, 3), (2, 3)])
+def test_row_gather_reuses_its_buffers_gloo(rows, world):
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = 29750 + 10 * world + rows
+    procs = [ctx.Process(target=_row_gather_worker, args=(r, world, port, rows, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = [q.get(timeout=120) for _ in procs]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert all(ok for _, ok in res)
+
+
 @pytest.mark.parametrize("rows,world", [(10, 2), (7, 2), (7, 3), (2, 3)])   # (2, 3): a rank holds no rows
 def test_all_gather_rows_gloo(rows, world):
     ctx = mp.get_context("spawn")
@@ -78,3 +111,16 @@ def test_balanced_shards_even_out_causal_work(attn_lib):
     assert sum(jobs_bal) == full["jobs"] == sum(jobs_eq)
     assert max(jobs_eq) > 1.3 * (full["jobs"] / world)         # equal rows: imbalanced
     assert max(jobs_bal) < 1.15 * (full["jobs"] / world)       # balanced within 15 %
+
+
+def test_bench_shard_rows_plan_partitions_the_sequence(attn_lib):
+    """bench.py --shard-rows: the shards it plans cover every query row once, in order, for
+    the long block-dense sequence (range form on the host) and a causal batch."""
+    import bench
+    for wl in (W.config(5), W.config(4)):
+        lq_max = max(wl.lq(b) for b in range(wl.batch))
+        for world in (1, 2, 4, 8):
+            sh = bench.shard_rows_plan(attn_lib, wl, world)
+            assert len(sh) == world and sh[0][0] == 0 and sh[-1][1] == lq_max
+            assert all(a[1] == b[0] and a[0] <= a[1] for a, b in zip(sh, sh[1:]))
+            assert all(b % 128 == 0 or b == lq_max for _, b in sh)
