@@ -3,9 +3,12 @@ gradients (oracle/backward.py), on ragged contiguous batches of every mask kind,
 64 and 128, grouped-query heads, rows that see no key and keys no query sees.
 
 Tolerance: P and dS enter the tensor cores as bf16 (relative rounding 2^-9 each) with fp32
-accumulation, and the gradients are stored as bf16; with the forward's bf16 out in
-delta = dout . out the expected error is a few 1e-3 of the gradient scale. The bound
-used: max |err| <= 2e-2 * max |ref| and mean |err| <= 1e-2 * mean |ref|, per tensor."""
+accumulation, and the gradients are stored as bf16 (relative rounding 2^-9, i.e. a mean
+error of about 2e-3 of the mean magnitude from the storage alone); with the forward's bf16
+out in delta = dout . out the expected error is a few 1e-3 of the gradient scale. Measured
+over every case of this file on B200: worst max |err| / max |ref| = 7.2e-3 (dq), worst
+mean |err| / mean |ref| = 3.0e-3. The bound used, per tensor: max |err| <= 1.2e-2 * max |ref|
+and mean |err| <= 5e-3 * mean |ref|."""
 import numpy as np
 import pytest
 import torch
@@ -17,7 +20,7 @@ from tests import gpu_helpers as G
 pytestmark = pytest.mark.gpu
 
 KINDS = ["FULL", "CAUSAL", "SLIDING_WINDOW", "PREFIX_LM", "CHUNK_CAUSAL", "RANGES", "CUSTOM", "BLOCK_SPARSE"]
-REL_MAX, REL_MEAN = 2e-2, 1e-2
+REL_MAX, REL_MEAN = 1.2e-2, 5e-3
 
 
 @pytest.fixture(scope="module", autouse=True)
