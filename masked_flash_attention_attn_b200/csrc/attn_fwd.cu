@@ -5,13 +5,12 @@
 // run of key tiles; empty key tiles never appear in the run, full key tiles carry no mask,
 // partial ones carry the index of a 2 KiB tile-transposed bit mask. Three kernels:
 //
-//   masked_attn_fwd_kernel       (bf16, head_dim 64 / 128): the two query tiles take turns
-//       in one S accumulator in TMEM, P has a TMEM slot of its own per tile, Q K^T and P V
-//       are issued by two different threads (see the kernel's comment).
-//   masked_attn_fwd_e4m3_kernel  (e4m3, head_dim 128): S double buffered, P written over S,
-//       one issuing thread; Q, K and V^T in e4m3 with .kind::f8f6f4 MMAs.
+//   masked_attn_fwd_kernel       (head_dim 64 / 128 in bf16, 128 in e4m3): the two query
+//       tiles take turns in one S accumulator in TMEM, P has a TMEM slot of its own per tile,
+//       Q K^T and P V are issued by two different threads (see the kernel's comment).
 //   masked_attn_fwd_pair_kernel  (head_dim 256, bf16 or e4m3): a CTA pair, one query tile per
-//       CTA, 2-SM MMAs (cta_group::2) so each SM streams half of every K and V tile.
+//       CTA, 2-SM MMAs (cta_group::2) so each SM streams half of every K and V tile; S double
+//       buffered per tile, P written over S.
 //
 // Every wait on an mbarrier is bounded (globaltimer). When a wait expires the thread
 // records ATTN_ERR_TIMEOUT in the plan's status word, raises a shared abort flag that
@@ -51,55 +50,6 @@ struct Params {
   float scale_log2;
   float v_scale;       // e4m3 forward: the value tensor's scale (1 for bf16)
   int64_t timeout_ns;
-};
-
-// Configuration of masked_attn_fwd_e4m3_kernel (FP8_ = true: e4m3 Q, K and V, the latter
-// transposed, [Hkv][d][keys], .kind::f8f6f4 MMAs, P quantised to e4m3 in TMEM; head_dim 128).
-// Warp roles (128 * (1 + NQ) threads): warp 0 TMA producer (Q tiles once per item, K and V
-// tiles through a ring of STAGES chunks); warp 1 MMA issuer (one thread: S = Q K^T into one
-// of two TMEM S slots, O += P V with P read from TMEM); warpgroup 1 + t the softmax of query
-// tile t, one thread per row, P written back over the S columns. The jobs of an item are
-// issued as S(0), S(1), then P V(u), S(u + 2) for u = 0, 1, ...; TMEM: S slot 0 at column 0,
-// S slot 1 at 128, O of tile t at 256 + t D.
-template <int D_, int NQ_, int STAGES_, bool PAGED_, int EMU_ = 0, bool FP8_ = false>
-struct Cfg {
-  static constexpr int D = D_, NQ = NQ_, STAGES = STAGES_;
-  static constexpr int EMU = EMU_;               // of every 8 column pairs, EMU use exp2_poly
-  static constexpr bool PAGED = PAGED_;
-  static constexpr bool FP8 = FP8_;
-  static constexpr int BOX_COLS = FP8 ? 128 : 64;  // elements per 128-byte box row
-  static constexpr int CH = D < 128 ? D : 128;   // columns of one ring chunk
-  static constexpr int NCH = D / CH;             // ring chunks per K or V tile
-  static constexpr int NBOX = CH / BOX_COLS;     // 128-byte boxes per chunk
-  static constexpr int QBOX = D / BOX_COLS;      // 128-byte boxes per Q tile
-  static constexpr int BOX_BYTES = 128 * 128;    // 128 rows x 128 bytes
-  static constexpr int Q_BYTES = QBOX * BOX_BYTES;
-  static constexpr int CHUNK_BYTES = NBOX * BOX_BYTES;
-  static constexpr int OFF_Q = 0;
-  static constexpr int OFF_RING = NQ * Q_BYTES;
-  static constexpr int OFF_BAR = OFF_RING + STAGES * CHUNK_BYTES;
-  // mbarrier indices
-  static constexpr int B_QFULL = 0, B_QEMPTY = 1, B_KVFULL = 2, B_KVEMPTY = B_KVFULL + STAGES,
-                       B_SFULL = B_KVEMPTY + STAGES, B_PFULL = B_SFULL + 2, B_PVDONE = B_PFULL + 2,
-                       B_OEMPTY = B_PVDONE + NQ, B_DRAIN = B_OEMPTY + NQ, NBAR = B_DRAIN + 1;
-  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;  // [0] TMEM base, [1] abort flag
-  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + slack to align the base to 1 KiB
-  static constexpr int THREADS = 128 * (1 + NQ);
-  // register split for NQ = 2: 128 threads at REG_LOW, 256 at REG_HIGH
-  static constexpr bool REG_SPLIT = NQ == 2;
-  static constexpr int REG_LOW = 64, REG_HIGH = 208;
-  static constexpr int REG_SPLIT_TOTAL = 128 * REG_LOW + 128 * NQ * REG_HIGH;
-  static constexpr int TM_O = 256;
-  // instruction descriptors: fp32 accumulate (bit 4); A / B types bf16 (1 at bits 7 / 10) or
-  // e4m3 (0); B major-ness bit 16; N / 8 at bit 17; M / 16 at bit 24
-  static constexpr uint32_t AB_TYPES = FP8 ? 0u : (1u << 7) | (1u << 10);
-  static constexpr uint32_t IDESC_QK =  // M=128, N=128, both K-major
-      (1u << 4) | AB_TYPES | (uint32_t(128 >> 3) << 17) | (uint32_t(128 >> 4) << 24);
-  static constexpr uint32_t IDESC_PV =  // M=128, N=CH, A (P) from TMEM; B: V MN-major (bf16), V^T K-major (e4m3)
-      (1u << 4) | AB_TYPES | (FP8 ? 0u : (1u << 16)) | (uint32_t(CH >> 3) << 17) | (uint32_t(128 >> 4) << 24);
-  static_assert(!FP8 || (D == 128 && !PAGED && NCH == 1), "e4m3 forward: head_dim 128, contiguous K/V");
-  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-  static_assert(2 * 128 + NQ * D <= 512, "TMEM budget");
 };
 
 #include "device_common.cuh"
@@ -303,280 +253,7 @@ enum : int32_t {
   kWaitQEmpty = 0x100, kWaitKvEmpty, kWaitQFull, kWaitKvFull, kWaitPFull, kWaitOEmpty, kWaitSFull, kWaitPvDone
 };
 
-template <class C>
-__global__ void __launch_bounds__(C::THREADS, 1) masked_attn_fwd_e4m3_kernel(const __grid_constant__ Params p) {
-  extern __shared__ uint8_t smem_raw[];
-  const uint32_t raw = smem_u32(smem_raw);
-  const uint32_t sbase = (raw + 1023u) & ~1023u;
-  uint32_t* misc = reinterpret_cast<uint32_t*>(smem_raw + (sbase - raw) + C::OFF_MISC);
-  const uint32_t bar0 = sbase + C::OFF_BAR;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const Guard guard{smem_u32(misc + 1), 0u, p.status, p.timeout_ns};
-#define BAR(i) (bar0 + 8u * uint32_t(i))
-
-  if (tid == 0) {
-    mbar_init(BAR(C::B_QFULL), 1);
-    mbar_init(BAR(C::B_QEMPTY), 1);
-    for (int s = 0; s < C::STAGES; ++s) {
-      mbar_init(BAR(C::B_KVFULL + s), 1);
-      mbar_init(BAR(C::B_KVEMPTY + s), 1);
-    }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(BAR(C::B_SFULL + s), 1);
-      mbar_init(BAR(C::B_PFULL + s), 128);
-    }
-    for (int t = 0; t < C::NQ; ++t) {
-      mbar_init(BAR(C::B_PVDONE + t), 1);
-      mbar_init(BAR(C::B_OEMPTY + t), 128);
-    }
-    mbar_init(BAR(C::B_DRAIN), 1);
-    misc[1] = 0u;
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    prefetch_tmap(&p.tm_q);
-    prefetch_tmap(&p.tm_k);
-    prefetch_tmap(&p.tm_v);
-  }
-  if (warp == 1) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(smem_u32(misc))
-                 : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = misc[0];
-  const int i_begin = p.cta_off[blockIdx.x], i_end = p.cta_off[blockIdx.x + 1];
-
-  // Registers move from the producer / MMA warpgroup to the softmax warpgroups (NQ = 2);
-  // the host launches only when the block's launch registers cover the split.
-  if (warp < 4) {
-  if constexpr (C::REG_SPLIT) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::REG_LOW));
-  if (warp == 0) {
-    // ================================ TMA producer ================================
-    if (lane == 0) {
-      uint32_t rc = 0;            // ring chunks issued
-      int n = 0;
-      int q_last = -1;            // last item whose Q load was armed
-      for (int ii = i_begin; ii < i_end; ++ii, ++n) {
-        const WorkItem it = p.items[p.cta_items[ii]];
-        if constexpr (C::PAGED) {
-          // first page-table lines of this item and of the next one
-          prefetch_l1(p.page_table + it.k_base);
-          if (ii + 1 < i_end) prefetch_l1(p.page_table + p.items[p.cta_items[ii + 1]].k_base);
-        }
-        if (!wait_bounded(BAR(C::B_QEMPTY), (n & 1) ^ 1, guard, kWaitQEmpty)) break;
-        if (!((p.debug_flags & 1) && n == 0)) {
-          mbar_expect_tx(BAR(C::B_QFULL), C::NQ * C::Q_BYTES);
-          q_last = n;
-          for (int t = 0; t < C::NQ; ++t)
-            for (int hh = 0; hh < p.hp; ++hh)
-              for (int c = 0; c < C::QBOX; ++c)
-                tma_load_3d(sbase + C::OFF_Q + t * C::Q_BYTES + c * C::BOX_BYTES + hh * p.R * 128, &p.tm_q,
-                            c * C::BOX_COLS, it.head[t] + hh, it.tok[t], BAR(C::B_QFULL));
-        }
-        const int T = C::NQ * it.job_count;
-        auto load_tile = [&](bool is_v, int j) -> bool {
-          const int kt = p.jobs[it.job_start + j].k_tile;
-          const CUtensorMap* tm = is_v ? &p.tm_v : &p.tm_k;
-          for (int h = 0; h < C::NCH; ++h, ++rc) {
-            const uint32_t slot = rc % C::STAGES;
-            if (!wait_bounded(BAR(C::B_KVEMPTY + slot), ((rc / C::STAGES) & 1) ^ 1, guard, kWaitKvEmpty))
-              return false;
-            mbar_expect_tx(BAR(C::B_KVFULL + slot), C::CHUNK_BYTES);
-            const uint32_t dst = sbase + C::OFF_RING + slot * C::CHUNK_BYTES;
-            if constexpr (C::FP8) {
-              // K: 128 keys x 128 bytes; V^T ([Hkv][d][keys]): d = 128 rows x 128 keys
-              if (is_v) tma_load_3d(dst, tm, it.vt_base + kt * 128, 0, it.kv_head, BAR(C::B_KVFULL + slot));
-              else tma_load_3d(dst, tm, 0, it.kv_head, it.k_base + kt * 128, BAR(C::B_KVFULL + slot));
-            } else if constexpr (!C::PAGED) {
-              for (int c = 0; c < C::NBOX; ++c)
-                tma_load_3d(dst + c * C::BOX_BYTES, tm, h * C::CH + c * C::BOX_COLS, it.kv_head, it.k_base + kt * 128,
-                            BAR(C::B_KVFULL + slot));
-            } else {
-              const int ps = p.page_size, ppt = 128 / ps;
-              // the page ids of the key tile two ahead go to L1 now; this tile's ids were
-              // prefetched the same way, so the loads below hit L1
-              if (!is_v && h == 0) {
-                const int ahead = (kt + 2) * ppt;
-                if (ahead < it.npages) prefetch_l1(p.page_table + it.k_base + ahead);
-              }
-              // all page ids of the tile are requested before the first is used
-              int32_t page[8];
-#pragma unroll
-              for (int pg = 0; pg < 8; ++pg) {
-                const int idx = kt * ppt + pg;
-                page[pg] = (pg < ppt && idx < it.npages) ? __ldg(p.page_table + it.k_base + idx) : -1;
-              }
-#pragma unroll
-              for (int pg = 0; pg < 8; ++pg) {
-                if (pg >= ppt) break;
-                int32_t row = p.num_pages * ps;  // fully out of bounds: the box reads zeros
-                if (page[pg] >= 0 && page[pg] < p.num_pages) row = page[pg] * ps;
-                for (int c = 0; c < C::NBOX; ++c)
-                  tma_load_3d(dst + c * C::BOX_BYTES + pg * ps * 128, tm, h * C::CH + c * C::BOX_COLS, it.kv_head, row,
-                              BAR(C::B_KVFULL + slot));
-              }
-            }
-          }
-          return true;
-        };
-        // loads in the order the MMA issuer consumes them
-        bool ok = load_tile(false, 0);
-        if (ok && T > 1 && C::NQ == 1) ok = load_tile(false, 1);
-        for (int u = 0; ok && u < T; ++u) {
-          if (u % C::NQ == 0) ok = load_tile(true, u / C::NQ);
-          const int t = u + 2;
-          if (ok && t < T && t % C::NQ == 0) ok = load_tile(false, t / C::NQ);
-        }
-        if (!ok) break;
-      }
-      // let every copy this thread issued land before the CTA may exit
-      for (uint32_t r = rc > uint32_t(C::STAGES) ? rc - C::STAGES : 0u; r < rc; ++r)
-        wait_drain(BAR(C::B_KVFULL + r % C::STAGES), (r / C::STAGES) & 1, p.timeout_ns);
-      if (q_last >= 0) wait_drain(BAR(C::B_QFULL), q_last & 1, p.timeout_ns);
-    }
-    __syncwarp();
-  } else if (warp == 1) {
-    // ================================ MMA issuer ================================
-    if (lane == 0) {
-      uint32_t rc = 0, sj = 0;
-      int n = 0;
-      for (int ii = i_begin; ii < i_end; ++ii, ++n) {
-        const WorkItem it = p.items[p.cta_items[ii]];
-        if (!wait_bounded(BAR(C::B_QFULL), n & 1, guard, kWaitQFull)) break;
-        tc_fence_after();
-        const int T = C::NQ * it.job_count;
-        uint32_t rk = 0, rv = 0;
-        auto qk = [&](int t) -> bool {
-          const int q = t % C::NQ;
-          if (q == 0) {
-            rk = rc;
-            for (int h = 0; h < C::NCH; ++h, ++rc)
-              if (!wait_bounded(BAR(C::B_KVFULL + rc % C::STAGES), (rc / C::STAGES) & 1, guard, kWaitKvFull))
-                return false;
-            tc_fence_after();
-          }
-          const uint32_t slot = (sj + t) & 1;
-          const uint32_t d_s = tmem + 128 * slot;
-          const uint32_t qlo = desc_lo(sbase + C::OFF_Q + q * C::Q_BYTES, 16);
-          static_assert(C::NCH == 1, "single-CTA kernel: one ring chunk per K or V tile");
-#pragma unroll
-          for (int h = 0; h < C::NCH; ++h) {
-            const uint32_t klo = desc_lo(sbase + C::OFF_RING + ((rk + h) % C::STAGES) * C::CHUNK_BYTES, 16);
-            if constexpr (C::FP8) mma8_ss_x4_k128(d_s, desc_of(qlo), desc_of(klo), C::IDESC_QK, 0u);
-            else if constexpr (C::D == 128) mma_ss_x8_k128(d_s, desc_of(qlo), desc_of(klo), C::IDESC_QK, 0u);
-            else mma_ss_x4_k64(d_s, desc_of(qlo), desc_of(klo), C::IDESC_QK, 0u);
-            // the chunk is free once these MMAs complete (commit tracks all earlier MMAs)
-            if (q == C::NQ - 1) mma_commit(BAR(C::B_KVEMPTY + (rk + h) % C::STAGES));
-          }
-          mma_commit(BAR(C::B_SFULL + slot));
-          if (t == T - 1) mma_commit(BAR(C::B_QEMPTY));
-          return true;
-        };
-        auto pv = [&](int u) -> bool {
-          const int q = u % C::NQ;
-          const uint32_t g = sj + u, slot = g & 1;
-          if (!wait_bounded(BAR(C::B_PFULL + slot), (g >> 1) & 1, guard, kWaitPFull)) return false;
-          if (u < C::NQ && !wait_bounded(BAR(C::B_OEMPTY + q), (n & 1) ^ 1, guard, kWaitOEmpty)) return false;
-          if (q == 0) {
-            rv = rc;
-            for (int h = 0; h < C::NCH; ++h, ++rc)
-              if (!wait_bounded(BAR(C::B_KVFULL + rc % C::STAGES), (rc / C::STAGES) & 1, guard, kWaitKvFull))
-                return false;
-          }
-          tc_fence_after();
-          const uint32_t first = u < C::NQ ? 1u : 0u;
-#pragma unroll
-          for (int h = 0; h < C::NCH; ++h) {
-            const uint32_t vbase = sbase + C::OFF_RING + ((rv + h) % C::STAGES) * C::CHUNK_BYTES;
-            const uint32_t d_o = tmem + C::TM_O + q * C::D + h * 128, a_p = tmem + 128 * slot;
-            if constexpr (C::FP8) mma8_ts_x4_k128(d_o, a_p, desc_of(desc_lo(vbase, 16)), C::IDESC_PV, first ^ 1u);
-            else mma_ts_x8(d_o, a_p, desc_of(desc_lo(vbase, C::BOX_BYTES)), C::IDESC_PV, first ^ 1u);
-            if (q == C::NQ - 1) mma_commit(BAR(C::B_KVEMPTY + (rv + h) % C::STAGES));
-          }
-          mma_commit(BAR(C::B_PVDONE + q));
-          return true;
-        };
-        bool ok = qk(0);
-        if (ok && T > 1) ok = qk(1);
-        for (int u = 0; ok && u < T; ++u) {
-          ok = pv(u);
-          if (ok && u + 2 < T) ok = qk(u + 2);
-        }
-        if (!ok) break;
-        sj += T;
-      }
-      // all MMAs this thread issued complete before TMEM may be freed
-      mma_commit(BAR(C::B_DRAIN));
-      wait_drain(BAR(C::B_DRAIN), 0, p.timeout_ns);
-    }
-    __syncwarp();
-  }
-  } else {
-    if constexpr (C::REG_SPLIT) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(C::REG_HIGH));
-    // ================================ softmax warpgroup ================================
-    const int q = warp / 4 - 1;                       // query tile of this warpgroup
-    const int r = tid - 128 * (1 + q);                // row of the tile = TMEM lane
-    const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
-    const uint32_t t_o = tmem + lane_base + C::TM_O + q * C::D;
-    const float sl2 = p.scale_log2;
-    uint32_t sj = 0, pvc = 0;
-    bool ok = true;
-    for (int ii = i_begin; ok && ii < i_end; ++ii) {
-      const WorkItem it = p.items[p.cta_items[ii]];
-      const int T = C::NQ * it.job_count;
-      RowState st{-INFINITY, 0.f};
-      for (int t = q; t < T; t += C::NQ) {
-        const uint32_t g = sj + t, slot = g & 1;
-        const int mi = p.jobs[it.job_start + t / C::NQ].mask[q];
-        uint4 bits = make_uint4(0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu);
-        if (mi >= 0) bits = __ldg(p.mask_tiles + int64_t(mi) * 128 + r);
-        else if (mi == kMaskNone) bits = make_uint4(0u, 0u, 0u, 0u);
-        if (!__all_sync(0xffffffffu, wait_bounded(BAR(C::B_SFULL + slot), (g >> 1) & 1, guard, kWaitSFull))) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        bool need;
-        const float alpha = softmax_tile<C::EMU, C::FP8>(tmem + lane_base + 128 * slot, mi, bits, sl2, st, need);
-        if (t >= C::NQ) {
-          // the previous P V of this tile must be done before O is touched or P is published
-          if (!__all_sync(0xffffffffu, wait_bounded(BAR(C::B_PVDONE + q), pvc & 1, guard, kWaitPvDone))) {
-            ok = false;
-            break;
-          }
-          ++pvc;
-          tc_fence_after();
-          if (__any_sync(0xffffffffu, need)) rescale_o<C::D>(t_o, alpha);
-        }
-        tc_fence_before();
-        mbar_arrive(BAR(C::B_PFULL + slot));
-      }
-      if (!ok) break;
-      // ---- epilogue ----
-      if (!__all_sync(0xffffffffu, wait_bounded(BAR(C::B_PVDONE + q), pvc & 1, guard, kWaitPvDone))) break;
-      ++pvc;
-      tc_fence_after();
-      const int lr = r % p.R, hh = r / p.R;
-      if (it.part < 0)
-        store_row<C::D>(t_o, st, lr < it.rows[q], int64_t(it.tok[q] + lr) * p.hq + it.head[q] + hh, p.out, p.lse,
-                        p.v_scale);
-      else
-        store_partial<C::D>(t_o, st, lr < it.rows[q], int64_t(it.part + q) * kSlotRows + r, p.part_o, p.part_lse,
-                            p.v_scale);
-      tc_fence_before();
-      mbar_arrive(BAR(C::B_OEMPTY + q));
-      sj += T;
-    }
-  }
-#undef BAR
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  if (warp == 1) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem) : "memory");
-}
-
-// ================================ shared-S kernel (head_dim 64 / 128, bf16) ================================
+// ================================ shared-S kernel (head_dim 64 / 128 bf16, 128 e4m3) ================================
 // One persistent CTA per SM, two 128-row query tiles per work item. The two query tiles take
 // turns in ONE S accumulator (TMEM columns 0-127): a softmax warpgroup frees it as soon as it
 // has read its scores into registers, so the next Q K^T (of the other tile) runs while it
@@ -593,15 +270,20 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_fwd_e4m3_kernel(con
 //                row's mask bits (partial tiles), updates the online max / sum, writes P into
 //                its slot once the previous P V of the tile is done, rescales O when the
 //                running maximum grows by more than 2^8, and finally writes out / lse.
-template <int D_, bool PAGED_, int EMU_ = 0>
+// FP8_: e4m3 Q and K (one 128-byte box per 128-row tile), V transposed per head
+// ([Hkv][d][keys]: a chunk is d = 128 rows x 128 keys), .kind::f8f6f4 MMAs of K = 32, and P
+// quantised to e4m3 (four per TMEM column: a 32-column P slot); head_dim 128, contiguous K/V.
+template <int D_, bool PAGED_, int EMU_ = 0, bool FP8_ = false>
 struct SCfg {
   static constexpr int D = D_, EMU = EMU_;
   static constexpr bool PAGED = PAGED_;
-  static constexpr int NBOX = D / 64;                 // 128-byte boxes per Q tile and per K / V chunk
+  static constexpr bool FP8 = FP8_;
+  static constexpr int NBOX = FP8 ? 1 : D / 64;       // 128-byte boxes per Q tile and per K / V chunk
   static constexpr int BOX_BYTES = 128 * 128;         // 128 rows x 128 bytes
   static constexpr int Q_BYTES = NBOX * BOX_BYTES;
   static constexpr int CHUNK_BYTES = NBOX * BOX_BYTES;
-  static constexpr int STAGES = D == 128 ? 5 : 10;
+  static constexpr int STAGES = FP8 ? 12 : D == 128 ? 5 : 10;
+  static constexpr int P_COLS = FP8 ? 32 : 64;        // TMEM columns of a P slot
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_RING = 2 * Q_BYTES;
   static constexpr int OFF_BAR = OFF_RING + STAGES * CHUNK_BYTES;
@@ -614,12 +296,13 @@ struct SCfg {
   static constexpr int REG_LOW = 64, REG_HIGH = 208;
   static constexpr int REG_SPLIT_TOTAL = 128 * REG_LOW + 256 * REG_HIGH;
   static constexpr int TM_S = 0, TM_P = 128, TM_O = 256;
-  static constexpr uint32_t AB_TYPES = (1u << 7) | (1u << 10);   // bf16 A and B
+  static constexpr uint32_t AB_TYPES = FP8 ? 0u : (1u << 7) | (1u << 10);   // bf16 (1) or e4m3 (0)
   static constexpr uint32_t IDESC_QK =  // M=128, N=128, both K-major, fp32 accumulate
       (1u << 4) | AB_TYPES | (uint32_t(128 >> 3) << 17) | (uint32_t(128 >> 4) << 24);
-  static constexpr uint32_t IDESC_PV =  // M=128, N=D, A (P) from TMEM, B (V) MN-major
-      (1u << 4) | AB_TYPES | (1u << 16) | (uint32_t(D >> 3) << 17) | (uint32_t(128 >> 4) << 24);
+  static constexpr uint32_t IDESC_PV =  // M=128, N=D, A (P) from TMEM, B: V MN-major (bf16), V^T K-major (e4m3)
+      (1u << 4) | AB_TYPES | (FP8 ? 0u : (1u << 16)) | (uint32_t(D >> 3) << 17) | (uint32_t(128 >> 4) << 24);
   static_assert(D == 64 || D == 128, "shared-S kernel: head_dim 64 or 128");
+  static_assert(!FP8 || (D == 128 && !PAGED), "e4m3 shared-S kernel: head_dim 128, contiguous K/V");
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
   static_assert(TM_O + 2 * D <= 512, "TMEM budget");
 };
@@ -632,7 +315,8 @@ __device__ __forceinline__ int v_pos(int j, int J) { return j == J - 1 ? 2 * J -
 // Softmax step of a shared-S tile: the row's 128 scores at t_s (fp32) into registers, then
 // `freed()` (the S accumulator may be overwritten), mask / max / exponentials / row sum, and
 // P (bf16 pairs) into pk[64]. Returns the factor by which O and l must be multiplied.
-template <int EMU, class Freed>
+// FP8: P as e4m3, four per word (pk[0 .. 31]) instead of bf16 pairs (pk[0 .. 63]).
+template <int EMU, bool FP8, class Freed>
 __device__ __forceinline__ float softmax_regs(uint32_t t_s, int mi, const uint4& bits, float sl2, RowState& st,
                                               bool& need, uint32_t (&pk)[64], Freed freed) {
   float s[128];
@@ -672,6 +356,7 @@ __device__ __forceinline__ float softmax_regs(uint32_t t_s, int mi, const uint4&
   const float mref = st.m_run == -INFINITY ? 0.f : st.m_run;
   const uint64_t sl2x2 = pk2(sl2, sl2), nm2 = pk2(-mref, -mref);
   uint64_t lsum2[4] = {pk2(0.f, 0.f), pk2(0.f, 0.f), pk2(0.f, 0.f), pk2(0.f, 0.f)};
+  float pprev0 = 0.f, pprev1 = 0.f;
 #pragma unroll
   for (int e = 0; e < 64; ++e) {
     float x0, x1;
@@ -682,7 +367,13 @@ __device__ __forceinline__ float softmax_regs(uint32_t t_s, int mi, const uint4&
     lsum2[e & 3] = fadd2(lsum2[e & 3], p01);
     float p0, p1;
     unpk2(p01, p0, p1);
-    pk[e] = pack_bf16(p0, p1);
+    if constexpr (FP8) {
+      if (e & 1) pk[e >> 1] = pack_e4m3x4(pprev0, pprev1, p0, p1);
+      pprev0 = p0;
+      pprev1 = p1;
+    } else {
+      pk[e] = pack_bf16(p0, p1);
+    }
   }
   float a, b;
   unpk2(fadd2(fadd2(lsum2[0], lsum2[1]), fadd2(lsum2[2], lsum2[3])), a, b);
@@ -753,8 +444,8 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_fwd_kernel(const __
           for (int t = 0; t < 2; ++t)
             for (int hh = 0; hh < p.hp; ++hh)
               for (int c = 0; c < C::NBOX; ++c)
-                tma_load_3d(sbase + C::OFF_Q + t * C::Q_BYTES + c * C::BOX_BYTES + hh * p.R * 128, &p.tm_q, c * 64,
-                            it.head[t] + hh, it.tok[t], BAR(C::B_QFULL));
+                tma_load_3d(sbase + C::OFF_Q + t * C::Q_BYTES + c * C::BOX_BYTES + hh * p.R * 128, &p.tm_q,
+                            c * (C::FP8 ? 128 : 64), it.head[t] + hh, it.tok[t], BAR(C::B_QFULL));
         }
         auto load_tile = [&](bool is_v, int j) -> bool {
           const int kt = p.jobs[it.job_start + j].k_tile;
@@ -763,7 +454,11 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_fwd_kernel(const __
           if (!wait_bounded(BAR(C::B_KVEMPTY + slot), ((rc / C::STAGES) & 1) ^ 1, guard, kWaitKvEmpty)) return false;
           mbar_expect_tx(BAR(C::B_KVFULL + slot), C::CHUNK_BYTES);
           const uint32_t dst = sbase + C::OFF_RING + slot * C::CHUNK_BYTES;
-          if constexpr (!C::PAGED) {
+          if constexpr (C::FP8) {
+            // K: 128 keys x 128 bytes; V^T ([Hkv][d][keys]): d = 128 rows x 128 keys
+            if (is_v) tma_load_3d(dst, tm, it.vt_base + kt * 128, 0, it.kv_head, BAR(C::B_KVFULL + slot));
+            else tma_load_3d(dst, tm, 0, it.kv_head, it.k_base + kt * 128, BAR(C::B_KVFULL + slot));
+          } else if constexpr (!C::PAGED) {
             for (int c = 0; c < C::NBOX; ++c)
               tma_load_3d(dst + c * C::BOX_BYTES, tm, c * 64, it.kv_head, it.k_base + kt * 128, BAR(C::B_KVFULL + slot));
           } else {
@@ -834,7 +529,8 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_fwd_kernel(const __
             }
             tc_fence_after();
             const uint32_t qlo = desc_lo(sbase + C::OFF_Q + t * C::Q_BYTES, 16);
-            if constexpr (C::D == 128) mma_ss_x8_k128(tmem + C::TM_S, desc_of(qlo), desc_of(klo), C::IDESC_QK, 0u);
+            if constexpr (C::FP8) mma8_ss_x4_k128(tmem + C::TM_S, desc_of(qlo), desc_of(klo), C::IDESC_QK, 0u);
+            else if constexpr (C::D == 128) mma_ss_x8_k128(tmem + C::TM_S, desc_of(qlo), desc_of(klo), C::IDESC_QK, 0u);
             else mma_ss_x4_k64(tmem + C::TM_S, desc_of(qlo), desc_of(klo), C::IDESC_QK, 0u);
             mma_commit(BAR(C::B_SFULL + t));
             ++produced;
@@ -884,8 +580,12 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_fwd_kernel(const __
               break;
             }
             tc_fence_after();
-            mma_ts_x8(tmem + C::TM_O + t * C::D, tmem + C::TM_P + 64 * t, desc_of(desc_lo(vbase, C::BOX_BYTES)),
-                      C::IDESC_PV, j == 0 ? 0u : 1u);
+            if constexpr (C::FP8)
+              mma8_ts_x4_k128(tmem + C::TM_O + t * C::D, tmem + C::TM_P + C::P_COLS * t, desc_of(desc_lo(vbase, 16)),
+                              C::IDESC_PV, j == 0 ? 0u : 1u);
+            else
+              mma_ts_x8(tmem + C::TM_O + t * C::D, tmem + C::TM_P + C::P_COLS * t,
+                        desc_of(desc_lo(vbase, C::BOX_BYTES)), C::IDESC_PV, j == 0 ? 0u : 1u);
             mma_commit(BAR(C::B_PVDONE + t));
           }
           if (!ok) break;
@@ -906,7 +606,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_fwd_kernel(const __
     const int r = tid - 128 * (1 + q);                // row of the tile = TMEM lane
     const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
     const uint32_t t_o = tmem + lane_base + C::TM_O + q * C::D;
-    const uint32_t t_p = tmem + lane_base + C::TM_P + 64 * q;
+    const uint32_t t_p = tmem + lane_base + C::TM_P + C::P_COLS * q;
     const float sl2 = p.scale_log2;
     uint32_t sc = 0, pc = 0;   // S phases consumed, P published
     bool ok = true;
@@ -931,7 +631,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_fwd_kernel(const __
         tc_fence_after();
         bool need;
         uint32_t pk[64];
-        const float alpha = softmax_regs<C::EMU>(tmem + lane_base + C::TM_S, mi, bits, sl2, st, need, pk, [&] {
+        const float alpha = softmax_regs<C::EMU, C::FP8>(tmem + lane_base + C::TM_S, mi, bits, sl2, st, need, pk, [&] {
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(BAR(C::B_SFREE + q));
@@ -943,10 +643,14 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_fwd_kernel(const __
         }
         tc_fence_after();
         if (j > 0 && __any_sync(0xffffffffu, need)) rescale_o<C::D>(t_o, alpha);
-        tmem_st32x16(t_p + 0, pk + 0);
-        tmem_st32x16(t_p + 16, pk + 16);
-        tmem_st32x16(t_p + 32, pk + 32);
-        tmem_st32x16(t_p + 48, pk + 48);
+        if constexpr (C::FP8) {
+          tmem_st32x32(t_p, pk);
+        } else {
+          tmem_st32x16(t_p + 0, pk + 0);
+          tmem_st32x16(t_p + 16, pk + 16);
+          tmem_st32x16(t_p + 32, pk + 32);
+          tmem_st32x16(t_p + 48, pk + 48);
+        }
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
@@ -959,9 +663,11 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_fwd_kernel(const __
       tc_fence_after();
       const int lr = r % p.R, hh = r / p.R;
       if (it.part < 0)
-        store_row<C::D>(t_o, st, lr < it.rows[q], int64_t(it.tok[q] + lr) * p.hq + it.head[q] + hh, p.out, p.lse);
+        store_row<C::D>(t_o, st, lr < it.rows[q], int64_t(it.tok[q] + lr) * p.hq + it.head[q] + hh, p.out, p.lse,
+                        p.v_scale);
       else
-        store_partial<C::D>(t_o, st, lr < it.rows[q], int64_t(it.part + q) * kSlotRows + r, p.part_o, p.part_lse);
+        store_partial<C::D>(t_o, st, lr < it.rows[q], int64_t(it.part + q) * kSlotRows + r, p.part_o, p.part_lse,
+                            p.v_scale);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(BAR(C::B_OEMPTY + q));
@@ -1351,24 +1057,6 @@ __global__ void fill_empty_kernel(float* lse, int64_t n) {
 
 
 template <class C>
-attn_status_t launch(const attn_plan_t* plan, Params& p, cudaStream_t stream) {
-  const cudaError_t attr = once_per_device([] {
-    cudaError_t e = cudaFuncSetAttribute(masked_attn_fwd_e4m3_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         C::SMEM_BYTES);
-    if (e == cudaSuccess && C::REG_SPLIT) {
-      // setmaxnreg.inc draws on the registers the block was launched with: the split must fit
-      cudaFuncAttributes fa{};
-      e = cudaFuncGetAttributes(&fa, masked_attn_fwd_e4m3_kernel<C>);
-      if (e == cudaSuccess && fa.numRegs * C::THREADS < C::REG_SPLIT_TOTAL) e = cudaErrorInvalidConfiguration;
-    }
-    return e;
-  });
-  if (attr != cudaSuccess) return ATTN_ERR_CUDA;
-  masked_attn_fwd_e4m3_kernel<C><<<plan->ctas, C::THREADS, C::SMEM_BYTES, stream>>>(p);
-  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
-}
-
-template <class C>
 attn_status_t launch_sharedS(const attn_plan_t* plan, Params& p, cudaStream_t stream) {
   const cudaError_t attr = once_per_device([] {
     cudaError_t e = cudaFuncSetAttribute(masked_attn_fwd_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1502,7 +1190,7 @@ attn_status_t mfa_launch_forward_fp8(const attn_plan_t* plan, const void* q, con
   p.scale_log2 = plan->scale * q_scale * k_scale * 1.4426950408889634f;
   p.v_scale = v_scale;
   const attn_status_t st = pair ? launch_pair<PairCfg<256, 10, false, 0, true>>(plan, p, stream)
-                                : launch<Cfg<128, 2, 10, false, 0, true>>(plan, p, stream);
+                                : launch_sharedS<SCfg<128, false, 0, true>>(plan, p, stream);
   return st != ATTN_OK ? st : merge_if_split(plan, out, lse, stream);
 }
 
