@@ -7,22 +7,33 @@
 //   bwd_delta_kernel    delta_i for every (row, query head): one warp per row.
 //   dQ kernel           one persistent CTA per SM over dQ items (a 128-row query tile of one
 //                       query head and its non-empty key tiles): S = Q K^T and dP = dO V^T
-//                       into TMEM, the elementwise warpgroup turns them into dS (bf16, written
+//                       into TMEM, the elementwise warpgroups turn them into dS (bf16, written
 //                       over S), then dQ += dS K accumulates in TMEM.
 //   dK/dV kernel        one persistent CTA per SM over dK/dV items (a 128-key tile of one
 //                       key/value head and every (query head, query tile) that sees it):
-//                       S^T = K Q^T and dP^T = V dO^T into TMEM, the warpgroup writes P^T and
-//                       dS^T (bf16) over them, then dV += P^T dO and dK += dS^T Q accumulate in
+//                       S^T = K Q^T and dP^T = V dO^T into TMEM, the warpgroups write P^T
+//                       and dS^T (bf16) over them, then dV += P^T dO and dK += dS^T Q accumulate in
 //                       TMEM.
-// Both recompute P from the forward's lse instead of storing it. Warp roles as in the
-// forward: warp 0 TMA producer, warp 1 MMA issuer (one thread), warps 4-7 the elementwise
-// warpgroup, one TMEM lane (= one tile row) per thread. Tiles are 128 rows of one head,
-// 64-column boxes with the 128-byte swizzle; a ring of STAGES tile slots streams the
-// per-job operands (dQ: K and V tiles; dK/dV: Q and dO tiles). Each job runs as two half
-// jobs of 64 columns (keys for dQ, query rows for dK/dV) with two S / dP slots in TMEM, so
-// the S / dP MMAs of the next half job overlap the elementwise work on the current one.
-// TMEM: S slots at columns 0 and 64, dP slots at 128 and 192, the accumulators from 256
-// (dQ: D columns; dK/dV: dV then dK). Every mbarrier wait is bounded as in the forward.
+// Both recompute P from the forward's lse instead of storing it. Warp roles: warp 0 TMA
+// producer; warp 1 issues the S / dP MMAs (one thread), warp 2 the accumulating MMAs (dQ, or
+// dV and dK; one thread); warps 4-11 two elementwise warpgroups, one TMEM lane (= one tile
+// row) per thread, the first warpgroup on columns 0..63 of every job and the second on
+// columns 64..127. Tiles are 128 rows of one head, 64-column boxes with the 128-byte swizzle;
+// a ring of STAGES tile slots streams the per-job operands (dQ: K and V tiles; dK/dV: Q and
+// dO tiles). A job is one 128 x 128 block, its S and dP MMAs M = 128, N = 128: the tensor
+// core reads 8 KiB of shared memory per 128 x 128 x 16 step, the rate its 64-cycle step can
+// take (narrower N re-reads A for every N block). The hand-offs are per operand, so each MMA
+// starts as soon as the TMEM it reads or overwrites allows:
+//   dQ:    S slots 0 / 1 (TMEM columns 0 and 128), one dP slot (256), dQ (384). S of job g+1
+//          runs while the warpgroups work on job g; dP of job g+1 once they have read dP of
+//          job g (they read it first); dQ += dS K once they have written dS over S.
+//   dK/dV: one S^T slot (0), one dP^T slot (128), dV (256) and dK (256 + D). The warpgroups
+//          write P^T over S^T (dV += P^T dO starts), then dS^T over dP^T (dK += dS^T Q
+//          starts); S^T of job g+1 once dV of job g has completed, dP^T once dK has.
+// bf16 P / dS pairs of columns 0..63 go to TMEM columns 0..31 of their slot and those of
+// columns 64..127 to 64..95, each within the columns its warpgroup has already read. Every
+// mbarrier wait is bounded as in the forward.
+
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_bf16.h>
@@ -59,58 +70,94 @@ struct BwdParams {
   int64_t timeout_ns;
 };
 
-template <int D_>
+// Shared-memory layout, TMEM columns and mbarriers of the two kernels. A job is one
+// 128 x 128 tile pair, S and dP (dQ) or S^T and dP^T (dK/dV) computed as M = 128, N = 128
+// MMAs; the accumulators take D (dQ) or 2 D (dV, dK) TMEM columns.
+template <int D_, bool DKV_>
 struct BwdCfg {
   static constexpr int D = D_;
+  static constexpr bool DKV = DKV_;
   static constexpr int NBOX = D / 64;                  // 64-column boxes per tile
   static constexpr int BOX_BYTES = 128 * 128;          // 128 rows x 128 bytes
   static constexpr int TILE_BYTES = NBOX * BOX_BYTES;  // one 128-row tile of one head
   static constexpr int STAGES = D == 128 ? 4 : 8;      // ring tile slots (two per job)
+  // TMEM: dQ -- S slots at 0 and 128, dP at 256, dQ at 384; dK/dV -- S^T at 0, dP^T at
+  // 128, dV at 256, dK at 256 + D
+  static constexpr int NS = DKV ? 1 : 2;               // S slots
+  static constexpr int TM_S = 0, TM_P = 128 * NS, TM_ACC = TM_P + 128;
   static constexpr int OFF_A = 0, OFF_B = TILE_BYTES, OFF_RING = 2 * TILE_BYTES;
   static constexpr int OFF_ROWV = OFF_RING + STAGES * TILE_BYTES;  // dK/dV: per warp 128 lse2 + 128 delta
-  static constexpr int OFF_BAR = OFF_ROWV + 4 * 2 * 128 * 4;
+  static constexpr int OFF_BAR = OFF_ROWV + (DKV ? 8 * 2 * 128 * 4 : 0);
+  // dQ:   SFULL[s] S of the slot computed, DPFULL dP computed, DPREAD dP read by the
+  //       warpgroups, DSREADY[s] dS written, SFREE[s] dQ MMA of the slot completed.
+  // dK/dV: SFULL S^T computed, DPFULL dP^T computed, PREADY P^T written, DSREADY dS^T
+  //       written, SFREE the dV MMA (reader of P^T) completed, DPFREE the dK MMA completed.
   static constexpr int B_AFULL = 0, B_AEMPTY = 1, B_RFULL = 2, B_REMPTY = B_RFULL + STAGES,
-                       B_SFULL = B_REMPTY + STAGES, B_PFULL = B_SFULL + 2, B_ACCFULL = B_PFULL + 2,
-                       B_ACCEMPTY = B_ACCFULL + 1, B_DRAIN = B_ACCEMPTY + 1, NBAR = B_DRAIN + 1;
+                       B_SFULL = B_REMPTY + STAGES, B_DPFULL = B_SFULL + NS, B_DPREAD = B_DPFULL + 1,
+                       B_PREADY = B_DPREAD + 1, B_DSREADY = B_PREADY + 1, B_SFREE = B_DSREADY + NS,
+                       B_DPFREE = B_SFREE + NS, B_ACCFULL = B_DPFREE + 1, B_ACCEMPTY = B_ACCFULL + 1,
+                       B_DRAIN = B_ACCEMPTY + 1, B_DRAIN2 = B_DRAIN + 1, NBAR = B_DRAIN2 + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;       // [0] TMEM base, [1] abort flag
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;   // + slack to align the base to 1 KiB
-  static constexpr int THREADS = 256;
-  // TMEM: S half-job slots at 0 and 64, dP slots at 128 and 192, accumulators from 256
-  static constexpr int TM_S = 0, TM_P = 128, TM_ACC = 256;
-  static constexpr int HALF_BYTES = 64 * 128;  // 64 rows of every 64-column box (8 swizzle atoms)
-  static constexpr uint32_t IDESC_SS =  // M=128, N=64 (a half job), bf16 x bf16 -> fp32, both K-major
-      (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(64 >> 3) << 17) | (uint32_t(128 >> 4) << 24);
+  static constexpr int THREADS = 384;
+  static constexpr int EW = 256;                            // elementwise threads (two warpgroups)
+  static constexpr uint32_t IDESC_SS =  // M=128, N=128, bf16 x bf16 -> fp32, both K-major
+      (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(128 >> 3) << 17) | (uint32_t(128 >> 4) << 24);
   static constexpr uint32_t IDESC_TS =  // M=128, N=D, A from TMEM, B MN-major
       (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) | (uint32_t(D >> 3) << 17) | (uint32_t(128 >> 4) << 24);
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-  static_assert(TM_ACC + 2 * D <= 512, "TMEM budget");
+  static_assert(TM_ACC + (DKV ? 2 * D : D) <= 512, "TMEM budget");
 };
 
 enum : int32_t {
   kBwdWaitAEmpty = 0x200, kBwdWaitREmpty, kBwdWaitAFull, kBwdWaitRFull, kBwdWaitPFull, kBwdWaitAccEmpty,
-  kBwdWaitSFull, kBwdWaitAccFull
+  kBwdWaitSFull, kBwdWaitAccFull, kBwdWaitSFree, kBwdWaitDpFull, kBwdWaitDpRead, kBwdWaitDsReady, kBwdWaitDpFree
 };
 
-// C[128 x 64] (TMEM, fp32) = A[128 x D] . B[64 x D]^T: A a whole tile, B 64 rows of a tile
-// (b_smem = tile + half * HALF_BYTES); both K-major in shared memory.
+// C[128 x 128] (TMEM, fp32) = A[128 x D] . B[128 x D]^T, both whole tiles, K-major in
+// shared memory.
 template <int D>
-__device__ __forceinline__ void mma_half_ss(uint32_t d, uint32_t a_smem, uint32_t b_smem, uint32_t idesc) {
+__device__ __forceinline__ void mma_tile_ss(uint32_t d, uint32_t a_smem, uint32_t b_smem, uint32_t idesc) {
   if constexpr (D == 128) mma_ss_x8_k128(d, desc_of(desc_lo(a_smem, 16)), desc_of(desc_lo(b_smem, 16)), idesc, 0u);
   else mma_ss_x4_k64(d, desc_of(desc_lo(a_smem, 16)), desc_of(desc_lo(b_smem, 16)), idesc, 0u);
 }
 
-// C[128 x D] (+)= A[128 x 64] (bf16 in TMEM, 32 columns) . B[64 x D] (64 rows of a tile in
-// shared memory, MN-major).
-__device__ __forceinline__ void mma_half_ts(uint32_t d, uint32_t a_tmem, uint32_t b_smem, uint32_t idesc,
-                                            uint32_t acc) {
-  mma_ts_x4(d, a_tmem, desc_of(desc_lo(b_smem, 128 * 128)), idesc, acc);
+// C[128 x D] (+)= A[128 x 128] . B[128 x D]: A is bf16 in TMEM, its 128 K columns (64 TMEM
+// columns) in two runs of 32 -- columns a .. a + 31 (K 0..63, written by the first
+// elementwise warpgroup) and a + 64 .. a + 95 (K 64..127, the second) -- and B a whole tile
+// in shared memory, MN-major.
+__device__ __forceinline__ void mma_tile_ts(uint32_t d, uint32_t a, uint32_t b_smem, uint32_t idesc, uint32_t acc) {
+  const uint64_t b = desc_of(desc_lo(b_smem, 128 * 128));
+  asm volatile(
+      "{\n\t.reg .pred p, t;\n\t.reg .b32 ta, bl, bh;\n\t.reg .b64 bx;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\tsetp.eq.u32 t, 0, 0;\n\t"
+      "mov.b64 {bl, bh}, %2;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t"
+      "add.u32 ta, %1, 8;\n\tadd.u32 bl, bl, 128;\n\tmov.b64 bx, {bl, bh};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], bx, %3, t;\n\t"
+      "add.u32 ta, %1, 16;\n\tadd.u32 bl, bl, 128;\n\tmov.b64 bx, {bl, bh};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], bx, %3, t;\n\t"
+      "add.u32 ta, %1, 24;\n\tadd.u32 bl, bl, 128;\n\tmov.b64 bx, {bl, bh};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], bx, %3, t;\n\t"
+      "add.u32 ta, %1, 64;\n\tadd.u32 bl, bl, 128;\n\tmov.b64 bx, {bl, bh};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], bx, %3, t;\n\t"
+      "add.u32 ta, %1, 72;\n\tadd.u32 bl, bl, 128;\n\tmov.b64 bx, {bl, bh};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], bx, %3, t;\n\t"
+      "add.u32 ta, %1, 80;\n\tadd.u32 bl, bl, 128;\n\tmov.b64 bx, {bl, bh};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], bx, %3, t;\n\t"
+      "add.u32 ta, %1, 88;\n\tadd.u32 bl, bl, 128;\n\tmov.b64 bx, {bl, bh};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], bx, %3, t;\n\t"
+      "}" ::"r"(d),
+      "r"(a), "l"(b), "r"(idesc), "r"(acc)
+      : "memory");
 }
 
-// One 128-row x D tile of bf16 gradients from TMEM (fp32, times `mul`) to global memory.
-template <int D>
-__device__ __forceinline__ void store_grad_row(uint32_t t_acc, float mul, bool valid, __nv_bfloat16* dst) {
+// NC columns of a 128-row tile of gradients from TMEM (fp32, times `mul`) to global memory as
+// bf16 (dst: this row's first column of the run).
+template <int NC>
+__device__ __forceinline__ void store_grad_cols(uint32_t t_acc, float mul, bool valid, __nv_bfloat16* dst) {
 #pragma unroll 1
-  for (int cc = 0; cc < D / 32; ++cc) {
+  for (int cc = 0; cc < NC / 32; ++cc) {
     uint32_t o[32];
     tmem_ld32x32(t_acc + cc * 32, o);
     tmem_wait_ld();
@@ -148,6 +195,13 @@ __global__ void bwd_delta_kernel(const __nv_bfloat16* __restrict__ out, const __
   }
 }
 
+// Row r's 128 mask bits of a job: the packed partial tile, all ones (fully visible) or all
+// zeros (a filler job that sees nothing).
+__device__ __forceinline__ uint4 row_bits(const uint4* __restrict__ tiles, int mi, int r) {
+  if (mi >= 0) return __ldg(tiles + int64_t(mi) * 128 + r);
+  return mi == kMaskNone ? make_uint4(0u, 0u, 0u, 0u) : make_uint4(0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu);
+}
+
 // ================================ dQ ================================
 template <class C>
 __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd_dq_kernel(const __grid_constant__ BwdParams p) {
@@ -166,13 +220,17 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd_dq_kernel(const
       mbar_init(BAR(C::B_RFULL + s), 1);
       mbar_init(BAR(C::B_REMPTY + s), 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < C::NS; ++b) {
       mbar_init(BAR(C::B_SFULL + b), 1);
-      mbar_init(BAR(C::B_PFULL + b), 128);
+      mbar_init(BAR(C::B_DSREADY + b), C::EW);
+      mbar_init(BAR(C::B_SFREE + b), 1);
     }
+    mbar_init(BAR(C::B_DPFULL), 1);
+    mbar_init(BAR(C::B_DPREAD), C::EW);
     mbar_init(BAR(C::B_ACCFULL), 1);
-    mbar_init(BAR(C::B_ACCEMPTY), 128);
+    mbar_init(BAR(C::B_ACCEMPTY), C::EW);
     mbar_init(BAR(C::B_DRAIN), 1);
+    mbar_init(BAR(C::B_DRAIN2), 1);
     misc[1] = 0u;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     prefetch_tmap(&p.tm_a);
@@ -190,6 +248,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd_dq_kernel(const
   tc_fence_after();
   const uint32_t tmem = misc[0];
   const int i_begin = p.cta_off[blockIdx.x], i_end = p.cta_off[blockIdx.x + 1];
+  auto ring = [&](uint32_t r) { return sbase + C::OFF_RING + (r % C::STAGES) * C::TILE_BYTES; };
 
   if (warp == 0) {
     // ---- TMA producer: Q and dO once per item, then K and V tiles of every job ----
@@ -230,67 +289,72 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd_dq_kernel(const
     }
     __syncwarp();
   } else if (warp == 1) {
-    // ---- MMA issuer: half jobs u = 2 j + h (keys 64 h .. 64 h + 63 of job j's tiles) ----
-    // issued S(0), dP(0), S(1), dP(1), then dQ(u), S(u + 2), dP(u + 2): the MMAs of the next
-    // half job run while the warpgroup works on the current one (two S / dP slots).
+    // ---- S / dP issuer. Job g (counted over the CTA's items): S = Q K^T into S slot g % 2
+    // once the dQ MMA of job g - 2 has completed, then dP = dO V^T once the warpgroups have
+    // read dP of job g - 1 (one dP slot).
     if (lane == 0) {
-      uint32_t rc = 0, gu = 0;
+      uint32_t rc = 0, g = 0;
       int n = 0;
       bool ok = true;
       for (int ii = i_begin; ok && ii < i_end; ++ii, ++n) {
         const BwdItem it = p.items[p.cta_items[ii]];
         if (!wait_bounded(BAR(C::B_AFULL), n & 1, guard, kBwdWaitAFull)) break;
-        tc_fence_after();
-        const uint32_t base = rc;   // job j: K tile at ring index base + 2 j, V tile at base + 2 j + 1
-        rc += 2 * uint32_t(it.job_count);
-        const int U = 2 * it.job_count;
-        auto ring = [&](uint32_t r) { return sbase + C::OFF_RING + (r % C::STAGES) * C::TILE_BYTES; };
-        auto ss = [&](int u) -> bool {
-          const uint32_t slot = (gu + u) & 1, rk = base + 2 * (u >> 1), rv = rk + 1, h = u & 1;
-          if (h == 0) {
-            if (!wait_bounded(BAR(C::B_RFULL + rk % C::STAGES), (rk / C::STAGES) & 1, guard, kBwdWaitRFull) ||
-                !wait_bounded(BAR(C::B_RFULL + rv % C::STAGES), (rv / C::STAGES) & 1, guard, kBwdWaitRFull))
-              return false;
-            tc_fence_after();
-          }
-          mma_half_ss<C::D>(tmem + C::TM_S + 64 * slot, sbase + C::OFF_A, ring(rk) + h * C::HALF_BYTES,
-                            C::IDESC_SS);   // S = Q K^T
-          mma_half_ss<C::D>(tmem + C::TM_P + 64 * slot, sbase + C::OFF_B, ring(rv) + h * C::HALF_BYTES,
-                            C::IDESC_SS);   // dP = dO V^T
-          if (h == 1) mma_commit(BAR(C::B_REMPTY + rv % C::STAGES));
-          mma_commit(BAR(C::B_SFULL + slot));
-          return true;
-        };
-        auto ts = [&](int u) -> bool {
-          const uint32_t g = gu + u, slot = g & 1, rk = base + 2 * (u >> 1), h = u & 1;
-          if (!wait_bounded(BAR(C::B_PFULL + slot), (g >> 1) & 1, guard, kBwdWaitPFull)) return false;
-          if (u == 0 && !wait_bounded(BAR(C::B_ACCEMPTY), (n & 1) ^ 1, guard, kBwdWaitAccEmpty)) return false;
+        for (int j = 0; ok && j < it.job_count; ++j, ++g, rc += 2) {
+          const uint32_t s = g & 1, rk = rc, rv = rc + 1;
+          ok = wait_bounded(BAR(C::B_SFREE + s), ((g >> 1) & 1) ^ 1, guard, kBwdWaitSFree) &&
+               wait_bounded(BAR(C::B_RFULL + rk % C::STAGES), (rk / C::STAGES) & 1, guard, kBwdWaitRFull);
+          if (!ok) break;
           tc_fence_after();
-          mma_half_ts(tmem + C::TM_ACC, tmem + C::TM_S + 64 * slot, ring(rk) + h * C::HALF_BYTES, C::IDESC_TS,
-                      u > 0 ? 1u : 0u);     // dQ += dS K
-          if (h == 1) mma_commit(BAR(C::B_REMPTY + rk % C::STAGES));
-          return true;
-        };
-        ok = ss(0) && ss(1);
-        for (int u = 0; ok && u < U; ++u) {
-          ok = ts(u);
-          if (ok && u + 2 < U) ok = ss(u + 2);
+          mma_tile_ss<C::D>(tmem + C::TM_S + 128 * s, sbase + C::OFF_A, ring(rk), C::IDESC_SS);   // S = Q K^T
+          mma_commit(BAR(C::B_SFULL + s));
+          ok = wait_bounded(BAR(C::B_DPREAD), (g & 1) ^ 1, guard, kBwdWaitDpRead) &&
+               wait_bounded(BAR(C::B_RFULL + rv % C::STAGES), (rv / C::STAGES) & 1, guard, kBwdWaitRFull);
+          if (!ok) break;
+          tc_fence_after();
+          mma_tile_ss<C::D>(tmem + C::TM_P, sbase + C::OFF_B, ring(rv), C::IDESC_SS);   // dP = dO V^T
+          mma_commit(BAR(C::B_DPFULL));
+          mma_commit(BAR(C::B_REMPTY + rv % C::STAGES));   // V is read by this MMA only
         }
         if (!ok) break;
-        mma_commit(BAR(C::B_ACCFULL));
-        mma_commit(BAR(C::B_AEMPTY));
-        gu += U;
+        mma_commit(BAR(C::B_AEMPTY));   // Q and dO are read by these MMAs only
       }
       mma_commit(BAR(C::B_DRAIN));
       wait_drain(BAR(C::B_DRAIN), 0, p.timeout_ns);
     }
     __syncwarp();
+  } else if (warp == 2) {
+    // ---- dQ issuer: dQ += dS K once the warpgroups have written dS over the job's S slot;
+    // frees the slot and the K tile on completion
+    if (lane == 0) {
+      uint32_t rc = 0, g = 0;
+      int n = 0;
+      bool ok = true;
+      for (int ii = i_begin; ok && ii < i_end; ++ii, ++n) {
+        const BwdItem it = p.items[p.cta_items[ii]];
+        for (int j = 0; ok && j < it.job_count; ++j, ++g, rc += 2) {
+          const uint32_t s = g & 1;
+          ok = wait_bounded(BAR(C::B_DSREADY + s), (g >> 1) & 1, guard, kBwdWaitDsReady);
+          if (ok && j == 0) ok = wait_bounded(BAR(C::B_ACCEMPTY), (n & 1) ^ 1, guard, kBwdWaitAccEmpty);
+          if (!ok) break;
+          tc_fence_after();
+          mma_tile_ts(tmem + C::TM_ACC, tmem + C::TM_S + 128 * s, ring(rc), C::IDESC_TS, j > 0 ? 1u : 0u);
+          mma_commit(BAR(C::B_SFREE + s));
+          mma_commit(BAR(C::B_REMPTY + rc % C::STAGES));
+        }
+        if (!ok) break;
+        mma_commit(BAR(C::B_ACCFULL));
+      }
+      mma_commit(BAR(C::B_DRAIN2));
+      wait_drain(BAR(C::B_DRAIN2), 0, p.timeout_ns);
+    }
+    __syncwarp();
   } else if (warp >= 4) {
-    // ---- elementwise warpgroup: thread r owns row r of the query tile ----
-    const int r = tid - 128;
+    // ---- two elementwise warpgroups: thread r of warpgroup w owns row r of the query tile
+    // and keys 64 w .. 64 w + 63 of every job ----
+    const int r = (warp & 3) * 32 + lane, w = (warp - 4) >> 2;
     const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
     const float sl2 = p.scale_log2;
-    uint32_t gu = 0;
+    uint32_t g = 0;
     int n = 0;
     bool ok = true;
     for (int ii = i_begin; ok && ii < i_end; ++ii, ++n) {
@@ -303,52 +367,77 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd_dq_kernel(const
         lse2 = l == -INFINITY ? INFINITY : l * 1.4426950408889634f;
         dlt = p.delta[grow];
       }
-      for (int u = 0; ok && u < 2 * it.job_count; ++u) {
-        const int mi = p.jobs[it.job_start + (u >> 1)].mask;
-        const int h = u & 1;
-        uint2 bits = make_uint2(0xffffffffu, 0xffffffffu);   // this half job's 64 key bits
-        if (mi >= 0) {
-          const uint4 b4 = __ldg(p.mask_tiles + int64_t(mi) * 128 + r);
-          bits = h ? make_uint2(b4.z, b4.w) : make_uint2(b4.x, b4.y);
-        } else if (mi == kMaskNone) {
-          bits = make_uint2(0u, 0u);
-        }
-        const uint32_t g = gu + u, slot = g & 1;
-        if (!__all_sync(0xffffffffu, wait_bounded(BAR(C::B_SFULL + slot), (g >> 1) & 1, guard, kBwdWaitSFull))) {
+      // mask bits one job ahead, mask tile indices two jobs ahead: no global load latency
+      // between two jobs
+      const int nj = it.job_count;
+      int mi_next = nj > 1 ? p.jobs[it.job_start + 1].mask : kMaskNone;
+      uint4 bits_next = row_bits(p.mask_tiles, p.jobs[it.job_start].mask, r);
+      for (int j = 0; ok && j < nj; ++j, ++g) {
+        const uint4 bits4 = bits_next;
+        bits_next = row_bits(p.mask_tiles, mi_next, r);
+        mi_next = j + 2 < nj ? p.jobs[it.job_start + j + 2].mask : kMaskNone;
+        const uint32_t s = g & 1;
+        if (!__all_sync(0xffffffffu, wait_bounded(BAR(C::B_SFULL + s), (g >> 1) & 1, guard, kBwdWaitSFull) &&
+                                         wait_bounded(BAR(C::B_DPFULL), g & 1, guard, kBwdWaitDpFull))) {
           ok = false;
           break;
         }
         tc_fence_after();
+        const uint32_t ts = tmem + lane_base + C::TM_S + 128 * s + 64 * w;
+        // this warpgroup's 64 dP columns, then the slot is free for the next job's dP
+        uint32_t dv[64], sv[32];
+        tmem_ld32x32(tmem + lane_base + C::TM_P + 64 * w, dv);
+        tmem_ld32x32(tmem + lane_base + C::TM_P + 64 * w + 32, dv + 32);
+        tmem_ld32x32(ts, sv);
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(BAR(C::B_DPREAD));
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
-          uint32_t sv[32], dv[32];
-          tmem_ld32x32(tmem + lane_base + C::TM_S + 64 * slot + 32 * c, sv);
-          tmem_ld32x32(tmem + lane_base + C::TM_P + 64 * slot + 32 * c, dv);
-          tmem_wait_ld();
-          const uint32_t w = c ? bits.y : bits.x;
-          uint32_t pk[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            float ds[2];
-#pragma unroll
-            for (int q = 0; q < 2; ++q) {
-              const float pr = ((w >> (2 * e + q)) & 1u) ? ex2(fmaf(__uint_as_float(sv[2 * e + q]), sl2, -lse2)) : 0.f;
-              ds[q] = pr * (__uint_as_float(dv[2 * e + q]) - dlt);
-            }
-            pk[e] = pack_bf16(ds[0], ds[1]);
+          if (c == 1) {
+            tmem_ld32x32(ts + 32, sv);
+            tmem_wait_ld();
           }
-          // dS of the slot's columns 32c .. 32c+31 over its S columns 16c .. 16c+15 (already read)
-          tmem_st32x16(tmem + lane_base + C::TM_S + 64 * slot + 16 * c, pk);
+          const uint32_t wb = w ? (c ? bits4.w : bits4.z) : (c ? bits4.y : bits4.x);   // keys 64 w + 32 c ..
+          const uint32_t* d32 = dv + 32 * c;
+          uint32_t pk[16];
+          if (wb == 0xffffffffu) {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              float ds[2];
+#pragma unroll
+              for (int q = 0; q < 2; ++q) {
+                const float pr = ex2(fmaf(__uint_as_float(sv[2 * e + q]), sl2, -lse2));
+                ds[q] = pr * (__uint_as_float(d32[2 * e + q]) - dlt);
+              }
+              pk[e] = pack_bf16(ds[0], ds[1]);
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              float ds[2];
+#pragma unroll
+              for (int q = 0; q < 2; ++q) {
+                const float pr =
+                    ((wb >> (2 * e + q)) & 1u) ? ex2(fmaf(__uint_as_float(sv[2 * e + q]), sl2, -lse2)) : 0.f;
+                ds[q] = pr * (__uint_as_float(d32[2 * e + q]) - dlt);
+              }
+              pk[e] = pack_bf16(ds[0], ds[1]);
+            }
+          }
+          // dS (bf16 pairs) of keys 64 w + 32 c .. over S columns 64 w + 16 c .. (already read)
+          tmem_st32x16(ts + 16 * c, pk);
         }
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(BAR(C::B_PFULL + slot));
+        mbar_arrive(BAR(C::B_DSREADY + s));
       }
-      gu += 2 * it.job_count;
       if (!ok) break;
       if (!__all_sync(0xffffffffu, wait_bounded(BAR(C::B_ACCFULL), n & 1, guard, kBwdWaitAccFull))) break;
       tc_fence_after();
-      store_grad_row<C::D>(tmem + lane_base + C::TM_ACC, p.scale, valid, p.g0 + grow * C::D);
+      // warpgroup w stores columns D/2 w .. D/2 w + D/2 - 1 of the row's dq
+      store_grad_cols<C::D / 2>(tmem + lane_base + C::TM_ACC + (C::D / 2) * w, p.scale, valid,
+                                p.g0 + grow * C::D + (C::D / 2) * w);
       tc_fence_before();
       mbar_arrive(BAR(C::B_ACCEMPTY));
     }
@@ -379,13 +468,16 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd_dkv_kernel(cons
       mbar_init(BAR(C::B_RFULL + s), 1);
       mbar_init(BAR(C::B_REMPTY + s), 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(BAR(C::B_SFULL + b), 1);
-      mbar_init(BAR(C::B_PFULL + b), 128);
-    }
+    mbar_init(BAR(C::B_SFULL), 1);
+    mbar_init(BAR(C::B_DPFULL), 1);
+    mbar_init(BAR(C::B_PREADY), C::EW);
+    mbar_init(BAR(C::B_DSREADY), C::EW);
+    mbar_init(BAR(C::B_SFREE), 1);
+    mbar_init(BAR(C::B_DPFREE), 1);
     mbar_init(BAR(C::B_ACCFULL), 1);
-    mbar_init(BAR(C::B_ACCEMPTY), 128);
+    mbar_init(BAR(C::B_ACCEMPTY), C::EW);
     mbar_init(BAR(C::B_DRAIN), 1);
+    mbar_init(BAR(C::B_DRAIN2), 1);
     misc[1] = 0u;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     prefetch_tmap(&p.tm_a);
@@ -403,6 +495,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd_dkv_kernel(cons
   tc_fence_after();
   const uint32_t tmem = misc[0];
   const int i_begin = p.cta_off[blockIdx.x], i_end = p.cta_off[blockIdx.x + 1];
+  auto ring = [&](uint32_t r) { return sbase + C::OFF_RING + (r % C::STAGES) * C::TILE_BYTES; };
 
   if (warp == 0) {
     // ---- TMA producer: K and V once per item, then Q and dO tiles of every job ----
@@ -443,146 +536,209 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd_dkv_kernel(cons
     }
     __syncwarp();
   } else if (warp == 1) {
-    // ---- MMA issuer: half jobs u = 2 j + h (query rows 64 h .. 64 h + 63 of job j's tiles),
-    // issued as in the dQ kernel: S^T(0), dP^T(0), S^T(1), dP^T(1), then dV, dK (u), S^T, dP^T (u + 2)
+    // ---- S^T / dP^T issuer. Job g: S^T = K Q^T once the dV MMA of job g - 1 (the reader of
+    // P^T, written over S^T) has completed; dP^T = V dO^T once the dK MMA of job g - 1 has.
     if (lane == 0) {
-      uint32_t rc = 0, gu = 0;
+      uint32_t rc = 0, g = 0;
       int n = 0;
       bool ok = true;
       for (int ii = i_begin; ok && ii < i_end; ++ii, ++n) {
         const BwdItem it = p.items[p.cta_items[ii]];
         if (!wait_bounded(BAR(C::B_AFULL), n & 1, guard, kBwdWaitAFull)) break;
-        tc_fence_after();
-        const uint32_t base = rc;   // job j: Q tile at ring index base + 2 j, dO tile at base + 2 j + 1
-        rc += 2 * uint32_t(it.job_count);
-        const int U = 2 * it.job_count;
-        auto ring = [&](uint32_t r) { return sbase + C::OFF_RING + (r % C::STAGES) * C::TILE_BYTES; };
-        auto ss = [&](int u) -> bool {
-          const uint32_t slot = (gu + u) & 1, rq = base + 2 * (u >> 1), rd = rq + 1, h = u & 1;
-          if (h == 0) {
-            if (!wait_bounded(BAR(C::B_RFULL + rq % C::STAGES), (rq / C::STAGES) & 1, guard, kBwdWaitRFull) ||
-                !wait_bounded(BAR(C::B_RFULL + rd % C::STAGES), (rd / C::STAGES) & 1, guard, kBwdWaitRFull))
-              return false;
-            tc_fence_after();
-          }
-          mma_half_ss<C::D>(tmem + C::TM_S + 64 * slot, sbase + C::OFF_A, ring(rq) + h * C::HALF_BYTES,
-                            C::IDESC_SS);   // S^T = K Q^T
-          mma_half_ss<C::D>(tmem + C::TM_P + 64 * slot, sbase + C::OFF_B, ring(rd) + h * C::HALF_BYTES,
-                            C::IDESC_SS);   // dP^T = V dO^T
-          mma_commit(BAR(C::B_SFULL + slot));
-          return true;
-        };
-        auto ts = [&](int u) -> bool {
-          const uint32_t g = gu + u, slot = g & 1, rq = base + 2 * (u >> 1), rd = rq + 1, h = u & 1;
-          if (!wait_bounded(BAR(C::B_PFULL + slot), (g >> 1) & 1, guard, kBwdWaitPFull)) return false;
-          if (u == 0 && !wait_bounded(BAR(C::B_ACCEMPTY), (n & 1) ^ 1, guard, kBwdWaitAccEmpty)) return false;
+        for (int j = 0; ok && j < it.job_count; ++j, ++g, rc += 2) {
+          const uint32_t rq = rc, rd = rc + 1;
+          ok = wait_bounded(BAR(C::B_SFREE), (g & 1) ^ 1, guard, kBwdWaitSFree) &&
+               wait_bounded(BAR(C::B_RFULL + rq % C::STAGES), (rq / C::STAGES) & 1, guard, kBwdWaitRFull);
+          if (!ok) break;
           tc_fence_after();
-          const uint32_t acc = u > 0 ? 1u : 0u;
-          mma_half_ts(tmem + C::TM_ACC, tmem + C::TM_S + 64 * slot, ring(rd) + h * C::HALF_BYTES, C::IDESC_TS,
-                      acc);                 // dV += P^T dO
-          mma_half_ts(tmem + C::TM_ACC + C::D, tmem + C::TM_P + 64 * slot, ring(rq) + h * C::HALF_BYTES,
-                      C::IDESC_TS, acc);    // dK += dS^T Q
-          if (h == 1) {
-            mma_commit(BAR(C::B_REMPTY + rq % C::STAGES));
-            mma_commit(BAR(C::B_REMPTY + rd % C::STAGES));
-          }
-          return true;
-        };
-        ok = ss(0) && ss(1);
-        for (int u = 0; ok && u < U; ++u) {
-          ok = ts(u);
-          if (ok && u + 2 < U) ok = ss(u + 2);
+          mma_tile_ss<C::D>(tmem + C::TM_S, sbase + C::OFF_A, ring(rq), C::IDESC_SS);   // S^T = K Q^T
+          mma_commit(BAR(C::B_SFULL));
+          ok = wait_bounded(BAR(C::B_DPFREE), (g & 1) ^ 1, guard, kBwdWaitDpFree) &&
+               wait_bounded(BAR(C::B_RFULL + rd % C::STAGES), (rd / C::STAGES) & 1, guard, kBwdWaitRFull);
+          if (!ok) break;
+          tc_fence_after();
+          mma_tile_ss<C::D>(tmem + C::TM_P, sbase + C::OFF_B, ring(rd), C::IDESC_SS);   // dP^T = V dO^T
+          mma_commit(BAR(C::B_DPFULL));
         }
         if (!ok) break;
-        mma_commit(BAR(C::B_ACCFULL));
-        mma_commit(BAR(C::B_AEMPTY));
-        gu += U;
+        mma_commit(BAR(C::B_AEMPTY));   // K and V are read by these MMAs only
       }
       mma_commit(BAR(C::B_DRAIN));
       wait_drain(BAR(C::B_DRAIN), 0, p.timeout_ns);
     }
     __syncwarp();
+  } else if (warp == 2) {
+    // ---- dV / dK issuer: dV += P^T dO once P^T is in TMEM (frees S^T on completion), dK +=
+    // dS^T Q once dS^T is (frees dP^T and the job's Q and dO tiles)
+    if (lane == 0) {
+      uint32_t rc = 0, g = 0;
+      int n = 0;
+      bool ok = true;
+      for (int ii = i_begin; ok && ii < i_end; ++ii, ++n) {
+        const BwdItem it = p.items[p.cta_items[ii]];
+        for (int j = 0; ok && j < it.job_count; ++j, ++g, rc += 2) {
+          const uint32_t rq = rc, rd = rc + 1, acc = j > 0 ? 1u : 0u;
+          ok = wait_bounded(BAR(C::B_PREADY), g & 1, guard, kBwdWaitPFull);
+          if (ok && j == 0) ok = wait_bounded(BAR(C::B_ACCEMPTY), (n & 1) ^ 1, guard, kBwdWaitAccEmpty);
+          if (!ok) break;
+          tc_fence_after();
+          mma_tile_ts(tmem + C::TM_ACC, tmem + C::TM_S, ring(rd), C::IDESC_TS, acc);   // dV += P^T dO
+          mma_commit(BAR(C::B_SFREE));
+          if (!wait_bounded(BAR(C::B_DSREADY), g & 1, guard, kBwdWaitDsReady)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          mma_tile_ts(tmem + C::TM_ACC + C::D, tmem + C::TM_P, ring(rq), C::IDESC_TS, acc);   // dK += dS^T Q
+          mma_commit(BAR(C::B_DPFREE));
+          // Q and dO: their last readers are this dK MMA and the dV MMA before it (dP^T of
+          // the job completed before the warpgroups wrote dS^T)
+          mma_commit(BAR(C::B_REMPTY + rq % C::STAGES));
+          mma_commit(BAR(C::B_REMPTY + rd % C::STAGES));
+        }
+        if (!ok) break;
+        mma_commit(BAR(C::B_ACCFULL));
+      }
+      mma_commit(BAR(C::B_DRAIN2));
+      wait_drain(BAR(C::B_DRAIN2), 0, p.timeout_ns);
+    }
+    __syncwarp();
   } else if (warp >= 4) {
-    // ---- elementwise warpgroup: thread r owns key row r of the key tile ----
-    const int r = tid - 128;
+    // ---- two elementwise warpgroups: thread r of warpgroup w owns key row r of the key tile
+    // and query rows 64 w .. 64 w + 63 of every job ----
+    const int r = (warp & 3) * 32 + lane, w = (warp - 4) >> 2;
     const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
     const float sl2 = p.scale_log2;
     // this warp's copy of the job's per-query-row terms (no barrier across warps)
     float* rl2 = reinterpret_cast<float*>(sgen + C::OFF_ROWV) + (warp - 4) * 256;
     float* rdl = rl2 + 128;
-    uint32_t gu = 0;
+    uint32_t g = 0;
     int n = 0;
     bool ok = true;
     for (int ii = i_begin; ok && ii < i_end; ++ii, ++n) {
       const BwdItem it = p.items[p.cta_items[ii]];
-      uint4 bits = make_uint4(0u, 0u, 0u, 0u);
-      for (int u = 0; ok && u < 2 * it.job_count; ++u) {
-        const int h = u & 1;
-        if (h == 0) {
-          // a new job: its query rows' lse (log2 e scaled) and delta into this warp's copy
-          const BwdJob jb = p.jobs[it.job_start + (u >> 1)];
-          __syncwarp();   // the previous job's reads of rl2 / rdl are done
+      // The next job's lse / delta and mask bits are loaded while this job runs, the job
+      // record two jobs ahead: only an item's first job waits for global memory.
+      const int nj = it.job_count;
+      const BwdJob none{0, kMaskNone, 0, 0};
+      BwdJob jb_next = nj > 1 ? p.jobs[it.job_start + 1] : none;
+      float nl[4], nd[4];
+      auto load_terms = [&](const BwdJob& jb) {
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const int qr = 4 * lane + k;
-            float l2 = INFINITY, dl = 0.f;
-            if (qr < jb.rows) {
-              const int64_t g = int64_t(jb.tok + qr) * p.hq + jb.head;
-              const float l = p.lse[g];
-              l2 = l == -INFINITY ? INFINITY : l * 1.4426950408889634f;
-              dl = p.delta[g];
-            }
-            rl2[qr] = l2;
-            rdl[qr] = dl;
+        for (int q = 0; q < 4; ++q) {
+          const int qr = 4 * lane + q;
+          nl[q] = -INFINITY;
+          nd[q] = 0.f;
+          if (qr < jb.rows) {
+            const int64_t gi = int64_t(jb.tok + qr) * p.hq + jb.head;
+            nl[q] = p.lse[gi];
+            nd[q] = p.delta[gi];
           }
-          __syncwarp();
-          bits = make_uint4(0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu);
-          if (jb.mask >= 0) bits = __ldg(p.mask_tiles + int64_t(jb.mask) * 128 + r);
-          else if (jb.mask == kMaskNone) bits = make_uint4(0u, 0u, 0u, 0u);
         }
-        const uint32_t g = gu + u, slot = g & 1;
-        if (!__all_sync(0xffffffffu, wait_bounded(BAR(C::B_SFULL + slot), (g >> 1) & 1, guard, kBwdWaitSFull))) {
+      };
+      uint4 bits_next;
+      {
+        const BwdJob j0 = p.jobs[it.job_start];
+        load_terms(j0);
+        bits_next = row_bits(p.mask_tiles, j0.mask, r);
+      }
+      for (int j = 0; ok && j < nj; ++j, ++g) {
+        // the job's query rows' lse (log2 e scaled; -inf, no key, as +inf) and delta into this
+        // warp's copy
+        __syncwarp();   // the previous job's reads of rl2 / rdl are done
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          rl2[4 * lane + q] = nl[q] == -INFINITY ? INFINITY : nl[q] * 1.4426950408889634f;
+          rdl[4 * lane + q] = nd[q];
+        }
+        __syncwarp();
+        const uint4 bits = bits_next;
+        load_terms(jb_next);
+        bits_next = row_bits(p.mask_tiles, jb_next.mask, r);
+        jb_next = j + 2 < nj ? p.jobs[it.job_start + j + 2] : none;
+
+        if (!__all_sync(0xffffffffu, wait_bounded(BAR(C::B_SFULL), g & 1, guard, kBwdWaitSFull))) {
           ok = false;
           break;
         }
         tc_fence_after();
+        // P^T for query rows 64 w .. 64 w + 63: kept in registers for dS^T, written (bf16
+        // pairs) over S^T columns 64 w .. 64 w + 31
+        const uint32_t ts = tmem + lane_base + C::TM_S + 64 * w;
+        float pr[64];
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
-          uint32_t sv[32], dv[32];
-          tmem_ld32x32(tmem + lane_base + C::TM_S + 64 * slot + 32 * c, sv);
-          tmem_ld32x32(tmem + lane_base + C::TM_P + 64 * slot + 32 * c, dv);
+          uint32_t sv[32];
+          tmem_ld32x32(ts + 32 * c, sv);
           tmem_wait_ld();
-          const int q0 = 64 * h + 32 * c;   // first query row of the chunk
-          const uint32_t w = h ? (c ? bits.w : bits.z) : (c ? bits.y : bits.x);
-          uint32_t pp[16], pd[16];
+          const uint32_t wb = w ? (c ? bits.w : bits.z) : (c ? bits.y : bits.x);
+          const float4* l2v = reinterpret_cast<const float4*>(rl2 + 64 * w + 32 * c);
+          if (wb == 0xffffffffu) {
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            float pr[2], ds[2];
-#pragma unroll
-            for (int q = 0; q < 2; ++q) {
-              const int qi = q0 + 2 * e + q;
-              pr[q] = ((w >> (2 * e + q)) & 1u) ? ex2(fmaf(__uint_as_float(sv[2 * e + q]), sl2, -rl2[qi])) : 0.f;
-              ds[q] = pr[q] * (__uint_as_float(dv[2 * e + q]) - rdl[qi]);
+            for (int f = 0; f < 8; ++f) {
+              const float4 la = l2v[f];
+              pr[32 * c + 4 * f + 0] = ex2(fmaf(__uint_as_float(sv[4 * f + 0]), sl2, -la.x));
+              pr[32 * c + 4 * f + 1] = ex2(fmaf(__uint_as_float(sv[4 * f + 1]), sl2, -la.y));
+              pr[32 * c + 4 * f + 2] = ex2(fmaf(__uint_as_float(sv[4 * f + 2]), sl2, -la.z));
+              pr[32 * c + 4 * f + 3] = ex2(fmaf(__uint_as_float(sv[4 * f + 3]), sl2, -la.w));
             }
-            pp[e] = pack_bf16(pr[0], pr[1]);
-            pd[e] = pack_bf16(ds[0], ds[1]);
+          } else {
+#pragma unroll
+            for (int f = 0; f < 8; ++f) {
+              const float4 la = l2v[f];
+              const float lq[4] = {la.x, la.y, la.z, la.w};
+#pragma unroll
+              for (int q = 0; q < 4; ++q)
+                pr[32 * c + 4 * f + q] = ((wb >> (4 * f + q)) & 1u)
+                                             ? ex2(fmaf(__uint_as_float(sv[4 * f + q]), sl2, -lq[q]))
+                                             : 0.f;
+            }
           }
-          // P^T over the slot's S^T columns 16c.., dS^T over its dP^T columns 16c.. (already read)
-          tmem_st32x16(tmem + lane_base + C::TM_S + 64 * slot + 16 * c, pp);
-          tmem_st32x16(tmem + lane_base + C::TM_P + 64 * slot + 16 * c, pd);
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) pk[e] = pack_bf16(pr[32 * c + 2 * e], pr[32 * c + 2 * e + 1]);
+          tmem_st32x16(ts + 16 * c, pk);
         }
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(BAR(C::B_PFULL + slot));
+        mbar_arrive(BAR(C::B_PREADY));
+        // dS^T = P^T (dP^T - delta) over dP^T columns 64 w .. 64 w + 31
+        if (!__all_sync(0xffffffffu, wait_bounded(BAR(C::B_DPFULL), g & 1, guard, kBwdWaitDpFull))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t tp = tmem + lane_base + C::TM_P + 64 * w;
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          uint32_t dv[32];
+          tmem_ld32x32(tp + 32 * c, dv);
+          tmem_wait_ld();
+          const float4* dlv = reinterpret_cast<const float4*>(rdl + 64 * w + 32 * c);
+          uint32_t pk[16];
+#pragma unroll
+          for (int f = 0; f < 8; ++f) {
+            const float4 da = dlv[f];
+            const float* pp = pr + 32 * c + 4 * f;
+            pk[2 * f] = pack_bf16(pp[0] * (__uint_as_float(dv[4 * f + 0]) - da.x),
+                                  pp[1] * (__uint_as_float(dv[4 * f + 1]) - da.y));
+            pk[2 * f + 1] = pack_bf16(pp[2] * (__uint_as_float(dv[4 * f + 2]) - da.z),
+                                      pp[3] * (__uint_as_float(dv[4 * f + 3]) - da.w));
+          }
+          tmem_st32x16(tp + 16 * c, pk);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(BAR(C::B_DSREADY));
       }
-      gu += 2 * it.job_count;
       if (!ok) break;
       if (!__all_sync(0xffffffffu, wait_bounded(BAR(C::B_ACCFULL), n & 1, guard, kBwdWaitAccFull))) break;
       tc_fence_after();
+      // warpgroup 0 stores the row's dv, warpgroup 1 its dk
       const bool valid = r < it.rows;
       const int64_t grow = int64_t(it.tok + r) * p.hkv + it.kv_head;
-      store_grad_row<C::D>(tmem + lane_base + C::TM_ACC, 1.f, valid, p.g1 + grow * C::D);           // dv
-      store_grad_row<C::D>(tmem + lane_base + C::TM_ACC + C::D, p.scale, valid, p.g0 + grow * C::D);  // dk
+      if (w == 0) store_grad_cols<C::D>(tmem + lane_base + C::TM_ACC, 1.f, valid, p.g1 + grow * C::D);
+      else store_grad_cols<C::D>(tmem + lane_base + C::TM_ACC + C::D, p.scale, valid, p.g0 + grow * C::D);
       tc_fence_before();
       mbar_arrive(BAR(C::B_ACCEMPTY));
     }
@@ -594,16 +750,22 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd_dkv_kernel(cons
   if (warp == 1) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem) : "memory");
 }
 
-template <class C, bool DKV>
+template <class C>
 attn_status_t launch_bwd(int ctas, const BwdParams& p, cudaStream_t stream) {
-  const cudaError_t attr = once_per_device([] {
-    return DKV ? cudaFuncSetAttribute(masked_attn_bwd_dkv_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      C::SMEM_BYTES)
-               : cudaFuncSetAttribute(masked_attn_bwd_dq_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      C::SMEM_BYTES);
-  });
-  if (attr != cudaSuccess) return ATTN_ERR_CUDA;
-  if (DKV) masked_attn_bwd_dkv_kernel<C><<<ctas, C::THREADS, C::SMEM_BYTES, stream>>>(p);
+  if constexpr (C::DKV) {
+    const cudaError_t attr = once_per_device([] {
+      return cudaFuncSetAttribute(masked_attn_bwd_dkv_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  C::SMEM_BYTES);
+    });
+    if (attr != cudaSuccess) return ATTN_ERR_CUDA;
+  } else {
+    const cudaError_t attr = once_per_device([] {
+      return cudaFuncSetAttribute(masked_attn_bwd_dq_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  C::SMEM_BYTES);
+    });
+    if (attr != cudaSuccess) return ATTN_ERR_CUDA;
+  }
+  if constexpr (C::DKV) masked_attn_bwd_dkv_kernel<C><<<ctas, C::THREADS, C::SMEM_BYTES, stream>>>(p);
   else masked_attn_bwd_dq_kernel<C><<<ctas, C::THREADS, C::SMEM_BYTES, stream>>>(p);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
@@ -663,11 +825,11 @@ attn_status_t mfa_launch_backward(const attn_plan_t* plan, const void* q, const 
   pk.g1 = static_cast<__nv_bfloat16*>(dv);
   attn_status_t st;
   if (D == 64) {
-    st = launch_bwd<BwdCfg<64>, false>(plan->bq_ctas, pq, stream);
-    if (st == ATTN_OK) st = launch_bwd<BwdCfg<64>, true>(plan->bkv_ctas, pk, stream);
+    st = launch_bwd<BwdCfg<64, false>>(plan->bq_ctas, pq, stream);
+    if (st == ATTN_OK) st = launch_bwd<BwdCfg<64, true>>(plan->bkv_ctas, pk, stream);
   } else {
-    st = launch_bwd<BwdCfg<128>, false>(plan->bq_ctas, pq, stream);
-    if (st == ATTN_OK) st = launch_bwd<BwdCfg<128>, true>(plan->bkv_ctas, pk, stream);
+    st = launch_bwd<BwdCfg<128, false>>(plan->bq_ctas, pq, stream);
+    if (st == ATTN_OK) st = launch_bwd<BwdCfg<128, true>>(plan->bkv_ctas, pk, stream);
   }
   return st;
 }
