@@ -19,8 +19,8 @@
 // dV and dK; one thread); warps 4-11 two elementwise warpgroups, one TMEM lane (= one tile
 // row) per thread, the first warpgroup on columns 0..63 of every job and the second on
 // columns 64..127. Tiles are 128 rows of one head, 64-column boxes with the 128-byte swizzle;
-// a ring of STAGES tile slots streams the per-job operands (dQ: K and V tiles; dK/dV: Q and
-// dO tiles). A job is one 128 x 128 block, its S and dP MMAs M = 128, N = 128: the tensor
+// rings of tile slots stream the per-job operands (dQ: a ring of K tiles, held until the
+// dQ MMA, and a shallower one of V tiles; dK/dV: one ring of Q and dO tiles). A job is one 128 x 128 block, its S and dP MMAs M = 128, N = 128: the tensor
 // core reads 8 KiB of shared memory per 128 x 128 x 16 step, the rate its 64-cycle step can
 // take (narrower N re-reads A for every N block). The hand-offs are per operand, so each MMA
 // starts as soon as the TMEM it reads or overwrites allows:
@@ -80,20 +80,25 @@ struct BwdCfg {
   static constexpr int NBOX = D / 64;                  // 64-column boxes per tile
   static constexpr int BOX_BYTES = 128 * 128;          // 128 rows x 128 bytes
   static constexpr int TILE_BYTES = NBOX * BOX_BYTES;  // one 128-row tile of one head
-  static constexpr int STAGES = D == 128 ? 4 : 8;      // ring tile slots (two per job)
+  // Ring tile slots. dK/dV: one ring of Q and dO tiles, two per job. dQ: a ring of K tiles
+  // and a ring of V tiles -- K is held until the job's dQ MMA, V only until its dP MMA, so the
+  // K ring is the deeper one.
+  static constexpr int STAGES = D == 128 ? 4 : 8;
+  static constexpr int KST = D == 128 ? 3 : 5, VST = D == 128 ? 2 : 3;
+  static constexpr int RING = DKV ? STAGES : KST + VST;
   // TMEM: dQ -- S slots at 0 and 128, dP at 256, dQ at 384; dK/dV -- S^T at 0, dP^T at
   // 128, dV at 256, dK at 256 + D
   static constexpr int NS = DKV ? 1 : 2;               // S slots
   static constexpr int TM_S = 0, TM_P = 128 * NS, TM_ACC = TM_P + 128;
   static constexpr int OFF_A = 0, OFF_B = TILE_BYTES, OFF_RING = 2 * TILE_BYTES;
-  static constexpr int OFF_ROWV = OFF_RING + STAGES * TILE_BYTES;  // dK/dV: per warp 128 lse2 + 128 delta
+  static constexpr int OFF_ROWV = OFF_RING + RING * TILE_BYTES;  // dK/dV: per warp 128 lse2 + 128 delta
   static constexpr int OFF_BAR = OFF_ROWV + (DKV ? 8 * 2 * 128 * 4 : 0);
   // dQ:   SFULL[s] S of the slot computed, DPFULL dP computed, DPREAD dP read by the
   //       warpgroups, DSREADY[s] dS written, SFREE[s] dQ MMA of the slot completed.
   // dK/dV: SFULL S^T computed, DPFULL dP^T computed, PREADY P^T written, DSREADY dS^T
   //       written, SFREE the dV MMA (reader of P^T) completed, DPFREE the dK MMA completed.
-  static constexpr int B_AFULL = 0, B_AEMPTY = 1, B_RFULL = 2, B_REMPTY = B_RFULL + STAGES,
-                       B_SFULL = B_REMPTY + STAGES, B_DPFULL = B_SFULL + NS, B_DPREAD = B_DPFULL + 1,
+  static constexpr int B_AFULL = 0, B_AEMPTY = 1, B_RFULL = 2, B_REMPTY = B_RFULL + RING,
+                       B_SFULL = B_REMPTY + RING, B_DPFULL = B_SFULL + NS, B_DPREAD = B_DPFULL + 1,
                        B_PREADY = B_DPREAD + 1, B_DSREADY = B_PREADY + 1, B_SFREE = B_DSREADY + NS,
                        B_DPFREE = B_SFREE + NS, B_ACCFULL = B_DPFREE + 1, B_ACCEMPTY = B_ACCFULL + 1,
                        B_DRAIN = B_ACCEMPTY + 1, B_DRAIN2 = B_DRAIN + 1, NBAR = B_DRAIN2 + 1;
@@ -216,7 +221,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd_dq_kernel(const
   if (tid == 0) {
     mbar_init(BAR(C::B_AFULL), 1);
     mbar_init(BAR(C::B_AEMPTY), 1);
-    for (int s = 0; s < C::STAGES; ++s) {
+    for (int s = 0; s < C::RING; ++s) {
       mbar_init(BAR(C::B_RFULL + s), 1);
       mbar_init(BAR(C::B_REMPTY + s), 1);
     }
@@ -248,12 +253,15 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd_dq_kernel(const
   tc_fence_after();
   const uint32_t tmem = misc[0];
   const int i_begin = p.cta_off[blockIdx.x], i_end = p.cta_off[blockIdx.x + 1];
-  auto ring = [&](uint32_t r) { return sbase + C::OFF_RING + (r % C::STAGES) * C::TILE_BYTES; };
+  // job g's K tile in slot g % KST of the K ring, its V tile in slot KST + g % VST
+  auto kslot = [](uint32_t g) { return g % C::KST; };
+  auto vslot = [](uint32_t g) { return C::KST + g % C::VST; };
+  auto tile = [&](uint32_t slot) { return sbase + C::OFF_RING + slot * C::TILE_BYTES; };
 
   if (warp == 0) {
     // ---- TMA producer: Q and dO once per item, then K and V tiles of every job ----
     if (lane == 0) {
-      uint32_t rc = 0;
+      uint32_t g = 0;
       int n = 0, a_last = -1;
       bool ok = true;
       for (int ii = i_begin; ok && ii < i_end; ++ii, ++n) {
@@ -267,24 +275,26 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd_dq_kernel(const
             tma_load_3d(sbase + C::OFF_B + c * C::BOX_BYTES, &p.tm_b, c * 64, it.head, it.tok, BAR(C::B_AFULL));
           }
         }
-        for (int j = 0; ok && j < it.job_count; ++j) {
+        for (int j = 0; ok && j < it.job_count; ++j, ++g) {
           const BwdJob jb = p.jobs[it.job_start + j];
-          for (int op = 0; op < 2; ++op, ++rc) {
-            const uint32_t slot = rc % C::STAGES;
-            if (!wait_bounded(BAR(C::B_REMPTY + slot), ((rc / C::STAGES) & 1) ^ 1, guard, kBwdWaitREmpty)) {
+          for (int op = 0; op < 2; ++op) {
+            const uint32_t slot = op == 0 ? kslot(g) : vslot(g), use = op == 0 ? g / C::KST : g / C::VST;
+            if (!wait_bounded(BAR(C::B_REMPTY + slot), (use & 1) ^ 1, guard, kBwdWaitREmpty)) {
               ok = false;
               break;
             }
             mbar_expect_tx(BAR(C::B_RFULL + slot), C::TILE_BYTES);
             const CUtensorMap* tm = op == 0 ? &p.tm_c : &p.tm_d;
             for (int c = 0; c < C::NBOX; ++c)
-              tma_load_3d(sbase + C::OFF_RING + slot * C::TILE_BYTES + c * C::BOX_BYTES, tm, c * 64, it.kv_head,
-                          jb.tok, BAR(C::B_RFULL + slot));
+              tma_load_3d(tile(slot) + c * C::BOX_BYTES, tm, c * 64, it.kv_head, jb.tok, BAR(C::B_RFULL + slot));
           }
         }
       }
-      for (uint32_t r = rc > uint32_t(C::STAGES) ? rc - C::STAGES : 0u; r < rc; ++r)
-        wait_drain(BAR(C::B_RFULL + r % C::STAGES), (r / C::STAGES) & 1, p.timeout_ns);
+      // let the loads in flight land before the CTA exits
+      for (uint32_t x = g > uint32_t(C::KST) ? g - C::KST : 0u; x < g; ++x)
+        wait_drain(BAR(C::B_RFULL + kslot(x)), (x / C::KST) & 1, p.timeout_ns);
+      for (uint32_t x = g > uint32_t(C::VST) ? g - C::VST : 0u; x < g; ++x)
+        wait_drain(BAR(C::B_RFULL + vslot(x)), (x / C::VST) & 1, p.timeout_ns);
       if (a_last >= 0) wait_drain(BAR(C::B_AFULL), a_last & 1, p.timeout_ns);
     }
     __syncwarp();
@@ -293,27 +303,27 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd_dq_kernel(const
     // once the dQ MMA of job g - 2 has completed, then dP = dO V^T once the warpgroups have
     // read dP of job g - 1 (one dP slot).
     if (lane == 0) {
-      uint32_t rc = 0, g = 0;
+      uint32_t g = 0;
       int n = 0;
       bool ok = true;
       for (int ii = i_begin; ok && ii < i_end; ++ii, ++n) {
         const BwdItem it = p.items[p.cta_items[ii]];
         if (!wait_bounded(BAR(C::B_AFULL), n & 1, guard, kBwdWaitAFull)) break;
-        for (int j = 0; ok && j < it.job_count; ++j, ++g, rc += 2) {
-          const uint32_t s = g & 1, rk = rc, rv = rc + 1;
+        for (int j = 0; ok && j < it.job_count; ++j, ++g) {
+          const uint32_t s = g & 1, ks = kslot(g), vs = vslot(g);
           ok = wait_bounded(BAR(C::B_SFREE + s), ((g >> 1) & 1) ^ 1, guard, kBwdWaitSFree) &&
-               wait_bounded(BAR(C::B_RFULL + rk % C::STAGES), (rk / C::STAGES) & 1, guard, kBwdWaitRFull);
+               wait_bounded(BAR(C::B_RFULL + ks), (g / C::KST) & 1, guard, kBwdWaitRFull);
           if (!ok) break;
           tc_fence_after();
-          mma_tile_ss<C::D>(tmem + C::TM_S + 128 * s, sbase + C::OFF_A, ring(rk), C::IDESC_SS);   // S = Q K^T
+          mma_tile_ss<C::D>(tmem + C::TM_S + 128 * s, sbase + C::OFF_A, tile(ks), C::IDESC_SS);   // S = Q K^T
           mma_commit(BAR(C::B_SFULL + s));
           ok = wait_bounded(BAR(C::B_DPREAD), (g & 1) ^ 1, guard, kBwdWaitDpRead) &&
-               wait_bounded(BAR(C::B_RFULL + rv % C::STAGES), (rv / C::STAGES) & 1, guard, kBwdWaitRFull);
+               wait_bounded(BAR(C::B_RFULL + vs), (g / C::VST) & 1, guard, kBwdWaitRFull);
           if (!ok) break;
           tc_fence_after();
-          mma_tile_ss<C::D>(tmem + C::TM_P, sbase + C::OFF_B, ring(rv), C::IDESC_SS);   // dP = dO V^T
+          mma_tile_ss<C::D>(tmem + C::TM_P, sbase + C::OFF_B, tile(vs), C::IDESC_SS);   // dP = dO V^T
           mma_commit(BAR(C::B_DPFULL));
-          mma_commit(BAR(C::B_REMPTY + rv % C::STAGES));   // V is read by this MMA only
+          mma_commit(BAR(C::B_REMPTY + vs));   // V is read by this MMA only
         }
         if (!ok) break;
         mma_commit(BAR(C::B_AEMPTY));   // Q and dO are read by these MMAs only
@@ -326,20 +336,20 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd_dq_kernel(const
     // ---- dQ issuer: dQ += dS K once the warpgroups have written dS over the job's S slot;
     // frees the slot and the K tile on completion
     if (lane == 0) {
-      uint32_t rc = 0, g = 0;
+      uint32_t g = 0;
       int n = 0;
       bool ok = true;
       for (int ii = i_begin; ok && ii < i_end; ++ii, ++n) {
         const BwdItem it = p.items[p.cta_items[ii]];
-        for (int j = 0; ok && j < it.job_count; ++j, ++g, rc += 2) {
-          const uint32_t s = g & 1;
+        for (int j = 0; ok && j < it.job_count; ++j, ++g) {
+          const uint32_t s = g & 1, ks = kslot(g);
           ok = wait_bounded(BAR(C::B_DSREADY + s), (g >> 1) & 1, guard, kBwdWaitDsReady);
           if (ok && j == 0) ok = wait_bounded(BAR(C::B_ACCEMPTY), (n & 1) ^ 1, guard, kBwdWaitAccEmpty);
           if (!ok) break;
           tc_fence_after();
-          mma_tile_ts(tmem + C::TM_ACC, tmem + C::TM_S + 128 * s, ring(rc), C::IDESC_TS, j > 0 ? 1u : 0u);
+          mma_tile_ts(tmem + C::TM_ACC, tmem + C::TM_S + 128 * s, tile(ks), C::IDESC_TS, j > 0 ? 1u : 0u);
           mma_commit(BAR(C::B_SFREE + s));
-          mma_commit(BAR(C::B_REMPTY + rc % C::STAGES));
+          mma_commit(BAR(C::B_REMPTY + ks));
         }
         if (!ok) break;
         mma_commit(BAR(C::B_ACCFULL));
@@ -568,8 +578,8 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd_dkv_kernel(cons
     }
     __syncwarp();
   } else if (warp == 2) {
-    // ---- dV / dK issuer: dV += P^T dO once P^T is in TMEM (frees S^T on completion), dK +=
-    // dS^T Q once dS^T is (frees dP^T and the job's Q and dO tiles)
+    // ---- dV / dK issuer: dV += P^T dO once P^T is in TMEM (frees S^T and the dO tile on
+    // completion), dK += dS^T Q once dS^T is (frees dP^T and the Q tile)
     if (lane == 0) {
       uint32_t rc = 0, g = 0;
       int n = 0;
@@ -584,6 +594,12 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd_dkv_kernel(cons
           tc_fence_after();
           mma_tile_ts(tmem + C::TM_ACC, tmem + C::TM_S, ring(rd), C::IDESC_TS, acc);   // dV += P^T dO
           mma_commit(BAR(C::B_SFREE));
+          // dO: read by this dV MMA and the job's dP^T MMA; the tile is free once both completed
+          if (!wait_bounded(BAR(C::B_DPFULL), g & 1, guard, kBwdWaitDpFull)) {
+            ok = false;
+            break;
+          }
+          mma_commit(BAR(C::B_REMPTY + rd % C::STAGES));
           if (!wait_bounded(BAR(C::B_DSREADY), g & 1, guard, kBwdWaitDsReady)) {
             ok = false;
             break;
@@ -591,10 +607,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd_dkv_kernel(cons
           tc_fence_after();
           mma_tile_ts(tmem + C::TM_ACC + C::D, tmem + C::TM_P, ring(rq), C::IDESC_TS, acc);   // dK += dS^T Q
           mma_commit(BAR(C::B_DPFREE));
-          // Q and dO: their last readers are this dK MMA and the dV MMA before it (dP^T of
-          // the job completed before the warpgroups wrote dS^T)
-          mma_commit(BAR(C::B_REMPTY + rq % C::STAGES));
-          mma_commit(BAR(C::B_REMPTY + rd % C::STAGES));
+          mma_commit(BAR(C::B_REMPTY + rq % C::STAGES));   // Q: read by S^T and this MMA
         }
         if (!ok) break;
         mma_commit(BAR(C::B_ACCFULL));
