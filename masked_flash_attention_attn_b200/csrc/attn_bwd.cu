@@ -15,14 +15,16 @@
 //                       and dS^T (bf16) over them, then dV += P^T dO and dK += dS^T Q accumulate in
 //                       TMEM.
 // Both recompute P from the forward's lse instead of storing it. Warp roles: warp 0 TMA
-// producer; warp 1 issues the S / dP MMAs (one thread), warp 2 the accumulating MMAs (dQ, or
-// dV and dK; one thread); warps 4-11 two elementwise warpgroups, one TMEM lane (= one tile
-// row) per thread, the first warpgroup on columns 0..63 of every job and the second on
-// columns 64..127. Tiles are 128 rows of one head, 64-column boxes with the 128-byte swizzle;
-// rings of tile slots stream the per-job operands (dQ: a ring of K tiles, held until the
-// dQ MMA, and a shallower one of V tiles; dK/dV: one ring of Q and dO tiles). A job is one 128 x 128 block, its S and dP MMAs M = 128, N = 128: the tensor
-// core reads 8 KiB of shared memory per 128 x 128 x 16 step, the rate its 64-cycle step can
-// take (narrower N re-reads A for every N block). The hand-offs are per operand, so each MMA
+// producer; warp 1 issues the S (S^T) MMAs, warp 3 the dP (dP^T) MMAs and warp 2 the
+// accumulating MMAs (dQ, or dV and dK), one thread each, so that no MMA waits behind another
+// kind's dependency in a shared issue order; warps 4-11 two elementwise warpgroups, one TMEM
+// lane (= one tile row) per thread, the first warpgroup on columns 0..63 of every job and the
+// second on columns 64..127. Tiles are 128 rows of one head, 64-column boxes with the
+// 128-byte swizzle; rings of tile slots stream the per-job operands (dQ: a ring of K tiles,
+// held until the dQ MMA, and a shallower one of V tiles; dK/dV: one ring of Q and dO tiles).
+// A job is one 128 x 128 block, its S and dP MMAs M = 128, N = 128: the tensor core reads
+// 8 KiB of shared memory per 128 x 128 x 16 step, the rate its 64-cycle step can take
+// (narrower N re-reads A for every N block). The hand-offs are per operand, so each MMA
 // starts as soon as the TMEM it reads or overwrites allows:
 //   dQ:    S slots 0 / 1 (TMEM columns 0 and 128), one dP slot (256), dQ (384). S of job g+1
 //          runs while the warpgroups work on job g; dP of job g+1 once they have read dP of
@@ -101,7 +103,8 @@ struct BwdCfg {
                        B_SFULL = B_REMPTY + RING, B_DPFULL = B_SFULL + NS, B_DPREAD = B_DPFULL + 1,
                        B_PREADY = B_DPREAD + 1, B_DSREADY = B_PREADY + 1, B_SFREE = B_DSREADY + NS,
                        B_DPFREE = B_SFREE + NS, B_ACCFULL = B_DPFREE + 1, B_ACCEMPTY = B_ACCFULL + 1,
-                       B_DRAIN = B_ACCEMPTY + 1, B_DRAIN2 = B_DRAIN + 1, NBAR = B_DRAIN2 + 1;
+                       B_DRAIN = B_ACCEMPTY + 1, B_DRAIN2 = B_DRAIN + 1, B_DRAIN3 = B_DRAIN2 + 1,
+                       NBAR = B_DRAIN3 + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;       // [0] TMEM base, [1] abort flag
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;   // + slack to align the base to 1 KiB
   static constexpr int THREADS = 384;
@@ -220,7 +223,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd_dq_kernel(const
 #define BAR(i) (bar0 + 8u * uint32_t(i))
   if (tid == 0) {
     mbar_init(BAR(C::B_AFULL), 1);
-    mbar_init(BAR(C::B_AEMPTY), 1);
+    mbar_init(BAR(C::B_AEMPTY), 2);   // both S-side issuers commit
     for (int s = 0; s < C::RING; ++s) {
       mbar_init(BAR(C::B_RFULL + s), 1);
       mbar_init(BAR(C::B_REMPTY + s), 1);
@@ -236,6 +239,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd_dq_kernel(const
     mbar_init(BAR(C::B_ACCEMPTY), C::EW);
     mbar_init(BAR(C::B_DRAIN), 1);
     mbar_init(BAR(C::B_DRAIN2), 1);
+    mbar_init(BAR(C::B_DRAIN3), 1);
     misc[1] = 0u;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     prefetch_tmap(&p.tm_a);
@@ -299,9 +303,8 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd_dq_kernel(const
     }
     __syncwarp();
   } else if (warp == 1) {
-    // ---- S / dP issuer. Job g (counted over the CTA's items): S = Q K^T into S slot g % 2
-    // once the dQ MMA of job g - 2 has completed, then dP = dO V^T once the warpgroups have
-    // read dP of job g - 1 (one dP slot).
+    // ---- S issuer. Job g (counted over the CTA's items): S = Q K^T into S slot g % 2 once
+    // the dQ MMA of job g - 2 has completed
     if (lane == 0) {
       uint32_t g = 0;
       int n = 0;
@@ -310,13 +313,33 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd_dq_kernel(const
         const BwdItem it = p.items[p.cta_items[ii]];
         if (!wait_bounded(BAR(C::B_AFULL), n & 1, guard, kBwdWaitAFull)) break;
         for (int j = 0; ok && j < it.job_count; ++j, ++g) {
-          const uint32_t s = g & 1, ks = kslot(g), vs = vslot(g);
+          const uint32_t s = g & 1, ks = kslot(g);
           ok = wait_bounded(BAR(C::B_SFREE + s), ((g >> 1) & 1) ^ 1, guard, kBwdWaitSFree) &&
                wait_bounded(BAR(C::B_RFULL + ks), (g / C::KST) & 1, guard, kBwdWaitRFull);
           if (!ok) break;
           tc_fence_after();
           mma_tile_ss<C::D>(tmem + C::TM_S + 128 * s, sbase + C::OFF_A, tile(ks), C::IDESC_SS);   // S = Q K^T
           mma_commit(BAR(C::B_SFULL + s));
+        }
+        if (!ok) break;
+        mma_commit(BAR(C::B_AEMPTY));   // Q is read by these MMAs only
+      }
+      mma_commit(BAR(C::B_DRAIN));
+      wait_drain(BAR(C::B_DRAIN), 0, p.timeout_ns);
+    }
+    __syncwarp();
+  } else if (warp == 3) {
+    // ---- dP issuer: dP = dO V^T of job g into the dP slot once the warpgroups have read dP
+    // of job g - 1
+    if (lane == 0) {
+      uint32_t g = 0;
+      int n = 0;
+      bool ok = true;
+      for (int ii = i_begin; ok && ii < i_end; ++ii, ++n) {
+        const BwdItem it = p.items[p.cta_items[ii]];
+        if (!wait_bounded(BAR(C::B_AFULL), n & 1, guard, kBwdWaitAFull)) break;
+        for (int j = 0; ok && j < it.job_count; ++j, ++g) {
+          const uint32_t vs = vslot(g);
           ok = wait_bounded(BAR(C::B_DPREAD), (g & 1) ^ 1, guard, kBwdWaitDpRead) &&
                wait_bounded(BAR(C::B_RFULL + vs), (g / C::VST) & 1, guard, kBwdWaitRFull);
           if (!ok) break;
@@ -326,10 +349,10 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd_dq_kernel(const
           mma_commit(BAR(C::B_REMPTY + vs));   // V is read by this MMA only
         }
         if (!ok) break;
-        mma_commit(BAR(C::B_AEMPTY));   // Q and dO are read by these MMAs only
+        mma_commit(BAR(C::B_AEMPTY));   // dO is read by these MMAs only
       }
-      mma_commit(BAR(C::B_DRAIN));
-      wait_drain(BAR(C::B_DRAIN), 0, p.timeout_ns);
+      mma_commit(BAR(C::B_DRAIN3));
+      wait_drain(BAR(C::B_DRAIN3), 0, p.timeout_ns);
     }
     __syncwarp();
   } else if (warp == 2) {
@@ -473,7 +496,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd_dkv_kernel(cons
 #define BAR(i) (bar0 + 8u * uint32_t(i))
   if (tid == 0) {
     mbar_init(BAR(C::B_AFULL), 1);
-    mbar_init(BAR(C::B_AEMPTY), 1);
+    mbar_init(BAR(C::B_AEMPTY), 2);   // both S-side issuers commit
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(BAR(C::B_RFULL + s), 1);
       mbar_init(BAR(C::B_REMPTY + s), 1);
@@ -488,6 +511,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd_dkv_kernel(cons
     mbar_init(BAR(C::B_ACCEMPTY), C::EW);
     mbar_init(BAR(C::B_DRAIN), 1);
     mbar_init(BAR(C::B_DRAIN2), 1);
+    mbar_init(BAR(C::B_DRAIN3), 1);
     misc[1] = 0u;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     prefetch_tmap(&p.tm_a);
@@ -546,8 +570,8 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd_dkv_kernel(cons
     }
     __syncwarp();
   } else if (warp == 1) {
-    // ---- S^T / dP^T issuer. Job g: S^T = K Q^T once the dV MMA of job g - 1 (the reader of
-    // P^T, written over S^T) has completed; dP^T = V dO^T once the dK MMA of job g - 1 has.
+    // ---- S^T issuer. Job g: S^T = K Q^T once the dV MMA of job g - 1 (the reader of P^T,
+    // written over S^T) has completed
     if (lane == 0) {
       uint32_t rc = 0, g = 0;
       int n = 0;
@@ -556,13 +580,33 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd_dkv_kernel(cons
         const BwdItem it = p.items[p.cta_items[ii]];
         if (!wait_bounded(BAR(C::B_AFULL), n & 1, guard, kBwdWaitAFull)) break;
         for (int j = 0; ok && j < it.job_count; ++j, ++g, rc += 2) {
-          const uint32_t rq = rc, rd = rc + 1;
+          const uint32_t rq = rc;
           ok = wait_bounded(BAR(C::B_SFREE), (g & 1) ^ 1, guard, kBwdWaitSFree) &&
                wait_bounded(BAR(C::B_RFULL + rq % C::STAGES), (rq / C::STAGES) & 1, guard, kBwdWaitRFull);
           if (!ok) break;
           tc_fence_after();
           mma_tile_ss<C::D>(tmem + C::TM_S, sbase + C::OFF_A, ring(rq), C::IDESC_SS);   // S^T = K Q^T
           mma_commit(BAR(C::B_SFULL));
+        }
+        if (!ok) break;
+        mma_commit(BAR(C::B_AEMPTY));   // K is read by these MMAs only
+      }
+      mma_commit(BAR(C::B_DRAIN));
+      wait_drain(BAR(C::B_DRAIN), 0, p.timeout_ns);
+    }
+    __syncwarp();
+  } else if (warp == 3) {
+    // ---- dP^T issuer: dP^T = V dO^T of job g once the dK MMA of job g - 1 (the reader of
+    // dS^T, written over dP^T) has completed
+    if (lane == 0) {
+      uint32_t rc = 0, g = 0;
+      int n = 0;
+      bool ok = true;
+      for (int ii = i_begin; ok && ii < i_end; ++ii, ++n) {
+        const BwdItem it = p.items[p.cta_items[ii]];
+        if (!wait_bounded(BAR(C::B_AFULL), n & 1, guard, kBwdWaitAFull)) break;
+        for (int j = 0; ok && j < it.job_count; ++j, ++g, rc += 2) {
+          const uint32_t rd = rc + 1;
           ok = wait_bounded(BAR(C::B_DPFREE), (g & 1) ^ 1, guard, kBwdWaitDpFree) &&
                wait_bounded(BAR(C::B_RFULL + rd % C::STAGES), (rd / C::STAGES) & 1, guard, kBwdWaitRFull);
           if (!ok) break;
@@ -571,10 +615,10 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd_dkv_kernel(cons
           mma_commit(BAR(C::B_DPFULL));
         }
         if (!ok) break;
-        mma_commit(BAR(C::B_AEMPTY));   // K and V are read by these MMAs only
+        mma_commit(BAR(C::B_AEMPTY));   // V is read by these MMAs only
       }
-      mma_commit(BAR(C::B_DRAIN));
-      wait_drain(BAR(C::B_DRAIN), 0, p.timeout_ns);
+      mma_commit(BAR(C::B_DRAIN3));
+      wait_drain(BAR(C::B_DRAIN3), 0, p.timeout_ns);
     }
     __syncwarp();
   } else if (warp == 2) {
