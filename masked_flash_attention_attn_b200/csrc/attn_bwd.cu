@@ -29,11 +29,14 @@
 //   dQ:    S slots 0 / 1 (TMEM columns 0 and 128), one dP slot (256), dQ (384). S of job g+1
 //          runs while the warpgroups work on job g; dP of job g+1 once they have read dP of
 //          job g (they read it first); dQ += dS K once they have written dS over S.
-//   dK/dV: one S^T slot (0), one dP^T slot (128), dV (256) and dK (256 + D). The warpgroups
-//          write P^T over S^T (dV += P^T dO starts), then dS^T over dP^T (dK += dS^T Q
-//          starts); S^T of job g+1 once dV of job g has completed, dP^T once dK has.
-// bf16 P / dS pairs of columns 0..63 go to TMEM columns 0..31 of their slot and those of
-// columns 64..127 to 64..95, each within the columns its warpgroup has already read. Every
+//   dK/dV: two job slots (TMEM columns 0 and 128), dV (256) and dK (256 + D). Job g uses
+//          slot g % 2 three times over: S^T, which the warpgroups read into registers; then
+//          dP^T, computed over it; then P^T and dS^T (bf16), which the warpgroups write over
+//          dP^T and dV += P^T dO, dK += dS^T Q read. Two jobs are in flight: S^T of job g+1
+//          runs while the warpgroups work on job g.
+// dQ: bf16 dS pairs of columns 0..63 go to TMEM columns 0..31 of the S slot and those of
+// columns 64..127 to 64..95; dK/dV: P^T pairs to columns 0..31 / 64..95 of the slot and dS^T
+// pairs to 32..63 / 96..127. Each warpgroup writes only columns it has already read. Every
 // mbarrier wait is bounded as in the forward.
 
 #include <cuda.h>
@@ -88,23 +91,23 @@ struct BwdCfg {
   static constexpr int STAGES = D == 128 ? 4 : 8;
   static constexpr int KST = D == 128 ? 3 : 5, VST = D == 128 ? 2 : 3;
   static constexpr int RING = DKV ? STAGES : KST + VST;
-  // TMEM: dQ -- S slots at 0 and 128, dP at 256, dQ at 384; dK/dV -- S^T at 0, dP^T at
-  // 128, dV at 256, dK at 256 + D
-  static constexpr int NS = DKV ? 1 : 2;               // S slots
-  static constexpr int TM_S = 0, TM_P = 128 * NS, TM_ACC = TM_P + 128;
+  // TMEM: dQ -- S slots at 0 and 128, dP at 256, dQ at 384; dK/dV -- two job slots at 0 and
+  // 128 (S^T, then dP^T over it, then P^T and dS^T), dV at 256, dK at 256 + D
+  static constexpr int NS = 2;                         // S (dQ) or job (dK/dV) slots
+  static constexpr int TM_S = 0, TM_P = 256, TM_ACC = DKV ? 256 : 384;
   static constexpr int OFF_A = 0, OFF_B = TILE_BYTES, OFF_RING = 2 * TILE_BYTES;
   static constexpr int OFF_ROWV = OFF_RING + RING * TILE_BYTES;  // dK/dV: per warp 128 lse2 + 128 delta
   static constexpr int OFF_BAR = OFF_ROWV + (DKV ? 8 * 2 * 128 * 4 : 0);
-  // dQ:   SFULL[s] S of the slot computed, DPFULL dP computed, DPREAD dP read by the
-  //       warpgroups, DSREADY[s] dS written, SFREE[s] dQ MMA of the slot completed.
-  // dK/dV: SFULL S^T computed, DPFULL dP^T computed, PREADY P^T written, DSREADY dS^T
-  //       written, SFREE the dV MMA (reader of P^T) completed, DPFREE the dK MMA completed.
+  // dQ:    SFULL[s] S of slot s computed, DPFULL[0] dP computed, READ[0] dP read by the
+  //        warpgroups, DSREADY[s] dS written, SFREE[s] the dQ MMA of slot s completed.
+  // dK/dV: SFULL[s] S^T of slot s computed, READ[s] S^T read by the warpgroups, DPFULL[s]
+  //        dP^T computed (over S^T), DSREADY[s] P^T and dS^T written (over dP^T), SFREE[s]
+  //        the dV and dK MMAs of slot s completed.
   static constexpr int B_AFULL = 0, B_AEMPTY = 1, B_RFULL = 2, B_REMPTY = B_RFULL + RING,
-                       B_SFULL = B_REMPTY + RING, B_DPFULL = B_SFULL + NS, B_DPREAD = B_DPFULL + 1,
-                       B_PREADY = B_DPREAD + 1, B_DSREADY = B_PREADY + 1, B_SFREE = B_DSREADY + NS,
-                       B_DPFREE = B_SFREE + NS, B_ACCFULL = B_DPFREE + 1, B_ACCEMPTY = B_ACCFULL + 1,
-                       B_DRAIN = B_ACCEMPTY + 1, B_DRAIN2 = B_DRAIN + 1, B_DRAIN3 = B_DRAIN2 + 1,
-                       NBAR = B_DRAIN3 + 1;
+                       B_SFULL = B_REMPTY + RING, B_DPFULL = B_SFULL + NS, B_READ = B_DPFULL + NS,
+                       B_DSREADY = B_READ + NS, B_SFREE = B_DSREADY + NS, B_ACCFULL = B_SFREE + NS,
+                       B_ACCEMPTY = B_ACCFULL + 1, B_DRAIN = B_ACCEMPTY + 1, B_DRAIN2 = B_DRAIN + 1,
+                       B_DRAIN3 = B_DRAIN2 + 1, NBAR = B_DRAIN3 + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;       // [0] TMEM base, [1] abort flag
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;   // + slack to align the base to 1 KiB
   static constexpr int THREADS = 384;
@@ -234,7 +237,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd_dq_kernel(const
       mbar_init(BAR(C::B_SFREE + b), 1);
     }
     mbar_init(BAR(C::B_DPFULL), 1);
-    mbar_init(BAR(C::B_DPREAD), C::EW);
+    mbar_init(BAR(C::B_READ), C::EW);
     mbar_init(BAR(C::B_ACCFULL), 1);
     mbar_init(BAR(C::B_ACCEMPTY), C::EW);
     mbar_init(BAR(C::B_DRAIN), 1);
@@ -340,7 +343,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd_dq_kernel(const
         if (!wait_bounded(BAR(C::B_AFULL), n & 1, guard, kBwdWaitAFull)) break;
         for (int j = 0; ok && j < it.job_count; ++j, ++g) {
           const uint32_t vs = vslot(g);
-          ok = wait_bounded(BAR(C::B_DPREAD), (g & 1) ^ 1, guard, kBwdWaitDpRead) &&
+          ok = wait_bounded(BAR(C::B_READ), (g & 1) ^ 1, guard, kBwdWaitDpRead) &&
                wait_bounded(BAR(C::B_RFULL + vs), (g / C::VST) & 1, guard, kBwdWaitRFull);
           if (!ok) break;
           tc_fence_after();
@@ -424,7 +427,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd_dq_kernel(const
         tmem_ld32x32(ts, sv);
         tmem_wait_ld();
         tc_fence_before();
-        mbar_arrive(BAR(C::B_DPREAD));
+        mbar_arrive(BAR(C::B_READ));
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
           if (c == 1) {
@@ -501,12 +504,13 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd_dkv_kernel(cons
       mbar_init(BAR(C::B_RFULL + s), 1);
       mbar_init(BAR(C::B_REMPTY + s), 1);
     }
-    mbar_init(BAR(C::B_SFULL), 1);
-    mbar_init(BAR(C::B_DPFULL), 1);
-    mbar_init(BAR(C::B_PREADY), C::EW);
-    mbar_init(BAR(C::B_DSREADY), C::EW);
-    mbar_init(BAR(C::B_SFREE), 1);
-    mbar_init(BAR(C::B_DPFREE), 1);
+    for (int b = 0; b < C::NS; ++b) {
+      mbar_init(BAR(C::B_SFULL + b), 1);
+      mbar_init(BAR(C::B_DPFULL + b), 1);
+      mbar_init(BAR(C::B_READ + b), C::EW);
+      mbar_init(BAR(C::B_DSREADY + b), C::EW);
+      mbar_init(BAR(C::B_SFREE + b), 1);
+    }
     mbar_init(BAR(C::B_ACCFULL), 1);
     mbar_init(BAR(C::B_ACCEMPTY), C::EW);
     mbar_init(BAR(C::B_DRAIN), 1);
@@ -570,8 +574,8 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd_dkv_kernel(cons
     }
     __syncwarp();
   } else if (warp == 1) {
-    // ---- S^T issuer. Job g: S^T = K Q^T once the dV MMA of job g - 1 (the reader of P^T,
-    // written over S^T) has completed
+    // ---- S^T issuer. Job g runs in TMEM slot g % 2: S^T = K Q^T once the dV and dK MMAs
+    // of job g - 2 have completed
     if (lane == 0) {
       uint32_t rc = 0, g = 0;
       int n = 0;
@@ -580,13 +584,13 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd_dkv_kernel(cons
         const BwdItem it = p.items[p.cta_items[ii]];
         if (!wait_bounded(BAR(C::B_AFULL), n & 1, guard, kBwdWaitAFull)) break;
         for (int j = 0; ok && j < it.job_count; ++j, ++g, rc += 2) {
-          const uint32_t rq = rc;
-          ok = wait_bounded(BAR(C::B_SFREE), (g & 1) ^ 1, guard, kBwdWaitSFree) &&
+          const uint32_t s = g & 1, rq = rc;
+          ok = wait_bounded(BAR(C::B_SFREE + s), ((g >> 1) & 1) ^ 1, guard, kBwdWaitSFree) &&
                wait_bounded(BAR(C::B_RFULL + rq % C::STAGES), (rq / C::STAGES) & 1, guard, kBwdWaitRFull);
           if (!ok) break;
           tc_fence_after();
-          mma_tile_ss<C::D>(tmem + C::TM_S, sbase + C::OFF_A, ring(rq), C::IDESC_SS);   // S^T = K Q^T
-          mma_commit(BAR(C::B_SFULL));
+          mma_tile_ss<C::D>(tmem + C::TM_S + 128 * s, sbase + C::OFF_A, ring(rq), C::IDESC_SS);   // S^T = K Q^T
+          mma_commit(BAR(C::B_SFULL + s));
         }
         if (!ok) break;
         mma_commit(BAR(C::B_AEMPTY));   // K is read by these MMAs only
@@ -596,8 +600,8 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd_dkv_kernel(cons
     }
     __syncwarp();
   } else if (warp == 3) {
-    // ---- dP^T issuer: dP^T = V dO^T of job g once the dK MMA of job g - 1 (the reader of
-    // dS^T, written over dP^T) has completed
+    // ---- dP^T issuer: dP^T = V dO^T of job g over S^T in slot g % 2 once the warpgroups have
+    // read S^T
     if (lane == 0) {
       uint32_t rc = 0, g = 0;
       int n = 0;
@@ -606,13 +610,13 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd_dkv_kernel(cons
         const BwdItem it = p.items[p.cta_items[ii]];
         if (!wait_bounded(BAR(C::B_AFULL), n & 1, guard, kBwdWaitAFull)) break;
         for (int j = 0; ok && j < it.job_count; ++j, ++g, rc += 2) {
-          const uint32_t rd = rc + 1;
-          ok = wait_bounded(BAR(C::B_DPFREE), (g & 1) ^ 1, guard, kBwdWaitDpFree) &&
+          const uint32_t s = g & 1, rd = rc + 1;
+          ok = wait_bounded(BAR(C::B_READ + s), (g >> 1) & 1, guard, kBwdWaitDpRead) &&
                wait_bounded(BAR(C::B_RFULL + rd % C::STAGES), (rd / C::STAGES) & 1, guard, kBwdWaitRFull);
           if (!ok) break;
           tc_fence_after();
-          mma_tile_ss<C::D>(tmem + C::TM_P, sbase + C::OFF_B, ring(rd), C::IDESC_SS);   // dP^T = V dO^T
-          mma_commit(BAR(C::B_DPFULL));
+          mma_tile_ss<C::D>(tmem + C::TM_S + 128 * s, sbase + C::OFF_B, ring(rd), C::IDESC_SS);   // dP^T = V dO^T
+          mma_commit(BAR(C::B_DPFULL + s));
         }
         if (!ok) break;
         mma_commit(BAR(C::B_AEMPTY));   // V is read by these MMAs only
@@ -622,8 +626,8 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd_dkv_kernel(cons
     }
     __syncwarp();
   } else if (warp == 2) {
-    // ---- dV / dK issuer: dV += P^T dO once P^T is in TMEM (frees S^T and the dO tile on
-    // completion), dK += dS^T Q once dS^T is (frees dP^T and the Q tile)
+    // ---- dV / dK issuer: dV += P^T dO and dK += dS^T Q once the warpgroups have written P^T
+    // and dS^T into the job's slot; frees the slot and the job's Q and dO tiles on completion
     if (lane == 0) {
       uint32_t rc = 0, g = 0;
       int n = 0;
@@ -631,27 +635,17 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd_dkv_kernel(cons
       for (int ii = i_begin; ok && ii < i_end; ++ii, ++n) {
         const BwdItem it = p.items[p.cta_items[ii]];
         for (int j = 0; ok && j < it.job_count; ++j, ++g, rc += 2) {
-          const uint32_t rq = rc, rd = rc + 1, acc = j > 0 ? 1u : 0u;
-          ok = wait_bounded(BAR(C::B_PREADY), g & 1, guard, kBwdWaitPFull);
+          const uint32_t s = g & 1, rq = rc, rd = rc + 1, acc = j > 0 ? 1u : 0u;
+          ok = wait_bounded(BAR(C::B_DSREADY + s), (g >> 1) & 1, guard, kBwdWaitDsReady);
           if (ok && j == 0) ok = wait_bounded(BAR(C::B_ACCEMPTY), (n & 1) ^ 1, guard, kBwdWaitAccEmpty);
           if (!ok) break;
           tc_fence_after();
-          mma_tile_ts(tmem + C::TM_ACC, tmem + C::TM_S, ring(rd), C::IDESC_TS, acc);   // dV += P^T dO
-          mma_commit(BAR(C::B_SFREE));
-          // dO: read by this dV MMA and the job's dP^T MMA; the tile is free once both completed
-          if (!wait_bounded(BAR(C::B_DPFULL), g & 1, guard, kBwdWaitDpFull)) {
-            ok = false;
-            break;
-          }
-          mma_commit(BAR(C::B_REMPTY + rd % C::STAGES));
-          if (!wait_bounded(BAR(C::B_DSREADY), g & 1, guard, kBwdWaitDsReady)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          mma_tile_ts(tmem + C::TM_ACC + C::D, tmem + C::TM_P, ring(rq), C::IDESC_TS, acc);   // dK += dS^T Q
-          mma_commit(BAR(C::B_DPFREE));
-          mma_commit(BAR(C::B_REMPTY + rq % C::STAGES));   // Q: read by S^T and this MMA
+          const uint32_t slot = tmem + C::TM_S + 128 * s;
+          mma_tile_ts(tmem + C::TM_ACC, slot, ring(rd), C::IDESC_TS, acc);               // dV += P^T dO
+          mma_tile_ts(tmem + C::TM_ACC + C::D, slot + 32, ring(rq), C::IDESC_TS, acc);   // dK += dS^T Q
+          mma_commit(BAR(C::B_SFREE + s));
+          mma_commit(BAR(C::B_REMPTY + rq % C::STAGES));   // Q: read by S^T and dK
+          mma_commit(BAR(C::B_REMPTY + rd % C::STAGES));   // dO: read by dP^T and dV
         }
         if (!ok) break;
         mma_commit(BAR(C::B_ACCFULL));
@@ -714,60 +708,60 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd_dkv_kernel(cons
         bits_next = row_bits(p.mask_tiles, jb_next.mask, r);
         jb_next = j + 2 < nj ? p.jobs[it.job_start + j + 2] : none;
 
-        if (!__all_sync(0xffffffffu, wait_bounded(BAR(C::B_SFULL), g & 1, guard, kBwdWaitSFull))) {
+        // S^T of query rows 64 w .. 64 w + 63 into registers; then dP^T may overwrite it
+        const uint32_t s = g & 1;
+        if (!__all_sync(0xffffffffu, wait_bounded(BAR(C::B_SFULL + s), (g >> 1) & 1, guard, kBwdWaitSFull))) {
           ok = false;
           break;
         }
         tc_fence_after();
-        // P^T for query rows 64 w .. 64 w + 63: kept in registers for dS^T, written (bf16
-        // pairs) over S^T columns 64 w .. 64 w + 31
-        const uint32_t ts = tmem + lane_base + C::TM_S + 64 * w;
+        const uint32_t ts = tmem + lane_base + C::TM_S + 128 * s + 64 * w;
         float pr[64];
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          uint32_t sv[32];
-          tmem_ld32x32(ts + 32 * c, sv);
+        {
+          uint32_t sv[64];
+          tmem_ld32x32(ts, sv);
+          tmem_ld32x32(ts + 32, sv + 32);
           tmem_wait_ld();
-          const uint32_t wb = w ? (c ? bits.w : bits.z) : (c ? bits.y : bits.x);
-          const float4* l2v = reinterpret_cast<const float4*>(rl2 + 64 * w + 32 * c);
-          if (wb == 0xffffffffu) {
+          tc_fence_before();
+          mbar_arrive(BAR(C::B_READ + s));
 #pragma unroll
-            for (int f = 0; f < 8; ++f) {
-              const float4 la = l2v[f];
-              pr[32 * c + 4 * f + 0] = ex2(fmaf(__uint_as_float(sv[4 * f + 0]), sl2, -la.x));
-              pr[32 * c + 4 * f + 1] = ex2(fmaf(__uint_as_float(sv[4 * f + 1]), sl2, -la.y));
-              pr[32 * c + 4 * f + 2] = ex2(fmaf(__uint_as_float(sv[4 * f + 2]), sl2, -la.z));
-              pr[32 * c + 4 * f + 3] = ex2(fmaf(__uint_as_float(sv[4 * f + 3]), sl2, -la.w));
-            }
-          } else {
+          for (int c = 0; c < 2; ++c) {
+            const uint32_t wb = w ? (c ? bits.w : bits.z) : (c ? bits.y : bits.x);
+            const float4* l2v = reinterpret_cast<const float4*>(rl2 + 64 * w + 32 * c);
+            if (wb == 0xffffffffu) {
 #pragma unroll
-            for (int f = 0; f < 8; ++f) {
-              const float4 la = l2v[f];
-              const float lq[4] = {la.x, la.y, la.z, la.w};
+              for (int f = 0; f < 8; ++f) {
+                const float4 la = l2v[f];
+                pr[32 * c + 4 * f + 0] = ex2(fmaf(__uint_as_float(sv[32 * c + 4 * f + 0]), sl2, -la.x));
+                pr[32 * c + 4 * f + 1] = ex2(fmaf(__uint_as_float(sv[32 * c + 4 * f + 1]), sl2, -la.y));
+                pr[32 * c + 4 * f + 2] = ex2(fmaf(__uint_as_float(sv[32 * c + 4 * f + 2]), sl2, -la.z));
+                pr[32 * c + 4 * f + 3] = ex2(fmaf(__uint_as_float(sv[32 * c + 4 * f + 3]), sl2, -la.w));
+              }
+            } else {
 #pragma unroll
-              for (int q = 0; q < 4; ++q)
-                pr[32 * c + 4 * f + q] = ((wb >> (4 * f + q)) & 1u)
-                                             ? ex2(fmaf(__uint_as_float(sv[4 * f + q]), sl2, -lq[q]))
-                                             : 0.f;
+              for (int f = 0; f < 8; ++f) {
+                const float4 la = l2v[f];
+                const float lq[4] = {la.x, la.y, la.z, la.w};
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                  pr[32 * c + 4 * f + q] = ((wb >> (4 * f + q)) & 1u)
+                                               ? ex2(fmaf(__uint_as_float(sv[32 * c + 4 * f + q]), sl2, -lq[q]))
+                                               : 0.f;
+              }
             }
           }
-          uint32_t pk[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e) pk[e] = pack_bf16(pr[32 * c + 2 * e], pr[32 * c + 2 * e + 1]);
-          tmem_st32x16(ts + 16 * c, pk);
         }
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(BAR(C::B_PREADY));
-        // dS^T = P^T (dP^T - delta) over dP^T columns 64 w .. 64 w + 31
-        if (!__all_sync(0xffffffffu, wait_bounded(BAR(C::B_DPFULL), g & 1, guard, kBwdWaitDpFull))) {
+        // dS^T = P^T (dP^T - delta). This warpgroup's dP^T columns 64 w .. 64 w + 63 then take
+        // P^T (bf16 pairs, columns 64 w .. 64 w + 31) and dS^T (64 w + 32 .. 64 w + 63); the
+        // second half is read first, so every write lands on columns already read.
+        if (!__all_sync(0xffffffffu, wait_bounded(BAR(C::B_DPFULL + s), (g >> 1) & 1, guard, kBwdWaitDpFull))) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t tp = tmem + lane_base + C::TM_P + 64 * w;
+        const uint32_t tp = ts;
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
+        for (int c = 1; c >= 0; --c) {
           uint32_t dv[32];
           tmem_ld32x32(tp + 32 * c, dv);
           tmem_wait_ld();
@@ -782,11 +776,18 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd_dkv_kernel(cons
             pk[2 * f + 1] = pack_bf16(pp[2] * (__uint_as_float(dv[4 * f + 2]) - da.z),
                                       pp[3] * (__uint_as_float(dv[4 * f + 3]) - da.w));
           }
+          tmem_st32x16(tp + 32 + 16 * c, pk);
+        }
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) pk[e] = pack_bf16(pr[32 * c + 2 * e], pr[32 * c + 2 * e + 1]);
           tmem_st32x16(tp + 16 * c, pk);
         }
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(BAR(C::B_DSREADY));
+        mbar_arrive(BAR(C::B_DSREADY + s));
       }
       if (!ok) break;
       if (!__all_sync(0xffffffffu, wait_bounded(BAR(C::B_ACCFULL), n & 1, guard, kBwdWaitAccFull))) break;
