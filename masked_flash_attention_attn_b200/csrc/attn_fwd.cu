@@ -428,58 +428,68 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_fwd_kernel(const __
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::REG_LOW));
   if (warp == 0) {
     // ================================ TMA producer ================================
-    if (lane == 0) {
+    // The whole warp runs the loop: lane 0 issues the Q copies and the contiguous K / V
+    // boxes; with a paged cache lane i issues the boxes of the chunk's page i (one TMA issue
+    // stream per page: a single thread issuing many small boxes is limited by its own issue
+    // rate). Waits are taken by every lane and agreed with a vote.
+    {
       uint32_t rc = 0;
       int n = 0, q_last = -1;
       for (int ii = i_begin; ii < i_end; ++ii, ++n) {
         const WorkItem it = p.items[p.cta_items[ii]];
         if constexpr (C::PAGED) {
-          prefetch_l1(p.page_table + it.k_base);
-          if (ii + 1 < i_end) prefetch_l1(p.page_table + p.items[p.cta_items[ii + 1]].k_base);
+          if (lane == 0) {
+            prefetch_l1(p.page_table + it.k_base);
+            if (ii + 1 < i_end) prefetch_l1(p.page_table + p.items[p.cta_items[ii + 1]].k_base);
+          }
         }
-        if (!wait_bounded(BAR(C::B_QEMPTY), (n & 1) ^ 1, guard, kWaitQEmpty)) break;
+        if (!__all_sync(0xffffffffu, wait_bounded(BAR(C::B_QEMPTY), (n & 1) ^ 1, guard, kWaitQEmpty))) break;
         if (!((p.debug_flags & 1) && n == 0)) {
-          mbar_expect_tx(BAR(C::B_QFULL), 2 * C::Q_BYTES);
           q_last = n;
-          for (int t = 0; t < 2; ++t)
-            for (int hh = 0; hh < p.hp; ++hh)
-              for (int c = 0; c < C::NBOX; ++c)
-                tma_load_3d(sbase + C::OFF_Q + t * C::Q_BYTES + c * C::BOX_BYTES + hh * p.R * 128, &p.tm_q,
-                            c * (C::FP8 ? 128 : 64), it.head[t] + hh, it.tok[t], BAR(C::B_QFULL));
+          if (lane == 0) {
+            mbar_expect_tx(BAR(C::B_QFULL), 2 * C::Q_BYTES);
+            for (int t = 0; t < 2; ++t)
+              for (int hh = 0; hh < p.hp; ++hh)
+                for (int c = 0; c < C::NBOX; ++c)
+                  tma_load_3d(sbase + C::OFF_Q + t * C::Q_BYTES + c * C::BOX_BYTES + hh * p.R * 128, &p.tm_q,
+                              c * (C::FP8 ? 128 : 64), it.head[t] + hh, it.tok[t], BAR(C::B_QFULL));
+          }
         }
         auto load_tile = [&](bool is_v, int j) -> bool {
           const int kt = p.jobs[it.job_start + j].k_tile;
           const CUtensorMap* tm = is_v ? &p.tm_v : &p.tm_k;
           const uint32_t slot = rc % C::STAGES;
-          if (!wait_bounded(BAR(C::B_KVEMPTY + slot), ((rc / C::STAGES) & 1) ^ 1, guard, kWaitKvEmpty)) return false;
-          mbar_expect_tx(BAR(C::B_KVFULL + slot), C::CHUNK_BYTES);
+          if (!__all_sync(0xffffffffu, wait_bounded(BAR(C::B_KVEMPTY + slot), ((rc / C::STAGES) & 1) ^ 1, guard,
+                                                    kWaitKvEmpty)))
+            return false;
           const uint32_t dst = sbase + C::OFF_RING + slot * C::CHUNK_BYTES;
+          if (lane == 0) mbar_expect_tx(BAR(C::B_KVFULL + slot), C::CHUNK_BYTES);
           if constexpr (C::FP8) {
             // K: 128 keys x 128 bytes; V^T ([Hkv][d][keys]): d = 128 rows x 128 keys
-            if (is_v) tma_load_3d(dst, tm, it.vt_base + kt * 128, 0, it.kv_head, BAR(C::B_KVFULL + slot));
-            else tma_load_3d(dst, tm, 0, it.kv_head, it.k_base + kt * 128, BAR(C::B_KVFULL + slot));
+            if (lane == 0) {
+              if (is_v) tma_load_3d(dst, tm, it.vt_base + kt * 128, 0, it.kv_head, BAR(C::B_KVFULL + slot));
+              else tma_load_3d(dst, tm, 0, it.kv_head, it.k_base + kt * 128, BAR(C::B_KVFULL + slot));
+            }
           } else if constexpr (!C::PAGED) {
-            for (int c = 0; c < C::NBOX; ++c)
-              tma_load_3d(dst + c * C::BOX_BYTES, tm, c * 64, it.kv_head, it.k_base + kt * 128, BAR(C::B_KVFULL + slot));
+            if (lane == 0)
+              for (int c = 0; c < C::NBOX; ++c)
+                tma_load_3d(dst + c * C::BOX_BYTES, tm, c * 64, it.kv_head, it.k_base + kt * 128,
+                            BAR(C::B_KVFULL + slot));
           } else {
             const int ps = p.page_size, ppt = 128 / ps;
-            if (!is_v) {
+            if (lane == 0 && !is_v) {
               const int ahead = (kt + 2) * ppt;
               if (ahead < it.npages) prefetch_l1(p.page_table + it.k_base + ahead);
             }
-            int32_t page[8];
-#pragma unroll
-            for (int pg = 0; pg < 8; ++pg) {
-              const int idx = kt * ppt + pg;
-              page[pg] = (pg < ppt && idx < it.npages) ? __ldg(p.page_table + it.k_base + idx) : -1;
-            }
-#pragma unroll
-            for (int pg = 0; pg < 8; ++pg) {
-              if (pg >= ppt) break;
+            __syncwarp();   // the expected byte count is posted before any of the chunk's copies
+            if (lane < ppt) {
+              const int idx = kt * ppt + lane;
+              const int32_t page = idx < it.npages ? __ldg(p.page_table + it.k_base + idx) : -1;
               int32_t row = p.num_pages * ps;  // fully out of bounds: the box reads zeros
-              if (page[pg] >= 0 && page[pg] < p.num_pages) row = page[pg] * ps;
+              if (page >= 0 && page < p.num_pages) row = page * ps;
               for (int c = 0; c < C::NBOX; ++c)
-                tma_load_3d(dst + c * C::BOX_BYTES + pg * ps * 128, tm, c * 64, it.kv_head, row, BAR(C::B_KVFULL + slot));
+                tma_load_3d(dst + c * C::BOX_BYTES + lane * ps * 128, tm, c * 64, it.kv_head, row,
+                            BAR(C::B_KVFULL + slot));
             }
           }
           ++rc;
@@ -494,9 +504,11 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_fwd_kernel(const __
         if (ok) ok = load_tile(true, J - 1);
         if (!ok) break;
       }
-      for (uint32_t r = rc > uint32_t(C::STAGES) ? rc - C::STAGES : 0u; r < rc; ++r)
-        wait_drain(BAR(C::B_KVFULL + r % C::STAGES), (r / C::STAGES) & 1, p.timeout_ns);
-      if (q_last >= 0) wait_drain(BAR(C::B_QFULL), q_last & 1, p.timeout_ns);
+      if (lane == 0) {
+        for (uint32_t r = rc > uint32_t(C::STAGES) ? rc - C::STAGES : 0u; r < rc; ++r)
+          wait_drain(BAR(C::B_KVFULL + r % C::STAGES), (r / C::STAGES) & 1, p.timeout_ns);
+        if (q_last >= 0) wait_drain(BAR(C::B_QFULL), q_last & 1, p.timeout_ns);
+      }
     }
     __syncwarp();
   } else if (warp == 1) {
