@@ -429,9 +429,9 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_fwd_kernel(const __
   if (warp == 0) {
     // ================================ TMA producer ================================
     // The whole warp runs the loop: lane 0 issues the Q copies and the contiguous K / V
-    // boxes; with a paged cache lane i issues the boxes of the chunk's page i (one TMA issue
-    // stream per page: a single thread issuing many small boxes is limited by its own issue
-    // rate). Waits are taken by every lane and agreed with a vote.
+    // boxes; with a paged cache lane i issues the boxes of the chunk's page i (a single thread
+    // issuing many small boxes is limited by its own issue rate; one lane per page measured
+    // faster than one lane per box). Waits are taken by every lane and agreed with a vote.
     {
       uint32_t rc = 0;
       int n = 0, q_last = -1;
@@ -482,7 +482,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_fwd_kernel(const __
               if (ahead < it.npages) prefetch_l1(p.page_table + it.k_base + ahead);
             }
             __syncwarp();   // the expected byte count is posted before any of the chunk's copies
-            if (lane < ppt) {
+            if (lane < ppt) {   // lane = page of the chunk
               const int idx = kt * ppt + lane;
               const int32_t page = idx < it.npages ? __ldg(p.page_table + it.k_base + idx) : -1;
               int32_t row = p.num_pages * ps;  // fully out of bounds: the box reads zeros
@@ -789,27 +789,34 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::THREADS, 1)
 
   if (warp == 0) {
     // ================================ TMA producer (both CTAs) ================================
-    if (lane == 0) {
+    // The whole warp runs the loop (waits agreed with a vote); lane 0 issues the Q copies
+    // and the contiguous K / V boxes, and with a paged cache every box of a half-chunk (page,
+    // 64-column block) has its own lane: one thread's TMA issue rate bounds many small boxes.
+    {
       const uint64_t pol_kv = l2_policy_evict_last(), pol_q = l2_policy_evict_first();
       uint32_t rc = 0;
       int n = 0, q_last = -1;
       for (int ii = i_begin; ii < i_end; ++ii, ++n) {
         const WorkItem it = p.items[p.cta_items[ii]];
-        if (!wait_bounded(BAR(C::B_QEMPTY), (n & 1) ^ 1, guard, kWaitQEmpty)) break;
+        if (!__all_sync(0xffffffffu, wait_bounded(BAR(C::B_QEMPTY), (n & 1) ^ 1, guard, kWaitQEmpty))) break;
         if (!((p.debug_flags & 1) && n == 0)) {
-          if (leader) mbar_expect_tx(BAR(C::B_QFULL), 2 * C::Q_BYTES);
           q_last = n;
-          for (int hh = 0; hh < p.hp; ++hh)
-            for (int c = 0; c < C::QBOX; ++c)
-              tma2_load_3d_hint(sbase + C::OFF_Q + c * 16384 + hh * p.R * 128, &p.tm_q, c * C::BOX_COLS,
-                                it.head[rank] + hh, it.tok[rank], LBAR(C::B_QFULL), pol_q);
+          if (lane == 0) {
+            if (leader) mbar_expect_tx(BAR(C::B_QFULL), 2 * C::Q_BYTES);
+            for (int hh = 0; hh < p.hp; ++hh)
+              for (int c = 0; c < C::QBOX; ++c)
+                tma2_load_3d_hint(sbase + C::OFF_Q + c * 16384 + hh * p.R * 128, &p.tm_q, c * C::BOX_COLS,
+                                  it.head[rank] + hh, it.tok[rank], LBAR(C::B_QFULL), pol_q);
+          }
         }
         const int T = it.job_count;
         auto load_half = [&](bool is_v, int j) -> bool {
           const int kt = p.jobs[it.job_start + j].k_tile;
           const uint32_t slot = rc % C::STAGES;
-          if (!wait_bounded(BAR(C::B_KVEMPTY + slot), ((rc / C::STAGES) & 1) ^ 1, guard, kWaitKvEmpty)) return false;
-          if (leader) mbar_expect_tx(BAR(C::B_KVFULL + slot), 2 * C::SLOT_BYTES);
+          if (!__all_sync(0xffffffffu, wait_bounded(BAR(C::B_KVEMPTY + slot), ((rc / C::STAGES) & 1) ^ 1, guard,
+                                                    kWaitKvEmpty)))
+            return false;
+          if (leader && lane == 0) mbar_expect_tx(BAR(C::B_KVFULL + slot), 2 * C::SLOT_BYTES);
           const uint32_t dst = sbase + C::OFF_RING + slot * C::SLOT_BYTES;
           const uint32_t fb = LBAR(C::B_KVFULL + slot);
           // K half: keys kt*128 + 64 rank .. +63, all D columns; V half: all 128 keys,
@@ -822,37 +829,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::THREADS, 1)
           const CUtensorMap* tm = is_v ? &p.tm_v : &p.tm_k;
           if constexpr (C::FP8) {
             // K half: 64 keys x two 128-byte boxes; V^T half: d / 2 rows x 128 keys
-            if (is_v)
+            if (lane != 0) {
+            } else if (is_v)
               tma2_load_3d_hint(dst, tm, it.vt_base + kt * 128, int(rank) * (C::D / 2), it.kv_head, fb, pol_kv);
             else
               for (int c = 0; c < nbox; ++c)
                 tma2_load_3d_hint(dst + c * box_bytes, tm, c * C::BOX_COLS, it.kv_head, it.k_base + key0, fb, pol_kv);
           } else if constexpr (!C::PAGED) {
-            for (int c = 0; c < nbox; ++c)
-              tma2_load_3d_hint(dst + c * box_bytes, tm, col0 + c * C::BOX_COLS, it.kv_head, it.k_base + key0, fb,
-                                pol_kv);
+            if (lane == 0)
+              for (int c = 0; c < nbox; ++c)
+                tma2_load_3d_hint(dst + c * box_bytes, tm, col0 + c * C::BOX_COLS, it.kv_head, it.k_base + key0, fb,
+                                  pol_kv);
           } else {
             const int ps = p.page_size;
             const int rows = ps < nkeys ? ps : nkeys;  // rows per box
             const int nb = nkeys / rows;               // boxes per 64-column block
-            if (!is_v) {
+            if (!is_v && lane == 0) {
               const int ahead = ((kt + 2) * 128) / ps;   // page-table line of the key tile two ahead
               if (ahead < it.npages) prefetch_l1(p.page_table + it.k_base + ahead);
             }
-            int32_t page[8];
-#pragma unroll
-            for (int pg = 0; pg < 8; ++pg) {
-              const int idx = (key0 + pg * rows) / ps;
-              page[pg] = (pg < nb && idx < it.npages) ? __ldg(p.page_table + it.k_base + idx) : -1;
-            }
-#pragma unroll
-            for (int pg = 0; pg < 8; ++pg) {
-              if (pg >= nb) break;
+            __syncwarp();   // this CTA's expected byte count is posted before its copies
+            if (lane < nb * nbox) {   // lane = (page block of the half-chunk, 64-column box)
+              const int pg = lane / nbox, c = lane % nbox, idx = (key0 + pg * rows) / ps;
+              const int32_t page = idx < it.npages ? __ldg(p.page_table + it.k_base + idx) : -1;
               int32_t row = p.num_pages * ps;  // fully out of bounds: the box reads zeros
-              if (page[pg] >= 0 && page[pg] < p.num_pages) row = page[pg] * ps + (key0 + pg * rows) % ps;
-              for (int c = 0; c < nbox; ++c)
-                tma2_load_3d_hint(dst + c * box_bytes + pg * rows * 128, tm, col0 + c * C::BOX_COLS, it.kv_head, row,
-                                  fb, pol_kv);
+              if (page >= 0 && page < p.num_pages) row = page * ps + (key0 + pg * rows) % ps;
+              tma2_load_3d_hint(dst + c * box_bytes + pg * rows * 128, tm, col0 + c * C::BOX_COLS, it.kv_head, row, fb,
+                                pol_kv);
             }
           }
           ++rc;
@@ -867,7 +870,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::THREADS, 1)
         if (!ok) break;
       }
       // let the copies land before the CTA may exit: the leader's barriers count both CTAs' bytes
-      if (leader) {
+      if (leader && lane == 0) {
         for (uint32_t r = rc > uint32_t(C::STAGES) ? rc - C::STAGES : 0u; r < rc; ++r)
           wait_drain(BAR(C::B_KVFULL + r % C::STAGES), (r / C::STAGES) & 1, p.timeout_ns);
         if (q_last >= 0) wait_drain(BAR(C::B_QFULL), q_last & 1, p.timeout_ns);
