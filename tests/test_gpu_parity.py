@@ -39,11 +39,14 @@ def test_small_paged(kind, d):
     G.check_full(wl, wl.masks[0], f"paged {kind} d={d}")
 
 
+@pytest.mark.parametrize("d", [64, 128, 256])
 @pytest.mark.parametrize("ps", [16, 32, 64, 128])
-def test_page_sizes(ps):
-    wl = W.random_small(seed=ps, kind="CAUSAL", batch=3, hq=2, hkv=1, d=128, lmin=1, lmax=300, paged=True,
+def test_page_sizes(ps, d):
+    # every page size against every head_dim: the producer issues one lane per page (one per
+    # box in the 2-SM kernel), so the lane count changes with both
+    wl = W.random_small(seed=ps + d, kind="CAUSAL", batch=3, hq=2, hkv=1, d=d, lmin=1, lmax=300, paged=True,
                         page_size=ps)
-    G.check_full(wl, wl.masks[0], f"page size {ps}")
+    G.check_full(wl, wl.masks[0], f"page size {ps} d={d}")
 
 
 @pytest.mark.parametrize("g,lmax", [(2, 64), (4, 32), (8, 16), (4, 64)])
