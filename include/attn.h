@@ -207,8 +207,8 @@ attn_status_t attn_masked_fwd(const attn_plan_t* plan, const void* q, const void
 
 /* Plan the forward AND the backward pass (gradients of out with respect to q, k, v).
  * Same arguments and errors as attn_plan(); the plan serves attn_masked_fwd() and
- * attn_masked_bwd(). Backward support: contiguous K/V and head_dim 64 or 128, otherwise
- * UNSUPPORTED. It adds a second device workspace: the dQ and dK/dV work lists over
+ * attn_masked_bwd(). Backward support: contiguous K/V (head_dim 64, 128 or 256); a paged
+ * cache gives UNSUPPORTED. It adds a second device workspace: the dQ and dK/dV work lists over
  * 128 x 128 tiles of one head, the partial-tile masks in query-major and key-major form,
  * and an fp32 [total_q][hq] buffer for the row terms dout . out. */
 attn_status_t attn_plan_bwd(const attn_problem_t* problem, const attn_mask_desc_t* mask,

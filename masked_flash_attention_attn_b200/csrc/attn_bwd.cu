@@ -71,6 +71,7 @@ struct BwdParams {
   int32_t* status;
   int32_t hq, hkv;
   int32_t debug_flags;   // bit 0: skip the first item's per-item loads (testing the timeout path)
+  int32_t dhalf;         // head_dim 256 dK/dV pass: the half of the head dimension accumulated
   float scale, scale_log2;
   int64_t timeout_ns;
 };
@@ -808,6 +809,438 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd_dkv_kernel(cons
   if (warp == 1) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem) : "memory");
 }
 
+// ============================== head_dim 256 ==============================
+// At d = 256 neither kernel's head_dim-128 structure fits: a 128-row tile of one head is
+// 64 KiB, so two resident tiles (Q and dO, or K and V) take 128 KiB and the streamed
+// operands are brought in as 32 KiB half-tiles (128 of the 256 columns) through a ring of
+// three slots; and dV plus dK would take all 512 TMEM columns, so the dK/dV kernel runs
+// twice, once per half of the head dimension (p.dhalf), accumulating dV and dK for those
+// 128 columns and recomputing S^T and dP^T (K = 256 as two K = 128 halves) in each pass.
+// One thread issues every MMA of a job in order: dP (dP^T), S (S^T), then the accumulating
+// MMAs once the warpgroups have written dS (P^T and dS^T); the tensor pipe runs one
+// thread's MMAs in issue order, so the next job's S / dP may overwrite the slots the
+// previous job's accumulating MMAs read. TMEM: S (S^T) 0, dP (dP^T) 128, accumulators 256
+// (dQ: 256 columns; dK/dV: dV 256, dK 384).
+struct Bwd256Cfg {
+  static constexpr int D = 256;
+  static constexpr int BOX_BYTES = 128 * 128;          // 128 rows x 64 columns
+  static constexpr int TILE_BYTES = 4 * BOX_BYTES;     // resident 128 x 256 tile
+  static constexpr int HALF_BYTES = 2 * BOX_BYTES;     // streamed 128 x 128 half-tile
+  static constexpr int RSLOTS = 3;
+  static constexpr int OFF_A = 0, OFF_B = TILE_BYTES, OFF_RING = 2 * TILE_BYTES;
+  static constexpr int OFF_BAR = OFF_RING + RSLOTS * HALF_BYTES;
+  static constexpr int B_AFULL = 0, B_AEMPTY = 1, B_RFULL = 2, B_REMPTY = B_RFULL + RSLOTS,
+                       B_SFULL = B_REMPTY + RSLOTS, B_DPFULL = B_SFULL + 1, B_READY = B_DPFULL + 1,
+                       B_ACCFULL = B_READY + 1, B_ACCEMPTY = B_ACCFULL + 1, B_DRAIN = B_ACCEMPTY + 1,
+                       NBAR = B_DRAIN + 1;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;       // [0] TMEM base, [1] abort flag
+  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;   // + slack to align the base to 1 KiB
+  static constexpr int THREADS = 384;
+  static constexpr int EW = 256;
+  static constexpr int TM_S = 0, TM_P = 128, TM_ACC = 256;
+  static constexpr uint32_t IDESC_SS =  // M=128, N=128, bf16 x bf16 -> fp32, both K-major
+      (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(128 >> 3) << 17) | (uint32_t(128 >> 4) << 24);
+  static constexpr uint32_t IDESC_TS =  // M=128, N=128 (one half of the head dimension), A from TMEM
+      (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) | (uint32_t(128 >> 3) << 17) | (uint32_t(128 >> 4) << 24);
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+};
+
+// C[128 x 128] (+)= A . B^T over K = 256: A a resident tile (two 32 KiB halves), B two
+// half-tiles in ring slots b0 (columns 0..127) and b1 (128..255).
+__device__ __forceinline__ void mma_ss_k256(uint32_t d, uint32_t a_tile, uint32_t b0, uint32_t b1, uint32_t idesc) {
+  mma_ss_x8_k128(d, desc_of(desc_lo(a_tile, 16)), desc_of(desc_lo(b0, 16)), idesc, 0u);
+  mma_ss_x8_k128(d, desc_of(desc_lo(a_tile + Bwd256Cfg::HALF_BYTES, 16)), desc_of(desc_lo(b1, 16)), idesc, 1u);
+}
+
+// Producer for the d = 256 kernels: the two resident tiles once per item (tm_a, tm_b at
+// the item's rows and head), then four half-tiles per job in the order `order` names
+// (each entry: 0 / 1 = tm_c half 0 / 1, 2 / 3 = tm_d half 0 / 1) through the ring.
+template <class C>
+__device__ __forceinline__ void bwd256_produce(const BwdParams& p, uint32_t sbase, uint32_t bar0, const Guard& guard,
+                                               int i_begin, int i_end, bool dkv, const int order[4]) {
+#define BAR(i) (bar0 + 8u * uint32_t(i))
+  uint32_t rc = 0;
+  int n = 0, a_last = -1;
+  bool ok = true;
+  for (int ii = i_begin; ok && ii < i_end; ++ii, ++n) {
+    const BwdItem it = p.items[p.cta_items[ii]];
+    const int a_head = dkv ? it.kv_head : it.head;
+    if (!wait_bounded(BAR(C::B_AEMPTY), (n & 1) ^ 1, guard, kBwdWaitAEmpty)) break;
+    if (!((p.debug_flags & 1) && n == 0)) {
+      mbar_expect_tx(BAR(C::B_AFULL), 2 * C::TILE_BYTES);
+      a_last = n;
+      for (int c = 0; c < 4; ++c) {
+        tma_load_3d(sbase + C::OFF_A + c * C::BOX_BYTES, &p.tm_a, c * 64, a_head, it.tok, BAR(C::B_AFULL));
+        tma_load_3d(sbase + C::OFF_B + c * C::BOX_BYTES, &p.tm_b, c * 64, a_head, it.tok, BAR(C::B_AFULL));
+      }
+    }
+    for (int j = 0; ok && j < it.job_count; ++j) {
+      const BwdJob jb = p.jobs[it.job_start + j];
+      const int head = dkv ? jb.head : it.kv_head;
+      for (int q = 0; q < 4; ++q, ++rc) {
+        const uint32_t slot = rc % C::RSLOTS;
+        if (!wait_bounded(BAR(C::B_REMPTY + slot), ((rc / C::RSLOTS) & 1) ^ 1, guard, kBwdWaitREmpty)) {
+          ok = false;
+          break;
+        }
+        mbar_expect_tx(BAR(C::B_RFULL + slot), C::HALF_BYTES);
+        const CUtensorMap* tm = order[q] < 2 ? &p.tm_c : &p.tm_d;
+        const int col = (order[q] & 1) * 128;
+        for (int c = 0; c < 2; ++c)
+          tma_load_3d(sbase + C::OFF_RING + slot * C::HALF_BYTES + c * C::BOX_BYTES, tm, col + c * 64, head, jb.tok,
+                      BAR(C::B_RFULL + slot));
+      }
+    }
+  }
+  for (uint32_t r = rc > uint32_t(C::RSLOTS) ? rc - C::RSLOTS : 0u; r < rc; ++r)
+    wait_drain(BAR(C::B_RFULL + r % C::RSLOTS), (r / C::RSLOTS) & 1, p.timeout_ns);
+  if (a_last >= 0) wait_drain(BAR(C::B_AFULL), a_last & 1, p.timeout_ns);
+#undef BAR
+}
+
+template <class C>
+__device__ __forceinline__ void bwd256_setup(uint32_t bar0, uint32_t* misc, const BwdParams& p, int tid) {
+#define BAR(i) (bar0 + 8u * uint32_t(i))
+  if (tid == 0) {
+    mbar_init(BAR(C::B_AFULL), 1);
+    mbar_init(BAR(C::B_AEMPTY), 1);
+    for (int s = 0; s < C::RSLOTS; ++s) {
+      mbar_init(BAR(C::B_RFULL + s), 1);
+      mbar_init(BAR(C::B_REMPTY + s), 1);
+    }
+    mbar_init(BAR(C::B_SFULL), 1);
+    mbar_init(BAR(C::B_DPFULL), 1);
+    mbar_init(BAR(C::B_READY), C::EW);
+    mbar_init(BAR(C::B_ACCFULL), 1);
+    mbar_init(BAR(C::B_ACCEMPTY), C::EW);
+    mbar_init(BAR(C::B_DRAIN), 1);
+    misc[1] = 0u;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    prefetch_tmap(&p.tm_a);
+    prefetch_tmap(&p.tm_b);
+    prefetch_tmap(&p.tm_c);
+    prefetch_tmap(&p.tm_d);
+  }
+#undef BAR
+}
+
+// dQ at d = 256. Per job the ring carries V half 0, V half 1, K half 0, K half 1.
+template <class C>
+__global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd256_dq_kernel(const __grid_constant__ BwdParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t sbase = (raw + 1023u) & ~1023u;
+  uint32_t* misc = reinterpret_cast<uint32_t*>(smem_raw + (sbase - raw) + C::OFF_MISC);
+  const uint32_t bar0 = sbase + C::OFF_BAR;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const Guard guard{smem_u32(misc + 1), 0u, p.status, p.timeout_ns};
+#define BAR(i) (bar0 + 8u * uint32_t(i))
+  bwd256_setup<C>(bar0, misc, p, tid);
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(smem_u32(misc))
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = misc[0];
+  const int i_begin = p.cta_off[blockIdx.x], i_end = p.cta_off[blockIdx.x + 1];
+  auto ring = [&](uint32_t r) { return sbase + C::OFF_RING + (r % C::RSLOTS) * C::HALF_BYTES; };
+
+  if (warp == 0) {
+    // ---- TMA producer: Q and dO once per item; V halves, then K halves of every job ----
+    if (lane == 0) {
+      const int order[4] = {2, 3, 0, 1};   // tm_c = K, tm_d = V
+      bwd256_produce<C>(p, sbase, bar0, guard, i_begin, i_end, false, order);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ---- MMA issuer: dP = dO V^T, S = Q K^T, then dQ += dS K for each job ----
+    if (lane == 0) {
+      uint32_t rc = 0, g = 0;
+      int n = 0;
+      bool ok = true;
+      for (int ii = i_begin; ok && ii < i_end; ++ii, ++n) {
+        const BwdItem it = p.items[p.cta_items[ii]];
+        if (!wait_bounded(BAR(C::B_AFULL), n & 1, guard, kBwdWaitAFull)) break;
+        for (int j = 0; ok && j < it.job_count; ++j, ++g, rc += 4) {
+          const uint32_t rv0 = rc, rv1 = rc + 1, rk0 = rc + 2, rk1 = rc + 3;
+          ok = wait_bounded(BAR(C::B_RFULL + rv0 % C::RSLOTS), (rv0 / C::RSLOTS) & 1, guard, kBwdWaitRFull) &&
+               wait_bounded(BAR(C::B_RFULL + rv1 % C::RSLOTS), (rv1 / C::RSLOTS) & 1, guard, kBwdWaitRFull);
+          if (!ok) break;
+          tc_fence_after();
+          mma_ss_k256(tmem + C::TM_P, sbase + C::OFF_B, ring(rv0), ring(rv1), C::IDESC_SS);   // dP = dO V^T
+          mma_commit(BAR(C::B_DPFULL));
+          mma_commit(BAR(C::B_REMPTY + rv0 % C::RSLOTS));
+          mma_commit(BAR(C::B_REMPTY + rv1 % C::RSLOTS));
+          ok = wait_bounded(BAR(C::B_RFULL + rk0 % C::RSLOTS), (rk0 / C::RSLOTS) & 1, guard, kBwdWaitRFull) &&
+               wait_bounded(BAR(C::B_RFULL + rk1 % C::RSLOTS), (rk1 / C::RSLOTS) & 1, guard, kBwdWaitRFull);
+          if (!ok) break;
+          tc_fence_after();
+          mma_ss_k256(tmem + C::TM_S, sbase + C::OFF_A, ring(rk0), ring(rk1), C::IDESC_SS);   // S = Q K^T
+          mma_commit(BAR(C::B_SFULL));
+          ok = wait_bounded(BAR(C::B_READY), g & 1, guard, kBwdWaitDsReady);
+          if (ok && j == 0) ok = wait_bounded(BAR(C::B_ACCEMPTY), (n & 1) ^ 1, guard, kBwdWaitAccEmpty);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t acc = j > 0 ? 1u : 0u;
+          mma_tile_ts(tmem + C::TM_ACC, tmem + C::TM_S, ring(rk0), C::IDESC_TS, acc);         // dQ[:, 0:128]
+          mma_tile_ts(tmem + C::TM_ACC + 128, tmem + C::TM_S, ring(rk1), C::IDESC_TS, acc);   // dQ[:, 128:256]
+          mma_commit(BAR(C::B_REMPTY + rk0 % C::RSLOTS));
+          mma_commit(BAR(C::B_REMPTY + rk1 % C::RSLOTS));
+        }
+        if (!ok) break;
+        mma_commit(BAR(C::B_ACCFULL));
+        mma_commit(BAR(C::B_AEMPTY));
+      }
+      mma_commit(BAR(C::B_DRAIN));
+      wait_drain(BAR(C::B_DRAIN), 0, p.timeout_ns);
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ---- two elementwise warpgroups: thread r of warpgroup w owns row r of the query tile
+    // and keys 64 w .. 64 w + 63 of every job ----
+    const int r = (warp & 3) * 32 + lane, w = (warp - 4) >> 2;
+    const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
+    const float sl2 = p.scale_log2;
+    uint32_t g = 0;
+    int n = 0;
+    bool ok = true;
+    for (int ii = i_begin; ok && ii < i_end; ++ii, ++n) {
+      const BwdItem it = p.items[p.cta_items[ii]];
+      const bool valid = r < it.rows;
+      const int64_t grow = int64_t(it.tok + r) * p.hq + it.head;
+      float lse2 = INFINITY, dlt = 0.f;
+      if (valid) {
+        const float l = p.lse[grow];
+        lse2 = l == -INFINITY ? INFINITY : l * 1.4426950408889634f;
+        dlt = p.delta[grow];
+      }
+      for (int j = 0; ok && j < it.job_count; ++j, ++g) {
+        const uint4 bits4 = row_bits(p.mask_tiles, p.jobs[it.job_start + j].mask, r);
+        if (!__all_sync(0xffffffffu, wait_bounded(BAR(C::B_SFULL), g & 1, guard, kBwdWaitSFull) &&
+                                         wait_bounded(BAR(C::B_DPFULL), g & 1, guard, kBwdWaitDpFull))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t ts = tmem + lane_base + C::TM_S + 64 * w;
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          uint32_t sv[32], dv[32];
+          tmem_ld32x32(ts + 32 * c, sv);
+          tmem_ld32x32(tmem + lane_base + C::TM_P + 64 * w + 32 * c, dv);
+          tmem_wait_ld();
+          const uint32_t wb = w ? (c ? bits4.w : bits4.z) : (c ? bits4.y : bits4.x);
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            float ds[2];
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+              const float pr =
+                  ((wb >> (2 * e + q)) & 1u) ? ex2(fmaf(__uint_as_float(sv[2 * e + q]), sl2, -lse2)) : 0.f;
+              ds[q] = pr * (__uint_as_float(dv[2 * e + q]) - dlt);
+            }
+            pk[e] = pack_bf16(ds[0], ds[1]);
+          }
+          tmem_st32x16(ts + 16 * c, pk);   // over S columns this warpgroup has read
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(BAR(C::B_READY));
+      }
+      if (!ok) break;
+      if (!__all_sync(0xffffffffu, wait_bounded(BAR(C::B_ACCFULL), n & 1, guard, kBwdWaitAccFull))) break;
+      tc_fence_after();
+      store_grad_cols<128>(tmem + lane_base + C::TM_ACC + 128 * w, p.scale, valid, p.g0 + grow * C::D + 128 * w);
+      tc_fence_before();
+      mbar_arrive(BAR(C::B_ACCEMPTY));
+    }
+  }
+#undef BAR
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem) : "memory");
+}
+
+// dK / dV at d = 256 for head-dim half h = p.dhalf. Per job the ring carries Q half 1-h,
+// Q half h, dO half 1-h, dO half h: the other halves are needed for S^T and dP^T only and
+// their slots free first.
+template <class C>
+__global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd256_dkv_kernel(const __grid_constant__ BwdParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t sbase = (raw + 1023u) & ~1023u;
+  uint32_t* misc = reinterpret_cast<uint32_t*>(smem_raw + (sbase - raw) + C::OFF_MISC);
+  const uint32_t bar0 = sbase + C::OFF_BAR;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int h = p.dhalf;
+  const Guard guard{smem_u32(misc + 1), 0u, p.status, p.timeout_ns};
+#define BAR(i) (bar0 + 8u * uint32_t(i))
+  bwd256_setup<C>(bar0, misc, p, tid);
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(smem_u32(misc))
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = misc[0];
+  const int i_begin = p.cta_off[blockIdx.x], i_end = p.cta_off[blockIdx.x + 1];
+  auto ring = [&](uint32_t r) { return sbase + C::OFF_RING + (r % C::RSLOTS) * C::HALF_BYTES; };
+
+  if (warp == 0) {
+    // ---- TMA producer: K and V once per item; Q and dO halves of every job ----
+    if (lane == 0) {
+      const int order[4] = {1 - h, h, 2 + (1 - h), 2 + h};   // tm_c = Q, tm_d = dO
+      bwd256_produce<C>(p, sbase, bar0, guard, i_begin, i_end, true, order);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ---- MMA issuer: S^T = K Q^T, dP^T = V dO^T, then dV_h += P^T dO_h and dK_h += dS^T Q_h ----
+    if (lane == 0) {
+      uint32_t rc = 0, g = 0;
+      int n = 0;
+      bool ok = true;
+      for (int ii = i_begin; ok && ii < i_end; ++ii, ++n) {
+        const BwdItem it = p.items[p.cta_items[ii]];
+        if (!wait_bounded(BAR(C::B_AFULL), n & 1, guard, kBwdWaitAFull)) break;
+        for (int j = 0; ok && j < it.job_count; ++j, ++g, rc += 4) {
+          // ring positions of Q half 0 / 1 and dO half 0 / 1 (half 1-h comes first)
+          const uint32_t rq[2] = {rc + uint32_t(h == 0 ? 1 : 0), rc + uint32_t(h == 0 ? 0 : 1)};
+          const uint32_t rd[2] = {rc + 2 + uint32_t(h == 0 ? 1 : 0), rc + 2 + uint32_t(h == 0 ? 0 : 1)};
+          ok = wait_bounded(BAR(C::B_RFULL + rc % C::RSLOTS), (rc / C::RSLOTS) & 1, guard, kBwdWaitRFull) &&
+               wait_bounded(BAR(C::B_RFULL + (rc + 1) % C::RSLOTS), ((rc + 1) / C::RSLOTS) & 1, guard, kBwdWaitRFull);
+          if (!ok) break;
+          tc_fence_after();
+          mma_ss_k256(tmem + C::TM_S, sbase + C::OFF_A, ring(rq[0]), ring(rq[1]), C::IDESC_SS);   // S^T = K Q^T
+          mma_commit(BAR(C::B_SFULL));
+          mma_commit(BAR(C::B_REMPTY + rc % C::RSLOTS));   // Q half 1-h: read by S^T only
+          ok = wait_bounded(BAR(C::B_RFULL + (rc + 2) % C::RSLOTS), ((rc + 2) / C::RSLOTS) & 1, guard, kBwdWaitRFull) &&
+               wait_bounded(BAR(C::B_RFULL + (rc + 3) % C::RSLOTS), ((rc + 3) / C::RSLOTS) & 1, guard, kBwdWaitRFull);
+          if (!ok) break;
+          tc_fence_after();
+          mma_ss_k256(tmem + C::TM_P, sbase + C::OFF_B, ring(rd[0]), ring(rd[1]), C::IDESC_SS);   // dP^T = V dO^T
+          mma_commit(BAR(C::B_DPFULL));
+          mma_commit(BAR(C::B_REMPTY + (rc + 2) % C::RSLOTS));   // dO half 1-h: read by dP^T only
+          ok = wait_bounded(BAR(C::B_READY), g & 1, guard, kBwdWaitDsReady);
+          if (ok && j == 0) ok = wait_bounded(BAR(C::B_ACCEMPTY), (n & 1) ^ 1, guard, kBwdWaitAccEmpty);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t acc = j > 0 ? 1u : 0u;
+          mma_tile_ts(tmem + C::TM_ACC, tmem + C::TM_S, ring(rc + 3), C::IDESC_TS, acc);         // dV_h += P^T dO_h
+          mma_tile_ts(tmem + C::TM_ACC + 128, tmem + C::TM_P, ring(rc + 1), C::IDESC_TS, acc);   // dK_h += dS^T Q_h
+          mma_commit(BAR(C::B_REMPTY + (rc + 1) % C::RSLOTS));
+          mma_commit(BAR(C::B_REMPTY + (rc + 3) % C::RSLOTS));
+        }
+        if (!ok) break;
+        mma_commit(BAR(C::B_ACCFULL));
+        mma_commit(BAR(C::B_AEMPTY));
+      }
+      mma_commit(BAR(C::B_DRAIN));
+      wait_drain(BAR(C::B_DRAIN), 0, p.timeout_ns);
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ---- two elementwise warpgroups: thread r of warpgroup w owns key row r of the key tile
+    // and query rows 64 w .. 64 w + 63 of every job; lane i of a warp fetches the lse and
+    // delta of the chunk's query row i and the warp shares them by shuffles ----
+    const int r = (warp & 3) * 32 + lane, w = (warp - 4) >> 2;
+    const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
+    const float sl2 = p.scale_log2;
+    uint32_t g = 0;
+    int n = 0;
+    bool ok = true;
+    for (int ii = i_begin; ok && ii < i_end; ++ii, ++n) {
+      const BwdItem it = p.items[p.cta_items[ii]];
+      for (int j = 0; ok && j < it.job_count; ++j, ++g) {
+        const BwdJob jb = p.jobs[it.job_start + j];
+        const uint4 bits = row_bits(p.mask_tiles, jb.mask, r);
+        float l2c[2], dlc[2];   // this lane's query row of chunk 0 / 1
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          const int qr = 64 * w + 32 * c + lane;
+          l2c[c] = INFINITY;
+          dlc[c] = 0.f;
+          if (qr < jb.rows) {
+            const int64_t gi = int64_t(jb.tok + qr) * p.hq + jb.head;
+            const float l = p.lse[gi];
+            l2c[c] = l == -INFINITY ? INFINITY : l * 1.4426950408889634f;
+            dlc[c] = p.delta[gi];
+          }
+        }
+        if (!__all_sync(0xffffffffu, wait_bounded(BAR(C::B_SFULL), g & 1, guard, kBwdWaitSFull))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        // P^T of query rows 64 w .. 64 w + 63 (kept for dS^T), bf16 pairs over S^T columns
+        // this warpgroup has read
+        const uint32_t ts = tmem + lane_base + C::TM_S + 64 * w;
+        float pr[64];
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          uint32_t sv[32];
+          tmem_ld32x32(ts + 32 * c, sv);
+          tmem_wait_ld();
+          const uint32_t wb = w ? (c ? bits.w : bits.z) : (c ? bits.y : bits.x);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const float l2 = __shfl_sync(0xffffffffu, l2c[c], e);
+            pr[32 * c + e] = ((wb >> e) & 1u) ? ex2(fmaf(__uint_as_float(sv[e]), sl2, -l2)) : 0.f;
+          }
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) pk[e] = pack_bf16(pr[32 * c + 2 * e], pr[32 * c + 2 * e + 1]);
+          tmem_st32x16(ts + 16 * c, pk);
+        }
+        if (!__all_sync(0xffffffffu, wait_bounded(BAR(C::B_DPFULL), g & 1, guard, kBwdWaitDpFull))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t tp = tmem + lane_base + C::TM_P + 64 * w;
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          uint32_t dv[32];
+          tmem_ld32x32(tp + 32 * c, dv);
+          tmem_wait_ld();
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const float d0 = __shfl_sync(0xffffffffu, dlc[c], 2 * e), d1 = __shfl_sync(0xffffffffu, dlc[c], 2 * e + 1);
+            pk[e] = pack_bf16(pr[32 * c + 2 * e] * (__uint_as_float(dv[2 * e]) - d0),
+                              pr[32 * c + 2 * e + 1] * (__uint_as_float(dv[2 * e + 1]) - d1));
+          }
+          tmem_st32x16(tp + 16 * c, pk);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(BAR(C::B_READY));
+      }
+      if (!ok) break;
+      if (!__all_sync(0xffffffffu, wait_bounded(BAR(C::B_ACCFULL), n & 1, guard, kBwdWaitAccFull))) break;
+      tc_fence_after();
+      // warpgroup 0 stores columns 128 h .. 128 h + 127 of the row's dv, warpgroup 1 of its dk
+      const bool valid = r < it.rows;
+      const int64_t grow = int64_t(it.tok + r) * p.hkv + it.kv_head;
+      if (w == 0) store_grad_cols<128>(tmem + lane_base + C::TM_ACC, 1.f, valid, p.g1 + grow * C::D + 128 * h);
+      else store_grad_cols<128>(tmem + lane_base + C::TM_ACC + 128, p.scale, valid, p.g0 + grow * C::D + 128 * h);
+      tc_fence_before();
+      mbar_arrive(BAR(C::B_ACCEMPTY));
+    }
+  }
+#undef BAR
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem) : "memory");
+}
+
 template <class C>
 attn_status_t launch_bwd(int ctas, const BwdParams& p, cudaStream_t stream) {
   if constexpr (C::DKV) {
@@ -825,6 +1258,27 @@ attn_status_t launch_bwd(int ctas, const BwdParams& p, cudaStream_t stream) {
   }
   if constexpr (C::DKV) masked_attn_bwd_dkv_kernel<C><<<ctas, C::THREADS, C::SMEM_BYTES, stream>>>(p);
   else masked_attn_bwd_dq_kernel<C><<<ctas, C::THREADS, C::SMEM_BYTES, stream>>>(p);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+template <bool DKV>
+attn_status_t launch_bwd256(int ctas, const BwdParams& p, cudaStream_t stream) {
+  using C = Bwd256Cfg;
+  if constexpr (DKV) {
+    const cudaError_t attr = once_per_device([] {
+      return cudaFuncSetAttribute(masked_attn_bwd256_dkv_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  C::SMEM_BYTES);
+    });
+    if (attr != cudaSuccess) return ATTN_ERR_CUDA;
+    masked_attn_bwd256_dkv_kernel<C><<<ctas, C::THREADS, C::SMEM_BYTES, stream>>>(p);
+  } else {
+    const cudaError_t attr = once_per_device([] {
+      return cudaFuncSetAttribute(masked_attn_bwd256_dq_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  C::SMEM_BYTES);
+    });
+    if (attr != cudaSuccess) return ATTN_ERR_CUDA;
+    masked_attn_bwd256_dq_kernel<C><<<ctas, C::THREADS, C::SMEM_BYTES, stream>>>(p);
+  }
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
@@ -885,9 +1339,15 @@ attn_status_t mfa_launch_backward(const attn_plan_t* plan, const void* q, const 
   if (D == 64) {
     st = launch_bwd<BwdCfg<64, false>>(plan->bq_ctas, pq, stream);
     if (st == ATTN_OK) st = launch_bwd<BwdCfg<64, true>>(plan->bkv_ctas, pk, stream);
-  } else {
+  } else if (D == 128) {
     st = launch_bwd<BwdCfg<128, false>>(plan->bq_ctas, pq, stream);
     if (st == ATTN_OK) st = launch_bwd<BwdCfg<128, true>>(plan->bkv_ctas, pk, stream);
+  } else {
+    st = launch_bwd256<false>(plan->bq_ctas, pq, stream);
+    for (int h = 0; h < 2 && st == ATTN_OK; ++h) {
+      pk.dhalf = h;
+      st = launch_bwd256<true>(plan->bkv_ctas, pk, stream);
+    }
   }
   return st;
 }

@@ -976,7 +976,7 @@ void transpose_tile(const uint32_t* src, uint32_t* dst) {
 
 attn_status_t plan_backward(const attn_mask_desc_t* mask, const Shape& s, RowSource& src, int num_sms,
                             cudaStream_t stream, attn_plan_t* plan) {
-  if (s.paged || (s.d != 64 && s.d != 128)) return ATTN_ERR_UNSUPPORTED;
+  if (s.paged) return ATTN_ERR_UNSUPPORTED;
   std::vector<std::vector<int32_t>> cnts(s.B);
   if (mask->kind == ATTN_MASK_CUSTOM) {
     attn_status_t st = custom_counts(mask, s, kTile, stream, cnts);
@@ -1097,7 +1097,7 @@ attn_status_t plan_impl(const attn_problem_t* problem, const attn_mask_desc_t* m
   if (st != ATTN_OK) return st;
   st = validate_mask(mask, s);
   if (st != ATTN_OK) return st;
-  if (with_bwd && (s.paged || (s.d != 64 && s.d != 128))) return ATTN_ERR_UNSUPPORTED;
+  if (with_bwd && s.paged) return ATTN_ERR_UNSUPPORTED;
 
   int dev = 0, num_sms = 148;
   cudaError_t e = cudaGetDevice(&dev);

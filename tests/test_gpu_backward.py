@@ -1,6 +1,6 @@
 """GPU parity of the backward pass (dQ, dK, dV) through the C ABI against the fp64 oracle
 gradients (oracle/backward.py), on ragged contiguous batches of every mask kind, head dims
-64 and 128, grouped-query heads, rows that see no key and keys no query sees.
+64, 128 and 256, grouped-query heads, rows that see no key and keys no query sees.
 
 Tolerance: P and dS enter the tensor cores as bf16 (relative rounding 2^-9 each) with fp32
 accumulation, and the gradients are stored as bf16 (relative rounding 2^-9, i.e. a mean
@@ -55,7 +55,7 @@ def check_backward(wl, spec, what, seed=0, with_dlse=False):
     _close(dv, rv, f"{what} dv")
 
 
-@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("d", [64, 128, 256])
 @pytest.mark.parametrize("kind", KINDS)
 def test_backward_all_kinds(kind, d):
     wl = W.random_small(seed=500 + d + 3 * KINDS.index(kind), kind=kind, batch=3, hq=4, hkv=2, d=d,
@@ -70,10 +70,20 @@ def test_backward_with_lse_gradient(kind):
     check_backward(wl, wl.masks[0], f"bwd dlse {kind}", seed=3, with_dlse=True)
 
 
+@pytest.mark.parametrize("d", [128, 256])
 @pytest.mark.parametrize("g", [1, 4])
-def test_backward_gqa_long(g):
-    wl = W.random_small(seed=70 + g, kind="CAUSAL", batch=2, hq=2 * g, hkv=2, d=128, lmin=200, lmax=700)
-    check_backward(wl, wl.masks[0], f"bwd gqa g={g}")
+def test_backward_gqa_long(g, d):
+    # several items per CTA and several jobs per item (the head_dim 256 kernels stream
+    # their operands in half-tiles through a three-slot ring and run dK / dV in two passes)
+    wl = W.random_small(seed=70 + g + d, kind="CAUSAL", batch=2, hq=2 * g, hkv=2, d=d, lmin=200, lmax=700)
+    check_backward(wl, wl.masks[0], f"bwd gqa g={g} d={d}")
+
+
+def test_backward_gemma2_shape_sliding_window():
+    # the Gemma2 workload's shape at reduced length: head_dim 256, 2 query heads per KV head,
+    # a sliding window narrower than the sequences
+    wl = W.random_small(seed=77, kind="SLIDING_WINDOW", batch=2, hq=4, hkv=2, d=256, lmin=300, lmax=900)
+    check_backward(wl, wl.masks[0], "bwd d=256 sliding window")
 
 
 def test_backward_rows_without_keys_and_unseen_keys():
@@ -108,10 +118,12 @@ def test_backward_plan_required_and_unsupported():
     with pytest.raises(G.M.AttnError) as e:
         G.M.backward(plan, q, k, v, out, lse, torch.zeros_like(out))
     assert e.value.status == 1
-    wl = W.random_small(seed=3, kind="CAUSAL", batch=2, hq=2, hkv=1, d=256, lmin=10, lmax=50)
+    # no backward over a paged cache
+    wl = W.random_small(seed=3, kind="CAUSAL", batch=2, hq=2, hkv=1, d=128, lmin=10, lmax=50, paged=True)
     with pytest.raises(G.M.AttnError) as e:
-        G.M.attn_plan(hq=2, hkv=1, head_dim=256, cu_seqlens_q=wl.cu_seqlens_q, cu_seqlens_k=wl.cu_seqlens_k,
-                      mask=wl.masks[0], backward=True)
+        G.M.attn_plan(hq=2, hkv=1, head_dim=128, cu_seqlens_q=wl.cu_seqlens_q, kv_lens=wl.kv_lens,
+                      page_table=torch.from_numpy(wl.page_table).cuda(), page_size=wl.page_size,
+                      num_pages=wl.k_cache.shape[0], mask=wl.masks[0], backward=True)
     assert e.value.status == 2
 
 
@@ -149,11 +161,12 @@ def test_backward_full_size_chunk_causal_sampled():
     _close(got_v, rv, "full-size dv")
 
 
-def test_backward_timeout_reports_and_context_survives():
+@pytest.mark.parametrize("d", [128, 256])
+def test_backward_timeout_reports_and_context_survives(d):
     """The forced missing arrival of the debug hook in both backward kernels: a bounded wait
     expires, the status word reports ATTN_ERR_TIMEOUT, the kernels return through their abort
     paths, and the next backward on the same plan is correct."""
-    wl = W.random_small(seed=6, kind="CAUSAL", batch=2, hq=4, hkv=2, d=128, lmin=100, lmax=300)
+    wl = W.random_small(seed=6, kind="CAUSAL", batch=2, hq=4, hkv=2, d=d, lmin=100, lmax=300)
     q, k, v = G.device_inputs(wl)
     plan = G.M.attn_plan(hq=wl.hq, hkv=wl.hkv, head_dim=wl.d, cu_seqlens_q=wl.cu_seqlens_q,
                          cu_seqlens_k=wl.cu_seqlens_k, mask=wl.masks[0], scale=wl.scale, backward=True)
