@@ -72,6 +72,8 @@ struct BwdParams {
   int32_t hq, hkv;
   int32_t debug_flags;   // bit 0: skip the first item's per-item loads (testing the timeout path)
   int32_t dhalf;         // head_dim 256 dK/dV pass: the half of the head dimension accumulated
+  const int32_t* page_table;   // paged K/V: [batch][maxp] pages of each sequence's keys
+  int32_t page_size, num_pages, maxp;
   float scale, scale_log2;
   int64_t timeout_ns;
 };
@@ -79,10 +81,11 @@ struct BwdParams {
 // Shared-memory layout, TMEM columns and mbarriers of the two kernels. A job is one
 // 128 x 128 tile pair, S and dP (dQ) or S^T and dP^T (dK/dV) computed as M = 128, N = 128
 // MMAs; the accumulators take D (dQ) or 2 D (dV, dK) TMEM columns.
-template <int D_, bool DKV_>
+template <int D_, bool DKV_, bool PAGED_ = false>
 struct BwdCfg {
   static constexpr int D = D_;
   static constexpr bool DKV = DKV_;
+  static constexpr bool PAGED = PAGED_;   // K / V from a paged cache
   static constexpr int NBOX = D / 64;                  // 64-column boxes per tile
   static constexpr int BOX_BYTES = 128 * 128;          // 128 rows x 128 bytes
   static constexpr int TILE_BYTES = NBOX * BOX_BYTES;  // one 128-row tile of one head
@@ -214,6 +217,37 @@ __device__ __forceinline__ uint4 row_bits(const uint4* __restrict__ tiles, int m
   return mi == kMaskNone ? make_uint4(0u, 0u, 0u, 0u) : make_uint4(0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu);
 }
 
+// Paged K/V: one key tile (128 keys from tile-local row 0) of sequence `seq` into `dst`, the
+// tile's pages issued by lanes 0 .. 128 / page_size - 1 of the calling warp (one TMA issue
+// stream per page). Pages past the sequence's last, or outside the cache, read as zeros.
+template <int NBOX>
+__device__ __forceinline__ void load_paged_tile(const BwdParams& p, const CUtensorMap* tm, uint32_t dst, int seq,
+                                                int key0, int npages, int kv_head, uint32_t bar, int lane) {
+  const int ps = p.page_size, ppt = 128 / ps;
+  if (lane < ppt) {
+    const int idx = key0 / ps + lane;
+    const int32_t page = idx < npages ? __ldg(p.page_table + int64_t(seq) * p.maxp + idx) : -1;
+    int32_t row = p.num_pages * ps;   // fully out of bounds: the box reads zeros
+    if (page >= 0 && page < p.num_pages) row = page * ps;
+    for (int c = 0; c < NBOX; ++c) tma_load_3d(dst + c * 128 * 128 + lane * ps * 128, tm, c * 64, kv_head, row, bar);
+  }
+}
+
+// Rows r0 .. 127 of a tile of NBOX 64-column boxes set to zero by one thread (a paged cache
+// holds stale rows past a sequence's last key in its last page; a zero row times a zero
+// score weight must stay zero in the MMAs), then made visible to the tensor core.
+template <int NBOX>
+__device__ __forceinline__ void zero_tile_rows(uint32_t tile, int r0) {
+  for (int i = 0; i < (128 - r0) * NBOX * 8; ++i) {
+    const int row = r0 + i / (NBOX * 8), rem = i % (NBOX * 8);
+    asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(tile + uint32_t((rem >> 3) * 16384 + row * 128 +
+                                                                                   (rem & 7) * 16)),
+                 "r"(0u)
+                 : "memory");
+  }
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // ================================ dQ ================================
 template <class C>
 __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd_dq_kernel(const __grid_constant__ BwdParams p) {
@@ -267,43 +301,54 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd_dq_kernel(const
   auto tile = [&](uint32_t slot) { return sbase + C::OFF_RING + slot * C::TILE_BYTES; };
 
   if (warp == 0) {
-    // ---- TMA producer: Q and dO once per item, then K and V tiles of every job ----
-    if (lane == 0) {
+    // ---- TMA producer: Q and dO once per item, then K and V tiles of every job (paged: one
+    // lane per page); the whole warp runs the loop ----
+    {
       uint32_t g = 0;
       int n = 0, a_last = -1;
       bool ok = true;
       for (int ii = i_begin; ok && ii < i_end; ++ii, ++n) {
         const BwdItem it = p.items[p.cta_items[ii]];
-        if (!wait_bounded(BAR(C::B_AEMPTY), (n & 1) ^ 1, guard, kBwdWaitAEmpty)) break;
+        if (!__all_sync(0xffffffffu, wait_bounded(BAR(C::B_AEMPTY), (n & 1) ^ 1, guard, kBwdWaitAEmpty))) break;
         if (!((p.debug_flags & 1) && n == 0)) {
-          mbar_expect_tx(BAR(C::B_AFULL), 2 * C::TILE_BYTES);
           a_last = n;
-          for (int c = 0; c < C::NBOX; ++c) {
-            tma_load_3d(sbase + C::OFF_A + c * C::BOX_BYTES, &p.tm_a, c * 64, it.head, it.tok, BAR(C::B_AFULL));
-            tma_load_3d(sbase + C::OFF_B + c * C::BOX_BYTES, &p.tm_b, c * 64, it.head, it.tok, BAR(C::B_AFULL));
+          if (lane == 0) {
+            mbar_expect_tx(BAR(C::B_AFULL), 2 * C::TILE_BYTES);
+            for (int c = 0; c < C::NBOX; ++c) {
+              tma_load_3d(sbase + C::OFF_A + c * C::BOX_BYTES, &p.tm_a, c * 64, it.head, it.tok, BAR(C::B_AFULL));
+              tma_load_3d(sbase + C::OFF_B + c * C::BOX_BYTES, &p.tm_b, c * 64, it.head, it.tok, BAR(C::B_AFULL));
+            }
           }
         }
         for (int j = 0; ok && j < it.job_count; ++j, ++g) {
           const BwdJob jb = p.jobs[it.job_start + j];
           for (int op = 0; op < 2; ++op) {
             const uint32_t slot = op == 0 ? kslot(g) : vslot(g), use = op == 0 ? g / C::KST : g / C::VST;
-            if (!wait_bounded(BAR(C::B_REMPTY + slot), (use & 1) ^ 1, guard, kBwdWaitREmpty)) {
+            if (!__all_sync(0xffffffffu, wait_bounded(BAR(C::B_REMPTY + slot), (use & 1) ^ 1, guard, kBwdWaitREmpty))) {
               ok = false;
               break;
             }
-            mbar_expect_tx(BAR(C::B_RFULL + slot), C::TILE_BYTES);
             const CUtensorMap* tm = op == 0 ? &p.tm_c : &p.tm_d;
-            for (int c = 0; c < C::NBOX; ++c)
-              tma_load_3d(tile(slot) + c * C::BOX_BYTES, tm, c * 64, it.kv_head, jb.tok, BAR(C::B_RFULL + slot));
+            if (lane == 0) mbar_expect_tx(BAR(C::B_RFULL + slot), C::TILE_BYTES);
+            if constexpr (C::PAGED) {
+              __syncwarp();   // the expected byte count is posted before the copies
+              load_paged_tile<C::NBOX>(p, tm, tile(slot), it.seq, jb.tok, it.npages, it.kv_head, BAR(C::B_RFULL + slot),
+                                       lane);
+            } else if (lane == 0) {
+              for (int c = 0; c < C::NBOX; ++c)
+                tma_load_3d(tile(slot) + c * C::BOX_BYTES, tm, c * 64, it.kv_head, jb.tok, BAR(C::B_RFULL + slot));
+            }
           }
         }
       }
       // let the loads in flight land before the CTA exits
-      for (uint32_t x = g > uint32_t(C::KST) ? g - C::KST : 0u; x < g; ++x)
-        wait_drain(BAR(C::B_RFULL + kslot(x)), (x / C::KST) & 1, p.timeout_ns);
-      for (uint32_t x = g > uint32_t(C::VST) ? g - C::VST : 0u; x < g; ++x)
-        wait_drain(BAR(C::B_RFULL + vslot(x)), (x / C::VST) & 1, p.timeout_ns);
-      if (a_last >= 0) wait_drain(BAR(C::B_AFULL), a_last & 1, p.timeout_ns);
+      if (lane == 0) {
+        for (uint32_t x = g > uint32_t(C::KST) ? g - C::KST : 0u; x < g; ++x)
+          wait_drain(BAR(C::B_RFULL + kslot(x)), (x / C::KST) & 1, p.timeout_ns);
+        for (uint32_t x = g > uint32_t(C::VST) ? g - C::VST : 0u; x < g; ++x)
+          wait_drain(BAR(C::B_RFULL + vslot(x)), (x / C::VST) & 1, p.timeout_ns);
+        if (a_last >= 0) wait_drain(BAR(C::B_AFULL), a_last & 1, p.timeout_ns);
+      }
     }
     __syncwarp();
   } else if (warp == 1) {
@@ -322,6 +367,10 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd_dq_kernel(const
                wait_bounded(BAR(C::B_RFULL + ks), (g / C::KST) & 1, guard, kBwdWaitRFull);
           if (!ok) break;
           tc_fence_after();
+          if constexpr (C::PAGED) {
+            const int kr = p.jobs[it.job_start + j].rows;
+            if (kr < 128) zero_tile_rows<C::NBOX>(tile(ks), kr);
+          }
           mma_tile_ss<C::D>(tmem + C::TM_S + 128 * s, sbase + C::OFF_A, tile(ks), C::IDESC_SS);   // S = Q K^T
           mma_commit(BAR(C::B_SFULL + s));
         }
@@ -348,6 +397,10 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd_dq_kernel(const
                wait_bounded(BAR(C::B_RFULL + vs), (g / C::VST) & 1, guard, kBwdWaitRFull);
           if (!ok) break;
           tc_fence_after();
+          if constexpr (C::PAGED) {
+            const int kr = p.jobs[it.job_start + j].rows;
+            if (kr < 128) zero_tile_rows<C::NBOX>(tile(vs), kr);
+          }
           mma_tile_ss<C::D>(tmem + C::TM_P, sbase + C::OFF_B, tile(vs), C::IDESC_SS);   // dP = dO V^T
           mma_commit(BAR(C::B_DPFULL));
           mma_commit(BAR(C::B_REMPTY + vs));   // V is read by this MMA only
@@ -537,41 +590,55 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd_dkv_kernel(cons
   auto ring = [&](uint32_t r) { return sbase + C::OFF_RING + (r % C::STAGES) * C::TILE_BYTES; };
 
   if (warp == 0) {
-    // ---- TMA producer: K and V once per item, then Q and dO tiles of every job ----
-    if (lane == 0) {
+    // ---- TMA producer: K and V once per item (paged: one lane per page), then Q and dO
+    // tiles of every job; the whole warp runs the loop ----
+    {
       uint32_t rc = 0;
       int n = 0, a_last = -1;
       bool ok = true;
       for (int ii = i_begin; ok && ii < i_end; ++ii, ++n) {
         const BwdItem it = p.items[p.cta_items[ii]];
-        if (!wait_bounded(BAR(C::B_AEMPTY), (n & 1) ^ 1, guard, kBwdWaitAEmpty)) break;
+        if (!__all_sync(0xffffffffu, wait_bounded(BAR(C::B_AEMPTY), (n & 1) ^ 1, guard, kBwdWaitAEmpty))) break;
         if (!((p.debug_flags & 1) && n == 0)) {
-          mbar_expect_tx(BAR(C::B_AFULL), 2 * C::TILE_BYTES);
           a_last = n;
-          for (int c = 0; c < C::NBOX; ++c) {
-            tma_load_3d(sbase + C::OFF_A + c * C::BOX_BYTES, &p.tm_a, c * 64, it.kv_head, it.tok, BAR(C::B_AFULL));
-            tma_load_3d(sbase + C::OFF_B + c * C::BOX_BYTES, &p.tm_b, c * 64, it.kv_head, it.tok, BAR(C::B_AFULL));
+          if (lane == 0) mbar_expect_tx(BAR(C::B_AFULL), 2 * C::TILE_BYTES);
+          if constexpr (C::PAGED) {
+            __syncwarp();   // the expected byte count is posted before the copies
+            load_paged_tile<C::NBOX>(p, &p.tm_a, sbase + C::OFF_A, it.seq, it.tok, it.npages, it.kv_head,
+                                     BAR(C::B_AFULL), lane);
+            load_paged_tile<C::NBOX>(p, &p.tm_b, sbase + C::OFF_B, it.seq, it.tok, it.npages, it.kv_head,
+                                     BAR(C::B_AFULL), lane);
+          } else if (lane == 0) {
+            for (int c = 0; c < C::NBOX; ++c) {
+              tma_load_3d(sbase + C::OFF_A + c * C::BOX_BYTES, &p.tm_a, c * 64, it.kv_head, it.tok, BAR(C::B_AFULL));
+              tma_load_3d(sbase + C::OFF_B + c * C::BOX_BYTES, &p.tm_b, c * 64, it.kv_head, it.tok, BAR(C::B_AFULL));
+            }
           }
         }
         for (int j = 0; ok && j < it.job_count; ++j) {
           const BwdJob jb = p.jobs[it.job_start + j];
           for (int op = 0; op < 2; ++op, ++rc) {
             const uint32_t slot = rc % C::STAGES;
-            if (!wait_bounded(BAR(C::B_REMPTY + slot), ((rc / C::STAGES) & 1) ^ 1, guard, kBwdWaitREmpty)) {
+            if (!__all_sync(0xffffffffu, wait_bounded(BAR(C::B_REMPTY + slot), ((rc / C::STAGES) & 1) ^ 1, guard,
+                                                      kBwdWaitREmpty))) {
               ok = false;
               break;
             }
-            mbar_expect_tx(BAR(C::B_RFULL + slot), C::TILE_BYTES);
             const CUtensorMap* tm = op == 0 ? &p.tm_c : &p.tm_d;
-            for (int c = 0; c < C::NBOX; ++c)
-              tma_load_3d(sbase + C::OFF_RING + slot * C::TILE_BYTES + c * C::BOX_BYTES, tm, c * 64, jb.head, jb.tok,
-                          BAR(C::B_RFULL + slot));
+            if (lane == 0) {
+              mbar_expect_tx(BAR(C::B_RFULL + slot), C::TILE_BYTES);
+              for (int c = 0; c < C::NBOX; ++c)
+                tma_load_3d(sbase + C::OFF_RING + slot * C::TILE_BYTES + c * C::BOX_BYTES, tm, c * 64, jb.head, jb.tok,
+                            BAR(C::B_RFULL + slot));
+            }
           }
         }
       }
-      for (uint32_t r = rc > uint32_t(C::STAGES) ? rc - C::STAGES : 0u; r < rc; ++r)
-        wait_drain(BAR(C::B_RFULL + r % C::STAGES), (r / C::STAGES) & 1, p.timeout_ns);
-      if (a_last >= 0) wait_drain(BAR(C::B_AFULL), a_last & 1, p.timeout_ns);
+      if (lane == 0) {
+        for (uint32_t r = rc > uint32_t(C::STAGES) ? rc - C::STAGES : 0u; r < rc; ++r)
+          wait_drain(BAR(C::B_RFULL + r % C::STAGES), (r / C::STAGES) & 1, p.timeout_ns);
+        if (a_last >= 0) wait_drain(BAR(C::B_AFULL), a_last & 1, p.timeout_ns);
+      }
     }
     __syncwarp();
   } else if (warp == 1) {
@@ -793,9 +860,16 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd_dkv_kernel(cons
       if (!ok) break;
       if (!__all_sync(0xffffffffu, wait_bounded(BAR(C::B_ACCFULL), n & 1, guard, kBwdWaitAccFull))) break;
       tc_fence_after();
-      // warpgroup 0 stores the row's dv, warpgroup 1 its dk
-      const bool valid = r < it.rows;
-      const int64_t grow = int64_t(it.tok + r) * p.hkv + it.kv_head;
+      // warpgroup 0 stores the row's dv, warpgroup 1 its dk (paged: into the row's cache slot)
+      bool valid = r < it.rows;
+      int64_t krow = it.tok + r;
+      if constexpr (C::PAGED) {
+        const int key = it.tok + r;
+        const int32_t page = valid ? __ldg(p.page_table + int64_t(it.seq) * p.maxp + key / p.page_size) : -1;
+        valid = valid && page >= 0 && page < p.num_pages;
+        krow = int64_t(page) * p.page_size + key % p.page_size;
+      }
+      const int64_t grow = krow * p.hkv + it.kv_head;
       if (w == 0) store_grad_cols<C::D>(tmem + lane_base + C::TM_ACC, 1.f, valid, p.g1 + grow * C::D);
       else store_grad_cols<C::D>(tmem + lane_base + C::TM_ACC + C::D, p.scale, valid, p.g0 + grow * C::D);
       tc_fence_before();
@@ -1302,11 +1376,19 @@ attn_status_t mfa_launch_backward(const attn_plan_t* plan, const void* q, const 
                                                 static_cast<const __nv_bfloat16*>(dout), dlse, plan->d_bdelta, qrows, D);
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
   BwdParams pq{}, pk{};
+  // paged: K / V boxes of one page; dk / dv cover the whole cache, and the rows no sequence
+  // reads (other pages, the tail of a sequence's last page) stay zero
+  const uint32_t kv_box = plan->paged ? uint32_t(plan->page_size) : 128u;
   if (!encode3d(&pq.tm_a, q, D, plan->hq, plan->total_q, 128) ||
       !encode3d(&pq.tm_b, dout, D, plan->hq, plan->total_q, 128) ||
-      !encode3d(&pq.tm_c, k, D, plan->hkv, plan->total_kv_rows, 128) ||
-      !encode3d(&pq.tm_d, v, D, plan->hkv, plan->total_kv_rows, 128))
+      !encode3d(&pq.tm_c, k, D, plan->hkv, plan->total_kv_rows, kv_box) ||
+      !encode3d(&pq.tm_d, v, D, plan->hkv, plan->total_kv_rows, kv_box))
     return ATTN_ERR_CUDA;
+  if (plan->paged) {
+    cudaError_t e = cudaMemsetAsync(dk, 0, size_t(krows) * D * 2, stream);
+    if (e == cudaSuccess) e = cudaMemsetAsync(dv, 0, size_t(krows) * D * 2, stream);
+    if (e != cudaSuccess) return ATTN_ERR_CUDA;
+  }
   pk.tm_a = pq.tm_c;   // K
   pk.tm_b = pq.tm_d;   // V
   pk.tm_c = pq.tm_a;   // Q
@@ -1321,6 +1403,10 @@ attn_status_t mfa_launch_backward(const attn_plan_t* plan, const void* q, const 
     p->scale = plan->scale;
     p->scale_log2 = plan->scale * 1.4426950408889634f;
     p->timeout_ns = plan->timeout_ns;
+    p->page_table = plan->page_table;
+    p->page_size = plan->page_size;
+    p->num_pages = plan->num_pages;
+    p->maxp = plan->max_pages;
   }
   pq.items = plan->d_bq_items;
   pq.jobs = plan->d_bq_jobs;
@@ -1336,7 +1422,15 @@ attn_status_t mfa_launch_backward(const attn_plan_t* plan, const void* q, const 
   pk.g0 = static_cast<__nv_bfloat16*>(dk);
   pk.g1 = static_cast<__nv_bfloat16*>(dv);
   attn_status_t st;
-  if (D == 64) {
+  if (plan->paged && D == 64) {
+    st = launch_bwd<BwdCfg<64, false, true>>(plan->bq_ctas, pq, stream);
+    if (st == ATTN_OK) st = launch_bwd<BwdCfg<64, true, true>>(plan->bkv_ctas, pk, stream);
+  } else if (plan->paged && D == 128) {
+    st = launch_bwd<BwdCfg<128, false, true>>(plan->bq_ctas, pq, stream);
+    if (st == ATTN_OK) st = launch_bwd<BwdCfg<128, true, true>>(plan->bkv_ctas, pk, stream);
+  } else if (plan->paged) {
+    st = ATTN_ERR_UNSUPPORTED;
+  } else if (D == 64) {
     st = launch_bwd<BwdCfg<64, false>>(plan->bq_ctas, pq, stream);
     if (st == ATTN_OK) st = launch_bwd<BwdCfg<64, true>>(plan->bkv_ctas, pk, stream);
   } else if (D == 128) {

@@ -71,17 +71,19 @@ struct alignas(16) BwdItem {
   int32_t seq, kv_head;
   int32_t head;        // dQ: the query head
   int32_t tok;         // dQ: first query token of the tile; dK/dV: first key row of the tile
+                       // (paged: sequence-local key index)
   int32_t rows;        // valid rows of the tile (queries, or keys)
   int32_t job_start, job_count;
-  int32_t pad;
+  int32_t npages;      // paged K/V: pages of the sequence's keys (0 for contiguous K/V)
 };
 static_assert(sizeof(BwdItem) == 32, "BwdItem layout");
 
 struct alignas(16) BwdJob {
-  int32_t tok;         // dQ: first key row of the key tile; dK/dV: first query token of the query tile
+  int32_t tok;         // dQ: first key row of the key tile (paged: sequence-local key index);
+                       // dK/dV: first query token of the query tile
   int32_t mask;        // kMaskFull, kMaskNone, or a mask tile (dQ: query-major; dK/dV: key-major)
   int32_t head;        // dK/dV: the query head
-  int32_t rows;        // dK/dV: valid query rows of the query tile
+  int32_t rows;        // dK/dV: valid query rows of the query tile; dQ: valid keys of the key tile
 };
 static_assert(sizeof(BwdJob) == 16, "BwdJob layout");
 

@@ -857,12 +857,16 @@ struct BwdLists {
   std::vector<TileRef> tiles;
 };
 
+// Key positions in the lists: contiguous K/V -- key rows of the K / V tensors; paged --
+// sequence-local key indices (the kernels map them through row `seq` of the page table),
+// with each item's page count in `pad` and each dQ job's valid keys in `rows`.
 void build_bwd(const Shape& s, const std::vector<std::vector<int32_t>>& cnts, int num_sms, BwdLists& bl) {
   const int g = s.hq / s.hkv;
   std::vector<int64_t> q_cost, kv_cost, q_group, kv_group;
   for (int b = 0; b < s.B; ++b) {
     const int lq = s.lq[b], lk = s.lk[b];
     const int n_qt = (lq + kTile - 1) / kTile, n_kt = (lk + kTile - 1) / kTile;
+    const int32_t kbase = s.paged ? 0 : s.koff[b], npg = s.paged ? (lk + s.ps - 1) / s.ps : 0;
     const std::vector<int32_t>& cnt = cnts[b];
     // How every (query tile, key tile) is masked, the same for all heads; partial tiles are
     // numbered in row-major order. Row lists serve the dQ items, column lists the dK/dV items.
@@ -907,17 +911,18 @@ void build_bwd(const Shape& s, const std::vector<std::vector<int32_t>>& cnts, in
       // dQ items
       for (int h = kh * g; h < (kh + 1) * g; ++h)
         for (int qt = 0; qt < n_qt; ++qt) {
-          BwdItem it{b, kh, h, s.qoff[b] + qt * kTile, std::min(kTile, lq - qt * kTile), int32_t(bl.q_jobs.size()), 0, 0};
+          BwdItem it{b, kh, h, s.qoff[b] + qt * kTile, std::min(kTile, lq - qt * kTile), int32_t(bl.q_jobs.size()), 0,
+                     npg};
           if (q_start[qt] >= 0) {
             it.job_start = q_start[qt];
             it.job_count = q_count[qt];
           } else {
             for (int32_t e = row_off[qt]; e < row_off[qt + 1]; ++e) {
               const int kt = row_kt[e];
-              bl.q_jobs.push_back(BwdJob{s.koff[b] + kt * kTile, tab[size_t(qt) * n_kt + kt], h, 0});
+              bl.q_jobs.push_back(BwdJob{kbase + kt * kTile, tab[size_t(qt) * n_kt + kt], h, std::min(kTile, lk - kt * kTile)});
             }
             if (bl.q_jobs.size() == size_t(it.job_start))   // no key anywhere: one hidden job writes dq = 0
-              bl.q_jobs.push_back(BwdJob{s.koff[b], kMaskNone, h, 0});
+              bl.q_jobs.push_back(BwdJob{kbase, kMaskNone, h, 0});
             it.job_count = int32_t(bl.q_jobs.size()) - it.job_start;
             q_start[qt] = it.job_start;
             q_count[qt] = it.job_count;
@@ -928,8 +933,8 @@ void build_bwd(const Shape& s, const std::vector<std::vector<int32_t>>& cnts, in
         }
       // dK/dV items
       for (int kt = 0; kt < n_kt; ++kt) {
-        BwdItem it{b, kh, kh * g, s.koff[b] + kt * kTile, std::min(kTile, lk - kt * kTile),
-                   int32_t(bl.kv_jobs.size()), 0, 0};
+        BwdItem it{b, kh, kh * g, kbase + kt * kTile, std::min(kTile, lk - kt * kTile),
+                   int32_t(bl.kv_jobs.size()), 0, npg};
         for (int h = kh * g; h < (kh + 1) * g; ++h)
           for (int32_t e = col_off[kt]; e < col_off[kt + 1]; ++e) {
             const int qt = col_qt[e];
@@ -976,7 +981,26 @@ void transpose_tile(const uint32_t* src, uint32_t* dst) {
 
 attn_status_t plan_backward(const attn_mask_desc_t* mask, const Shape& s, RowSource& src, int num_sms,
                             cudaStream_t stream, attn_plan_t* plan) {
-  if (s.paged) return ATTN_ERR_UNSUPPORTED;
+  if (s.paged) {
+    // The gradient of a cache page shared by two sequences would be the sum of both
+    // sequences' contributions; the dK/dV kernel writes each page's rows from one work item,
+    // so every page a sequence reads (entries in [0, num_pages)) must belong to it alone.
+    if (s.d == 256) return ATTN_ERR_UNSUPPORTED;
+    std::vector<int32_t> pt(size_t(s.B) * s.maxp);
+    if (!pt.empty()) {
+      cudaError_t e = cudaMemcpyAsync(pt.data(), plan->page_table, pt.size() * 4, cudaMemcpyDeviceToHost, stream);
+      if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+      if (e != cudaSuccess) return ATTN_ERR_CUDA;
+    }
+    std::vector<uint8_t> seen(size_t(s.npages), 0);
+    for (int b = 0; b < s.B; ++b)
+      for (int i = 0; i < (s.lk[b] + s.ps - 1) / s.ps; ++i) {
+        const int32_t pg = pt[size_t(b) * s.maxp + i];
+        if (pg < 0 || pg >= s.npages) continue;
+        if (seen[size_t(pg)]) return ATTN_ERR_UNSUPPORTED;
+        seen[size_t(pg)] = 1;
+      }
+  }
   std::vector<std::vector<int32_t>> cnts(s.B);
   if (mask->kind == ATTN_MASK_CUSTOM) {
     attn_status_t st = custom_counts(mask, s, kTile, stream, cnts);
@@ -1097,7 +1121,7 @@ attn_status_t plan_impl(const attn_problem_t* problem, const attn_mask_desc_t* m
   if (st != ATTN_OK) return st;
   st = validate_mask(mask, s);
   if (st != ATTN_OK) return st;
-  if (with_bwd && s.paged) return ATTN_ERR_UNSUPPORTED;
+  if (with_bwd && s.paged && s.d == 256) return ATTN_ERR_UNSUPPORTED;
 
   int dev = 0, num_sms = 148;
   cudaError_t e = cudaGetDevice(&dev);

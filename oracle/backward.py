@@ -49,34 +49,44 @@ def attention_backward_one_head(q, k, v, mask, scale, dout, dlse=None):
 
 
 def masked_attention_backward(wl, spec, dout, dlse=None):
-    """Gradients over a contiguous workload: dout [total_q, Hq, d], dlse [total_q, Hq] or None
-    (torch or numpy). Returns (dq fp64 [total_q, Hq, d], dk, dv fp64 [total_k, Hkv, d])."""
-    if wl.paged:
-        raise ValueError("backward oracle: contiguous K/V only")
+    """Gradients: dout [total_q, Hq, d], dlse [total_q, Hq] or None (torch or numpy).
+    Returns dq fp64 [total_q, Hq, d] and dk, dv fp64 shaped like the keys: [total_k, Hkv, d]
+    for contiguous K/V; for a paged cache [num_pages, page_size, Hkv, d], key j of sequence b
+    being cache row (page_table[b, j // page_size], j % page_size) -- a cache entry's
+    gradient is the sum over the keys stored there, and entries no sequence reads get 0."""
     dout = dout.to(__import__("torch").float64).numpy() if hasattr(dout, "numpy") else np.asarray(dout, np.float64)
     if dlse is not None:
         dlse = dlse.to(__import__("torch").float64).numpy() if hasattr(dlse, "numpy") else np.asarray(dlse, np.float64)
     g = wl.hq // wl.hkv
-    total_q, total_k = int(wl.cu_seqlens_q[-1]), int(wl.cu_seqlens_k[-1])
+    total_q = int(wl.cu_seqlens_q[-1])
     dq = np.zeros((total_q, wl.hq, wl.d))
-    dk = np.zeros((total_k, wl.hkv, wl.d))
-    dv = np.zeros((total_k, wl.hkv, wl.d))
+    if wl.paged:
+        dk = np.zeros((wl.k_cache.shape[0], wl.page_size, wl.hkv, wl.d))
+    else:
+        dk = np.zeros((int(wl.cu_seqlens_k[-1]), wl.hkv, wl.d))
+    dv = np.zeros_like(dk)
     for b in range(wl.batch):
         lq, lk = wl.lq(b), wl.lk(b)
-        q0, k0 = int(wl.cu_seqlens_q[b]), int(wl.cu_seqlens_k[b])
+        q0 = int(wl.cu_seqlens_q[b])
         if lq == 0 or lk == 0:
             continue
         m = dense_mask(spec, b, lq, lk)
         kk, vv = wl.kv_of_seq(b)
         kk, vv = _f64(kk), _f64(vv)
+        if wl.paged:   # cache (page, slot) of every key of the sequence
+            keys = np.arange(lk)
+            rows = (np.asarray(wl.page_table[b], np.int64)[keys // wl.page_size], keys % wl.page_size)
+        else:
+            k0 = int(wl.cu_seqlens_k[b])
+            rows = (np.arange(k0, k0 + lk),)
         for h in range(wl.hq):
             kh = h // g
             a, bk, bv = attention_backward_one_head(_f64(wl.q[q0:q0 + lq, h]), kk[:, kh], vv[:, kh], m, wl.scale,
                                                     dout[q0:q0 + lq, h],
                                                     None if dlse is None else dlse[q0:q0 + lq, h])
             dq[q0:q0 + lq, h] = a
-            dk[k0:k0 + lk, kh] += bk
-            dv[k0:k0 + lk, kh] += bv
+            np.add.at(dk, rows + (kh,), bk)
+            np.add.at(dv, rows + (kh,), bv)
     return dq, dk, dv
 
 

@@ -38,10 +38,20 @@ def _close(got, ref, what):
     assert err.mean() <= REL_MEAN * scale_mean, f"{what}: mean err {err.mean():.3e} vs scale {scale_mean:.3e}"
 
 
-def check_backward(wl, spec, what, seed=0, with_dlse=False):
-    q, k, v = G.device_inputs(wl)
-    plan = G.M.attn_plan(hq=wl.hq, hkv=wl.hkv, head_dim=wl.d, cu_seqlens_q=wl.cu_seqlens_q,
-                         cu_seqlens_k=wl.cu_seqlens_k, mask=spec, scale=wl.scale, backward=True)
+def _bwd_plan(wl, spec):
+    kw = dict(hq=wl.hq, hkv=wl.hkv, head_dim=wl.d, cu_seqlens_q=wl.cu_seqlens_q, mask=spec, scale=wl.scale,
+              backward=True)
+    if wl.paged:
+        kw.update(kv_lens=wl.kv_lens, page_table=torch.from_numpy(wl.page_table).cuda(), page_size=wl.page_size,
+                  num_pages=wl.k_cache.shape[0])
+    else:
+        kw.update(cu_seqlens_k=wl.cu_seqlens_k)
+    return G.M.attn_plan(**kw)
+
+
+def check_backward(wl, spec, what, seed=0, with_dlse=False, inputs=None):
+    q, k, v = inputs if inputs is not None else G.device_inputs(wl)
+    plan = _bwd_plan(wl, spec)
     out, lse = G.M.forward(plan, q, k, v)
     gen = torch.Generator().manual_seed(1000 + seed)
     dout_h = W.randn_bf16(gen, q.shape[0], wl.hq, wl.d)
@@ -118,12 +128,16 @@ def test_backward_plan_required_and_unsupported():
     with pytest.raises(G.M.AttnError) as e:
         G.M.backward(plan, q, k, v, out, lse, torch.zeros_like(out))
     assert e.value.status == 1
-    # no backward over a paged cache
-    wl = W.random_small(seed=3, kind="CAUSAL", batch=2, hq=2, hkv=1, d=128, lmin=10, lmax=50, paged=True)
+    # paged backward: not at head_dim 256, and not when two sequences read the same page (its
+    # gradient would be the sum of both)
+    wl = W.random_small(seed=3, kind="CAUSAL", batch=2, hq=2, hkv=1, d=256, lmin=10, lmax=50, paged=True)
     with pytest.raises(G.M.AttnError) as e:
-        G.M.attn_plan(hq=2, hkv=1, head_dim=128, cu_seqlens_q=wl.cu_seqlens_q, kv_lens=wl.kv_lens,
-                      page_table=torch.from_numpy(wl.page_table).cuda(), page_size=wl.page_size,
-                      num_pages=wl.k_cache.shape[0], mask=wl.masks[0], backward=True)
+        _bwd_plan(wl, wl.masks[0])
+    assert e.value.status == 2
+    wl = W.random_small(seed=4, kind="CAUSAL", batch=2, hq=2, hkv=1, d=128, lmin=40, lmax=60, paged=True)
+    wl.page_table[1, 0] = wl.page_table[0, 0]
+    with pytest.raises(G.M.AttnError) as e:
+        _bwd_plan(wl, wl.masks[0])
     assert e.value.status == 2
 
 
@@ -183,3 +197,30 @@ def test_backward_timeout_reports_and_context_survives(d):
     _close(dq, rq, "after timeout dq")
     _close(dk, rk, "after timeout dk")
     _close(dv, rv, "after timeout dv")
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("ps", [16, 64])
+@pytest.mark.parametrize("kind", ["CAUSAL", "SLIDING_WINDOW", "CUSTOM"])
+def test_backward_paged(kind, ps, d):
+    # K / V from a paged cache (pages permuted, spare pages no sequence reads); dk / dv come
+    # back in the cache layout, zero on every row no sequence reads
+    wl = W.random_small(seed=80 + ps + d + len(kind), kind=kind, batch=3, hq=4, hkv=2, d=d, lmin=1, lmax=330,
+                        paged=True, page_size=ps)
+    check_backward(wl, wl.masks[0], f"bwd paged {kind} ps={ps} d={d}")
+
+
+@pytest.mark.parametrize("poison", [1e30, float("nan")])
+def test_backward_paged_poison_in_unused_slots(poison):
+    # the slots past each sequence's last key in its last page hold garbage; the dQ kernel
+    # zeroes those K / V rows in shared memory, so the gradients are those of clean caches
+    wl = W.random_small(seed=88, kind="CAUSAL", batch=3, hq=4, hkv=2, d=128, lmin=20, lmax=300, paged=True,
+                        page_size=64)
+    kc, vc = wl.k_cache.clone(), wl.v_cache.clone()
+    for b in range(wl.batch):
+        n = wl.lk(b)
+        if n % wl.page_size:
+            last = int(wl.page_table[b, n // wl.page_size])
+            kc[last, n % wl.page_size:] = poison
+            vc[last, n % wl.page_size:] = poison
+    check_backward(wl, wl.masks[0], f"bwd paged poison {poison}", inputs=(wl.q.cuda(), kc.cuda(), vc.cuda()))

@@ -153,3 +153,32 @@ def test_finite_differences_with_lse_gradient(seed):
     assert np.allclose(dq, _fd(lambda x: loss(x, k, v), q), rtol=1e-6, atol=1e-8)
     assert np.allclose(dk, _fd(lambda x: loss(q, x, v), k), rtol=1e-6, atol=1e-8)
     assert np.allclose(dv, _fd(lambda x: loss(q, k, x), v), rtol=1e-6, atol=1e-8)
+
+
+def test_paged_gradients_are_the_contiguous_ones_through_the_page_table():
+    """A paged cache's gradients: the same keys laid out contiguously give the same per-key
+    dk / dv, and the paged oracle puts key j of sequence b at cache row (page_table[b, j //
+    page_size], j % page_size); rows no sequence reads (spare pages, the tail of a last
+    page) are exactly zero."""
+    wl = W.random_small(seed=91, kind="CAUSAL", batch=3, hq=4, hkv=2, d=16, lmin=5, lmax=70, paged=True,
+                        page_size=16)
+    kv = [wl.kv_of_seq(b) for b in range(wl.batch)]
+    lk = np.asarray([wl.lk(b) for b in range(wl.batch)])
+    twin = W.Workload(name="contiguous twin", hq=wl.hq, hkv=wl.hkv, d=wl.d, scale=wl.scale,
+                      cu_seqlens_q=wl.cu_seqlens_q, q=wl.q, masks=wl.masks, cu_seqlens_k=W.cu_from_lengths(lk),
+                      k=torch.cat([a for a, _ in kv]), v=torch.cat([b for _, b in kv]), seed=wl.seed)
+    dout = torch.randn(int(wl.cu_seqlens_q[-1]), wl.hq, wl.d, generator=torch.Generator().manual_seed(5),
+                       dtype=torch.float64)
+    dq_p, dk_p, dv_p = oracle.masked_attention_backward(wl, wl.masks[0], dout)
+    dq_c, dk_c, dv_c = oracle.masked_attention_backward(twin, twin.masks[0], dout)
+    assert np.array_equal(dq_p, dq_c)
+    assert dk_p.shape == (wl.k_cache.shape[0], wl.page_size, wl.hkv, wl.d)
+    used = np.zeros(dk_p.shape[:2], bool)
+    for b in range(wl.batch):
+        k0 = int(twin.cu_seqlens_k[b])
+        for j in range(int(lk[b])):
+            pg, sl = int(wl.page_table[b, j // wl.page_size]), j % wl.page_size
+            used[pg, sl] = True
+            assert np.array_equal(dk_p[pg, sl], dk_c[k0 + j]) and np.array_equal(dv_p[pg, sl], dv_c[k0 + j])
+    assert not dk_p[~used].any() and not dv_p[~used].any()
+    assert (~used).sum() >= 7 * wl.page_size   # the spare pages are among the unread rows
