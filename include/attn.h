@@ -207,8 +207,10 @@ attn_status_t attn_masked_fwd(const attn_plan_t* plan, const void* q, const void
 
 /* Plan the forward AND the backward pass (gradients of out with respect to q, k, v).
  * Same arguments and errors as attn_plan(); the plan serves attn_masked_fwd() and
- * attn_masked_bwd(). Backward support: contiguous K/V (head_dim 64, 128 or 256); a paged
- * cache gives UNSUPPORTED. It adds a second device workspace: the dQ and dK/dV work lists over
+ * attn_masked_bwd(). Backward support: contiguous K/V at head_dim 64, 128 or 256; a paged
+ * cache at head_dim 64 or 128 when no cache page is read by two sequences (its gradient
+ * would be the sum of both; the page table is copied to the host to check). Otherwise
+ * UNSUPPORTED. It adds a second device workspace: the dQ and dK/dV work lists over
  * 128 x 128 tiles of one head, the partial-tile masks in query-major and key-major form,
  * and an fp32 [total_q][hq] buffer for the row terms dout . out. */
 attn_status_t attn_plan_bwd(const attn_problem_t* problem, const attn_mask_desc_t* mask,
@@ -222,9 +224,10 @@ attn_status_t attn_plan_bwd(const attn_problem_t* problem, const attn_mask_desc_
  * its query heads. Asynchronous on `stream`; all DEVICE pointers, 16-byte aligned:
  *   q, out, dout  bf16 [total_q][hq][head_dim]; lse fp32 [total_q][hq] as attn_masked_fwd wrote it
  *   dlse          fp32 [total_q][hq], or NULL (no gradient on lse)
- *   k, v          bf16 [total_k][hkv][head_dim]
+ *   k, v          bf16 [total_k][hkv][head_dim], or the paged caches [num_pages][page_size][hkv][head_dim]
  *   dq            bf16 [total_q][hq][head_dim]  (0 on rows that see no key)
- *   dk, dv        bf16 [total_k][hkv][head_dim] (0 on keys that no query sees)
+ *   dk, dv        bf16 shaped like k / v (0 on keys that no query sees; paged: 0 on every
+ *                 cache row that no sequence reads, the whole cache is written)
  * The plan must come from attn_plan_bwd(). Allocates nothing. Errors: INVALID_ARG (plan
  * without backward lists, null or misaligned pointer, another current device than the
  * plan's), CUDA. */
