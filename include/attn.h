@@ -324,7 +324,7 @@ const char* attn_status_string(attn_status_t status);
  *   - The plan is copied into the array on `stream` and the forward is enqueued behind it;
  *     the call returns once the host copy source has been consumed.
  *   - The first call on a device looks up the array's device address (once per device,
- *     with that device current); make that first call before any stream capture.
+ *     with that device current).
  *   - Every call reuses the same array and overwrites what the previous call left there
  *     (the status word is cleared each time), so calls whose work overlaps on the GPU --
  *     different streams, or another host thread -- race; serialise them on one stream.
