@@ -375,9 +375,34 @@ def kv_bytes_read(wl):
     return sum(wl.lk(b) for b in range(wl.batch)) * wl.hkv * wl.d * 2 * 2
 
 
-def choose_peak(clocks, fp8=False):
+def measure_e4m3_gemm_tflops(dev, n=8192, iters=20):
+    """Dense e4m3 tensor rate of this GPU, measured: cuBLASLt's fp8 GEMM (torch._scaled_mm,
+    n x n x n, e4m3 inputs, bf16 out) timed with CUDA events after warm-up -- the e4m3
+    counterpart of the driver's cuBLAS bf16 figure. None when the call is not available."""
+    import torch
+    try:
+        gen = torch.Generator(device=dev).manual_seed(0)
+        a = torch.randn(n, n, generator=gen, device=dev).to(torch.float8_e4m3fn)
+        b = torch.randn(n, n, generator=gen, device=dev).to(torch.float8_e4m3fn).t()   # column-major operand
+        one = torch.ones((), device=dev)
+        for _ in range(3):
+            torch._scaled_mm(a, b, scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        t0.record()
+        for _ in range(iters):
+            torch._scaled_mm(a, b, scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+        t1.record()
+        torch.cuda.synchronize()
+        return 2.0 * n ** 3 * iters / (t0.elapsed_time(t1) * 1e-3) / 1e12
+    except Exception:   # noqa: BLE001 -- no fp8 GEMM here: the caller falls back to the ratio rule
+        return None
+
+
+def choose_peak(clocks, fp8=False, e4m3_tflops=None):
     """Tensor peak for the roofline: the measured burst cuBLAS bf16 figure, or the sustained
-    one when the sampled SM clock fell below 90 % of its maximum (a long run at the power cap)."""
+    one when the sampled SM clock fell below 90 % of its maximum (a long run at the power cap).
+    e4m3: the fp8 GEMM rate measured in this run when given, else bf16 x 2 (the nominal ratio)."""
     pk, pk_src = peaks()
     burst = float(pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     sustained = float(pk.get("bf16_tflops_sustained", burst))
@@ -385,7 +410,9 @@ def choose_peak(clocks, fp8=False):
         clocks["sm_mhz"] < 0.9 * clocks["sm_max_mhz"]
     peak = sustained if use_sustained else burst
     pk_src += " bf16_tflops_sustained" if use_sustained else " bf16_tflops (burst)"
-    if fp8:   # e4m3 tensor rate: the measured bf16 figure x the nominal fp8 / bf16 ratio (4.5 / 2.25)
+    if fp8 and e4m3_tflops:
+        peak, pk_src = e4m3_tflops, "measured in this run: cuBLASLt e4m3 GEMM (torch._scaled_mm, 8192^3, bf16 out)"
+    elif fp8:   # e4m3 tensor rate: the measured bf16 figure x the nominal fp8 / bf16 ratio (4.5 / 2.25)
         peak *= 2.0
         pk_src += " x 2 (nominal e4m3 / bf16 ratio)"
     hbm = float(pk.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
@@ -781,7 +808,7 @@ def run_ours(args, rank, world, local_rank):
     # power cap) and the SM clock stays near its maximum (see "clocks"), so the burst cuBLAS
     # figure is the denominator; the sustained one is used only when the sampled clock fell
     # below 90 % of the maximum.
-    peak, pk_src, hbm_peak = choose_peak(clocks, fp8)
+    peak, pk_src, hbm_peak = choose_peak(clocks, fp8, measure_e4m3_gemm_tflops(dev) if fp8 else None)
     avg_launch_ms = sum(sum(x) for x in launch_ms) / sum(len(x) for x in launch_ms)
     achieved = (sum(flops) / len(flops)) / (avg_launch_ms * 1e-3) / 1e12
     tr = None if (bwd or fp8) else traffic_for(wl.name)
