@@ -207,10 +207,9 @@ attn_status_t attn_masked_fwd(const attn_plan_t* plan, const void* q, const void
 
 /* Plan the forward AND the backward pass (gradients of out with respect to q, k, v).
  * Same arguments and errors as attn_plan(); the plan serves attn_masked_fwd() and
- * attn_masked_bwd(). Backward support: contiguous K/V at head_dim 64, 128 or 256; a paged
- * cache at head_dim 64 or 128 when no cache page is read by two sequences (its gradient
- * would be the sum of both; the page table is copied to the host to check). Otherwise
- * UNSUPPORTED. It adds a second device workspace: the dQ and dK/dV work lists over
+ * attn_masked_bwd(). Backward support: head_dim 64, 128 or 256, contiguous K/V, or a paged
+ * cache when no cache page is read by two sequences (its gradient would be the sum of both;
+ * the page table is copied to the host to check, else UNSUPPORTED). It adds a second device workspace: the dQ and dK/dV work lists over
  * 128 x 128 tiles of one head, the partial-tile masks in query-major and key-major form,
  * and an fp32 [total_q][hq] buffer for the row terms dout . out. */
 attn_status_t attn_plan_bwd(const attn_problem_t* problem, const attn_mask_desc_t* mask,

@@ -895,8 +895,10 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd_dkv_kernel(cons
 // thread's MMAs in issue order, so the next job's S / dP may overwrite the slots the
 // previous job's accumulating MMAs read. TMEM: S (S^T) 0, dP (dP^T) 128, accumulators 256
 // (dQ: 256 columns; dK/dV: dV 256, dK 384).
+template <bool PAGED_ = false>
 struct Bwd256Cfg {
   static constexpr int D = 256;
+  static constexpr bool PAGED = PAGED_;   // K / V from a paged cache
   static constexpr int BOX_BYTES = 128 * 128;          // 128 rows x 64 columns
   static constexpr int TILE_BYTES = 4 * BOX_BYTES;     // resident 128 x 256 tile
   static constexpr int HALF_BYTES = 2 * BOX_BYTES;     // streamed 128 x 128 half-tile
@@ -923,15 +925,18 @@ struct Bwd256Cfg {
 // half-tiles in ring slots b0 (columns 0..127) and b1 (128..255).
 __device__ __forceinline__ void mma_ss_k256(uint32_t d, uint32_t a_tile, uint32_t b0, uint32_t b1, uint32_t idesc) {
   mma_ss_x8_k128(d, desc_of(desc_lo(a_tile, 16)), desc_of(desc_lo(b0, 16)), idesc, 0u);
-  mma_ss_x8_k128(d, desc_of(desc_lo(a_tile + Bwd256Cfg::HALF_BYTES, 16)), desc_of(desc_lo(b1, 16)), idesc, 1u);
+  mma_ss_x8_k128(d, desc_of(desc_lo(a_tile + Bwd256Cfg<>::HALF_BYTES, 16)), desc_of(desc_lo(b1, 16)), idesc, 1u);
 }
 
-// Producer for the d = 256 kernels: the two resident tiles once per item (tm_a, tm_b at
-// the item's rows and head), then four half-tiles per job in the order `order` names
-// (each entry: 0 / 1 = tm_c half 0 / 1, 2 / 3 = tm_d half 0 / 1) through the ring.
+// Producer for the d = 256 kernels, run by the whole warp (waits agreed with a vote): the
+// two resident tiles once per item (tm_a, tm_b at the item's rows and head), then four
+// half-tiles per job in the order `order` names (each entry: 0 / 1 = tm_c half 0 / 1,
+// 2 / 3 = tm_d half 0 / 1) through the ring. Lane 0 issues the contiguous copies; K / V from
+// a paged cache (the dK/dV kernel's resident tiles, the dQ kernel's half-tiles) come one
+// lane per page.
 template <class C>
 __device__ __forceinline__ void bwd256_produce(const BwdParams& p, uint32_t sbase, uint32_t bar0, const Guard& guard,
-                                               int i_begin, int i_end, bool dkv, const int order[4]) {
+                                               int i_begin, int i_end, bool dkv, const int order[4], int lane) {
 #define BAR(i) (bar0 + 8u * uint32_t(i))
   uint32_t rc = 0;
   int n = 0, a_last = -1;
@@ -939,13 +944,19 @@ __device__ __forceinline__ void bwd256_produce(const BwdParams& p, uint32_t sbas
   for (int ii = i_begin; ok && ii < i_end; ++ii, ++n) {
     const BwdItem it = p.items[p.cta_items[ii]];
     const int a_head = dkv ? it.kv_head : it.head;
-    if (!wait_bounded(BAR(C::B_AEMPTY), (n & 1) ^ 1, guard, kBwdWaitAEmpty)) break;
+    if (!__all_sync(0xffffffffu, wait_bounded(BAR(C::B_AEMPTY), (n & 1) ^ 1, guard, kBwdWaitAEmpty))) break;
     if (!((p.debug_flags & 1) && n == 0)) {
-      mbar_expect_tx(BAR(C::B_AFULL), 2 * C::TILE_BYTES);
       a_last = n;
-      for (int c = 0; c < 4; ++c) {
-        tma_load_3d(sbase + C::OFF_A + c * C::BOX_BYTES, &p.tm_a, c * 64, a_head, it.tok, BAR(C::B_AFULL));
-        tma_load_3d(sbase + C::OFF_B + c * C::BOX_BYTES, &p.tm_b, c * 64, a_head, it.tok, BAR(C::B_AFULL));
+      if (lane == 0) mbar_expect_tx(BAR(C::B_AFULL), 2 * C::TILE_BYTES);
+      if (C::PAGED && dkv) {
+        __syncwarp();   // the expected byte count is posted before the copies
+        load_paged_tile<4>(p, &p.tm_a, sbase + C::OFF_A, it.seq, it.tok, it.npages, it.kv_head, BAR(C::B_AFULL), lane);
+        load_paged_tile<4>(p, &p.tm_b, sbase + C::OFF_B, it.seq, it.tok, it.npages, it.kv_head, BAR(C::B_AFULL), lane);
+      } else if (lane == 0) {
+        for (int c = 0; c < 4; ++c) {
+          tma_load_3d(sbase + C::OFF_A + c * C::BOX_BYTES, &p.tm_a, c * 64, a_head, it.tok, BAR(C::B_AFULL));
+          tma_load_3d(sbase + C::OFF_B + c * C::BOX_BYTES, &p.tm_b, c * 64, a_head, it.tok, BAR(C::B_AFULL));
+        }
       }
     }
     for (int j = 0; ok && j < it.job_count; ++j) {
@@ -953,22 +964,38 @@ __device__ __forceinline__ void bwd256_produce(const BwdParams& p, uint32_t sbas
       const int head = dkv ? jb.head : it.kv_head;
       for (int q = 0; q < 4; ++q, ++rc) {
         const uint32_t slot = rc % C::RSLOTS;
-        if (!wait_bounded(BAR(C::B_REMPTY + slot), ((rc / C::RSLOTS) & 1) ^ 1, guard, kBwdWaitREmpty)) {
+        if (!__all_sync(0xffffffffu,
+                        wait_bounded(BAR(C::B_REMPTY + slot), ((rc / C::RSLOTS) & 1) ^ 1, guard, kBwdWaitREmpty))) {
           ok = false;
           break;
         }
-        mbar_expect_tx(BAR(C::B_RFULL + slot), C::HALF_BYTES);
+        if (lane == 0) mbar_expect_tx(BAR(C::B_RFULL + slot), C::HALF_BYTES);
         const CUtensorMap* tm = order[q] < 2 ? &p.tm_c : &p.tm_d;
         const int col = (order[q] & 1) * 128;
-        for (int c = 0; c < 2; ++c)
-          tma_load_3d(sbase + C::OFF_RING + slot * C::HALF_BYTES + c * C::BOX_BYTES, tm, col + c * 64, head, jb.tok,
-                      BAR(C::B_RFULL + slot));
+        const uint32_t dst = sbase + C::OFF_RING + slot * C::HALF_BYTES;
+        if (C::PAGED && !dkv) {
+          __syncwarp();
+          const int ps = p.page_size;
+          if (lane < 128 / ps) {   // lane = page of the key tile
+            const int idx = jb.tok / ps + lane;
+            const int32_t page = idx < it.npages ? __ldg(p.page_table + int64_t(it.seq) * p.maxp + idx) : -1;
+            int32_t row = p.num_pages * ps;   // fully out of bounds: the box reads zeros
+            if (page >= 0 && page < p.num_pages) row = page * ps;
+            for (int c = 0; c < 2; ++c)
+              tma_load_3d(dst + c * C::BOX_BYTES + lane * ps * 128, tm, col + c * 64, head, row, BAR(C::B_RFULL + slot));
+          }
+        } else if (lane == 0) {
+          for (int c = 0; c < 2; ++c)
+            tma_load_3d(dst + c * C::BOX_BYTES, tm, col + c * 64, head, jb.tok, BAR(C::B_RFULL + slot));
+        }
       }
     }
   }
-  for (uint32_t r = rc > uint32_t(C::RSLOTS) ? rc - C::RSLOTS : 0u; r < rc; ++r)
-    wait_drain(BAR(C::B_RFULL + r % C::RSLOTS), (r / C::RSLOTS) & 1, p.timeout_ns);
-  if (a_last >= 0) wait_drain(BAR(C::B_AFULL), a_last & 1, p.timeout_ns);
+  if (lane == 0) {
+    for (uint32_t r = rc > uint32_t(C::RSLOTS) ? rc - C::RSLOTS : 0u; r < rc; ++r)
+      wait_drain(BAR(C::B_RFULL + r % C::RSLOTS), (r / C::RSLOTS) & 1, p.timeout_ns);
+    if (a_last >= 0) wait_drain(BAR(C::B_AFULL), a_last & 1, p.timeout_ns);
+  }
 #undef BAR
 }
 
@@ -1024,10 +1051,8 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd256_dq_kernel(co
 
   if (warp == 0) {
     // ---- TMA producer: Q and dO once per item; V halves, then K halves of every job ----
-    if (lane == 0) {
-      const int order[4] = {2, 3, 0, 1};   // tm_c = K, tm_d = V
-      bwd256_produce<C>(p, sbase, bar0, guard, i_begin, i_end, false, order);
-    }
+    const int order[4] = {2, 3, 0, 1};   // tm_c = K, tm_d = V
+    bwd256_produce<C>(p, sbase, bar0, guard, i_begin, i_end, false, order, lane);
     __syncwarp();
   } else if (warp == 1) {
     // ---- MMA issuer: dP = dO V^T, S = Q K^T, then dQ += dS K for each job ----
@@ -1044,6 +1069,11 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd256_dq_kernel(co
                wait_bounded(BAR(C::B_RFULL + rv1 % C::RSLOTS), (rv1 / C::RSLOTS) & 1, guard, kBwdWaitRFull);
           if (!ok) break;
           tc_fence_after();
+          const int kr = C::PAGED ? p.jobs[it.job_start + j].rows : 128;
+          if (kr < 128) {   // a paged cache's stale rows past the sequence's last key
+            zero_tile_rows<2>(ring(rv0), kr);
+            zero_tile_rows<2>(ring(rv1), kr);
+          }
           mma_ss_k256(tmem + C::TM_P, sbase + C::OFF_B, ring(rv0), ring(rv1), C::IDESC_SS);   // dP = dO V^T
           mma_commit(BAR(C::B_DPFULL));
           mma_commit(BAR(C::B_REMPTY + rv0 % C::RSLOTS));
@@ -1052,6 +1082,10 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd256_dq_kernel(co
                wait_bounded(BAR(C::B_RFULL + rk1 % C::RSLOTS), (rk1 / C::RSLOTS) & 1, guard, kBwdWaitRFull);
           if (!ok) break;
           tc_fence_after();
+          if (kr < 128) {
+            zero_tile_rows<2>(ring(rk0), kr);
+            zero_tile_rows<2>(ring(rk1), kr);
+          }
           mma_ss_k256(tmem + C::TM_S, sbase + C::OFF_A, ring(rk0), ring(rk1), C::IDESC_SS);   // S = Q K^T
           mma_commit(BAR(C::B_SFULL));
           ok = wait_bounded(BAR(C::B_READY), g & 1, guard, kBwdWaitDsReady);
@@ -1169,10 +1203,8 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd256_dkv_kernel(c
 
   if (warp == 0) {
     // ---- TMA producer: K and V once per item; Q and dO halves of every job ----
-    if (lane == 0) {
-      const int order[4] = {1 - h, h, 2 + (1 - h), 2 + h};   // tm_c = Q, tm_d = dO
-      bwd256_produce<C>(p, sbase, bar0, guard, i_begin, i_end, true, order);
-    }
+    const int order[4] = {1 - h, h, 2 + (1 - h), 2 + h};   // tm_c = Q, tm_d = dO
+    bwd256_produce<C>(p, sbase, bar0, guard, i_begin, i_end, true, order, lane);
     __syncwarp();
   } else if (warp == 1) {
     // ---- MMA issuer: S^T = K Q^T, dP^T = V dO^T, then dV_h += P^T dO_h and dK_h += dS^T Q_h ----
@@ -1300,8 +1332,16 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd256_dkv_kernel(c
       if (!__all_sync(0xffffffffu, wait_bounded(BAR(C::B_ACCFULL), n & 1, guard, kBwdWaitAccFull))) break;
       tc_fence_after();
       // warpgroup 0 stores columns 128 h .. 128 h + 127 of the row's dv, warpgroup 1 of its dk
-      const bool valid = r < it.rows;
-      const int64_t grow = int64_t(it.tok + r) * p.hkv + it.kv_head;
+      // (paged: into the key's cache slot)
+      bool valid = r < it.rows;
+      int64_t krow = it.tok + r;
+      if constexpr (C::PAGED) {
+        const int key = it.tok + r;
+        const int32_t page = valid ? __ldg(p.page_table + int64_t(it.seq) * p.maxp + key / p.page_size) : -1;
+        valid = valid && page >= 0 && page < p.num_pages;
+        krow = int64_t(page) * p.page_size + key % p.page_size;
+      }
+      const int64_t grow = krow * p.hkv + it.kv_head;
       if (w == 0) store_grad_cols<128>(tmem + lane_base + C::TM_ACC, 1.f, valid, p.g1 + grow * C::D + 128 * h);
       else store_grad_cols<128>(tmem + lane_base + C::TM_ACC + 128, p.scale, valid, p.g0 + grow * C::D + 128 * h);
       tc_fence_before();
@@ -1335,9 +1375,9 @@ attn_status_t launch_bwd(int ctas, const BwdParams& p, cudaStream_t stream) {
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
-template <bool DKV>
+template <bool DKV, bool PAGED>
 attn_status_t launch_bwd256(int ctas, const BwdParams& p, cudaStream_t stream) {
-  using C = Bwd256Cfg;
+  using C = Bwd256Cfg<PAGED>;
   if constexpr (DKV) {
     const cudaError_t attr = once_per_device([] {
       return cudaFuncSetAttribute(masked_attn_bwd256_dkv_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1429,7 +1469,11 @@ attn_status_t mfa_launch_backward(const attn_plan_t* plan, const void* q, const 
     st = launch_bwd<BwdCfg<128, false, true>>(plan->bq_ctas, pq, stream);
     if (st == ATTN_OK) st = launch_bwd<BwdCfg<128, true, true>>(plan->bkv_ctas, pk, stream);
   } else if (plan->paged) {
-    st = ATTN_ERR_UNSUPPORTED;
+    st = launch_bwd256<false, true>(plan->bq_ctas, pq, stream);
+    for (int h = 0; h < 2 && st == ATTN_OK; ++h) {
+      pk.dhalf = h;
+      st = launch_bwd256<true, true>(plan->bkv_ctas, pk, stream);
+    }
   } else if (D == 64) {
     st = launch_bwd<BwdCfg<64, false>>(plan->bq_ctas, pq, stream);
     if (st == ATTN_OK) st = launch_bwd<BwdCfg<64, true>>(plan->bkv_ctas, pk, stream);
@@ -1437,10 +1481,10 @@ attn_status_t mfa_launch_backward(const attn_plan_t* plan, const void* q, const 
     st = launch_bwd<BwdCfg<128, false>>(plan->bq_ctas, pq, stream);
     if (st == ATTN_OK) st = launch_bwd<BwdCfg<128, true>>(plan->bkv_ctas, pk, stream);
   } else {
-    st = launch_bwd256<false>(plan->bq_ctas, pq, stream);
+    st = launch_bwd256<false, false>(plan->bq_ctas, pq, stream);
     for (int h = 0; h < 2 && st == ATTN_OK; ++h) {
       pk.dhalf = h;
-      st = launch_bwd256<true>(plan->bkv_ctas, pk, stream);
+      st = launch_bwd256<true, false>(plan->bkv_ctas, pk, stream);
     }
   }
   return st;

@@ -985,7 +985,6 @@ attn_status_t plan_backward(const attn_mask_desc_t* mask, const Shape& s, RowSou
     // The gradient of a cache page shared by two sequences would be the sum of both
     // sequences' contributions; the dK/dV kernel writes each page's rows from one work item,
     // so every page a sequence reads (entries in [0, num_pages)) must belong to it alone.
-    if (s.d == 256) return ATTN_ERR_UNSUPPORTED;
     std::vector<int32_t> pt(size_t(s.B) * s.maxp);
     if (!pt.empty()) {
       cudaError_t e = cudaMemcpyAsync(pt.data(), plan->page_table, pt.size() * 4, cudaMemcpyDeviceToHost, stream);
@@ -1121,7 +1120,6 @@ attn_status_t plan_impl(const attn_problem_t* problem, const attn_mask_desc_t* m
   if (st != ATTN_OK) return st;
   st = validate_mask(mask, s);
   if (st != ATTN_OK) return st;
-  if (with_bwd && s.paged && s.d == 256) return ATTN_ERR_UNSUPPORTED;
 
   int dev = 0, num_sms = 148;
   cudaError_t e = cudaGetDevice(&dev);
