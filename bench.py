@@ -11,7 +11,8 @@ of the five benchmark workloads that fit one GPU.
 Metric: effective TFLOP/s = 4 * d * (unmasked pairs) * Hq / time, summed over the masks of
 the step (masked pairs are not counted). Prints ONE JSON line on rank 0. After the
 headline, the other four benchmark workloads are timed one by one and reported in the same
-line under "per_config" (--no-per-config skips them).
+line under "per_config", and the backward of the chunk-causal (d=128) and Gemma2 (d=256)
+workloads under "backward" (--no-per-config skips both).
 
 Multi-GPU (torchrun, one rank per GPU): every rank runs its own independent batch of the
 same workload (seed offset by rank); there is no collective on the data path. Timing is
@@ -340,7 +341,8 @@ def make_plan(M, wl, spec, dev, kv_splits=0, backward=False, q_rows=None):
 def kernel_name(wl, fp8=False, bwd=False):
     """The kernel a forward (or backward) of this workload launches."""
     if bwd:
-        return f"masked_attn_bwd_dq_kernel + masked_attn_bwd_dkv_kernel d={wl.d}"
+        pre = "masked_attn_bwd256" if wl.d == 256 else "masked_attn_bwd"
+        return f"{pre}_dq_kernel + {pre}_dkv_kernel d={wl.d}{' paged' if wl.paged else ''}"
     base = "masked_attn_fwd_pair_kernel (2-SM)" if wl.d == 256 else "masked_attn_fwd_kernel"
     return f"{base}{' e4m3' if fp8 else ''} d={wl.d}{' paged' if wl.paged else ''}"
 
@@ -419,20 +421,27 @@ def choose_peak(clocks, fp8=False, e4m3_tflops=None):
     return peak, pk_src, hbm
 
 
-def time_config(M, cfg, dev, stream, steps, warmup, peak, hbm_peak):
-    """Forward of one benchmark workload (every mask of it) on this GPU: CUDA-event time of
-    each launch over `steps` steps after `warmup`, L2 flushed between launches when the
-    inputs fit in it. Returns the per-config entry of the bench line."""
+def time_config(M, cfg, dev, stream, steps, warmup, peak, hbm_peak, bwd=False):
+    """Forward (or, with `bwd`, backward) of one benchmark workload (every mask of it) on this
+    GPU: CUDA-event time of each launch over `steps` steps after `warmup`, L2 flushed between
+    launches when the inputs fit in it. Returns the per-config entry of the bench line."""
     import torch
     wl = workload(cfg, 0)
     q, k, v = device_inputs(wl, dev)
-    plans, plan_ms = build_plans(M, wl, dev)
+    plans, plan_ms = build_plans(M, wl, dev, backward=bwd)
     stats = [M.attn_plan_get_stats(p) for p in plans]
-    flops = [flops_of(s, wl) for s in stats]
+    flops = [flops_of(s, wl) * (2.5 if bwd else 1.0) for s in stats]
     tq = q.shape[0]
     outs = [torch.empty(tq, wl.hq, wl.d, dtype=torch.bfloat16, device=dev) for _ in plans]
     lses = [torch.empty(tq, wl.hq, dtype=torch.float32, device=dev) for _ in plans]
     in_bytes = (q.numel() + k.numel() + v.numel()) * 2
+    if bwd:
+        for i, p in enumerate(plans):
+            M.attn_masked_fwd(p, q, k, v, outs[i], lses[i], stream)
+        gen = torch.Generator(device=dev).manual_seed(wl.seed + 101)
+        dout = torch.randn(tq, wl.hq, wl.d, generator=gen, device=dev).to(torch.bfloat16)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        in_bytes += sum(o.numel() * 2 + l.numel() * 4 for o, l in zip(outs, lses)) + dout.numel() * 2
     flush = torch.empty(256 * 2**20, dtype=torch.uint8, device=dev) if in_bytes <= L2_BYTES else None
     ev = [[[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in plans] for _ in range(steps)]
     for s in range(warmup + steps):
@@ -441,19 +450,23 @@ def time_config(M, cfg, dev, stream, steps, warmup, peak, hbm_peak):
                 flush.fill_(s & 255)
             if s >= warmup:
                 ev[s - warmup][i][0].record(stream)
-            M.attn_masked_fwd(p, q, k, v, outs[i], lses[i], stream)
+            if bwd:
+                M.attn_masked_bwd(p, q, k, v, outs[i], lses[i], dout, dq, dk, dv, stream)
+            else:
+                M.attn_masked_fwd(p, q, k, v, outs[i], lses[i], stream)
             if s >= warmup:
                 ev[s - warmup][i][1].record(stream)
     torch.cuda.synchronize()
     for p in plans:
         st = M.attn_plan_check_status(p)
         if st != 0:
-            raise RuntimeError(f"workload {cfg}: forward reported {M.STATUS.get(st, st)}")
+            raise RuntimeError(f"workload {cfg}: {'backward' if bwd else 'forward'} reported {M.STATUS.get(st, st)}")
     launch_ms = [[ev[s][i][0].elapsed_time(ev[s][i][1]) for s in range(steps)] for i in range(len(plans))]
     mean_ms = [statistics.mean(x) for x in launch_ms]
     step_ms = sum(mean_ms)
     tflops = sum(flops) / (step_ms * 1e-3) / 1e12
-    entry = {"config": cfg, "workload": wl.name, "kernel": kernel_name(wl), "steps": steps,
+    entry = {"config": cfg, "workload": wl.name, "pass": "bwd" if bwd else "fwd",
+             "kernel": kernel_name(wl, bwd=bwd), "steps": steps,
              "ms_per_step": step_ms, "tflops_per_s": tflops, "frac": tflops / peak,
              "per_mask": [{"mask": m.kind, "ms": mm, "ms_median": statistics.median(x),
                            "tflops_per_s": f / (mm * 1e-3) / 1e12, "frac": f / (mm * 1e-3) / 1e12 / peak,
@@ -463,7 +476,7 @@ def time_config(M, cfg, dev, stream, steps, warmup, peak, hbm_peak):
                           for m, s, f, x, mm, pm in zip(wl.masks, stats, flops, launch_ms, mean_ms, plan_ms)],
              "l2": "L2 flushed between launches" if flush is not None else
                    f"inputs {in_bytes / 2**20:.0f} MiB vs 126 MiB L2; no flush"}
-    if wl.paged:
+    if wl.paged and not bwd:
         # the K/V stream: bytes of the keys every request holds, read once per launch at least
         kvb = kv_bytes_read(wl)
         gbs = kvb / (step_ms / len(plans) * 1e-3) / 1e9
@@ -471,6 +484,9 @@ def time_config(M, cfg, dev, stream, steps, warmup, peak, hbm_peak):
                               "frac_of_hbm": gbs / hbm_peak}
     mask_bytes = sum(s["mask_tile_reads"] for s in stats) * 2048.0
     entry["mask_gbs"] = mask_bytes / (step_ms * 1e-3) / 1e9
+    if bwd:
+        entry["flops_note"] = "10 d FLOPs per unmasked pair and head (2.5 x the forward's 4 d)"
+        del dout, dq, dk, dv
     del q, k, v, outs, lses, flush, plans
     torch.cuda.empty_cache()
     return entry
@@ -858,6 +874,9 @@ def run_ours(args, rank, world, local_rank):
         torch.cuda.empty_cache()
         line["per_config"] = [time_config(M, c, dev, stream, max(3, min(args.steps, 30)), 3, peak, hbm_peak)
                               for c in (1, 2, 3, 4, 5) if c != args.config]
+        # the backward of the chunk-causal (d = 128) and Gemma2 (d = 256) workloads
+        line["backward"] = [time_config(M, c, dev, stream, max(3, min(args.steps, 20)), 3, peak, hbm_peak, bwd=True)
+                            for c in (4, 2)]
     if world == 1 and not args.no_cpu_baseline and not bwd and not fp8:
         pairs, secs, desc = oracle_sample(wl, wl.masks, args.cpu_seconds)
         line["cpu_baseline"] = {"value": 4.0 * wl.d * pairs / secs / 1e12, "unit": "TFLOP/s",

@@ -312,12 +312,12 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd_dq_kernel(const
         if (!__all_sync(0xffffffffu, wait_bounded(BAR(C::B_AEMPTY), (n & 1) ^ 1, guard, kBwdWaitAEmpty))) break;
         if (!((p.debug_flags & 1) && n == 0)) {
           a_last = n;
-          if (lane == 0) {
-            mbar_expect_tx(BAR(C::B_AFULL), 2 * C::TILE_BYTES);
-            for (int c = 0; c < C::NBOX; ++c) {
-              tma_load_3d(sbase + C::OFF_A + c * C::BOX_BYTES, &p.tm_a, c * 64, it.head, it.tok, BAR(C::B_AFULL));
-              tma_load_3d(sbase + C::OFF_B + c * C::BOX_BYTES, &p.tm_b, c * 64, it.head, it.tok, BAR(C::B_AFULL));
-            }
+          if (lane == 0) mbar_expect_tx(BAR(C::B_AFULL), 2 * C::TILE_BYTES);
+          __syncwarp();   // the expected byte count is posted before the copies
+          if (lane < 2 * C::NBOX) {   // one box per lane: one issuing thread caps the copy rate
+            const int c = lane % C::NBOX;
+            tma_load_3d(sbase + (lane < C::NBOX ? C::OFF_A : C::OFF_B) + c * C::BOX_BYTES,
+                        lane < C::NBOX ? &p.tm_a : &p.tm_b, c * 64, it.head, it.tok, BAR(C::B_AFULL));
           }
         }
         for (int j = 0; ok && j < it.job_count; ++j, ++g) {
@@ -330,13 +330,12 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd_dq_kernel(const
             }
             const CUtensorMap* tm = op == 0 ? &p.tm_c : &p.tm_d;
             if (lane == 0) mbar_expect_tx(BAR(C::B_RFULL + slot), C::TILE_BYTES);
+            __syncwarp();   // the expected byte count is posted before the copies
             if constexpr (C::PAGED) {
-              __syncwarp();   // the expected byte count is posted before the copies
               load_paged_tile<C::NBOX>(p, tm, tile(slot), it.seq, jb.tok, it.npages, it.kv_head, BAR(C::B_RFULL + slot),
                                        lane);
-            } else if (lane == 0) {
-              for (int c = 0; c < C::NBOX; ++c)
-                tma_load_3d(tile(slot) + c * C::BOX_BYTES, tm, c * 64, it.kv_head, jb.tok, BAR(C::B_RFULL + slot));
+            } else if (lane < C::NBOX) {
+              tma_load_3d(tile(slot) + lane * C::BOX_BYTES, tm, lane * 64, it.kv_head, jb.tok, BAR(C::B_RFULL + slot));
             }
           }
         }
@@ -608,10 +607,12 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd_dkv_kernel(cons
                                      BAR(C::B_AFULL), lane);
             load_paged_tile<C::NBOX>(p, &p.tm_b, sbase + C::OFF_B, it.seq, it.tok, it.npages, it.kv_head,
                                      BAR(C::B_AFULL), lane);
-          } else if (lane == 0) {
-            for (int c = 0; c < C::NBOX; ++c) {
-              tma_load_3d(sbase + C::OFF_A + c * C::BOX_BYTES, &p.tm_a, c * 64, it.kv_head, it.tok, BAR(C::B_AFULL));
-              tma_load_3d(sbase + C::OFF_B + c * C::BOX_BYTES, &p.tm_b, c * 64, it.kv_head, it.tok, BAR(C::B_AFULL));
+          } else {
+            __syncwarp();
+            if (lane < 2 * C::NBOX) {   // one box per lane
+              const int c = lane % C::NBOX;
+              tma_load_3d(sbase + (lane < C::NBOX ? C::OFF_A : C::OFF_B) + c * C::BOX_BYTES,
+                          lane < C::NBOX ? &p.tm_a : &p.tm_b, c * 64, it.kv_head, it.tok, BAR(C::B_AFULL));
             }
           }
         }
@@ -625,12 +626,11 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd_dkv_kernel(cons
               break;
             }
             const CUtensorMap* tm = op == 0 ? &p.tm_c : &p.tm_d;
-            if (lane == 0) {
-              mbar_expect_tx(BAR(C::B_RFULL + slot), C::TILE_BYTES);
-              for (int c = 0; c < C::NBOX; ++c)
-                tma_load_3d(sbase + C::OFF_RING + slot * C::TILE_BYTES + c * C::BOX_BYTES, tm, c * 64, jb.head, jb.tok,
-                            BAR(C::B_RFULL + slot));
-            }
+            if (lane == 0) mbar_expect_tx(BAR(C::B_RFULL + slot), C::TILE_BYTES);
+            __syncwarp();
+            if (lane < C::NBOX)   // one box per lane
+              tma_load_3d(sbase + C::OFF_RING + slot * C::TILE_BYTES + lane * C::BOX_BYTES, tm, lane * 64, jb.head,
+                          jb.tok, BAR(C::B_RFULL + slot));
           }
         }
       }
@@ -931,9 +931,9 @@ __device__ __forceinline__ void mma_ss_k256(uint32_t d, uint32_t a_tile, uint32_
 // Producer for the d = 256 kernels, run by the whole warp (waits agreed with a vote): the
 // two resident tiles once per item (tm_a, tm_b at the item's rows and head), then four
 // half-tiles per job in the order `order` names (each entry: 0 / 1 = tm_c half 0 / 1,
-// 2 / 3 = tm_d half 0 / 1) through the ring. Lane 0 issues the contiguous copies; K / V from
-// a paged cache (the dK/dV kernel's resident tiles, the dQ kernel's half-tiles) come one
-// lane per page.
+// 2 / 3 = tm_d half 0 / 1) through the ring. Contiguous copies go one box per lane; K / V from
+// a paged cache (the dK/dV kernel's resident tiles, the dQ kernel's half-tiles) one lane per
+// page.
 template <class C>
 __device__ __forceinline__ void bwd256_produce(const BwdParams& p, uint32_t sbase, uint32_t bar0, const Guard& guard,
                                                int i_begin, int i_end, bool dkv, const int order[4], int lane) {
@@ -948,15 +948,14 @@ __device__ __forceinline__ void bwd256_produce(const BwdParams& p, uint32_t sbas
     if (!((p.debug_flags & 1) && n == 0)) {
       a_last = n;
       if (lane == 0) mbar_expect_tx(BAR(C::B_AFULL), 2 * C::TILE_BYTES);
+      __syncwarp();   // the expected byte count is posted before the copies
       if (C::PAGED && dkv) {
-        __syncwarp();   // the expected byte count is posted before the copies
         load_paged_tile<4>(p, &p.tm_a, sbase + C::OFF_A, it.seq, it.tok, it.npages, it.kv_head, BAR(C::B_AFULL), lane);
         load_paged_tile<4>(p, &p.tm_b, sbase + C::OFF_B, it.seq, it.tok, it.npages, it.kv_head, BAR(C::B_AFULL), lane);
-      } else if (lane == 0) {
-        for (int c = 0; c < 4; ++c) {
-          tma_load_3d(sbase + C::OFF_A + c * C::BOX_BYTES, &p.tm_a, c * 64, a_head, it.tok, BAR(C::B_AFULL));
-          tma_load_3d(sbase + C::OFF_B + c * C::BOX_BYTES, &p.tm_b, c * 64, a_head, it.tok, BAR(C::B_AFULL));
-        }
+      } else if (lane < 8) {   // one box per lane
+        const int c = lane & 3;
+        tma_load_3d(sbase + (lane < 4 ? C::OFF_A : C::OFF_B) + c * C::BOX_BYTES, lane < 4 ? &p.tm_a : &p.tm_b, c * 64,
+                    a_head, it.tok, BAR(C::B_AFULL));
       }
     }
     for (int j = 0; ok && j < it.job_count; ++j) {
@@ -970,11 +969,11 @@ __device__ __forceinline__ void bwd256_produce(const BwdParams& p, uint32_t sbas
           break;
         }
         if (lane == 0) mbar_expect_tx(BAR(C::B_RFULL + slot), C::HALF_BYTES);
+        __syncwarp();
         const CUtensorMap* tm = order[q] < 2 ? &p.tm_c : &p.tm_d;
         const int col = (order[q] & 1) * 128;
         const uint32_t dst = sbase + C::OFF_RING + slot * C::HALF_BYTES;
         if (C::PAGED && !dkv) {
-          __syncwarp();
           const int ps = p.page_size;
           if (lane < 128 / ps) {   // lane = page of the key tile
             const int idx = jb.tok / ps + lane;
@@ -984,9 +983,8 @@ __device__ __forceinline__ void bwd256_produce(const BwdParams& p, uint32_t sbas
             for (int c = 0; c < 2; ++c)
               tma_load_3d(dst + c * C::BOX_BYTES + lane * ps * 128, tm, col + c * 64, head, row, BAR(C::B_RFULL + slot));
           }
-        } else if (lane == 0) {
-          for (int c = 0; c < 2; ++c)
-            tma_load_3d(dst + c * C::BOX_BYTES, tm, col + c * 64, head, jb.tok, BAR(C::B_RFULL + slot));
+        } else if (lane < 2) {   // one box per lane
+          tma_load_3d(dst + lane * C::BOX_BYTES, tm, col + lane * 64, head, jb.tok, BAR(C::B_RFULL + slot));
         }
       }
     }
