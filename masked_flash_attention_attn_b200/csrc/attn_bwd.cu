@@ -54,6 +54,28 @@ namespace {
 
 #include "device_common.cuh"
 
+// The elementwise loops work on packed fp32 pairs (one f32x2 instruction per two elements):
+// the two warps of each sub-partition are limited by issue slots and the MUFU exponentials.
+__device__ __forceinline__ uint64_t fmul2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
+// 2^x of a packed pair (MUFU).
+__device__ __forceinline__ uint64_t exp2_pair(uint64_t x) {
+  float x0, x1;
+  unpk2(x, x0, x1);
+  return pk2(ex2(x0), ex2(x1));
+}
+
+// Two bf16 of a packed pair (lower element in the low half).
+__device__ __forceinline__ uint32_t pack_bf16x2(uint64_t v) {
+  float a, b;
+  unpk2(v, a, b);
+  return pack_bf16(a, b);
+}
+
 struct BwdParams {
   CUtensorMap tm_a;   // per item:  dQ: Q    dK/dV: K
   CUtensorMap tm_b;   // per item:  dQ: dO   dK/dV: V
@@ -456,6 +478,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd_dq_kernel(const
         lse2 = l == -INFINITY ? INFINITY : l * 1.4426950408889634f;
         dlt = p.delta[grow];
       }
+      const uint64_t sl2x2 = pk2(sl2, sl2), nlse2x2 = pk2(-lse2, -lse2), ndlt2 = pk2(-dlt, -dlt);
       // mask bits one job ahead, mask tile indices two jobs ahead: no global load latency
       // between two jobs
       const int nj = it.job_count;
@@ -493,13 +516,11 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd_dq_kernel(const
           if (wb == 0xffffffffu) {
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
-              float ds[2];
-#pragma unroll
-              for (int q = 0; q < 2; ++q) {
-                const float pr = ex2(fmaf(__uint_as_float(sv[2 * e + q]), sl2, -lse2));
-                ds[q] = pr * (__uint_as_float(d32[2 * e + q]) - dlt);
-              }
-              pk[e] = pack_bf16(ds[0], ds[1]);
+              // packed pairs: x = s sl2 - lse2, ds = 2^x (dp - delta)
+              const uint64_t x = ffma2(pk2(__uint_as_float(sv[2 * e]), __uint_as_float(sv[2 * e + 1])), sl2x2, nlse2x2);
+              const uint64_t pr = exp2_pair(x);
+              const uint64_t dd = fadd2(pk2(__uint_as_float(d32[2 * e]), __uint_as_float(d32[2 * e + 1])), ndlt2);
+              pk[e] = pack_bf16x2(fmul2(pr, dd));
             }
           } else {
 #pragma unroll
@@ -728,7 +749,9 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd_dkv_kernel(cons
     const int r = (warp & 3) * 32 + lane, w = (warp - 4) >> 2;
     const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
     const float sl2 = p.scale_log2;
-    // this warp's copy of the job's per-query-row terms (no barrier across warps)
+    const uint64_t sl2x2 = pk2(sl2, sl2);
+    // this warp's copy of the job's per-query-row terms, -lse log2 e and -delta (no barrier
+    // across warps)
     float* rl2 = reinterpret_cast<float*>(sgen + C::OFF_ROWV) + (warp - 4) * 256;
     float* rdl = rl2 + 128;
     uint32_t g = 0;
@@ -767,8 +790,8 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd_dkv_kernel(cons
         __syncwarp();   // the previous job's reads of rl2 / rdl are done
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          rl2[4 * lane + q] = nl[q] == -INFINITY ? INFINITY : nl[q] * 1.4426950408889634f;
-          rdl[4 * lane + q] = nd[q];
+          rl2[4 * lane + q] = nl[q] == -INFINITY ? -INFINITY : -(nl[q] * 1.4426950408889634f);   // -lse2
+          rdl[4 * lane + q] = -nd[q];                                                             // -delta
         }
         __syncwarp();
         const uint4 bits = bits_next;
@@ -799,11 +822,13 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd_dkv_kernel(cons
             if (wb == 0xffffffffu) {
 #pragma unroll
               for (int f = 0; f < 8; ++f) {
-                const float4 la = l2v[f];
-                pr[32 * c + 4 * f + 0] = ex2(fmaf(__uint_as_float(sv[32 * c + 4 * f + 0]), sl2, -la.x));
-                pr[32 * c + 4 * f + 1] = ex2(fmaf(__uint_as_float(sv[32 * c + 4 * f + 1]), sl2, -la.y));
-                pr[32 * c + 4 * f + 2] = ex2(fmaf(__uint_as_float(sv[32 * c + 4 * f + 2]), sl2, -la.z));
-                pr[32 * c + 4 * f + 3] = ex2(fmaf(__uint_as_float(sv[32 * c + 4 * f + 3]), sl2, -la.w));
+                const float4 la = l2v[f];   // -lse2 of four query rows
+                const uint32_t* s4 = sv + 32 * c + 4 * f;
+                const uint64_t x01 = ffma2(pk2(__uint_as_float(s4[0]), __uint_as_float(s4[1])), sl2x2, pk2(la.x, la.y));
+                const uint64_t x23 = ffma2(pk2(__uint_as_float(s4[2]), __uint_as_float(s4[3])), sl2x2, pk2(la.z, la.w));
+                float* p4 = pr + 32 * c + 4 * f;
+                unpk2(exp2_pair(x01), p4[0], p4[1]);
+                unpk2(exp2_pair(x23), p4[2], p4[3]);
               }
             } else {
 #pragma unroll
@@ -813,7 +838,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd_dkv_kernel(cons
 #pragma unroll
                 for (int q = 0; q < 4; ++q)
                   pr[32 * c + 4 * f + q] = ((wb >> (4 * f + q)) & 1u)
-                                               ? ex2(fmaf(__uint_as_float(sv[32 * c + 4 * f + q]), sl2, -lq[q]))
+                                               ? ex2(fmaf(__uint_as_float(sv[32 * c + 4 * f + q]), sl2, lq[q]))
                                                : 0.f;
               }
             }
@@ -837,12 +862,14 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd_dkv_kernel(cons
           uint32_t pk[16];
 #pragma unroll
           for (int f = 0; f < 8; ++f) {
-            const float4 da = dlv[f];
+            const float4 da = dlv[f];   // -delta of four query rows
             const float* pp = pr + 32 * c + 4 * f;
-            pk[2 * f] = pack_bf16(pp[0] * (__uint_as_float(dv[4 * f + 0]) - da.x),
-                                  pp[1] * (__uint_as_float(dv[4 * f + 1]) - da.y));
-            pk[2 * f + 1] = pack_bf16(pp[2] * (__uint_as_float(dv[4 * f + 2]) - da.z),
-                                      pp[3] * (__uint_as_float(dv[4 * f + 3]) - da.w));
+            pk[2 * f] = pack_bf16x2(fmul2(pk2(pp[0], pp[1]),
+                                          fadd2(pk2(__uint_as_float(dv[4 * f]), __uint_as_float(dv[4 * f + 1])),
+                                                pk2(da.x, da.y))));
+            pk[2 * f + 1] = pack_bf16x2(fmul2(pk2(pp[2], pp[3]),
+                                              fadd2(pk2(__uint_as_float(dv[4 * f + 2]), __uint_as_float(dv[4 * f + 3])),
+                                                    pk2(da.z, da.w))));
           }
           tmem_st32x16(tp + 32 + 16 * c, pk);
         }
@@ -1123,6 +1150,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd256_dq_kernel(co
         lse2 = l == -INFINITY ? INFINITY : l * 1.4426950408889634f;
         dlt = p.delta[grow];
       }
+      const uint64_t sl2x2 = pk2(sl2, sl2), nlse2x2 = pk2(-lse2, -lse2), ndlt2 = pk2(-dlt, -dlt);
       for (int j = 0; ok && j < it.job_count; ++j, ++g) {
         const uint4 bits4 = row_bits(p.mask_tiles, p.jobs[it.job_start + j].mask, r);
         if (!__all_sync(0xffffffffu, wait_bounded(BAR(C::B_SFULL), g & 1, guard, kBwdWaitSFull) &&
@@ -1140,16 +1168,25 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd256_dq_kernel(co
           tmem_wait_ld();
           const uint32_t wb = w ? (c ? bits4.w : bits4.z) : (c ? bits4.y : bits4.x);
           uint32_t pk[16];
+          if (wb == 0xffffffffu) {
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            float ds[2];
-#pragma unroll
-            for (int q = 0; q < 2; ++q) {
-              const float pr =
-                  ((wb >> (2 * e + q)) & 1u) ? ex2(fmaf(__uint_as_float(sv[2 * e + q]), sl2, -lse2)) : 0.f;
-              ds[q] = pr * (__uint_as_float(dv[2 * e + q]) - dlt);
+            for (int e = 0; e < 16; ++e) {
+              const uint64_t x = ffma2(pk2(__uint_as_float(sv[2 * e]), __uint_as_float(sv[2 * e + 1])), sl2x2, nlse2x2);
+              const uint64_t dd = fadd2(pk2(__uint_as_float(dv[2 * e]), __uint_as_float(dv[2 * e + 1])), ndlt2);
+              pk[e] = pack_bf16x2(fmul2(exp2_pair(x), dd));
             }
-            pk[e] = pack_bf16(ds[0], ds[1]);
+          } else {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              float ds[2];
+#pragma unroll
+              for (int q = 0; q < 2; ++q) {
+                const float pr =
+                    ((wb >> (2 * e + q)) & 1u) ? ex2(fmaf(__uint_as_float(sv[2 * e + q]), sl2, -lse2)) : 0.f;
+                ds[q] = pr * (__uint_as_float(dv[2 * e + q]) - dlt);
+              }
+              pk[e] = pack_bf16(ds[0], ds[1]);
+            }
           }
           tmem_st32x16(ts + 16 * c, pk);   // over S columns this warpgroup has read
         }
@@ -1264,17 +1301,17 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd256_dkv_kernel(c
       for (int j = 0; ok && j < it.job_count; ++j, ++g) {
         const BwdJob jb = p.jobs[it.job_start + j];
         const uint4 bits = row_bits(p.mask_tiles, jb.mask, r);
-        float l2c[2], dlc[2];   // this lane's query row of chunk 0 / 1
+        float l2c[2], dlc[2];   // -lse log2 e and -delta of this lane's query row of chunk 0 / 1
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
           const int qr = 64 * w + 32 * c + lane;
-          l2c[c] = INFINITY;
+          l2c[c] = -INFINITY;
           dlc[c] = 0.f;
           if (qr < jb.rows) {
             const int64_t gi = int64_t(jb.tok + qr) * p.hq + jb.head;
             const float l = p.lse[gi];
-            l2c[c] = l == -INFINITY ? INFINITY : l * 1.4426950408889634f;
-            dlc[c] = p.delta[gi];
+            l2c[c] = l == -INFINITY ? -INFINITY : -(l * 1.4426950408889634f);
+            dlc[c] = -p.delta[gi];
           }
         }
         if (!__all_sync(0xffffffffu, wait_bounded(BAR(C::B_SFULL), g & 1, guard, kBwdWaitSFull))) {
@@ -1295,7 +1332,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd256_dkv_kernel(c
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
             const float l2 = __shfl_sync(0xffffffffu, l2c[c], e);
-            pr[32 * c + e] = ((wb >> e) & 1u) ? ex2(fmaf(__uint_as_float(sv[e]), sl2, -l2)) : 0.f;
+            pr[32 * c + e] = ((wb >> e) & 1u) ? ex2(fmaf(__uint_as_float(sv[e]), sl2, l2)) : 0.f;
           }
           uint32_t pk[16];
 #pragma unroll
@@ -1317,8 +1354,9 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd256_dkv_kernel(c
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
             const float d0 = __shfl_sync(0xffffffffu, dlc[c], 2 * e), d1 = __shfl_sync(0xffffffffu, dlc[c], 2 * e + 1);
-            pk[e] = pack_bf16(pr[32 * c + 2 * e] * (__uint_as_float(dv[2 * e]) - d0),
-                              pr[32 * c + 2 * e + 1] * (__uint_as_float(dv[2 * e + 1]) - d1));
+            pk[e] = pack_bf16x2(fmul2(pk2(pr[32 * c + 2 * e], pr[32 * c + 2 * e + 1]),
+                                      fadd2(pk2(__uint_as_float(dv[2 * e]), __uint_as_float(dv[2 * e + 1])),
+                                            pk2(d0, d1))));
           }
           tmem_st32x16(tp + 16 * c, pk);
         }
