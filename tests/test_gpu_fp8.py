@@ -8,8 +8,10 @@ values are exact, and the sums stay well inside fp32 precision), so the error co
 rounding P to e4m3 for the P V product: with p_ij = exp(s_ij - lse_i) (rows sum to one)
 and the kernel's l >= 1 (its reference maximum never exceeds the row maximum), each
 rounded P is off by at most max(2^-4 p_ij, 2^-10) in units of l (half an e4m3 ulp:
-2^-4 relative for normal values, 2^-10 absolute for subnormals), so
-    |out_i - ref_i| <= v_scale sum_j max(2^-4 p_ij, 2^-10) |v8_j| + 2^-8 |ref_i| + 1e-5,
+2^-4 relative for normal values, 2^-10 absolute for subnormals), plus the error of the
+exponential before rounding: a quarter of the columns use the FMA-pipe polynomial, whose
+relative error (7.5e-5, pinned by its own test) is below 2^-13, so
+    |out_i - ref_i| <= v_scale sum_j (max(2^-4 p_ij, 2^-10) + 2^-13 p_ij) |v8_j| + 2^-8 |ref_i| + 1e-5,
 the second term covering the bf16 rounding of out. lse uses P before rounding: 1e-3."""
 import numpy as np
 import pytest
@@ -67,7 +69,7 @@ def _bound(wl_deq, spec):
             s = wl_deq.scale * q @ k.T
             has = np.isfinite(lse)
             p = np.where(m & has[:, None], np.exp(np.where(m, s, 0) - np.where(has, lse, 0)[:, None]), 0)
-            w = np.where(m & has[:, None], np.maximum(2.0 ** -4 * p, 2.0 ** -10), 0)
+            w = np.where(m & has[:, None], np.maximum(2.0 ** -4 * p, 2.0 ** -10) + 2.0 ** -13 * p, 0)
             bound[q0:q0 + lq, h] = w @ np.abs(v).max(axis=1)
     return bound
 
