@@ -212,23 +212,50 @@ __device__ __forceinline__ void store_grad_cols(uint32_t t_acc, float mul, bool 
   }
 }
 
-// delta[r][h] = dout[r][h] . out[r][h] - dlse[r][h] (fp32; dlse may be null), one warp per
-// (row, head). With a gradient on lse, ds = p (dp - delta) picks up + p dlse.
+// delta[r][h] = dout[r][h] . out[r][h] - dlse[r][h] (fp32; dlse may be null) over the rows
+// r = (token, head) of D bf16 values. With a gradient on lse, ds = p (dp - delta) picks up
+// + p dlse. A row is read by D / 8 lanes, 16 bytes of each tensor per lane (both 16-byte
+// aligned), and every lane keeps four rows' loads in flight: one warp per row with 4-byte
+// loads left the read at under half of the HBM rate.
+__device__ __forceinline__ float dot8_bf16(const uint4& a, const uint4& b) {
+  const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, bw[4] = {b.x, b.y, b.z, b.w};
+  float acc = 0.f;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&aw[i]));
+    const float2 y = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&bw[i]));
+    acc = fmaf(x.x, y.x, acc);
+    acc = fmaf(x.y, y.y, acc);
+  }
+  return acc;
+}
+
+template <int D>
 __global__ void bwd_delta_kernel(const __nv_bfloat16* __restrict__ out, const __nv_bfloat16* __restrict__ dout,
-                                 const float* __restrict__ dlse, float* __restrict__ delta, int64_t rows, int D) {
-  const int lane = threadIdx.x & 31;
-  const int64_t warps = int64_t(gridDim.x) * (blockDim.x >> 5);
-  for (int64_t r = int64_t(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); r < rows; r += warps) {
-    float acc = 0.f;
-    for (int c = 2 * lane; c < D; c += 64) {
-      const __nv_bfloat162 o = *reinterpret_cast<const __nv_bfloat162*>(out + r * D + c);
-      const __nv_bfloat162 g = *reinterpret_cast<const __nv_bfloat162*>(dout + r * D + c);
-      acc = fmaf(__low2float(o), __low2float(g), acc);
-      acc = fmaf(__high2float(o), __high2float(g), acc);
+                                 const float* __restrict__ dlse, float* __restrict__ delta, int64_t rows) {
+  constexpr int L = D / 8, RPW = 32 / L, U = 4;   // lanes per row, rows per warp pass, passes in flight
+  const int lane = threadIdx.x & 31, sub = lane % L, grp = lane / L;
+  const int64_t warp0 = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = (int64_t(gridDim.x) * blockDim.x) >> 5;
+  for (int64_t base = warp0 * (RPW * U); base < rows; base += nwarps * (RPW * U)) {   // warp-uniform
+    uint4 o[U], g[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int64_t r = base + u * RPW + grp;
+      o[u] = g[u] = make_uint4(0u, 0u, 0u, 0u);
+      if (r < rows) {
+        o[u] = __ldg(reinterpret_cast<const uint4*>(out + r * D) + sub);
+        g[u] = __ldg(reinterpret_cast<const uint4*>(dout + r * D) + sub);
+      }
     }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-    if (lane == 0) delta[r] = dlse ? acc - dlse[r] : acc;
+    for (int u = 0; u < U; ++u) {
+      float acc = dot8_bf16(o[u], g[u]);
+#pragma unroll
+      for (int m = L / 2; m > 0; m >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m);
+      const int64_t r = base + u * RPW + grp;
+      if (sub == 0 && r < rows) delta[r] = dlse ? acc - dlse[r] : acc;
+    }
   }
 }
 
@@ -1448,8 +1475,13 @@ attn_status_t mfa_launch_backward(const attn_plan_t* plan, const void* q, const 
     if (e == cudaSuccess) e = cudaMemsetAsync(dv, 0, size_t(krows) * D * 2, stream);
     return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
   }
-  bwd_delta_kernel<<<4 * 148, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(out),
-                                                static_cast<const __nv_bfloat16*>(dout), dlse, plan->d_bdelta, qrows, D);
+  {
+    const auto* o16 = static_cast<const __nv_bfloat16*>(out);
+    const auto* g16 = static_cast<const __nv_bfloat16*>(dout);
+    if (D == 64) bwd_delta_kernel<64><<<8 * 148, 256, 0, stream>>>(o16, g16, dlse, plan->d_bdelta, qrows);
+    else if (D == 128) bwd_delta_kernel<128><<<8 * 148, 256, 0, stream>>>(o16, g16, dlse, plan->d_bdelta, qrows);
+    else bwd_delta_kernel<256><<<8 * 148, 256, 0, stream>>>(o16, g16, dlse, plan->d_bdelta, qrows);
+  }
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
   BwdParams pq{}, pk{};
   // paged: K / V boxes of one page; dk / dv cover the whole cache, and the rows no sequence
