@@ -4,7 +4,7 @@
 // delta_i = dout_i . out_i and ds_ij = p_ij (dp_ij - delta_i):
 //     dq_i = scale sum_j ds_ij k_j,   dk_j = scale sum_i ds_ij q_i,   dv_j = sum_i p_ij dout_i,
 // dk and dv of a key/value head summed over the query heads that read it. Three kernels:
-//   bwd_delta_kernel    delta_i for every (row, query head): one warp per row.
+//   bwd_delta_kernel    delta_i for every (row, query head): d / 8 lanes per row.
 //   dQ kernel           one persistent CTA per SM over dQ items (a 128-row query tile of one
 //                       query head and its non-empty key tiles): S = Q K^T and dP = dO V^T
 //                       into TMEM, the elementwise warpgroups turn them into dS (bf16, written
@@ -37,7 +37,9 @@
 // dQ: bf16 dS pairs of columns 0..63 go to TMEM columns 0..31 of the S slot and those of
 // columns 64..127 to 64..95; dK/dV: P^T pairs to columns 0..31 / 64..95 of the slot and dS^T
 // pairs to 32..63 / 96..127. Each warpgroup writes only columns it has already read. Every
-// mbarrier wait is bounded as in the forward.
+// mbarrier wait is bounded as in the forward. At head_dim 256 (Bwd256Cfg) the tiles are too
+// large for this layout: the streamed operands come as half-tiles, one thread issues a job's
+// MMAs in order, and dK / dV take two passes, one per head-dim half of the accumulators.
 
 #include <cuda.h>
 #include <cudaTypedefs.h>
