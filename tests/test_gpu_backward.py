@@ -171,6 +171,56 @@ def test_backward_full_size_chunk_causal_sampled():
     _close(got_v, rv, "full-size dv")
 
 
+def _full_size_sampled(cfg, seed, n_rows, key_pairs, n_keys, compare_forms):
+    """Backward of a benchmark workload at full size, every mask of it, in the launch the
+    benchmark times: dq on sampled rows (first / middle / last rows of every sequence and
+    random ones), dk and dv on sampled keys of the given (sequence, KV head) pairs, against
+    the oracle evaluated at those places; with `compare_forms`, the masks are two descriptor
+    forms of one mask and must give identical gradients."""
+    wl = W.config(cfg)
+    q, k, v = G.device_inputs(wl)
+    gen = torch.Generator().manual_seed(seed)
+    dout_h = W.randn_bf16(gen, q.shape[0], wl.hq, wl.d)
+    dout = dout_h.cuda()
+    rng = np.random.default_rng(seed)
+    qs = G.sample_rows(wl, n_rows, seed=seed)
+    ks = [(b, kh, int(j)) for b, kh in key_pairs
+          for j in list(rng.integers(0, wl.lk(b), size=n_keys)) + [0, wl.lk(b) - 1]]
+    grads = []
+    for spec in wl.masks:
+        plan = G.M.attn_plan(hq=wl.hq, hkv=wl.hkv, head_dim=wl.d, cu_seqlens_q=wl.cu_seqlens_q,
+                             cu_seqlens_k=wl.cu_seqlens_k, mask=spec, scale=wl.scale, backward=True)
+        out, lse = G.M.forward(plan, q, k, v)
+        dq, dk, dv = G.M.backward(plan, q, k, v, out, lse, dout)
+        assert G.M.attn_plan_check_status(plan) == 0
+        grads.append((spec, dq.cpu(), dk.cpu(), dv.cpu()))
+    if compare_forms:
+        for a, b in zip(grads[0][1:], grads[1][1:]):
+            assert torch.equal(a, b)
+        grads = grads[:1]
+    for spec, dq, dk, dv in grads:
+        rq, rk, rv = oracle.sampled_backward(wl, spec, dout_h, qs, ks)
+        got_q = torch.stack([dq[int(wl.cu_seqlens_q[b]) + i, h] for b, h, i in qs])
+        got_k = torch.stack([dk[int(wl.cu_seqlens_k[b]) + j, kh] for b, kh, j in ks])
+        got_v = torch.stack([dv[int(wl.cu_seqlens_k[b]) + j, kh] for b, kh, j in ks])
+        _close(got_q, rq, f"workload {cfg} {spec.kind} dq")
+        _close(got_k, rk, f"workload {cfg} {spec.kind} dk")
+        _close(got_v, rv, f"workload {cfg} {spec.kind} dv")
+
+
+def test_backward_full_size_gemma2_sampled():
+    """The Gemma2 workload (4 sequences up to 7028 tokens, 16 / 8 heads, d = 256), its
+    sliding-window and causal masks, through the head_dim 256 kernels."""
+    _full_size_sampled(2, seed=45, n_rows=24, key_pairs=[(0, 3), (2, 6)], n_keys=6, compare_forms=False)
+
+
+def test_backward_full_size_block_dense_sampled():
+    """The block-dense workload (one sequence of 29576 tokens, 32 / 8 heads, d = 128), as
+    packed bits and as ranges (identical gradients), on sampled rows and on keys of one
+    KV head, among them keys of the causal blocks past 24576."""
+    _full_size_sampled(5, seed=46, n_rows=24, key_pairs=[(0, 5)], n_keys=6, compare_forms=True)
+
+
 @pytest.mark.parametrize("d", [128, 256])
 def test_backward_timeout_reports_and_context_survives(d):
     """The forced missing arrival of the debug hook in both backward kernels: a bounded wait
