@@ -963,7 +963,8 @@ struct Bwd256Cfg {
   static constexpr int OFF_BAR = OFF_RING + RSLOTS * HALF_BYTES;
   static constexpr int B_AFULL = 0, B_AEMPTY = 1, B_RFULL = 2, B_REMPTY = B_RFULL + RSLOTS,
                        B_SFULL = B_REMPTY + RSLOTS, B_DPFULL = B_SFULL + 1, B_READY = B_DPFULL + 1,
-                       B_ACCFULL = B_READY + 1, B_ACCEMPTY = B_ACCFULL + 1, B_DRAIN = B_ACCEMPTY + 1,
+                       B_PREADY = B_READY + 1,   // dK/dV: P^T written (dV may start before dS^T)
+                       B_ACCFULL = B_PREADY + 1, B_ACCEMPTY = B_ACCFULL + 1, B_DRAIN = B_ACCEMPTY + 1,
                        NBAR = B_DRAIN + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;       // [0] TMEM base, [1] abort flag
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;   // + slack to align the base to 1 KiB
@@ -1066,6 +1067,7 @@ __device__ __forceinline__ void bwd256_setup(uint32_t bar0, uint32_t* misc, cons
     mbar_init(BAR(C::B_SFULL), 1);
     mbar_init(BAR(C::B_DPFULL), 1);
     mbar_init(BAR(C::B_READY), C::EW);
+    mbar_init(BAR(C::B_PREADY), C::EW);
     mbar_init(BAR(C::B_ACCFULL), 1);
     mbar_init(BAR(C::B_ACCEMPTY), C::EW);
     mbar_init(BAR(C::B_DRAIN), 1);
@@ -1271,7 +1273,8 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd256_dkv_kernel(c
     bwd256_produce<C>(p, sbase, bar0, guard, i_begin, i_end, true, order, lane);
     __syncwarp();
   } else if (warp == 1) {
-    // ---- MMA issuer: S^T = K Q^T, dP^T = V dO^T, then dV_h += P^T dO_h and dK_h += dS^T Q_h ----
+    // ---- MMA issuer: S^T = K Q^T, dP^T = V dO^T, then dV_h += P^T dO_h once the warpgroups
+    // have written P^T (they then compute dS^T) and dK_h += dS^T Q_h ----
     if (lane == 0) {
       uint32_t rc = 0, g = 0;
       int n = 0;
@@ -1297,15 +1300,18 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd256_dkv_kernel(c
           mma_ss_k256(tmem + C::TM_P, sbase + C::OFF_B, ring(rd[0]), ring(rd[1]), C::IDESC_SS);   // dP^T = V dO^T
           mma_commit(BAR(C::B_DPFULL));
           mma_commit(BAR(C::B_REMPTY + (rc + 2) % C::RSLOTS));   // dO half 1-h: read by dP^T only
-          ok = wait_bounded(BAR(C::B_READY), g & 1, guard, kBwdWaitDsReady);
+          ok = wait_bounded(BAR(C::B_PREADY), g & 1, guard, kBwdWaitPFull);
           if (ok && j == 0) ok = wait_bounded(BAR(C::B_ACCEMPTY), (n & 1) ^ 1, guard, kBwdWaitAccEmpty);
           if (!ok) break;
           tc_fence_after();
           const uint32_t acc = j > 0 ? 1u : 0u;
-          mma_tile_ts(tmem + C::TM_ACC, tmem + C::TM_S, ring(rc + 3), C::IDESC_TS, acc);         // dV_h += P^T dO_h
+          mma_tile_ts(tmem + C::TM_ACC, tmem + C::TM_S, ring(rc + 3), C::IDESC_TS, acc);   // dV_h += P^T dO_h
+          mma_commit(BAR(C::B_REMPTY + (rc + 3) % C::RSLOTS));                            // dO half h
+          ok = wait_bounded(BAR(C::B_READY), g & 1, guard, kBwdWaitDsReady);
+          if (!ok) break;
+          tc_fence_after();
           mma_tile_ts(tmem + C::TM_ACC + 128, tmem + C::TM_P, ring(rc + 1), C::IDESC_TS, acc);   // dK_h += dS^T Q_h
-          mma_commit(BAR(C::B_REMPTY + (rc + 1) % C::RSLOTS));
-          mma_commit(BAR(C::B_REMPTY + (rc + 3) % C::RSLOTS));
+          mma_commit(BAR(C::B_REMPTY + (rc + 1) % C::RSLOTS));                                  // Q half h
         }
         if (!ok) break;
         mma_commit(BAR(C::B_ACCFULL));
@@ -1368,6 +1374,9 @@ __global__ void __launch_bounds__(C::THREADS, 1) masked_attn_bwd256_dkv_kernel(c
           for (int e = 0; e < 16; ++e) pk[e] = pack_bf16(pr[32 * c + 2 * e], pr[32 * c + 2 * e + 1]);
           tmem_st32x16(ts + 16 * c, pk);
         }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(BAR(C::B_PREADY));   // dV_h += P^T dO_h may run while dS^T is computed
         if (!__all_sync(0xffffffffu, wait_bounded(BAR(C::B_DPFULL), g & 1, guard, kBwdWaitDpFull))) {
           ok = false;
           break;
