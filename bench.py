@@ -872,11 +872,18 @@ def run_ours(args, rank, world, local_rank):
         # its timed region): every configuration's throughput in the same line
         del q, k, v, outs, lses
         torch.cuda.empty_cache()
-        line["per_config"] = [time_config(M, c, dev, stream, max(3, min(args.steps, 30)), 3, peak, hbm_peak)
+        def section(cfg, **kw):
+            # a failure here is reported in the entry; the headline above stands on its own
+            try:
+                return time_config(M, cfg, dev, stream, peak=peak, hbm_peak=hbm_peak, **kw)
+            except Exception as e:   # noqa: BLE001 -- recorded in the line, not swallowed
+                torch.cuda.synchronize()
+                return {"config": cfg, "pass": "bwd" if kw.get("bwd") else "fwd", "error": f"{type(e).__name__}: {e}"}
+
+        line["per_config"] = [section(c, steps=max(3, min(args.steps, 30)), warmup=3)
                               for c in (1, 2, 3, 4, 5) if c != args.config]
         # the backward of the chunk-causal (d = 128) and Gemma2 (d = 256) workloads
-        line["backward"] = [time_config(M, c, dev, stream, max(3, min(args.steps, 20)), 3, peak, hbm_peak, bwd=True)
-                            for c in (4, 2)]
+        line["backward"] = [section(c, steps=max(3, min(args.steps, 20)), warmup=3, bwd=True) for c in (4, 2)]
     if world == 1 and not args.no_cpu_baseline and not bwd and not fp8:
         pairs, secs, desc = oracle_sample(wl, wl.masks, args.cpu_seconds)
         line["cpu_baseline"] = {"value": 4.0 * wl.d * pairs / secs / 1e12, "unit": "TFLOP/s",
