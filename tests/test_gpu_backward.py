@@ -1,6 +1,8 @@
 """GPU parity of the backward pass (dQ, dK, dV) through the C ABI against the fp64 oracle
-gradients (oracle/backward.py), on ragged contiguous batches of every mask kind, head dims
-64, 128 and 256, grouped-query heads, rows that see no key and keys no query sees.
+gradients (oracle/backward.py), on ragged batches of every mask kind, head dims 64, 128 and
+256, contiguous K/V and paged caches (dk / dv in the cache layout; unused slots poisoned),
+grouped-query heads, rows that see no key and keys no query sees; and three benchmark
+workloads at full size on sampled rows and keys.
 
 Tolerance: P and dS enter the tensor cores as bf16 (relative rounding 2^-9 each) with fp32
 accumulation, and the gradients are stored as bf16 (relative rounding 2^-9, i.e. a mean
