@@ -36,7 +36,8 @@
  *     GPUs, each computing its rows against all (all-gathered) keys;
  *   - attn_plan_bwd() + attn_masked_bwd(): dq, dk, dv;
  *   - attn_fp8_transpose_v() + attn_masked_fwd_fp8(): the forward on e4m3 inputs;
- *   - attn_plan_dry_run(): the plan statistics on the host, without a GPU;
+ *   - attn_plan_dry_run() / attn_plan_bwd_dry_run(): the forward / backward plan
+ *     statistics on the host, without a GPU;
  *   - attn_masked_fwd_noalloc(): plan + forward without any device allocation.
  *
  * Errors. Every call returns an attn_status_t; nothing is thrown across the ABI and
@@ -303,6 +304,26 @@ attn_status_t attn_classify_host(const attn_problem_t* problem, const attn_mask_
  * (num_sms <= 0 or as attn_plan), UNSUPPORTED (CUSTOM, or as attn_plan), OOM. */
 attn_status_t attn_plan_dry_run(const attn_problem_t* problem, const attn_mask_desc_t* mask, int32_t num_sms,
                                 attn_plan_stats_t* stats);
+
+/* Statistics of the backward work lists (attn_plan_bwd() builds the same lists over
+ * 128 x 128 tiles of one head). */
+typedef struct {
+  int64_t dq_items, dq_jobs;        /* dQ items (query tile, query head) and the key tiles they run */
+  int64_t dkv_items, dkv_jobs;      /* dK/dV items (key tile, KV head) and the (query head, query tile)s they run */
+  int64_t mask_tiles;               /* tiles that carry a mask (partial, or cut by the end of the keys or queries) */
+  int32_t dq_ctas, dkv_ctas;        /* persistent CTAs of the two kernels */
+  int64_t dq_cost, dkv_cost;        /* sum over items of (jobs + 2), the planner's cost unit */
+  int64_t dq_max_cta_cost, dkv_max_cta_cost; /* largest per-CTA cost after the longest-first assignment */
+  int64_t dq_max_item_cost, dkv_max_item_cost;
+} attn_bwd_stats_t;
+
+/* Host-only dry run of attn_plan_bwd() for the analytic kinds: the same validation and
+ * backward work lists for a GPU of `num_sms` SMs, with no CUDA call and no device memory.
+ * A paged problem's page table is not read (the check that no page is read by two
+ * sequences needs it on the device). Errors: INVALID_ARG (num_sms <= 0 or as attn_plan),
+ * UNSUPPORTED (CUSTOM, or as attn_plan_bwd), OOM. */
+attn_status_t attn_plan_bwd_dry_run(const attn_problem_t* problem, const attn_mask_desc_t* mask, int32_t num_sms,
+                                    attn_bwd_stats_t* stats);
 
 const char* attn_status_string(attn_status_t status);
 

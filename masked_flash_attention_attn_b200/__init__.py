@@ -47,7 +47,7 @@ EXPORTS = ("attn_plan", "attn_masked_fwd", "attn_plan_get_tile_classes", "attn_p
            "attn_plan_check_status", "attn_plan_set_debug", "attn_plan_destroy", "attn_classify_host",
            "attn_status_string", "attn_masked_fwd_noalloc", "attn_test_exp2_poly", "attn_plan_dry_run",
            "attn_plan_bwd", "attn_masked_bwd", "attn_masked_fwd_fp8", "attn_fp8_transpose_v",
-           "attn_test_transpose_mask_tile", "attn_test_noalloc_debug")
+           "attn_test_transpose_mask_tile", "attn_test_noalloc_debug", "attn_plan_bwd_dry_run")
 
 
 class AttnError(RuntimeError):
@@ -75,6 +75,14 @@ class attn_problem_t(ctypes.Structure):
                 ("cu_seqlens_k", ctypes.c_void_p), ("kv_lens", ctypes.c_void_p), ("page_table", ctypes.c_void_p),
                 ("page_size", ctypes.c_int32), ("max_pages_per_seq", ctypes.c_int32), ("num_pages", ctypes.c_int32),
                 ("kv_splits", ctypes.c_int32), ("q_begin", ctypes.c_int32), ("q_end", ctypes.c_int32)]
+
+
+class attn_bwd_stats_t(ctypes.Structure):
+    _fields_ = [("dq_items", ctypes.c_int64), ("dq_jobs", ctypes.c_int64), ("dkv_items", ctypes.c_int64),
+                ("dkv_jobs", ctypes.c_int64), ("mask_tiles", ctypes.c_int64), ("dq_ctas", ctypes.c_int32),
+                ("dkv_ctas", ctypes.c_int32), ("dq_cost", ctypes.c_int64), ("dkv_cost", ctypes.c_int64),
+                ("dq_max_cta_cost", ctypes.c_int64), ("dkv_max_cta_cost", ctypes.c_int64),
+                ("dq_max_item_cost", ctypes.c_int64), ("dkv_max_item_cost", ctypes.c_int64)]
 
 
 class attn_plan_stats_t(ctypes.Structure):
@@ -120,6 +128,8 @@ def lib() -> ctypes.CDLL:
         L.attn_test_transpose_mask_tile.argtypes = [vp, vp]
         L.attn_plan_dry_run.argtypes = [ctypes.POINTER(attn_problem_t), ctypes.POINTER(attn_mask_desc_t), i32,
                                         ctypes.POINTER(attn_plan_stats_t)]
+        L.attn_plan_bwd_dry_run.argtypes = [ctypes.POINTER(attn_problem_t), ctypes.POINTER(attn_mask_desc_t), i32,
+                                            ctypes.POINTER(attn_bwd_stats_t)]
         L.attn_masked_fwd_noalloc.argtypes = [ctypes.POINTER(attn_problem_t), ctypes.POINTER(attn_mask_desc_t),
                                               vp, vp, vp, vp, vp, vp]
         L.attn_test_noalloc_debug.argtypes = [i32, i64]
@@ -429,6 +439,22 @@ def attn_plan_dry_run(*, hq: int, hkv: int, head_dim: int, cu_seqlens_q, mask, n
     _check(lib().attn_plan_dry_run(ctypes.byref(pr), ctypes.byref(d), int(num_sms), ctypes.byref(st)),
            "attn_plan_dry_run")
     return {n: getattr(st, n) for n, _ in attn_plan_stats_t._fields_}
+
+
+def attn_plan_bwd_dry_run(*, hq: int, hkv: int, head_dim: int, cu_seqlens_q, mask, num_sms: int = 148,
+                          cu_seqlens_k=None, kv_lens=None, page_size: int = 0, max_pages_per_seq: int = 0,
+                          num_pages: int = 0) -> dict:
+    """Host-only attn_plan_bwd() work lists (analytic kinds) for a GPU of ``num_sms`` SMs: their statistics."""
+    m = _Marshal()
+    pr = _problem(m, hq=hq, hkv=hkv, head_dim=head_dim, cu_seqlens_q=cu_seqlens_q, cu_seqlens_k=cu_seqlens_k,
+                  kv_lens=kv_lens)
+    if kv_lens is not None:
+        pr.page_size, pr.max_pages_per_seq, pr.num_pages = page_size, max_pages_per_seq, num_pages
+    d = _mask_desc(m, mask, cu_seqlens_q=cu_seqlens_q)
+    st = attn_bwd_stats_t()
+    _check(lib().attn_plan_bwd_dry_run(ctypes.byref(pr), ctypes.byref(d), int(num_sms), ctypes.byref(st)),
+           "attn_plan_bwd_dry_run")
+    return {n: getattr(st, n) for n, _ in attn_bwd_stats_t._fields_}
 
 
 def attn_classify_host(*, hq: int, hkv: int, head_dim: int, cu_seqlens_q, mask, cu_seqlens_k=None, kv_lens=None,

@@ -1289,6 +1289,55 @@ attn_status_t attn_test_transpose_mask_tile(const uint32_t* src, uint32_t* dst) 
   return ATTN_OK;
 }
 
+attn_status_t attn_plan_bwd_dry_run(const attn_problem_t* problem, const attn_mask_desc_t* mask, int32_t num_sms,
+                                    attn_bwd_stats_t* stats) {
+  try {
+    if (!stats || num_sms <= 0) return ATTN_ERR_INVALID_ARG;
+    if (mask && mask->kind == ATTN_MASK_CUSTOM) return ATTN_ERR_UNSUPPORTED;
+    Shape s;
+    attn_status_t st = validate_problem(problem, s, /*need_device_ptrs=*/false);
+    if (st != ATTN_OK) return st;
+    st = validate_mask(mask, s);
+    if (st != ATTN_OK) return st;
+    std::vector<std::vector<int32_t>> cnts(s.B);
+    RowSource src(mask, s);
+    for (int b = 0; b < s.B; ++b) {
+      src.prepare(b);
+      count_sequence(src, b, s, kTile, cnts[b]);
+    }
+    BwdLists bl;
+    build_bwd(s, cnts, num_sms, bl);
+    attn_bwd_stats_t out{};
+    auto side = [](const std::vector<BwdItem>& items, const std::vector<int32_t>& off,
+                   const std::vector<int32_t>& list, int64_t& n_items, int64_t& n_jobs, int32_t& ctas,
+                   int64_t& cost, int64_t& max_cta, int64_t& max_item) {
+      n_items = int64_t(items.size());
+      for (const BwdItem& it : items) {
+        n_jobs += it.job_count;
+        cost += it.job_count + 2;
+        max_item = std::max<int64_t>(max_item, it.job_count + 2);
+      }
+      ctas = int32_t(off.size()) - 1;
+      for (int32_t c = 0; c < ctas; ++c) {
+        int64_t load = 0;
+        for (int32_t e = off[c]; e < off[c + 1]; ++e) load += items[size_t(list[e])].job_count + 2;
+        max_cta = std::max(max_cta, load);
+      }
+    };
+    side(bl.q_items, bl.q_off, bl.q_list, out.dq_items, out.dq_jobs, out.dq_ctas, out.dq_cost, out.dq_max_cta_cost,
+         out.dq_max_item_cost);
+    side(bl.kv_items, bl.kv_off, bl.kv_list, out.dkv_items, out.dkv_jobs, out.dkv_ctas, out.dkv_cost,
+         out.dkv_max_cta_cost, out.dkv_max_item_cost);
+    out.mask_tiles = int64_t(bl.tiles.size());
+    *stats = out;
+    return ATTN_OK;
+  } catch (const std::bad_alloc&) {
+    return ATTN_ERR_OOM;
+  } catch (...) {
+    return ATTN_ERR_INVALID_ARG;
+  }
+}
+
 attn_status_t attn_plan_dry_run(const attn_problem_t* problem, const attn_mask_desc_t* mask, int32_t num_sms,
                                 attn_plan_stats_t* stats) {
   try {
