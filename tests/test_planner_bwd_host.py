@@ -101,3 +101,16 @@ def test_custom_and_bad_arguments_are_refused(attn_lib):
     with pytest.raises(M.AttnError) as e:
         M.attn_plan_bwd_dry_run(**_kw(wl, wl.masks[0], 0))
     assert e.value.status == 1
+
+
+def test_chunk_causal_workload_closed_form(attn_lib):
+    # 8 sequences of 8192 = 64 x 128 rows, causal over [0, 4096) then chunk-causal (chunk 2)
+    # over [4096, 8192): per sequence and head 2016 full + 64 partial non-empty tiles (the
+    # forward's tile classes), no tile cut by a sequence end, every query tile sees a key and
+    # every key tile is seen -- so both kernels run 16 x 8 x 2080 jobs and 8 x 64 tiles carry a mask
+    wl = W.config(4)
+    for spec in wl.masks:   # both descriptor forms
+        st = attn_lib.attn_plan_bwd_dry_run(**_kw(wl, spec, 148))
+        assert st["dq_items"] == st["dkv_items"] == 16 * 8 * 64
+        assert st["dq_jobs"] == st["dkv_jobs"] == 16 * 8 * 2080
+        assert st["mask_tiles"] == 8 * 64
